@@ -1,0 +1,264 @@
+"""Seeded synthetic inputs: decoder geometries, workloads and random tensors.
+
+This module holds shapes and random numbers only -- none of the decoder's
+arithmetic.  The CUDA library and the parity oracle both consume the float32
+arrays it produces.
+
+Random numbers: SplitMix64 (Steele, Lea & Flood, "Fast splittable
+pseudorandom number generators", OOPSLA 2014) used as a counter-based stream --
+the i-th 64-bit word of stream ``seed`` is mix(seed + (i + 1) * 0x9E3779B97F4A7C15)
+-- and the Box-Muller transform (Box & Muller 1958) on consecutive pairs of
+words: u1 = ((w0 >> 11) + 1) / 2^53, u2 = (w1 >> 11) / 2^53,
+n0 = sqrt(-2 ln u1) cos(2 pi u2), n1 = sqrt(-2 ln u1) sin(2 pi u2).
+One stream per workload; the input is drawn first, then the parameters in
+module order (``param_layout``), each tensor taking the next normals.
+"""
+from __future__ import annotations
+
+import dataclasses
+from dataclasses import dataclass, field
+from typing import List, Sequence, Tuple
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+M1 = np.uint64(0xBF58476D1CE4E5B9)
+M2 = np.uint64(0x94D049BB133111EB)
+
+
+def splitmix64_words(seed: int, start: int, count: int) -> np.ndarray:
+    """Words start .. start+count-1 of SplitMix64 stream ``seed``."""
+    i = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed) + i * GAMMA
+        z = (z ^ (z >> np.uint64(30))) * M1
+        z = (z ^ (z >> np.uint64(27))) * M2
+    return z ^ (z >> np.uint64(31))
+
+
+class NormalStream:
+    """Consecutive standard normals from one seeded SplitMix64 stream."""
+
+    CHUNK = 1 << 22
+
+    def __init__(self, seed: int):
+        self.seed = int(seed)
+        self.pos = 0  # index of the next normal
+
+    def _normals(self, start: int, count: int) -> np.ndarray:
+        # normals 2k and 2k+1 come from words 2k and 2k+1
+        p0 = start // 2
+        p1 = (start + count + 1) // 2
+        w = splitmix64_words(self.seed, 2 * p0, 2 * (p1 - p0))
+        u1 = ((w[0::2] >> np.uint64(11)) + np.uint64(1)).astype(np.float64) * 2.0 ** -53
+        u2 = (w[1::2] >> np.uint64(11)).astype(np.float64) * 2.0 ** -53
+        r = np.sqrt(-2.0 * np.log(u1))
+        th = 2.0 * np.pi * u2
+        out = np.empty(2 * (p1 - p0), np.float64)
+        out[0::2] = r * np.cos(th)
+        out[1::2] = r * np.sin(th)
+        off = start - 2 * p0
+        return out[off:off + count]
+
+    def normal(self, shape, mean=0.0, std=1.0) -> np.ndarray:
+        n = int(np.prod(shape)) if len(shape) else 1
+        out = np.empty(n, np.float32)
+        done = 0
+        while done < n:
+            c = min(self.CHUNK, n - done)
+            out[done:done + c] = (mean + std * self._normals(self.pos + done, c)).astype(np.float32)
+            done += c
+        self.pos += n
+        return out.reshape(shape)
+
+
+# ----------------------------------------------------------------- geometry
+
+
+@dataclass(frozen=True)
+class DecoderGeometry:
+    """Shape of a BigVGAN-style decoder (conv_pre -> ConvT stages with AMP
+    blocks averaged per stage -> act_post -> conv_post -> final op)."""
+    in_channels: int
+    pre_channels: int
+    pre_kernel: int
+    up_rates: Tuple[int, ...]
+    up_kernels: Tuple[int, ...]
+    up_channels: Tuple[int, ...]
+    block_kernels: Tuple[int, ...]
+    dilations: Tuple[int, ...]
+    post_kernel: int
+    out_channels: int
+    final_act: str  # "none" | "clamp" | "tanh"
+    sample_rate: int
+
+    @property
+    def hop(self) -> int:
+        h = 1
+        for r in self.up_rates:
+            h *= r
+        return h
+
+    def replace(self, **kw) -> "DecoderGeometry":
+        return dataclasses.replace(self, **kw)
+
+
+def param_layout(g: DecoderGeometry) -> List[Tuple[str, Tuple[int, ...], str]]:
+    """(name, shape, kind) of every decoder parameter in module order; kind is
+    'w' (conv weight), 'b' (bias) or 'snake' (log alpha / log beta)."""
+    out = []
+    C = g.pre_channels
+    out.append(("conv_pre.w", (C, g.in_channels, g.pre_kernel), "w"))
+    out.append(("conv_pre.b", (C,), "b"))
+    for i, (s, k, co) in enumerate(zip(g.up_rates, g.up_kernels, g.up_channels)):
+        out.append((f"ups.{i}.w", (C, co, k), "w"))
+        out.append((f"ups.{i}.b", (co,), "b"))
+        C = co
+        for j, kb in enumerate(g.block_kernels):
+            for u, _d in enumerate(g.dilations):
+                p = f"stage{i}.block{j}.unit{u}"
+                out += [(f"{p}.act1.log_alpha", (C,), "snake"),
+                        (f"{p}.act1.log_beta", (C,), "snake"),
+                        (f"{p}.conv1.w", (C, C, kb), "w"),
+                        (f"{p}.conv1.b", (C,), "b"),
+                        (f"{p}.act2.log_alpha", (C,), "snake"),
+                        (f"{p}.act2.log_beta", (C,), "snake"),
+                        (f"{p}.conv2.w", (C, C, kb), "w"),
+                        (f"{p}.conv2.b", (C,), "b")]
+    out.append(("act_post.log_alpha", (C,), "snake"))
+    out.append(("act_post.log_beta", (C,), "snake"))
+    out.append(("conv_post.w", (g.out_channels, C, g.post_kernel), "w"))
+    out.append(("conv_post.b", (g.out_channels,), "b"))
+    return out
+
+
+def param_count(g: DecoderGeometry) -> int:
+    return int(sum(int(np.prod(s)) for _, s, _ in param_layout(g)))
+
+
+# The parameter distributions of the synthetic decoders: conv and ConvT
+# weights and biases N(0, 0.02), SnakeBeta log-alpha / log-beta N(0, 0.1).
+WEIGHT_STD = 0.02
+BIAS_STD = 0.02
+SNAKE_STD = 0.1
+
+
+def _draw_params(stream: NormalStream, layout) -> np.ndarray:
+    total = sum(int(np.prod(s)) for _, s, _ in layout)
+    flat = np.empty(total, np.float32)
+    off = 0
+    for _, shape, kind in layout:
+        n = int(np.prod(shape))
+        std = {"w": WEIGHT_STD, "b": BIAS_STD, "snake": SNAKE_STD}[kind]
+        flat[off:off + n] = stream.normal((n,), 0.0, std)
+        off += n
+    return flat
+
+
+# ---------------------------------------------------------------- workloads
+
+H3 = DecoderGeometry(
+    in_channels=32, pre_channels=1536, pre_kernel=7,
+    up_rates=(5, 5, 2, 2, 2, 2, 2), up_kernels=(10, 10, 4, 4, 4, 4, 4),
+    up_channels=(768, 384, 192, 96, 48, 24, 12),
+    block_kernels=(3, 7, 11), dilations=(1, 3, 5),
+    post_kernel=7, out_channels=1, final_act="tanh", sample_rate=32000)
+
+LTX = DecoderGeometry(
+    in_channels=64, pre_channels=1024, pre_kernel=7,
+    up_rates=(5, 2, 2, 2, 2, 2), up_kernels=(10, 4, 4, 4, 4, 4),
+    up_channels=(512, 256, 128, 64, 32, 16),
+    block_kernels=(3, 7, 11), dilations=(1, 3, 5),
+    post_kernel=7, out_channels=1, final_act="clamp", sample_rate=16000)
+
+
+@dataclass(frozen=True)
+class DecoderWorkload:
+    name: str
+    geometry: DecoderGeometry
+    batch: int
+    frames: int
+    seed: int
+    input_mean: float = 0.0
+    input_std: float = 1.0
+    tile_frames: int = 0
+    overlap_frames: int = 0
+
+    def audio_seconds(self) -> float:
+        """Seconds of audio per side (stereo counts once)."""
+        return self.frames * self.geometry.hop / self.geometry.sample_rate
+
+    def make(self):
+        """(z [B, in_ch, frames], flat params) drawn from this workload's seed."""
+        s = NormalStream(self.seed)
+        z = s.normal((self.batch, self.geometry.in_channels, self.frames),
+                     self.input_mean, self.input_std)
+        return z, _draw_params(s, param_layout(self.geometry))
+
+
+@dataclass(frozen=True)
+class AmpWorkload:
+    name: str
+    batch: int
+    channels: int
+    length: int
+    kernel: int
+    dilations: Tuple[int, ...]
+    seed: int
+
+    def layout(self):
+        C, K = self.channels, self.kernel
+        out = []
+        for u, _ in enumerate(self.dilations):
+            out += [(f"unit{u}.act1.log_alpha", (C,), "snake"),
+                    (f"unit{u}.act1.log_beta", (C,), "snake"),
+                    (f"unit{u}.conv1.w", (C, C, K), "w"), (f"unit{u}.conv1.b", (C,), "b"),
+                    (f"unit{u}.act2.log_alpha", (C,), "snake"),
+                    (f"unit{u}.act2.log_beta", (C,), "snake"),
+                    (f"unit{u}.conv2.w", (C, C, K), "w"), (f"unit{u}.conv2.b", (C,), "b")]
+        return out
+
+    def make(self):
+        s = NormalStream(self.seed)
+        x = s.normal((self.batch, self.channels, self.length))
+        return x, _draw_params(s, self.layout())
+
+
+@dataclass(frozen=True)
+class ActivationWorkload:
+    name: str
+    batch: int
+    channels: int
+    length: int
+    seed: int
+
+    def make(self):
+        s = NormalStream(self.seed)
+        x = s.normal((self.batch, self.channels, self.length))
+        la = s.normal((self.channels,), 0.0, SNAKE_STD)
+        lb = s.normal((self.channels,), 0.0, SNAKE_STD)
+        return x, la, lb
+
+
+AMP_BLOCK_C32 = AmpWorkload("amp_block_c32_t8192", 1, 32, 8192, 3, (1, 3, 5), seed=0)
+ACT_SWEEP = ActivationWorkload("activation_c512_t65536", 2, 512, 65536, seed=1)
+ACT_SWEEP_GRID = [(c, t) for c in (64, 128, 256, 512, 768, 1024, 1536)
+                  for t in (4096, 16384, 65536, 262144)]
+H3_10S = DecoderWorkload("h3_decoder_10s_stereo", H3, 2, 400, seed=2)
+LTX_VOCODER = DecoderWorkload("ltx_vocoder_500f_stereo", LTX, 2, 500, seed=3,
+                              input_mean=-4.0, input_std=2.0)
+H3_60S_TILED = DecoderWorkload("h3_decoder_60s_stereo_tiled", H3, 2, 2400, seed=4,
+                               tile_frames=200, overlap_frames=16)
+
+DECODER_WORKLOADS = {w.name: w for w in (H3_10S, LTX_VOCODER, H3_60S_TILED)}
+
+
+def tiny_geometry(**kw) -> DecoderGeometry:
+    """A small decoder with the same structure, for tests the oracle runs in
+    seconds (both stride parities, several blocks and dilations)."""
+    base = DecoderGeometry(
+        in_channels=8, pre_channels=48, pre_kernel=7,
+        up_rates=(5, 2, 2), up_kernels=(10, 4, 4), up_channels=(32, 16, 8),
+        block_kernels=(3, 7, 11), dilations=(1, 3, 5),
+        post_kernel=7, out_channels=1, final_act="tanh", sample_rate=32000)
+    return base.replace(**kw)

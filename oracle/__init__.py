@@ -1,0 +1,284 @@
+"""Parity oracle for the BigVGAN alias-free decoder (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the bench's CPU-baseline
+leg may import this package.  It is a plain single-threaded C statement of
+the decoder (``bv_oracle.c``) that accumulates in double, loaded through
+ctypes; it shares nothing with the CUDA library.
+
+Functions take and return numpy float32 arrays in [B, C, T] layout.  The
+decoder geometry is passed as a mapping or an object with the attributes
+``in_channels, pre_channels, pre_kernel, up_rates, up_kernels, up_channels,
+block_kernels, dilations, post_kernel, out_channels, final_act``.
+
+Sources: docs.rs cortiq-engine 0.5.74 ``audiovae.rs`` (MiniMax-H3 BigVGAN),
+0.6.3 ``ltxaudio.rs`` (LTX-2.5 BigVGAN v2), 0.5.89 ``music3.rs`` (windowing).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_LIB = None
+
+_f32p = ctypes.POINTER(ctypes.c_float)
+_f64p = ctypes.POINTER(ctypes.c_double)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_i32p = ctypes.POINTER(ctypes.c_int)
+
+FINAL_ACTS = {"none": 0, "clamp": 1, "tanh": 2}
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.orc_bessel_i0.restype = ctypes.c_double
+        L.orc_bessel_i0.argtypes = [ctypes.c_double]
+        L.orc_sinc.restype = ctypes.c_double
+        L.orc_sinc.argtypes = [ctypes.c_double]
+        L.orc_kaiser_sinc.argtypes = [ctypes.c_double, ctypes.c_double, ctypes.c_int, _f64p]
+        L.orc_activation1d.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       _f32p, _f32p, _f32p, _f32p, ctypes.c_int,
+                                       ctypes.c_double, ctypes.c_int, _f32p]
+        L.orc_conv1d.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
+                                 _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_int, ctypes.c_int, _f32p]
+        L.orc_conv_transpose1d.argtypes = L.orc_conv1d.argtypes
+        L.orc_conv1d_points.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                        _f32p, _f32p, ctypes.c_int, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int, _i64p, ctypes.c_int,
+                                        _f64p]
+        L.orc_conv_transpose1d_points.argtypes = L.orc_conv1d_points.argtypes
+        L.orc_activation1d_points.argtypes = [_f32p, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, _f32p, _f32p, _f32p, _f32p,
+                                              ctypes.c_int, ctypes.c_double, _i64p,
+                                              ctypes.c_int, _f64p]
+        L.orc_decoder_param_count.restype = ctypes.c_long
+        L.orc_decoder_param_count.argtypes = [_i32p]
+        L.orc_decoder_hop.restype = ctypes.c_long
+        L.orc_decoder_hop.argtypes = [_i32p]
+        L.orc_decoder_raw_len.restype = ctypes.c_long
+        L.orc_decoder_raw_len.argtypes = [_i32p, ctypes.c_int]
+        L.orc_decode.argtypes = [_i32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, _f32p,
+                                 _f32p, ctypes.c_int, ctypes.c_double, ctypes.c_int, _f32p]
+        L.orc_decode_tiled.argtypes = [_i32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, _f32p, _f32p, ctypes.c_int,
+                                       ctypes.c_double, ctypes.c_int, _f32p, _f32p]
+        L.orc_tile_count.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        _LIB = L
+    return _LIB
+
+
+def _f32(a):
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _p32(a):
+    return None if a is None else a.ctypes.data_as(_f32p)
+
+
+def _check(rc, what):
+    if rc != 0:
+        raise ValueError(f"oracle {what} failed with code {rc}")
+
+
+# ------------------------------------------------------------------ filter
+
+
+def bessel_i0(x: float) -> float:
+    return lib().orc_bessel_i0(float(x))
+
+
+def sinc(x: float) -> float:
+    return lib().orc_sinc(float(x))
+
+
+def kaiser_sinc_f64(cutoff=0.25, half_width=0.3, k=12) -> np.ndarray:
+    out = np.zeros(k, np.float64)
+    _check(lib().orc_kaiser_sinc(cutoff, half_width, k, out.ctypes.data_as(_f64p)),
+           "kaiser_sinc")
+    return out
+
+
+def kaiser_sinc(cutoff=0.25, half_width=0.3, k=12) -> np.ndarray:
+    """The designed filter as the pages hand it out: float taps."""
+    return kaiser_sinc_f64(cutoff, half_width, k).astype(np.float32)
+
+
+# ------------------------------------------------------------------ layers
+
+
+def activation1d(x, log_alpha, log_beta, up=None, down=None, eps=1e-9, store_f64=False):
+    x = _f32(x)
+    B, C, T = x.shape
+    up = kaiser_sinc() if up is None else _f32(up)
+    down = up if down is None else _f32(down)
+    la, lb = _f32(log_alpha), _f32(log_beta)
+    y = np.empty_like(x)
+    _check(lib().orc_activation1d(_p32(x), B, C, T, _p32(la), _p32(lb), _p32(up),
+                                  _p32(down), len(up), eps, int(store_f64), _p32(y)),
+           "activation1d")
+    return y
+
+
+def conv1d(x, w, bias, dilation=1, pad=None, store_f64=False):
+    x, w = _f32(x), _f32(w)
+    B, Cin, T = x.shape
+    Cout, Cin2, K = w.shape
+    assert Cin2 == Cin
+    if pad is None:
+        pad = (K * dilation - dilation) // 2
+    Tout = T + 2 * pad - dilation * (K - 1)
+    b = None if bias is None else _f32(bias)
+    y = np.empty((B, Cout, Tout), np.float32)
+    _check(lib().orc_conv1d(_p32(x), B, Cin, T, _p32(w), _p32(b), Cout, K, dilation,
+                            pad, int(store_f64), _p32(y)), "conv1d")
+    return y
+
+
+def conv_transpose1d(x, w, bias, stride, pad=None, store_f64=False):
+    x, w = _f32(x), _f32(w)
+    B, Cin, T = x.shape
+    Cin2, Cout, K = w.shape
+    assert Cin2 == Cin
+    if pad is None:
+        pad = (K - stride) // 2
+    Tout = (T - 1) * stride + K - 2 * pad
+    b = None if bias is None else _f32(bias)
+    y = np.empty((B, Cout, Tout), np.float32)
+    _check(lib().orc_conv_transpose1d(_p32(x), B, Cin, T, _p32(w), _p32(b), Cout, K,
+                                      stride, pad, int(store_f64), _p32(y)),
+           "conv_transpose1d")
+    return y
+
+
+def _idx(points):
+    idx = np.ascontiguousarray(np.asarray(points, dtype=np.int64).reshape(-1, 3))
+    return idx, idx.shape[0]
+
+
+def conv1d_points(x, w, bias, dilation, pad, points):
+    x, w = _f32(x), _f32(w)
+    B, Cin, T = x.shape
+    Cout, _, K = w.shape
+    b = None if bias is None else _f32(bias)
+    idx, n = _idx(points)
+    out = np.empty(n, np.float64)
+    _check(lib().orc_conv1d_points(_p32(x), B, Cin, T, _p32(w), _p32(b), Cout, K,
+                                   dilation, pad, idx.ctypes.data_as(_i64p), n,
+                                   out.ctypes.data_as(_f64p)), "conv1d_points")
+    return out
+
+
+def conv_transpose1d_points(x, w, bias, stride, pad, points):
+    x, w = _f32(x), _f32(w)
+    B, Cin, T = x.shape
+    _, Cout, K = w.shape
+    b = None if bias is None else _f32(bias)
+    idx, n = _idx(points)
+    out = np.empty(n, np.float64)
+    _check(lib().orc_conv_transpose1d_points(_p32(x), B, Cin, T, _p32(w), _p32(b), Cout,
+                                             K, stride, pad, idx.ctypes.data_as(_i64p), n,
+                                             out.ctypes.data_as(_f64p)),
+           "conv_transpose1d_points")
+    return out
+
+
+def activation1d_points(x, log_alpha, log_beta, points, up=None, down=None, eps=1e-9):
+    x = _f32(x)
+    B, C, T = x.shape
+    up = kaiser_sinc() if up is None else _f32(up)
+    down = up if down is None else _f32(down)
+    la, lb = _f32(log_alpha), _f32(log_beta)
+    idx, n = _idx(points)
+    out = np.empty(n, np.float64)
+    _check(lib().orc_activation1d_points(_p32(x), B, C, T, _p32(la), _p32(lb), _p32(up),
+                                         _p32(down), len(up), eps,
+                                         idx.ctypes.data_as(_i64p), n,
+                                         out.ctypes.data_as(_f64p)), "activation1d_points")
+    return out
+
+
+# ----------------------------------------------------------------- decoder
+
+
+def _get(geo, name):
+    return geo[name] if isinstance(geo, dict) else getattr(geo, name)
+
+
+def geometry_ints(geo) -> np.ndarray:
+    g = np.zeros(41, np.int32)
+    rates, upk, upch = (list(_get(geo, n)) for n in ("up_rates", "up_kernels", "up_channels"))
+    bk, dil = list(_get(geo, "block_kernels")), list(_get(geo, "dilations"))
+    fa = _get(geo, "final_act")
+    g[0], g[1], g[2], g[3] = (_get(geo, "in_channels"), _get(geo, "pre_channels"),
+                              _get(geo, "pre_kernel"), len(rates))
+    g[4:4 + len(rates)] = rates
+    g[12:12 + len(upk)] = upk
+    g[20:20 + len(upch)] = upch
+    g[28] = len(bk)
+    g[29:29 + len(bk)] = bk
+    g[33] = len(dil)
+    g[34:34 + len(dil)] = dil
+    g[38], g[39] = _get(geo, "post_kernel"), _get(geo, "out_channels")
+    g[40] = FINAL_ACTS[fa] if isinstance(fa, str) else int(fa)
+    return g
+
+
+def param_count(geo) -> int:
+    g = geometry_ints(geo)
+    n = lib().orc_decoder_param_count(g.ctypes.data_as(_i32p))
+    if n < 0:
+        raise ValueError("bad decoder geometry")
+    return int(n)
+
+
+def hop(geo) -> int:
+    g = geometry_ints(geo)
+    return int(lib().orc_decoder_hop(g.ctypes.data_as(_i32p)))
+
+
+def raw_len(geo, frames) -> int:
+    g = geometry_ints(geo)
+    return int(lib().orc_decoder_raw_len(g.ctypes.data_as(_i32p), int(frames)))
+
+
+def decode(geo, params, z, filt=None, eps=1e-9, store_f64=False):
+    """z [B, in_ch, frames] -> waveform [B, out_ch, frames * hop]."""
+    g = geometry_ints(geo)
+    z, params = _f32(z), _f32(params)
+    if params.size != param_count(geo):
+        raise ValueError(f"params has {params.size} values, geometry needs {param_count(geo)}")
+    B, _, F = z.shape
+    f = kaiser_sinc() if filt is None else _f32(filt)
+    y = np.empty((B, int(g[39]), F * hop(geo)), np.float32)
+    _check(lib().orc_decode(g.ctypes.data_as(_i32p), _p32(params), _p32(z), B, F,
+                            _p32(f), _p32(f), len(f), eps, int(store_f64), _p32(y)),
+           "decode")
+    return y
+
+
+def tile_count(frames, tile, overlap) -> int:
+    return int(lib().orc_tile_count(int(frames), int(tile), int(overlap)))
+
+
+def decode_tiled(geo, params, z, tile, overlap, tiles=None, filt=None, eps=1e-9,
+                 store_f64=False):
+    """Tiled decode; ``tiles=(lo, hi)`` restricts which tiles are decoded (the
+    samples no chosen tile covers come back as NaN).  Returns (y, count)."""
+    g = geometry_ints(geo)
+    z, params = _f32(z), _f32(params)
+    B, _, F = z.shape
+    lo, hi = (0, tile_count(F, tile, overlap)) if tiles is None else tiles
+    f = kaiser_sinc() if filt is None else _f32(filt)
+    L = F * hop(geo)
+    y = np.empty((B, int(g[39]), L), np.float32)
+    cnt = np.empty(L, np.float32)
+    _check(lib().orc_decode_tiled(g.ctypes.data_as(_i32p), _p32(params), _p32(z), B, F,
+                                  tile, overlap, lo, hi, _p32(f), _p32(f), len(f), eps,
+                                  int(store_f64), _p32(y), _p32(cnt)), "decode_tiled")
+    return y, cnt
