@@ -1,0 +1,339 @@
+#!/usr/bin/env python
+"""Decoder throughput on B200: seconds of audio decoded per second.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   # the plain CPU oracle, timed on the host
+
+One step = one whole decode (conv_pre, every ConvT stage with its AMP blocks,
+act_post, conv_post, final op) of one batch of the workload, weights and
+latent resident in HBM.  With N > 1 (torchrun) every rank decodes its own
+batch on its own GPU (independent replicas, no collective on the data path);
+the step time is the max over ranks.  Prints one JSON line on rank 0.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from bigvgan_waveform_decoder_alias_b200 import synth  # noqa: E402
+
+METRIC = "audio-seconds decoded per second (1 B200); activation GB/s and conv pipe % of peak"
+UNIT = "audio_s/s"
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=synth.H3_10S.name, choices=sorted(synth.DECODER_WORKLOADS))
+    ap.add_argument("--cpu-sample-frames", type=int, default=12,
+                    help="latent frames (one side) of the oracle's timed sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d.get("hbm_gbs", 6650.0), d.get("sm_max_mhz", 1965.0), "measured"
+    return 6650.0, 1965.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_baseline(workload, frames, steps=1):
+    """The oracle as it stands, single-threaded, on a bounded sample: one side
+    of the workload's decoder on its first `frames` latent frames."""
+    import oracle
+    z, params = workload.make()
+    zs = np.ascontiguousarray(z[:1, :, :frames])
+    oracle.decode(workload.geometry, params, zs)  # warm the library and caches
+    times = []
+    for _ in range(steps):
+        t = time.perf_counter()
+        oracle.decode(workload.geometry, params, zs)
+        times.append(time.perf_counter() - t)
+    audio = frames * workload.geometry.hop / workload.geometry.sample_rate
+    return audio / statistics.mean(times), times, audio
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = synth.DECODER_WORKLOADS[args.workload]
+    import oracle
+    z, params = w.make()
+    frames = 3
+    zs = np.ascontiguousarray(z[:1, :, :frames])
+    audio = frames * w.geometry.hop / w.geometry.sample_rate
+    for _ in range(args.warmup):
+        oracle.decode(w.geometry, params, zs)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        oracle.decode(w.geometry, params, zs)
+        times.append(time.perf_counter() - t)
+    value = audio / statistics.mean(times)
+    sample = (f"oracle decode of one side, first {frames} latent frames "
+              f"({audio:.3f} s of audio) of {w.name}")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * statistics.mean(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": 1, "frames": frames},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_init()
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+
+    import torch
+    import torch.distributed as dist
+    from bigvgan_waveform_decoder_alias_b200 import native
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    w = synth.DECODER_WORKLOADS[args.workload]
+    z, params = w.make()
+    if rank > 0:  # each replica decodes its own latent
+        z = synth.NormalStream(w.seed + 1000 * rank).normal(z.shape, w.input_mean, w.input_std)
+    dec = native.Decoder(w.geometry, params, tile_frames=w.tile_frames,
+                         overlap_frames=w.overlap_frames, device=dev)
+    zd = torch.from_numpy(z).to(dev)
+    B, _, F = z.shape
+    L = dec.output_length(F)
+    y = torch.empty((B, w.geometry.out_channels, L), device=dev)
+    ws = dec.workspace(B, F)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(max(args.warmup, 3)):
+        dec.decode(zd, y=y, workspace=ws)
+    torch.cuda.synchronize()
+
+    # ---------------------------------------------------------- timed region
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    n0 = native.launch_count()
+    with ClockSampler(dev.index) as clk:
+        for k in range(args.steps):
+            flush.fill_(float(k))  # evict L2 between steps, outside the events
+            ev[k][0].record(stream)
+            dec.decode(zd, y=y, workspace=ws)
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = native.launch_count() - n0
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    audio_per_step = w.audio_seconds()
+    value = world * audio_per_step / (ms_per_step / 1000.0)
+    y_check = y.detach().float()
+    finite = bool(torch.isfinite(y_check).all().item())
+
+    # -------------------------------------------- end to end through host memory
+    zh = torch.from_numpy(z).pin_memory()
+    yh = torch.empty((B, w.geometry.out_channels, L), dtype=torch.float32).pin_memory()
+    wsh = dec.workspace(B, F, host=True)
+    dec.decode_host(zh, yh, workspace=wsh)
+    torch.cuda.synchronize()
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        ev2[k][0].record(stream)
+        dec.decode_host(zh, yh, workspace=wsh)
+        ev2[k][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = world * audio_per_step / (e2e_ms / args.steps / 1000.0)
+
+    # ----------------------------------------- per-kernel timing (roofline)
+    import ctypes
+    Lb = native.lib()
+    Lb.bv_timing_enable(1)
+    Lb.bv_timing_reset()
+    prof_steps = min(args.steps, 5)
+    for k in range(prof_steps):
+        flush.fill_(float(k))
+        dec.decode(zd, y=y, workspace=ws)
+    torch.cuda.synchronize()
+    Stats = native.KernelStats * 16
+    st = Stats()
+    n = Lb.bv_timing_read(st, 16)
+    Lb.bv_timing_enable(0)
+    kernels = {}
+    for i in range(max(n, 0)):
+        s = st[i]
+        kernels[s.name.decode()] = {"launches_per_step": s.launches / prof_steps,
+                                    "ms_per_step": s.ms / prof_steps,
+                                    "flops": s.flops / max(s.launches, 1),
+                                    "bytes": s.bytes / max(s.launches, 1),
+                                    "avg_launch_ms": s.ms / max(s.launches, 1)}
+    hbm, sm_max_mhz, src = peaks()
+    fp32_peak = SMS * FP32_LANES_PER_SM * 2 * sm_max_mhz * 1e6 / 1e12  # TFLOP/s
+    dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
+    roof = None
+    if dom:
+        kd = kernels[dom]
+        if kd["flops"] > 0:
+            ach = kd["flops"] / (kd["avg_launch_ms"] / 1000.0) / 1e12
+            roof = {"kernel": dom, "bound": "alu", "achieved": ach, "peak": fp32_peak,
+                    "unit": "TFLOP/s", "frac": ach / fp32_peak, "traffic": None,
+                    "peak_source": f"FP32 pipe: {SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 x "
+                                   f"{sm_max_mhz:.0f} MHz"}
+        else:
+            ach = kd["bytes"] / (kd["avg_launch_ms"] / 1000.0) / 1e9
+            roof = {"kernel": dom, "bound": "hbm", "achieved": ach, "peak": hbm,
+                    "unit": "GB/s", "frac": ach / hbm, "traffic": None,
+                    "peak_source": f"{src} hbm_gbs"}
+    act = None
+    if "activation" in kernels:
+        ka = kernels["activation"]
+        gbs = ka["bytes"] / (ka["avg_launch_ms"] / 1000.0) / 1e9
+        act = {"achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, times, audio = cpu_baseline(w, args.cpu_sample_frames)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"oracle decode of one side, first {args.cpu_sample_frames} latent "
+                         f"frames ({audio:.3f} s of audio) of {w.name}, "
+                         f"{statistics.mean(times):.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "frames": F,
+                       "audio_seconds_per_step": audio_per_step,
+                       "sample_rate": w.geometry.sample_rate,
+                       "l2": "flushed between steps (256 MiB write outside the timed events)",
+                       "parallelism": f"replicas x{world}"},
+            "e2e": {"value": e2e_value, "unit": UNIT,
+                    "h2d_bytes_per_step": int(zh.numel() * 4),
+                    "d2h_bytes_per_step": int(yh.numel() * 4)},
+            "gpu_launches": int(launches),
+            "roofline": roof,
+            "activation": act,
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "clocks": clk.summary(),
+            "output_finite": finite,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,724 @@
+// The C ABI of libbv: argument checks, the filter design, and the host-side
+// orchestration of the AMP block and the decoder.  Every step of the
+// computation runs in the CUDA kernels of this library.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "bv.h"
+#include "common.cuh"
+#include "tiles.cuh"
+
+#define BV_VERSION "bv 0.1.0 (sm_100a)"
+
+namespace bv {
+
+namespace {
+thread_local char g_err[512] = "";
+uint64_t g_launches = 0;
+}  // namespace
+
+__device__ int g_device_status = 0;
+
+int *device_status_ptr() {
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+  return static_cast<int *>(p);
+}
+
+bv_status fail(bv_status st, const char *fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+bv_status check_launch(const char *what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(BV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return BV_OK;
+}
+
+void count_launch(uint64_t n) { __atomic_fetch_add(&g_launches, n, __ATOMIC_RELAXED); }
+
+// ------------------------------------------------------------ launch timing
+
+namespace {
+struct TimerRec {
+  std::string cls;
+  cudaEvent_t start = nullptr, stop = nullptr;
+  double flops = 0, bytes = 0;
+  bool used = false;
+};
+std::atomic<bool> g_timing_on{false};
+std::mutex g_timer_mu;
+std::vector<TimerRec> g_timers;
+size_t g_timer_next = 0;  // records [0, next) are live
+}  // namespace
+
+LaunchTimer::LaunchTimer(cudaStream_t st, const char *cls, double flops, double bytes) : st_(st) {
+  if (!g_timing_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_timer_mu);
+  if (g_timer_next == g_timers.size()) {
+    TimerRec r;
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) {
+      cudaGetLastError();
+      return;
+    }
+    g_timers.push_back(r);
+  }
+  TimerRec &r = g_timers[g_timer_next];
+  r.cls = cls;
+  r.flops = flops;
+  r.bytes = bytes;
+  r.used = true;
+  slot_ = (int)g_timer_next++;
+  cudaEventRecord(r.start, st_);
+}
+
+LaunchTimer::~LaunchTimer() {
+  if (slot_ < 0) return;
+  std::lock_guard<std::mutex> lk(g_timer_mu);
+  cudaEventRecord(g_timers[slot_].stop, st_);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+// The current device must be an sm_100 part; checked once per device.
+bv_status check_device() {
+  static int ok_mask = 0;  // bit per device id < 32 that passed
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(BV_ERR_CUDA, "no CUDA device: %s", cudaGetErrorString(e));
+  if (dev < 32 && (ok_mask >> dev) & 1) return BV_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10)
+    return fail(BV_ERR_CUDA, "device %d is sm_%d%d; this library is built for sm_100a", dev,
+                major, minor);
+  if (dev < 32) ok_mask |= 1 << dev;
+  return BV_OK;
+}
+
+#define BV_TRY(expr)                 \
+  do {                               \
+    bv_status _s = (expr);           \
+    if (_s != BV_OK) return _s;      \
+  } while (0)
+
+// ------------------------------------------------------------- filter design
+
+// Modified Bessel I0 by its power series; terms (x/2)^{2k}/(k!)^2 accumulate
+// until they fall below 1e-18 of the sum (at most 39 of them).
+double bessel_i0(double x) {
+  double s = 1.0, term = 1.0;
+  const double h = 0.5 * x;
+  for (int k = 1; k <= 39; ++k) {
+    term *= (h / k) * (h / k);
+    s += term;
+    if (term < 1e-18 * s) break;
+  }
+  return s;
+}
+
+double sinc_pi(double v) { return v == 0.0 ? 1.0 : std::sin(M_PI * v) / (M_PI * v); }
+
+}  // namespace
+}  // namespace bv
+
+using namespace bv;
+
+extern "C" {
+
+const char *bv_last_error(void) { return g_err; }
+
+const char *bv_version(void) { return BV_VERSION; }
+
+uint64_t bv_launch_count(void) { return __atomic_load_n(&g_launches, __ATOMIC_RELAXED); }
+
+void bv_timing_enable(int on) { g_timing_on.store(on != 0); }
+
+void bv_timing_reset(void) {
+  std::lock_guard<std::mutex> lk(g_timer_mu);
+  g_timer_next = 0;
+}
+
+int bv_timing_read(bv_kernel_stats *out, int max) {
+  std::lock_guard<std::mutex> lk(g_timer_mu);
+  std::map<std::string, bv_kernel_stats> acc;
+  for (size_t i = 0; i < g_timer_next; ++i) {
+    TimerRec &r = g_timers[i];
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) return -1;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) return -1;
+    bv_kernel_stats &k = acc[r.cls];
+    if (k.launches == 0) {
+      std::memset(&k, 0, sizeof(k));
+      snprintf(k.name, sizeof(k.name), "%s", r.cls.c_str());
+    }
+    k.launches += 1;
+    k.ms += ms;
+    k.flops += r.flops;
+    k.bytes += r.bytes;
+  }
+  int n = 0;
+  for (auto &kv : acc) {
+    if (n < max && out) out[n] = kv.second;
+    ++n;
+  }
+  return n;
+}
+
+bv_status bv_sync_status(void *stream) {
+  g_err[0] = 0;
+  BV_TRY(check_device());
+  int h = 0;
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemcpyFromSymbolAsync(&h, g_device_status, sizeof(int), 0,
+                                            cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return fail(BV_ERR_CUDA, "bv_sync_status: %s", cudaGetErrorString(e));
+  if (h != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
+    cudaStreamSynchronize(st);
+    return fail(BV_ERR_TIMEOUT, "a bounded device wait gave up (code %d)", h);
+  }
+  return BV_OK;
+}
+
+bv_status bv_filter_design(double cutoff, double half_width, int taps, float *out_host) {
+  g_err[0] = 0;
+  if (!out_host) return fail(BV_ERR_ARG, "bv_filter_design: null output");
+  if (taps < 1 || taps > 64) return fail(BV_ERR_ARG, "bv_filter_design: taps %d", taps);
+  if (!(cutoff > 0.0 && cutoff <= 0.5) || !(half_width > 0.0))
+    return fail(BV_ERR_ARG, "bv_filter_design: cutoff %g half_width %g", cutoff, half_width);
+  // Kaiser's attenuation estimate and beta for a transition of 4 half_width
+  const int half = taps / 2;
+  const double atten = 2.285 * (half - 1) * M_PI * (4.0 * half_width) + 7.95;
+  double beta = 0.0;
+  if (atten > 50.0) beta = 0.1102 * (atten - 8.7);
+  else if (atten >= 21.0) beta = 0.5842 * std::pow(atten - 21.0, 0.4) + 0.07886 * (atten - 21.0);
+  const double i0b = bessel_i0(beta);
+  const double centre = (taps % 2 == 0) ? half - 0.5 : (double)half;
+  std::vector<double> f(taps);
+  double total = 0.0;
+  for (int i = 0; i < taps; ++i) {
+    const double r = taps > 1 ? 2.0 * i / (taps - 1) - 1.0 : 0.0;
+    const double win = bessel_i0(beta * std::sqrt(std::fmax(0.0, 1.0 - r * r))) / i0b;
+    f[i] = 2.0 * cutoff * win * sinc_pi(2.0 * cutoff * (i - centre));
+    total += f[i];
+  }
+  for (int i = 0; i < taps; ++i) out_host[i] = (float)(f[i] / total);
+  return BV_OK;
+}
+
+bv_status bv_activation1d(const float *x, float *y, int B, int C, int T, const float *log_alpha,
+                          const float *log_beta, const float *up_filter,
+                          const float *down_filter, float eps, void *stream) {
+  g_err[0] = 0;
+  if (!x || !y || !log_alpha || !log_beta || !up_filter || !down_filter)
+    return fail(BV_ERR_ARG, "bv_activation1d: null pointer");
+  if (B < 1 || C < 1 || T < 1) return fail(BV_ERR_SHAPE, "bv_activation1d: B=%d C=%d T=%d", B, C, T);
+  const size_t n = (size_t)B * C * T;
+  if (n >= (1ull << 40)) return fail(BV_ERR_SHAPE, "bv_activation1d: tensor too large");
+  if (!aligned4(x) || !aligned4(y)) return fail(BV_ERR_ARG, "bv_activation1d: misaligned pointer");
+  if (overlaps(x, n, y, n)) return fail(BV_ERR_ARG, "bv_activation1d: x and y overlap");
+  BV_TRY(check_device());
+  return launch_activation(x, y, B, C, T, log_alpha, log_beta, up_filter, down_filter, eps,
+                           as_stream(stream));
+}
+
+bv_status bv_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
+                    int Cout, int K, int dilation, int pad, const bv_epilogue *ep, float *y,
+                    void *stream) {
+  g_err[0] = 0;
+  if (!x || !w || !y) return fail(BV_ERR_ARG, "bv_conv1d: null pointer");
+  if (B < 1 || Cin < 1 || T < 1 || Cout < 1 || K < 1 || K > 32 || dilation < 1 || pad < 0)
+    return fail(BV_ERR_SHAPE, "bv_conv1d: B=%d Cin=%d T=%d Cout=%d K=%d d=%d pad=%d", B, Cin, T,
+                Cout, K, dilation, pad);
+  const long long Tout = (long long)T + 2LL * pad - (long long)dilation * (K - 1);
+  if (Tout < 1 || Tout > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "bv_conv1d: output length %lld", Tout);
+  const size_t nin = (size_t)B * Cin * T, nout = (size_t)B * Cout * Tout;
+  if (overlaps(x, nin, y, nout)) return fail(BV_ERR_ARG, "bv_conv1d: x and y overlap");
+  Epi e{nullptr, 1.0f, 0, 0};
+  if (ep) {
+    e.residual = ep->residual;
+    e.scale = ep->scale;
+    e.accumulate = ep->accumulate ? 1 : 0;
+    e.final_act = ep->final_act;
+    if (e.final_act < 0 || e.final_act > 2) return fail(BV_ERR_ARG, "bv_conv1d: final_act %d", e.final_act);
+    if (e.residual && e.residual != y && overlaps(e.residual, nout, y, nout))
+      return fail(BV_ERR_ARG, "bv_conv1d: residual partially overlaps y");
+  }
+  BV_TRY(check_device());
+  return launch_conv1d(x, B, Cin, T, w, bias, Cout, K, dilation, pad, e, y, (int)Tout, (int)Tout,
+                       as_stream(stream));
+}
+
+bv_status bv_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,
+                              const float *bias, int Cout, int K, int stride, int pad, float *y,
+                              void *stream) {
+  g_err[0] = 0;
+  if (!x || !w || !y) return fail(BV_ERR_ARG, "bv_conv_transpose1d: null pointer");
+  if (B < 1 || Cin < 1 || T < 1 || Cout < 1 || K < 1 || K > 64 || stride < 1 || stride > 16 ||
+      pad < 0)
+    return fail(BV_ERR_SHAPE, "bv_conv_transpose1d: B=%d Cin=%d T=%d Cout=%d K=%d s=%d pad=%d",
+                B, Cin, T, Cout, K, stride, pad);
+  const long long Tout = (long long)(T - 1) * stride + K - 2LL * pad;
+  if (Tout < 1 || Tout > 0x7fffffffLL)
+    return fail(BV_ERR_SHAPE, "bv_conv_transpose1d: output length %lld", Tout);
+  if (overlaps(x, (size_t)B * Cin * T, y, (size_t)B * Cout * Tout))
+    return fail(BV_ERR_ARG, "bv_conv_transpose1d: x and y overlap");
+  BV_TRY(check_device());
+  return launch_conv_transpose1d(x, B, Cin, T, w, bias, Cout, K, stride, pad, y,
+                                 as_stream(stream));
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------- AMP block
+
+namespace bv {
+namespace {
+
+bv_status check_amp_params(const bv_amp_params *p, int C) {
+  (void)C;
+  if (!p) return fail(BV_ERR_ARG, "amp block: null params");
+  if (p->kernel_size < 1 || p->kernel_size % 2 == 0 || p->kernel_size > 32)
+    return fail(BV_ERR_SHAPE, "amp block: kernel_size %d (odd, <= 31)", p->kernel_size);
+  if (p->n_dilations < 1 || p->n_dilations > BV_MAX_DIL)
+    return fail(BV_ERR_SHAPE, "amp block: n_dilations %d", p->n_dilations);
+  if (!p->up_filter || !p->down_filter) return fail(BV_ERR_ARG, "amp block: null filter");
+  for (int u = 0; u < p->n_dilations; ++u) {
+    if (p->dilation[u] < 1) return fail(BV_ERR_SHAPE, "amp block: dilation %d", p->dilation[u]);
+    if (!p->conv1_w[u] || !p->conv2_w[u] || !p->act_log_alpha[2 * u] ||
+        !p->act_log_beta[2 * u] || !p->act_log_alpha[2 * u + 1] || !p->act_log_beta[2 * u + 1])
+      return fail(BV_ERR_ARG, "amp block: null weight in unit %d", u);
+  }
+  return BV_OK;
+}
+
+struct AmpScratch {
+  float *cur, *h1, *h2;
+};
+
+// y = (accumulate ? y : 0) + scale * AMP(x); x, y and the scratch are disjoint.
+bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params &p, float *y,
+                        float scale, int accumulate, const AmpScratch &s, cudaStream_t st) {
+  const int K = p.kernel_size, n = p.n_dilations;
+  const float eps = 1e-9f;
+  for (int u = 0; u < n; ++u) {
+    const float *src = (u == 0) ? x : s.cur;
+    const int d = p.dilation[u];
+    BV_TRY(launch_activation(src, s.h1, B, C, T, p.act_log_alpha[2 * u], p.act_log_beta[2 * u],
+                             p.up_filter, p.down_filter, eps, st));
+    Epi plain{nullptr, 1.0f, 0, 0};
+    BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv1_w[u], p.conv1_b[u], C, K, d, (K * d - d) / 2,
+                         plain, s.h2, T, T, st));
+    BV_TRY(launch_activation(s.h2, s.h1, B, C, T, p.act_log_alpha[2 * u + 1],
+                             p.act_log_beta[2 * u + 1], p.up_filter, p.down_filter, eps, st));
+    if (u == n - 1) {
+      Epi last{src, scale, accumulate, 0};
+      BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, last,
+                           y, T, T, st));
+    } else {
+      Epi res{src, 1.0f, 0, 0};  // cur = src + conv2(...); src may be cur itself
+      BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, res,
+                           s.cur, T, T, st));
+    }
+  }
+  return BV_OK;
+}
+
+}  // namespace
+}  // namespace bv
+
+extern "C" {
+
+size_t bv_amp_block_workspace_size(int B, int C, int T) {
+  if (B < 1 || C < 1 || T < 1) return 0;
+  return 3 * align_up((size_t)B * C * T * sizeof(float));
+}
+
+bv_status bv_amp_block(const float *x, int B, int C, int T, const bv_amp_params *p, float *y,
+                       float scale, int accumulate, void *workspace, size_t ws_bytes,
+                       void *stream) {
+  g_err[0] = 0;
+  if (!x || !y) return fail(BV_ERR_ARG, "bv_amp_block: null x or y");
+  if (B < 1 || C < 1 || T < 1) return fail(BV_ERR_SHAPE, "bv_amp_block: B=%d C=%d T=%d", B, C, T);
+  BV_TRY(check_amp_params(p, C));
+  const size_t n = (size_t)B * C * T;
+  const size_t need = bv_amp_block_workspace_size(B, C, T);
+  if (!workspace || ws_bytes < need)
+    return fail(BV_ERR_WORKSPACE, "bv_amp_block: workspace %zu bytes, need %zu", ws_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_amp_block: workspace not 256-byte aligned");
+  const float *wsf = static_cast<const float *>(workspace);
+  if (overlaps(x, n, y, n) || overlaps(x, n, wsf, need / 4) || overlaps(y, n, wsf, need / 4))
+    return fail(BV_ERR_ARG, "bv_amp_block: x, y and workspace must be disjoint");
+  BV_TRY(check_device());
+  char *w8 = static_cast<char *>(workspace);
+  const size_t sz = align_up(n * sizeof(float));
+  AmpScratch s{reinterpret_cast<float *>(w8), reinterpret_cast<float *>(w8 + sz),
+               reinterpret_cast<float *>(w8 + 2 * sz)};
+  return run_amp_block(x, B, C, T, *p, y, scale, accumulate, s, as_stream(stream));
+}
+
+}  // extern "C"
+
+// --------------------------------------------------------------- decoder
+
+namespace bv {
+namespace {
+
+bv_status check_config(const bv_decoder_config *c) {
+  if (!c) return fail(BV_ERR_ARG, "decoder: null config");
+  if (c->in_channels < 1 || c->pre_channels < 1 || c->out_channels < 1)
+    return fail(BV_ERR_SHAPE, "decoder: channel counts must be >= 1");
+  if (c->pre_kernel < 1 || c->pre_kernel % 2 == 0 || c->pre_kernel > 31 || c->post_kernel < 1 ||
+      c->post_kernel % 2 == 0 || c->post_kernel > 31)
+    return fail(BV_ERR_SHAPE, "decoder: pre/post kernels must be odd and <= 31");
+  if (c->n_up < 0 || c->n_up > BV_MAX_UP) return fail(BV_ERR_SHAPE, "decoder: n_up %d", c->n_up);
+  for (int i = 0; i < c->n_up; ++i) {
+    if (c->up_rate[i] < 1 || c->up_rate[i] > 16 || c->up_kernel[i] < c->up_rate[i] ||
+        c->up_kernel[i] > 64 || c->up_channels[i] < 1)
+      return fail(BV_ERR_SHAPE, "decoder: stage %d rate %d kernel %d channels %d", i,
+                  c->up_rate[i], c->up_kernel[i], c->up_channels[i]);
+  }
+  if (c->n_blocks < 1 || c->n_blocks > BV_MAX_BLOCKS)
+    return fail(BV_ERR_SHAPE, "decoder: n_blocks %d", c->n_blocks);
+  for (int j = 0; j < c->n_blocks; ++j)
+    if (c->block_kernel[j] < 1 || c->block_kernel[j] % 2 == 0 || c->block_kernel[j] > 31)
+      return fail(BV_ERR_SHAPE, "decoder: block kernel %d must be odd", c->block_kernel[j]);
+  if (c->n_dilations < 1 || c->n_dilations > BV_MAX_DIL)
+    return fail(BV_ERR_SHAPE, "decoder: n_dilations %d", c->n_dilations);
+  for (int u = 0; u < c->n_dilations; ++u)
+    if (c->dilation[u] < 1) return fail(BV_ERR_SHAPE, "decoder: dilation %d", c->dilation[u]);
+  if (c->final_act < 0 || c->final_act > 2) return fail(BV_ERR_ARG, "decoder: final_act %d", c->final_act);
+  if (c->tile_frames < 0 || c->overlap_frames < 0 ||
+      (c->tile_frames > 0 && c->overlap_frames >= c->tile_frames))
+    return fail(BV_ERR_SHAPE, "decoder: tile %d overlap %d", c->tile_frames, c->overlap_frames);
+  return BV_OK;
+}
+
+long long hop_of(const bv_decoder_config *c) {
+  long long h = 1;
+  for (int i = 0; i < c->n_up; ++i) h *= c->up_rate[i];
+  return h;
+}
+
+// Largest B*C*T over the stored layers of an untiled decode (z excluded).
+long long max_elems(const bv_decoder_config *c, long long B, long long F) {
+  long long n = F, m = B * c->pre_channels * F;
+  for (int i = 0; i < c->n_up; ++i) {
+    const int s = c->up_rate[i], k = c->up_kernel[i];
+    n = (n - 1) * s + k - 2 * ((k - s) / 2);
+    const long long e = B * c->up_channels[i] * n;
+    if (e > m) m = e;
+  }
+  return m;
+}
+
+size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
+  return 5 * align_up((size_t)max_elems(c, B, F) * sizeof(float));
+}
+
+struct TilePlan {
+  bool tiled = false;
+  int step = 0, n_tiles = 1;
+  int n_full = 0;   // tiles of tile_frames frames
+  int last_len = 0; // frames of a shorter last tile (0: none)
+};
+
+TilePlan plan_tiles(const bv_decoder_config *c, int F) {
+  TilePlan p;
+  if (c->tile_frames <= 0 || c->tile_frames >= F) return p;
+  p.tiled = true;
+  p.step = c->tile_frames - c->overlap_frames;
+  int start = 0, n = 1;
+  while (start + c->tile_frames < F) {
+    start += p.step;
+    ++n;
+  }
+  p.n_tiles = n;
+  const int last = F - start;
+  if (last == c->tile_frames) {
+    p.n_full = n;
+  } else {
+    p.n_full = n - 1;
+    p.last_len = last;
+  }
+  return p;
+}
+
+size_t decode_ws(const bv_decoder_config *c, int B, int F) {
+  const TilePlan tp = plan_tiles(c, F);
+  const long long hop = hop_of(c);
+  if (!tp.tiled) return core_ws(c, B, F);
+  size_t s = 0;
+  const long long rows_full = (long long)B * tp.n_full;
+  s += align_up((size_t)rows_full * c->in_channels * c->tile_frames * sizeof(float));
+  s += align_up((size_t)rows_full * c->out_channels * c->tile_frames * hop * sizeof(float));
+  size_t core = core_ws(c, rows_full, c->tile_frames);
+  if (tp.last_len > 0) {
+    s += align_up((size_t)B * c->in_channels * tp.last_len * sizeof(float));
+    s += align_up((size_t)B * c->out_channels * tp.last_len * hop * sizeof(float));
+    const size_t c2 = core_ws(c, B, tp.last_len);
+    if (c2 > core) core = c2;
+  }
+  return s + core;
+}
+
+bv_status check_weights(const bv_decoder_config *c, const bv_decoder_weights *w) {
+  if (!w) return fail(BV_ERR_ARG, "decoder: null weights");
+  if (!w->pre_w || !w->post_w || !w->post_log_alpha || !w->post_log_beta || !w->up_filter ||
+      !w->down_filter)
+    return fail(BV_ERR_ARG, "decoder: null conv_pre / act_post / conv_post weight or filter");
+  for (int i = 0; i < c->n_up; ++i) {
+    if (!w->up_w[i]) return fail(BV_ERR_ARG, "decoder: null ups.%d weight", i);
+    for (int j = 0; j < c->n_blocks; ++j) {
+      const bv_amp_params &p = w->amp[i][j];
+      BV_TRY(check_amp_params(&p, c->up_channels[i]));
+      if (p.kernel_size != c->block_kernel[j] || p.n_dilations != c->n_dilations)
+        return fail(BV_ERR_ARG, "decoder: amp[%d][%d] kernel/dilations differ from the config", i, j);
+      for (int u = 0; u < c->n_dilations; ++u)
+        if (p.dilation[u] != c->dilation[u])
+          return fail(BV_ERR_ARG, "decoder: amp[%d][%d] dilation differs from the config", i, j);
+    }
+  }
+  return BV_OK;
+}
+
+// One untiled decode of B rows into y rows of length F*hop.
+bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                      int B, int F, float *y, char *ws, cudaStream_t st) {
+  const size_t sz = align_up((size_t)max_elems(c, B, F) * sizeof(float));
+  float *A = reinterpret_cast<float *>(ws);
+  float *S = reinterpret_cast<float *>(ws + sz);
+  AmpScratch s{reinterpret_cast<float *>(ws + 2 * sz), reinterpret_cast<float *>(ws + 3 * sz),
+               reinterpret_cast<float *>(ws + 4 * sz)};
+  int C = c->pre_channels, n = F;
+  Epi plain{nullptr, 1.0f, 0, 0};
+  BV_TRY(launch_conv1d(z, B, c->in_channels, F, w->pre_w, w->pre_b, C, c->pre_kernel, 1,
+                       (c->pre_kernel - 1) / 2, plain, A, F, F, st));
+  for (int i = 0; i < c->n_up; ++i) {
+    const int sr = c->up_rate[i], k = c->up_kernel[i], Co = c->up_channels[i];
+    const int pad = (k - sr) / 2;
+    const int n2 = (n - 1) * sr + k - 2 * pad;
+    BV_TRY(launch_conv_transpose1d(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S, st));
+    C = Co;
+    n = n2;
+    const float scale = 1.0f / (float)c->n_blocks;
+    for (int j = 0; j < c->n_blocks; ++j)
+      BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], A, scale, j > 0, s, st));
+  }
+  BV_TRY(launch_activation(A, s.h1, B, C, n, w->post_log_alpha, w->post_log_beta, w->up_filter,
+                           w->down_filter, 1e-9f, st));
+  const long long L = (long long)F * hop_of(c);
+  Epi fin{nullptr, 1.0f, 0, c->final_act};
+  return launch_conv1d(s.h1, B, C, n, w->post_w, w->post_b, c->out_channels, c->post_kernel, 1,
+                       (c->post_kernel - 1) / 2, fin, y, (int)L, (int)L, st);
+}
+
+bv_status decode_impl(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                      int B, int F, float *y, char *ws, cudaStream_t st) {
+  const TilePlan tp = plan_tiles(c, F);
+  if (!tp.tiled) return decode_core(c, w, z, B, F, y, ws, st);
+  const long long hop = hop_of(c);
+  const int Ft = c->tile_frames;
+  const long long rows_full = (long long)B * tp.n_full;
+  char *p = ws;
+  float *zf = reinterpret_cast<float *>(p);
+  p += align_up((size_t)rows_full * c->in_channels * Ft * sizeof(float));
+  float *yf = reinterpret_cast<float *>(p);
+  p += align_up((size_t)rows_full * c->out_channels * Ft * hop * sizeof(float));
+  float *zl = nullptr, *yl = nullptr;
+  if (tp.last_len > 0) {
+    zl = reinterpret_cast<float *>(p);
+    p += align_up((size_t)B * c->in_channels * tp.last_len * sizeof(float));
+    yl = reinterpret_cast<float *>(p);
+    p += align_up((size_t)B * c->out_channels * tp.last_len * hop * sizeof(float));
+  }
+  TileGroups g{};
+  g.n = 0;
+  if (tp.n_full > 0) {
+    BV_TRY(launch_gather_tiles(z, zf, B, c->in_channels, F, tp.step, Ft, 0, tp.n_full, st));
+    BV_TRY(decode_core(c, w, zf, (int)rows_full, Ft, yf, p, st));
+    g.data[g.n] = yf;
+    g.k0[g.n] = 0;
+    g.count[g.n] = tp.n_full;
+    g.len_samples[g.n] = Ft * hop;
+    ++g.n;
+  }
+  if (tp.last_len > 0) {
+    BV_TRY(launch_gather_tiles(z, zl, B, c->in_channels, F, tp.step, tp.last_len, tp.n_full, 1, st));
+    BV_TRY(decode_core(c, w, zl, B, tp.last_len, yl, p, st));
+    g.data[g.n] = yl;
+    g.k0[g.n] = tp.n_full;
+    g.count[g.n] = 1;
+    g.len_samples[g.n] = tp.last_len * hop;
+    ++g.n;
+  }
+  g.max_len_samples = Ft * hop;
+  return launch_stitch_tiles(g, y, B, c->out_channels, (long long)F * hop, (int)(tp.step * hop), st);
+}
+
+}  // namespace
+}  // namespace bv
+
+extern "C" {
+
+int64_t bv_decoder_param_count(const bv_decoder_config *c) {
+  if (check_config(c) != BV_OK) return -1;
+  int64_t n = (int64_t)c->pre_channels * c->in_channels * c->pre_kernel + c->pre_channels;
+  int64_t C = c->pre_channels;
+  for (int i = 0; i < c->n_up; ++i) {
+    const int64_t Co = c->up_channels[i];
+    n += C * Co * c->up_kernel[i] + Co;
+    for (int j = 0; j < c->n_blocks; ++j)
+      n += (int64_t)c->n_dilations * (4 * Co + 2 * (Co * Co * c->block_kernel[j] + Co));
+    C = Co;
+  }
+  n += 2 * C + (int64_t)c->out_channels * C * c->post_kernel + c->out_channels;
+  return n;
+}
+
+bv_status bv_decoder_weights_from_flat(const bv_decoder_config *c, const float *flat,
+                                       const float *up_filter, const float *down_filter,
+                                       bv_decoder_weights *out) {
+  g_err[0] = 0;
+  BV_TRY(check_config(c));
+  if (!flat || !up_filter || !down_filter || !out)
+    return fail(BV_ERR_ARG, "bv_decoder_weights_from_flat: null pointer");
+  std::memset(out, 0, sizeof(*out));
+  const float *p = flat;
+  auto take = [&](size_t n) {
+    const float *q = p;
+    p += n;
+    return q;
+  };
+  size_t C = c->pre_channels;
+  out->pre_w = take(C * c->in_channels * c->pre_kernel);
+  out->pre_b = take(C);
+  for (int i = 0; i < c->n_up; ++i) {
+    const size_t Co = c->up_channels[i];
+    out->up_w[i] = take(C * Co * c->up_kernel[i]);
+    out->up_b[i] = take(Co);
+    C = Co;
+    for (int j = 0; j < c->n_blocks; ++j) {
+      bv_amp_params &a = out->amp[i][j];
+      const size_t K = c->block_kernel[j];
+      a.kernel_size = (int)K;
+      a.n_dilations = c->n_dilations;
+      a.up_filter = up_filter;
+      a.down_filter = down_filter;
+      for (int u = 0; u < c->n_dilations; ++u) {
+        a.dilation[u] = c->dilation[u];
+        a.act_log_alpha[2 * u] = take(C);
+        a.act_log_beta[2 * u] = take(C);
+        a.conv1_w[u] = take(C * C * K);
+        a.conv1_b[u] = take(C);
+        a.act_log_alpha[2 * u + 1] = take(C);
+        a.act_log_beta[2 * u + 1] = take(C);
+        a.conv2_w[u] = take(C * C * K);
+        a.conv2_b[u] = take(C);
+      }
+    }
+  }
+  out->post_log_alpha = take(C);
+  out->post_log_beta = take(C);
+  out->post_w = take((size_t)c->out_channels * C * c->post_kernel);
+  out->post_b = take(c->out_channels);
+  out->up_filter = up_filter;
+  out->down_filter = down_filter;
+  return BV_OK;
+}
+
+int64_t bv_decoder_output_length(const bv_decoder_config *c, int frames) {
+  if (check_config(c) != BV_OK || frames < 1) return -1;
+  return (int64_t)frames * hop_of(c);
+}
+
+size_t bv_decode_workspace_size(const bv_decoder_config *c, int B, int frames) {
+  g_err[0] = 0;
+  if (check_config(c) != BV_OK) return 0;
+  if (B < 1 || frames < 1) {
+    fail(BV_ERR_SHAPE, "bv_decode_workspace_size: B=%d frames=%d", B, frames);
+    return 0;
+  }
+  return decode_ws(c, B, frames);
+}
+
+bv_status bv_decode(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                    int B, int frames, float *y, void *workspace, size_t ws_bytes,
+                    void *stream) {
+  g_err[0] = 0;
+  BV_TRY(check_config(c));
+  if (!z || !y) return fail(BV_ERR_ARG, "bv_decode: null z or y");
+  if (B < 1 || frames < 1) return fail(BV_ERR_SHAPE, "bv_decode: B=%d frames=%d", B, frames);
+  const long long L = (long long)frames * hop_of(c);
+  if (L > 0x7fffffffLL || max_elems(c, B, frames) > (1LL << 40))
+    return fail(BV_ERR_SHAPE, "bv_decode: request too large");
+  BV_TRY(check_weights(c, w));
+  const size_t need = decode_ws(c, B, frames);
+  if (!workspace || ws_bytes < need)
+    return fail(BV_ERR_WORKSPACE, "bv_decode: workspace %zu bytes, need %zu", ws_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_decode: workspace not 256-byte aligned");
+  const size_t nz = (size_t)B * c->in_channels * frames, ny = (size_t)B * c->out_channels * L;
+  const float *wsf = static_cast<const float *>(workspace);
+  if (overlaps(z, nz, y, ny) || overlaps(z, nz, wsf, need / 4) || overlaps(y, ny, wsf, need / 4))
+    return fail(BV_ERR_ARG, "bv_decode: z, y and workspace must be disjoint");
+  BV_TRY(check_device());
+  return decode_impl(c, w, z, B, frames, y, static_cast<char *>(workspace), as_stream(stream));
+}
+
+size_t bv_decode_host_workspace_size(const bv_decoder_config *c, int B, int frames) {
+  const size_t core = bv_decode_workspace_size(c, B, frames);
+  if (core == 0) return 0;
+  const long long L = (long long)frames * hop_of(c);
+  return core + align_up((size_t)B * c->in_channels * frames * sizeof(float)) +
+         align_up((size_t)B * c->out_channels * L * sizeof(float));
+}
+
+bv_status bv_decode_host(const bv_decoder_config *c, const bv_decoder_weights *w,
+                         const float *z_host, int B, int frames, float *y_host, void *workspace,
+                         size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  BV_TRY(check_config(c));
+  if (!z_host || !y_host) return fail(BV_ERR_ARG, "bv_decode_host: null z or y");
+  if (B < 1 || frames < 1) return fail(BV_ERR_SHAPE, "bv_decode_host: B=%d frames=%d", B, frames);
+  const size_t need = bv_decode_host_workspace_size(c, B, frames);
+  if (!workspace || ws_bytes < need)
+    return fail(BV_ERR_WORKSPACE, "bv_decode_host: workspace %zu bytes, need %zu", ws_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_decode_host: workspace not 256-byte aligned");
+  BV_TRY(check_weights(c, w));
+  BV_TRY(check_device());
+  const long long L = (long long)frames * hop_of(c);
+  const size_t zb = (size_t)B * c->in_channels * frames * sizeof(float);
+  const size_t yb = (size_t)B * c->out_channels * L * sizeof(float);
+  char *p = static_cast<char *>(workspace);
+  float *zd = reinterpret_cast<float *>(p);
+  float *yd = reinterpret_cast<float *>(p + align_up(zb));
+  char *core = p + align_up(zb) + align_up(yb);
+  cudaStream_t st = as_stream(stream);
+  cudaError_t e = cudaMemcpyAsync(zd, z_host, zb, cudaMemcpyHostToDevice, st);
+  if (e != cudaSuccess) return fail(BV_ERR_CUDA, "bv_decode_host: H2D: %s", cudaGetErrorString(e));
+  BV_TRY(decode_impl(c, w, zd, B, frames, yd, core, st));
+  e = cudaMemcpyAsync(y_host, yd, yb, cudaMemcpyDeviceToHost, st);
+  if (e != cudaSuccess) return fail(BV_ERR_CUDA, "bv_decode_host: D2H: %s", cudaGetErrorString(e));
+  return BV_OK;
+}
+
+}  // extern "C"

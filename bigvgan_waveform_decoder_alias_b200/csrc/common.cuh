@@ -1,0 +1,88 @@
+// Shared host/device helpers of libbv (error state, launch accounting).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <cstdarg>
+#include <cstdio>
+
+#include "bv.h"
+
+namespace bv {
+
+// Records a message for bv_last_error() and returns `st`.
+bv_status fail(bv_status st, const char *fmt, ...);
+
+// Checks the last launch; BV_ERR_CUDA with the CUDA message on failure.
+bv_status check_launch(const char *what);
+
+// Counts kernel launches issued by the library.
+void count_launch(uint64_t n = 1);
+
+// Address of the device status word that bounded waits set when they give
+// up (kernels take it as an argument); nullptr if it cannot be resolved.
+int *device_status_ptr();
+
+// Per-launch event timing (bv_timing_enable).  Construct right before a
+// launch and let it go out of scope right after it.
+class LaunchTimer {
+ public:
+  LaunchTimer(cudaStream_t st, const char *cls, double flops, double bytes);
+  ~LaunchTimer();
+  LaunchTimer(const LaunchTimer &) = delete;
+  LaunchTimer &operator=(const LaunchTimer &) = delete;
+
+ private:
+  int slot_ = -1;
+  cudaStream_t st_;
+};
+
+inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// [a, a+na) and [b, b+nb) (in floats) overlap?
+inline bool overlaps(const float *a, size_t na, const float *b, size_t nb) {
+  const char *a0 = reinterpret_cast<const char *>(a), *b0 = reinterpret_cast<const char *>(b);
+  return a0 < b0 + nb * sizeof(float) && b0 < a0 + na * sizeof(float);
+}
+
+inline bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// Epilogue in device-friendly form.
+struct Epi {
+  const float *residual;  // may equal y
+  float scale;
+  int accumulate;
+  int final_act;
+};
+
+__device__ __forceinline__ float apply_epilogue(float acc, float bias, const Epi &e,
+                                                const float *yp, size_t idx) {
+  float v = acc + bias;
+  if (e.residual) v += e.residual[idx];  // may alias y: plain load
+  v *= e.scale;
+  if (e.accumulate) v += yp[idx];
+  if (e.final_act == 1) v = fminf(fmaxf(v, -1.0f), 1.0f);
+  else if (e.final_act == 2) v = tanhf(v);
+  return v;
+}
+
+// ---- launchers shared by the ABI and the decoder orchestration -------------
+
+// Alias-free activation over rows (b, c) of length T.
+bv_status launch_activation(const float *x, float *y, int B, int C, int T, const float *la,
+                            const float *lb, const float *fu, const float *fd, float eps,
+                            cudaStream_t st);
+
+// Conv1d; writes y rows of length y_len (<= Tout: the first y_len outputs),
+// row pitch y_pitch floats.
+bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
+                        int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
+                        int y_pitch, cudaStream_t st);
+
+// ConvTranspose1d.
+bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,
+                                  const float *bias, int Cout, int K, int stride, int pad,
+                                  float *y, cudaStream_t st);
+
+}  // namespace bv

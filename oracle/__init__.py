@@ -56,6 +56,9 @@ def lib():
                                               ctypes.c_int, _f32p, _f32p, _f32p, _f32p,
                                               ctypes.c_int, ctypes.c_double, _i64p,
                                               ctypes.c_int, _f64p]
+        L.orc_amp_block.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
+                                    ctypes.c_int, _i32p, ctypes.c_int, _f32p, _f32p,
+                                    ctypes.c_int, ctypes.c_double, ctypes.c_int, _f32p]
         L.orc_decoder_param_count.restype = ctypes.c_long
         L.orc_decoder_param_count.argtypes = [_i32p]
         L.orc_decoder_hop.restype = ctypes.c_long
@@ -201,6 +204,22 @@ def activation1d_points(x, log_alpha, log_beta, points, up=None, down=None, eps=
                                          idx.ctypes.data_as(_i64p), n,
                                          out.ctypes.data_as(_f64p)), "activation1d_points")
     return out
+
+
+def amp_block(x, params, kernel_size, dilations, filt=None, eps=1e-9, store_f64=False):
+    """One AMP block; `params` flat in the block's module order."""
+    x, params = _f32(x), _f32(params)
+    B, C, T = x.shape
+    d = np.ascontiguousarray(np.asarray(dilations, np.int32))
+    need = len(d) * (4 * C + 2 * (C * C * kernel_size + C))
+    if params.size != need:
+        raise ValueError(f"amp block params: {params.size} values, need {need}")
+    f = kaiser_sinc() if filt is None else _f32(filt)
+    y = np.empty_like(x)
+    _check(lib().orc_amp_block(_p32(x), B, C, T, _p32(params), kernel_size,
+                               d.ctypes.data_as(_i32p), len(d), _p32(f), _p32(f), len(f), eps,
+                               int(store_f64), _p32(y)), "amp_block")
+    return y
 
 
 # ----------------------------------------------------------------- decoder

@@ -487,6 +487,34 @@ static const float *amp_block(double *cur, int B, int C, int n, int K,
     return p;
 }
 
+/* One AMP block on x [B, C, T] -> y, parameters in the block's module order
+ * (per dilation: act1 log_alpha, log_beta, conv1 w, b, act2 log_alpha,
+ * log_beta, conv2 w, b).  Same definition as inside the decoder. */
+int orc_amp_block(const float *x, int B, int C, int T, const float *params, int K,
+                  const int *dil, int nd, const float *up, const float *down, int FK,
+                  double eps, int store_f64, float *y) {
+    if (B <= 0 || C <= 0 || T <= 0 || K <= 0 || K % 2 == 0 || nd <= 0 || nd > 4 ||
+        !up_filter_ok(FK) || FK > 64)
+        return ORC_ERR_ARG;
+    for (int u = 0; u < nd; ++u) if (dil[u] <= 0) return ORC_ERR_ARG;
+    double fu[64], fd[64];
+    for (int j = 0; j < FK; ++j) { fu[j] = up[j]; fd[j] = down[j]; }
+    size_t n = (size_t)B * C * T;
+    double *cur = to_d(x, n);
+    double *h1 = (double *)malloc(n * sizeof(double));
+    double *h2 = (double *)malloc(n * sizeof(double));
+    double *acc = (double *)malloc((size_t)(T + 8) * sizeof(double));
+    double *work = (double *)malloc((size_t)2 * (2 * T + 2 * FK + 8) * sizeof(double));
+    if (!cur || !h1 || !h2 || !acc || !work) {
+        free(cur); free(h1); free(h2); free(acc); free(work);
+        return ORC_ERR_NOMEM;
+    }
+    amp_block(cur, B, C, T, K, dil, nd, params, fu, fd, FK, eps, h1, h2, acc, work, store_f64);
+    to_f(cur, y, n);
+    free(cur); free(h1); free(h2); free(acc); free(work);
+    return ORC_OK;
+}
+
 /* Decode z [B, in_ch, frames] -> y [B, out_ch, frames * hop] (the first
  * frames*hop samples of the full-rate signal; the pages' odd-stride ConvT
  * makes the raw signal a few samples longer, and the extra samples sit at

@@ -1,0 +1,382 @@
+"""Parity of the CUDA path (through the C ABI) with the oracle, element by
+element on the same seeded inputs.
+
+Tolerances (the decoder's accuracy target): a single layer within 1e-5
+relative L2 of the oracle given the same float input, the whole waveform
+within 1e-4.  Spot checks of full-size tensors compare sampled outputs that
+the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+from bigvgan_waveform_decoder_alias_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+LAYER_TOL = 1e-5
+WAVE_TOL = 1e-4
+
+
+def rel_l2(got, want):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    return float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-300))
+
+
+@pytest.fixture(scope="module")
+def nat():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from bigvgan_waveform_decoder_alias_b200 import build_native, native
+    build_native.build()
+    native.lib()
+    return native
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
+
+
+def host(t):
+    torch.cuda.synchronize()
+    return t.detach().cpu().numpy()
+
+
+@pytest.fixture(scope="module")
+def filt(oracle, nat):
+    f = nat.bv_filter_design(0.25, 0.3, 12)
+    np.testing.assert_array_equal(f, oracle.kaiser_sinc())
+    return dev(f)
+
+
+# -------------------------------------------------------------- activation
+
+ACT_SHAPES = [(1, 1, 1), (1, 1, 2), (1, 3, 3), (2, 1, 5), (1, 2, 13), (1, 1, 1023),
+              (2, 3, 1024), (1, 2, 1025), (2, 2, 2049), (1, 5, 5000), (3, 4, 4100)]
+
+
+@pytest.mark.parametrize("B,C,T", ACT_SHAPES)
+def test_activation_matches_oracle(nat, oracle, filt, B, C, T):
+    s = synth.NormalStream(1000 + 7 * T + C)
+    x = s.normal((B, C, T), 0.0, 2.0)
+    la, lb = s.normal((C,), 0.0, 0.3), s.normal((C,), 0.0, 0.3)
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    want = oracle.activation1d(x, la, lb)
+    assert y.shape == want.shape
+    assert rel_l2(y, want) < LAYER_TOL
+    np.testing.assert_allclose(y, want, rtol=1e-5, atol=1e-5)
+
+
+def test_activation_constant_rows_exact_form(nat, filt):
+    """Constant rows map to c + sin^2(e^a c)/(e^b + eps) everywhere, edges too."""
+    C, T = 4, 3000
+    cs = np.array([0.3, -1.7, 2.5, np.pi / 2], np.float32)
+    la = np.array([0.05, -0.2, 0.1, 0.0], np.float32)
+    lb = np.array([-0.1, 0.15, 0.0, 0.0], np.float32)
+    x = np.repeat(cs[None, :, None], T, axis=2)
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    for c in range(C):
+        want = cs[c] + np.sin(np.exp(la[c]) * cs[c]) ** 2 / (np.exp(lb[c]) + 1e-9)
+        np.testing.assert_allclose(y[0, c], want, rtol=2e-6, atol=2e-6)
+
+
+def test_activation_full_size_sweep_point(nat, oracle, filt):
+    """The activation workload at full size [2, 512, 65536], every element."""
+    w = synth.ACT_SWEEP
+    x, la, lb = w.make()
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    want = oracle.activation1d(x, la, lb)
+    assert rel_l2(y, want) < LAYER_TOL
+    assert np.abs(y - want).max() < 1e-4
+
+
+@pytest.mark.parametrize("C,T", [(64, 262144), (1536, 4096), (768, 16384)])
+def test_activation_sweep_shapes_sampled(nat, oracle, filt, C, T):
+    s = synth.NormalStream(C + T)
+    x = s.normal((2, C, T))
+    la, lb = s.normal((C,), 0.0, 0.1), s.normal((C,), 0.0, 0.1)
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    rng = np.random.default_rng(C + T)
+    pts = np.stack([rng.integers(0, 2, 3000), rng.integers(0, C, 3000),
+                    rng.integers(0, T, 3000)], 1)
+    pts = np.concatenate([pts, [[0, 0, 0], [1, C - 1, T - 1], [0, 1, T - 2]]])
+    want = oracle.activation1d_points(x, la, lb, pts)
+    got = y[pts[:, 0], pts[:, 1], pts[:, 2]]
+    assert rel_l2(got, want) < LAYER_TOL
+
+
+# ------------------------------------------------------------------- convs
+
+CONV_CASES = [(C, K, d, T) for (C, T) in ((12, 1000), (32, 333), (48, 257), (96, 130), (128, 300))
+              for K in (3, 7, 11) for d in (1, 3, 5)]
+
+
+@pytest.mark.parametrize("C,K,d,T", CONV_CASES)
+def test_conv1d_matches_oracle(nat, oracle, C, K, d, T):
+    s = synth.NormalStream(3000 + C * 7 + K * 3 + d + T)
+    B = 2
+    x = s.normal((B, C, T))
+    w = s.normal((C, C, K), 0.0, 0.02)
+    b = s.normal((C,), 0.0, 0.02)
+    pad = (K * d - d) // 2
+    y = host(nat.bv_conv1d(dev(x), dev(w), dev(b), d, pad))
+    want = oracle.conv1d(x, w, b, d, pad)
+    assert rel_l2(y, want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("Cin,Cout,K,T", [(32, 1536, 7, 400), (64, 1024, 7, 500),
+                                          (12, 1, 7, 5001), (16, 1, 7, 777), (3, 5, 1, 9),
+                                          (7, 9, 5, 1), (1, 1, 3, 2), (200, 130, 3, 65)])
+def test_conv1d_channel_changes(nat, oracle, Cin, Cout, K, T):
+    s = synth.NormalStream(Cin * 1000 + Cout + K + T)
+    x = s.normal((2, Cin, T))
+    w = s.normal((Cout, Cin, K), 0.0, 0.05)
+    b = s.normal((Cout,), 0.0, 0.05)
+    y = host(nat.bv_conv1d(dev(x), dev(w), dev(b), 1, (K - 1) // 2))
+    assert rel_l2(y, oracle.conv1d(x, w, b, 1, (K - 1) // 2)) < LAYER_TOL
+
+
+def test_conv1d_unpadded_no_bias(nat, oracle):
+    s = synth.NormalStream(17)
+    x = s.normal((1, 20, 100))
+    w = s.normal((30, 20, 5), 0.0, 0.1)
+    y = host(nat.bv_conv1d(dev(x), dev(w), None, 3, 0))
+    want = oracle.conv1d(x, w, None, 3, 0)
+    assert y.shape == (1, 30, 88) and rel_l2(y, want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("final_act", [0, 1, 2])
+def test_conv1d_epilogue(nat, oracle, final_act):
+    """y = final(scale * (conv + bias + residual) + y_old)."""
+    s = synth.NormalStream(50 + final_act)
+    C, T = 48, 700
+    x = s.normal((2, C, T))
+    w = s.normal((C, C, 7), 0.0, 0.1)
+    b = s.normal((C,), 0.0, 0.1)
+    r = s.normal((2, C, T))
+    y0 = s.normal((2, C, T))
+    yd = dev(y0)
+    nat.bv_conv1d(dev(x), dev(w), dev(b), 3, 9, residual=dev(r), scale=1.0 / 3.0,
+                  accumulate=True, final_act=final_act, y=yd)
+    got = host(yd).astype(np.float64)
+    conv = oracle.conv1d(x, w, b, 3, 9, store_f64=True).astype(np.float64)
+    want = (conv + r) * (1.0 / 3.0) + y0
+    if final_act == 1:
+        want = np.clip(want, -1, 1)
+    elif final_act == 2:
+        want = np.tanh(want)
+    assert rel_l2(got, want) < LAYER_TOL
+
+
+def test_conv1d_inplace_residual(nat, oracle):
+    s = synth.NormalStream(77)
+    C, T = 96, 513
+    x = s.normal((1, C, T))
+    w = s.normal((C, C, 3), 0.0, 0.05)
+    cur = s.normal((1, C, T))
+    cd = dev(cur)
+    nat.bv_conv1d(dev(x), dev(w), None, 5, 5, residual=cd, y=cd)
+    want = oracle.conv1d(x, w, None, 5, 5, store_f64=True).astype(np.float64) + cur
+    assert rel_l2(host(cd), want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("S,T,Cin,Cout", [(5, 400, 64, 48), (5, 1, 16, 8), (2, 2001, 48, 24),
+                                          (2, 3, 12, 12), (3, 50, 20, 10), (4, 77, 24, 40),
+                                          (6, 33, 16, 16), (8, 20, 8, 12)])
+def test_conv_transpose1d_matches_oracle(nat, oracle, S, T, Cin, Cout):
+    s = synth.NormalStream(4000 + S * 100 + T)
+    K = 2 * S
+    pad = (K - S) // 2
+    x = s.normal((2, Cin, T))
+    w = s.normal((Cin, Cout, K), 0.0, 0.05)
+    b = s.normal((Cout,), 0.0, 0.05)
+    y = host(nat.bv_conv_transpose1d(dev(x), dev(w), dev(b), S, pad))
+    want = oracle.conv_transpose1d(x, w, b, S, pad)
+    assert y.shape == want.shape
+    assert rel_l2(y, want) < LAYER_TOL
+
+
+def test_conv_transpose1d_general_kernel(nat, oracle):
+    s = synth.NormalStream(99)
+    x = s.normal((1, 10, 37))
+    for S, K, pad in ((5, 11, 3), (2, 3, 0), (4, 4, 0), (3, 9, 4)):
+        w = s.normal((10, 6, K), 0.0, 0.1)
+        y = host(nat.bv_conv_transpose1d(dev(x), dev(w), None, S, pad))
+        assert rel_l2(y, oracle.conv_transpose1d(x, w, None, S, pad)) < LAYER_TOL
+
+
+# Full-size layer shapes of the MiniMax-H3 decoder, on seeded inputs,
+# checked at sampled outputs.
+H3_STAGES = [(768, 2001), (384, 10006), (192, 20012), (96, 40024), (48, 80048),
+             (24, 160096), (12, 320192)]
+
+
+@pytest.mark.parametrize("C,T", H3_STAGES)
+def test_full_size_stage_layers_sampled(nat, oracle, filt, C, T):
+    s = synth.NormalStream(C * 31 + T)
+    B = 2
+    x = s.normal((B, C, T))
+    xd = dev(x)
+    rng = np.random.default_rng(C)
+    n = 48 if C >= 384 else 200
+    pts = np.stack([rng.integers(0, B, n), rng.integers(0, C, n), rng.integers(0, T, n)], 1)
+    pts = np.concatenate([pts, [[0, 0, 0], [1, C - 1, T - 1], [0, C // 2, 1], [1, 1, T - 3]]])
+    for K, d in ((3, 1), (7, 3), (11, 5)):
+        w = s.normal((C, C, K), 0.0, 0.02)
+        b = s.normal((C,), 0.0, 0.02)
+        pad = (K * d - d) // 2
+        y = host(nat.bv_conv1d(xd, dev(w), dev(b), d, pad))
+        want = oracle.conv1d_points(x, w, b, d, pad, pts)
+        assert rel_l2(y[pts[:, 0], pts[:, 1], pts[:, 2]], want) < LAYER_TOL, (K, d)
+    la, lb = s.normal((C,), 0.0, 0.1), s.normal((C,), 0.0, 0.1)
+    y = host(nat.bv_activation1d(xd, dev(la), dev(lb), filt))
+    want = oracle.activation1d_points(x, la, lb, pts)
+    assert rel_l2(y[pts[:, 0], pts[:, 1], pts[:, 2]], want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("Cin,Cout,S,T", [(1536, 768, 5, 400), (768, 384, 5, 2001),
+                                          (384, 192, 2, 10006), (24, 12, 2, 160096)])
+def test_full_size_conv_transpose_sampled(nat, oracle, Cin, Cout, S, T):
+    s = synth.NormalStream(Cin + T)
+    K = 2 * S
+    pad = (K - S) // 2
+    x = s.normal((2, Cin, T))
+    w = s.normal((Cin, Cout, K), 0.0, 0.02)
+    b = s.normal((Cout,), 0.0, 0.02)
+    y = host(nat.bv_conv_transpose1d(dev(x), dev(w), dev(b), S, pad))
+    Tout = (T - 1) * S + K - 2 * pad
+    rng = np.random.default_rng(T)
+    pts = np.stack([rng.integers(0, 2, 40), rng.integers(0, Cout, 40),
+                    rng.integers(0, Tout, 40)], 1)
+    pts = np.concatenate([pts, [[0, 0, 0], [1, Cout - 1, Tout - 1], [0, 1, Tout - 2]]])
+    want = oracle.conv_transpose1d_points(x, w, b, S, pad, pts)
+    assert rel_l2(y[pts[:, 0], pts[:, 1], pts[:, 2]], want) < LAYER_TOL
+
+
+# -------------------------------------------------------------- AMP block
+
+
+def _amp_tensors(layout, flat):
+    out, off = {}, 0
+    for name, shape, _ in layout:
+        n = int(np.prod(shape))
+        out[name] = dev(flat[off:off + n].reshape(shape))
+        off += n
+    return out
+
+
+def test_amp_block_workload_matches_oracle(nat, oracle, filt):
+    w = synth.AMP_BLOCK_C32
+    x, flat = w.make()
+    tens = _amp_tensors(w.layout(), flat)
+    p = nat.amp_params(w.kernel, w.dilations, tens, filt)
+    y = host(nat.bv_amp_block(dev(x), p))
+    want = oracle.amp_block(x, flat, w.kernel, w.dilations)
+    assert rel_l2(y, want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("C,T,K,dils", [(12, 3001, 11, (1, 3, 5)), (96, 517, 7, (1, 3, 5)),
+                                        (130, 64, 3, (2,)), (16, 5, 7, (1, 3, 5, 7))])
+def test_amp_block_shapes(nat, oracle, filt, C, T, K, dils):
+    wl = synth.AmpWorkload("t", 2, C, T, K, dils, seed=C + T)
+    x, flat = wl.make()
+    tens = _amp_tensors(wl.layout(), flat)
+    p = nat.amp_params(K, dils, tens, filt)
+    y0 = synth.NormalStream(5).normal((2, C, T))
+    yd = dev(y0)
+    nat.bv_amp_block(dev(x), p, y=yd, scale=0.5, accumulate=True)
+    want = 0.5 * oracle.amp_block(x, flat, K, dils).astype(np.float64) + y0
+    assert rel_l2(host(yd), want) < LAYER_TOL
+
+
+# ----------------------------------------------------------------- decoder
+
+
+def _decoder(nat, geo, params, filt, tile=0, overlap=0):
+    return nat.Decoder(geo, params, filt=host(filt), tile_frames=tile, overlap_frames=overlap)
+
+
+@pytest.mark.parametrize("final_act", ["none", "clamp", "tanh"])
+def test_tiny_decoder_matches_oracle(nat, oracle, filt, final_act):
+    geo = synth.tiny_geometry(final_act=final_act)
+    s = synth.NormalStream(8)
+    z = s.normal((2, geo.in_channels, 9))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.1)
+    dec = _decoder(nat, geo, params, filt)
+    y = host(dec.decode(dev(z)))
+    want = oracle.decode(geo, params, z)
+    assert y.shape == want.shape == (2, 1, 9 * geo.hop)
+    assert rel_l2(y, want) < WAVE_TOL
+
+
+@pytest.mark.parametrize("wname,frames", [("h3_decoder_10s_stereo", 3),
+                                          ("ltx_vocoder_500f_stereo", 4)])
+def test_real_geometry_short_latent(nat, oracle, filt, wname, frames):
+    """The full-size channel plan of each decoder on a few latent frames,
+    checked over the whole waveform (every layer kind and stride at its real
+    channel count)."""
+    w = synth.DECODER_WORKLOADS[wname]
+    z, params = w.make()
+    z = np.ascontiguousarray(z[..., :frames])
+    dec = _decoder(nat, w.geometry, params, filt)
+    y = host(dec.decode(dev(z)))
+    want = oracle.decode(w.geometry, params, z)
+    assert y.shape == want.shape
+    assert rel_l2(y, want) < WAVE_TOL
+
+
+def test_decoder_batch_independence_and_determinism(nat, filt):
+    geo = synth.tiny_geometry()
+    s = synth.NormalStream(12)
+    z = s.normal((3, geo.in_channels, 7))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.1)
+    dec = _decoder(nat, geo, params, filt)
+    y = host(dec.decode(dev(z)))
+    y2 = host(dec.decode(dev(z)))
+    np.testing.assert_array_equal(y, y2)
+    for b in range(3):
+        np.testing.assert_array_equal(host(dec.decode(dev(z[b:b + 1]))), y[b:b + 1])
+
+
+def test_tiled_decoder_matches_oracle(nat, oracle, filt):
+    geo = synth.tiny_geometry()
+    s = synth.NormalStream(13)
+    z = s.normal((2, geo.in_channels, 23))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.1)
+    for tile, ov in ((6, 2), (5, 1), (23, 4), (30, 3), (8, 0)):
+        dec = _decoder(nat, geo, params, filt, tile, ov)
+        y = host(dec.decode(dev(z)))
+        want, _ = oracle.decode_tiled(geo, params, z, tile, ov)
+        assert rel_l2(y, want) < WAVE_TOL, (tile, ov)
+
+
+def test_decode_host_matches_device(nat, filt):
+    geo = synth.tiny_geometry()
+    s = synth.NormalStream(14)
+    z = s.normal((2, geo.in_channels, 5))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.1)
+    dec = _decoder(nat, geo, params, filt)
+    yd = host(dec.decode(dev(z)))
+    zh = torch.from_numpy(z).pin_memory()
+    yh = torch.empty((2, 1, 5 * geo.hop), dtype=torch.float32).pin_memory()
+    dec.decode_host(zh, yh)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(yh.numpy(), yd)
+
+
+def test_decode_in_cuda_graph(nat, filt):
+    geo = synth.tiny_geometry()
+    s = synth.NormalStream(15)
+    z = dev(s.normal((2, geo.in_channels, 5)))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.1)
+    dec = _decoder(nat, geo, params, filt)
+    ref = host(dec.decode(z))
+    y = torch.empty((2, 1, 5 * geo.hop), device="cuda")
+    ws = dec.workspace(2, 5)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dec.decode(z, y=y, workspace=ws)
+    y.zero_()
+    g.replay()
+    np.testing.assert_array_equal(host(y), ref)
