@@ -43,7 +43,56 @@ def parse():
     ap.add_argument("--cpu-sample-frames", type=int, default=12,
                     help="latent frames (one side) of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None,
+                    help="time one kernel on one shape instead of the decoder (for profiling): "
+                         "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s")
     return ap.parse_args()
+
+
+def run_case(args):
+    """One kernel on one seeded shape, W warm-up and K timed launches."""
+    import torch
+    from bigvgan_waveform_decoder_alias_b200 import native
+    kind, shape, *rest = args.case.split(":")
+    B, C, T = (int(v) for v in shape.split("x"))
+    s = synth.NormalStream(7)
+    x = torch.from_numpy(s.normal((B, C, T))).cuda()
+    filt = torch.from_numpy(native.bv_filter_design()).cuda()
+    if kind == "activation":
+        la = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
+        lb = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
+        y = torch.empty_like(x)
+        fn = lambda: native.bv_activation1d(x, la, lb, filt, y=y)  # noqa: E731
+        work, unit = 8.0 * B * C * T, "GB/s"
+    elif kind == "conv1d":
+        K, d = int(rest[0]), int(rest[1])
+        w = torch.from_numpy(s.normal((C, C, K), 0, 0.02)).cuda()
+        b = torch.from_numpy(s.normal((C,), 0, 0.02)).cuda()
+        y = torch.empty_like(x)
+        fn = lambda: native.bv_conv1d(x, w, b, d, (K * d - d) // 2, y=y)  # noqa: E731
+        work, unit = 2.0 * B * C * C * K * T, "TFLOP/s"
+    elif kind == "convt":
+        Co, st = int(rest[0]), int(rest[1])
+        w = torch.from_numpy(s.normal((C, Co, 2 * st), 0, 0.02)).cuda()
+        b = torch.from_numpy(s.normal((Co,), 0, 0.02)).cuda()
+        fn = lambda: native.bv_conv_transpose1d(x, w, b, st)  # noqa: E731
+        work, unit = 2.0 * B * C * Co * 2 * st * T, "TFLOP/s"
+    else:
+        raise SystemExit(f"unknown case {kind}")
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    for a, b_ in ev:
+        a.record()
+        fn()
+        b_.record()
+    torch.cuda.synchronize()
+    ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
+    rate = work / (ms / 1000) / (1e9 if unit == "GB/s" else 1e12)
+    print(json.dumps({"case": args.case, "ms_median": ms, "achieved": rate, "unit": unit}))
+    return 0
 
 
 def peaks():
@@ -166,6 +215,8 @@ def run_reference(args, world, rank):
 def main():
     args = parse()
     world, rank, local = dist_init()
+    if args.case:
+        return run_case(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
 
