@@ -109,6 +109,8 @@ def lib():
     L.bv_amp_block_workspace_size.argtypes = [c_int, c_int, c_int]
     L.bv_amp_block.argtypes = [_fp, c_int, c_int, c_int, ctypes.POINTER(AmpParams), _fp, c_float,
                                c_int, _fp, c_size, _fp]
+    L.bv_amp_block_static.argtypes = [_fp, c_int, c_int, c_int, ctypes.POINTER(AmpParams), _fp,
+                                      c_float, c_int, _fp]
     L.bv_decoder_param_count.restype = ctypes.c_int64
     L.bv_decoder_param_count.argtypes = [ctypes.POINTER(DecoderConfig)]
     L.bv_decoder_weights_from_flat.argtypes = [ctypes.POINTER(DecoderConfig), _fp, _fp, _fp,

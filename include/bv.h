@@ -208,6 +208,31 @@ bv_status bv_amp_block(const float *x, int B, int C, int T,
                        void *stream);
 
 /* ------------------------------------------------------------------------
+ * bv_amp_block without a workspace argument.  The pages have no counterpart
+ * to this entry point: it exists for callers that cannot allocate device
+ * memory when they run the block -- a real-time audio thread (a plugin's
+ * render callback must not call cudaMalloc, which may block on the driver),
+ * or a host that fixes its device memory budget before the decoder runs.
+ * The scratch lives in a static device array inside libbv, sized for
+ * B*C*T <= BV_AMP_STATIC_MAX_ELEMS (three tensors of that many floats,
+ * 12 MiB); every GPU that loads the library holds it until the process
+ * exits.  Larger requests return BV_ERR_WORKSPACE and leave y untouched.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture begins.  All calls share the one array and it
+ * keeps the last call's contents (nothing in it needs to start at zero):
+ * calls whose GPU work can overlap -- on different streams or from
+ * different host threads -- race on it, so serialise them.  Arguments and
+ * results are those of bv_amp_block.
+ * ---------------------------------------------------------------------- */
+#define BV_AMP_STATIC_MAX_ELEMS (1 << 20)
+
+bv_status bv_amp_block_static(const float *x, int B, int C, int T,
+                              const bv_amp_params *p, float *y, float scale,
+                              int accumulate, void *stream);
+
+/* ------------------------------------------------------------------------
  * The whole decoder ([H3] `AudioVae::decode`, [LTX] `Vocoder::forward`):
  *   conv_pre (pad (pre_kernel-1)/2)
  *   -> for each stage i: ConvT (rate up_rate[i], kernel up_kernel[i],
