@@ -238,6 +238,16 @@ bv_status bv_activation1d(const float *x, float *y, int B, int C, int T, const f
                            as_stream(stream));
 }
 
+bv_status bv_sin_squared(const float *z, float *out, int64_t n, void *stream) {
+  g_err[0] = 0;
+  if (!z || !out) return fail(BV_ERR_ARG, "bv_sin_squared: null pointer");
+  if (n < 0) return fail(BV_ERR_SHAPE, "bv_sin_squared: n=%lld", (long long)n);
+  if (z != out && overlaps(z, (size_t)n, out, (size_t)n))
+    return fail(BV_ERR_ARG, "bv_sin_squared: z and out partially overlap");
+  BV_TRY(check_device());
+  return launch_sin_squared(z, out, n, as_stream(stream));
+}
+
 bv_status bv_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
                     int Cout, int K, int dilation, int pad, const bv_epilogue *ep, float *y,
                     void *stream) {

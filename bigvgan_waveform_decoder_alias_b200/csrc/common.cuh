@@ -74,11 +74,21 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
                             const float *lb, const float *fu, const float *fd, float eps,
                             cudaStream_t st);
 
+// The activation's sin^2, elementwise (for accuracy tests).
+bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream_t st);
+
 // Conv1d; writes y rows of length y_len (<= Tout: the first y_len outputs),
 // row pitch y_pitch floats.
 bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
                         int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
                         int y_pitch, cudaStream_t st);
+
+// Conv1d on the tensor cores (tcgen05, 3xTF32); supported() says whether the
+// shape qualifies (launch_conv1d picks it automatically).
+bool conv1d_tc_supported(int Cin, int Cout, int K, int dil);
+bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
+                           float *y, int y_len, int y_pitch, cudaStream_t st);
 
 // ConvTranspose1d.
 bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,

@@ -140,7 +140,7 @@ bv_status run_conv(const float *x, int B, int Cin, int T, const float *w, const 
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d: grid too large");
   {
     const double outs = (double)B * Cout * y_len;
-    LaunchTimer tm(st, "conv1d", 2.0 * outs * Cin * K,
+    LaunchTimer tm(st, "conv1d_simt", 2.0 * outs * Cin * K,
                    4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                           outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
     kern<<<grid, Cfg::THREADS, smem, st>>>(x, w, bias, y, Cin, T, Cout, K, dil, pad, y_len,
@@ -156,6 +156,8 @@ bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, c
                         int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
                         int y_pitch, cudaStream_t st) {
   if (B <= 0 || y_len <= 0) return BV_OK;
+  if (conv1d_tc_supported(Cin, Cout, K, dil) && (reinterpret_cast<uintptr_t>(w) & 15u) == 0)
+    return launch_conv1d_tc(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
   if (Cout >= 96)
     return run_conv<128, 128, 8, 8, 8>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len,
                                        y_pitch, st);

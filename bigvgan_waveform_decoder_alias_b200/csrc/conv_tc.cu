@@ -1,0 +1,513 @@
+// Dilated Conv1d as an implicit GEMM on the 5th-generation tensor cores
+// (tcgen05, accumulator in TMEM), with FP32 accuracy from a 3xTF32 split.
+//
+//   y[b,o,t] = bias[o] + sum_i sum_j w[o,i,j] x[b,i,t + j d - pad]
+// (docs.rs cortiq-engine audiovae.rs `Conv1d::apply`, whose note states the
+// im2col identity used here; ltxaudio.rs `Conv1d::forward`).
+//
+// GEMM view: D[o, t] = sum_kk A[o, kk] B[kk, t] with kk = i K + j (the order
+// of w's own [Cout][Cin][K] layout, so A is w read as a [Cout, Cin K] matrix)
+// and B[kk, t] = x[b, i, t + j d - pad] (im2col, never materialised).
+// Each CTA owns a 128 (o) x 128 (t) output tile and walks kk in chunks of 32:
+//   - a TMA load brings the weight chunk A [128 x 32] into shared memory in
+//     the 128-byte-swizzled K-major layout the tensor core reads;
+//   - four converter warps split it in place into A_hi = tf32(A) (low 13
+//     mantissa bits cleared) and A_lo = A - A_hi, and build B_hi / B_lo
+//     [128 t x 32 kk] (K-major, same swizzle) from input rows staged in shared
+//     memory with cp.async;
+//   - one thread issues three tcgen05.mma.kind::tf32 per 8-wide k step,
+//     A_hi B_hi + A_hi B_lo + A_lo B_hi, into one FP32 TMEM accumulator (the
+//     3xTF32 scheme: the dropped A_lo B_lo term is 2^-22 relative);
+//   - runs of RUN chunks accumulate in one of two TMEM accumulators, starting
+//     from zero; the converter warps read each finished run and add it into
+//     FP32 registers (the tensor core's accumulation truncates, so its error
+//     would otherwise grow with Cin K);
+//   - the epilogue adds bias / residual, scales, accumulates and applies the
+//     final op, staged through shared memory so that global reads and writes
+//     are row-contiguous.
+// Two operand stages overlap conversion with the MMAs.  Every mbarrier wait
+// is bounded; a wait that runs out sets the device status word and the CTA
+// unwinds (its output tile is then unspecified) after freeing its TMEM.
+#include <cuda.h>
+
+#include "common.cuh"
+
+namespace bv {
+namespace {
+
+constexpr int BM = 128;             // output channels per CTA (UMMA M)
+constexpr int BN = 128;             // time samples per CTA (UMMA N)
+constexpr int BK = 32;              // kk per chunk: one 128-byte swizzle row of fp32
+constexpr int NSTAGE = 2;           // operand stages
+constexpr int CB = 32;              // input channels per staged x block
+constexpr int MAX_HALO = 56;        // (K - 1) d the staged rows can hold
+constexpr int XW = BN + MAX_HALO + 8;  // staged row width (floats)
+constexpr int TILE_BYTES = BM * BK * 4;  // 16 KB: one A or B operand tile
+constexpr int THREADS = 256;
+constexpr int CONV_WARP0 = 4;       // warps 4..7 convert and run the epilogue
+constexpr int NCONV = 128;
+constexpr long long WAIT_LIMIT = 1ll << 26;  // try_wait polls before giving up
+constexpr int TMEM_COLS = 256;     // two 128-column accumulators
+constexpr int RUN = 4;              // chunks accumulated in TMEM before an FP32 add
+constexpr int MAX_K = 32;           // largest kernel size (offset table rows)
+constexpr int DS_PITCH = BN + 1;    // epilogue staging row pitch (floats)
+
+// shared memory layout (bytes from a 1024-aligned base)
+constexpr int OFF_A = 0;                                  // A raw -> A_hi, per stage
+constexpr int OFF_ALO = OFF_A + NSTAGE * TILE_BYTES;      // A_lo
+constexpr int OFF_BHI = OFF_ALO + NSTAGE * TILE_BYTES;    // B_hi
+constexpr int OFF_BLO = OFF_BHI + NSTAGE * TILE_BYTES;    // B_lo
+constexpr int OFF_X = OFF_BLO + NSTAGE * TILE_BYTES;      // x blocks [2][CB][XW]
+constexpr int X_BYTES = 2 * CB * XW * 4;
+constexpr int OFF_BAR = OFF_X + X_BYTES;                  // mbarriers
+constexpr int SMEM_USED = OFF_BAR + 256;
+constexpr int SMEM_BYTES = SMEM_USED + 1024;              // room to align the base
+static_assert(BM * DS_PITCH * 4 <= OFF_X, "epilogue staging must fit in the operand area");
+
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+  return (unsigned)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(unsigned bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(unsigned bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(unsigned bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+struct Ctl {
+  int abort;        // a bounded wait gave up somewhere in the CTA
+  unsigned tmem;    // TMEM base address from tcgen05.alloc
+};
+
+// Bounded wait on an mbarrier phase.  On running out it marks the CTA
+// aborted and records the failure in the device status word.
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
+                                          int *status, int code) {
+  for (long long it = 0; it < WAIT_LIMIT; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255) == 255 && ctl->abort) return false;
+  }
+  ctl->abort = 1;
+  if (status) atomicExch(status, code);
+  return false;
+}
+
+// Bounded wait that does not return early on abort: used to drain copies that
+// are still in flight before the CTA exits.
+__device__ __forceinline__ void mbar_drain(unsigned bar, unsigned parity) {
+  for (long long it = 0; it < (1ll << 22); ++it)
+    if (mbar_try_wait(bar, parity)) return;
+}
+
+__device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool valid) {
+  const unsigned d = smem_u32(dst);
+  const int n = valid ? 4 : 0;
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+}
+__device__ __forceinline__ void conv_bar_sync() {  // the four converter warps
+  asm volatile("bar.sync 1, %0;\n" ::"n"(NCONV) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1.
+__device__ __forceinline__ uint64_t sw128_desc(unsigned addr) {
+  return (uint64_t)((addr >> 4) & 0x3FFF) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+// Instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = 128.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                            ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void mma_tf32(unsigned tmem_d, uint64_t a, uint64_t b, unsigned acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit(unsigned bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// Byte offset of element (row r, column k < 32) in a K-major SW128 tile of
+// 128-byte rows: 8-row groups of 1024 bytes, 16-byte chunk index XOR (r % 8).
+__device__ __forceinline__ int sw128_off(int r, int k) {
+  return (r >> 3) * 1024 + (r & 7) * 128 + ((((k >> 2) ^ (r & 7))) << 4) + ((k & 3) << 2);
+}
+
+__device__ __forceinline__ float tf32_hi(float v) {
+  return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+}
+
+// Converter-side wait: lane 0 polls the barrier, the warp follows it, so the
+// polling does not compete with the conversion for shared-memory bandwidth.
+__device__ __forceinline__ void warp_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
+                                          int *status, int code) {
+  if ((threadIdx.x & 31) == 0) mbar_wait(bar, parity, ctl, status, code);
+  __syncwarp();
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ x,
+                 const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
+                 int dil, int pad, int y_len, int y_pitch, Epi ep, int *status) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
+  __shared__ Ctl ctl;
+  __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block, entry e
+  // barriers: A landed (TMA) / operands ready / stage free, per stage; run
+  // accumulated / run accumulator read, per TMEM accumulator
+  const unsigned bar_full_a = smem_u32(&bars[0]);
+  const unsigned bar_ready = smem_u32(&bars[2]);
+  const unsigned bar_empty = smem_u32(&bars[4]);
+  const unsigned bar_run_full = smem_u32(&bars[6]);
+  const unsigned bar_run_free = smem_u32(&bars[8]);
+  float *xs = reinterpret_cast<float *>(smem + OFF_X);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * BN;
+  const int o0 = blockIdx.y * BM;
+  const int b = blockIdx.z;
+  const int KK = Cin * K;
+  const int n_chunks = (KK + BK - 1) / BK;
+  const int n_runs = (n_chunks + RUN - 1) / RUN;
+  const int halo = (K - 1) * dil;
+  const int xt0 = t0 - pad;  // time of staged column 0
+
+  if (threadIdx.x == 0) {
+    ctl.abort = 0;
+    for (int s = 0; s < NSTAGE; ++s) {
+      mbar_init(bar_full_a + 8 * s, 1);
+      mbar_init(bar_ready + 8 * s, NCONV / 32);
+      mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_run_full + 8 * s, 1);
+      mbar_init(bar_run_free + 8 * s, NCONV / 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  // chunk m of an x block covers block-local kk = 32 m + e = i K + j
+  for (int idx = threadIdx.x; idx < K * BK; idx += THREADS) {
+    const int i = idx / K, j = idx - i * K;
+    xoff[idx] = i * XW + j * dil;
+  }
+  if (warp == 1) {  // two TMEM accumulators of 128 lanes x 128 fp32 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_u32(&ctl.tmem)),
+                 "n"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const unsigned tmem = ctl.tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % NSTAGE, u = c / NSTAGE;
+        // After an abort every wait returns at once and the loops run to the end
+        // without blocking, so all roles reach the final barrier.
+        if (u > 0) mbar_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 101);
+        const unsigned dst = smem_u32(smem + OFF_A + s * TILE_BYTES);
+        mbar_arrive_tx(bar_full_a + 8 * s, TILE_BYTES);
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+            "l"(reinterpret_cast<uint64_t>(&tmap_w)), "r"(c * BK), "r"(o0),
+            "r"(bar_full_a + 8 * s)
+            : "memory");
+      }
+      // drain: the last loads of each stage must land before the CTA can exit
+      for (int c = n_chunks - NSTAGE; c < n_chunks; ++c)
+        if (c >= 0) mbar_drain(bar_full_a + 8 * (c % NSTAGE), (c / NSTAGE) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    // Runs of RUN chunks accumulate into alternating TMEM accumulators, each
+    // run starting from zero; the converter warps add finished runs in FP32
+    // registers.  Short runs keep the tensor core's truncating accumulation
+    // from growing with Cin K.
+    if (lane == 0) {
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % NSTAGE, u = c / NSTAGE;
+        const int r = c / RUN, ra = r & 1;
+        const bool first = (c % RUN) == 0;
+        const bool last = (c % RUN) == RUN - 1 || c == n_chunks - 1;
+        if (first && r >= 2)  // the converters have read this accumulator's run r - 2
+          mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 106);
+        mbar_wait(bar_ready + 8 * s, u & 1, &ctl, status, 102);
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        const unsigned acc = tmem + (unsigned)(ra * BN);
+        const unsigned a_hi = smem_u32(smem + OFF_A + s * TILE_BYTES);
+        const unsigned a_lo = smem_u32(smem + OFF_ALO + s * TILE_BYTES);
+        const unsigned b_hi = smem_u32(smem + OFF_BHI + s * TILE_BYTES);
+        const unsigned b_lo = smem_u32(smem + OFF_BLO + s * TILE_BYTES);
+#pragma unroll
+        for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes per MMA
+          const unsigned off = 32 * k;
+          mma_tf32(acc, sw128_desc(a_lo + off), sw128_desc(b_hi + off),
+                   (first && k == 0) ? 0u : 1u);
+          mma_tf32(acc, sw128_desc(a_hi + off), sw128_desc(b_lo + off), 1u);
+          mma_tf32(acc, sw128_desc(a_hi + off), sw128_desc(b_hi + off), 1u);
+        }
+        mma_commit(bar_empty + 8 * s);  // stage s may be refilled once these finish
+        if (last) mma_commit(bar_run_full + 8 * ra);
+      }
+    }
+  } else if (warp >= CONV_WARP0) {
+    // ------------------------------------------------------ converters + sums
+    const int ct = threadIdx.x - CONV_WARP0 * 32;  // row of B this thread builds
+    const int q = warp - CONV_WARP0;                // TMEM lane quarter
+    const float *xb = x + (size_t)b * Cin * T;
+    float sum[BN];  // this thread's output row (o = o0 + 32 q + lane), FP32 run sums
+#pragma unroll
+    for (int e = 0; e < BN; ++e) sum[e] = 0.0f;
+
+    // stage x block blk (channels [CB blk, CB blk + CB)) into xs[blk & 1];
+    // channels >= Cin and times outside [0, T) read as zero
+    auto stage_x = [&](int blk) {
+      float *dst = xs + (blk & 1) * CB * XW;
+      const int i0 = blk * CB;
+      const int width = BN + halo;
+      for (int idx = ct; idx < CB * width; idx += NCONV) {
+        const int ci = idx / width, n = idx - ci * width;
+        const int i = i0 + ci, t = xt0 + n;
+        const bool valid = (i < Cin) && (t >= 0) && (t < T);
+        const float *src = valid ? xb + (size_t)i * T + t : xb;
+        cp_async4_zfill(dst + ci * XW + n, src, valid);
+      }
+      cp_async_commit();
+    };
+    // add finished run p into the row sums and hand its accumulator back
+    auto promote = [&](int p) {
+      const int ra = p & 1;
+      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 105);
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t v[32];
+        const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * BN + c0);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
+            "[%32];\n"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+              "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+              "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]),
+              "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+              "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+              "=r"(v[30]), "=r"(v[31])
+            : "r"(taddr)
+            : "memory");
+        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_run_free + 8 * ra);
+    };
+
+    stage_x(0);
+    int ready_blk = -1;
+    int promoted = 0;  // runs added so far
+    for (int c = 0; c < n_chunks; ++c) {
+      const int s = c % NSTAGE, u = c / NSTAGE;
+      const int kk0 = c * BK;
+      // x blocks hold CB channels = CB K kk, a multiple of BK: a chunk never
+      // straddles two blocks
+      const int blk = (kk0 / K) / CB;
+      const int m = c - blk * K;  // chunk index inside the block
+      if (blk > ready_blk) {
+        cp_async_wait_all();
+        conv_bar_sync();  // everyone's copies of this block landed; the old block is free
+        ready_blk = blk;
+        if ((blk + 1) * CB < Cin) stage_x(blk + 1);
+      }
+      if (u > 0) warp_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 103);
+      warp_wait(bar_full_a + 8 * s, u & 1, &ctl, status, 104);
+      // A: split in place into hi and lo (elementwise over the swizzled tile)
+      unsigned char *a_raw = smem + OFF_A + s * TILE_BYTES;
+      unsigned char *a_lo = smem + OFF_ALO + s * TILE_BYTES;
+#pragma unroll
+      for (int rr = 0; rr < TILE_BYTES / 16 / NCONV; ++rr) {
+        const int qo = (ct + rr * NCONV) * 16;
+        const float4 v = *reinterpret_cast<const float4 *>(a_raw + qo);
+        const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+        *reinterpret_cast<float4 *>(a_raw + qo) = h;
+        *reinterpret_cast<float4 *>(a_lo + qo) =
+            make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+      }
+      // B: row t = ct of the im2col chunk, block-local kk = 32 m .. 32 m + 31
+      unsigned char *b_hi = smem + OFF_BHI + s * TILE_BYTES;
+      unsigned char *b_lo = smem + OFF_BLO + s * TILE_BYTES;
+      const float *xrow = xs + (blk & 1) * CB * XW + ct;
+      const int *offs = xoff + m * BK;
+      float xv[BK];
+#pragma unroll
+      for (int e = 0; e < BK; e += 4) {
+        const int4 o4 = *reinterpret_cast<const int4 *>(offs + e);
+        xv[e] = xrow[o4.x];
+        xv[e + 1] = xrow[o4.y];
+        xv[e + 2] = xrow[o4.z];
+        xv[e + 3] = xrow[o4.w];
+      }
+#pragma unroll
+      for (int qq = 0; qq < BK / 4; ++qq) {
+        float hv[4], lv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hv[e] = tf32_hi(xv[4 * qq + e]);
+          lv[e] = xv[4 * qq + e] - hv[e];
+        }
+        const int off = sw128_off(ct, 4 * qq);
+        *reinterpret_cast<float4 *>(b_hi + off) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<float4 *>(b_lo + off) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      }
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_ready + 8 * s);
+      // a run whose MMAs were issued two chunks ago is complete by now
+      if (c >= (promoted + 1) * RUN + 1) promote(promoted++);
+    }
+    cp_async_wait_all();
+    while (promoted < n_runs) promote(promoted++);
+
+    // ------------------------------------------------------------- epilogue
+    float *ds = reinterpret_cast<float *>(smem);  // [BM][DS_PITCH]; operands are dead now
+    const int row = 32 * q + lane;
+#pragma unroll
+    for (int e = 0; e < BN; ++e) ds[row * DS_PITCH + e] = sum[e];
+    conv_bar_sync();
+    if (!ctl.abort) {
+      // row-contiguous write-out: each warp takes rows, lanes take columns
+      for (int r = q; r < BM; r += 4) {
+        const int o = o0 + r;
+        if (o >= Cout) break;
+        const float bo = bias ? __ldg(bias + o) : 0.0f;
+        const size_t rowoff = ((size_t)b * Cout + o) * y_pitch;
+        for (int cc = lane; cc < BN; cc += 32) {
+          const int t = t0 + cc;
+          if (t < y_len)
+            y[rowoff + t] = apply_epilogue(ds[r * DS_PITCH + cc], bo, ep, y, rowoff + t);
+        }
+      }
+    }
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == 1) {
+    // no MMA may still write an accumulator when it is freed
+    if (lane == 0 && n_runs > 0) {
+      mbar_drain(bar_run_full + 8 * ((n_runs - 1) & 1), ((n_runs - 1) >> 1) & 1);
+      if (n_runs > 1) mbar_drain(bar_run_full + 8 * ((n_runs - 2) & 1), ((n_runs - 2) >> 1) & 1);
+    }
+    __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                 "n"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  }
+  return fn;
+}
+
+}  // namespace
+
+bool conv1d_tc_supported(int Cin, int Cout, int K, int dil) {
+  return Cout >= 64 && K <= MAX_K && (Cin * K) % 4 == 0 && (K - 1) * dil <= MAX_HALO &&
+         Cin * K >= BK &&
+         encode_fn() != nullptr;
+}
+
+bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
+                           float *y, int y_len, int y_pitch, cudaStream_t st) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: no cuTensorMapEncodeTiled");
+  if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0)
+    return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: weights not 16-byte aligned");
+  CUtensorMap tmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)Cin * K, (cuuint64_t)Cout};
+  const cuuint64_t strides[1] = {(cuuint64_t)Cin * K * sizeof(float)};
+  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BV_ERR_CUDA, "conv1d_tc: tensor map encode failed (%d)", (int)r);
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(conv1d_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return check_launch("conv1d_tc smem attribute");
+    configured = true;
+  }
+  int *status = device_status_ptr();
+  dim3 grid((y_len + BN - 1) / BN, (Cout + BM - 1) / BM, B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
+  {
+    const double outs = (double)B * Cout * y_len;
+    LaunchTimer tm(st, "conv1d_tc", 2.0 * outs * Cin * K,
+                   4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
+                          outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
+    conv1d_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, x, bias, y, Cin, T, Cout, K, dil,
+                                                        pad, y_len, y_pitch, ep, status);
+  }
+  count_launch();
+  return check_launch("conv1d_tc_kernel");
+}
+
+}  // namespace bv

@@ -101,6 +101,7 @@ def lib():
     L.bv_timing_read.restype = c_int
     L.bv_filter_design.argtypes = [c_double, c_double, c_int, ctypes.POINTER(c_float)]
     L.bv_activation1d.argtypes = [_fp, _fp, c_int, c_int, c_int, _fp, _fp, _fp, _fp, c_float, _fp]
+    L.bv_sin_squared.argtypes = [_fp, _fp, ctypes.c_int64, _fp]
     L.bv_conv1d.argtypes = [_fp, c_int, c_int, c_int, _fp, _fp, c_int, c_int, c_int, c_int,
                             ctypes.POINTER(Epilogue), _fp, _fp]
     L.bv_conv_transpose1d.argtypes = [_fp, c_int, c_int, c_int, _fp, _fp, c_int, c_int, c_int,
@@ -199,6 +200,12 @@ def bv_activation1d(x, log_alpha, log_beta, up_filter, down_filter=None, eps=1e-
     _check(lib().bv_activation1d(_ptr(x), _ptr(y), B, C, T, _ptr(log_alpha), _ptr(log_beta),
                                  _ptr(up_filter), _ptr(down_filter), eps, _stream(stream)))
     return y
+
+
+def bv_sin_squared(z, out=None, stream=None):
+    out = torch.empty_like(z) if out is None else out
+    _check(lib().bv_sin_squared(_ptr(z), _ptr(out), z.numel(), _stream(stream)))
+    return out
 
 
 def bv_conv1d(x, w, bias, dilation=1, pad=None, residual=None, scale=1.0, accumulate=False,

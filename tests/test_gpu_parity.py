@@ -81,6 +81,26 @@ def test_activation_constant_rows_exact_form(nat, filt):
         np.testing.assert_allclose(y[0, c], want, rtol=2e-6, atol=2e-6)
 
 
+def test_sin_squared_accuracy(nat):
+    """The kernel's own sin^2 (Cody-Waite reduction by pi, Taylor series of
+    sin to r^13) against double precision, and against CUDA's sinf squared."""
+    rng = np.random.default_rng(0)
+    z = np.concatenate([np.linspace(-8, 8, 20001), rng.normal(0, 30, 200000),
+                        rng.uniform(-65536, 65536, 200000),
+                        np.array([0.0, np.pi / 2, np.pi, 1e-30, -1e-30, 65536.0, 65537.0,
+                                  1e5, -3e6, 1e30])]).astype(np.float32)
+    zd = dev(z)
+    got = host(nat.bv_sin_squared(zd)).astype(np.float64)
+    exact = np.sin(z.astype(np.float64)) ** 2
+    # the argument is exact (a float); the error is the reduction and series
+    err = np.abs(got - exact)
+    small = np.abs(z) <= 1024
+    assert err[small].max() < 4e-7, err[small].max()
+    assert err.max() < 4e-6, err.max()
+    cuda_sinf2 = host(torch.sin(zd)).astype(np.float64) ** 2
+    assert np.abs(got - cuda_sinf2)[small].max() < 5e-7
+
+
 def test_activation_full_size_sweep_point(nat, oracle, filt):
     """The activation workload at full size [2, 512, 65536], every element."""
     w = synth.ACT_SWEEP
@@ -204,6 +224,80 @@ def test_conv_transpose1d_general_kernel(nat, oracle):
         w = s.normal((10, 6, K), 0.0, 0.1)
         y = host(nat.bv_conv_transpose1d(dev(x), dev(w), None, S, pad))
         assert rel_l2(y, oracle.conv_transpose1d(x, w, None, S, pad)) < LAYER_TOL
+
+
+# Shapes that take the tensor-core path (tcgen05, 3xTF32): partial output
+# tiles (Cout not a multiple of 128), partial k chunks (Cin K not a multiple
+# of 32), partial input-channel blocks, short and ragged time axes, the
+# largest halo, and every epilogue.
+TC_CASES = [(64, 64, 3, 1, 200), (128, 128, 3, 1, 1), (128, 128, 7, 3, 5), (96, 96, 11, 5, 130),
+            (192, 192, 11, 5, 257), (12, 128, 3, 1, 129), (40, 200, 7, 1, 300),
+            (384, 384, 11, 5, 127), (768, 768, 3, 1, 400), (32, 1536, 7, 1, 77),
+            (256, 256, 7, 3, 1024), (100, 300, 11, 1, 513)]
+
+
+def _kernel_classes(nat, fn):
+    nat.timing(True)
+    nat.timing_reset()
+    try:
+        fn()
+        torch.cuda.synchronize()
+        return nat.timing_read()
+    finally:
+        nat.timing(False)
+        nat.timing_reset()
+
+
+@pytest.mark.parametrize("Cin,Cout,K,d,T", TC_CASES)
+def test_conv1d_tensor_core_path(nat, oracle, Cin, Cout, K, d, T):
+    s = synth.NormalStream(6000 + Cin + Cout + K * d + T)
+    B = 2
+    x = s.normal((B, Cin, T))
+    w = s.normal((Cout, Cin, K), 0.0, 0.02)
+    b = s.normal((Cout,), 0.0, 0.02)
+    pad = (K * d - d) // 2
+    xd, wd, bd = dev(x), dev(w), dev(b)
+    out = {}
+    classes = _kernel_classes(nat, lambda: out.setdefault(
+        "y", nat.bv_conv1d(xd, wd, bd, d, pad)))
+    assert "conv1d_tc" in classes, classes
+    y = host(out["y"])
+    want = oracle.conv1d(x, w, b, d, pad)
+    assert rel_l2(y, want) < LAYER_TOL
+
+
+@pytest.mark.parametrize("final_act", [0, 1, 2])
+def test_conv1d_tensor_core_epilogue(nat, oracle, final_act):
+    s = synth.NormalStream(70 + final_act)
+    C, T = 160, 300
+    x = s.normal((2, C, T))
+    w = s.normal((C, C, 7), 0.0, 0.05)
+    b = s.normal((C,), 0.0, 0.05)
+    r = s.normal((2, C, T))
+    y0 = s.normal((2, C, T))
+    yd = dev(y0)
+    nat.bv_conv1d(dev(x), dev(w), dev(b), 3, 9, residual=dev(r), scale=1.0 / 3.0,
+                  accumulate=True, final_act=final_act, y=yd)
+    got = host(yd).astype(np.float64)
+    conv = oracle.conv1d(x, w, b, 3, 9, store_f64=True).astype(np.float64)
+    want = (conv + r) * (1.0 / 3.0) + y0
+    if final_act == 1:
+        want = np.clip(want, -1, 1)
+    elif final_act == 2:
+        want = np.tanh(want)
+    assert rel_l2(got, want) < LAYER_TOL
+
+
+def test_conv1d_tensor_core_inplace_residual(nat, oracle):
+    s = synth.NormalStream(78)
+    C, T = 128, 1000
+    x = s.normal((2, C, T))
+    w = s.normal((C, C, 11), 0.0, 0.02)
+    cur = s.normal((2, C, T))
+    cd = dev(cur)
+    nat.bv_conv1d(dev(x), dev(w), None, 5, 25, residual=cd, y=cd)
+    want = oracle.conv1d(x, w, None, 5, 25, store_f64=True).astype(np.float64) + cur
+    assert rel_l2(host(cd), want) < LAYER_TOL
 
 
 # Full-size layer shapes of the MiniMax-H3 decoder, on seeded inputs,
