@@ -14,41 +14,71 @@
 //
 // Persistent CTAs walk row tiles of TILE outputs.  While a CTA computes one
 // tile, the next tile's input x[t0-8 .. t0+TILE+8) (clamped at the row ends)
-// is already streaming into the other half of a double buffer with cp.async
-// (16-byte copies when the row is 16-byte aligned and the tile is interior).
-// Per tile: stage A computes v[2 t0 - 6 + k], k < 2 TILE + 12, into shared
-// memory; stage B filters v into the TILE outputs.
+// streams into the other half of a double buffer with cp.async.  Per tile,
+// stage A computes v[2 t0 - 6 + k], k < 2 TILE + 12, into shared memory and
+// stage B filters v into the TILE outputs.  Each thread works on two
+// positions half a tile apart at once, with packed f32x2 arithmetic (FFMA2):
+// both positions have the same polyphase taps, so every filter tap and every
+// step of the sin^2 evaluation is one paired instruction.
 #include "common.cuh"
 #include "sin2.cuh"
 
 namespace bv {
 namespace {
 
-constexpr int TILE = 1024;         // outputs per tile
-constexpr int THREADS = 256;       // 4 outputs and 8 up-sampled values each
+constexpr int TILE = 2048;         // outputs per tile
+constexpr int HALF = TILE / 2;     // the two positions of a thread are HALF apart
+constexpr int THREADS = 256;       // per half tile: 4 outputs and 8 up-sampled values each
 constexpr int XS = TILE + 16;      // x[t0 - 8 + i]
 constexpr int VS = 2 * TILE + 16;  // v[2 t0 - 6 + k], k < 2 TILE + 12 used
+static_assert(HALF == 4 * THREADS, "one thread per 4 outputs of a half tile");
+
+__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+
+// Scalar SnakeBeta (tails and edge fix-ups).
+__device__ __forceinline__ float snake1(float u, float a, float inv_b) {
+  return fmaf(sin_squared(a * u), inv_b, u);
+}
+
+// Paired SnakeBeta: u + sin^2(a u) inv_b for two values, with the sin^2 of
+// sin2.cuh (reduction by pi in three parts, Taylor series of sin to r^13).
+// The nearest integer to z/pi comes from adding and removing 1.5 * 2^23.
+__device__ __forceinline__ float2 snake2(float2 u, float a, float inv_b) {
+  using namespace sin2c;
+  const float2 z = mul2(u, f2(a));
+  if (fmaxf(fabsf(z.x), fabsf(z.y)) > kFastLimit)
+    return make_float2(snake1(u.x, a, inv_b), snake1(u.y, a, inv_b));
+  const float2 k = add2(fma2(z, f2(kInvPi), f2(12582912.0f)), f2(-12582912.0f));
+  float2 r = fma2(k, f2(-kC1), z);
+  r = fma2(k, f2(-kC2), r);
+  r = fma2(k, f2(-kC3), r);
+  const float2 r2 = mul2(r, r);
+  float2 p = fma2(r2, f2(kT6), f2(kT5));
+  p = fma2(r2, p, f2(kT4));
+  p = fma2(r2, p, f2(kT3));
+  p = fma2(r2, p, f2(kT2));
+  p = fma2(r2, p, f2(kT1));
+  p = fma2(r2, p, f2(1.0f));
+  const float2 s = mul2(r, p);
+  return fma2(mul2(s, s), f2(inv_b), u);
+}
 
 struct Taps {
   float up2[12];  // 2 * f_up
   float dn[12];
 };
 
-__device__ __forceinline__ float snake(float u, float a, float inv_b) {
-  return fmaf(sin_squared(a * u), inv_b, u);
-}
-
-// u at phase r (0: even output index, 1: odd) from 6 consecutive x values
-// x0..x5 = x[p + r - 3 .. p + r + 2]:  u[2p+r] = sum_l 2 f[2l+1-r] x[p+2+r-l],
-// where term l pairs with x_{5-l}.
-__device__ __forceinline__ float up_phase(const Taps &tp, int r, float x0, float x1, float x2,
-                                          float x3, float x4, float x5) {
-  if (r == 0) {
-    return tp.up2[1] * x5 + tp.up2[3] * x4 + tp.up2[5] * x3 + tp.up2[7] * x2 + tp.up2[9] * x1 +
-           tp.up2[11] * x0;
-  }
-  return tp.up2[0] * x5 + tp.up2[2] * x4 + tp.up2[4] * x3 + tp.up2[6] * x2 + tp.up2[8] * x1 +
-         tp.up2[10] * x0;
+// u at phase r (0: even index, 1: odd) from six consecutive x values
+// xp[0..5] = x[p + r - 3 .. p + r + 2]:  u[2p+r] = sum_l 2 f[2l+1-r] x[p+2+r-l],
+// where term l pairs with xp[5-l].
+__device__ __forceinline__ float up1(const Taps &tp, int r, const float *xp) {
+  float u = tp.up2[1 - r] * xp[5];
+#pragma unroll
+  for (int l = 1; l < 6; ++l) u = fmaf(tp.up2[2 * l + 1 - r], xp[5 - l], u);
+  return u;
 }
 
 __device__ __forceinline__ void cp_async4(float *dst, const float *src) {
@@ -67,12 +97,9 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Issue the copies of tile `tile_id`'s input into xs (x[t0 - 8 + i], clamped).
-__device__ __forceinline__ void issue_tile(const float *__restrict__ x, float *xs,
-                                           long long tile_id, int tiles_per_row, int T, int tid) {
-  const long long row = tile_id / tiles_per_row;
-  const int t0 = (int)(tile_id - row * tiles_per_row) * TILE;
-  const float *xr = x + row * (long long)T;
+// Issue the copies of one tile's input into xs: x[t0 - 8 + i], clamped.
+__device__ __forceinline__ void issue_tile(const float *__restrict__ xr, float *xs, int t0, int T,
+                                           int tid) {
   const bool vec =
       ((reinterpret_cast<uintptr_t>(xr) & 15u) == 0) && (t0 >= 8) && (t0 + TILE + 8 <= T);
   if (vec) {
@@ -87,13 +114,26 @@ __device__ __forceinline__ void issue_tile(const float *__restrict__ x, float *x
   }
 }
 
+__device__ __forceinline__ void store4(float *yr, int t, int T, float o0, float o1, float o2,
+                                       float o3) {
+  if (t + 3 < T && ((reinterpret_cast<uintptr_t>(yr + t) & 15u) == 0)) {
+    __stcs(reinterpret_cast<float4 *>(yr + t), make_float4(o0, o1, o2, o3));
+  } else {
+    if (t < T) yr[t] = o0;
+    if (t + 1 < T) yr[t + 1] = o1;
+    if (t + 2 < T) yr[t + 2] = o2;
+    if (t + 3 < T) yr[t + 3] = o3;
+  }
+}
+
 __global__ void __launch_bounds__(THREADS)
 activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int T,
-                  int tiles_per_row, long long n_tiles, const float *__restrict__ log_alpha,
+                  int tiles_per_row, int n_tiles, const float *__restrict__ log_alpha,
                   const float *__restrict__ log_beta, const float *__restrict__ f_up,
                   const float *__restrict__ f_dn, float eps) {
   __shared__ __align__(16) float xs[2][XS];
   __shared__ __align__(16) float vs[VS];
+  __shared__ float snake_ab[2];  // a, inv_b of the current tile's channel
   const int tid = threadIdx.x;
 
   Taps tp;
@@ -103,93 +143,121 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
     tp.dn[j] = __ldg(f_dn + j);
   }
 
-  long long tile_id = blockIdx.x;
-  if (tile_id < n_tiles) issue_tile(x, xs[0], tile_id, tiles_per_row, T, tid);
+  // tiles are visited as tile_id = blockIdx.x + k gridDim.x; (row, tile) are
+  // carried along incrementally
+  const int step_row = gridDim.x / tiles_per_row, step_tile = gridDim.x % tiles_per_row;
+  int tile_id = blockIdx.x;
+  int row = tile_id / tiles_per_row, tile = tile_id % tiles_per_row;
+  if (tile_id < n_tiles) issue_tile(x + (size_t)row * T, xs[0], tile * TILE, T, tid);
   cp_async_commit();
   int buf = 0;
   for (; tile_id < n_tiles; tile_id += gridDim.x, buf ^= 1) {
-    const long long next = tile_id + gridDim.x;
-    if (next < n_tiles) issue_tile(x, xs[buf ^ 1], next, tiles_per_row, T, tid);
+    int nrow = row + step_row, ntile = tile + step_tile;
+    if (ntile >= tiles_per_row) {
+      ntile -= tiles_per_row;
+      ++nrow;
+    }
+    if (tile_id + (int)gridDim.x < n_tiles)
+      issue_tile(x + (size_t)nrow * T, xs[buf ^ 1], ntile * TILE, T, tid);
     cp_async_commit();
+    if (tid == 0) {
+      const int c = row % C;
+      snake_ab[0] = expf(__ldg(log_alpha + c));
+      snake_ab[1] = 1.0f / (expf(__ldg(log_beta + c)) + eps);
+    }
     cp_async_wait<1>();  // this tile's copies are done; the next tile's may be in flight
     __syncthreads();
 
-    const long long row = tile_id / tiles_per_row;
-    const int t0 = (int)(tile_id - row * tiles_per_row) * TILE;
-    const int c = (int)(row % C);
-    const float a = expf(__ldg(log_alpha + c));
-    const float inv_b = 1.0f / (expf(__ldg(log_beta + c)) + eps);
+    const int t0 = tile * TILE;
+    const float a = snake_ab[0], inv_b = snake_ab[1];
     const float *xb = xs[buf];
 
-    // ---- stage A: v[m] for m = 2 t0 - 6 + k, k in [0, 2 TILE + 12)
-    const bool interior = (2 * t0 - 6 >= 0) && (2 * t0 + 2 * TILE + 5 <= 2 * T - 1);
-    if (interior) {
-      // k = 2q + r, p = t0 - 3 + q; x[p + r - 3 + k'] = x[t0 - 6 + q + r + k'] sits at
-      // xb[2 + q + r + k'].  Thread owns q in [4 tid, 4 tid + 4).
+    // ---- stage A: v[2 t0 - 6 + k]; k = 2q + r holds p = t0 - 3 + q and
+    // x[p + r - 3 + k'] sits at xb[2 + q + r + k'].  The thread owns
+    // q in [4 tid, 4 tid + 4) of each half tile.
+    {
       const int q0 = 4 * tid;
-      const float4 w0 = *reinterpret_cast<const float4 *>(xb + q0);
-      const float4 w1 = *reinterpret_cast<const float4 *>(xb + q0 + 4);
-      const float4 w2 = *reinterpret_cast<const float4 *>(xb + q0 + 8);
-      const float xw[12] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y,
-                            w1.z, w1.w, w2.x, w2.y, w2.z, w2.w};
-      float vv[8];
+      float2 X[12];
+#pragma unroll
+      for (int w = 0; w < 3; ++w) {
+        const float4 lo = *reinterpret_cast<const float4 *>(xb + q0 + 4 * w);
+        const float4 hi = *reinterpret_cast<const float4 *>(xb + HALF + q0 + 4 * w);
+        X[4 * w] = make_float2(lo.x, hi.x);
+        X[4 * w + 1] = make_float2(lo.y, hi.y);
+        X[4 * w + 2] = make_float2(lo.z, hi.z);
+        X[4 * w + 3] = make_float2(lo.w, hi.w);
+      }
+      float2 V[8];
 #pragma unroll
       for (int qq = 0; qq < 4; ++qq) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
           const int b0 = 2 + qq + r;
-          const float u = up_phase(tp, r, xw[b0], xw[b0 + 1], xw[b0 + 2], xw[b0 + 3],
-                                   xw[b0 + 4], xw[b0 + 5]);
-          vv[2 * qq + r] = snake(u, a, inv_b);
+          float2 u = mul2(f2(tp.up2[1 - r]), X[b0 + 5]);
+#pragma unroll
+          for (int l = 1; l < 6; ++l) u = fma2(f2(tp.up2[2 * l + 1 - r]), X[b0 + 5 - l], u);
+          V[2 * qq + r] = snake2(u, a, inv_b);
         }
       }
-      *reinterpret_cast<float4 *>(vs + 2 * q0) = make_float4(vv[0], vv[1], vv[2], vv[3]);
-      *reinterpret_cast<float4 *>(vs + 2 * q0 + 4) = make_float4(vv[4], vv[5], vv[6], vv[7]);
-      if (tid < 12) {  // k in [2 TILE, 2 TILE + 12): q in [TILE, TILE + 6)
+      *reinterpret_cast<float4 *>(vs + 2 * q0) = make_float4(V[0].x, V[1].x, V[2].x, V[3].x);
+      *reinterpret_cast<float4 *>(vs + 2 * q0 + 4) = make_float4(V[4].x, V[5].x, V[6].x, V[7].x);
+      *reinterpret_cast<float4 *>(vs + 2 * HALF + 2 * q0) =
+          make_float4(V[0].y, V[1].y, V[2].y, V[3].y);
+      *reinterpret_cast<float4 *>(vs + 2 * HALF + 2 * q0 + 4) =
+          make_float4(V[4].y, V[5].y, V[6].y, V[7].y);
+      if (tid < 12) {  // k in [2 TILE, 2 TILE + 12)
         const int k = 2 * TILE + tid;
         const int q = k >> 1, r = k & 1;
-        const float *xp = xb + 2 + q + r;
-        vs[k] = snake(up_phase(tp, r, xp[0], xp[1], xp[2], xp[3], xp[4], xp[5]), a, inv_b);
+        vs[k] = snake1(up1(tp, r, xb + 2 + q + r), a, inv_b);
       }
-    } else {
-      // edge tiles: clamp m into [0, 2T - 1] and take v there
-      for (int k = tid; k < 2 * TILE + 12; k += THREADS) {
-        int m = 2 * t0 - 6 + k;
-        m = m < 0 ? 0 : (m > 2 * T - 1 ? 2 * T - 1 : m);
-        const int p = m >> 1, r = m & 1;
-        // x[p + r - 3 + k'] sits at xb[p + r - 3 + k' - (t0 - 8)]
-        const float *xp = xb + (p + r + 5 - t0);
-        vs[k] = snake(up_phase(tp, r, xp[0], xp[1], xp[2], xp[3], xp[4], xp[5]), a, inv_b);
+    }
+    // Near a row end the pages pad the 2x signal by replication: v at an index
+    // m outside [0, 2T-1] is v at the clamped index.  Only m in [-6, -1] and
+    // [2T, 2T + 4] are read by outputs t < T.
+    const bool edge = (2 * t0 - 6 < 0) || (2 * t0 + 2 * TILE + 5 > 2 * T - 1);
+    if (edge) {
+      __syncthreads();
+      if (tid < 11) {
+        const int m = tid < 6 ? tid - 6 : 2 * T + (tid - 6);
+        const int k = m - (2 * t0 - 6);
+        if (k >= 0 && k < 2 * TILE + 12) {
+          const int mc = m < 0 ? 0 : 2 * T - 1;
+          const int p = mc >> 1, r = mc & 1;
+          // x[p + r - 3 + k'] sits at xb[p + r + 5 - t0 + k'] (in range: the tile
+          // reaches that row end)
+          vs[k] = snake1(up1(tp, r, xb + (p + r + 5 - t0)), a, inv_b);
+        }
       }
     }
     __syncthreads();
 
     // ---- stage B: y[t] = sum_j f_dn[j] v[2t + j - 5]; v[2t + j - 5] is vs[2 (t - t0) + j + 1]
-    const int tl = 4 * tid;
-    const float4 a0 = *reinterpret_cast<const float4 *>(vs + 2 * tl);
-    const float4 a1 = *reinterpret_cast<const float4 *>(vs + 2 * tl + 4);
-    const float4 a2 = *reinterpret_cast<const float4 *>(vs + 2 * tl + 8);
-    const float4 a3 = *reinterpret_cast<const float4 *>(vs + 2 * tl + 12);
-    const float4 a4 = *reinterpret_cast<const float4 *>(vs + 2 * tl + 16);
-    const float vw[20] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w, a2.x, a2.y,
-                          a2.z, a2.w, a3.x, a3.y, a3.z, a3.w, a4.x, a4.y, a4.z, a4.w};
-    float out[4];
+    {
+      const int tl = 4 * tid;
+      float2 W[20];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float acc = 0.0f;
+      for (int w = 0; w < 5; ++w) {
+        const float4 lo = *reinterpret_cast<const float4 *>(vs + 2 * tl + 4 * w);
+        const float4 hi = *reinterpret_cast<const float4 *>(vs + 2 * HALF + 2 * tl + 4 * w);
+        W[4 * w] = make_float2(lo.x, hi.x);
+        W[4 * w + 1] = make_float2(lo.y, hi.y);
+        W[4 * w + 2] = make_float2(lo.z, hi.z);
+        W[4 * w + 3] = make_float2(lo.w, hi.w);
+      }
+      float2 out[4];
 #pragma unroll
-      for (int j = 0; j < 12; ++j) acc = fmaf(tp.dn[j], vw[2 * e + j + 1], acc);
-      out[e] = acc;
+      for (int e = 0; e < 4; ++e) {
+        float2 acc = mul2(f2(tp.dn[0]), W[2 * e + 1]);
+#pragma unroll
+        for (int j = 1; j < 12; ++j) acc = fma2(f2(tp.dn[j]), W[2 * e + j + 1], acc);
+        out[e] = acc;
+      }
+      float *yr = y + (size_t)row * T;
+      store4(yr, t0 + tl, T, out[0].x, out[1].x, out[2].x, out[3].x);
+      store4(yr, t0 + HALF + tl, T, out[0].y, out[1].y, out[2].y, out[3].y);
     }
-    float *yr = y + row * (long long)T;
-    const int t = t0 + tl;
-    if (t + 3 < T && ((reinterpret_cast<uintptr_t>(yr + t) & 15u) == 0)) {
-      __stcs(reinterpret_cast<float4 *>(yr + t), make_float4(out[0], out[1], out[2], out[3]));
-    } else {
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        if (t + e < T) yr[t + e] = out[e];
-    }
+    row = nrow;
+    tile = ntile;
   }
   cp_async_wait<0>();
 }
@@ -201,7 +269,7 @@ __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restric
     out[i] = sin_squared(z[i]);
 }
 
-// CTAs that are resident at once for the activation kernel on this device.
+// CTAs resident at once for the activation kernel on this device.
 int persistent_ctas() {
   static int n = 0;
   if (n == 0) {
@@ -235,12 +303,13 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
   const int tiles = (T + TILE - 1) / TILE;
   const long long n_tiles = rows * tiles;
   if (n_tiles <= 0) return BV_OK;
+  if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "activation: too many tiles");
   const int ctas = persistent_ctas();
   const long long grid = n_tiles < ctas ? n_tiles : ctas;
   {
     LaunchTimer tm(st, "activation", 0.0, 8.0 * (double)rows * T);
-    activation_kernel<<<(unsigned)grid, THREADS, 0, st>>>(x, y, C, T, tiles, n_tiles, la, lb,
-                                                          fu, fd, eps);
+    activation_kernel<<<(unsigned)grid, THREADS, 0, st>>>(x, y, C, T, tiles, (int)n_tiles, la,
+                                                          lb, fu, fd, eps);
   }
   count_launch();
   return check_launch("activation_kernel");

@@ -53,14 +53,17 @@ constexpr int MAX_K = 32;           // largest kernel size (offset table rows)
 constexpr int DS_PITCH = BN + 1;    // epilogue staging row pitch (floats)
 
 // shared memory layout (bytes from a 1024-aligned base)
-constexpr int OFF_A = 0;                                  // A raw -> A_hi, per stage
+constexpr int NRAW = 2;                                   // TMA ring of raw weight chunks
+constexpr int OFF_A = 0;                                  // A_hi, per operand stage
 constexpr int OFF_ALO = OFF_A + NSTAGE * TILE_BYTES;      // A_lo
 constexpr int OFF_BHI = OFF_ALO + NSTAGE * TILE_BYTES;    // B_hi
 constexpr int OFF_BLO = OFF_BHI + NSTAGE * TILE_BYTES;    // B_lo
-constexpr int OFF_X = OFF_BLO + NSTAGE * TILE_BYTES;      // x blocks [2][CB][XW]
+constexpr int OFF_RAW = OFF_BLO + NSTAGE * TILE_BYTES;    // raw A chunks from TMA
+constexpr int OFF_X = OFF_RAW + NRAW * TILE_BYTES;        // x blocks [2][CB][XW]
 constexpr int X_BYTES = 2 * CB * XW * 4;
 constexpr int OFF_BAR = OFF_X + X_BYTES;                  // mbarriers
 constexpr int SMEM_USED = OFF_BAR + 256;
+static_assert(SMEM_USED + 1024 + 4 * 1024 + 64 <= 227 * 1024, "shared memory budget");
 constexpr int SMEM_BYTES = SMEM_USED + 1024;              // room to align the base
 static_assert(BM * DS_PITCH * 4 <= OFF_X, "epilogue staging must fit in the operand area");
 
@@ -182,13 +185,15 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   __shared__ Ctl ctl;
   __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block, entry e
-  // barriers: A landed (TMA) / operands ready / stage free, per stage; run
-  // accumulated / run accumulator read, per TMEM accumulator
+  // barriers: raw A landed (TMA) / raw A read, per raw slot; operands ready /
+  // operand stage free, per stage; run accumulated / run accumulator read,
+  // per TMEM accumulator
   const unsigned bar_full_a = smem_u32(&bars[0]);
   const unsigned bar_ready = smem_u32(&bars[2]);
   const unsigned bar_empty = smem_u32(&bars[4]);
   const unsigned bar_run_full = smem_u32(&bars[6]);
   const unsigned bar_run_free = smem_u32(&bars[8]);
+  const unsigned bar_raw_free = smem_u32(&bars[10]);
   float *xs = reinterpret_cast<float *>(smem + OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -204,11 +209,14 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
   if (threadIdx.x == 0) {
     ctl.abort = 0;
     for (int s = 0; s < NSTAGE; ++s) {
-      mbar_init(bar_full_a + 8 * s, 1);
       mbar_init(bar_ready + 8 * s, NCONV / 32);
       mbar_init(bar_empty + 8 * s, 1);
       mbar_init(bar_run_full + 8 * s, 1);
       mbar_init(bar_run_free + 8 * s, NCONV / 32);
+    }
+    for (int s = 0; s < NRAW; ++s) {
+      mbar_init(bar_full_a + 8 * s, 1);
+      mbar_init(bar_raw_free + 8 * s, NCONV / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -233,11 +241,12 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % NSTAGE, u = c / NSTAGE;
+        const int s = c % NRAW, u = c / NRAW;
         // After an abort every wait returns at once and the loops run to the end
-        // without blocking, so all roles reach the final barrier.
-        if (u > 0) mbar_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 101);
-        const unsigned dst = smem_u32(smem + OFF_A + s * TILE_BYTES);
+        // without blocking, so all roles reach the final barrier.  The raw slot
+        // is free once the converters have split the chunk it held.
+        if (u > 0) mbar_wait(bar_raw_free + 8 * s, (u - 1) & 1, &ctl, status, 101);
+        const unsigned dst = smem_u32(smem + OFF_RAW + s * TILE_BYTES);
         mbar_arrive_tx(bar_full_a + 8 * s, TILE_BYTES);
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
@@ -247,8 +256,8 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
             : "memory");
       }
       // drain: the last loads of each stage must land before the CTA can exit
-      for (int c = n_chunks - NSTAGE; c < n_chunks; ++c)
-        if (c >= 0) mbar_drain(bar_full_a + 8 * (c % NSTAGE), (c / NSTAGE) & 1);
+      for (int c = n_chunks - NRAW; c < n_chunks; ++c)
+        if (c >= 0) mbar_drain(bar_full_a + 8 * (c % NRAW), (c / NRAW) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -353,17 +362,25 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
         ready_blk = blk;
         if ((blk + 1) * CB < Cin) stage_x(blk + 1);
       }
+      const int sr = c % NRAW;
       if (u > 0) warp_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 103);
-      warp_wait(bar_full_a + 8 * s, u & 1, &ctl, status, 104);
-      // A: split in place into hi and lo (elementwise over the swizzled tile)
-      unsigned char *a_raw = smem + OFF_A + s * TILE_BYTES;
+      warp_wait(bar_full_a + 8 * sr, (c / NRAW) & 1, &ctl, status, 104);
+      // A: split into hi and lo (elementwise over the swizzled tile)
+      const unsigned char *a_raw = smem + OFF_RAW + sr * TILE_BYTES;
+      unsigned char *a_hi = smem + OFF_A + s * TILE_BYTES;
       unsigned char *a_lo = smem + OFF_ALO + s * TILE_BYTES;
+      float4 av[TILE_BYTES / 16 / NCONV];
+#pragma unroll
+      for (int rr = 0; rr < TILE_BYTES / 16 / NCONV; ++rr)
+        av[rr] = *reinterpret_cast<const float4 *>(a_raw + (ct + rr * NCONV) * 16);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_raw_free + 8 * sr);  // the TMA may refill the slot
 #pragma unroll
       for (int rr = 0; rr < TILE_BYTES / 16 / NCONV; ++rr) {
         const int qo = (ct + rr * NCONV) * 16;
-        const float4 v = *reinterpret_cast<const float4 *>(a_raw + qo);
+        const float4 v = av[rr];
         const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-        *reinterpret_cast<float4 *>(a_raw + qo) = h;
+        *reinterpret_cast<float4 *>(a_hi + qo) = h;
         *reinterpret_cast<float4 *>(a_lo + qo) =
             make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
       }
