@@ -5,26 +5,26 @@
 // (docs.rs cortiq-engine audiovae.rs `Conv1d::apply`, whose note states the
 // im2col identity used here; ltxaudio.rs `Conv1d::forward`).
 //
-// GEMM view: D[o, t] = sum_kk A[o, kk] B[kk, t] with kk = i K + j (the order
-// of w's own [Cout][Cin][K] layout, so A is w read as a [Cout, Cin K] matrix)
-// and B[kk, t] = x[b, i, t + j d - pad] (im2col, never materialised).
-// Each CTA owns a 128 (o) x 128 (t) output tile and walks kk in chunks of 32:
-//   - a TMA load brings the weight chunk A [128 x 32] into shared memory in
-//     the 128-byte-swizzled K-major layout the tensor core reads;
-//   - four converter warps split it in place into A_hi = tf32(A) (low 13
-//     mantissa bits cleared) and A_lo = A - A_hi, and build B_hi / B_lo
-//     [128 t x 32 kk] (K-major, same swizzle) from input rows staged in shared
-//     memory with cp.async;
+// GEMM view: D[t, o] = sum_kk X[t, kk] W[o, kk] with kk = i K + j (the order of
+// w's own [Cout][Cin][K] layout, so W is w read as a [Cout, Cin K] matrix) and
+// X[t, kk] = x[b, i, t + j d - pad] (im2col, never materialised).  Time is the
+// MMA's M side (128 per CTA) and output channels its N side (NT per CTA, a
+// multiple of 16 sized to Cout, so narrow layers waste no tensor work).
+// Each CTA walks kk in chunks of 32 (one 128-byte swizzle row of fp32):
+//   - TMA brings the weight chunk W [NT x 32] into a ring of raw slots;
+//   - four converter warps split it into W_hi = tf32(W) (low 13 mantissa bits
+//     cleared) and W_lo = W - W_hi, and build X_hi / X_lo [128 t x 32 kk] from
+//     input rows staged in shared memory with cp.async, all in the K-major
+//     128-byte-swizzled layout the tensor core reads;
 //   - one thread issues three tcgen05.mma.kind::tf32 per 8-wide k step,
-//     A_hi B_hi + A_hi B_lo + A_lo B_hi, into one FP32 TMEM accumulator (the
-//     3xTF32 scheme: the dropped A_lo B_lo term is 2^-22 relative);
-//   - runs of RUN chunks accumulate in one of two TMEM accumulators, starting
-//     from zero; the converter warps read each finished run and add it into
-//     FP32 registers (the tensor core's accumulation truncates, so its error
-//     would otherwise grow with Cin K);
-//   - the epilogue adds bias / residual, scales, accumulates and applies the
-//     final op, staged through shared memory so that global reads and writes
-//     are row-contiguous.
+//     X_lo W_hi + X_hi W_lo + X_hi W_hi, into an FP32 TMEM accumulator (the
+//     3xTF32 scheme: the dropped X_lo W_lo term is 2^-22 relative);
+//   - runs of RUN chunks accumulate in one of two TMEM accumulators starting
+//     from zero, and the converter warps add each finished run into FP32
+//     registers: the tensor core's accumulation truncates, so its error would
+//     otherwise grow with Cin K;
+//   - the epilogue (bias, residual, scale, accumulate, final op) has one
+//     thread per time sample, so global reads and writes are coalesced.
 // Two operand stages overlap conversion with the MMAs.  Every mbarrier wait
 // is bounded; a wait that runs out sets the device status word and the CTA
 // unwinds (its output tile is then unspecified) after freeing its TMEM.
@@ -35,37 +35,36 @@
 namespace bv {
 namespace {
 
-constexpr int BM = 128;             // output channels per CTA (UMMA M)
-constexpr int BN = 128;             // time samples per CTA (UMMA N)
-constexpr int BK = 32;              // kk per chunk: one 128-byte swizzle row of fp32
-constexpr int NSTAGE = 2;           // operand stages
-constexpr int CB = 32;              // input channels per staged x block
-constexpr int MAX_HALO = 56;        // (K - 1) d the staged rows can hold
-constexpr int XW = BN + MAX_HALO + 8;  // staged row width (floats)
-constexpr int TILE_BYTES = BM * BK * 4;  // 16 KB: one A or B operand tile
+constexpr int BM = 128;                  // time samples per CTA (UMMA M)
+constexpr int MAX_NT = 128;              // output channels per CTA (UMMA N), at most
+constexpr int BK = 32;                   // kk per chunk
+constexpr int NSTAGE = 2;                // operand stages
+constexpr int NRAW = 2;                  // TMA ring of raw weight chunks
+constexpr int CB = 32;                   // input channels per staged x block
+constexpr int MAX_HALO = 56;             // (K - 1) d the staged rows can hold
+constexpr int XW = BM + MAX_HALO + 8;    // staged row width (floats)
+constexpr int X_TILE = BM * BK * 4;      // 16 KB: one im2col operand tile
+constexpr int W_TILE = MAX_NT * BK * 4;  // 16 KB: one weight operand tile (at most)
 constexpr int THREADS = 256;
-constexpr int CONV_WARP0 = 4;       // warps 4..7 convert and run the epilogue
+constexpr int CONV_WARP0 = 4;            // warps 4..7 convert, add runs, write out
 constexpr int NCONV = 128;
 constexpr long long WAIT_LIMIT = 1ll << 26;  // try_wait polls before giving up
-constexpr int TMEM_COLS = 256;     // two 128-column accumulators
-constexpr int RUN = 4;              // chunks accumulated in TMEM before an FP32 add
-constexpr int MAX_K = 32;           // largest kernel size (offset table rows)
-constexpr int DS_PITCH = BN + 1;    // epilogue staging row pitch (floats)
+constexpr int TMEM_COLS = 256;           // two accumulators of up to 128 columns
+constexpr int RUN = 4;                   // chunks accumulated in TMEM before an FP32 add
+constexpr int MAX_K = 32;                // largest kernel size (offset table rows)
 
 // shared memory layout (bytes from a 1024-aligned base)
-constexpr int NRAW = 2;                                   // TMA ring of raw weight chunks
-constexpr int OFF_A = 0;                                  // A_hi, per operand stage
-constexpr int OFF_ALO = OFF_A + NSTAGE * TILE_BYTES;      // A_lo
-constexpr int OFF_BHI = OFF_ALO + NSTAGE * TILE_BYTES;    // B_hi
-constexpr int OFF_BLO = OFF_BHI + NSTAGE * TILE_BYTES;    // B_lo
-constexpr int OFF_RAW = OFF_BLO + NSTAGE * TILE_BYTES;    // raw A chunks from TMA
-constexpr int OFF_X = OFF_RAW + NRAW * TILE_BYTES;        // x blocks [2][CB][XW]
+constexpr int OFF_XHI = 0;                               // per operand stage
+constexpr int OFF_XLO = OFF_XHI + NSTAGE * X_TILE;
+constexpr int OFF_WHI = OFF_XLO + NSTAGE * X_TILE;
+constexpr int OFF_WLO = OFF_WHI + NSTAGE * W_TILE;
+constexpr int OFF_RAW = OFF_WLO + NSTAGE * W_TILE;       // raw weight chunks from TMA
+constexpr int OFF_X = OFF_RAW + NRAW * W_TILE;           // x blocks [2][CB][XW]
 constexpr int X_BYTES = 2 * CB * XW * 4;
-constexpr int OFF_BAR = OFF_X + X_BYTES;                  // mbarriers
+constexpr int OFF_BAR = OFF_X + X_BYTES;                 // mbarriers
 constexpr int SMEM_USED = OFF_BAR + 256;
-static_assert(SMEM_USED + 1024 + 4 * 1024 + 64 <= 227 * 1024, "shared memory budget");
-constexpr int SMEM_BYTES = SMEM_USED + 1024;              // room to align the base
-static_assert(BM * DS_PITCH * 4 <= OFF_X, "epilogue staging must fit in the operand area");
+constexpr int SMEM_BYTES = SMEM_USED + 1024;             // room to align the base
+static_assert(SMEM_BYTES + 4 * 1024 + 64 <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) {
   return (unsigned)__cvta_generic_to_shared(p);
@@ -93,8 +92,8 @@ __device__ __forceinline__ bool mbar_try_wait(unsigned bar, unsigned parity) {
 }
 
 struct Ctl {
-  int abort;        // a bounded wait gave up somewhere in the CTA
-  unsigned tmem;    // TMEM base address from tcgen05.alloc
+  int abort;      // a bounded wait gave up somewhere in the CTA
+  unsigned tmem;  // TMEM base address from tcgen05.alloc
 };
 
 // Bounded wait on an mbarrier phase.  On running out it marks the CTA
@@ -115,6 +114,14 @@ __device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, volatil
 __device__ __forceinline__ void mbar_drain(unsigned bar, unsigned parity) {
   for (long long it = 0; it < (1ll << 22); ++it)
     if (mbar_try_wait(bar, parity)) return;
+}
+
+// Converter-side wait: lane 0 polls the barrier, the warp follows it, so the
+// polling does not compete with the conversion for shared-memory bandwidth.
+__device__ __forceinline__ void warp_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
+                                          int *status, int code) {
+  if ((threadIdx.x & 31) == 0) mbar_wait(bar, parity, ctl, status, code);
+  __syncwarp();
 }
 
 __device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool valid) {
@@ -140,21 +147,24 @@ __device__ __forceinline__ uint64_t sw128_desc(unsigned addr) {
          ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
-// Instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = 128.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(BN >> 3) << 17) |
-                            ((uint32_t)(BM >> 4) << 24);
+// Instruction descriptor: D f32, A and B tf32, both K-major, M = 128, N = nt.
+__host__ __device__ constexpr uint32_t make_idesc(int nt) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(nt >> 3) << 17) |
+         ((uint32_t)(BM >> 4) << 24);
+}
 
-__device__ __forceinline__ void mma_tf32(unsigned tmem_d, uint64_t a, uint64_t b, unsigned acc) {
+__device__ __forceinline__ void mma_tf32(unsigned tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         unsigned acc) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(acc)
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
       : "memory");
 }
 __device__ __forceinline__ void mma_commit(unsigned bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(
-                   bar)
-               : "memory");
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(bar)
+      : "memory");
 }
 
 // Byte offset of element (row r, column k < 32) in a K-major SW128 tile of
@@ -167,38 +177,34 @@ __device__ __forceinline__ float tf32_hi(float v) {
   return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
 }
 
-// Converter-side wait: lane 0 polls the barrier, the warp follows it, so the
-// polling does not compete with the conversion for shared-memory bandwidth.
-__device__ __forceinline__ void warp_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
-                                          int *status, int code) {
-  if ((threadIdx.x & 31) == 0) mbar_wait(bar, parity, ctl, status, code);
-  __syncwarp();
-}
-
+template <int NT>
 __global__ void __launch_bounds__(THREADS, 1)
 conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ x,
                  const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
                  int dil, int pad, int y_len, int y_pitch, Epi ep, int *status) {
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
+  constexpr int W_BYTES = NT * BK * 4;  // bytes of one weight chunk (TMA box)
+  constexpr uint32_t IDESC = make_idesc(NT);
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   __shared__ Ctl ctl;
-  __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block, entry e
-  // barriers: raw A landed (TMA) / raw A read, per raw slot; operands ready /
-  // operand stage free, per stage; run accumulated / run accumulator read,
-  // per TMEM accumulator
-  const unsigned bar_full_a = smem_u32(&bars[0]);
-  const unsigned bar_ready = smem_u32(&bars[2]);
-  const unsigned bar_empty = smem_u32(&bars[4]);
-  const unsigned bar_run_full = smem_u32(&bars[6]);
-  const unsigned bar_run_free = smem_u32(&bars[8]);
-  const unsigned bar_raw_free = smem_u32(&bars[10]);
+  __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block
+  // barriers: raw weights landed (TMA) / raw weights read, per raw slot;
+  // operands ready / operand stage free, per stage; run accumulated / run
+  // accumulator read, per TMEM accumulator
+  const unsigned bar_full_w = smem_u32(&bars[0]);
+  const unsigned bar_raw_free = smem_u32(&bars[2]);
+  const unsigned bar_ready = smem_u32(&bars[4]);
+  const unsigned bar_empty = smem_u32(&bars[6]);
+  const unsigned bar_run_full = smem_u32(&bars[8]);
+  const unsigned bar_run_free = smem_u32(&bars[10]);
   float *xs = reinterpret_cast<float *>(smem + OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * BN;
-  const int o0 = blockIdx.y * BM;
+  const int t0 = blockIdx.x * BM;
+  const int o0 = blockIdx.y * NT;
   const int b = blockIdx.z;
   const int KK = Cin * K;
   const int n_chunks = (KK + BK - 1) / BK;
@@ -208,15 +214,13 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
 
   if (threadIdx.x == 0) {
     ctl.abort = 0;
-    for (int s = 0; s < NSTAGE; ++s) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_full_w + 8 * s, 1);
+      mbar_init(bar_raw_free + 8 * s, NCONV / 32);
       mbar_init(bar_ready + 8 * s, NCONV / 32);
       mbar_init(bar_empty + 8 * s, 1);
       mbar_init(bar_run_full + 8 * s, 1);
       mbar_init(bar_run_free + 8 * s, NCONV / 32);
-    }
-    for (int s = 0; s < NRAW; ++s) {
-      mbar_init(bar_full_a + 8 * s, 1);
-      mbar_init(bar_raw_free + 8 * s, NCONV / 32);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
@@ -225,7 +229,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     const int i = idx / K, j = idx - i * K;
     xoff[idx] = i * XW + j * dil;
   }
-  if (warp == 1) {  // two TMEM accumulators of 128 lanes x 128 fp32 columns
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      smem_u32(&ctl.tmem)),
                  "n"(TMEM_COLS)
@@ -243,28 +247,24 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % NRAW, u = c / NRAW;
         // After an abort every wait returns at once and the loops run to the end
-        // without blocking, so all roles reach the final barrier.  The raw slot
+        // without blocking, so all roles reach the final barrier.  A raw slot
         // is free once the converters have split the chunk it held.
         if (u > 0) mbar_wait(bar_raw_free + 8 * s, (u - 1) & 1, &ctl, status, 101);
-        const unsigned dst = smem_u32(smem + OFF_RAW + s * TILE_BYTES);
-        mbar_arrive_tx(bar_full_a + 8 * s, TILE_BYTES);
+        const unsigned dst = smem_u32(smem + OFF_RAW + s * W_TILE);
+        mbar_arrive_tx(bar_full_w + 8 * s, W_BYTES);
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
             "l"(reinterpret_cast<uint64_t>(&tmap_w)), "r"(c * BK), "r"(o0),
-            "r"(bar_full_a + 8 * s)
+            "r"(bar_full_w + 8 * s)
             : "memory");
       }
-      // drain: the last loads of each stage must land before the CTA can exit
+      // drain: the last loads must land before the CTA can exit
       for (int c = n_chunks - NRAW; c < n_chunks; ++c)
-        if (c >= 0) mbar_drain(bar_full_a + 8 * (c % NRAW), (c / NRAW) & 1);
+        if (c >= 0) mbar_drain(bar_full_w + 8 * (c % NRAW), (c / NRAW) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
-    // Runs of RUN chunks accumulate into alternating TMEM accumulators, each
-    // run starting from zero; the converter warps add finished runs in FP32
-    // registers.  Short runs keep the tensor core's truncating accumulation
-    // from growing with Cin K.
     if (lane == 0) {
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % NSTAGE, u = c / NSTAGE;
@@ -275,18 +275,18 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
           mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 106);
         mbar_wait(bar_ready + 8 * s, u & 1, &ctl, status, 102);
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        const unsigned acc = tmem + (unsigned)(ra * BN);
-        const unsigned a_hi = smem_u32(smem + OFF_A + s * TILE_BYTES);
-        const unsigned a_lo = smem_u32(smem + OFF_ALO + s * TILE_BYTES);
-        const unsigned b_hi = smem_u32(smem + OFF_BHI + s * TILE_BYTES);
-        const unsigned b_lo = smem_u32(smem + OFF_BLO + s * TILE_BYTES);
+        const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
+        const unsigned x_hi = smem_u32(smem + OFF_XHI + s * X_TILE);
+        const unsigned x_lo = smem_u32(smem + OFF_XLO + s * X_TILE);
+        const unsigned w_hi = smem_u32(smem + OFF_WHI + s * W_TILE);
+        const unsigned w_lo = smem_u32(smem + OFF_WLO + s * W_TILE);
 #pragma unroll
         for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes per MMA
           const unsigned off = 32 * k;
-          mma_tf32(acc, sw128_desc(a_lo + off), sw128_desc(b_hi + off),
+          mma_tf32(acc, sw128_desc(x_lo + off), sw128_desc(w_hi + off), IDESC,
                    (first && k == 0) ? 0u : 1u);
-          mma_tf32(acc, sw128_desc(a_hi + off), sw128_desc(b_lo + off), 1u);
-          mma_tf32(acc, sw128_desc(a_hi + off), sw128_desc(b_hi + off), 1u);
+          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_lo + off), IDESC, 1u);
+          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_hi + off), IDESC, 1u);
         }
         mma_commit(bar_empty + 8 * s);  // stage s may be refilled once these finish
         if (last) mma_commit(bar_run_full + 8 * ra);
@@ -294,19 +294,19 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     }
   } else if (warp >= CONV_WARP0) {
     // ------------------------------------------------------ converters + sums
-    const int ct = threadIdx.x - CONV_WARP0 * 32;  // row of B this thread builds
-    const int q = warp - CONV_WARP0;                // TMEM lane quarter
+    const int ct = threadIdx.x - CONV_WARP0 * 32;  // time row of X this thread builds
+    const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
     const float *xb = x + (size_t)b * Cin * T;
-    float sum[BN];  // this thread's output row (o = o0 + 32 q + lane), FP32 run sums
+    float sum[NT];  // time sample t0 + ct, channels o0 .. o0 + NT - 1: FP32 run sums
 #pragma unroll
-    for (int e = 0; e < BN; ++e) sum[e] = 0.0f;
+    for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
 
     // stage x block blk (channels [CB blk, CB blk + CB)) into xs[blk & 1];
     // channels >= Cin and times outside [0, T) read as zero
     auto stage_x = [&](int blk) {
       float *dst = xs + (blk & 1) * CB * XW;
       const int i0 = blk * CB;
-      const int width = BN + halo;
+      const int width = BM + halo;
       for (int idx = ct; idx < CB * width; idx += NCONV) {
         const int ci = idx / width, n = idx - ci * width;
         const int i = i0 + ci, t = xt0 + n;
@@ -316,30 +316,26 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
       }
       cp_async_commit();
     };
-    // add finished run p into the row sums and hand its accumulator back
+    // add finished run p into the sums and hand its accumulator back
     auto promote = [&](int p) {
       const int ra = p & 1;
       warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 105);
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 #pragma unroll
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t v[32];
-        const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * BN + c0);
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        uint32_t v[16];
+        const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * MAX_NT + c0);
         asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-            "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, "
-            "[%32];\n"
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15}, [%16];\n"
             : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
               "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-              "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]),
-              "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
-              "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
-              "=r"(v[30]), "=r"(v[31])
+              "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
             : "r"(taddr)
             : "memory");
         asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+        for (int e = 0; e < 16; ++e) sum[c0 + e] += __uint_as_float(v[e]);
       }
       asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
       __syncwarp();
@@ -351,6 +347,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     int promoted = 0;  // runs added so far
     for (int c = 0; c < n_chunks; ++c) {
       const int s = c % NSTAGE, u = c / NSTAGE;
+      const int sr = c % NRAW;
       const int kk0 = c * BK;
       // x blocks hold CB channels = CB K kk, a multiple of BK: a chunk never
       // straddles two blocks
@@ -362,31 +359,36 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
         ready_blk = blk;
         if ((blk + 1) * CB < Cin) stage_x(blk + 1);
       }
-      const int sr = c % NRAW;
       if (u > 0) warp_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 103);
-      warp_wait(bar_full_a + 8 * sr, (c / NRAW) & 1, &ctl, status, 104);
-      // A: split into hi and lo (elementwise over the swizzled tile)
-      const unsigned char *a_raw = smem + OFF_RAW + sr * TILE_BYTES;
-      unsigned char *a_hi = smem + OFF_A + s * TILE_BYTES;
-      unsigned char *a_lo = smem + OFF_ALO + s * TILE_BYTES;
-      float4 av[TILE_BYTES / 16 / NCONV];
+      warp_wait(bar_full_w + 8 * sr, (c / NRAW) & 1, &ctl, status, 104);
+      // W: split into hi and lo (elementwise over the swizzled tile)
+      const unsigned char *w_raw = smem + OFF_RAW + sr * W_TILE;
+      unsigned char *w_hi = smem + OFF_WHI + s * W_TILE;
+      unsigned char *w_lo = smem + OFF_WLO + s * W_TILE;
+      constexpr int WCH = W_BYTES / 16;  // 16-byte chunks of the weight tile
+      constexpr int WPT = (WCH + NCONV - 1) / NCONV;
+      float4 wv[WPT];
 #pragma unroll
-      for (int rr = 0; rr < TILE_BYTES / 16 / NCONV; ++rr)
-        av[rr] = *reinterpret_cast<const float4 *>(a_raw + (ct + rr * NCONV) * 16);
+      for (int rr = 0; rr < WPT; ++rr)
+        if (ct + rr * NCONV < WCH)
+          wv[rr] = *reinterpret_cast<const float4 *>(w_raw + (ct + rr * NCONV) * 16);
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_raw_free + 8 * sr);  // the TMA may refill the slot
 #pragma unroll
-      for (int rr = 0; rr < TILE_BYTES / 16 / NCONV; ++rr) {
-        const int qo = (ct + rr * NCONV) * 16;
-        const float4 v = av[rr];
-        const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
-        *reinterpret_cast<float4 *>(a_hi + qo) = h;
-        *reinterpret_cast<float4 *>(a_lo + qo) =
-            make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+      for (int rr = 0; rr < WPT; ++rr) {
+        if (ct + rr * NCONV < WCH) {
+          const int qo = (ct + rr * NCONV) * 16;
+          const float4 v = wv[rr];
+          const float4 h =
+              make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+          *reinterpret_cast<float4 *>(w_hi + qo) = h;
+          *reinterpret_cast<float4 *>(w_lo + qo) =
+              make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+        }
       }
-      // B: row t = ct of the im2col chunk, block-local kk = 32 m .. 32 m + 31
-      unsigned char *b_hi = smem + OFF_BHI + s * TILE_BYTES;
-      unsigned char *b_lo = smem + OFF_BLO + s * TILE_BYTES;
+      // X: time row ct of the im2col chunk, block-local kk = 32 m .. 32 m + 31
+      unsigned char *x_hi = smem + OFF_XHI + s * X_TILE;
+      unsigned char *x_lo = smem + OFF_XLO + s * X_TILE;
       const float *xrow = xs + (blk & 1) * CB * XW + ct;
       const int *offs = xoff + m * BK;
       float xv[BK];
@@ -407,8 +409,8 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
           lv[e] = xv[4 * qq + e] - hv[e];
         }
         const int off = sw128_off(ct, 4 * qq);
-        *reinterpret_cast<float4 *>(b_hi + off) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-        *reinterpret_cast<float4 *>(b_lo + off) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+        *reinterpret_cast<float4 *>(x_hi + off) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+        *reinterpret_cast<float4 *>(x_lo + off) = make_float4(lv[0], lv[1], lv[2], lv[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
       __syncwarp();
@@ -420,22 +422,17 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     while (promoted < n_runs) promote(promoted++);
 
     // ------------------------------------------------------------- epilogue
-    float *ds = reinterpret_cast<float *>(smem);  // [BM][DS_PITCH]; operands are dead now
-    const int row = 32 * q + lane;
+    // one thread per time sample: for each channel, the warp's 32 lanes touch
+    // 32 consecutive samples of that channel's row
+    const int t = t0 + ct;
+    if (!ctl.abort && t < y_len) {
 #pragma unroll
-    for (int e = 0; e < BN; ++e) ds[row * DS_PITCH + e] = sum[e];
-    conv_bar_sync();
-    if (!ctl.abort) {
-      // row-contiguous write-out: each warp takes rows, lanes take columns
-      for (int r = q; r < BM; r += 4) {
-        const int o = o0 + r;
-        if (o >= Cout) break;
-        const float bo = bias ? __ldg(bias + o) : 0.0f;
-        const size_t rowoff = ((size_t)b * Cout + o) * y_pitch;
-        for (int cc = lane; cc < BN; cc += 32) {
-          const int t = t0 + cc;
-          if (t < y_len)
-            y[rowoff + t] = apply_epilogue(ds[r * DS_PITCH + cc], bo, ep, y, rowoff + t);
+      for (int e = 0; e < NT; ++e) {
+        const int o = o0 + e;
+        if (o < Cout) {
+          const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
+          const float bo = bias ? __ldg(bias + o) : 0.0f;
+          y[idx] = apply_epilogue(sum[e], bo, ep, y, idx);
         }
       }
     }
@@ -481,12 +478,42 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Channels per CTA: split Cout into the fewest tiles of at most 128 and round
+// each to a multiple of 16 (the UMMA N granularity for M = 128).
+int pick_nt(int Cout) {
+  const int tiles = (Cout + MAX_NT - 1) / MAX_NT;
+  const int per = (Cout + tiles - 1) / tiles;
+  return (per + 15) / 16 * 16;
+}
+
+template <int NT>
+bv_status run_tc(const CUtensorMap &tmap, const float *x, int B, int Cin, int T,
+                 const float *bias, int Cout, int K, int dil, int pad, const Epi &ep, float *y,
+                 int y_len, int y_pitch, cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(conv1d_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return check_launch("conv1d_tc smem attribute");
+    configured = true;
+  }
+  dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
+  conv1d_tc_kernel<NT><<<grid, THREADS, SMEM_BYTES, st>>>(
+      tmap, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, device_status_ptr());
+  return BV_OK;
+}
+
 }  // namespace
 
+// The tensor-core path pays a fixed cost per CTA (barriers, TMEM, pipeline
+// fill) that narrow layers cannot amortise: measured on B200, the FP32 SIMT
+// kernel is as fast or faster below about 40 output channels or 192 reduction
+// terms (e.g. 12- and 24-channel stages, 48 channels with k = 3, and the
+// 1-channel conv_post), and the tensor cores win from 48 channels with k >= 7.
 bool conv1d_tc_supported(int Cin, int Cout, int K, int dil) {
-  return Cout >= 64 && K <= MAX_K && (Cin * K) % 4 == 0 && (K - 1) * dil <= MAX_HALO &&
-         Cin * K >= BK &&
-         encode_fn() != nullptr;
+  return Cout >= 40 && Cin * K >= 192 && K <= MAX_K && (Cin * K) % 4 == 0 &&
+         (K - 1) * dil <= MAX_HALO && encode_fn() != nullptr;
 }
 
 bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
@@ -496,33 +523,41 @@ bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w
   if (!enc) return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: no cuTensorMapEncodeTiled");
   if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: weights not 16-byte aligned");
+  const int nt = pick_nt(Cout);
   CUtensorMap tmap;
   const cuuint64_t dims[2] = {(cuuint64_t)Cin * K, (cuuint64_t)Cout};
   const cuuint64_t strides[1] = {(cuuint64_t)Cin * K * sizeof(float)};
-  const cuuint32_t box[2] = {BK, BM};
+  const cuuint32_t box[2] = {BK, (cuuint32_t)nt};
   const cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return fail(BV_ERR_CUDA, "conv1d_tc: tensor map encode failed (%d)", (int)r);
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(conv1d_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return check_launch("conv1d_tc smem attribute");
-    configured = true;
-  }
-  int *status = device_status_ptr();
-  dim3 grid((y_len + BN - 1) / BN, (Cout + BM - 1) / BM, B);
-  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
+  if (r != CUDA_SUCCESS)
+    return fail(BV_ERR_CUDA, "conv1d_tc: tensor map encode failed (%d)", (int)r);
+  bv_status s;
   {
     const double outs = (double)B * Cout * y_len;
     LaunchTimer tm(st, "conv1d_tc", 2.0 * outs * Cin * K,
                    4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                           outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
-    conv1d_tc_kernel<<<grid, THREADS, SMEM_BYTES, st>>>(tmap, x, bias, y, Cin, T, Cout, K, dil,
-                                                        pad, y_len, y_pitch, ep, status);
+#define BV_TC_CASE(N)                                                                        \
+  case N:                                                                                    \
+    s = run_tc<N>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
+    break;
+    switch (nt) {
+      BV_TC_CASE(16)
+      BV_TC_CASE(32)
+      BV_TC_CASE(48)
+      BV_TC_CASE(64)
+      BV_TC_CASE(80)
+      BV_TC_CASE(96)
+      BV_TC_CASE(112)
+      default:
+        s = run_tc<128>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
+    }
+#undef BV_TC_CASE
   }
+  if (s != BV_OK) return s;
   count_launch();
   return check_launch("conv1d_tc_kernel");
 }

@@ -231,9 +231,10 @@ def test_conv_transpose1d_general_kernel(nat, oracle):
 # of 32), partial input-channel blocks, short and ragged time axes, the
 # largest halo, and every epilogue.
 TC_CASES = [(64, 64, 3, 1, 200), (128, 128, 3, 1, 1), (128, 128, 7, 3, 5), (96, 96, 11, 5, 130),
-            (192, 192, 11, 5, 257), (12, 128, 3, 1, 129), (40, 200, 7, 1, 300),
+            (192, 192, 11, 5, 257), (64, 128, 3, 1, 129), (40, 200, 7, 1, 300),
             (384, 384, 11, 5, 127), (768, 768, 3, 1, 400), (32, 1536, 7, 1, 77),
-            (256, 256, 7, 3, 1024), (100, 300, 11, 1, 513)]
+            (256, 256, 7, 3, 1024), (100, 300, 11, 1, 513), (48, 48, 7, 3, 700),
+            (48, 48, 11, 5, 77), (64, 40, 3, 1, 300), (96, 112, 7, 1, 130), (80, 80, 3, 1, 9)]
 
 
 def _kernel_classes(nat, fn):
