@@ -30,7 +30,11 @@ constexpr int TILE = 2048;         // outputs per tile
 constexpr int HALF = TILE / 2;     // the two positions of a thread are HALF apart
 constexpr int THREADS = 256;       // per half tile: 4 outputs and 8 up-sampled values each
 constexpr int XS = TILE + 16;      // x[t0 - 8 + i]
-constexpr int VS = 2 * TILE + 16;  // v[2 t0 - 6 + k], k < 2 TILE + 12 used
+// v[2 t0 - 6 + k], k < 2 TILE + 12, stored at vidx(k): 4 floats of padding
+// after every 32 spread the 32-byte-strided float4 accesses of a warp over all
+// banks
+__device__ __forceinline__ int vidx(int k) { return k + 4 * (k >> 5); }
+constexpr int VS = (2 * TILE + 16) + 4 * ((2 * TILE + 16) / 32 + 1);
 static_assert(HALF == 4 * THREADS, "one thread per 4 outputs of a half tile");
 
 __device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
@@ -126,7 +130,7 @@ __device__ __forceinline__ void store4(float *yr, int t, int T, float o0, float 
   }
 }
 
-__global__ void __launch_bounds__(THREADS)
+__global__ void __launch_bounds__(THREADS, 2)
 activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int T,
                   int tiles_per_row, int n_tiles, const float *__restrict__ log_alpha,
                   const float *__restrict__ log_beta, const float *__restrict__ f_up,
@@ -199,16 +203,19 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
           V[2 * qq + r] = snake2(u, a, inv_b);
         }
       }
-      *reinterpret_cast<float4 *>(vs + 2 * q0) = make_float4(V[0].x, V[1].x, V[2].x, V[3].x);
-      *reinterpret_cast<float4 *>(vs + 2 * q0 + 4) = make_float4(V[4].x, V[5].x, V[6].x, V[7].x);
-      *reinterpret_cast<float4 *>(vs + 2 * HALF + 2 * q0) =
+      *reinterpret_cast<float4 *>(vs + vidx(2 * q0)) = make_float4(V[0].x, V[1].x, V[2].x, V[3].x);
+      *reinterpret_cast<float4 *>(vs + vidx(2 * q0 + 4)) =
+          make_float4(V[4].x, V[5].x, V[6].x, V[7].x);
+      *reinterpret_cast<float4 *>(vs + vidx(2 * HALF + 2 * q0)) =
           make_float4(V[0].y, V[1].y, V[2].y, V[3].y);
-      *reinterpret_cast<float4 *>(vs + 2 * HALF + 2 * q0 + 4) =
+      *reinterpret_cast<float4 *>(vs + vidx(2 * HALF + 2 * q0 + 4)) =
           make_float4(V[4].y, V[5].y, V[6].y, V[7].y);
-      if (tid < 12) {  // k in [2 TILE, 2 TILE + 12)
-        const int k = 2 * TILE + tid;
+      // k in [2 TILE, 2 TILE + 12): one or two per warp, lane 0 and lane 1
+      if ((tid & 31) < 2 && (tid >> 5) + 8 * (tid & 31) < 12) {
+        const int i = (tid >> 5) + 8 * (tid & 31);
+        const int k = 2 * TILE + i;
         const int q = k >> 1, r = k & 1;
-        vs[k] = snake1(up1(tp, r, xb + 2 + q + r), a, inv_b);
+        vs[vidx(k)] = snake1(up1(tp, r, xb + 2 + q + r), a, inv_b);
       }
     }
     // Near a row end the pages pad the 2x signal by replication: v at an index
@@ -225,7 +232,7 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
           const int p = mc >> 1, r = mc & 1;
           // x[p + r - 3 + k'] sits at xb[p + r + 5 - t0 + k'] (in range: the tile
           // reaches that row end)
-          vs[k] = snake1(up1(tp, r, xb + (p + r + 5 - t0)), a, inv_b);
+          vs[vidx(k)] = snake1(up1(tp, r, xb + (p + r + 5 - t0)), a, inv_b);
         }
       }
     }
@@ -237,8 +244,8 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
       float2 W[20];
 #pragma unroll
       for (int w = 0; w < 5; ++w) {
-        const float4 lo = *reinterpret_cast<const float4 *>(vs + 2 * tl + 4 * w);
-        const float4 hi = *reinterpret_cast<const float4 *>(vs + 2 * HALF + 2 * tl + 4 * w);
+        const float4 lo = *reinterpret_cast<const float4 *>(vs + vidx(2 * tl + 4 * w));
+        const float4 hi = *reinterpret_cast<const float4 *>(vs + vidx(2 * HALF + 2 * tl + 4 * w));
         W[4 * w] = make_float2(lo.x, hi.x);
         W[4 * w + 1] = make_float2(lo.y, hi.y);
         W[4 * w + 2] = make_float2(lo.z, hi.z);

@@ -439,8 +439,24 @@ long long max_elems(const bv_decoder_config *c, long long B, long long F) {
   return m;
 }
 
+// Repacked ConvT weights for the tensor-core path (one buffer, reused by
+// every stage that takes that path).
+size_t convt_ws(const bv_decoder_config *c) {
+  size_t m = 0;
+  int C = c->pre_channels;
+  for (int i = 0; i < c->n_up; ++i) {
+    if (conv_transpose1d_tc_supported(C, c->up_channels[i], c->up_kernel[i], c->up_rate[i])) {
+      const size_t b = conv_transpose1d_tc_workspace(C, c->up_channels[i], c->up_kernel[i],
+                                                     c->up_rate[i]);
+      if (b > m) m = b;
+    }
+    C = c->up_channels[i];
+  }
+  return align_up(m);
+}
+
 size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
-  return 5 * align_up((size_t)max_elems(c, B, F) * sizeof(float));
+  return 5 * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
 }
 
 struct TilePlan {
@@ -517,6 +533,7 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, c
   float *S = reinterpret_cast<float *>(ws + sz);
   AmpScratch s{reinterpret_cast<float *>(ws + 2 * sz), reinterpret_cast<float *>(ws + 3 * sz),
                reinterpret_cast<float *>(ws + 4 * sz)};
+  float *WP = reinterpret_cast<float *>(ws + 5 * sz);  // repacked ConvT weights
   int C = c->pre_channels, n = F;
   Epi plain{nullptr, 1.0f, 0, 0};
   BV_TRY(launch_conv1d(z, B, c->in_channels, F, w->pre_w, w->pre_b, C, c->pre_kernel, 1,
@@ -525,7 +542,11 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, c
     const int sr = c->up_rate[i], k = c->up_kernel[i], Co = c->up_channels[i];
     const int pad = (k - sr) / 2;
     const int n2 = (n - 1) * sr + k - 2 * pad;
-    BV_TRY(launch_conv_transpose1d(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S, st));
+    if (conv_transpose1d_tc_supported(C, Co, k, sr))
+      BV_TRY(launch_conv_transpose1d_tc(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S,
+                                        WP, st));
+    else
+      BV_TRY(launch_conv_transpose1d(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S, st));
     C = Co;
     n = n2;
     const float scale = 1.0f / (float)c->n_blocks;

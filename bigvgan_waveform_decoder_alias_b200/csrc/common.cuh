@@ -90,6 +90,15 @@ bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w
                            const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
                            float *y, int y_len, int y_pitch, cudaStream_t st);
 
+// ConvTranspose1d on the tensor cores: each output phase is an ordinary conv
+// over the input samples with repacked weights (wp: workspace of
+// conv_transpose1d_tc_workspace bytes, rewritten by every call).
+bool conv_transpose1d_tc_supported(int Cin, int Cout, int K, int S);
+size_t conv_transpose1d_tc_workspace(int Cin, int Cout, int K, int S);
+bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                                     const float *bias, int Cout, int K, int S, int pad, float *y,
+                                     float *wp, cudaStream_t st);
+
 // ConvTranspose1d.
 bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,
                                   const float *bias, int Cout, int K, int stride, int pad,

@@ -177,11 +177,18 @@ __device__ __forceinline__ float tf32_hi(float v) {
   return __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
 }
 
+// Where conv output t goes: sample stride * t + offset of a row of len
+// samples; phases > 1 runs that many weight sets (blockIdx.z = b phases + r),
+// phase r reading weight rows r Cout .. and writing offset + r.
+struct OutMap {
+  int stride, offset, len, phases;
+};
+
 template <int NT>
 __global__ void __launch_bounds__(THREADS, 1)
 conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ x,
                  const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
-                 int dil, int pad, int y_len, int y_pitch, Epi ep, int *status) {
+                 int dil, int pad, int y_len, int y_pitch, Epi ep, OutMap om, int *status) {
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
   constexpr int W_BYTES = NT * BK * 4;  // bytes of one weight chunk (TMA box)
   constexpr uint32_t IDESC = make_idesc(NT);
@@ -205,7 +212,9 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * BM;
   const int o0 = blockIdx.y * NT;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z / om.phases;
+  const int phase = blockIdx.z - b * om.phases;
+  const int w_row0 = phase * Cout + o0;  // this phase's weight rows in the tensor map
   const int KK = Cin * K;
   const int n_chunks = (KK + BK - 1) / BK;
   const int n_runs = (n_chunks + RUN - 1) / RUN;
@@ -255,7 +264,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
-            "l"(reinterpret_cast<uint64_t>(&tmap_w)), "r"(c * BK), "r"(o0),
+            "l"(reinterpret_cast<uint64_t>(&tmap_w)), "r"(c * BK), "r"(w_row0),
             "r"(bar_full_w + 8 * s)
             : "memory");
       }
@@ -423,14 +432,16 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
 
     // ------------------------------------------------------------- epilogue
     // one thread per time sample: for each channel, the warp's 32 lanes touch
-    // 32 consecutive samples of that channel's row
+    // 32 consecutive samples of that channel's row (every stride-th sample for
+    // a transposed-conv phase)
     const int t = t0 + ct;
-    if (!ctl.abort && t < y_len) {
+    const int p = om.stride * t + om.offset + phase;
+    if (!ctl.abort && t < y_len && p >= 0 && p < om.len) {
 #pragma unroll
       for (int e = 0; e < NT; ++e) {
         const int o = o0 + e;
         if (o < Cout) {
-          const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
+          const size_t idx = ((size_t)b * Cout + o) * y_pitch + p;
           const float bo = bias ? __ldg(bias + o) : 0.0f;
           y[idx] = apply_epilogue(sum[e], bo, ep, y, idx);
         }
@@ -489,7 +500,7 @@ int pick_nt(int Cout) {
 template <int NT>
 bv_status run_tc(const CUtensorMap &tmap, const float *x, int B, int Cin, int T,
                  const float *bias, int Cout, int K, int dil, int pad, const Epi &ep, float *y,
-                 int y_len, int y_pitch, cudaStream_t st) {
+                 int y_len, int y_pitch, const OutMap &om, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(conv1d_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -497,10 +508,10 @@ bv_status run_tc(const CUtensorMap &tmap, const float *x, int B, int Cin, int T,
       return check_launch("conv1d_tc smem attribute");
     configured = true;
   }
-  dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B);
+  dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B * om.phases);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
   conv1d_tc_kernel<NT><<<grid, THREADS, SMEM_BYTES, st>>>(
-      tmap, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, device_status_ptr());
+      tmap, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, om, device_status_ptr());
   return BV_OK;
 }
 
@@ -516,16 +527,21 @@ bool conv1d_tc_supported(int Cin, int Cout, int K, int dil) {
          (K - 1) * dil <= MAX_HALO && encode_fn() != nullptr;
 }
 
-bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
-                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
-                           float *y, int y_len, int y_pitch, cudaStream_t st) {
+namespace {
+
+// Encode the weight tensor map ([rows, Cin K] fp32, box 32 x nt, 128-byte
+// swizzle) and launch the NT instance.
+bv_status launch_tc_impl(const char *cls, const float *x, int B, int Cin, int T, const float *w,
+                         int w_rows, const float *bias, int Cout, int K, int dil, int pad,
+                         const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
+                         double flops, double bytes, cudaStream_t st) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: no cuTensorMapEncodeTiled");
   if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: weights not 16-byte aligned");
   const int nt = pick_nt(Cout);
   CUtensorMap tmap;
-  const cuuint64_t dims[2] = {(cuuint64_t)Cin * K, (cuuint64_t)Cout};
+  const cuuint64_t dims[2] = {(cuuint64_t)Cin * K, (cuuint64_t)w_rows};
   const cuuint64_t strides[1] = {(cuuint64_t)Cin * K * sizeof(float)};
   const cuuint32_t box[2] = {BK, (cuuint32_t)nt};
   const cuuint32_t estr[2] = {1, 1};
@@ -536,13 +552,11 @@ bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w
     return fail(BV_ERR_CUDA, "conv1d_tc: tensor map encode failed (%d)", (int)r);
   bv_status s;
   {
-    const double outs = (double)B * Cout * y_len;
-    LaunchTimer tm(st, "conv1d_tc", 2.0 * outs * Cin * K,
-                   4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
-                          outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
-#define BV_TC_CASE(N)                                                                        \
-  case N:                                                                                    \
-    s = run_tc<N>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
+    LaunchTimer tm(st, cls, flops, bytes);
+#define BV_TC_CASE(N)                                                                      \
+  case N:                                                                                  \
+    s = run_tc<N>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, om, \
+                  st);                                                                     \
     break;
     switch (nt) {
       BV_TC_CASE(16)
@@ -553,13 +567,84 @@ bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w
       BV_TC_CASE(96)
       BV_TC_CASE(112)
       default:
-        s = run_tc<128>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
+        s = run_tc<128>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, om,
+                        st);
     }
 #undef BV_TC_CASE
   }
   if (s != BV_OK) return s;
   count_launch();
   return check_launch("conv1d_tc_kernel");
+}
+
+// wp[r][o][i nt + j] = w[i][o][r + s (nt - 1 - j)] (zero past K): phase r of
+// the transposed conv as an ordinary nt-tap conv over the input samples.
+__global__ void convt_repack_kernel(const float *__restrict__ w, float *__restrict__ wp, int Cin,
+                                    int Cout, int K, int S, int nt) {
+  const long long total = (long long)S * Cout * Cin * nt;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int j = (int)(idx % nt);
+    long long rest = idx / nt;
+    const int i = (int)(rest % Cin);
+    rest /= Cin;
+    const int o = (int)(rest % Cout);
+    const int r = (int)(rest / Cout);
+    const int k = r + S * (nt - 1 - j);
+    wp[idx] = k < K ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
+  }
+}
+
+}  // namespace
+
+bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
+                           float *y, int y_len, int y_pitch, cudaStream_t st) {
+  const double outs = (double)B * Cout * y_len;
+  const OutMap om{1, 0, y_len, 1};
+  return launch_tc_impl("conv1d_tc", x, B, Cin, T, w, Cout, bias, Cout, K, dil, pad, ep, y,
+                        y_len, y_pitch, om, 2.0 * outs * Cin * K,
+                        4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
+                               outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)),
+                        st);
+}
+
+int convt_taps(int K, int S) { return (K + S - 1) / S; }
+
+bool conv_transpose1d_tc_supported(int Cin, int Cout, int K, int S) {
+  const int nt = convt_taps(K, S);
+  return conv1d_tc_supported(Cin, Cout, nt, 1);
+}
+
+size_t conv_transpose1d_tc_workspace(int Cin, int Cout, int K, int S) {
+  return (size_t)S * Cout * Cin * convt_taps(K, S) * sizeof(float);
+}
+
+bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                                     const float *bias, int Cout, int K, int S, int pad, float *y,
+                                     float *wp, cudaStream_t st) {
+  const int nt = convt_taps(K, S);
+  const int Tout = (T - 1) * S + K - 2 * pad;
+  const long long total = (long long)S * Cout * Cin * nt;
+  {
+    LaunchTimer tm(st, "convt_repack", 0.0, 8.0 * (double)total);
+    const long long blocks = (total + 255) / 256;
+    convt_repack_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
+        w, wp, Cin, Cout, K, S, nt);
+  }
+  count_launch();
+  bv_status s = check_launch("convt_repack_kernel");
+  if (s != BV_OK) return s;
+  // phase r: conv output P (input-grid index, P < T + nt - 1) lands on sample
+  // S P + r - pad of the output row
+  const OutMap om{S, -pad, Tout, S};
+  const Epi plain{nullptr, 1.0f, 0, 0};
+  return launch_tc_impl("conv_transpose1d_tc", x, B, Cin, T, wp, S * Cout, bias, Cout, nt, 1,
+                        nt - 1, plain, y, T + nt - 1, Tout, om,
+                        2.0 * B * Cin * (double)Cout * K * T,
+                        4.0 * ((double)B * Cin * T + (double)Cin * Cout * K +
+                               (double)B * Cout * Tout),
+                        st);
 }
 
 }  // namespace bv

@@ -421,6 +421,23 @@ def test_real_geometry_short_latent(nat, oracle, filt, wname, frames):
     assert rel_l2(y, want) < WAVE_TOL
 
 
+@pytest.mark.parametrize("frames", [1, 2, 5, 27])
+def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
+    """A decoder wide enough that its ConvT stages (both stride parities) and
+    its AMP convs take the tensor-core path, on short and ragged latents."""
+    geo = synth.tiny_geometry(pre_channels=256, up_channels=(128, 96, 48), in_channels=16)
+    s = synth.NormalStream(40 + frames)
+    z = s.normal((2, geo.in_channels, frames))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.02)  # the workloads' weight scale
+    dec = _decoder(nat, geo, params, filt)
+    zd = dev(z)
+    out = {}
+    classes = _kernel_classes(nat, lambda: out.setdefault("y", dec.decode(zd)))
+    assert "conv_transpose1d_tc" in classes and "conv1d_tc" in classes, classes
+    want = oracle.decode(geo, params, z)
+    assert rel_l2(host(out["y"]), want) < WAVE_TOL
+
+
 def test_decoder_batch_independence_and_determinism(nat, filt):
     geo = synth.tiny_geometry()
     s = synth.NormalStream(12)
