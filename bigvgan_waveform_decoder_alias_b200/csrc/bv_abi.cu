@@ -322,9 +322,16 @@ struct AmpScratch {
   float *cur, *h1, *h2;
 };
 
+// Pre-split tensor-core weights of one AMP block's convs (nullptr: the conv
+// splits its own weights).
+struct AmpSplit {
+  const float *conv1[BV_MAX_DIL], *conv2[BV_MAX_DIL];
+};
+
 // y = (accumulate ? y : 0) + scale * AMP(x); x, y and the scratch are disjoint.
 bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params &p, float *y,
-                        float scale, int accumulate, const AmpScratch &s, cudaStream_t st) {
+                        float scale, int accumulate, const AmpScratch &s, cudaStream_t st,
+                        const AmpSplit *sp = nullptr) {
   const int K = p.kernel_size, n = p.n_dilations;
   const float eps = 1e-9f;
   for (int u = 0; u < n; ++u) {
@@ -334,17 +341,17 @@ bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params
                              p.up_filter, p.down_filter, eps, st));
     Epi plain{nullptr, 1.0f, 0, 0};
     BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv1_w[u], p.conv1_b[u], C, K, d, (K * d - d) / 2,
-                         plain, s.h2, T, T, st));
+                         plain, s.h2, T, T, st, sp ? sp->conv1[u] : nullptr));
     BV_TRY(launch_activation(s.h2, s.h1, B, C, T, p.act_log_alpha[2 * u + 1],
                              p.act_log_beta[2 * u + 1], p.up_filter, p.down_filter, eps, st));
     if (u == n - 1) {
       Epi last{src, scale, accumulate, 0};
       BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, last,
-                           y, T, T, st));
+                           y, T, T, st, sp ? sp->conv2[u] : nullptr));
     } else {
       Epi res{src, 1.0f, 0, 0};  // cur = src + conv2(...); src may be cur itself
       BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, res,
-                           s.cur, T, T, st));
+                           s.cur, T, T, st, sp ? sp->conv2[u] : nullptr));
     }
   }
   return BV_OK;
@@ -455,6 +462,75 @@ size_t convt_ws(const bv_decoder_config *c) {
   return align_up(m);
 }
 
+// Pre-split weights of every conv the tensor-core path takes: tf32(W) then
+// W - tf32(W), written once per decode call and read by every tile group.
+struct DecoderSplit {
+  const float *pre = nullptr, *post = nullptr;
+  AmpSplit amp[BV_MAX_UP][BV_MAX_BLOCKS] = {};
+};
+
+// Walk the decoder's convs in a fixed order; f(Cin, Cout, K, dil, src, slot)
+// is called for each conv the tensor-core path supports (src may be null when
+// only sizes are wanted).
+template <class F>
+void for_each_tc_conv(const bv_decoder_config *c, const bv_decoder_weights *w, F &&f) {
+  if (conv1d_tc_supported(c->in_channels, c->pre_channels, c->pre_kernel, 1))
+    f(c->in_channels, c->pre_channels, c->pre_kernel, w ? w->pre_w : nullptr, 0, -1, -1, -1);
+  for (int i = 0; i < c->n_up; ++i) {
+    const int C = c->up_channels[i];
+    for (int j = 0; j < c->n_blocks; ++j) {
+      const int K = c->block_kernel[j];
+      for (int u = 0; u < c->n_dilations; ++u) {
+        if (conv1d_tc_supported(C, C, K, c->dilation[u]))
+          f(C, C, K, w ? w->amp[i][j].conv1_w[u] : nullptr, 1, i, j, u);
+        if (conv1d_tc_supported(C, C, K, 1))
+          f(C, C, K, w ? w->amp[i][j].conv2_w[u] : nullptr, 2, i, j, u);
+      }
+    }
+  }
+  const int Cl = c->n_up > 0 ? c->up_channels[c->n_up - 1] : c->pre_channels;
+  if (conv1d_tc_supported(Cl, c->out_channels, c->post_kernel, 1))
+    f(Cl, c->out_channels, c->post_kernel, w ? w->post_w : nullptr, 3, -1, -1, -1);
+}
+
+size_t split_ws(const bv_decoder_config *c) {
+  size_t s = 0;
+  for_each_tc_conv(c, nullptr, [&](int Cin, int Cout, int K, const float *, int, int, int, int) {
+    s += align_up(2 * (size_t)Cin * Cout * K * sizeof(float));
+  });
+  return s;
+}
+
+// Fill `out` with slots in ws (size split_ws) and launch the split kernels.
+bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w, char *ws,
+                        DecoderSplit *out, cudaStream_t st) {
+  SplitTable tab;
+  tab.n = 0;
+  bv_status status = BV_OK;
+  size_t off = 0;
+  for_each_tc_conv(c, w, [&](int Cin, int Cout, int K, const float *src, int kind, int i, int j,
+                             int u) {
+    if (status != BV_OK) return;
+    const long long count = (long long)Cin * Cout * K;
+    float *dst = reinterpret_cast<float *>(ws + off);
+    off += align_up(2 * (size_t)count * sizeof(float));
+    if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return;  // SIMT path: no split needed
+    if (kind == 0) out->pre = dst;
+    else if (kind == 1) out->amp[i][j].conv1[u] = dst;
+    else if (kind == 2) out->amp[i][j].conv2[u] = dst;
+    else out->post = dst;
+    tab.src[tab.n] = src;
+    tab.dst[tab.n] = dst;
+    tab.count[tab.n] = count;
+    if (++tab.n == kMaxSplit) {
+      status = launch_split_weights(tab, st);
+      tab.n = 0;
+    }
+  });
+  if (status != BV_OK) return status;
+  return launch_split_weights(tab, st);
+}
+
 size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
   return 5 * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
 }
@@ -490,8 +566,8 @@ TilePlan plan_tiles(const bv_decoder_config *c, int F) {
 size_t decode_ws(const bv_decoder_config *c, int B, int F) {
   const TilePlan tp = plan_tiles(c, F);
   const long long hop = hop_of(c);
-  if (!tp.tiled) return core_ws(c, B, F);
-  size_t s = 0;
+  if (!tp.tiled) return split_ws(c) + core_ws(c, B, F);
+  size_t s = split_ws(c);
   const long long rows_full = (long long)B * tp.n_full;
   s += align_up((size_t)rows_full * c->in_channels * c->tile_frames * sizeof(float));
   s += align_up((size_t)rows_full * c->out_channels * c->tile_frames * hop * sizeof(float));
@@ -526,8 +602,9 @@ bv_status check_weights(const bv_decoder_config *c, const bv_decoder_weights *w)
 }
 
 // One untiled decode of B rows into y rows of length F*hop.
-bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
-                      int B, int F, float *y, char *ws, cudaStream_t st) {
+bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
+                      const DecoderSplit &sw, const float *z, int B, int F, float *y, char *ws,
+                      cudaStream_t st) {
   const size_t sz = align_up((size_t)max_elems(c, B, F) * sizeof(float));
   float *A = reinterpret_cast<float *>(ws);
   float *S = reinterpret_cast<float *>(ws + sz);
@@ -537,7 +614,7 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, c
   int C = c->pre_channels, n = F;
   Epi plain{nullptr, 1.0f, 0, 0};
   BV_TRY(launch_conv1d(z, B, c->in_channels, F, w->pre_w, w->pre_b, C, c->pre_kernel, 1,
-                       (c->pre_kernel - 1) / 2, plain, A, F, F, st));
+                       (c->pre_kernel - 1) / 2, plain, A, F, F, st, sw.pre));
   for (int i = 0; i < c->n_up; ++i) {
     const int sr = c->up_rate[i], k = c->up_kernel[i], Co = c->up_channels[i];
     const int pad = (k - sr) / 2;
@@ -551,20 +628,23 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w, c
     n = n2;
     const float scale = 1.0f / (float)c->n_blocks;
     for (int j = 0; j < c->n_blocks; ++j)
-      BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], A, scale, j > 0, s, st));
+      BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], A, scale, j > 0, s, st, &sw.amp[i][j]));
   }
   BV_TRY(launch_activation(A, s.h1, B, C, n, w->post_log_alpha, w->post_log_beta, w->up_filter,
                            w->down_filter, 1e-9f, st));
   const long long L = (long long)F * hop_of(c);
   Epi fin{nullptr, 1.0f, 0, c->final_act};
   return launch_conv1d(s.h1, B, C, n, w->post_w, w->post_b, c->out_channels, c->post_kernel, 1,
-                       (c->post_kernel - 1) / 2, fin, y, (int)L, (int)L, st);
+                       (c->post_kernel - 1) / 2, fin, y, (int)L, (int)L, st, sw.post);
 }
 
 bv_status decode_impl(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
                       int B, int F, float *y, char *ws, cudaStream_t st) {
   const TilePlan tp = plan_tiles(c, F);
-  if (!tp.tiled) return decode_core(c, w, z, B, F, y, ws, st);
+  DecoderSplit sw;
+  BV_TRY(split_weights(c, w, ws, &sw, st));
+  ws += split_ws(c);
+  if (!tp.tiled) return decode_core(c, w, sw, z, B, F, y, ws, st);
   const long long hop = hop_of(c);
   const int Ft = c->tile_frames;
   const long long rows_full = (long long)B * tp.n_full;
@@ -584,7 +664,7 @@ bv_status decode_impl(const bv_decoder_config *c, const bv_decoder_weights *w, c
   g.n = 0;
   if (tp.n_full > 0) {
     BV_TRY(launch_gather_tiles(z, zf, B, c->in_channels, F, tp.step, Ft, 0, tp.n_full, st));
-    BV_TRY(decode_core(c, w, zf, (int)rows_full, Ft, yf, p, st));
+    BV_TRY(decode_core(c, w, sw, zf, (int)rows_full, Ft, yf, p, st));
     g.data[g.n] = yf;
     g.k0[g.n] = 0;
     g.count[g.n] = tp.n_full;
@@ -593,7 +673,7 @@ bv_status decode_impl(const bv_decoder_config *c, const bv_decoder_weights *w, c
   }
   if (tp.last_len > 0) {
     BV_TRY(launch_gather_tiles(z, zl, B, c->in_channels, F, tp.step, tp.last_len, tp.n_full, 1, st));
-    BV_TRY(decode_core(c, w, zl, B, tp.last_len, yl, p, st));
+    BV_TRY(decode_core(c, w, sw, zl, B, tp.last_len, yl, p, st));
     g.data[g.n] = yl;
     g.k0[g.n] = tp.n_full;
     g.count[g.n] = 1;

@@ -81,14 +81,28 @@ bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream
 // row pitch y_pitch floats.
 bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
                         int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
-                        int y_pitch, cudaStream_t st);
+                        int y_pitch, cudaStream_t st, const float *w_split = nullptr);
 
 // Conv1d on the tensor cores (tcgen05, 3xTF32); supported() says whether the
 // shape qualifies (launch_conv1d picks it automatically).
+// w_split: tf32(W) followed by W - tf32(W), each in w's layout (written by
+// launch_split_weights), or nullptr, in which case the kernel splits w itself.
 bool conv1d_tc_supported(int Cin, int Cout, int K, int dil);
 bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
-                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
-                           float *y, int y_len, int y_pitch, cudaStream_t st);
+                           const float *w_split, const float *bias, int Cout, int K, int dil,
+                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                           cudaStream_t st);
+
+// tf32(W) and W - tf32(W) of a batch of weight tensors in one launch: entry e
+// writes dst[e][0, count) = tf32(src[e]) and dst[e][count, 2 count) = the rest.
+constexpr int kMaxSplit = 128;  // keeps the table under 4 KB of kernel parameters
+struct SplitTable {
+  int n;
+  const float *src[kMaxSplit];
+  float *dst[kMaxSplit];
+  long long count[kMaxSplit];
+};
+bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
 
 // ConvTranspose1d on the tensor cores: each output phase is an ordinary conv
 // over the input samples with repacked weights (wp: workspace of

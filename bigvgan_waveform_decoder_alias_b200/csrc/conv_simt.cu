@@ -154,10 +154,12 @@ bv_status run_conv(const float *x, int B, int Cin, int T, const float *w, const 
 
 bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, const float *bias,
                         int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
-                        int y_pitch, cudaStream_t st) {
+                        int y_pitch, cudaStream_t st, const float *w_split) {
   if (B <= 0 || y_len <= 0) return BV_OK;
-  if (conv1d_tc_supported(Cin, Cout, K, dil) && (reinterpret_cast<uintptr_t>(w) & 15u) == 0)
-    return launch_conv1d_tc(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
+  if (conv1d_tc_supported(Cin, Cout, K, dil) && (reinterpret_cast<uintptr_t>(w) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(w_split) & 15u) == 0)
+    return launch_conv1d_tc(x, B, Cin, T, w, w_split, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch,
+                            st);
   if (Cout >= 96)
     return run_conv<128, 128, 8, 8, 8>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len,
                                        y_pitch, st);

@@ -53,16 +53,26 @@ constexpr int TMEM_COLS = 256;           // two accumulators of up to 128 column
 constexpr int RUN = 4;                   // chunks accumulated in TMEM before an FP32 add
 constexpr int MAX_K = 32;                // largest kernel size (offset table rows)
 
-// shared memory layout (bytes from a 1024-aligned base)
+// shared memory layout (bytes from a 1024-aligned base): im2col operand
+// stages, then a weight region of six 16 KB tiles, then the staged x blocks.
+// The weight region holds W_hi[2], W_lo[2] and the raw TMA ring[2] when the
+// kernel splits the weights itself, or W_hi[3], W_lo[3] (a three-slot TMA
+// ring) when the split weights come from global memory.
+constexpr int NWSLOT = 3;                                // pre-split weight ring
 constexpr int OFF_XHI = 0;                               // per operand stage
 constexpr int OFF_XLO = OFF_XHI + NSTAGE * X_TILE;
-constexpr int OFF_WHI = OFF_XLO + NSTAGE * X_TILE;
-constexpr int OFF_WLO = OFF_WHI + NSTAGE * W_TILE;
-constexpr int OFF_RAW = OFF_WLO + NSTAGE * W_TILE;       // raw weight chunks from TMA
-constexpr int OFF_X = OFF_RAW + NRAW * W_TILE;           // x blocks [2][CB][XW]
+constexpr int OFF_W = OFF_XLO + NSTAGE * X_TILE;         // weight region
+constexpr int OFF_X = OFF_W + 6 * W_TILE;                // x blocks [2][CB][XW]
+static_assert(NSTAGE * 2 + NRAW == 6 && NWSLOT * 2 == 6, "weight region layout");
+template <bool PRESPLIT>
+struct WLayout {
+  __host__ __device__ static constexpr int hi(int s) { return OFF_W + s * W_TILE; }
+  __host__ __device__ static constexpr int lo(int s) { return OFF_W + (PRESPLIT ? NWSLOT : NSTAGE) * W_TILE + s * W_TILE; }
+  __host__ __device__ static constexpr int raw(int r) { return OFF_W + 2 * NSTAGE * W_TILE + r * W_TILE; }
+};
 constexpr int X_BYTES = 2 * CB * XW * 4;
 constexpr int OFF_BAR = OFF_X + X_BYTES;                 // mbarriers
-constexpr int SMEM_USED = OFF_BAR + 256;
+constexpr int SMEM_USED = OFF_BAR + 16 * 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;             // room to align the base
 static_assert(SMEM_BYTES + 4 * 1024 + 64 <= 227 * 1024, "shared memory budget");
 
@@ -184,9 +194,10 @@ struct OutMap {
   int stride, offset, len, phases;
 };
 
-template <int NT>
+template <int NT, bool PRESPLIT>
 __global__ void __launch_bounds__(THREADS, 1)
-conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__restrict__ x,
+conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
+                 const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ x,
                  const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
                  int dil, int pad, int y_len, int y_pitch, Epi ep, OutMap om, int *status) {
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
@@ -198,15 +209,17 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   __shared__ Ctl ctl;
   __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block
-  // barriers: raw weights landed (TMA) / raw weights read, per raw slot;
+  using WL = WLayout<PRESPLIT>;
+  constexpr int NWRING = PRESPLIT ? NWSLOT : NRAW;  // weight TMA ring slots
+  // barriers: weights landed (TMA) / weight slot free, per ring slot;
   // operands ready / operand stage free, per stage; run accumulated / run
   // accumulator read, per TMEM accumulator
   const unsigned bar_full_w = smem_u32(&bars[0]);
-  const unsigned bar_raw_free = smem_u32(&bars[2]);
-  const unsigned bar_ready = smem_u32(&bars[4]);
-  const unsigned bar_empty = smem_u32(&bars[6]);
-  const unsigned bar_run_full = smem_u32(&bars[8]);
-  const unsigned bar_run_free = smem_u32(&bars[10]);
+  const unsigned bar_raw_free = smem_u32(&bars[3]);
+  const unsigned bar_ready = smem_u32(&bars[6]);
+  const unsigned bar_empty = smem_u32(&bars[8]);
+  const unsigned bar_run_full = smem_u32(&bars[10]);
+  const unsigned bar_run_free = smem_u32(&bars[12]);
   float *xs = reinterpret_cast<float *>(smem + OFF_X);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -223,9 +236,12 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
 
   if (threadIdx.x == 0) {
     ctl.abort = 0;
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < NWRING; ++s) {
       mbar_init(bar_full_w + 8 * s, 1);
-      mbar_init(bar_raw_free + 8 * s, NCONV / 32);
+      // a pre-split slot is freed by the MMA's commit, a raw slot by the converters
+      mbar_init(bar_raw_free + 8 * s, PRESPLIT ? 1 : NCONV / 32);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar_ready + 8 * s, NCONV / 32);
       mbar_init(bar_empty + 8 * s, 1);
       mbar_init(bar_run_full + 8 * s, 1);
@@ -254,23 +270,31 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % NRAW, u = c / NRAW;
+        const int s = c % NWRING, u = c / NWRING;
         // After an abort every wait returns at once and the loops run to the end
         // without blocking, so all roles reach the final barrier.  A raw slot
-        // is free once the converters have split the chunk it held.
+        // is free once the converters have split the chunk it held; a
+        // pre-split slot once the MMAs that read it have finished.
         if (u > 0) mbar_wait(bar_raw_free + 8 * s, (u - 1) & 1, &ctl, status, 101);
-        const unsigned dst = smem_u32(smem + OFF_RAW + s * W_TILE);
-        mbar_arrive_tx(bar_full_w + 8 * s, W_BYTES);
+        const unsigned dst = smem_u32(smem + (PRESPLIT ? WL::hi(s) : WL::raw(s)));
+        mbar_arrive_tx(bar_full_w + 8 * s, PRESPLIT ? 2 * W_BYTES : W_BYTES);
         asm volatile(
             "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
             " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
             "l"(reinterpret_cast<uint64_t>(&tmap_w)), "r"(c * BK), "r"(w_row0),
             "r"(bar_full_w + 8 * s)
             : "memory");
+        if (PRESPLIT)
+          asm volatile(
+              "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+              " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(smem + WL::lo(s))),
+              "l"(reinterpret_cast<uint64_t>(&tmap_wlo)), "r"(c * BK), "r"(w_row0),
+              "r"(bar_full_w + 8 * s)
+              : "memory");
       }
       // drain: the last loads must land before the CTA can exit
-      for (int c = n_chunks - NRAW; c < n_chunks; ++c)
-        if (c >= 0) mbar_drain(bar_full_w + 8 * (c % NRAW), (c / NRAW) & 1);
+      for (int c = n_chunks - NWRING; c < n_chunks; ++c)
+        if (c >= 0) mbar_drain(bar_full_w + 8 * (c % NWRING), (c / NWRING) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
@@ -283,12 +307,14 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
         if (first && r >= 2)  // the converters have read this accumulator's run r - 2
           mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 106);
         mbar_wait(bar_ready + 8 * s, u & 1, &ctl, status, 102);
+        const int ws = PRESPLIT ? c % NWSLOT : s;  // weight slot of this chunk
+        if (PRESPLIT) mbar_wait(bar_full_w + 8 * ws, (c / NWSLOT) & 1, &ctl, status, 107);
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
         const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
         const unsigned x_hi = smem_u32(smem + OFF_XHI + s * X_TILE);
         const unsigned x_lo = smem_u32(smem + OFF_XLO + s * X_TILE);
-        const unsigned w_hi = smem_u32(smem + OFF_WHI + s * W_TILE);
-        const unsigned w_lo = smem_u32(smem + OFF_WLO + s * W_TILE);
+        const unsigned w_hi = smem_u32(smem + WL::hi(ws));
+        const unsigned w_lo = smem_u32(smem + WL::lo(ws));
 #pragma unroll
         for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes per MMA
           const unsigned off = 32 * k;
@@ -298,6 +324,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
           mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_hi + off), IDESC, 1u);
         }
         mma_commit(bar_empty + 8 * s);  // stage s may be refilled once these finish
+        if (PRESPLIT) mma_commit(bar_raw_free + 8 * ws);  // and the weight slot
         if (last) mma_commit(bar_run_full + 8 * ra);
       }
     }
@@ -369,11 +396,12 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
         if ((blk + 1) * CB < Cin) stage_x(blk + 1);
       }
       if (u > 0) warp_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 103);
+      if (!PRESPLIT) {
       warp_wait(bar_full_w + 8 * sr, (c / NRAW) & 1, &ctl, status, 104);
       // W: split into hi and lo (elementwise over the swizzled tile)
-      const unsigned char *w_raw = smem + OFF_RAW + sr * W_TILE;
-      unsigned char *w_hi = smem + OFF_WHI + s * W_TILE;
-      unsigned char *w_lo = smem + OFF_WLO + s * W_TILE;
+      const unsigned char *w_raw = smem + WL::raw(sr);
+      unsigned char *w_hi = smem + WL::hi(s);
+      unsigned char *w_lo = smem + WL::lo(s);
       constexpr int WCH = W_BYTES / 16;  // 16-byte chunks of the weight tile
       constexpr int WPT = (WCH + NCONV - 1) / NCONV;
       float4 wv[WPT];
@@ -394,6 +422,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const float *__rest
           *reinterpret_cast<float4 *>(w_lo + qo) =
               make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
         }
+      }
       }
       // X: time row ct of the im2col chunk, block-local kk = 32 m .. 32 m + 31
       unsigned char *x_hi = smem + OFF_XHI + s * X_TILE;
@@ -497,21 +526,23 @@ int pick_nt(int Cout) {
   return (per + 15) / 16 * 16;
 }
 
-template <int NT>
-bv_status run_tc(const CUtensorMap &tmap, const float *x, int B, int Cin, int T,
-                 const float *bias, int Cout, int K, int dil, int pad, const Epi &ep, float *y,
-                 int y_len, int y_pitch, const OutMap &om, cudaStream_t st) {
+template <int NT, bool PRESPLIT>
+bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const float *x, int B,
+                 int Cin, int T, const float *bias, int Cout, int K, int dil, int pad,
+                 const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
+                 cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
-    if (cudaFuncSetAttribute(conv1d_tc_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(conv1d_tc_kernel<NT, PRESPLIT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
       return check_launch("conv1d_tc smem attribute");
     configured = true;
   }
   dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B * om.phases);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
-  conv1d_tc_kernel<NT><<<grid, THREADS, SMEM_BYTES, st>>>(
-      tmap, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, om, device_status_ptr());
+  conv1d_tc_kernel<NT, PRESPLIT><<<grid, THREADS, SMEM_BYTES, st>>>(
+      tmap, tmap_lo, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, om,
+      device_status_ptr());
   return BV_OK;
 }
 
@@ -529,34 +560,50 @@ bool conv1d_tc_supported(int Cin, int Cout, int K, int dil) {
 
 namespace {
 
-// Encode the weight tensor map ([rows, Cin K] fp32, box 32 x nt, 128-byte
-// swizzle) and launch the NT instance.
-bv_status launch_tc_impl(const char *cls, const float *x, int B, int Cin, int T, const float *w,
-                         int w_rows, const float *bias, int Cout, int K, int dil, int pad,
-                         const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
-                         double flops, double bytes, cudaStream_t st) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: no cuTensorMapEncodeTiled");
+// Weight tensor map: [rows, Cin K] fp32, box 32 x nt, 128-byte swizzle.
+bv_status encode_w(CUtensorMap *tmap, const float *w, int rows, int KK, int nt) {
   if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: weights not 16-byte aligned");
-  const int nt = pick_nt(Cout);
-  CUtensorMap tmap;
-  const cuuint64_t dims[2] = {(cuuint64_t)Cin * K, (cuuint64_t)w_rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)Cin * K * sizeof(float)};
+  const cuuint64_t dims[2] = {(cuuint64_t)KK, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)KK * sizeof(float)};
   const cuuint32_t box[2] = {BK, (cuuint32_t)nt};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims,
-                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(BV_ERR_CUDA, "conv1d_tc: tensor map encode failed (%d)", (int)r);
-  bv_status s;
+  return BV_OK;
+}
+
+// Launch the NT instance.  w: the [w_rows, Cin K] weight matrix; or, when
+// split is set, w holds tf32(W) followed by W - tf32(W) (each [w_rows, Cin K])
+// and both operands go straight from global memory to the MMA, otherwise the
+// kernel splits the raw weights itself.
+bv_status launch_tc_impl(const char *cls, const float *x, int B, int Cin, int T, const float *w,
+                         bool split, int w_rows, const float *bias, int Cout, int K, int dil,
+                         int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                         const OutMap &om, double flops, double bytes, cudaStream_t st) {
+  if (!encode_fn()) return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: no cuTensorMapEncodeTiled");
+  const int nt = pick_nt(Cout);
+  CUtensorMap tmap, tmap_lo;
+  bv_status s = encode_w(&tmap, w, w_rows, Cin * K, nt);
+  if (s != BV_OK) return s;
+  if (split) {
+    s = encode_w(&tmap_lo, w + (size_t)w_rows * Cin * K, w_rows, Cin * K, nt);
+    if (s != BV_OK) return s;
+  } else {
+    tmap_lo = tmap;
+  }
   {
     LaunchTimer tm(st, cls, flops, bytes);
-#define BV_TC_CASE(N)                                                                      \
-  case N:                                                                                  \
-    s = run_tc<N>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, om, \
-                  st);                                                                     \
+#define BV_TC_CASE(N)                                                                          \
+  case N:                                                                                      \
+    s = split ? run_tc<N, true>(tmap, tmap_lo, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y,   \
+                               y_len, y_pitch, om, st)                                         \
+              : run_tc<N, false>(tmap, tmap_lo, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y,  \
+                                y_len, y_pitch, om, st);                                       \
     break;
     switch (nt) {
       BV_TC_CASE(16)
@@ -566,9 +613,9 @@ bv_status launch_tc_impl(const char *cls, const float *x, int B, int Cin, int T,
       BV_TC_CASE(80)
       BV_TC_CASE(96)
       BV_TC_CASE(112)
+      BV_TC_CASE(128)
       default:
-        s = run_tc<128>(tmap, x, B, Cin, T, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, om,
-                        st);
+        return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: tile %d", nt);
     }
 #undef BV_TC_CASE
   }
@@ -579,8 +626,9 @@ bv_status launch_tc_impl(const char *cls, const float *x, int B, int Cin, int T,
 
 // wp[r][o][i nt + j] = w[i][o][r + s (nt - 1 - j)] (zero past K): phase r of
 // the transposed conv as an ordinary nt-tap conv over the input samples.
-__global__ void convt_repack_kernel(const float *__restrict__ w, float *__restrict__ wp, int Cin,
-                                    int Cout, int K, int S, int nt) {
+__global__ void convt_repack_kernel(const float *__restrict__ w, float *__restrict__ wp,
+                                    float *__restrict__ wp_lo, int Cin, int Cout, int K, int S,
+                                    int nt) {
   const long long total = (long long)S * Cout * Cin * nt;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -591,18 +639,64 @@ __global__ void convt_repack_kernel(const float *__restrict__ w, float *__restri
     const int o = (int)(rest % Cout);
     const int r = (int)(rest / Cout);
     const int k = r + S * (nt - 1 - j);
-    wp[idx] = k < K ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
+    const float v = k < K ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
+    const float h = tf32_hi(v);
+    wp[idx] = h;
+    wp_lo[idx] = v - h;
+  }
+}
+
+// dst[0 .. n) = tf32(src), dst[n .. 2n) = src - tf32(src), per table entry
+// (float4 where the entry allows it)
+__global__ void split_weights_kernel(SplitTable tab) {
+  for (int e = blockIdx.y; e < tab.n; e += gridDim.y) {
+    const float *__restrict__ src = tab.src[e];
+    float *__restrict__ hi = tab.dst[e];
+    const long long n = tab.count[e];
+    float *__restrict__ lo = hi + n;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long i0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
+    const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) &&
+                     ((reinterpret_cast<uintptr_t>(hi) & 15u) == 0);
+    if (vec) {
+      for (long long i = i0; i < n / 4; i += stride) {
+        const float4 v = reinterpret_cast<const float4 *>(src)[i];
+        const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
+        reinterpret_cast<float4 *>(hi)[i] = h;
+        reinterpret_cast<float4 *>(lo)[i] = make_float4(v.x - h.x, v.y - h.y, v.z - h.z, v.w - h.w);
+      }
+    } else {
+      for (long long i = i0; i < n; i += stride) {
+        const float v = src[i], h = tf32_hi(v);
+        hi[i] = h;
+        lo[i] = v - h;
+      }
+    }
   }
 }
 
 }  // namespace
 
+bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st) {
+  if (tab.n <= 0) return BV_OK;
+  if (tab.n > kMaxSplit) return fail(BV_ERR_SHAPE, "split_weights: %d entries", tab.n);
+  double bytes = 0;
+  for (int e = 0; e < tab.n; ++e) bytes += 12.0 * tab.count[e];
+  {
+    LaunchTimer tm(st, "weight_split", 0.0, bytes);
+    split_weights_kernel<<<dim3(32, tab.n), 256, 0, st>>>(tab);
+  }
+  count_launch();
+  return check_launch("split_weights_kernel");
+}
+
 bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w,
-                           const float *bias, int Cout, int K, int dil, int pad, const Epi &ep,
-                           float *y, int y_len, int y_pitch, cudaStream_t st) {
+                           const float *w_split, const float *bias, int Cout, int K, int dil,
+                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                           cudaStream_t st) {
   const double outs = (double)B * Cout * y_len;
   const OutMap om{1, 0, y_len, 1};
-  return launch_tc_impl("conv1d_tc", x, B, Cin, T, w, Cout, bias, Cout, K, dil, pad, ep, y,
+  return launch_tc_impl("conv1d_tc", x, B, Cin, T, w_split ? w_split : w, w_split != nullptr, Cout, bias, Cout, K, dil, pad, ep, y,
                         y_len, y_pitch, om, 2.0 * outs * Cin * K,
                         4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                                outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)),
@@ -617,7 +711,7 @@ bool conv_transpose1d_tc_supported(int Cin, int Cout, int K, int S) {
 }
 
 size_t conv_transpose1d_tc_workspace(int Cin, int Cout, int K, int S) {
-  return (size_t)S * Cout * Cin * convt_taps(K, S) * sizeof(float);
+  return 2 * (size_t)S * Cout * Cin * convt_taps(K, S) * sizeof(float);  // wp and its lo part
 }
 
 bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
@@ -630,7 +724,7 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
     LaunchTimer tm(st, "convt_repack", 0.0, 8.0 * (double)total);
     const long long blocks = (total + 255) / 256;
     convt_repack_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
-        w, wp, Cin, Cout, K, S, nt);
+        w, wp, wp + total, Cin, Cout, K, S, nt);
   }
   count_launch();
   bv_status s = check_launch("convt_repack_kernel");
@@ -639,7 +733,8 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
   // S P + r - pad of the output row
   const OutMap om{S, -pad, Tout, S};
   const Epi plain{nullptr, 1.0f, 0, 0};
-  return launch_tc_impl("conv_transpose1d_tc", x, B, Cin, T, wp, S * Cout, bias, Cout, nt, 1,
+  return launch_tc_impl("conv_transpose1d_tc", x, B, Cin, T, wp, true, S * Cout, bias, Cout,
+                        nt, 1,
                         nt - 1, plain, y, T + nt - 1, Tout, om,
                         2.0 * B * Cin * (double)Cout * K * T,
                         4.0 * ((double)B * Cin * T + (double)Cin * Cout * K +
