@@ -109,12 +109,6 @@ bv_status check_device() {
   return BV_OK;
 }
 
-#define BV_TRY(expr)                 \
-  do {                               \
-    bv_status _s = (expr);           \
-    if (_s != BV_OK) return _s;      \
-  } while (0)
-
 // ------------------------------------------------------------- filter design
 
 // Modified Bessel I0 by its power series; terms (x/2)^{2k}/(k!)^2 accumulate
@@ -318,41 +312,54 @@ bv_status check_amp_params(const bv_amp_params *p, int C) {
   return BV_OK;
 }
 
+// xhi / xlo: two [B, T, C] planes for the time-major tensor-core convs
+// (nullptr: every conv reads h1 in [B, C, T]).
 struct AmpScratch {
   float *cur, *h1, *h2;
+  float *xhi = nullptr, *xlo = nullptr;
 };
 
 // Pre-split tensor-core weights of one AMP block's convs (nullptr: the conv
-// splits its own weights).
+// splits its own weights); tm marks tap-major weights for the time-major conv.
 struct AmpSplit {
   const float *conv1[BV_MAX_DIL], *conv2[BV_MAX_DIL];
+  bool tm1[BV_MAX_DIL], tm2[BV_MAX_DIL];
 };
+
+// act -> conv with the activation's output in h1: through the time-major
+// planes when the block's scratch and weights are set up for it.
+bv_status act_conv(const float *in, int B, int C, int T, const float *la, const float *lb,
+                   const bv_amp_params &p, const float *w, const float *bias, const float *w_split,
+                   bool tm, int dil, const Epi &ep, float *out, const AmpScratch &s,
+                   cudaStream_t st) {
+  const int K = p.kernel_size, pad = (K * dil - dil) / 2;
+  BV_TRY(launch_activation(in, s.h1, B, C, T, la, lb, p.up_filter, p.down_filter, 1e-9f, st));
+  if (tm && w_split && s.xhi) {
+    BV_TRY(launch_transpose_split(s.h1, s.xhi, s.xlo, B, C, T, st));
+    return launch_conv1d_tm(s.xhi, s.xlo, B, C, T, w_split, bias, C, K, dil, pad, ep, out, T, T,
+                            st);
+  }
+  return launch_conv1d(s.h1, B, C, T, w, bias, C, K, dil, pad, ep, out, T, T, st, w_split);
+}
 
 // y = (accumulate ? y : 0) + scale * AMP(x); x, y and the scratch are disjoint.
 bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params &p, float *y,
                         float scale, int accumulate, const AmpScratch &s, cudaStream_t st,
                         const AmpSplit *sp = nullptr) {
-  const int K = p.kernel_size, n = p.n_dilations;
-  const float eps = 1e-9f;
+  const int n = p.n_dilations;
   for (int u = 0; u < n; ++u) {
     const float *src = (u == 0) ? x : s.cur;
-    const int d = p.dilation[u];
-    BV_TRY(launch_activation(src, s.h1, B, C, T, p.act_log_alpha[2 * u], p.act_log_beta[2 * u],
-                             p.up_filter, p.down_filter, eps, st));
-    Epi plain{nullptr, 1.0f, 0, 0};
-    BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv1_w[u], p.conv1_b[u], C, K, d, (K * d - d) / 2,
-                         plain, s.h2, T, T, st, sp ? sp->conv1[u] : nullptr));
-    BV_TRY(launch_activation(s.h2, s.h1, B, C, T, p.act_log_alpha[2 * u + 1],
-                             p.act_log_beta[2 * u + 1], p.up_filter, p.down_filter, eps, st));
-    if (u == n - 1) {
-      Epi last{src, scale, accumulate, 0};
-      BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, last,
-                           y, T, T, st, sp ? sp->conv2[u] : nullptr));
-    } else {
-      Epi res{src, 1.0f, 0, 0};  // cur = src + conv2(...); src may be cur itself
-      BV_TRY(launch_conv1d(s.h1, B, C, T, p.conv2_w[u], p.conv2_b[u], C, K, 1, (K - 1) / 2, res,
-                           s.cur, T, T, st, sp ? sp->conv2[u] : nullptr));
-    }
+    const Epi plain{nullptr, 1.0f, 0, 0};
+    BV_TRY(act_conv(src, B, C, T, p.act_log_alpha[2 * u], p.act_log_beta[2 * u], p, p.conv1_w[u],
+                    p.conv1_b[u], sp ? sp->conv1[u] : nullptr, sp && sp->tm1[u], p.dilation[u],
+                    plain, s.h2, s, st));
+    // last unit: y (+)= scale (src + conv2(...)); otherwise cur = src + conv2(...),
+    // where src may be cur itself
+    const bool last = (u == n - 1);
+    const Epi res = last ? Epi{src, scale, accumulate, 0} : Epi{src, 1.0f, 0, 0};
+    BV_TRY(act_conv(s.h2, B, C, T, p.act_log_alpha[2 * u + 1], p.act_log_beta[2 * u + 1], p,
+                    p.conv2_w[u], p.conv2_b[u], sp ? sp->conv2[u] : nullptr, sp && sp->tm2[u], 1,
+                    res, last ? y : s.cur, s, st));
   }
   return BV_OK;
 }
@@ -469,35 +476,39 @@ struct DecoderSplit {
   AmpSplit amp[BV_MAX_UP][BV_MAX_BLOCKS] = {};
 };
 
-// Walk the decoder's convs in a fixed order; f(Cin, Cout, K, dil, src, slot)
-// is called for each conv the tensor-core path supports (src may be null when
-// only sizes are wanted).
+// Walk the decoder's convs in a fixed order; f(Cin, Cout, K, src, kind, i, j,
+// u, tm) is called for each conv a tensor-core path supports (src may be null
+// when only sizes are wanted); tm: the AMP conv takes the time-major path.
 template <class F>
 void for_each_tc_conv(const bv_decoder_config *c, const bv_decoder_weights *w, F &&f) {
   if (conv1d_tc_supported(c->in_channels, c->pre_channels, c->pre_kernel, 1))
-    f(c->in_channels, c->pre_channels, c->pre_kernel, w ? w->pre_w : nullptr, 0, -1, -1, -1);
+    f(c->in_channels, c->pre_channels, c->pre_kernel, w ? w->pre_w : nullptr, 0, -1, -1, -1,
+      false);
   for (int i = 0; i < c->n_up; ++i) {
     const int C = c->up_channels[i];
     for (int j = 0; j < c->n_blocks; ++j) {
       const int K = c->block_kernel[j];
       for (int u = 0; u < c->n_dilations; ++u) {
-        if (conv1d_tc_supported(C, C, K, c->dilation[u]))
-          f(C, C, K, w ? w->amp[i][j].conv1_w[u] : nullptr, 1, i, j, u);
-        if (conv1d_tc_supported(C, C, K, 1))
-          f(C, C, K, w ? w->amp[i][j].conv2_w[u] : nullptr, 2, i, j, u);
+        const int d = c->dilation[u];
+        const bool tm1 = conv1d_tm_supported(C, C, K, d), tm2 = conv1d_tm_supported(C, C, K, 1);
+        if (tm1 || conv1d_tc_supported(C, C, K, d))
+          f(C, C, K, w ? w->amp[i][j].conv1_w[u] : nullptr, 1, i, j, u, tm1);
+        if (tm2 || conv1d_tc_supported(C, C, K, 1))
+          f(C, C, K, w ? w->amp[i][j].conv2_w[u] : nullptr, 2, i, j, u, tm2);
       }
     }
   }
   const int Cl = c->n_up > 0 ? c->up_channels[c->n_up - 1] : c->pre_channels;
   if (conv1d_tc_supported(Cl, c->out_channels, c->post_kernel, 1))
-    f(Cl, c->out_channels, c->post_kernel, w ? w->post_w : nullptr, 3, -1, -1, -1);
+    f(Cl, c->out_channels, c->post_kernel, w ? w->post_w : nullptr, 3, -1, -1, -1, false);
 }
 
 size_t split_ws(const bv_decoder_config *c) {
   size_t s = 0;
-  for_each_tc_conv(c, nullptr, [&](int Cin, int Cout, int K, const float *, int, int, int, int) {
-    s += align_up(2 * (size_t)Cin * Cout * K * sizeof(float));
-  });
+  for_each_tc_conv(c, nullptr,
+                   [&](int Cin, int Cout, int K, const float *, int, int, int, int, bool) {
+                     s += align_up(2 * (size_t)Cin * Cout * K * sizeof(float));
+                   });
   return s;
 }
 
@@ -509,19 +520,29 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
   bv_status status = BV_OK;
   size_t off = 0;
   for_each_tc_conv(c, w, [&](int Cin, int Cout, int K, const float *src, int kind, int i, int j,
-                             int u) {
+                             int u, bool tm) {
     if (status != BV_OK) return;
     const long long count = (long long)Cin * Cout * K;
     float *dst = reinterpret_cast<float *>(ws + off);
     off += align_up(2 * (size_t)count * sizeof(float));
-    if ((reinterpret_cast<uintptr_t>(src) & 15u) != 0) return;  // SIMT path: no split needed
-    if (kind == 0) out->pre = dst;
-    else if (kind == 1) out->amp[i][j].conv1[u] = dst;
-    else if (kind == 2) out->amp[i][j].conv2[u] = dst;
-    else out->post = dst;
+    // an unaligned weight sends a [B, C, T] conv to the SIMT path: no split needed
+    if (!tm && (reinterpret_cast<uintptr_t>(src) & 15u) != 0) return;
+    if (kind == 0) {
+      out->pre = dst;
+    } else if (kind == 1) {
+      out->amp[i][j].conv1[u] = dst;
+      out->amp[i][j].tm1[u] = tm;
+    } else if (kind == 2) {
+      out->amp[i][j].conv2[u] = dst;
+      out->amp[i][j].tm2[u] = tm;
+    } else {
+      out->post = dst;
+    }
     tab.src[tab.n] = src;
     tab.dst[tab.n] = dst;
     tab.count[tab.n] = count;
+    tab.cin[tab.n] = tm ? Cin : 0;
+    tab.k[tab.n] = K;
     if (++tab.n == kMaxSplit) {
       status = launch_split_weights(tab, st);
       tab.n = 0;
@@ -531,8 +552,10 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
   return launch_split_weights(tab, st);
 }
 
+// A, S, cur, h1, h2 in [B, C, T] and the two time-major planes, then the
+// repacked transposed-conv weights.
 size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
-  return 5 * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
+  return 7 * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
 }
 
 struct TilePlan {
@@ -609,8 +632,9 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
   float *A = reinterpret_cast<float *>(ws);
   float *S = reinterpret_cast<float *>(ws + sz);
   AmpScratch s{reinterpret_cast<float *>(ws + 2 * sz), reinterpret_cast<float *>(ws + 3 * sz),
-               reinterpret_cast<float *>(ws + 4 * sz)};
-  float *WP = reinterpret_cast<float *>(ws + 5 * sz);  // repacked ConvT weights
+               reinterpret_cast<float *>(ws + 4 * sz), reinterpret_cast<float *>(ws + 5 * sz),
+               reinterpret_cast<float *>(ws + 6 * sz)};
+  float *WP = reinterpret_cast<float *>(ws + 7 * sz);  // repacked ConvT weights
   int C = c->pre_channels, n = F;
   Epi plain{nullptr, 1.0f, 0, 0};
   BV_TRY(launch_conv1d(z, B, c->in_channels, F, w->pre_w, w->pre_b, C, c->pre_kernel, 1,

@@ -85,6 +85,12 @@ bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, c
 
 // Conv1d on the tensor cores (tcgen05, 3xTF32); supported() says whether the
 // shape qualifies (launch_conv1d picks it automatically).
+#define BV_TRY(expr)            \
+  do {                          \
+    bv_status _s = (expr);      \
+    if (_s != BV_OK) return _s; \
+  } while (0)
+
 // w_split: tf32(W) followed by W - tf32(W), each in w's layout (written by
 // launch_split_weights), or nullptr, in which case the kernel splits w itself.
 bool conv1d_tc_supported(int Cin, int Cout, int K, int dil);
@@ -95,14 +101,33 @@ bv_status launch_conv1d_tc(const float *x, int B, int Cin, int T, const float *w
 
 // tf32(W) and W - tf32(W) of a batch of weight tensors in one launch: entry e
 // writes dst[e][0, count) = tf32(src[e]) and dst[e][count, 2 count) = the rest.
-constexpr int kMaxSplit = 128;  // keeps the table under 4 KB of kernel parameters
+constexpr int kMaxSplit = 96;  // keeps the table under 4 KB of kernel parameters
 struct SplitTable {
   int n;
   const float *src[kMaxSplit];
   float *dst[kMaxSplit];
   long long count[kMaxSplit];
+  // tap-major entries: src is [rows][cin][k] and dst[o][j cin + i] = src[o][i][j];
+  // cin = 0 keeps src's order
+  int cin[kMaxSplit], k[kMaxSplit];
 };
 bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
+
+// Time-major tensor-core conv: x_hi / x_lo are [B, T, Cin] planes with
+// x = x_hi + x_lo, x_hi = tf32(x) (launch_transpose_split writes them);
+// w_split holds tf32(W') then W' - tf32(W') for the tap-major weight matrix
+// W'[o, j Cin + i] = w[o, i, j] (launch_split_weights with tap_major set).
+// Output and epilogue as launch_conv1d ([B, Cout, y_pitch]).
+bool conv1d_tm_supported(int Cin, int Cout, int K, int dil);
+bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                           const float *w_split, const float *bias, int Cout, int K, int dil,
+                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                           cudaStream_t st);
+
+// [B, C, T] -> time-major planes hi[b, t, c] = tf32(x[b, c, t]),
+// lo = x - hi (C a multiple of 32).
+bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
+                                 cudaStream_t st);
 
 // ConvTranspose1d on the tensor cores: each output phase is an ordinary conv
 // over the input samples with repacked weights (wp: workspace of

@@ -546,6 +546,243 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
   return BV_OK;
 }
 
+// ---------------------------------------------------------------------------
+// Time-major variant: the input arrives as two [B, T, Cin] planes, X_hi =
+// tf32(x) and X_lo = x - X_hi (written by launch_transpose_split), and the
+// weights as tap-major [Cout, K Cin] hi / lo matrices, W'[o, j Cin + i] =
+// w[o, i, j].  Reduction chunk c = (tap j, 32-channel block cb) is then a
+// plain 2-D box of each plane: rows t0 - pad + j d .. + 127 (zero outside
+// [0, T), which is the conv's zero padding) by channels 32 cb .. 32 cb + 31,
+// already K-major with 128-byte rows.  So all four operand tiles of a chunk
+// come by TMA and no warp touches them: one thread issues the loads, one the
+// MMAs, and four warps add finished runs into FP32 registers and write the
+// [B, Cout, T] output with the usual epilogue.
+constexpr int TM_STAGES = 3;
+constexpr int TM_TILE = 16384;                        // one 128 x 32 fp32 operand tile
+constexpr int TM_STAGE_BYTES = 4 * TM_TILE;           // X_hi, X_lo, W_hi, W_lo
+constexpr int TM_OFF_BAR = TM_STAGES * TM_STAGE_BYTES;
+constexpr int TM_SMEM_BYTES = TM_OFF_BAR + 16 * 8 + 1024;
+static_assert(TM_SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+template <int NT>
+__global__ void __launch_bounds__(THREADS, 1)
+conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
+                 const __grid_constant__ CUtensorMap tmap_xlo,
+                 const __grid_constant__ CUtensorMap tmap_whi,
+                 const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ bias,
+                 float *y, int Cin, int Cout, int K, int dil, int pad, int y_len, int y_pitch,
+                 Epi ep, int *status) {
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
+  constexpr uint32_t IDESC = make_idesc(NT);
+  constexpr unsigned STAGE_TX = 2 * TM_TILE + 2 * NT * BK * 4;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char *smem = reinterpret_cast<unsigned char *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TM_OFF_BAR);
+  __shared__ Ctl ctl;
+  // barriers: stage loaded (TMA) / stage consumed (MMA commit), per stage;
+  // run accumulated / run accumulator read, per TMEM accumulator
+  const unsigned bar_full = smem_u32(&bars[0]);
+  const unsigned bar_empty = smem_u32(&bars[TM_STAGES]);
+  const unsigned bar_run_full = smem_u32(&bars[2 * TM_STAGES]);
+  const unsigned bar_run_free = smem_u32(&bars[2 * TM_STAGES + 2]);
+  auto xhi_at = [&](int s) { return smem + s * TM_STAGE_BYTES; };
+  auto xlo_at = [&](int s) { return smem + s * TM_STAGE_BYTES + TM_TILE; };
+  auto whi_at = [&](int s) { return smem + s * TM_STAGE_BYTES + 2 * TM_TILE; };
+  auto wlo_at = [&](int s) { return smem + s * TM_STAGE_BYTES + 3 * TM_TILE; };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = blockIdx.x * BM;
+  const int o0 = blockIdx.y * NT;
+  const int b = blockIdx.z;
+  const int n_cb = Cin / BK;  // 32-channel blocks per tap
+  const int n_chunks = K * n_cb;
+  const int n_runs = (n_chunks + RUN - 1) / RUN;
+
+  if (threadIdx.x == 0) {
+    ctl.abort = 0;
+    for (int s = 0; s < TM_STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_run_full + 8 * s, 1);
+      mbar_init(bar_run_free + 8 * s, NCONV / 32);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+                     smem_u32(&ctl.tmem)),
+                 "n"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+  const unsigned tmem = ctl.tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % TM_STAGES, u = c / TM_STAGES;
+        // after an abort every wait returns at once, so all roles run to the end
+        if (u > 0) mbar_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 111);
+        const int j = c / n_cb, cb = c - j * n_cb;
+        const int xt = t0 - pad + j * dil;  // first input time of the box (may be < 0)
+        const unsigned fb = bar_full + 8 * s;
+        mbar_arrive_tx(fb, STAGE_TX);
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(xhi_at(s))),
+            "l"(reinterpret_cast<uint64_t>(&tmap_xhi)), "r"(cb * BK), "r"(xt), "r"(b), "r"(fb)
+            : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(xlo_at(s))),
+            "l"(reinterpret_cast<uint64_t>(&tmap_xlo)), "r"(cb * BK), "r"(xt), "r"(b), "r"(fb)
+            : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(whi_at(s))),
+            "l"(reinterpret_cast<uint64_t>(&tmap_whi)), "r"(c * BK), "r"(o0), "r"(fb)
+            : "memory");
+        asm volatile(
+            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+            " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(wlo_at(s))),
+            "l"(reinterpret_cast<uint64_t>(&tmap_wlo)), "r"(c * BK), "r"(o0), "r"(fb)
+            : "memory");
+      }
+      // drain: the last loads must land before the CTA can exit
+      for (int c = n_chunks - TM_STAGES; c < n_chunks; ++c)
+        if (c >= 0) mbar_drain(bar_full + 8 * (c % TM_STAGES), (c / TM_STAGES) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % TM_STAGES, u = c / TM_STAGES;
+        const int r = c / RUN, ra = r & 1;
+        const bool first = (c % RUN) == 0;
+        const bool last = (c % RUN) == RUN - 1 || c == n_chunks - 1;
+        if (first && r >= 2)  // the sum warps have read this accumulator's run r - 2
+          mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 112);
+        mbar_wait(bar_full + 8 * s, u & 1, &ctl, status, 113);
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
+        const unsigned x_hi = smem_u32(xhi_at(s)), x_lo = smem_u32(xlo_at(s));
+        const unsigned w_hi = smem_u32(whi_at(s)), w_lo = smem_u32(wlo_at(s));
+#pragma unroll
+        for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes per MMA
+          const unsigned off = 32 * k;
+          mma_tf32(acc, sw128_desc(x_lo + off), sw128_desc(w_hi + off), IDESC,
+                   (first && k == 0) ? 0u : 1u);
+          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_lo + off), IDESC, 1u);
+          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_hi + off), IDESC, 1u);
+        }
+        mma_commit(bar_empty + 8 * s);  // the stage may be refilled once these finish
+        if (last) mma_commit(bar_run_full + 8 * ra);
+      }
+    }
+  } else if (warp >= CONV_WARP0) {
+    // ------------------------------------------------------ run sums + output
+    const int ct = threadIdx.x - CONV_WARP0 * 32;  // time row of this thread
+    const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
+    float sum[NT];
+#pragma unroll
+    for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
+    for (int p = 0; p < n_runs; ++p) {
+      const int ra = p & 1;
+      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 114);
+      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+      for (int c0 = 0; c0 < NT; c0 += 16) {
+        uint32_t v[16];
+        const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * MAX_NT + c0);
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15}, [%16];\n"
+            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+              "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+              "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+            : "r"(taddr)
+            : "memory");
+        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+      }
+      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_run_free + 8 * ra);
+    }
+    const int t = t0 + ct;
+    if (!ctl.abort && t < y_len) {
+#pragma unroll
+      for (int e = 0; e < NT; ++e) {
+        const int o = o0 + e;
+        if (o < Cout) {
+          const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
+          const float bo = bias ? __ldg(bias + o) : 0.0f;
+          y[idx] = apply_epilogue(sum[e], bo, ep, y, idx);
+        }
+      }
+    }
+  }
+
+  asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+  __syncthreads();
+  if (warp == 1) {
+    // no MMA may still write an accumulator when it is freed
+    if (lane == 0 && n_runs > 0) {
+      mbar_drain(bar_run_full + 8 * ((n_runs - 1) & 1), ((n_runs - 1) >> 1) & 1);
+      if (n_runs > 1) mbar_drain(bar_run_full + 8 * ((n_runs - 2) & 1), ((n_runs - 2) >> 1) & 1);
+    }
+    __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+                 "n"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+template <int NT>
+bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
+                 const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
+                 int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                 cudaStream_t st) {
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(conv1d_tm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             TM_SMEM_BYTES) != cudaSuccess)
+      return check_launch("conv1d_tm smem attribute");
+    configured = true;
+  }
+  dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tm: grid too large");
+  conv1d_tm_kernel<NT><<<grid, THREADS, TM_SMEM_BYTES, st>>>(
+      xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, device_status_ptr());
+  return BV_OK;
+}
+
+// [B, T, C] fp32 plane as a 3-D tensor map, box 32 channels x 128 times.
+bv_status encode_x_tm(CUtensorMap *tmap, const float *x, int B, int C, int T) {
+  if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0)
+    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: input not 16-byte aligned");
+  const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)C * sizeof(float), (cuuint64_t)T * C * sizeof(float)};
+  const cuuint32_t box[3] = {BK, BM, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(BV_ERR_CUDA, "conv1d_tm: tensor map encode failed (%d)", (int)r);
+  return BV_OK;
+}
+
 }  // namespace
 
 // The tensor-core path pays a fixed cost per CTA (barriers, TMEM, pipeline
@@ -647,7 +884,7 @@ __global__ void convt_repack_kernel(const float *__restrict__ w, float *__restri
 }
 
 // dst[0 .. n) = tf32(src), dst[n .. 2n) = src - tf32(src), per table entry
-// (float4 where the entry allows it)
+// (float4 where the entry allows it; tap-major entries reorder as they go)
 __global__ void split_weights_kernel(SplitTable tab) {
   for (int e = blockIdx.y; e < tab.n; e += gridDim.y) {
     const float *__restrict__ src = tab.src[e];
@@ -658,7 +895,18 @@ __global__ void split_weights_kernel(SplitTable tab) {
     const long long i0 = blockIdx.x * (long long)blockDim.x + threadIdx.x;
     const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) &&
                      ((reinterpret_cast<uintptr_t>(hi) & 15u) == 0);
-    if (vec) {
+    if (tab.cin[e] > 0) {
+      const int cin = tab.cin[e], k = tab.k[e];
+      const long long row = (long long)cin * k;
+      for (long long d = i0; d < n; d += stride) {  // d = o row + j cin + i
+        const long long o = d / row;
+        const int rem = (int)(d - o * row);
+        const int j = rem / cin, i = rem - j * cin;
+        const float v = src[o * row + (long long)i * k + j], h = tf32_hi(v);
+        hi[d] = h;
+        lo[d] = v - h;
+      }
+    } else if (vec) {
       for (long long i = i0; i < n / 4; i += stride) {
         const float4 v = reinterpret_cast<const float4 *>(src)[i];
         const float4 h = make_float4(tf32_hi(v.x), tf32_hi(v.y), tf32_hi(v.z), tf32_hi(v.w));
@@ -675,7 +923,50 @@ __global__ void split_weights_kernel(SplitTable tab) {
   }
 }
 
+// hi[b, t, c] = tf32(x[b, c, t]), lo = x - hi: 32 x 32 tiles through shared
+// memory, reads along t and writes along c both coalesced.
+__global__ void __launch_bounds__(256) transpose_split_kernel(const float *__restrict__ x,
+                                                               float *__restrict__ hi,
+                                                               float *__restrict__ lo, int C,
+                                                               int T) {
+  __shared__ float tile[32][33];
+  const int t0 = blockIdx.x * 32, c0 = blockIdx.y * 32, b = blockIdx.z;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32
+  const float *xb = x + (size_t)b * C * T;
+#pragma unroll
+  for (int r = ty; r < 32; r += 8) {
+    const int t = t0 + tx;
+    tile[r][tx] = t < T ? __ldcs(xb + (size_t)(c0 + r) * T + t) : 0.0f;
+  }
+  __syncthreads();
+  const size_t ob = (size_t)b * T * C;
+#pragma unroll
+  for (int r = ty; r < 32; r += 8) {
+    const int t = t0 + r;
+    if (t < T) {
+      const float v = tile[tx][r], h = tf32_hi(v);
+      const size_t idx = ob + (size_t)t * C + c0 + tx;
+      hi[idx] = h;
+      lo[idx] = v - h;
+    }
+  }
+}
+
 }  // namespace
+
+bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
+                                 cudaStream_t st) {
+  if (B <= 0 || T <= 0) return BV_OK;
+  if (C % 32 != 0) return fail(BV_ERR_SHAPE, "transpose_split: C %d not a multiple of 32", C);
+  dim3 grid((T + 31) / 32, C / 32, B);
+  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "transpose_split: grid");
+  {
+    LaunchTimer tm(st, "transpose_split", 0.0, 12.0 * B * C * T);
+    transpose_split_kernel<<<grid, 256, 0, st>>>(x, hi, lo, C, T);
+  }
+  count_launch();
+  return check_launch("transpose_split_kernel");
+}
 
 bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st) {
   if (tab.n <= 0) return BV_OK;
@@ -740,6 +1031,53 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
                         4.0 * ((double)B * Cin * T + (double)Cin * Cout * K +
                                (double)B * Cout * Tout),
                         st);
+}
+
+
+bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
+  (void)dil;
+  return Cin % BK == 0 && Cout >= 40 && Cin * K >= 192 && encode_fn() != nullptr;
+}
+
+bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                           const float *w_split, const float *bias, int Cout, int K, int dil,
+                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                           cudaStream_t st) {
+  if (B <= 0 || y_len <= 0) return BV_OK;
+  if (!conv1d_tm_supported(Cin, Cout, K, dil))
+    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
+  const int nt = pick_nt(Cout);
+  const int KK = Cin * K;
+  CUtensorMap xh, xl, wh, wl;
+  BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T));
+  BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T));
+  BV_TRY(encode_w(&wh, w_split, Cout, KK, nt));
+  BV_TRY(encode_w(&wl, w_split + (size_t)Cout * KK, Cout, KK, nt));
+  bv_status s;
+  {
+    const double outs = (double)B * Cout * y_len;
+    LaunchTimer tm(st, "conv1d_tc", 2.0 * outs * KK,
+                   4.0 * ((double)B * Cin * T + (double)Cout * KK +
+                          outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
+#define BV_TM_CASE(N)                                                                          \
+  case N:                                                                                      \
+    s = run_tm<N>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
+    break;
+    switch (nt) {
+      BV_TM_CASE(48)
+      BV_TM_CASE(64)
+      BV_TM_CASE(80)
+      BV_TM_CASE(96)
+      BV_TM_CASE(112)
+      BV_TM_CASE(128)
+      default:
+        return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: tile %d", nt);
+    }
+#undef BV_TM_CASE
+  }
+  if (s != BV_OK) return s;
+  count_launch();
+  return check_launch("conv1d_tm_kernel");
 }
 
 }  // namespace bv

@@ -424,7 +424,8 @@ def test_real_geometry_short_latent(nat, oracle, filt, wname, frames):
 @pytest.mark.parametrize("frames", [1, 2, 5, 27])
 def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     """A decoder wide enough that its ConvT stages (both stride parities) and
-    its AMP convs take the tensor-core path, on short and ragged latents."""
+    its AMP convs take the tensor-core paths (time-major input at 128 and 96
+    channels, [B, C, T] input at 48), on short and ragged latents."""
     geo = synth.tiny_geometry(pre_channels=256, up_channels=(128, 96, 48), in_channels=16)
     s = synth.NormalStream(40 + frames)
     z = s.normal((2, geo.in_channels, frames))
@@ -434,6 +435,7 @@ def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault("y", dec.decode(zd)))
     assert "conv_transpose1d_tc" in classes and "conv1d_tc" in classes, classes
+    assert "transpose_split" in classes, classes  # the 128/96-channel AMP convs run time-major
     want = oracle.decode(geo, params, z)
     assert rel_l2(host(out["y"]), want) < WAVE_TOL
 
