@@ -526,6 +526,14 @@ int pick_nt(int Cout) {
   return (per + 15) / 16 * 16;
 }
 
+// Channels per CTA pair: the fewest tiles of at most 128, each a multiple of
+// 32 (two halves of 16 rows, the smallest B half the pair's MMA takes).
+int pick_nt_pair(int Cout) {
+  const int tiles = (Cout + MAX_NT - 1) / MAX_NT;
+  const int per = (Cout + tiles - 1) / tiles;
+  return (per + 31) / 32 * 32;
+}
+
 template <int NT, bool PRESPLIT>
 bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const float *x, int B,
                  int Cin, int T, const float *bias, int Cout, int K, int dil, int pad,
@@ -547,155 +555,321 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
 }
 
 // ---------------------------------------------------------------------------
-// Time-major variant: the input arrives as two [B, T, Cin] planes, X_hi =
-// tf32(x) and X_lo = x - X_hi (written by launch_transpose_split), and the
-// weights as tap-major [Cout, K Cin] hi / lo matrices, W'[o, j Cin + i] =
-// w[o, i, j].  Reduction chunk c = (tap j, 32-channel block cb) is then a
-// plain 2-D box of each plane: rows t0 - pad + j d .. + 127 (zero outside
-// [0, T), which is the conv's zero padding) by channels 32 cb .. 32 cb + 31,
-// already K-major with 128-byte rows.  So all four operand tiles of a chunk
-// come by TMA and no warp touches them: one thread issues the loads, one the
-// MMAs, and four warps add finished runs into FP32 registers and write the
-// [B, Cout, T] output with the usual epilogue.
-constexpr int TM_STAGES = 3;
-constexpr int TM_TILE = 16384;                        // one 128 x 32 fp32 operand tile
-constexpr int TM_STAGE_BYTES = 4 * TM_TILE;           // X_hi, X_lo, W_hi, W_lo
-constexpr int TM_OFF_BAR = TM_STAGES * TM_STAGE_BYTES;
-constexpr int TM_SMEM_BYTES = TM_OFF_BAR + 16 * 8 + 1024;
-static_assert(TM_SMEM_BYTES <= 227 * 1024, "shared memory budget");
+// Time-major variant on CTA pairs.  The input arrives as two [B, T, Cin]
+// planes, X_hi = tf32(x) and X_lo = x - X_hi (written by
+// launch_transpose_split), and the weights as tap-major [Cout, K Cin] hi / lo
+// matrices, W'[o, j Cin + i] = w[o, i, j].
+//
+// Two CTAs of a cluster share each MMA (tcgen05 cta_group::2, M = 256): CTA r
+// of the pair owns time rows t0 + 128 r .. + 127 (its half of the A operand
+// and of the accumulator) and loads weight rows o0 + r NT/2 .. + NT/2 - 1
+// (its half of the B operand), so each SM fetches half the weight bytes a
+// lone CTA would; the weights are what every time tile re-reads from L2.
+//
+// For each 32-channel block cb, one TMA box per plane brings input rows
+// t0 - pad .. t0 - pad + 127 + (K - 1) d (zero outside [0, T), the conv's
+// zero padding) by the block's 32 channels: K-major rows of 128 bytes, the A
+// operand layout.  Tap j's A operand is the same box seen from row j d on:
+// its descriptor starts j d rows in.  Both the TMA write and the tensor core's
+// read place a 16-byte chunk by the absolute shared-memory address (chunk
+// bits XOR row bits 7-9), so a start inside an 8-row group needs no base
+// offset (measured on B200: setting the descriptor's base-offset field to the
+// row phase breaks the result).  The input is fetched once per channel block;
+// only the weight chunks (j, cb) stream through a ring.
+//
+// Roles: in each CTA one thread of warp 0 issues the weight loads and one of
+// warp 2 the x loads, completing on the even CTA's barriers (which expect both
+// CTAs' bytes); one thread of the even CTA issues the MMAs and commits to
+// barriers in both CTAs; four warps per CTA add finished runs into FP32
+// registers and write that CTA's rows of the [B, Cout, T] output with the
+// usual epilogue.  A chunk is two taps of one channel block (24 MMAs), so the
+// per-chunk cost of a barrier wait and a commit in the issuing thread is
+// spread over twice the tensor work.
+constexpr int TM_MAX_HALO = 56;                       // (K - 1) d the x box can hold
+constexpr int TM_W_PLANE = (MAX_NT / 2) * BK * 4;     // 8 KB: one CTA's half of a weight plane
+constexpr int TM_W_SLOT = 2 * 2 * TM_W_PLANE;         // a chunk: two taps, hi and lo
+constexpr int TM_MAX_WSLOTS = 6;
+constexpr int TM_RUN = 2;                              // chunks (up to 4 taps of 32) per run
+constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
+constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
+constexpr int TM_XSLOTS = 2;                          // x blocks in flight
+constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 + 2;
+static_assert(TM_SMEM_BYTES + 64 <= 227 * 1024, "shared memory budget");
+
+// Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
+__host__ __device__ constexpr int tm_x_plane(int rows) { return (rows * 128 + 1023) / 1024 * 1024; }
+// Weight ring slots that fit beside the x slots of `rows` rows.
+__host__ __device__ constexpr int tm_w_slots(int rows) {
+  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / TM_W_SLOT <
+                 TM_MAX_WSLOTS
+             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / TM_W_SLOT
+             : TM_MAX_WSLOTS;
+}
+static_assert(tm_w_slots(BM + TM_MAX_HALO) >= 4, "weight ring depth");
+static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 4 * TM_W_SLOT + TM_NBARS * 8 <=
+                  TM_BUDGET,
+              "shared memory layout");
+
+// Instruction descriptor for the pair: D f32, A and B tf32, K-major, M = 256.
+__host__ __device__ constexpr uint32_t make_idesc_pair(int nt) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(nt >> 3) << 17) |
+         ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ unsigned cluster_rank() {
+  unsigned r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\nbarrier.cluster.wait.acquire.aligned;\n" ::
+                   : "memory");
+}
+// Shared::cluster address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ unsigned map_to_rank(unsigned addr, unsigned rank) {
+  unsigned r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void mbar_arrive_remote(unsigned cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr)
+               : "memory");
+}
+// TMA loads of the pair: the destination is this CTA's shared memory, the
+// completion goes to the even CTA's barrier (peer bit cleared).
+constexpr unsigned kPeerBitMask = 0xFEFFFFFFu;
+__device__ __forceinline__ void tma_load_3d_pair(unsigned dst, const CUtensorMap *map, int c0, int c1,
+                                                 int c2, unsigned bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(bar & kPeerBitMask)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(unsigned dst, const CUtensorMap *map, int c0, int c1,
+                                                 unsigned bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar & kPeerBitMask)
+      : "memory");
+}
+// The A-collector qualifier: FILL keeps this MMA's A operand in the
+// collector buffer, LASTUSE takes A from there (the same descriptor) and frees
+// it, NONE reads A afresh.  Reusing A saves the tensor core one operand read.
+enum class ACol { NONE, FILL, LASTUSE };
+template <ACol C>
+__device__ __forceinline__ void mma_tf32_pair(unsigned tmem_d, uint64_t a, uint64_t b,
+                                              uint32_t idesc, unsigned acc) {
+  if constexpr (C == ACol::FILL)
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::tf32.collector::a::fill [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+  else if constexpr (C == ACol::LASTUSE)
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::tf32.collector::a::lastuse [%0], %1, %2, %3, p;\n}\n" ::
+            "r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+  else
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs once the MMAs issued so
+// far have completed.
+__device__ __forceinline__ void mma_commit_pair(unsigned bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n" ::"r"(bar),
+      "h"((unsigned short)3)
+      : "memory");
+}
 
 template <int NT>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_xlo,
                  const __grid_constant__ CUtensorMap tmap_whi,
                  const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ bias,
                  float *y, int Cin, int Cout, int K, int dil, int pad, int y_len, int y_pitch,
                  Epi ep, int *status) {
-  static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
-  constexpr uint32_t IDESC = make_idesc(NT);
-  constexpr unsigned STAGE_TX = 2 * TM_TILE + 2 * NT * BK * 4;
+  static_assert(NT % 32 == 0 && NT >= 32 && NT <= MAX_NT, "UMMA N for M = 256, halves of 16");
+  constexpr uint32_t IDESC = make_idesc_pair(NT);
+  constexpr unsigned W_TX_TAP = 2u * 2u * (NT / 2) * BK * 4;  // one tap: both CTAs, hi and lo
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + TM_OFF_BAR);
   __shared__ Ctl ctl;
-  // barriers: stage loaded (TMA) / stage consumed (MMA commit), per stage;
-  // run accumulated / run accumulator read, per TMEM accumulator
-  const unsigned bar_full = smem_u32(&bars[0]);
-  const unsigned bar_empty = smem_u32(&bars[TM_STAGES]);
-  const unsigned bar_run_full = smem_u32(&bars[2 * TM_STAGES]);
-  const unsigned bar_run_free = smem_u32(&bars[2 * TM_STAGES + 2]);
-  auto xhi_at = [&](int s) { return smem + s * TM_STAGE_BYTES; };
-  auto xlo_at = [&](int s) { return smem + s * TM_STAGE_BYTES + TM_TILE; };
-  auto whi_at = [&](int s) { return smem + s * TM_STAGE_BYTES + 2 * TM_TILE; };
-  auto wlo_at = [&](int s) { return smem + s * TM_STAGE_BYTES + 3 * TM_TILE; };
+  const unsigned rank = cluster_rank();
+  const bool leader = (rank == 0);
+  const int xrows = BM + (K - 1) * dil;  // rows of one x box
+  const int XP = tm_x_plane(xrows);
+  const int NW = tm_w_slots(xrows);
+  const unsigned X_TX = 2u * 2u * (unsigned)xrows * 128u;  // both CTAs, hi and lo
+  unsigned char *wbase = smem + 2 * TM_XSLOTS * XP;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + NW * TM_W_SLOT);
+  // barriers (the leader's full and run-free barriers serve the pair):
+  // x block loaded / consumed (TM_XSLOTS), weight chunk loaded / consumed
+  // (NW slots), run accumulated / run accumulator read (2)
+  const unsigned bar_xfull = smem_u32(&bars[0]);
+  const unsigned bar_xempty = smem_u32(&bars[TM_XSLOTS]);
+  const unsigned bar_wfull = smem_u32(&bars[2 * TM_XSLOTS]);
+  const unsigned bar_wempty = smem_u32(&bars[2 * TM_XSLOTS + TM_MAX_WSLOTS]);
+  const unsigned bar_run_full = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS]);
+  const unsigned bar_run_free = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2]);
+  // x slot s, plane (0 hi, 1 lo); weight slot s, tap t of the chunk, plane
+  auto x_at = [&](int slot, int plane) { return smem_u32(smem + (2 * slot + plane) * XP); };
+  auto w_at = [&](int slot, int tap, int plane) {
+    return smem_u32(wbase + slot * TM_W_SLOT + (2 * tap + plane) * TM_W_PLANE);
+  };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = blockIdx.x * BM;
+  const int t0 = (blockIdx.x >> 1) * (2 * BM) + (int)rank * BM;  // this CTA's rows
   const int o0 = blockIdx.y * NT;
   const int b = blockIdx.z;
-  const int n_cb = Cin / BK;  // 32-channel blocks per tap
-  const int n_chunks = K * n_cb;
-  const int n_runs = (n_chunks + RUN - 1) / RUN;
+  const int n_cb = Cin / BK;          // 32-channel blocks
+  const int n_tc = (K + 1) / 2;       // chunks per block: taps (0,1), (2,3), ...
+  const int n_chunks = n_cb * n_tc;
+  const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;
 
   if (threadIdx.x == 0) {
     ctl.abort = 0;
-    for (int s = 0; s < TM_STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 1);
+    for (int s = 0; s < TM_XSLOTS; ++s) {
+      mbar_init(bar_xfull + 8 * s, 1);
+      mbar_init(bar_xempty + 8 * s, 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar_run_full + 8 * s, 1);
-      mbar_init(bar_run_free + 8 * s, NCONV / 32);
+      mbar_init(bar_run_free + 8 * s, 2 * NCONV / 32);  // sum warps of both CTAs
+    }
+    for (int s = 0; s < NW; ++s) {
+      mbar_init(bar_wfull + 8 * s, 1);
+      mbar_init(bar_wempty + 8 * s, 1);
     }
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      smem_u32(&ctl.tmem)),
                  "n"(TMEM_COLS)
                  : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
   }
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before anyone signals them
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
   const unsigned tmem = ctl.tmem;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (warp == 2) {
+    // ---------------------------------------------------- TMA producer: x blocks
+    // (a thread of its own, so a block waiting for its slot never holds up
+    // the weight stream)
     if (lane == 0) {
-      for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % TM_STAGES, u = c / TM_STAGES;
-        // after an abort every wait returns at once, so all roles run to the end
-        if (u > 0) mbar_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 111);
-        const int j = c / n_cb, cb = c - j * n_cb;
-        const int xt = t0 - pad + j * dil;  // first input time of the box (may be < 0)
-        const unsigned fb = bar_full + 8 * s;
-        mbar_arrive_tx(fb, STAGE_TX);
-        asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(xhi_at(s))),
-            "l"(reinterpret_cast<uint64_t>(&tmap_xhi)), "r"(cb * BK), "r"(xt), "r"(b), "r"(fb)
-            : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3, %4}], [%5];\n" ::"r"(smem_u32(xlo_at(s))),
-            "l"(reinterpret_cast<uint64_t>(&tmap_xlo)), "r"(cb * BK), "r"(xt), "r"(b), "r"(fb)
-            : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(whi_at(s))),
-            "l"(reinterpret_cast<uint64_t>(&tmap_whi)), "r"(c * BK), "r"(o0), "r"(fb)
-            : "memory");
-        asm volatile(
-            "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
-            " [%0], [%1, {%2, %3}], [%4];\n" ::"r"(smem_u32(wlo_at(s))),
-            "l"(reinterpret_cast<uint64_t>(&tmap_wlo)), "r"(c * BK), "r"(o0), "r"(fb)
-            : "memory");
+      // after an abort every wait returns at once, so all roles run to the end
+      for (int cb = 0; cb < n_cb; ++cb) {
+        const int xs = cb % TM_XSLOTS, xu = cb / TM_XSLOTS;
+        if (xu > 0) mbar_wait(bar_xempty + 8 * xs, (xu - 1) & 1, &ctl, status, 111);
+        const unsigned fb = bar_xfull + 8 * xs;
+        if (leader) mbar_arrive_tx(fb, X_TX);
+        tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * BK, t0 - pad, b, fb);
+        tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * BK, t0 - pad, b, fb);
       }
-      // drain: the last loads must land before the CTA can exit
-      for (int c = n_chunks - TM_STAGES; c < n_chunks; ++c)
-        if (c >= 0) mbar_drain(bar_full + 8 * (c % TM_STAGES), (c / TM_STAGES) & 1);
+      if (leader)
+        for (int cb = n_cb - TM_XSLOTS; cb < n_cb; ++cb)
+          if (cb >= 0) mbar_drain(bar_xfull + 8 * (cb % TM_XSLOTS), (cb / TM_XSLOTS) & 1);
+    }
+  } else if (warp == 0) {
+    // ----------------------------------------------- TMA producer: weight chunks
+    if (lane == 0) {
+      const int row = o0 + (int)rank * (NT / 2);
+      int ws = 0, wphase = 0;
+      for (int cb = 0; cb < n_cb; ++cb) {
+        for (int q = 0; q < n_tc; ++q) {
+          if (cb * n_tc + q >= NW) mbar_wait(bar_wempty + 8 * ws, wphase ^ 1, &ctl, status, 112);
+          const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+          const unsigned fb = bar_wfull + 8 * ws;
+          if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
+          for (int t = 0; t < ntap; ++t) {
+            const int col = (j0 + t) * Cin + cb * BK;
+            tma_load_2d_pair(w_at(ws, t, 0), &tmap_whi, col, row, fb);
+            tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
+          }
+          if (++ws == NW) {
+            ws = 0;
+            wphase ^= 1;
+          }
+        }
+      }
+      // drain: the pair's last loads land before the leader can exit (the odd
+      // CTA's land before the leader's MMAs read them, which the final
+      // cluster barrier waits for)
+      if (leader)
+        for (int c = n_chunks - NW; c < n_chunks; ++c)
+          if (c >= 0) mbar_drain(bar_wfull + 8 * (c % NW), (c / NW) & 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      for (int c = 0; c < n_chunks; ++c) {
-        const int s = c % TM_STAGES, u = c / TM_STAGES;
-        const int r = c / RUN, ra = r & 1;
-        const bool first = (c % RUN) == 0;
-        const bool last = (c % RUN) == RUN - 1 || c == n_chunks - 1;
-        if (first && r >= 2)  // the sum warps have read this accumulator's run r - 2
-          mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 112);
-        mbar_wait(bar_full + 8 * s, u & 1, &ctl, status, 113);
-        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-        const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
-        const unsigned x_hi = smem_u32(xhi_at(s)), x_lo = smem_u32(xlo_at(s));
-        const unsigned w_hi = smem_u32(whi_at(s)), w_lo = smem_u32(wlo_at(s));
+    // ----------------------------------------------- MMA issuer (leader only)
+    if (leader && lane == 0) {
+      // descriptors are formed once per operand tile and advanced by adding
+      // the byte offset / 16 (the start-address field; shared addresses stay
+      // below 256 KB, so the field never carries)
+      int c = 0, ws = 0, wphase = 0;
+      for (int cb = 0; cb < n_cb; ++cb) {
+        const int xs = cb % TM_XSLOTS;
+        mbar_wait(bar_xfull + 8 * xs, (cb / TM_XSLOTS) & 1, &ctl, status, 113);
+        const uint64_t dxh = sw128_desc(x_at(xs, 0)), dxl = sw128_desc(x_at(xs, 1));
+        for (int q = 0; q < n_tc; ++q, ++c) {
+          const int r = c / TM_RUN, ra = r & 1;
+          const bool first = (c % TM_RUN) == 0;
+          const bool last = (c % TM_RUN) == TM_RUN - 1 || c == n_chunks - 1;
+          if (first && r >= 2)  // both CTAs' sum warps have read this accumulator's run r - 2
+            mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 114);
+          mbar_wait(bar_wfull + 8 * ws, wphase, &ctl, status, 115);
+          asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+          const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
+          const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+          for (int t = 0; t < ntap; ++t) {
+            const uint64_t rows = (uint64_t)((j0 + t) * dil * 8);  // tap's first row, in 16 B
+            const uint64_t ah = dxh + rows, al = dxl + rows;
+            const uint64_t bh = sw128_desc(w_at(ws, t, 0)), bl = sw128_desc(w_at(ws, t, 1));
 #pragma unroll
-        for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes per MMA
-          const unsigned off = 32 * k;
-          mma_tf32(acc, sw128_desc(x_lo + off), sw128_desc(w_hi + off), IDESC,
-                   (first && k == 0) ? 0u : 1u);
-          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_lo + off), IDESC, 1u);
-          mma_tf32(acc, sw128_desc(x_hi + off), sw128_desc(w_hi + off), IDESC, 1u);
+            for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes = 2 x 16 B per MMA
+              const uint64_t o = 2 * k;
+              // X_hi is the A operand of two products: read it once
+              mma_tf32_pair<ACol::FILL>(acc, ah + o, bh + o, IDESC,
+                                        (first && t == 0 && k == 0) ? 0u : 1u);
+              mma_tf32_pair<ACol::LASTUSE>(acc, ah + o, bl + o, IDESC, 1u);
+              mma_tf32_pair<ACol::NONE>(acc, al + o, bh + o, IDESC, 1u);
+            }
+          }
+          mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot
+          if (q == n_tc - 1) mma_commit_pair(bar_xempty + 8 * xs);  // and the x slot
+          if (last) mma_commit_pair(bar_run_full + 8 * ra);
+          if (++ws == NW) {
+            ws = 0;
+            wphase ^= 1;
+          }
         }
-        mma_commit(bar_empty + 8 * s);  // the stage may be refilled once these finish
-        if (last) mma_commit(bar_run_full + 8 * ra);
       }
     }
   } else if (warp >= CONV_WARP0) {
     // ------------------------------------------------------ run sums + output
     const int ct = threadIdx.x - CONV_WARP0 * 32;  // time row of this thread
     const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
+    const unsigned run_free_leader = map_to_rank(bar_run_free, 0);
     float sum[NT];
 #pragma unroll
     for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
     for (int p = 0; p < n_runs; ++p) {
       const int ra = p & 1;
-      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 114);
+      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 116);
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 #pragma unroll
       for (int c0 = 0; c0 < NT; c0 += 16) {
@@ -715,7 +889,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       }
       asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_run_free + 8 * ra);
+      if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
     }
     const int t = t0 + ct;
     if (!ctl.abort && t < y_len) {
@@ -732,16 +906,13 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  __syncthreads();
+  // every MMA of the pair has completed (each CTA's sum warps saw the last
+  // run) and every remote arrive has landed before either CTA frees TMEM or
+  // its shared memory
+  cluster_sync();
   if (warp == 1) {
-    // no MMA may still write an accumulator when it is freed
-    if (lane == 0 && n_runs > 0) {
-      mbar_drain(bar_run_full + 8 * ((n_runs - 1) & 1), ((n_runs - 1) >> 1) & 1);
-      if (n_runs > 1) mbar_drain(bar_run_full + 8 * ((n_runs - 2) & 1), ((n_runs - 2) >> 1) & 1);
-    }
-    __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
                  "n"(TMEM_COLS)
                  : "memory");
   }
@@ -759,20 +930,20 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
       return check_launch("conv1d_tm smem attribute");
     configured = true;
   }
-  dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B);
+  dim3 grid(2 * ((y_len + 2 * BM - 1) / (2 * BM)), (Cout + NT - 1) / NT, B);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tm: grid too large");
   conv1d_tm_kernel<NT><<<grid, THREADS, TM_SMEM_BYTES, st>>>(
       xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, device_status_ptr());
   return BV_OK;
 }
 
-// [B, T, C] fp32 plane as a 3-D tensor map, box 32 channels x 128 times.
-bv_status encode_x_tm(CUtensorMap *tmap, const float *x, int B, int C, int T) {
+// [B, T, C] fp32 plane as a 3-D tensor map, box 32 channels x `rows` times.
+bv_status encode_x_tm(CUtensorMap *tmap, const float *x, int B, int C, int T, int rows) {
   if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: input not 16-byte aligned");
   const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
   const cuuint64_t strides[2] = {(cuuint64_t)C * sizeof(float), (cuuint64_t)T * C * sizeof(float)};
-  const cuuint32_t box[3] = {BK, BM, 1};
+  const cuuint32_t box[3] = {BK, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -896,15 +1067,28 @@ __global__ void split_weights_kernel(SplitTable tab) {
     const bool vec = ((n & 3) == 0) && ((reinterpret_cast<uintptr_t>(src) & 15u) == 0) &&
                      ((reinterpret_cast<uintptr_t>(hi) & 15u) == 0);
     if (tab.cin[e] > 0) {
+      // one output row o at a time, 64 input channels per pass: the slice
+      // src[o][i0 .. i0 + 64)[0 .. k) is contiguous, and so is each tap's run
+      // dst[o][j cin + i0 .. + 64); shared memory turns one into the other
+      __shared__ float sl[64 * MAX_K];
       const int cin = tab.cin[e], k = tab.k[e];
       const long long row = (long long)cin * k;
-      for (long long d = i0; d < n; d += stride) {  // d = o row + j cin + i
-        const long long o = d / row;
-        const int rem = (int)(d - o * row);
-        const int j = rem / cin, i = rem - j * cin;
-        const float v = src[o * row + (long long)i * k + j], h = tf32_hi(v);
-        hi[d] = h;
-        lo[d] = v - h;
+      const long long rows = n / row;
+      for (long long o = blockIdx.x; o < rows; o += gridDim.x) {
+        for (int i0 = 0; i0 < cin; i0 += 64) {
+          const int ni = cin - i0 < 64 ? cin - i0 : 64;
+          const float *sp = src + o * row + (long long)i0 * k;
+          for (int q = threadIdx.x; q < ni * k; q += blockDim.x) sl[q] = sp[q];
+          __syncthreads();
+          for (int q = threadIdx.x; q < ni * k; q += blockDim.x) {
+            const int j = q / ni, ii = q - j * ni;
+            const float v = sl[ii * k + j], h = tf32_hi(v);
+            const long long d = o * row + (long long)j * cin + i0 + ii;
+            hi[d] = h;
+            lo[d] = v - h;
+          }
+          __syncthreads();
+        }
       }
     } else if (vec) {
       for (long long i = i0; i < n / 4; i += stride) {
@@ -975,7 +1159,7 @@ bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st) {
   for (int e = 0; e < tab.n; ++e) bytes += 12.0 * tab.count[e];
   {
     LaunchTimer tm(st, "weight_split", 0.0, bytes);
-    split_weights_kernel<<<dim3(32, tab.n), 256, 0, st>>>(tab);
+    split_weights_kernel<<<dim3(64, tab.n), 256, 0, st>>>(tab);
   }
   count_launch();
   return check_launch("split_weights_kernel");
@@ -1035,8 +1219,8 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
 
 
 bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
-  (void)dil;
-  return Cin % BK == 0 && Cout >= 40 && Cin * K >= 192 && encode_fn() != nullptr;
+  return Cin % BK == 0 && Cout >= 40 && Cin * K >= 192 && K >= 1 && K <= MAX_K && dil >= 1 &&
+         (K - 1) * dil <= TM_MAX_HALO && encode_fn() != nullptr;
 }
 
 bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
@@ -1046,13 +1230,13 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
   if (B <= 0 || y_len <= 0) return BV_OK;
   if (!conv1d_tm_supported(Cin, Cout, K, dil))
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
-  const int nt = pick_nt(Cout);
+  const int nt = pick_nt_pair(Cout);
   const int KK = Cin * K;
   CUtensorMap xh, xl, wh, wl;
-  BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T));
-  BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T));
-  BV_TRY(encode_w(&wh, w_split, Cout, KK, nt));
-  BV_TRY(encode_w(&wl, w_split + (size_t)Cout * KK, Cout, KK, nt));
+  BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T, BM + (K - 1) * dil));
+  BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T, BM + (K - 1) * dil));
+  BV_TRY(encode_w(&wh, w_split, Cout, KK, nt / 2));  // each CTA of a pair loads half the rows
+  BV_TRY(encode_w(&wl, w_split + (size_t)Cout * KK, Cout, KK, nt / 2));
   bv_status s;
   {
     const double outs = (double)B * Cout * y_len;
@@ -1064,11 +1248,8 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
     s = run_tm<N>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
     break;
     switch (nt) {
-      BV_TM_CASE(48)
       BV_TM_CASE(64)
-      BV_TM_CASE(80)
       BV_TM_CASE(96)
-      BV_TM_CASE(112)
       BV_TM_CASE(128)
       default:
         return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: tile %d", nt);
