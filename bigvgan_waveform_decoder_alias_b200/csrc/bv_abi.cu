@@ -506,8 +506,9 @@ void for_each_tc_conv(const bv_decoder_config *c, const bv_decoder_weights *w, F
 size_t split_ws(const bv_decoder_config *c) {
   size_t s = 0;
   for_each_tc_conv(c, nullptr,
-                   [&](int Cin, int Cout, int K, const float *, int, int, int, int, bool) {
-                     s += align_up(2 * (size_t)Cin * Cout * K * sizeof(float));
+                   [&](int Cin, int Cout, int K, const float *, int, int, int, int, bool tm) {
+                     s += align_up(2 * (size_t)(tm ? tm_cin_pad(Cin) : Cin) * Cout * K *
+                                   sizeof(float));
                    });
   return s;
 }
@@ -524,7 +525,7 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
     if (status != BV_OK) return;
     const long long count = (long long)Cin * Cout * K;
     float *dst = reinterpret_cast<float *>(ws + off);
-    off += align_up(2 * (size_t)count * sizeof(float));
+    off += align_up(2 * (size_t)(tm ? tm_cin_pad(Cin) : Cin) * Cout * K * sizeof(float));
     // an unaligned weight sends a [B, C, T] conv to the SIMT path: no split needed
     if (!tm && (reinterpret_cast<uintptr_t>(src) & 15u) != 0) return;
     if (kind == 0) {

@@ -56,6 +56,64 @@ struct Epi {
   int final_act;
 };
 
+// Grouped form for a thread that owns N outputs y[idx0 + e * stride]:
+// every value read (residual, the accumulated y) comes through the read-only
+// path and all N reads are issued before the N writes.  That is safe although
+// residual and y may be one buffer: each index is read once, by the thread
+// that then writes it, and what it reads was written by an earlier kernel.
+// (Plain loads would have to stay ordered after the previous group's stores
+// of the same buffer, and measured on B200 each then waited a full memory
+// round trip.)
+template <int N>
+__device__ __forceinline__ void epi_group(float *v, const float *bias_g, const Epi &e, float *y,
+                                          size_t idx0, size_t stride, int valid) {
+  if (!e.residual && !e.accumulate) {  // nothing to read: straight to the writes
+#pragma unroll
+    for (int q = 0; q < N; ++q) {
+      if (q < valid) {
+        float t = (v[q] + (bias_g ? __ldg(bias_g + q) : 0.0f)) * e.scale;
+        if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
+        else if (e.final_act == 2) t = tanhf(t);
+        y[idx0 + q * stride] = t;
+      }
+    }
+    return;
+  }
+  float r[N], a[N];
+#pragma unroll
+  for (int q = 0; q < N; ++q) {
+    r[q] = (e.residual && q < valid) ? __ldg(e.residual + idx0 + q * stride) : 0.0f;
+    a[q] = (e.accumulate && q < valid) ? __ldg(y + idx0 + q * stride) : 0.0f;
+  }
+#pragma unroll
+  for (int q = 0; q < N; ++q) {
+    if (q < valid) {
+      float t = (v[q] + (bias_g ? __ldg(bias_g + q) : 0.0f) + r[q]) * e.scale + a[q];
+      if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
+      else if (e.final_act == 2) t = tanhf(t);
+      y[idx0 + q * stride] = t;
+    }
+  }
+}
+
+// Two-phase form for a thread that owns many outputs: epi_load folds in
+// everything read from memory (bias, residual, the accumulated y) for all of
+// them before epi_store writes any, so the loads overlap instead of each one
+// waiting behind the previous store.  residual and y may be one buffer: every
+// index is read and then written by the same thread only.
+__device__ __forceinline__ float epi_load(float acc, float bias, const Epi &e, const float *yp,
+                                          size_t idx) {
+  float v = acc + bias;
+  if (e.residual) v += e.residual[idx];
+  v *= e.scale;
+  if (e.accumulate) v += yp[idx];
+  return v;
+}
+__device__ __forceinline__ float epi_final(float v, const Epi &e) {
+  if (e.final_act == 1) v = fminf(fmaxf(v, -1.0f), 1.0f);
+  else if (e.final_act == 2) v = tanhf(v);
+  return v;
+}
 __device__ __forceinline__ float apply_epilogue(float acc, float bias, const Epi &e,
                                                 const float *yp, size_t idx) {
   float v = acc + bias;
@@ -116,16 +174,20 @@ bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
 // Time-major tensor-core conv: x_hi / x_lo are [B, T, Cin] planes with
 // x = x_hi + x_lo, x_hi = tf32(x) (launch_transpose_split writes them);
 // w_split holds tf32(W') then W' - tf32(W') for the tap-major weight matrix
-// W'[o, j Cin + i] = w[o, i, j] (launch_split_weights with tap_major set).
+// W'[o, j Cp + i] = w[o, i, j], Cp = tm_cin_pad(Cin), zero for i >= Cin
+// (launch_split_weights with cin set).
 // Output and epilogue as launch_conv1d ([B, Cout, y_pitch]).
 bool conv1d_tm_supported(int Cin, int Cout, int K, int dil);
+// Channels per tap in the time-major conv's weight rows: Cin rounded up to
+// whole 32-channel blocks (the padding is zero).
+__host__ __device__ constexpr int tm_cin_pad(int cin) { return (cin + 31) / 32 * 32; }
 bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
                            const float *w_split, const float *bias, int Cout, int K, int dil,
                            int pad, const Epi &ep, float *y, int y_len, int y_pitch,
                            cudaStream_t st);
 
 // [B, C, T] -> time-major planes hi[b, t, c] = tf32(x[b, c, t]),
-// lo = x - hi (C a multiple of 32).
+// lo = x - hi.
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
                                  cudaStream_t st);
 

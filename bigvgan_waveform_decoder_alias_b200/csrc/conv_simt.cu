@@ -105,18 +105,36 @@ conv1d_simt_kernel(const float *__restrict__ x, const float *__restrict__ w,
     __syncthreads();
   }
 
-  // fused epilogue
+  // fused epilogue: all reads (bias, residual, accumulated y) first, then
+  // the writes, so the loads overlap
+  // (read-only path: each index is read once, by the thread that writes it)
 #pragma unroll
   for (int i = 0; i < TM; ++i) {
     const int o = m0 + ty * TM + i;
     if (o >= Cout) continue;
     const float bo = bias ? __ldg(bias + o) : 0.0f;
-    float *yrow = y + ((size_t)b * Cout + o) * y_pitch;
     const size_t rowoff = ((size_t)b * Cout + o) * y_pitch;
 #pragma unroll
     for (int q = 0; q < TN; ++q) {
       const int t = t0 + tx + q * Cfg::NTX;
-      if (t < y_len) yrow[t] = apply_epilogue(acc[i][q], bo, ep, y, rowoff + t);
+      if (t < y_len) {
+        float v = acc[i][q] + bo;
+        if (ep.residual) v += __ldg(ep.residual + rowoff + t);
+        v *= ep.scale;
+        if (ep.accumulate) v += __ldg(y + rowoff + t);
+        acc[i][q] = v;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int o = m0 + ty * TM + i;
+    if (o >= Cout) continue;
+    float *yrow = y + ((size_t)b * Cout + o) * y_pitch;
+#pragma unroll
+    for (int q = 0; q < TN; ++q) {
+      const int t = t0 + tx + q * Cfg::NTX;
+      if (t < y_len) yrow[t] = epi_final(acc[i][q], ep);
     }
   }
 }

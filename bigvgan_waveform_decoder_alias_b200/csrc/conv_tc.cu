@@ -466,15 +466,12 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
     const int t = t0 + ct;
     const int p = om.stride * t + om.offset + phase;
     if (!ctl.abort && t < y_len && p >= 0 && p < om.len) {
+      // 16 channels at a time: the group's reads, then its writes
+      const size_t base = (size_t)b * Cout * y_pitch + p;
 #pragma unroll
-      for (int e = 0; e < NT; ++e) {
-        const int o = o0 + e;
-        if (o < Cout) {
-          const size_t idx = ((size_t)b * Cout + o) * y_pitch + p;
-          const float bo = bias ? __ldg(bias + o) : 0.0f;
-          y[idx] = apply_epilogue(sum[e], bo, ep, y, idx);
-        }
-      }
+      for (int g = 0; g < NT; g += 16)
+        epi_group<16>(sum + g, bias ? bias + o0 + g : nullptr, ep, y,
+                      base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch, Cout - (o0 + g));
     }
   }
 
@@ -734,7 +731,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const int t0 = (blockIdx.x >> 1) * (2 * BM) + (int)rank * BM;  // this CTA's rows
   const int o0 = blockIdx.y * NT;
   const int b = blockIdx.z;
-  const int n_cb = Cin / BK;          // 32-channel blocks
+  const int n_cb = (Cin + BK - 1) / BK;  // 32-channel blocks (channels past Cin read as 0)
+  const int Cpad = n_cb * BK;            // weight row stride per tap
   const int n_tc = (K + 1) / 2;       // chunks per block: taps (0,1), (2,3), ...
   const int n_chunks = n_cb * n_tc;
   const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;
@@ -797,7 +795,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
           const unsigned fb = bar_wfull + 8 * ws;
           if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
           for (int t = 0; t < ntap; ++t) {
-            const int col = (j0 + t) * Cin + cb * BK;
+            const int col = (j0 + t) * Cpad + cb * BK;
             tma_load_2d_pair(w_at(ws, t, 0), &tmap_whi, col, row, fb);
             tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
           }
@@ -893,15 +891,12 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     }
     const int t = t0 + ct;
     if (!ctl.abort && t < y_len) {
+      // 16 channels at a time: the group's reads, then its writes
+      const size_t base = (size_t)b * Cout * y_pitch + t;
 #pragma unroll
-      for (int e = 0; e < NT; ++e) {
-        const int o = o0 + e;
-        if (o < Cout) {
-          const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
-          const float bo = bias ? __ldg(bias + o) : 0.0f;
-          y[idx] = apply_epilogue(sum[e], bo, ep, y, idx);
-        }
-      }
+      for (int g = 0; g < NT; g += 16)
+        epi_group<16>(sum + g, bias ? bias + o0 + g : nullptr, ep, y,
+                      base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch, Cout - (o0 + g));
     }
   }
 
@@ -1069,11 +1064,13 @@ __global__ void split_weights_kernel(SplitTable tab) {
     if (tab.cin[e] > 0) {
       // one output row o at a time, 64 input channels per pass: the slice
       // src[o][i0 .. i0 + 64)[0 .. k) is contiguous, and so is each tap's run
-      // dst[o][j cin + i0 .. + 64); shared memory turns one into the other
+      // dst[o][j cp + i0 .. + 64); shared memory turns one into the other.
+      // Rows are padded to cp = tm_cin_pad(cin) channels per tap with zeros.
       __shared__ float sl[64 * MAX_K];
-      const int cin = tab.cin[e], k = tab.k[e];
-      const long long row = (long long)cin * k;
+      const int cin = tab.cin[e], k = tab.k[e], cp = tm_cin_pad(cin);
+      const long long row = (long long)cin * k, drow = (long long)cp * k;
       const long long rows = n / row;
+      lo = hi + rows * drow;
       for (long long o = blockIdx.x; o < rows; o += gridDim.x) {
         for (int i0 = 0; i0 < cin; i0 += 64) {
           const int ni = cin - i0 < 64 ? cin - i0 : 64;
@@ -1083,11 +1080,17 @@ __global__ void split_weights_kernel(SplitTable tab) {
           for (int q = threadIdx.x; q < ni * k; q += blockDim.x) {
             const int j = q / ni, ii = q - j * ni;
             const float v = sl[ii * k + j], h = tf32_hi(v);
-            const long long d = o * row + (long long)j * cin + i0 + ii;
+            const long long d = o * drow + (long long)j * cp + i0 + ii;
             hi[d] = h;
             lo[d] = v - h;
           }
           __syncthreads();
+        }
+        for (int q = threadIdx.x; q < (cp - cin) * k; q += blockDim.x) {
+          const int j = q / (cp - cin), ii = cin + q - j * (cp - cin);
+          const long long d = o * drow + (long long)j * cp + ii;
+          hi[d] = 0.0f;
+          lo[d] = 0.0f;
         }
       }
     } else if (vec) {
@@ -1120,14 +1123,14 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__res
 #pragma unroll
   for (int r = ty; r < 32; r += 8) {
     const int t = t0 + tx;
-    tile[r][tx] = t < T ? __ldcs(xb + (size_t)(c0 + r) * T + t) : 0.0f;
+    tile[r][tx] = (t < T && c0 + r < C) ? __ldcs(xb + (size_t)(c0 + r) * T + t) : 0.0f;
   }
   __syncthreads();
   const size_t ob = (size_t)b * T * C;
 #pragma unroll
   for (int r = ty; r < 32; r += 8) {
     const int t = t0 + r;
-    if (t < T) {
+    if (t < T && c0 + tx < C) {
       const float v = tile[tx][r], h = tf32_hi(v);
       const size_t idx = ob + (size_t)t * C + c0 + tx;
       hi[idx] = h;
@@ -1141,8 +1144,7 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__res
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
                                  cudaStream_t st) {
   if (B <= 0 || T <= 0) return BV_OK;
-  if (C % 32 != 0) return fail(BV_ERR_SHAPE, "transpose_split: C %d not a multiple of 32", C);
-  dim3 grid((T + 31) / 32, C / 32, B);
+  dim3 grid((T + 31) / 32, (C + 31) / 32, B);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "transpose_split: grid");
   {
     LaunchTimer tm(st, "transpose_split", 0.0, 12.0 * B * C * T);
@@ -1219,7 +1221,10 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
 
 
 bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
-  return Cin % BK == 0 && Cout >= 40 && Cin * K >= 192 && K >= 1 && K <= MAX_K && dil >= 1 &&
+  // input rows of Cin floats must be 16-byte multiples (TMA strides); a
+  // partial last channel block costs padded tensor work, so at most a third
+  return Cin % 4 == 0 && 3 * tm_cin_pad(Cin) <= 4 * Cin && Cout >= 40 &&
+         tm_cin_pad(Cin) * K >= 192 && K >= 1 && K <= MAX_K && dil >= 1 &&
          (K - 1) * dil <= TM_MAX_HALO && encode_fn() != nullptr;
 }
 
@@ -1231,7 +1236,7 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
   if (!conv1d_tm_supported(Cin, Cout, K, dil))
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
   const int nt = pick_nt_pair(Cout);
-  const int KK = Cin * K;
+  const int KK = tm_cin_pad(Cin) * K;  // tap-major weight row, padded channels
   CUtensorMap xh, xl, wh, wl;
   BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T, BM + (K - 1) * dil));
   BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T, BM + (K - 1) * dil));
