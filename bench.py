@@ -197,6 +197,24 @@ def dist_init():
     return world, rank, local
 
 
+def max_over_ranks(value, world, device):
+    """The largest of every rank's `value` (each rank's device-timed total):
+    the job takes as long as its slowest replica."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, audio_seconds_per_step, ms_per_step):
+    """Whole-job audio-seconds per second: every replica decodes its own
+    workload in the (max-over-ranks) step time."""
+    return world * audio_seconds_per_step / (ms_per_step / 1000.0)
+
+
 def cpu_baseline(workload, frames, steps=1):
     """The oracle as it stands, single-threaded, on a bounded sample: one side
     of the workload's decoder on its first `frames` latent frames."""
@@ -305,14 +323,10 @@ def main():
     barrier()
     launches = native.launch_count() - n0
     step_ms = [a.elapsed_time(b) for a, b in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
     ms_per_step = total_ms / args.steps
     audio_per_step = w.audio_seconds()
-    value = world * audio_per_step / (ms_per_step / 1000.0)
+    value = job_throughput(world, audio_per_step, ms_per_step)
     y_check = y.detach().float()
     finite = bool(torch.isfinite(y_check).all().item())
 
@@ -332,12 +346,8 @@ def main():
         ev2[k][1].record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in ev2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = world * audio_per_step / (e2e_ms / args.steps / 1000.0)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev2), world, dev)
+    e2e_value = job_throughput(world, audio_per_step, e2e_ms / args.steps)
 
     # ----------------------------------------- per-kernel timing (roofline)
     import ctypes
