@@ -40,7 +40,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=synth.H3_10S.name, choices=sorted(synth.DECODER_WORKLOADS))
-    ap.add_argument("--cpu-sample-frames", type=int, default=12,
+    ap.add_argument("--cpu-sample-frames", type=int, default=40,
                     help="latent frames (one side) of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
@@ -113,11 +113,15 @@ def peaks():
             "source": "fallback"}
 
 
+# kernel classes that run 3xTF32 on the tensor cores
+TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc")
+
+
 def roofline_for(name, kd, pk):
     """Achieved vs peak for one kernel class; achieved = algorithmic work per
     launch / average launch time."""
     t = kd["avg_launch_ms"] / 1000.0
-    if name == "conv1d_tc":
+    if name in TENSOR_CLASSES:
         # useful FLOPs of the 3xTF32 conv; the tensor pipe issues 3 TF32 MMAs each
         peak = pk["bf16_sustained"] * TF32_PER_BF16 / 3.0
         ach = kd["flops"] / t / 1e12
@@ -377,7 +381,17 @@ def main():
         kernels[name]["roofline"] = r
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
     roof = dict(roofs[dom], kernel=dom) if dom else None
-    act = roofs.get("activation")
+    # the fused activation: algorithmic bytes / time
+    acts = [kernels[k] for k in ("activation",) if k in kernels]
+    act = None
+    if acts:
+        ms = sum(k["ms_per_step"] for k in acts)
+        by = sum(k["bytes"] * k["launches_per_step"] for k in acts)
+        gbs = by / (ms / 1000.0) / 1e9
+        act = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+               "frac": gbs / pk["hbm_gbs"], "traffic": None,
+               "peak_source": f"{pk['source']} hbm_gbs",
+               "kernels": [k for k in ("activation",) if k in kernels]}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -364,6 +364,47 @@ bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params
   return BV_OK;
 }
 
+// Split-weight bytes of an AMP block's time-major tensor-core convs (0 when
+// none qualifies): tf32 hi / lo of each tap-major [C, K, Cp] matrix.
+size_t amp_split_bytes(int C, const bv_amp_params &p) {
+  const int K = p.kernel_size;
+  size_t s = 0;
+  for (int u = 0; u < p.n_dilations; ++u) {
+    if (conv1d_tm_supported(C, C, K, p.dilation[u]))
+      s += align_up(2 * (size_t)tm_cin_pad(C) * C * K * sizeof(float));
+    if (conv1d_tm_supported(C, C, K, 1))
+      s += align_up(2 * (size_t)tm_cin_pad(C) * C * K * sizeof(float));
+  }
+  return s;
+}
+
+// Write the split weights of the block's time-major convs into ws (laid out
+// as amp_split_bytes counts them) and point `out` at them.
+bv_status split_amp_weights(int C, const bv_amp_params &p, char *ws, AmpSplit *out,
+                            cudaStream_t st) {
+  const int K = p.kernel_size;
+  SplitTable tab;
+  tab.n = 0;
+  size_t off = 0;
+  auto add = [&](const float *src, const float **slot, bool *tm) {
+    float *dst = reinterpret_cast<float *>(ws + off);
+    off += align_up(2 * (size_t)tm_cin_pad(C) * C * K * sizeof(float));
+    *slot = dst;
+    *tm = true;
+    tab.src[tab.n] = src;
+    tab.dst[tab.n] = dst;
+    tab.count[tab.n] = (long long)C * C * K;
+    tab.cin[tab.n] = C;
+    tab.k[tab.n] = K;
+    ++tab.n;
+  };
+  for (int u = 0; u < p.n_dilations; ++u) {
+    if (conv1d_tm_supported(C, C, K, p.dilation[u])) add(p.conv1_w[u], &out->conv1[u], &out->tm1[u]);
+    if (conv1d_tm_supported(C, C, K, 1)) add(p.conv2_w[u], &out->conv2[u], &out->tm2[u]);
+  }
+  return launch_split_weights(tab, st);
+}
+
 }  // namespace
 }  // namespace bv
 
@@ -372,6 +413,15 @@ extern "C" {
 size_t bv_amp_block_workspace_size(int B, int C, int T) {
   if (B < 1 || C < 1 || T < 1) return 0;
   return 3 * align_up((size_t)B * C * T * sizeof(float));
+}
+
+size_t bv_amp_block_workspace_size_tc(int B, int C, int T, const bv_amp_params *p) {
+  g_err[0] = 0;
+  if (B < 1 || C < 1 || T < 1 || check_amp_params(p, C) != BV_OK) return 0;
+  const size_t base = bv_amp_block_workspace_size(B, C, T);
+  const size_t split = bv::amp_split_bytes(C, *p);
+  if (split == 0) return base;
+  return base + 2 * bv::align_up((size_t)B * C * T * sizeof(float)) + split;
 }
 
 bv_status bv_amp_block(const float *x, int B, int C, int T, const bv_amp_params *p, float *y,
@@ -387,15 +437,27 @@ bv_status bv_amp_block(const float *x, int B, int C, int T, const bv_amp_params 
     return fail(BV_ERR_WORKSPACE, "bv_amp_block: workspace %zu bytes, need %zu", ws_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(BV_ERR_ARG, "bv_amp_block: workspace not 256-byte aligned");
-  const float *wsf = static_cast<const float *>(workspace);
-  if (overlaps(x, n, y, n) || overlaps(x, n, wsf, need / 4) || overlaps(y, n, wsf, need / 4))
-    return fail(BV_ERR_ARG, "bv_amp_block: x, y and workspace must be disjoint");
   BV_TRY(check_device());
-  char *w8 = static_cast<char *>(workspace);
   const size_t sz = align_up(n * sizeof(float));
+  const size_t split = amp_split_bytes(C, *p);
+  const bool tc = split > 0 && ws_bytes >= need + 2 * sz + split;  // time-major path fits
+  const size_t used = tc ? need + 2 * sz + split : need;
+  const float *wsf = static_cast<const float *>(workspace);
+  if (overlaps(x, n, y, n) || overlaps(x, n, wsf, used / 4) || overlaps(y, n, wsf, used / 4))
+    return fail(BV_ERR_ARG, "bv_amp_block: x, y and workspace must be disjoint");
+  char *w8 = static_cast<char *>(workspace);
   AmpScratch s{reinterpret_cast<float *>(w8), reinterpret_cast<float *>(w8 + sz),
                reinterpret_cast<float *>(w8 + 2 * sz)};
-  return run_amp_block(x, B, C, T, *p, y, scale, accumulate, s, as_stream(stream));
+  cudaStream_t st = as_stream(stream);
+  if (tc) {
+    // time-major tensor-core path: operand planes, then the split weights
+    s.xhi = reinterpret_cast<float *>(w8 + 3 * sz);
+    s.xlo = reinterpret_cast<float *>(w8 + 4 * sz);
+    AmpSplit sp{};
+    BV_TRY(split_amp_weights(C, *p, w8 + 5 * sz, &sp, st));
+    return run_amp_block(x, B, C, T, *p, y, scale, accumulate, s, st, &sp);
+  }
+  return run_amp_block(x, B, C, T, *p, y, scale, accumulate, s, st);
 }
 
 }  // extern "C"

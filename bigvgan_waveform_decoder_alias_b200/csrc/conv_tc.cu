@@ -1244,9 +1244,11 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
   BV_TRY(encode_w(&wl, w_split + (size_t)Cout * KK, Cout, KK, nt / 2));
   bv_status s;
   {
+    // algorithmic work: the useful products (Cin K per output), not the
+    // padded channel block or the three 3xTF32 terms
     const double outs = (double)B * Cout * y_len;
-    LaunchTimer tm(st, "conv1d_tc", 2.0 * outs * KK,
-                   4.0 * ((double)B * Cin * T + (double)Cout * KK +
+    LaunchTimer tm(st, "conv1d_tm", 2.0 * outs * Cin * K,
+                   4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                           outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
 #define BV_TM_CASE(N)                                                                          \
   case N:                                                                                      \

@@ -108,6 +108,8 @@ def lib():
                                       c_int, _fp, _fp]
     L.bv_amp_block_workspace_size.restype = c_size
     L.bv_amp_block_workspace_size.argtypes = [c_int, c_int, c_int]
+    L.bv_amp_block_workspace_size_tc.restype = c_size
+    L.bv_amp_block_workspace_size_tc.argtypes = [c_int, c_int, c_int, ctypes.POINTER(AmpParams)]
     L.bv_amp_block.argtypes = [_fp, c_int, c_int, c_int, ctypes.POINTER(AmpParams), _fp, c_float,
                                c_int, _fp, c_size, _fp]
     L.bv_amp_block_static.argtypes = [_fp, c_int, c_int, c_int, ctypes.POINTER(AmpParams), _fp,
@@ -259,11 +261,19 @@ def bv_amp_block_workspace_size(B, C, T) -> int:
     return int(lib().bv_amp_block_workspace_size(B, C, T))
 
 
+def bv_amp_block_workspace_size_tc(B, C, T, params: AmpParams) -> int:
+    return int(lib().bv_amp_block_workspace_size_tc(B, C, T, ctypes.byref(params)))
+
+
 def bv_amp_block(x, params: AmpParams, y=None, scale=1.0, accumulate=False, workspace=None,
-                 stream=None, keepalive=None):
+                 stream=None, keepalive=None, tensor_core=True):
+    """tensor_core: size a new workspace for the time-major tensor-core path
+    (taken by the block's qualifying convs); False keeps every conv on
+    [B, C, T] operands."""
     B, C, T = x.shape
     y = torch.empty_like(x) if y is None else y
-    need = bv_amp_block_workspace_size(B, C, T)
+    need = (bv_amp_block_workspace_size_tc(B, C, T, params) if tensor_core
+            else bv_amp_block_workspace_size(B, C, T))
     if workspace is None:
         workspace = torch.empty(need // 4 + 64, device=x.device, dtype=torch.float32)
     _check(lib().bv_amp_block(_ptr(x), B, C, T, ctypes.byref(params), _ptr(y), float(scale),

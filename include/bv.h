@@ -207,8 +207,19 @@ typedef struct {
 /* Workspace bytes bv_amp_block needs for [B, C, T]. */
 size_t bv_amp_block_workspace_size(int B, int C, int T);
 
-/* x, y [B, C, T] must not overlap each other or the workspace.  Errors:
- * BV_ERR_ARG, BV_ERR_SHAPE, BV_ERR_WORKSPACE. */
+/* Workspace bytes with which bv_amp_block runs the block's convs on the
+ * tensor cores from time-major operands (the path bv_decode takes): room for
+ * two [B, T, C] operand planes and the convs' weights split into tf32 hi / lo
+ * parts, besides the three [B, C, T] buffers.  Equals
+ * bv_amp_block_workspace_size when no conv of the block qualifies (narrow
+ * channel counts, or no tensor-core support); 0 for invalid arguments. */
+size_t bv_amp_block_workspace_size_tc(int B, int C, int T, const bv_amp_params *p);
+
+/* x, y [B, C, T] must not overlap each other or the workspace.  With a
+ * workspace of at least bv_amp_block_workspace_size_tc bytes the qualifying
+ * convs run time-major on the tensor cores; with at least
+ * bv_amp_block_workspace_size bytes all convs read [B, C, T] operands.
+ * Errors: BV_ERR_ARG, BV_ERR_SHAPE, BV_ERR_WORKSPACE. */
 bv_status bv_amp_block(const float *x, int B, int C, int T,
                        const bv_amp_params *p, float *y, float scale,
                        int accumulate, void *workspace, size_t ws_bytes,

@@ -371,16 +371,29 @@ def test_amp_block_workload_matches_oracle(nat, oracle, filt):
     assert rel_l2(y, want) < LAYER_TOL
 
 
-@pytest.mark.parametrize("C,T,K,dils", [(12, 3001, 11, (1, 3, 5)), (96, 517, 7, (1, 3, 5)),
-                                        (130, 64, 3, (2,)), (16, 5, 7, (1, 3, 5, 7))])
-def test_amp_block_shapes(nat, oracle, filt, C, T, K, dils):
+# (C, T, K, dilations, whether the time-major tensor-core conv qualifies)
+AMP_SHAPES = [(12, 3001, 11, (1, 3, 5), False), (96, 517, 7, (1, 3, 5), True),
+              (130, 64, 3, (2,), False), (16, 5, 7, (1, 3, 5, 7), False),
+              (128, 2001, 11, (1, 3, 5), True), (48, 1003, 7, (1, 3, 5), True),
+              (64, 300, 3, (1, 3, 5), True), (256, 130, 11, (5,), True)]
+
+
+@pytest.mark.parametrize("tensor_core", [False, True])
+@pytest.mark.parametrize("C,T,K,dils,tm", AMP_SHAPES)
+def test_amp_block_shapes(nat, oracle, filt, C, T, K, dils, tm, tensor_core):
+    """The AMP block (scale 0.5 accumulated onto y) against the oracle, with
+    its convs on [B, C, T] operands or, given the larger workspace, time-major
+    on the tensor cores (48 channels: a zero-padded channel block)."""
     wl = synth.AmpWorkload("t", 2, C, T, K, dils, seed=C + T)
     x, flat = wl.make()
     tens = _amp_tensors(wl.layout(), flat)
     p = nat.amp_params(K, dils, tens, filt)
     y0 = synth.NormalStream(5).normal((2, C, T))
     yd = dev(y0)
-    nat.bv_amp_block(dev(x), p, y=yd, scale=0.5, accumulate=True)
+    classes = _kernel_classes(nat, lambda: nat.bv_amp_block(dev(x), p, y=yd, scale=0.5,
+                                                            accumulate=True,
+                                                            tensor_core=tensor_core))
+    assert ("conv1d_tm" in classes) == (tm and tensor_core), classes
     want = 0.5 * oracle.amp_block(x, flat, K, dils).astype(np.float64) + y0
     assert rel_l2(host(yd), want) < LAYER_TOL
 
@@ -424,8 +437,9 @@ def test_real_geometry_short_latent(nat, oracle, filt, wname, frames):
 @pytest.mark.parametrize("frames", [1, 2, 5, 27])
 def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     """A decoder wide enough that its ConvT stages (both stride parities) and
-    its AMP convs take the tensor-core paths (time-major input at 128 and 96
-    channels, [B, C, T] input at 48), on short and ragged latents."""
+    its AMP convs take the time-major tensor-core path (128, 96 and 48
+    channels, the last with a zero-padded channel block), on short and ragged
+    latents."""
     geo = synth.tiny_geometry(pre_channels=256, up_channels=(128, 96, 48), in_channels=16)
     s = synth.NormalStream(40 + frames)
     z = s.normal((2, geo.in_channels, frames))
@@ -434,8 +448,9 @@ def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     zd = dev(z)
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault("y", dec.decode(zd)))
-    assert "conv_transpose1d_tc" in classes and "conv1d_tc" in classes, classes
-    assert "transpose_split" in classes, classes  # the 128/96-channel AMP convs run time-major
+    assert "conv_transpose1d_tc" in classes, classes
+    # the 128/96/48-channel AMP convs run time-major
+    assert "conv1d_tm" in classes and "transpose_split" in classes, classes
     want = oracle.decode(geo, params, z)
     assert rel_l2(host(out["y"]), want) < WAVE_TOL
 
