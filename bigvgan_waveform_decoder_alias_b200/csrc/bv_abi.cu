@@ -617,8 +617,43 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
 
 // A, S, cur, h1, h2 in [B, C, T] and the two time-major planes, then the
 // repacked transposed-conv weights.
+// Buffers of one untiled decode, each max B C T floats: A (stage output) and S
+// (ConvT output); per AMP block its scratch (cur, h1, h2 and the two
+// time-major planes); for blocks 1.. their own outputs, summed into A.
+int core_planes(const bv_decoder_config *c) { return 2 + 5 * c->n_blocks + (c->n_blocks - 1); }
+
 size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
-  return 7 * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
+  return core_planes(c) * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
+}
+
+// Streams on which the AMP blocks of a stage run side by side (one per block),
+// created once per device and kept until exit, with the events that fork them
+// from and join them back to the caller's stream.
+struct AuxStreams {
+  cudaStream_t s[BV_MAX_BLOCKS];
+  cudaEvent_t fork, join[BV_MAX_BLOCKS];
+  bool ok = false;
+};
+
+AuxStreams *aux_streams() {
+  static AuxStreams per_dev[32];
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 32) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  AuxStreams &a = per_dev[dev];
+  if (!a.ok) {
+    bool good = cudaEventCreateWithFlags(&a.fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int j = 0; j < BV_MAX_BLOCKS && good; ++j)
+      good = cudaStreamCreateWithFlags(&a.s[j], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&a.join[j], cudaEventDisableTiming) == cudaSuccess;
+    if (!good) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    a.ok = true;
+  }
+  return &a;
 }
 
 struct TilePlan {
@@ -692,12 +727,26 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
                       const DecoderSplit &sw, const float *z, int B, int F, float *y, char *ws,
                       cudaStream_t st) {
   const size_t sz = align_up((size_t)max_elems(c, B, F) * sizeof(float));
-  float *A = reinterpret_cast<float *>(ws);
-  float *S = reinterpret_cast<float *>(ws + sz);
-  AmpScratch s{reinterpret_cast<float *>(ws + 2 * sz), reinterpret_cast<float *>(ws + 3 * sz),
-               reinterpret_cast<float *>(ws + 4 * sz), reinterpret_cast<float *>(ws + 5 * sz),
-               reinterpret_cast<float *>(ws + 6 * sz)};
-  float *WP = reinterpret_cast<float *>(ws + 7 * sz);  // repacked ConvT weights
+  auto plane = [&](int k) { return reinterpret_cast<float *>(ws + (size_t)k * sz); };
+  float *A = plane(0);
+  float *S = plane(1);
+  const int nb = c->n_blocks;
+  AmpScratch sb[BV_MAX_BLOCKS];
+  float *Ab[BV_MAX_BLOCKS];  // block j's output (block 0 writes A)
+  for (int j = 0; j < nb; ++j) {
+    const int k = 2 + 5 * j;
+    sb[j] = AmpScratch{plane(k), plane(k + 1), plane(k + 2), plane(k + 3), plane(k + 4)};
+    Ab[j] = j == 0 ? A : plane(2 + 5 * nb + (j - 1));
+  }
+  const AmpScratch &s = sb[0];
+  float *WP = plane(core_planes(c));  // repacked ConvT weights
+  // The blocks of a stage are independent until their mean: they run side by
+  // side on one stream each and their outputs are summed in block order
+  // (bit-identical to accumulating them one after the other).  With the
+  // library's per-kernel timers on they run in order on the caller's stream,
+  // so that every launch's event time is its own.
+  AuxStreams *aux = (nb > 1 && !g_timing_on.load(std::memory_order_relaxed)) ? aux_streams()
+                                                                              : nullptr;
   int C = c->pre_channels, n = F;
   Epi plain{nullptr, 1.0f, 0, 0};
   BV_TRY(launch_conv1d(z, B, c->in_channels, F, w->pre_w, w->pre_b, C, c->pre_kernel, 1,
@@ -713,9 +762,24 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
       BV_TRY(launch_conv_transpose1d(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S, st));
     C = Co;
     n = n2;
-    const float scale = 1.0f / (float)c->n_blocks;
-    for (int j = 0; j < c->n_blocks; ++j)
-      BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], A, scale, j > 0, s, st, &sw.amp[i][j]));
+    const float scale = 1.0f / (float)nb;
+    if (aux) {
+      CUDA_TRY(cudaEventRecord(aux->fork, st));
+      for (int j = 0; j < nb; ++j) CUDA_TRY(cudaStreamWaitEvent(aux->s[j], aux->fork, 0));
+      for (int j = 0; j < nb; ++j)
+        BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], Ab[j], scale, 0, sb[j], aux->s[j],
+                             &sw.amp[i][j]));
+      for (int j = 0; j < nb; ++j) {
+        CUDA_TRY(cudaEventRecord(aux->join[j], aux->s[j]));
+        CUDA_TRY(cudaStreamWaitEvent(st, aux->join[j], 0));
+      }
+      Parts parts{nb - 1, {}};
+      for (int j = 1; j < nb; ++j) parts.p[j - 1] = Ab[j];
+      BV_TRY(launch_add_parts(A, parts, (long long)B * C * n, st));
+    } else {
+      for (int j = 0; j < nb; ++j)
+        BV_TRY(run_amp_block(S, B, C, n, w->amp[i][j], A, scale, j > 0, s, st, &sw.amp[i][j]));
+    }
   }
   BV_TRY(launch_activation(A, s.h1, B, C, n, w->post_log_alpha, w->post_log_beta, w->up_filter,
                            w->down_filter, 1e-9f, st));

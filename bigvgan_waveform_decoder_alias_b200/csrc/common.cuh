@@ -148,6 +148,11 @@ bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, c
     bv_status _s = (expr);      \
     if (_s != BV_OK) return _s; \
   } while (0)
+#define CUDA_TRY(expr)                                                               \
+  do {                                                                               \
+    cudaError_t _e = (expr);                                                         \
+    if (_e != cudaSuccess) return fail(BV_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(_e)); \
+  } while (0)
 
 // w_split: tf32(W) followed by W - tf32(W), each in w's layout (written by
 // launch_split_weights), or nullptr, in which case the kernel splits w itself.
@@ -170,6 +175,14 @@ struct SplitTable {
   int cin[kMaxSplit], k[kMaxSplit];
 };
 bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
+
+// acc += parts[0] + parts[1] + ... (n floats each), added in that order.
+constexpr int kMaxParts = 3;
+struct Parts {
+  int n;
+  const float *p[kMaxParts];
+};
+bv_status launch_add_parts(float *acc, const Parts &parts, long long n, cudaStream_t st);
 
 // Time-major tensor-core conv: x_hi / x_lo are [B, T, Cin] planes with
 // x = x_hi + x_lo, x_hi = tf32(x) (launch_transpose_split writes them);

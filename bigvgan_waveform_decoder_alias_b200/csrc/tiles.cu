@@ -58,7 +58,30 @@ __global__ void stitch_tiles_kernel(TileGroups g, float *__restrict__ y, int B, 
   }
 }
 
+// acc[i] = ((acc[i] + p[0][i]) + p[1][i]) + ... in that order
+__global__ void add_parts_kernel(float *__restrict__ acc, Parts parts, long long n) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n; i += stride) {
+    float v = acc[i];
+    for (int q = 0; q < parts.n; ++q) v += __ldg(parts.p[q] + i);
+    acc[i] = v;
+  }
+}
+
 }  // namespace
+
+bv_status launch_add_parts(float *acc, const Parts &parts, long long n, cudaStream_t st) {
+  if (n <= 0 || parts.n <= 0) return BV_OK;
+  const int threads = 256;
+  const long long blocks = (n + threads - 1) / threads;
+  {
+    LaunchTimer tm(st, "stage_sum", 0.0, 4.0 * (double)n * (parts.n + 2));
+    add_parts_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), threads, 0, st>>>(
+        acc, parts, n);
+  }
+  count_launch();
+  return check_launch("add_parts_kernel");
+}
 
 bv_status launch_gather_tiles(const float *z, float *zt, int B, int C, int frames, int step,
                               int len, int k0, int n_tiles, cudaStream_t st) {
