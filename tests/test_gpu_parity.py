@@ -375,7 +375,8 @@ def test_amp_block_workload_matches_oracle(nat, oracle, filt):
 AMP_SHAPES = [(12, 3001, 11, (1, 3, 5), False), (96, 517, 7, (1, 3, 5), True),
               (130, 64, 3, (2,), False), (16, 5, 7, (1, 3, 5, 7), False),
               (128, 2001, 11, (1, 3, 5), True), (48, 1003, 7, (1, 3, 5), True),
-              (64, 300, 3, (1, 3, 5), True), (256, 130, 11, (5,), True)]
+              (64, 300, 3, (1, 3, 5), True), (256, 130, 11, (5,), True),
+              (24, 700, 11, (1, 3, 5), False)]
 
 
 @pytest.mark.parametrize("tensor_core", [False, True])
