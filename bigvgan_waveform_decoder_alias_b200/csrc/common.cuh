@@ -56,39 +56,34 @@ struct Epi {
   int final_act;
 };
 
-// Grouped form for a thread that owns N outputs y[idx0 + e * stride]:
-// every value read (residual, the accumulated y) comes through the read-only
-// path and all N reads are issued before the N writes.  That is safe although
-// residual and y may be one buffer: each index is read once, by the thread
-// that then writes it, and what it reads was written by an earlier kernel.
-// (Plain loads would have to stay ordered after the previous group's stores
-// of the same buffer, and measured on B200 each then waited a full memory
-// round trip.)
+// Grouped form for a thread that owns N outputs y[idx0 + e * stride]: the
+// caller passes the group's biases already in registers (from shared memory),
+// every value read from global memory (residual, the accumulated y) comes
+// through the read-only path, and all N reads are issued before the N
+// writes.  That is safe although residual and y may be one buffer: each index
+// is read once, by the thread that then writes it, and what it reads was
+// written by an earlier kernel.  (Measured on B200: a global load issued
+// between stores to y -- a plain load, or even a read-only bias load -- waited
+// a full memory round trip each, which made the output loop of a tensor-core
+// conv tile several times longer than its stores.)
 template <int N>
-__device__ __forceinline__ void epi_group(float *v, const float *bias_g, const Epi &e, float *y,
-                                          size_t idx0, size_t stride, int valid) {
-  if (!e.residual && !e.accumulate) {  // nothing to read: straight to the writes
+__device__ __forceinline__ void epi_group(float *v, const float (&bias)[N], const Epi &e,
+                                          float *y, size_t idx0, size_t stride, int valid) {
+  float r[N], a[N];
+  if (e.residual || e.accumulate) {
 #pragma unroll
     for (int q = 0; q < N; ++q) {
-      if (q < valid) {
-        float t = (v[q] + (bias_g ? __ldg(bias_g + q) : 0.0f)) * e.scale;
-        if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
-        else if (e.final_act == 2) t = tanhf(t);
-        y[idx0 + q * stride] = t;
-      }
+      r[q] = (e.residual && q < valid) ? __ldg(e.residual + idx0 + q * stride) : 0.0f;
+      a[q] = (e.accumulate && q < valid) ? __ldg(y + idx0 + q * stride) : 0.0f;
     }
-    return;
-  }
-  float r[N], a[N];
+  } else {
 #pragma unroll
-  for (int q = 0; q < N; ++q) {
-    r[q] = (e.residual && q < valid) ? __ldg(e.residual + idx0 + q * stride) : 0.0f;
-    a[q] = (e.accumulate && q < valid) ? __ldg(y + idx0 + q * stride) : 0.0f;
+    for (int q = 0; q < N; ++q) r[q] = a[q] = 0.0f;
   }
 #pragma unroll
   for (int q = 0; q < N; ++q) {
     if (q < valid) {
-      float t = (v[q] + (bias_g ? __ldg(bias_g + q) : 0.0f) + r[q]) * e.scale + a[q];
+      float t = (v[q] + bias[q] + r[q]) * e.scale + a[q];
       if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
       else if (e.final_act == 2) t = tanhf(t);
       y[idx0 + q * stride] = t;

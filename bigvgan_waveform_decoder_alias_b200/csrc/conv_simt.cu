@@ -107,12 +107,19 @@ conv1d_simt_kernel(const float *__restrict__ x, const float *__restrict__ w,
 
   // fused epilogue: all reads (bias, residual, accumulated y) first, then
   // the writes, so the loads overlap
-  // (read-only path: each index is read once, by the thread that writes it)
+  // (read-only path: each index is read once, by the thread that writes it;
+  // the biases are read before any write too)
+  float bos[TM];
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int o = m0 + ty * TM + i;
+    bos[i] = (bias && o < Cout) ? __ldg(bias + o) : 0.0f;
+  }
 #pragma unroll
   for (int i = 0; i < TM; ++i) {
     const int o = m0 + ty * TM + i;
     if (o >= Cout) continue;
-    const float bo = bias ? __ldg(bias + o) : 0.0f;
+    const float bo = bos[i];
     const size_t rowoff = ((size_t)b * Cout + o) * y_pitch;
 #pragma unroll
     for (int q = 0; q < TN; ++q) {

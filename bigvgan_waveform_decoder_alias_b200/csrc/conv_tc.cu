@@ -74,7 +74,7 @@ constexpr int X_BYTES = 2 * CB * XW * 4;
 constexpr int OFF_BAR = OFF_X + X_BYTES;                 // mbarriers
 constexpr int SMEM_USED = OFF_BAR + 16 * 8;
 constexpr int SMEM_BYTES = SMEM_USED + 1024;             // room to align the base
-static_assert(SMEM_BYTES + 4 * 1024 + 64 <= 227 * 1024, "shared memory budget");
+static_assert(SMEM_BYTES + 4 * 1024 + 1024 <= 227 * 1024, "shared memory budget");
 
 __device__ __forceinline__ unsigned smem_u32(const void *p) {
   return (unsigned)__cvta_generic_to_shared(p);
@@ -208,6 +208,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + OFF_BAR);
   __shared__ Ctl ctl;
+  __shared__ float bias_s[MAX_NT];  // this tile's biases (0 past Cout or without bias)
   __shared__ __align__(16) int xoff[MAX_K * BK];  // im2col offsets of chunk m of a block
   using WL = WLayout<PRESPLIT>;
   constexpr int NWRING = PRESPLIT ? NWSLOT : NRAW;  // weight TMA ring slots
@@ -261,6 +262,8 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
   }
+  for (int i = threadIdx.x; i < MAX_NT; i += THREADS)
+    bias_s[i] = (bias && o0 + i < Cout) ? bias[o0 + i] : 0.0f;
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   __syncthreads();
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -469,9 +472,13 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
       // 16 channels at a time: the group's reads, then its writes
       const size_t base = (size_t)b * Cout * y_pitch + p;
 #pragma unroll
-      for (int g = 0; g < NT; g += 16)
-        epi_group<16>(sum + g, bias ? bias + o0 + g : nullptr, ep, y,
-                      base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch, Cout - (o0 + g));
+      for (int g = 0; g < NT; g += 16) {
+        float bb[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) bb[q] = bias_s[g + q];
+        epi_group<16>(sum + g, bb, ep, y, base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch,
+                      Cout - (o0 + g));
+      }
     }
   }
 
@@ -591,7 +598,7 @@ constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barrier
 constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
 constexpr int TM_XSLOTS = 2;                          // x blocks in flight
 constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 + 2;
-static_assert(TM_SMEM_BYTES + 64 <= 227 * 1024, "shared memory budget");
+static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
 __host__ __device__ constexpr int tm_x_plane(int rows) { return (rows * 128 + 1023) / 1024 * 1024; }
@@ -704,6 +711,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ Ctl ctl;
+  __shared__ float bias_s[MAX_NT];  // this tile's biases (0 past Cout or without bias)
   const unsigned rank = cluster_rank();
   const bool leader = (rank == 0);
   const int xrows = BM + (K - 1) * dil;  // rows of one x box
@@ -760,6 +768,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
   }
+  for (int i = threadIdx.x; i < MAX_NT; i += THREADS)
+    bias_s[i] = (bias && o0 + i < Cout) ? bias[o0 + i] : 0.0f;
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   cluster_sync();  // both CTAs' barriers exist before anyone signals them
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -894,9 +904,13 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       // 16 channels at a time: the group's reads, then its writes
       const size_t base = (size_t)b * Cout * y_pitch + t;
 #pragma unroll
-      for (int g = 0; g < NT; g += 16)
-        epi_group<16>(sum + g, bias ? bias + o0 + g : nullptr, ep, y,
-                      base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch, Cout - (o0 + g));
+      for (int g = 0; g < NT; g += 16) {
+        float bb[16];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) bb[q] = bias_s[g + q];
+        epi_group<16>(sum + g, bb, ep, y, base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch,
+                      Cout - (o0 + g));
+      }
     }
   }
 
