@@ -116,6 +116,12 @@ def peaks():
 # kernel classes that run 3xTF32 on the tensor cores
 TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc")
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of a full decode of the bench workload, per kernel class, for the
+# kernel code as committed with it (profiles/conv1d_tm_traffic_h3_10s.md);
+# a class missing here reports null.
+NCU_TRAFFIC_PER_LAUNCH = {"conv1d_tm": 84.1e6}
+
 
 def roofline_for(name, kd, pk):
     """Achieved vs peak for one kernel class; achieved = algorithmic work per
@@ -126,7 +132,7 @@ def roofline_for(name, kd, pk):
         peak = pk["bf16_sustained"] * TF32_PER_BF16 / 3.0
         ach = kd["flops"] / t / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
                 "peak_source": f"{pk['source']} bf16 sustained {pk['bf16_sustained']} TFLOP/s x "
                                f"tf32/bf16 {TF32_PER_BF16:.3f} / 3 (3xTF32)"}
     if kd["flops"] > 0:
