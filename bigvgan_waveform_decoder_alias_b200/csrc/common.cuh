@@ -171,6 +171,13 @@ struct SplitTable {
 };
 bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
 
+// Narrow conv on the FP32 pipe (at most 32 input and output channels, at
+// least 4 output channels); arguments as launch_conv1d.
+bool conv1d_small_supported(int Cin, int Cout, int K, int dil);
+bv_status launch_conv1d_small(const float *x, int B, int Cin, int T, const float *w,
+                              const float *bias, int Cout, int K, int dil, int pad,
+                              const Epi &ep, float *y, int y_len, int y_pitch, cudaStream_t st);
+
 // acc += parts[0] + parts[1] + ... (n floats each), added in that order.
 constexpr int kMaxParts = 3;
 struct Parts {

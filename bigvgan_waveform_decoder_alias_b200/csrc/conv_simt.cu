@@ -185,6 +185,9 @@ bv_status launch_conv1d(const float *x, int B, int Cin, int T, const float *w, c
       (reinterpret_cast<uintptr_t>(w_split) & 15u) == 0)
     return launch_conv1d_tc(x, B, Cin, T, w, w_split, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch,
                             st);
+  if (conv1d_small_supported(Cin, Cout, K, dil))
+    return launch_conv1d_small(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch,
+                               st);
   if (Cout >= 96)
     return run_conv<128, 128, 8, 8, 8>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len,
                                        y_pitch, st);

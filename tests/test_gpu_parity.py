@@ -166,11 +166,14 @@ def test_conv1d_unpadded_no_bias(nat, oracle):
     assert y.shape == (1, 30, 88) and rel_l2(y, want) < LAYER_TOL
 
 
+@pytest.mark.parametrize("C", [48, 24, 13])
 @pytest.mark.parametrize("final_act", [0, 1, 2])
-def test_conv1d_epilogue(nat, oracle, final_act):
-    """y = final(scale * (conv + bias + residual) + y_old)."""
-    s = synth.NormalStream(50 + final_act)
-    C, T = 48, 700
+def test_conv1d_epilogue(nat, oracle, final_act, C):
+    """y = final(scale * (conv + bias + residual) + y_old), on the tensor-core
+    path (48 channels) and the narrow FP32 kernel (24; 13 with an odd row
+    pitch and a partial channel group)."""
+    s = synth.NormalStream(50 + final_act + C)
+    T = 700 + C % 2
     x = s.normal((2, C, T))
     w = s.normal((C, C, 7), 0.0, 0.1)
     b = s.normal((C,), 0.0, 0.1)
@@ -189,9 +192,10 @@ def test_conv1d_epilogue(nat, oracle, final_act):
     assert rel_l2(got, want) < LAYER_TOL
 
 
-def test_conv1d_inplace_residual(nat, oracle):
-    s = synth.NormalStream(77)
-    C, T = 96, 513
+@pytest.mark.parametrize("C", [96, 24])
+def test_conv1d_inplace_residual(nat, oracle, C):
+    s = synth.NormalStream(77 + C)
+    T = 513
     x = s.normal((1, C, T))
     w = s.normal((C, C, 3), 0.0, 0.05)
     cur = s.normal((1, C, T))
