@@ -20,6 +20,8 @@
 // positions half a tile apart at once, with packed f32x2 arithmetic (FFMA2):
 // both positions have the same polyphase taps, so every filter tap and every
 // step of the sin^2 evaluation is one paired instruction.
+#include <type_traits>
+
 #include "common.cuh"
 #include "sin2.cuh"
 
@@ -50,10 +52,12 @@ __device__ __forceinline__ float snake1(float u, float a, float inv_b) {
 // Paired SnakeBeta: u + sin^2(a u) inv_b for two values, with the sin^2 of
 // sin2.cuh (reduction by pi in three parts, Taylor series of sin to r^13).
 // The nearest integer to z/pi comes from adding and removing 1.5 * 2^23.
+// CHECK = false when the caller has bounded |a u| by the fast-path limit.
+template <bool CHECK = true>
 __device__ __forceinline__ float2 snake2(float2 u, float a, float inv_b) {
   using namespace sin2c;
   const float2 z = mul2(u, f2(a));
-  if (fmaxf(fabsf(z.x), fabsf(z.y)) > kFastLimit)
+  if (CHECK && fmaxf(fabsf(z.x), fabsf(z.y)) > kFastLimit)
     return make_float2(snake1(u.x, a, inv_b), snake1(u.y, a, inv_b));
   const float2 k = add2(fma2(z, f2(kInvPi), f2(12582912.0f)), f2(-12582912.0f));
   float2 r = fma2(k, f2(-kC1), z);
@@ -77,12 +81,17 @@ struct Taps {
 
 // u at phase r (0: even index, 1: odd) from six consecutive x values
 // xp[0..5] = x[p + r - 3 .. p + r + 2]:  u[2p+r] = sum_l 2 f[2l+1-r] x[p+2+r-l],
-// where term l pairs with xp[5-l].
-__device__ __forceinline__ float up1(const Taps &tp, int r, const float *xp) {
-  float u = tp.up2[1 - r] * xp[5];
+// where term l pairs with xp[5-l].  (The phase is a template argument so the
+// taps are indexed statically and stay in registers.)
+template <int R>
+__device__ __forceinline__ float up1r(const Taps &tp, const float *xp) {
+  float u = tp.up2[1 - R] * xp[5];
 #pragma unroll
-  for (int l = 1; l < 6; ++l) u = fmaf(tp.up2[2 * l + 1 - r], xp[5 - l], u);
+  for (int l = 1; l < 6; ++l) u = fmaf(tp.up2[2 * l + 1 - R], xp[5 - l], u);
   return u;
+}
+__device__ __forceinline__ float up1(const Taps &tp, int r, const float *xp) {
+  return r ? up1r<1>(tp, xp) : up1r<0>(tp, xp);
 }
 
 __device__ __forceinline__ void cp_async4(float *dst, const float *src) {
@@ -146,6 +155,21 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
     tp.up2[j] = 2.0f * __ldg(f_up + j);
     tp.dn[j] = __ldg(f_dn + j);
   }
+  // the taps as broadcast pairs, formed once for every tile
+  float2 U2[12], D2[12];
+#pragma unroll
+  for (int j = 0; j < 12; ++j) {
+    U2[j] = f2(tp.up2[j]);
+    D2[j] = f2(tp.dn[j]);
+  }
+  // |u| <= up_abs * max |x| over the six inputs of either phase
+  float up_abs = 0.0f, up_abs1 = 0.0f;
+#pragma unroll
+  for (int l = 0; l < 6; ++l) {
+    up_abs += fabsf(tp.up2[2 * l + 1]);
+    up_abs1 += fabsf(tp.up2[2 * l]);
+  }
+  up_abs = fmaxf(up_abs, up_abs1);
 
   // tiles are visited as tile_id = blockIdx.x + k gridDim.x; (row, tile) are
   // carried along incrementally
@@ -191,18 +215,31 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
         X[4 * w + 2] = make_float2(lo.z, hi.z);
         X[4 * w + 3] = make_float2(lo.w, hi.w);
       }
+      // every u of this thread is bounded by up_abs times its largest input:
+      // when a times that bound is within sin^2's fast-path limit, the
+      // per-pair range check is skipped (thread-uniform branch)
+      float m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 12; ++j) m = fmaxf(m, fmaxf(fabsf(X[j].x), fabsf(X[j].y)));
+      const bool fast = a * (up_abs * m) <= sin2c::kFastLimit;
       float2 V[8];
+      auto stage_a = [&](auto check) {
 #pragma unroll
-      for (int qq = 0; qq < 4; ++qq) {
+        for (int qq = 0; qq < 4; ++qq) {
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int b0 = 2 + qq + r;
-          float2 u = mul2(f2(tp.up2[1 - r]), X[b0 + 5]);
+          for (int r = 0; r < 2; ++r) {
+            const int b0 = 2 + qq + r;
+            float2 u = mul2(U2[1 - r], X[b0 + 5]);
 #pragma unroll
-          for (int l = 1; l < 6; ++l) u = fma2(f2(tp.up2[2 * l + 1 - r]), X[b0 + 5 - l], u);
-          V[2 * qq + r] = snake2(u, a, inv_b);
+            for (int l = 1; l < 6; ++l) u = fma2(U2[2 * l + 1 - r], X[b0 + 5 - l], u);
+            V[2 * qq + r] = snake2<decltype(check)::value>(u, a, inv_b);
+          }
         }
-      }
+      };
+      if (fast)
+        stage_a(std::false_type{});
+      else
+        stage_a(std::true_type{});
       *reinterpret_cast<float4 *>(vs + vidx(2 * q0)) = make_float4(V[0].x, V[1].x, V[2].x, V[3].x);
       *reinterpret_cast<float4 *>(vs + vidx(2 * q0 + 4)) =
           make_float4(V[4].x, V[5].x, V[6].x, V[7].x);
@@ -254,9 +291,9 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int
       float2 out[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float2 acc = mul2(f2(tp.dn[0]), W[2 * e + 1]);
+        float2 acc = mul2(D2[0], W[2 * e + 1]);
 #pragma unroll
-        for (int j = 1; j < 12; ++j) acc = fma2(f2(tp.dn[j]), W[2 * e + j + 1], acc);
+        for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j + 1], acc);
         out[e] = acc;
       }
       float *yr = y + (size_t)row * T;

@@ -68,6 +68,20 @@ def test_activation_matches_oracle(nat, oracle, filt, B, C, T):
     np.testing.assert_allclose(y, want, rtol=1e-5, atol=1e-5)
 
 
+def test_activation_large_arguments(nat, oracle, filt):
+    """Inputs of scale 2e5, so that e^alpha u passes sin^2's fast-path limit in
+    most tiles (where the kernel range-checks every pair) while quiet rows stay
+    on the fast path; the result still matches the oracle."""
+    s = synth.NormalStream(99)
+    B, C, T = 2, 6, 5000
+    x = s.normal((B, C, T)) * np.where(np.arange(C) % 2 == 0, 2e5, 1.0)[None, :, None]
+    la = s.normal((C,), 0.0, 0.1)
+    lb = s.normal((C,), 0.0, 0.1)
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    want = oracle.activation1d(x, la, lb)
+    assert np.isfinite(y).all() and rel_l2(y, want) < LAYER_TOL
+
+
 def test_activation_constant_rows_exact_form(nat, filt):
     """Constant rows map to c + sin^2(e^a c)/(e^b + eps) everywhere, edges too."""
     C, T = 4, 3000
