@@ -11,24 +11,29 @@
 // of its channel tile.  Here a CTA takes SM_T consecutive outputs of one batch
 // row for every output channel.  It stages the input rows it needs (zero
 // outside [0, T)) and all the weights, reordered so that the output channels
-// of one (input channel, tap) are contiguous, then each thread accumulates 2
-// outputs x COUT channels in registers: per (i, j), two reads of x and COUT/4
-// broadcast 16-byte reads of w feed 2 COUT FMAs.
+// of one (input channel, tap) are contiguous, then each thread accumulates 4
+// consecutive outputs x COUT channels in registers: per (i, j), four reads of
+// x and COUT/4 broadcast 16-byte reads of w feed 4 COUT FMAs.  The common
+// kernel sizes are template arguments, so the tap loop unrolls.
 #include "common.cuh"
 
 namespace bv {
 namespace {
 
-constexpr int SM_T = 512;       // outputs per CTA
-constexpr int SM_THREADS = 256;  // 2 consecutive outputs each
+constexpr int SM_T = 512;        // outputs per CTA
+constexpr int SM_PER = 4;        // consecutive outputs per thread
+constexpr int SM_THREADS = SM_T / SM_PER;
 constexpr int SM_MAX_C = 32;
 
-template <int COUT>  // output channels rounded up to a multiple of 4
-__global__ void __launch_bounds__(SM_THREADS, 2)
+// COUT: output channels rounded up to a multiple of 4; KT: the kernel size
+// when fixed at compile time, 0 for a runtime K
+template <int COUT, int KT>
+__global__ void __launch_bounds__(SM_THREADS, COUT > 24 ? 2 : 3)
 conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
-                    const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
+                    const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int Kr,
                     int dil, int pad, int y_len, int y_pitch, Epi ep) {
   static_assert(COUT % 4 == 0 && COUT <= SM_MAX_C, "output channels");
+  const int K = KT > 0 ? KT : Kr;
   extern __shared__ __align__(16) float sm[];
   const int halo = (K - 1) * dil;
   const int XW = (SM_T + halo + 3) & ~3;  // staged row width
@@ -52,71 +57,79 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
   if (tid < COUT) bias_s[tid] = (bias && tid < Cout) ? __ldg(bias + tid) : 0.0f;
   __syncthreads();
 
-  const int tl = 2 * tid;  // this thread's outputs t0 + tl, t0 + tl + 1
-  float acc[COUT][2];
+  const int tl = SM_PER * tid;  // this thread's outputs t0 + tl .. t0 + tl + SM_PER - 1
+  float acc[COUT][SM_PER];
 #pragma unroll
-  for (int o = 0; o < COUT; ++o) acc[o][0] = acc[o][1] = 0.0f;
+  for (int o = 0; o < COUT; ++o)
+#pragma unroll
+    for (int e = 0; e < SM_PER; ++e) acc[o][e] = 0.0f;
   for (int i = 0; i < Cin; ++i) {
     const float *xr = xs + i * XW + tl;
     const float4 *wr = reinterpret_cast<const float4 *>(ws + i * K * COUT);
+#pragma unroll(KT > 0 ? KT : 1)
     for (int j = 0; j < K; ++j) {
-      const float x0 = xr[j * dil], x1 = xr[j * dil + 1];
+      float xv[SM_PER];
+#pragma unroll
+      for (int e = 0; e < SM_PER; ++e) xv[e] = xr[j * dil + e];
       const float4 *wj = wr + j * (COUT / 4);
 #pragma unroll
       for (int o4 = 0; o4 < COUT / 4; ++o4) {
         const float4 wv = wj[o4];
-        acc[4 * o4][0] = fmaf(wv.x, x0, acc[4 * o4][0]);
-        acc[4 * o4][1] = fmaf(wv.x, x1, acc[4 * o4][1]);
-        acc[4 * o4 + 1][0] = fmaf(wv.y, x0, acc[4 * o4 + 1][0]);
-        acc[4 * o4 + 1][1] = fmaf(wv.y, x1, acc[4 * o4 + 1][1]);
-        acc[4 * o4 + 2][0] = fmaf(wv.z, x0, acc[4 * o4 + 2][0]);
-        acc[4 * o4 + 2][1] = fmaf(wv.z, x1, acc[4 * o4 + 2][1]);
-        acc[4 * o4 + 3][0] = fmaf(wv.w, x0, acc[4 * o4 + 3][0]);
-        acc[4 * o4 + 3][1] = fmaf(wv.w, x1, acc[4 * o4 + 3][1]);
+#pragma unroll
+        for (int e = 0; e < SM_PER; ++e) {
+          acc[4 * o4][e] = fmaf(wv.x, xv[e], acc[4 * o4][e]);
+          acc[4 * o4 + 1][e] = fmaf(wv.y, xv[e], acc[4 * o4 + 1][e]);
+          acc[4 * o4 + 2][e] = fmaf(wv.z, xv[e], acc[4 * o4 + 2][e]);
+          acc[4 * o4 + 3][e] = fmaf(wv.w, xv[e], acc[4 * o4 + 3][e]);
+        }
       }
     }
   }
 
-  // epilogue, 8 channels at a time: every read (residual, accumulated y,
+  // epilogue, 4 channels at a time: every read (residual, accumulated y,
   // through the read-only path: each index is read once, by this thread,
   // before it writes it) ahead of the group's writes
   const int t = t0 + tl;
   if (t >= y_len) return;
-  const bool two = t + 1 < y_len;
-  const bool vec = two && ((((size_t)b * Cout) * y_pitch + t) % 2 == 0) && (y_pitch % 2 == 0) &&
-                   ((reinterpret_cast<uintptr_t>(y) & 7u) == 0);
+  const int n_out = y_len - t < SM_PER ? y_len - t : SM_PER;
+  const bool vec = n_out == SM_PER && (y_pitch % 4 == 0) &&
+                   ((reinterpret_cast<uintptr_t>(y) & 15u) == 0);  // t is a multiple of 4
 #pragma unroll
-  for (int g = 0; g < COUT; g += 8) {
-    float r[8][2], a[8][2];
+  for (int g = 0; g < COUT; g += 4) {
+    float r[4][SM_PER], a[4][SM_PER];
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const int o = g + q;
       const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
-      const bool ok = o < Cout;
-      r[q][0] = (ok && ep.residual) ? __ldg(ep.residual + idx) : 0.0f;
-      r[q][1] = (ok && two && ep.residual) ? __ldg(ep.residual + idx + 1) : 0.0f;
-      a[q][0] = (ok && ep.accumulate) ? __ldg(y + idx) : 0.0f;
-      a[q][1] = (ok && two && ep.accumulate) ? __ldg(y + idx + 1) : 0.0f;
+#pragma unroll
+      for (int e = 0; e < SM_PER; ++e) {
+        const bool ok = o < Cout && e < n_out;
+        r[q][e] = (ok && ep.residual) ? __ldg(ep.residual + idx + e) : 0.0f;
+        a[q][e] = (ok && ep.accumulate) ? __ldg(y + idx + e) : 0.0f;
+      }
     }
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
+    for (int q = 0; q < 4; ++q) {
       const int o = g + q;
       if (o < Cout) {
         const size_t idx = ((size_t)b * Cout + o) * y_pitch + t;
-        const float v0 = epi_final((acc[o][0] + bias_s[o] + r[q][0]) * ep.scale + a[q][0], ep);
-        const float v1 = epi_final((acc[o][1] + bias_s[o] + r[q][1]) * ep.scale + a[q][1], ep);
+        float v[SM_PER];
+#pragma unroll
+        for (int e = 0; e < SM_PER; ++e)
+          v[e] = epi_final((acc[o][e] + bias_s[o] + r[q][e]) * ep.scale + a[q][e], ep);
         if (vec) {
-          *reinterpret_cast<float2 *>(y + idx) = make_float2(v0, v1);
+          *reinterpret_cast<float4 *>(y + idx) = make_float4(v[0], v[1], v[2], v[3]);
         } else {
-          y[idx] = v0;
-          if (two) y[idx + 1] = v1;
+#pragma unroll
+          for (int e = 0; e < SM_PER; ++e)
+            if (e < n_out) y[idx + e] = v[e];
         }
       }
     }
   }
 }
 
-template <int COUT>
+template <int COUT, int KT>
 bv_status run_small(const float *x, int B, int Cin, int T, const float *w, const float *bias,
                     int Cout, int K, int dil, int pad, const Epi &ep, float *y, int y_len,
                     int y_pitch, cudaStream_t st) {
@@ -125,8 +138,8 @@ bv_status run_small(const float *x, int B, int Cin, int T, const float *w, const
   if (smem > 200 * 1024) return fail(BV_ERR_UNSUPPORTED, "conv1d_small: tile too large");
   static size_t configured = 0;
   if (smem > 48 * 1024 && smem > configured) {
-    if (cudaFuncSetAttribute(conv1d_small_kernel<COUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(conv1d_small_kernel<COUT, KT>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
       return check_launch("conv1d_small smem attribute");
     configured = smem;
   }
@@ -137,8 +150,8 @@ bv_status run_small(const float *x, int B, int Cin, int T, const float *w, const
     LaunchTimer tm(st, "conv1d_small", 2.0 * outs * Cin * K,
                    4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                           outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
-    conv1d_small_kernel<COUT><<<grid, SM_THREADS, smem, st>>>(x, w, bias, y, Cin, T, Cout, K, dil,
-                                                              pad, y_len, y_pitch, ep);
+    conv1d_small_kernel<COUT, KT><<<grid, SM_THREADS, smem, st>>>(x, w, bias, y, Cin, T, Cout, K,
+                                                                  dil, pad, y_len, y_pitch, ep);
   }
   count_launch();
   return check_launch("conv1d_small_kernel");
@@ -157,15 +170,23 @@ bv_status launch_conv1d_small(const float *x, int B, int Cin, int T, const float
   if (B <= 0 || y_len <= 0) return BV_OK;
   if (!conv1d_small_supported(Cin, Cout, K, dil))
     return fail(BV_ERR_UNSUPPORTED, "conv1d_small: Cin %d Cout %d", Cin, Cout);
+#define BV_SMALL_K(N, KK)                                                                     \
+  if (K == KK)                                                                                \
+    return run_small<N, KK>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
 #define BV_SMALL(N)                                                                           \
-  if (Cout <= N)                                                                              \
-    return run_small<N>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st);
+  if (Cout <= N) {                                                                            \
+    BV_SMALL_K(N, 3)                                                                          \
+    BV_SMALL_K(N, 7)                                                                          \
+    BV_SMALL_K(N, 11)                                                                         \
+    return run_small<N, 0>(x, B, Cin, T, w, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
+  }
   BV_SMALL(8)
   BV_SMALL(12)
   BV_SMALL(16)
   BV_SMALL(24)
   BV_SMALL(32)
 #undef BV_SMALL
+#undef BV_SMALL_K
   return fail(BV_ERR_UNSUPPORTED, "conv1d_small: Cout %d", Cout);
 }
 
