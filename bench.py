@@ -114,7 +114,7 @@ def peaks():
 
 
 # kernel classes that run 3xTF32 on the tensor cores
-TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc")
+TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm")
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of a full decode of the bench workload, per kernel class, for the

@@ -521,12 +521,14 @@ size_t convt_ws(const bv_decoder_config *c) {
   size_t m = 0;
   int C = c->pre_channels;
   for (int i = 0; i < c->n_up; ++i) {
-    if (conv_transpose1d_tc_supported(C, c->up_channels[i], c->up_kernel[i], c->up_rate[i])) {
-      const size_t b = conv_transpose1d_tc_workspace(C, c->up_channels[i], c->up_kernel[i],
-                                                     c->up_rate[i]);
-      if (b > m) m = b;
-    }
-    C = c->up_channels[i];
+    const int Co = c->up_channels[i], k = c->up_kernel[i], sr = c->up_rate[i];
+    size_t b = 0;
+    if (conv_transpose1d_tm_supported(C, Co, k, sr))
+      b = conv_transpose1d_tm_workspace(C, Co, k, sr);
+    else if (conv_transpose1d_tc_supported(C, Co, k, sr))
+      b = conv_transpose1d_tc_workspace(C, Co, k, sr);
+    if (b > m) m = b;
+    C = Co;
   }
   return align_up(m);
 }
@@ -755,7 +757,12 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
     const int sr = c->up_rate[i], k = c->up_kernel[i], Co = c->up_channels[i];
     const int pad = (k - sr) / 2;
     const int n2 = (n - 1) * sr + k - 2 * pad;
-    if (conv_transpose1d_tc_supported(C, Co, k, sr))
+    if (conv_transpose1d_tm_supported(C, Co, k, sr)) {
+      // time-major: the stage input goes to block 0's operand planes first
+      BV_TRY(launch_transpose_split(A, s.xhi, s.xlo, B, C, n, st));
+      BV_TRY(launch_conv_transpose1d_tm(s.xhi, s.xlo, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr,
+                                        pad, S, WP, st));
+    } else if (conv_transpose1d_tc_supported(C, Co, k, sr))
       BV_TRY(launch_conv_transpose1d_tc(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S,
                                         WP, st));
     else

@@ -201,6 +201,16 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
                            int pad, const Epi &ep, float *y, int y_len, int y_pitch,
                            cudaStream_t st);
 
+// Transposed conv on the time-major kernel: x_hi / x_lo [B, T, Cin] planes
+// (launch_transpose_split), each of the S output phases an ceil(K/S)-tap conv
+// over the input samples with its weights repacked tap-major into wp
+// (conv_transpose1d_tm_workspace bytes).
+bool conv_transpose1d_tm_supported(int Cin, int Cout, int K, int S);
+size_t conv_transpose1d_tm_workspace(int Cin, int Cout, int K, int S);
+bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                                     const float *w, const float *bias, int Cout, int K, int S,
+                                     int pad, float *y, float *wp, cudaStream_t st);
+
 // [B, C, T] -> time-major planes hi[b, t, c] = tf32(x[b, c, t]),
 // lo = x - hi.
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,

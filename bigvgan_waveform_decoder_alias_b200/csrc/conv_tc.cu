@@ -703,7 +703,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_whi,
                  const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ bias,
                  float *y, int Cin, int Cout, int K, int dil, int pad, int y_len, int y_pitch,
-                 Epi ep, int *status) {
+                 Epi ep, OutMap om, int *status) {
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= MAX_NT, "UMMA N for M = 256, halves of 16");
   constexpr uint32_t IDESC = make_idesc_pair(NT);
   constexpr unsigned W_TX_TAP = 2u * 2u * (NT / 2) * BK * 4;  // one tap: both CTAs, hi and lo
@@ -738,7 +738,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = (blockIdx.x >> 1) * (2 * BM) + (int)rank * BM;  // this CTA's rows
   const int o0 = blockIdx.y * NT;
-  const int b = blockIdx.z;
+  const int b = blockIdx.z / om.phases;
+  const int phase = blockIdx.z - b * om.phases;  // weight rows phase Cout .., output offset + phase
   const int n_cb = (Cin + BK - 1) / BK;  // 32-channel blocks (channels past Cin read as 0)
   const int Cpad = n_cb * BK;            // weight row stride per tap
   const int n_tc = (K + 1) / 2;       // chunks per block: taps (0,1), (2,3), ...
@@ -796,7 +797,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   } else if (warp == 0) {
     // ----------------------------------------------- TMA producer: weight chunks
     if (lane == 0) {
-      const int row = o0 + (int)rank * (NT / 2);
+      const int row = phase * Cout + o0 + (int)rank * (NT / 2);
       int ws = 0, wphase = 0;
       for (int cb = 0; cb < n_cb; ++cb) {
         for (int q = 0; q < n_tc; ++q) {
@@ -900,9 +901,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
     }
     const int t = t0 + ct;
-    if (!ctl.abort && t < y_len) {
+    const int p = om.stride * t + om.offset + phase;  // output sample of conv position t
+    if (!ctl.abort && t < y_len && p >= 0 && p < om.len) {
       // 16 channels at a time: the group's reads, then its writes
-      const size_t base = (size_t)b * Cout * y_pitch + t;
+      const size_t base = (size_t)b * Cout * y_pitch + p;
 #pragma unroll
       for (int g = 0; g < NT; g += 16) {
         float bb[16];
@@ -931,7 +933,7 @@ template <int NT>
 bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
                  int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
-                 cudaStream_t st) {
+                 const OutMap &om, cudaStream_t st) {
   static bool configured = false;
   if (!configured) {
     if (cudaFuncSetAttribute(conv1d_tm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -939,10 +941,11 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
       return check_launch("conv1d_tm smem attribute");
     configured = true;
   }
-  dim3 grid(2 * ((y_len + 2 * BM - 1) / (2 * BM)), (Cout + NT - 1) / NT, B);
+  dim3 grid(2 * ((y_len + 2 * BM - 1) / (2 * BM)), (Cout + NT - 1) / NT, B * om.phases);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tm: grid too large");
   conv1d_tm_kernel<NT><<<grid, THREADS, TM_SMEM_BYTES, st>>>(
-      xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, device_status_ptr());
+      xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
+      device_status_ptr());
   return BV_OK;
 }
 
@@ -1057,6 +1060,28 @@ __global__ void convt_repack_kernel(const float *__restrict__ w, float *__restri
     const int r = (int)(rest / Cout);
     const int k = r + S * (nt - 1 - j);
     const float v = k < K ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
+    const float h = tf32_hi(v);
+    wp[idx] = h;
+    wp_lo[idx] = v - h;
+  }
+}
+
+// Tap-major phase weights for the time-major kernel: wp[r][o][j cp + i] =
+// w[i][o][r + S (nt - 1 - j)] split into tf32 hi / lo (zero past K or Cin).
+__global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__restrict__ wp,
+                                       float *__restrict__ wp_lo, int Cin, int Cout, int K, int S,
+                                       int nt, int cp) {
+  const long long total = (long long)S * Cout * nt * cp;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(idx % cp);
+    long long rest = idx / cp;
+    const int j = (int)(rest % nt);
+    rest /= nt;
+    const int o = (int)(rest % Cout);
+    const int r = (int)(rest / Cout);
+    const int k = r + S * (nt - 1 - j);
+    const float v = (k < K && i < Cin) ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
     const float h = tf32_hi(v);
     wp[idx] = h;
     wp_lo[idx] = v - h;
@@ -1244,31 +1269,28 @@ bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
          (K - 1) * dil <= TM_MAX_HALO && encode_fn() != nullptr;
 }
 
-bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
-                           const float *w_split, const float *bias, int Cout, int K, int dil,
-                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
-                           cudaStream_t st) {
-  if (B <= 0 || y_len <= 0) return BV_OK;
-  if (!conv1d_tm_supported(Cin, Cout, K, dil))
-    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
+namespace {
+
+// The time-major launch: w_split holds hi then lo of a [w_rows, K Cp] tap-major
+// matrix (w_rows = phases Cout), outputs go through om.
+bv_status tm_impl(const char *cls, const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                  const float *w_split, int w_rows, const float *bias, int Cout, int K, int dil,
+                  int pad, const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
+                  double flops, double bytes, cudaStream_t st) {
   const int nt = pick_nt_pair(Cout);
   const int KK = tm_cin_pad(Cin) * K;  // tap-major weight row, padded channels
   CUtensorMap xh, xl, wh, wl;
   BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T, BM + (K - 1) * dil));
   BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T, BM + (K - 1) * dil));
-  BV_TRY(encode_w(&wh, w_split, Cout, KK, nt / 2));  // each CTA of a pair loads half the rows
-  BV_TRY(encode_w(&wl, w_split + (size_t)Cout * KK, Cout, KK, nt / 2));
+  BV_TRY(encode_w(&wh, w_split, w_rows, KK, nt / 2));  // each CTA of a pair loads half the rows
+  BV_TRY(encode_w(&wl, w_split + (size_t)w_rows * KK, w_rows, KK, nt / 2));
   bv_status s;
   {
-    // algorithmic work: the useful products (Cin K per output), not the
-    // padded channel block or the three 3xTF32 terms
-    const double outs = (double)B * Cout * y_len;
-    LaunchTimer tm(st, "conv1d_tm", 2.0 * outs * Cin * K,
-                   4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
-                          outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)));
-#define BV_TM_CASE(N)                                                                          \
-  case N:                                                                                      \
-    s = run_tm<N>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, st); \
+    LaunchTimer tm(st, cls, flops, bytes);
+#define BV_TM_CASE(N)                                                                      \
+  case N:                                                                                  \
+    s = run_tm<N>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, \
+                  om, st);                                                                 \
     break;
     switch (nt) {
       BV_TM_CASE(64)
@@ -1282,6 +1304,59 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
   if (s != BV_OK) return s;
   count_launch();
   return check_launch("conv1d_tm_kernel");
+}
+
+}  // namespace
+
+bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                           const float *w_split, const float *bias, int Cout, int K, int dil,
+                           int pad, const Epi &ep, float *y, int y_len, int y_pitch,
+                           cudaStream_t st) {
+  if (B <= 0 || y_len <= 0) return BV_OK;
+  if (!conv1d_tm_supported(Cin, Cout, K, dil))
+    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
+  // algorithmic work: the useful products (Cin K per output), not the padded
+  // channel block or the three 3xTF32 terms
+  const double outs = (double)B * Cout * y_len;
+  return tm_impl("conv1d_tm", x_hi, x_lo, B, Cin, T, w_split, Cout, bias, Cout, K, dil, pad, ep,
+                 y, y_len, y_pitch, OutMap{1, 0, y_len, 1}, 2.0 * outs * Cin * K,
+                 4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
+                        outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)),
+                 st);
+}
+
+bool conv_transpose1d_tm_supported(int Cin, int Cout, int K, int S) {
+  return conv1d_tm_supported(Cin, Cout, convt_taps(K, S), 1);
+}
+
+size_t conv_transpose1d_tm_workspace(int Cin, int Cout, int K, int S) {
+  return 2 * (size_t)S * Cout * tm_cin_pad(Cin) * convt_taps(K, S) * sizeof(float);
+}
+
+bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                                     const float *w, const float *bias, int Cout, int K, int S,
+                                     int pad, float *y, float *wp, cudaStream_t st) {
+  if (B <= 0 || T <= 0) return BV_OK;
+  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
+    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
+  const int nt = convt_taps(K, S), cp = tm_cin_pad(Cin);
+  const int Tout = (T - 1) * S + K - 2 * pad;
+  const long long total = (long long)S * Cout * nt * cp;
+  {
+    LaunchTimer tm(st, "convt_repack", 0.0, 4.0 * (double)Cin * Cout * K + 8.0 * (double)total);
+    const long long blocks = (total + 255) / 256;
+    convt_repack_tm_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
+        w, wp, wp + total, Cin, Cout, K, S, nt, cp);
+  }
+  count_launch();
+  BV_TRY(check_launch("convt_repack_tm_kernel"));
+  // phase r: conv output P (input-grid index, P < T + nt - 1) lands on sample
+  // S P + r - pad of the output row
+  return tm_impl("conv_transpose1d_tm", x_hi, x_lo, B, Cin, T, wp, S * Cout, bias, Cout, nt, 1,
+                 nt - 1, Epi{nullptr, 1.0f, 0, 0}, y, T + nt - 1, Tout, OutMap{S, -pad, Tout, S},
+                 2.0 * B * Cin * (double)Cout * K * T,
+                 4.0 * ((double)B * Cin * T + (double)Cin * Cout * K + (double)B * Cout * Tout),
+                 st);
 }
 
 }  // namespace bv

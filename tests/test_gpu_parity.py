@@ -467,7 +467,7 @@ def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     zd = dev(z)
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault("y", dec.decode(zd)))
-    assert "conv_transpose1d_tc" in classes, classes
+    assert "conv_transpose1d_tm" in classes, classes
     # the 128/96/48-channel AMP convs run time-major
     assert "conv1d_tm" in classes and "transpose_split" in classes, classes
     want = oracle.decode(geo, params, z)
