@@ -120,7 +120,7 @@ TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpo
 # ncu capture of a full decode of the bench workload, per kernel class, for the
 # kernel code as committed with it (profiles/conv1d_tm_traffic_h3_10s.md);
 # a class missing here reports null.
-NCU_TRAFFIC_PER_LAUNCH = {"conv1d_tm": 84.1e6}
+NCU_TRAFFIC_PER_LAUNCH = {"conv1d_tm": 84.65e6}
 
 
 def roofline_for(name, kd, pk):
