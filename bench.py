@@ -45,7 +45,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="time one kernel on one shape instead of the decoder (for profiling): "
-                         "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s")
+                         "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s | "
+                         "amp:BxCxT:K (an AMP block, dilations 1, 3, 5)")
     return ap.parse_args()
 
 
@@ -77,6 +78,23 @@ def run_case(args):
         b = torch.from_numpy(s.normal((Co,), 0, 0.02)).cuda()
         fn = lambda: native.bv_conv_transpose1d(x, w, b, st)  # noqa: E731
         work, unit = 2.0 * B * C * Co * 2 * st * T, "TFLOP/s"
+    elif kind == "amp":
+        K = int(rest[0])
+        wl = synth.AmpWorkload("case", B, C, T, K, (1, 3, 5), seed=7)
+        xa, flat = wl.make()
+        x = torch.from_numpy(xa).cuda()
+        tens, off = {}, 0
+        for name, shape, _ in wl.layout():
+            n = int(np.prod(shape))
+            tens[name] = torch.from_numpy(flat[off:off + n].reshape(shape)).cuda()
+            off += n
+        p = native.amp_params(K, (1, 3, 5), tens, filt)
+        y = torch.empty_like(x)
+        ws = torch.empty(native.bv_amp_block_workspace_size_tc(B, C, T, p) // 4 + 64,
+                         device="cuda")
+        fn = lambda: native.bv_amp_block(x, p, y=y, workspace=ws)  # noqa: E731
+        # the block's 6 convs (useful FLOPs); its activations are not counted
+        work, unit = 2.0 * 6 * B * C * C * K * T, "TFLOP/s"
     else:
         raise SystemExit(f"unknown case {kind}")
     for _ in range(args.warmup):
@@ -91,7 +109,8 @@ def run_case(args):
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
     rate = work / (ms / 1000) / (1e9 if unit == "GB/s" else 1e12)
-    print(json.dumps({"case": args.case, "ms_median": ms, "achieved": rate, "unit": unit}))
+    print(json.dumps({"case": args.case, "ms_median": ms, "achieved": rate, "unit": unit,
+                      "steps": args.steps, "warmup": args.warmup}))
     return 0
 
 
