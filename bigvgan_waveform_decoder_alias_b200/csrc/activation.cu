@@ -12,14 +12,26 @@
 // (the polyphase form of the pages' replicate pad 5 / stride-2 transposed
 // FIR / trim 15 / replicate pad 5|6 / stride-2 FIR).
 //
-// Persistent CTAs walk row tiles of TILE outputs.  While a CTA computes one
-// tile, the next tile's input x[t0-8 .. t0+TILE+8) (clamped at the row ends)
-// streams into the other half of a double buffer with cp.async.  Per tile,
-// stage A computes v[2 t0 - 6 + k], k < 2 TILE + 12, into shared memory and
-// stage B filters v into the TILE outputs.  Each thread works on two
-// positions half a tile apart at once, with packed f32x2 arithmetic (FFMA2):
-// both positions have the same polyphase taps, so every filter tap and every
-// step of the sin^2 evaluation is one paired instruction.
+// Work unit: a warp tile, TW outputs of two rows at once (rows r0 and r0 + 1;
+// channels may differ).  Everything in shared memory is stored as (row r0,
+// row r0 + 1) pairs, so every load yields operand pairs for packed f32x2
+// arithmetic (FFMA2) directly: the two rows share the filter taps, and their
+// SnakeBeta constants sit in pairs too.
+//
+// Every warp runs on its own, with no block-wide barrier: it owns a
+// contiguous range of warp tiles (row pair by row pair, left to right) and
+// its own shared memory -- a double buffer of input windows, filled with
+// cp.async one tile ahead, and a ring of two 2x-rate buffers.  Stage A of
+// tile j computes v[2 t0 - 5 + s], s < 2 TW, into the ring; stage B of tile j
+// also needs the first 10 values of tile j + 1, so it runs after stage A of
+// tile j + 1.  Only at the end of a row (replicate padding) or of the warp's
+// range does stage B follow its own stage A, after computing those 10 values
+// directly.
+//
+// SnakeBeta's sin^2 runs in units of pi: w = u a/pi, f = w - rint(w) in
+// [-1/2, 1/2] (exact), and sin(pi f) = f P(f^2) with a degree-4 polynomial P
+// (sin2.cuh).  The row's sqrt(inv_b) is folded into P, so v = u + g^2 with
+// g = f P'(f^2): eleven paired instructions per pair of values.
 #include <type_traits>
 
 #include "common.cuh"
@@ -28,79 +40,93 @@
 namespace bv {
 namespace {
 
-constexpr int TILE = 2048;         // outputs per tile
-constexpr int HALF = TILE / 2;     // the two positions of a thread are HALF apart
-constexpr int THREADS = 256;       // per half tile: 4 outputs and 8 up-sampled values each
-constexpr int XS = TILE + 16;      // x[t0 - 8 + i]
-// v[2 t0 - 6 + k], k < 2 TILE + 12, stored at vidx(k): 4 floats of padding
-// after every 32 spread the 32-byte-strided float4 accesses of a warp over all
-// banks
-__device__ __forceinline__ int vidx(int k) { return k + 4 * (k >> 5); }
-constexpr int VS = (2 * TILE + 16) + 4 * ((2 * TILE + 16) / 32 + 1);
-static_assert(HALF == 4 * THREADS, "one thread per 4 outputs of a half tile");
+constexpr int WARPS = 8;          // per CTA
+constexpr int THREADS = 32 * WARPS;
+constexpr int TW = 256;           // outputs per row of a warp tile
+constexpr int XP = TW + 16;       // input pairs x[t0 - 8 + i] of a warp tile
+constexpr int RING = 4 * TW;      // 2x-rate ring: two tiles of 2 TW pairs
+constexpr int XS_FLOATS = 2 * XP;
+constexpr int RING_FLOATS = 2 * RING;
+constexpr int WARP_FLOATS = 2 * XS_FLOATS + RING_FLOATS + 2 * 10;
+constexpr size_t SMEM_BYTES = (size_t)WARPS * WARP_FLOATS * sizeof(float);
+static_assert(TW == 2 * 4 * 32, "two passes of 4 outputs per lane");
+static_assert(XP % 16 == 0 && RING % 16 == 0, "whole swizzle blocks");
 
-__device__ __forceinline__ float2 f2(float v) { return make_float2(v, v); }
+// Shared-memory float offsets of pair i.  A 16-byte chunk holds two pairs;
+// chunks are XOR-swizzled inside blocks of 8 so that the 16-byte accesses of
+// a quarter warp hit 8 distinct bank groups.  Input pairs: stage A's lanes are
+// 2 chunks apart, and bit 3 of the chunk index flips bit 0.  2x-rate pairs:
+// stages A and B have lanes 4 chunks apart, and bits 3-4 of the chunk index
+// flip bits 0-1.
+__device__ __forceinline__ int xoff(int i) {
+  const int ch = i >> 1;
+  return 4 * (ch ^ ((ch >> 3) & 1)) + 2 * (i & 1);
+}
+__device__ __forceinline__ int voff(int s) {
+  const int ch = s >> 1;
+  return 4 * (ch ^ ((ch >> 3) & 3)) + 2 * (s & 1);
+}
+
+// |w| bound of the fast path: far inside the 2^22 where rint by adding and
+// removing 1.5 * 2^23 stays exact; |a u| <= pi * 16384 = 51472.
+constexpr float kWLimit = 16384.0f;
+
+// Per-row-pair constants, as (row r0, row r0 + 1) pairs.
+enum {
+  kA = 0,      // a / pi
+  kP = 1,      // P_j sqrt(inv_b), j < 5
+  kM = 6,      // 1.5 * 2^23 (both)
+  kNeg = 7,    // -1 (both)
+  kAraw = 8,   // a
+  kIb = 9,     // inv_b
+  kConsts = 10
+};
+
 __device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
 
-// Scalar SnakeBeta (tails and edge fix-ups).
-__device__ __forceinline__ float snake1(float u, float a, float inv_b) {
-  return fmaf(sin_squared(a * u), inv_b, u);
-}
-
-// Paired SnakeBeta: u + sin^2(a u) inv_b for two values, with the sin^2 of
-// sin2.cuh (reduction by pi in three parts, Taylor series of sin to r^13).
-// The nearest integer to z/pi comes from adding and removing 1.5 * 2^23.
-// CHECK = false when the caller has bounded |a u| by the fast-path limit.
-template <bool CHECK = true>
-__device__ __forceinline__ float2 snake2(float2 u, float a, float inv_b) {
-  using namespace sin2c;
-  const float2 z = mul2(u, f2(a));
-  if (CHECK && fmaxf(fabsf(z.x), fabsf(z.y)) > kFastLimit)
-    return make_float2(snake1(u.x, a, inv_b), snake1(u.y, a, inv_b));
-  const float2 k = add2(fma2(z, f2(kInvPi), f2(12582912.0f)), f2(-12582912.0f));
-  float2 r = fma2(k, f2(-kC1), z);
-  r = fma2(k, f2(-kC2), r);
-  r = fma2(k, f2(-kC3), r);
-  const float2 r2 = mul2(r, r);
-  float2 p = fma2(r2, f2(kT6), f2(kT5));
-  p = fma2(r2, p, f2(kT4));
-  p = fma2(r2, p, f2(kT3));
-  p = fma2(r2, p, f2(kT2));
-  p = fma2(r2, p, f2(kT1));
-  p = fma2(r2, p, f2(1.0f));
-  const float2 s = mul2(r, p);
-  return fma2(mul2(s, s), f2(inv_b), u);
-}
-
-struct Taps {
-  float up2[12];  // 2 * f_up
-  float dn[12];
+struct Snake {
+  float2 A, P[5], M, Neg;
 };
 
-// u at phase r (0: even index, 1: odd) from six consecutive x values
-// xp[0..5] = x[p + r - 3 .. p + r + 2]:  u[2p+r] = sum_l 2 f[2l+1-r] x[p+2+r-l],
-// where term l pairs with xp[5-l].  (The phase is a template argument so the
-// taps are indexed statically and stay in registers.)
-template <int R>
-__device__ __forceinline__ float up1r(const Taps &tp, const float *xp) {
-  float u = tp.up2[1 - R] * xp[5];
-#pragma unroll
-  for (int l = 1; l < 6; ++l) u = fmaf(tp.up2[2 * l + 1 - R], xp[5 - l], u);
-  return u;
+// Paired SnakeBeta for the two rows.  CHECK: range-check |w| per pair and
+// take the scalar sin^2 of sin2.cuh (Cody-Waite reduction, sinf beyond its
+// limit) for pairs outside the fast path.
+template <bool CHECK>
+__device__ __forceinline__ float2 snake2(float2 u, const Snake &k, const float2 *cst) {
+  const float2 w = mul2(u, k.A);
+  if (CHECK && fmaxf(fabsf(w.x), fabsf(w.y)) > kWLimit) {
+    const float2 a = cst[kAraw], ib = cst[kIb];
+    return make_float2(fmaf(sin_squared(a.x * u.x), ib.x, u.x),
+                       fmaf(sin_squared(a.y * u.y), ib.y, u.y));
+  }
+  const float2 t = add2(w, k.M);          // rint(w) + 1.5 * 2^23
+  const float2 nk = fma2(t, k.Neg, k.M);  // -rint(w), exact
+  const float2 f = add2(w, nk);           // in [-1/2, 1/2], exact
+  const float2 s = mul2(f, f);
+  float2 p = fma2(s, k.P[4], k.P[3]);
+  p = fma2(s, p, k.P[2]);
+  p = fma2(s, p, k.P[1]);
+  p = fma2(s, p, k.P[0]);
+  const float2 g = mul2(f, p);  // sqrt(inv_b) sin(pi f)
+  return fma2(g, g, u);
 }
-__device__ __forceinline__ float up1(const Taps &tp, int r, const float *xp) {
-  return r ? up1r<1>(tp, xp) : up1r<0>(tp, xp);
+
+// u pair at phase R from six consecutive input pairs xp[0..5] =
+// x[p + R - 3 .. p + R + 2]: u[2p+R] = sum_l 2 f_up[2l+1-R] x[p+2+R-l], term l
+// pairs with xp[5-l].
+template <int R>
+__device__ __forceinline__ float2 up2(const float2 *U2, const float2 *xp) {
+  float2 u = mul2(U2[1 - R], xp[5]);
+#pragma unroll
+  for (int l = 1; l < 6; ++l) u = fma2(U2[2 * l + 1 - R], xp[5 - l], u);
+  return u;
 }
 
 __device__ __forceinline__ void cp_async4(float *dst, const float *src) {
   const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(d), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async16(float *dst, const float *src) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
   asm volatile("cp.async.commit_group;\n" ::: "memory");
@@ -110,19 +136,33 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
 }
 
-// Issue the copies of one tile's input into xs: x[t0 - 8 + i], clamped.
-__device__ __forceinline__ void issue_tile(const float *__restrict__ xr, float *xs, int t0, int T,
-                                           int tid) {
-  const bool vec =
-      ((reinterpret_cast<uintptr_t>(xr) & 15u) == 0) && (t0 >= 8) && (t0 + TILE + 8 <= T);
-  if (vec) {
-    const float *src = xr + t0 - 8;
-    for (int c = tid; c < XS / 4; c += THREADS) cp_async16(xs + 4 * c, src + 4 * c);
+// Issue the copies of one warp tile's input: pair i = (x0[t0 - 8 + i],
+// x1[t0 - 8 + i]), positions clamped to [0, T).  Lane L copies pairs L + 32 j
+// of each row (j < 9, the last only for L < 16).
+__device__ __forceinline__ void issue_tile(const float *__restrict__ x0,
+                                           const float *__restrict__ x1, float *xs, int t0, int T,
+                                           int lane) {
+  float *d = xs + xoff(lane);  // xoff(L + 32 j) = xoff(L) + 64 j
+  const int base = t0 - 8 + lane;
+  if (t0 >= 8 && t0 - 8 + XP <= T) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cp_async4(d + 64 * j, x0 + base + 32 * j);
+      cp_async4(d + 64 * j + 1, x1 + base + 32 * j);
+    }
+    if (lane < XP - 256) {
+      cp_async4(d + 512, x0 + base + 256);
+      cp_async4(d + 513, x1 + base + 256);
+    }
   } else {
-    for (int i = tid; i < XS; i += THREADS) {
-      int p = t0 - 8 + i;
-      p = p < 0 ? 0 : (p > T - 1 ? T - 1 : p);
-      cp_async4(xs + i, xr + p);
+#pragma unroll
+    for (int j = 0; j < 9; ++j) {
+      if (j < 8 || lane < XP - 256) {
+        int p = base + 32 * j;
+        p = p < 0 ? 0 : (p > T - 1 ? T - 1 : p);
+        cp_async4(d + 64 * j, x0 + p);
+        cp_async4(d + 64 * j + 1, x1 + p);
+      }
     }
   }
 }
@@ -139,168 +179,254 @@ __device__ __forceinline__ void store4(float *yr, int t, int T, float o0, float 
   }
 }
 
+__device__ __forceinline__ void load_taps(float2 (&F)[12], const float2 *taps) {
+#pragma unroll
+  for (int j = 0; j < 6; ++j) {
+    const float4 v = reinterpret_cast<const float4 *>(taps)[j];
+    F[2 * j] = make_float2(v.x, v.y);
+    F[2 * j + 1] = make_float2(v.z, v.w);
+  }
+}
+
+// Stage A of one warp tile: the lane's 2x-rate pairs s = 256 h + 8 L + n
+// (pass h < 2, n < 8), i.e. k = s + 1 = 2q + r from (q0, 1) to (q0 + 4, 0)
+// with q0 = 128 h + 4 L relative to t0 - 3; their inputs are the pairs
+// q0 + 3 .. q0 + 11 (X[j] = pair q0 + 2 + j).  Ring slot of s: rb + s.
+__device__ __forceinline__ void stage_a(const float *xb, float *ring, int rb, const float2 *taps,
+                                        const float2 *cst, float up_abs, int lane) {
+  float2 U2[12];
+  load_taps(U2, taps);
+  Snake k;
+  {
+    const float4 *c4 = reinterpret_cast<const float4 *>(cst);
+    float4 v = c4[0];
+    k.A = make_float2(v.x, v.y);
+    k.P[0] = make_float2(v.z, v.w);
+    v = c4[1];
+    k.P[1] = make_float2(v.x, v.y);
+    k.P[2] = make_float2(v.z, v.w);
+    v = c4[2];
+    k.P[3] = make_float2(v.x, v.y);
+    k.P[4] = make_float2(v.z, v.w);
+    v = c4[3];
+    k.M = make_float2(v.x, v.y);
+    k.Neg = make_float2(v.z, v.w);
+  }
+  const float bound = up_abs * fmaxf(k.A.x, k.A.y);
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int q0 = 128 * h + 4 * lane;
+    float2 X[10];
+#pragma unroll
+    for (int m = 0; m < 5; ++m) {
+      const float4 v = *reinterpret_cast<const float4 *>(xb + xoff(q0 + 2 + 2 * m));
+      X[2 * m] = make_float2(v.x, v.y);
+      X[2 * m + 1] = make_float2(v.z, v.w);
+    }
+    // every u of this lane is bounded by up_abs times its largest input:
+    // when that keeps |w| within the fast path, the per-pair range check is
+    // skipped (lane-uniform branch)
+    float mx = 0.0f;
+#pragma unroll
+    for (int j = 1; j < 10; ++j) mx = fmaxf(mx, fmaxf(fabsf(X[j].x), fabsf(X[j].y)));
+    auto run = [&](auto check) {
+      constexpr bool CK = decltype(check)::value;
+#pragma unroll
+      for (int n = 0; n < 8; n += 2) {
+        // n (even): phase 1 at q0 + n/2; n + 1: phase 0 at q0 + n/2 + 1; both
+        // read the input pairs X[n/2 + 1 ..]
+        const float2 v0 = snake2<CK>(up2<1>(U2, X + n / 2 + 1), k, cst);
+        const float2 v1 = snake2<CK>(up2<0>(U2, X + n / 2 + 1), k, cst);
+        *reinterpret_cast<float4 *>(ring + voff((rb + 2 * q0 + n) & (RING - 1))) =
+            make_float4(v0.x, v0.y, v1.x, v1.y);
+      }
+    };
+    if (mx * bound <= kWLimit)
+      run(std::false_type{});
+    else
+      run(std::true_type{});
+  }
+}
+
+// The 10 pairs s in [2 TW, 2 TW + 10) of a tile, from its own input window:
+// k = s + 1 = 2 TW + 1 + i; lanes 0-4 take phase 1 (q = TW + L), lanes 5-9
+// phase 0 (q = TW + L - 4).
+__device__ __forceinline__ void stage_a_tail(const float *xb, float *ring, int rb,
+                                             const float2 *taps, const float2 *cst, int lane) {
+  if (lane >= 10) return;
+  float2 U2[12];
+  load_taps(U2, taps);
+  Snake k;
+  k.A = cst[kA];
+#pragma unroll
+  for (int j = 0; j < 5; ++j) k.P[j] = cst[kP + j];
+  k.M = cst[kM];
+  k.Neg = cst[kNeg];
+  const int R = lane < 5 ? 1 : 0;
+  const int q = lane < 5 ? TW + lane : TW + lane - 4;
+  float2 xp[6];
+#pragma unroll
+  for (int j = 0; j < 6; ++j) xp[j] = *reinterpret_cast<const float2 *>(xb + xoff(2 + q + R + j));
+  const float2 u = R ? up2<1>(U2, xp) : up2<0>(U2, xp);
+  *reinterpret_cast<float2 *>(ring + voff((rb + 2 * q + R - 1) & (RING - 1))) =
+      snake2<true>(u, k, cst);
+}
+
+// Stage B of one warp tile: y[t] = sum_j f_dn[j] v[2t + j - 5] with
+// v[2t + j - 5] at s = 2 (t - t0) + j; lane L writes t = t0 + 128 h + 4 L + e.
+__device__ __forceinline__ void stage_b(const float *ring, int rb, const float2 *taps,
+                                        float *y0, bool has_r1, int t0, int T, int lane) {
+  float2 D2[12];
+  load_taps(D2, taps + 12);
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    const int tl = 128 * h + 4 * lane;
+    float2 W[18];
+#pragma unroll
+    for (int m = 0; m < 9; ++m) {
+      const float4 v =
+          *reinterpret_cast<const float4 *>(ring + voff((rb + 2 * tl + 2 * m) & (RING - 1)));
+      W[2 * m] = make_float2(v.x, v.y);
+      W[2 * m + 1] = make_float2(v.z, v.w);
+    }
+    float2 out[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float2 acc = mul2(D2[0], W[2 * e]);
+#pragma unroll
+      for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j], acc);
+      out[e] = acc;
+    }
+    store4(y0, t0 + tl, T, out[0].x, out[1].x, out[2].x, out[3].x);
+    if (has_r1) store4(y0 + T, t0 + tl, T, out[0].y, out[1].y, out[2].y, out[3].y);
+  }
+}
+
 __global__ void __launch_bounds__(THREADS, 2)
-activation_kernel(const float *__restrict__ x, float *__restrict__ y, int C, int T,
-                  int tiles_per_row, int n_tiles, const float *__restrict__ log_alpha,
+activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, int C, int T,
+                  int tiles_per_row, long long n_tiles, const float *__restrict__ log_alpha,
                   const float *__restrict__ log_beta, const float *__restrict__ f_up,
                   const float *__restrict__ f_dn, float eps) {
-  __shared__ __align__(16) float xs[2][XS];
-  __shared__ __align__(16) float vs[VS];
-  __shared__ float snake_ab[2];  // a, inv_b of the current tile's channel
-  const int tid = threadIdx.x;
-
-  Taps tp;
-#pragma unroll
-  for (int j = 0; j < 12; ++j) {
-    tp.up2[j] = 2.0f * __ldg(f_up + j);
-    tp.dn[j] = __ldg(f_dn + j);
+  extern __shared__ __align__(16) float smem[];
+  __shared__ __align__(16) float2 taps[24];  // 2 f_up, then f_down, as broadcast pairs
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (threadIdx.x < 24) {
+    const float f =
+        threadIdx.x < 12 ? 2.0f * __ldg(f_up + threadIdx.x) : __ldg(f_dn + threadIdx.x - 12);
+    taps[threadIdx.x] = make_float2(f, f);
   }
-  // the taps as broadcast pairs, formed once for every tile
-  float2 U2[12], D2[12];
-#pragma unroll
-  for (int j = 0; j < 12; ++j) {
-    U2[j] = f2(tp.up2[j]);
-    D2[j] = f2(tp.dn[j]);
-  }
+  __syncthreads();  // the only block-wide barrier
   // |u| <= up_abs * max |x| over the six inputs of either phase
   float up_abs = 0.0f, up_abs1 = 0.0f;
 #pragma unroll
   for (int l = 0; l < 6; ++l) {
-    up_abs += fabsf(tp.up2[2 * l + 1]);
-    up_abs1 += fabsf(tp.up2[2 * l]);
+    up_abs += fabsf(taps[2 * l + 1].x);
+    up_abs1 += fabsf(taps[2 * l].x);
   }
   up_abs = fmaxf(up_abs, up_abs1);
 
-  // tiles are visited as tile_id = blockIdx.x + k gridDim.x; (row, tile) are
-  // carried along incrementally
-  const int step_row = gridDim.x / tiles_per_row, step_tile = gridDim.x % tiles_per_row;
-  int tile_id = blockIdx.x;
-  int row = tile_id / tiles_per_row, tile = tile_id % tiles_per_row;
-  if (tile_id < n_tiles) issue_tile(x + (size_t)row * T, xs[0], tile * TILE, T, tid);
+  float *wsm = smem + (size_t)warp * WARP_FLOATS;
+  float *xs0 = wsm, *xs1 = wsm + XS_FLOATS, *ring = wsm + 2 * XS_FLOATS;
+  float2 *cst = reinterpret_cast<float2 *>(ring + RING_FLOATS);
+
+  // this warp's contiguous range of tiles (row pair * tiles_per_row + tile)
+  const long long nw = (long long)gridDim.x * WARPS;
+  const long long gw = (long long)blockIdx.x * WARPS + warp;
+  const long long beg = gw * n_tiles / nw, end = (gw + 1) * n_tiles / nw;
+  if (beg >= end) return;
+  auto row_ptr = [&](int pr, int which) {
+    const int r = 2 * pr + which;
+    return x + (size_t)(r < rows ? r : rows - 1) * T;
+  };
+  int pair = (int)(beg / tiles_per_row), tile = (int)(beg % tiles_per_row);
+  issue_tile(row_ptr(pair, 0), row_ptr(pair, 1), xs0, tile * TW, T, lane);
   cp_async_commit();
-  int buf = 0;
-  for (; tile_id < n_tiles; tile_id += gridDim.x, buf ^= 1) {
-    int nrow = row + step_row, ntile = tile + step_tile;
-    if (ntile >= tiles_per_row) {
-      ntile -= tiles_per_row;
-      ++nrow;
+  int cur_pair = -1;
+  bool pending = false;  // stage B of the previous tile still to run
+  int p_t0 = 0, rb = 0;
+  for (long long id = beg; id < end; ++id, rb ^= 2 * TW) {
+    const int j = (int)(id - beg);
+    int npair = pair, ntile = tile + 1;
+    if (ntile == tiles_per_row) {
+      ntile = 0;
+      ++npair;
     }
-    if (tile_id + (int)gridDim.x < n_tiles)
-      issue_tile(x + (size_t)nrow * T, xs[buf ^ 1], ntile * TILE, T, tid);
+    __syncwarp();  // the previous iteration's reads of the buffers written below are done
+    if (id + 1 < end)
+      issue_tile(row_ptr(npair, 0), row_ptr(npair, 1), (j & 1) ? xs0 : xs1, ntile * TW, T, lane);
     cp_async_commit();
-    if (tid == 0) {
-      const int c = row % C;
-      snake_ab[0] = expf(__ldg(log_alpha + c));
-      snake_ab[1] = 1.0f / (expf(__ldg(log_beta + c)) + eps);
-    }
-    cp_async_wait<1>();  // this tile's copies are done; the next tile's may be in flight
-    __syncthreads();
-
-    const int t0 = tile * TILE;
-    const float a = snake_ab[0], inv_b = snake_ab[1];
-    const float *xb = xs[buf];
-
-    // ---- stage A: v[2 t0 - 6 + k]; k = 2q + r holds p = t0 - 3 + q and
-    // x[p + r - 3 + k'] sits at xb[2 + q + r + k'].  The thread owns
-    // q in [4 tid, 4 tid + 4) of each half tile.
-    {
-      const int q0 = 4 * tid;
-      float2 X[12];
+    if (pair != cur_pair) {
+      // the row pair's SnakeBeta constants (every lane computes the same values)
+      cur_pair = pair;
+      float *cf = reinterpret_cast<float *>(cst);
+      const int r1 = min(2 * pair + 1, rows - 1);
+      const int c0 = (2 * pair) % C, c1 = r1 % C;
+      const float a0 = expf(__ldg(log_alpha + c0)), a1 = expf(__ldg(log_alpha + c1));
+      const float ib0 = 1.0f / (expf(__ldg(log_beta + c0)) + eps);
+      const float ib1 = 1.0f / (expf(__ldg(log_beta + c1)) + eps);
+      const float sb0 = sqrtf(ib0), sb1 = sqrtf(ib1);
+      if (lane == 0) {
+        cf[2 * kA] = a0 * sin2p::kInvPi;
+        cf[2 * kA + 1] = a1 * sin2p::kInvPi;
 #pragma unroll
-      for (int w = 0; w < 3; ++w) {
-        const float4 lo = *reinterpret_cast<const float4 *>(xb + q0 + 4 * w);
-        const float4 hi = *reinterpret_cast<const float4 *>(xb + HALF + q0 + 4 * w);
-        X[4 * w] = make_float2(lo.x, hi.x);
-        X[4 * w + 1] = make_float2(lo.y, hi.y);
-        X[4 * w + 2] = make_float2(lo.z, hi.z);
-        X[4 * w + 3] = make_float2(lo.w, hi.w);
-      }
-      // every u of this thread is bounded by up_abs times its largest input:
-      // when a times that bound is within sin^2's fast-path limit, the
-      // per-pair range check is skipped (thread-uniform branch)
-      float m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 12; ++j) m = fmaxf(m, fmaxf(fabsf(X[j].x), fabsf(X[j].y)));
-      const bool fast = a * (up_abs * m) <= sin2c::kFastLimit;
-      float2 V[8];
-      auto stage_a = [&](auto check) {
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-#pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            const int b0 = 2 + qq + r;
-            float2 u = mul2(U2[1 - r], X[b0 + 5]);
-#pragma unroll
-            for (int l = 1; l < 6; ++l) u = fma2(U2[2 * l + 1 - r], X[b0 + 5 - l], u);
-            V[2 * qq + r] = snake2<decltype(check)::value>(u, a, inv_b);
-          }
+        for (int q = 0; q < 5; ++q) {
+          cf[2 * (kP + q)] = sin2p::coef(q) * sb0;
+          cf[2 * (kP + q) + 1] = sin2p::coef(q) * sb1;
         }
-      };
-      if (fast)
-        stage_a(std::false_type{});
-      else
-        stage_a(std::true_type{});
-      *reinterpret_cast<float4 *>(vs + vidx(2 * q0)) = make_float4(V[0].x, V[1].x, V[2].x, V[3].x);
-      *reinterpret_cast<float4 *>(vs + vidx(2 * q0 + 4)) =
-          make_float4(V[4].x, V[5].x, V[6].x, V[7].x);
-      *reinterpret_cast<float4 *>(vs + vidx(2 * HALF + 2 * q0)) =
-          make_float4(V[0].y, V[1].y, V[2].y, V[3].y);
-      *reinterpret_cast<float4 *>(vs + vidx(2 * HALF + 2 * q0 + 4)) =
-          make_float4(V[4].y, V[5].y, V[6].y, V[7].y);
-      // k in [2 TILE, 2 TILE + 12): one or two per warp, lane 0 and lane 1
-      if ((tid & 31) < 2 && (tid >> 5) + 8 * (tid & 31) < 12) {
-        const int i = (tid >> 5) + 8 * (tid & 31);
-        const int k = 2 * TILE + i;
-        const int q = k >> 1, r = k & 1;
-        vs[vidx(k)] = snake1(up1(tp, r, xb + 2 + q + r), a, inv_b);
+        cf[2 * kM] = cf[2 * kM + 1] = 12582912.0f;
+        cf[2 * kNeg] = cf[2 * kNeg + 1] = -1.0f;
+        cf[2 * kAraw] = a0;
+        cf[2 * kAraw + 1] = a1;
+        cf[2 * kIb] = ib0;
+        cf[2 * kIb + 1] = ib1;
       }
     }
-    // Near a row end the pages pad the 2x signal by replication: v at an index
-    // m outside [0, 2T-1] is v at the clamped index.  Only m in [-6, -1] and
-    // [2T, 2T + 4] are read by outputs t < T.
-    const bool edge = (2 * t0 - 6 < 0) || (2 * t0 + 2 * TILE + 5 > 2 * T - 1);
-    if (edge) {
-      __syncthreads();
-      if (tid < 11) {
-        const int m = tid < 6 ? tid - 6 : 2 * T + (tid - 6);
-        const int k = m - (2 * t0 - 6);
-        if (k >= 0 && k < 2 * TILE + 12) {
-          const int mc = m < 0 ? 0 : 2 * T - 1;
-          const int p = mc >> 1, r = mc & 1;
-          // x[p + r - 3 + k'] sits at xb[p + r + 5 - t0 + k'] (in range: the tile
-          // reaches that row end)
-          vs[vidx(k)] = snake1(up1(tp, r, xb + (p + r + 5 - t0)), a, inv_b);
-        }
+    cp_async_wait<1>();  // this tile's input has landed (the next one may be in flight)
+    __syncwarp();
+    const float *xb = (j & 1) ? xs1 : xs0;
+    const int t0 = tile * TW;
+    stage_a(xb, ring, rb, taps, cst, up_abs, lane);
+    __syncwarp();
+    // Replicate padding of the 2x signal: v[m] for m in [-5, -1] is v[0], for
+    // m in [2T, 2T + 4] it is v[2T - 1] (slot s = m - 2 t0 + 5; only m up to
+    // 2T + 4 are read).  The slots below 2 TW are fixed here, before the
+    // previous tile's stage B reads the first 10 of them.
+    const bool row_end = tile == tiles_per_row - 1;
+    const bool edge_r = T <= t0 + TW + 2;  // the tile's outputs read v[2T..]
+    const int s_end = 2 * (T - t0) + 4;    // slot of v[2T - 1]
+    if (t0 == 0 || edge_r) {
+      if (lane < 5) {
+        if (t0 == 0)
+          *reinterpret_cast<float2 *>(ring + voff(rb + lane)) =
+              *reinterpret_cast<const float2 *>(ring + voff(rb + 5));
+        if (edge_r && s_end + 1 + lane < 2 * TW)
+          *reinterpret_cast<float2 *>(ring + voff(rb + s_end + 1 + lane)) =
+              *reinterpret_cast<const float2 *>(ring + voff(rb + s_end));
       }
+      __syncwarp();
     }
-    __syncthreads();
-
-    // ---- stage B: y[t] = sum_j f_dn[j] v[2t + j - 5]; v[2t + j - 5] is vs[2 (t - t0) + j + 1]
-    {
-      const int tl = 4 * tid;
-      float2 W[20];
-#pragma unroll
-      for (int w = 0; w < 5; ++w) {
-        const float4 lo = *reinterpret_cast<const float4 *>(vs + vidx(2 * tl + 4 * w));
-        const float4 hi = *reinterpret_cast<const float4 *>(vs + vidx(2 * HALF + 2 * tl + 4 * w));
-        W[4 * w] = make_float2(lo.x, hi.x);
-        W[4 * w + 1] = make_float2(lo.y, hi.y);
-        W[4 * w + 2] = make_float2(lo.z, hi.z);
-        W[4 * w + 3] = make_float2(lo.w, hi.w);
+    float *yp = y + (size_t)(2 * pair) * T;
+    const bool has_r1 = 2 * pair + 1 < rows;
+    if (pending) stage_b(ring, rb ^ (2 * TW), taps, yp, has_r1, p_t0, T, lane);
+    if (row_end || id + 1 == end) {
+      // stage B of this tile now: its last 10 values come from its own window
+      __syncwarp();
+      stage_a_tail(xb, ring, rb, taps, cst, lane);
+      __syncwarp();
+      if (edge_r && lane < 5) {
+        const int s = s_end + 1 + lane;
+        if (s >= 2 * TW && s < 2 * TW + 10)
+          *reinterpret_cast<float2 *>(ring + voff((rb + s) & (RING - 1))) =
+              *reinterpret_cast<const float2 *>(ring + voff((rb + s_end) & (RING - 1)));
       }
-      float2 out[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float2 acc = mul2(D2[0], W[2 * e + 1]);
-#pragma unroll
-        for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j + 1], acc);
-        out[e] = acc;
-      }
-      float *yr = y + (size_t)row * T;
-      store4(yr, t0 + tl, T, out[0].x, out[1].x, out[2].x, out[3].x);
-      store4(yr, t0 + HALF + tl, T, out[0].y, out[1].y, out[2].y, out[3].y);
+      __syncwarp();
+      stage_b(ring, rb, taps, yp, has_r1, t0, T, lane);
+      pending = false;
+    } else {
+      pending = true;
+      p_t0 = t0;
     }
-    row = nrow;
+    pair = npair;
     tile = ntile;
   }
   cp_async_wait<0>();
@@ -320,7 +446,8 @@ int persistent_ctas() {
     int dev = 0, sms = 148, per_sm = 4;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_kernel, THREADS, 0) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_kernel, THREADS,
+                                                      SMEM_BYTES) !=
             cudaSuccess ||
         per_sm < 1)
       per_sm = 4;
@@ -344,16 +471,25 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
                             const float *lb, const float *fu, const float *fd, float eps,
                             cudaStream_t st) {
   const long long rows = (long long)B * C;
-  const int tiles = (T + TILE - 1) / TILE;
-  const long long n_tiles = rows * tiles;
+  const int tiles = (T + TW - 1) / TW;
+  const long long n_tiles = (rows + 1) / 2 * tiles;
   if (n_tiles <= 0) return BV_OK;
-  if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "activation: too many tiles");
-  const int ctas = persistent_ctas();
-  const long long grid = n_tiles < ctas ? n_tiles : ctas;
+  if (rows > 0x7fffffffLL || (rows + 1) / 2 > 0x7fffffffLL / 2)
+    return fail(BV_ERR_SHAPE, "activation: too many rows");
+  static bool configured = false;
+  if (!configured) {
+    if (cudaFuncSetAttribute(activation_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)SMEM_BYTES) != cudaSuccess)
+      return check_launch("activation smem attribute");
+    configured = true;
+  }
+  const long long ctas = persistent_ctas();
+  const long long need = (n_tiles + WARPS - 1) / WARPS;
+  const long long grid = need < ctas ? need : ctas;
   {
     LaunchTimer tm(st, "activation", 0.0, 8.0 * (double)rows * T);
-    activation_kernel<<<(unsigned)grid, THREADS, 0, st>>>(x, y, C, T, tiles, (int)n_tiles, la,
-                                                          lb, fu, fd, eps);
+    activation_kernel<<<(unsigned)grid, THREADS, SMEM_BYTES, st>>>(
+        x, y, (int)rows, C, T, tiles, n_tiles, la, lb, fu, fd, eps);
   }
   count_launch();
   return check_launch("activation_kernel");
