@@ -21,12 +21,12 @@
 // Every warp runs on its own, with no block-wide barrier: it owns a
 // contiguous range of warp tiles (row pair by row pair, left to right) and
 // its own shared memory -- a double buffer of input windows, filled with
-// cp.async one tile ahead, and a ring of two 2x-rate buffers.  Stage A of
-// tile j computes v[2 t0 - 5 + s], s < 2 TW, into the ring; stage B of tile j
-// also needs the first 10 values of tile j + 1, so it runs after stage A of
-// tile j + 1.  Only at the end of a row (replicate padding) or of the warp's
-// range does stage B follow its own stage A, after computing those 10 values
-// directly.
+// cp.async one tile ahead, and two 2x-rate buffers.  Stage A of tile j
+// computes v[2 t0 - 5 + s], s < 2 TW, into its buffer; stage B of tile j also
+// needs the first 10 values of tile j + 1 (slots 2 TW .. 2 TW + 9), so it runs
+// after stage A of tile j + 1, which writes those values into both buffers.
+// Only at the end of a row (replicate padding) or of the warp's range does
+// stage B follow its own stage A, after computing those 10 values directly.
 //
 // SnakeBeta's sin^2 runs in units of pi: w = u a/pi, f = w - rint(w) in
 // [-1/2, 1/2] (exact), and sin(pi f) = f P(f^2) with a degree-4 polynomial P
@@ -42,30 +42,26 @@ namespace {
 
 constexpr int WARPS = 8;          // per CTA
 constexpr int THREADS = 32 * WARPS;
-constexpr int TW = 256;           // outputs per row of a warp tile
+constexpr int TW = 128;           // outputs per row of a warp tile (4 per lane)
 constexpr int XP = TW + 16;       // input pairs x[t0 - 8 + i] of a warp tile
-constexpr int RING = 4 * TW;      // 2x-rate ring: two tiles of 2 TW pairs
-constexpr int XS_FLOATS = 2 * XP;
-constexpr int RING_FLOATS = 2 * RING;
-constexpr int WARP_FLOATS = 2 * XS_FLOATS + RING_FLOATS + 2 * 10;
-constexpr size_t SMEM_BYTES = (size_t)WARPS * WARP_FLOATS * sizeof(float);
-static_assert(TW == 2 * 4 * 32, "two passes of 4 outputs per lane");
-static_assert(XP % 16 == 0 && RING % 16 == 0, "whole swizzle blocks");
+constexpr int VP = 2 * TW + 10;   // 2x-rate pairs v[2 t0 - 5 + s] of a warp tile
 
-// Shared-memory float offsets of pair i.  A 16-byte chunk holds two pairs;
-// chunks are XOR-swizzled inside blocks of 8 so that the 16-byte accesses of
-// a quarter warp hit 8 distinct bank groups.  Input pairs: stage A's lanes are
-// 2 chunks apart, and bit 3 of the chunk index flips bit 0.  2x-rate pairs:
-// stages A and B have lanes 4 chunks apart, and bits 3-4 of the chunk index
-// flip bits 0-1.
-__device__ __forceinline__ int xoff(int i) {
-  const int ch = i >> 1;
-  return 4 * (ch ^ ((ch >> 3) & 1)) + 2 * (i & 1);
-}
-__device__ __forceinline__ int voff(int s) {
-  const int ch = s >> 1;
-  return 4 * (ch ^ ((ch >> 3) & 3)) + 2 * (s & 1);
-}
+// Shared-memory float offsets of pair i.  A 16-byte chunk c holds two pairs;
+// the chunks are padded so that the 16-byte accesses of a quarter warp hit 8
+// distinct bank groups while the address stays linear in the lane:
+//   input pairs: stage A's lanes are 2 chunks apart; chunk c at c + c/2,
+//     so lane L's chunks start at 3L (3L mod 8 distinct over 8 lanes);
+//   2x-rate pairs: stages A and B have lanes 4 chunks apart; chunk c at
+//     c + c/4, lane L's chunks start at 5L.
+__host__ __device__ constexpr int xoff(int i) { return 4 * ((i >> 1) + (i >> 2)) + 2 * (i & 1); }
+__host__ __device__ constexpr int voff(int s) { return 4 * ((s >> 1) + (s >> 3)) + 2 * (s & 1); }
+constexpr int XS_FLOATS = xoff(XP - 1) + 2;
+constexpr int VS_FLOATS = voff(VP - 1) + 2;
+constexpr int WARP_FLOATS = 2 * XS_FLOATS + 2 * VS_FLOATS + 2 * 10;
+constexpr size_t SMEM_BYTES = (size_t)WARPS * WARP_FLOATS * sizeof(float);
+static_assert(TW == 4 * 32, "4 outputs per lane");
+static_assert(XS_FLOATS % 4 == 0 && VS_FLOATS % 4 == 0 && WARP_FLOATS % 4 == 0, "16-byte alignment");
+static_assert(xoff(32) == xoff(0) + 96 && voff(2 * TW) == 640, "linear layouts");
 
 // |w| bound of the fast path: far inside the 2^22 where rint by adding and
 // removing 1.5 * 2^23 stays exact; |a u| <= pi * 16384 = 51472.
@@ -89,6 +85,22 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a
 struct Snake {
   float2 A, P[5], M, Neg;
 };
+
+__device__ __forceinline__ void load_snake(Snake &k, const float2 *cst) {
+  const float4 *c4 = reinterpret_cast<const float4 *>(cst);
+  float4 v = c4[0];
+  k.A = make_float2(v.x, v.y);
+  k.P[0] = make_float2(v.z, v.w);
+  v = c4[1];
+  k.P[1] = make_float2(v.x, v.y);
+  k.P[2] = make_float2(v.z, v.w);
+  v = c4[2];
+  k.P[3] = make_float2(v.x, v.y);
+  k.P[4] = make_float2(v.z, v.w);
+  v = c4[3];
+  k.M = make_float2(v.x, v.y);
+  k.Neg = make_float2(v.z, v.w);
+}
 
 // Paired SnakeBeta for the two rows.  CHECK: range-check |w| per pair and
 // take the scalar sin^2 of sin2.cuh (Cody-Waite reduction, sinf beyond its
@@ -138,30 +150,30 @@ __device__ __forceinline__ void cp_async_wait() {
 
 // Issue the copies of one warp tile's input: pair i = (x0[t0 - 8 + i],
 // x1[t0 - 8 + i]), positions clamped to [0, T).  Lane L copies pairs L + 32 j
-// of each row (j < 9, the last only for L < 16).
+// of each row (j < 5, the last only for L < 16).
 __device__ __forceinline__ void issue_tile(const float *__restrict__ x0,
                                            const float *__restrict__ x1, float *xs, int t0, int T,
                                            int lane) {
-  float *d = xs + xoff(lane);  // xoff(L + 32 j) = xoff(L) + 64 j
+  float *d = xs + xoff(lane);  // xoff(L + 32 j) = xoff(L) + 96 j
   const int base = t0 - 8 + lane;
   if (t0 >= 8 && t0 - 8 + XP <= T) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      cp_async4(d + 64 * j, x0 + base + 32 * j);
-      cp_async4(d + 64 * j + 1, x1 + base + 32 * j);
+    for (int j = 0; j < 4; ++j) {
+      cp_async4(d + 96 * j, x0 + base + 32 * j);
+      cp_async4(d + 96 * j + 1, x1 + base + 32 * j);
     }
-    if (lane < XP - 256) {
-      cp_async4(d + 512, x0 + base + 256);
-      cp_async4(d + 513, x1 + base + 256);
+    if (lane < XP - 128) {
+      cp_async4(d + 384, x0 + base + 128);
+      cp_async4(d + 385, x1 + base + 128);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 9; ++j) {
-      if (j < 8 || lane < XP - 256) {
+    for (int j = 0; j < 5; ++j) {
+      if (j < 4 || lane < XP - 128) {
         int p = base + 32 * j;
         p = p < 0 ? 0 : (p > T - 1 ? T - 1 : p);
-        cp_async4(d + 64 * j, x0 + p);
-        cp_async4(d + 64 * j + 1, x1 + p);
+        cp_async4(d + 96 * j, x0 + p);
+        cp_async4(d + 96 * j + 1, x1 + p);
       }
     }
   }
@@ -188,118 +200,101 @@ __device__ __forceinline__ void load_taps(float2 (&F)[12], const float2 *taps) {
   }
 }
 
-// Stage A of one warp tile: the lane's 2x-rate pairs s = 256 h + 8 L + n
-// (pass h < 2, n < 8), i.e. k = s + 1 = 2q + r from (q0, 1) to (q0 + 4, 0)
-// with q0 = 128 h + 4 L relative to t0 - 3; their inputs are the pairs
-// q0 + 3 .. q0 + 11 (X[j] = pair q0 + 2 + j).  Ring slot of s: rb + s.
-__device__ __forceinline__ void stage_a(const float *xb, float *ring, int rb, const float2 *taps,
-                                        const float2 *cst, float up_abs, int lane) {
+// Stage A of one warp tile: lane L's 2x-rate pairs s = 8 L + n, n < 8, i.e.
+// k = s + 1 = 2q + r from (q0, 1) to (q0 + 4, 0) with q0 = 4 L relative to
+// t0 - 3; their inputs are the pairs q0 + 3 .. q0 + 11 (X[j] = pair q0 + 2 + j,
+// whose chunks start at 3 L + 1 in the padded layout).  The slots s < 10 are
+// written to the other buffer's slots s + 2 TW too (mirror), where the
+// previous tile's stage B reads them.
+__device__ __forceinline__ void stage_a(const float *xb, float *vb, float *vmirror,
+                                        const float2 *taps, const float2 *cst, float up_abs,
+                                        int lane) {
   float2 U2[12];
   load_taps(U2, taps);
   Snake k;
-  {
-    const float4 *c4 = reinterpret_cast<const float4 *>(cst);
-    float4 v = c4[0];
-    k.A = make_float2(v.x, v.y);
-    k.P[0] = make_float2(v.z, v.w);
-    v = c4[1];
-    k.P[1] = make_float2(v.x, v.y);
-    k.P[2] = make_float2(v.z, v.w);
-    v = c4[2];
-    k.P[3] = make_float2(v.x, v.y);
-    k.P[4] = make_float2(v.z, v.w);
-    v = c4[3];
-    k.M = make_float2(v.x, v.y);
-    k.Neg = make_float2(v.z, v.w);
-  }
-  const float bound = up_abs * fmaxf(k.A.x, k.A.y);
-#pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    const int q0 = 128 * h + 4 * lane;
-    float2 X[10];
+  load_snake(k, cst);
+  float2 X[10];
+  const float *xl = xb + 12 * lane;  // xoff(4L + 2 + 2m) = 12 L + 4 (1 + m + (1 + m) / 2)
 #pragma unroll
-    for (int m = 0; m < 5; ++m) {
-      const float4 v = *reinterpret_cast<const float4 *>(xb + xoff(q0 + 2 + 2 * m));
-      X[2 * m] = make_float2(v.x, v.y);
-      X[2 * m + 1] = make_float2(v.z, v.w);
+  for (int m = 0; m < 5; ++m) {
+    const float4 v = *reinterpret_cast<const float4 *>(xl + 4 * (1 + m + (1 + m) / 2));
+    X[2 * m] = make_float2(v.x, v.y);
+    X[2 * m + 1] = make_float2(v.z, v.w);
+  }
+  // every u of this lane is bounded by up_abs times its largest input: when
+  // that keeps |w| within the fast path, the per-pair range check is skipped
+  // (lane-uniform branch)
+  float mx = 0.0f;
+#pragma unroll
+  for (int j = 1; j < 10; ++j) mx = fmaxf(mx, fmaxf(fabsf(X[j].x), fabsf(X[j].y)));
+  float *vl = vb + 20 * lane;  // voff(8L + n) = 20 L + 2n
+  auto run = [&](auto check) {
+    constexpr bool CK = decltype(check)::value;
+#pragma unroll
+    for (int n = 0; n < 8; n += 2) {
+      // n (even): phase 1 at q0 + n/2; n + 1: phase 0 at q0 + n/2 + 1; both
+      // read the input pairs X[n/2 + 1 ..]
+      const float2 v0 = snake2<CK>(up2<1>(U2, X + n / 2 + 1), k, cst);
+      const float2 v1 = snake2<CK>(up2<0>(U2, X + n / 2 + 1), k, cst);
+      const float4 o = make_float4(v0.x, v0.y, v1.x, v1.y);
+      *reinterpret_cast<float4 *>(vl + 2 * n) = o;
+      if (8 * lane + n < 10) *reinterpret_cast<float4 *>(vmirror + voff(8 * lane + n + 2 * TW)) = o;
     }
-    // every u of this lane is bounded by up_abs times its largest input:
-    // when that keeps |w| within the fast path, the per-pair range check is
-    // skipped (lane-uniform branch)
-    float mx = 0.0f;
-#pragma unroll
-    for (int j = 1; j < 10; ++j) mx = fmaxf(mx, fmaxf(fabsf(X[j].x), fabsf(X[j].y)));
-    auto run = [&](auto check) {
-      constexpr bool CK = decltype(check)::value;
-#pragma unroll
-      for (int n = 0; n < 8; n += 2) {
-        // n (even): phase 1 at q0 + n/2; n + 1: phase 0 at q0 + n/2 + 1; both
-        // read the input pairs X[n/2 + 1 ..]
-        const float2 v0 = snake2<CK>(up2<1>(U2, X + n / 2 + 1), k, cst);
-        const float2 v1 = snake2<CK>(up2<0>(U2, X + n / 2 + 1), k, cst);
-        *reinterpret_cast<float4 *>(ring + voff((rb + 2 * q0 + n) & (RING - 1))) =
-            make_float4(v0.x, v0.y, v1.x, v1.y);
-      }
-    };
-    if (mx * bound <= kWLimit)
-      run(std::false_type{});
-    else
-      run(std::true_type{});
-  }
+  };
+  if (mx * up_abs * fmaxf(k.A.x, k.A.y) <= kWLimit)
+    run(std::false_type{});
+  else
+    run(std::true_type{});
 }
 
 // The 10 pairs s in [2 TW, 2 TW + 10) of a tile, from its own input window:
 // k = s + 1 = 2 TW + 1 + i; lanes 0-4 take phase 1 (q = TW + L), lanes 5-9
 // phase 0 (q = TW + L - 4).
-__device__ __forceinline__ void stage_a_tail(const float *xb, float *ring, int rb,
-                                             const float2 *taps, const float2 *cst, int lane) {
+__device__ __forceinline__ void stage_a_tail(const float *xb, float *vb, const float2 *taps,
+                                             const float2 *cst, int lane) {
   if (lane >= 10) return;
   float2 U2[12];
   load_taps(U2, taps);
   Snake k;
-  k.A = cst[kA];
-#pragma unroll
-  for (int j = 0; j < 5; ++j) k.P[j] = cst[kP + j];
-  k.M = cst[kM];
-  k.Neg = cst[kNeg];
+  load_snake(k, cst);
   const int R = lane < 5 ? 1 : 0;
   const int q = lane < 5 ? TW + lane : TW + lane - 4;
   float2 xp[6];
 #pragma unroll
   for (int j = 0; j < 6; ++j) xp[j] = *reinterpret_cast<const float2 *>(xb + xoff(2 + q + R + j));
   const float2 u = R ? up2<1>(U2, xp) : up2<0>(U2, xp);
-  *reinterpret_cast<float2 *>(ring + voff((rb + 2 * q + R - 1) & (RING - 1))) =
-      snake2<true>(u, k, cst);
+  *reinterpret_cast<float2 *>(vb + voff(2 * q + R - 1)) = snake2<true>(u, k, cst);
 }
 
 // Stage B of one warp tile: y[t] = sum_j f_dn[j] v[2t + j - 5] with
-// v[2t + j - 5] at s = 2 (t - t0) + j; lane L writes t = t0 + 128 h + 4 L + e.
-__device__ __forceinline__ void stage_b(const float *ring, int rb, const float2 *taps,
-                                        float *y0, bool has_r1, int t0, int T, int lane) {
+// v[2t + j - 5] at s = 2 (t - t0) + j; lane L writes t = t0 + 4 L + e.
+__device__ __forceinline__ void stage_b(const float *vb, const float2 *taps, float *y0,
+                                        bool has_r1, int t0, int T, int lane) {
   float2 D2[12];
   load_taps(D2, taps + 12);
-#pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    const int tl = 128 * h + 4 * lane;
-    float2 W[18];
+  float2 W[18];
+  const float *vl = vb + 20 * lane;  // voff(8L + 2m) = 20 L + 4 (m + m / 4)
 #pragma unroll
-    for (int m = 0; m < 9; ++m) {
-      const float4 v =
-          *reinterpret_cast<const float4 *>(ring + voff((rb + 2 * tl + 2 * m) & (RING - 1)));
-      W[2 * m] = make_float2(v.x, v.y);
-      W[2 * m + 1] = make_float2(v.z, v.w);
-    }
-    float2 out[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      float2 acc = mul2(D2[0], W[2 * e]);
-#pragma unroll
-      for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j], acc);
-      out[e] = acc;
-    }
-    store4(y0, t0 + tl, T, out[0].x, out[1].x, out[2].x, out[3].x);
-    if (has_r1) store4(y0 + T, t0 + tl, T, out[0].y, out[1].y, out[2].y, out[3].y);
+  for (int m = 0; m < 9; ++m) {
+    const float4 v = *reinterpret_cast<const float4 *>(vl + 4 * (m + m / 4));
+    W[2 * m] = make_float2(v.x, v.y);
+    W[2 * m + 1] = make_float2(v.z, v.w);
   }
+  float2 out[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 acc = mul2(D2[0], W[2 * e]);
+#pragma unroll
+    for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j], acc);
+    out[e] = acc;
+  }
+  const int t = t0 + 4 * lane;
+  store4(y0, t, T, out[0].x, out[1].x, out[2].x, out[3].x);
+  if (has_r1) store4(y0 + T, t, T, out[0].y, out[1].y, out[2].y, out[3].y);
+}
+
+__device__ __forceinline__ void copy_pair(float *vb, int dst, int src) {
+  *reinterpret_cast<float2 *>(vb + voff(dst)) = *reinterpret_cast<const float2 *>(vb + voff(src));
 }
 
 __global__ void __launch_bounds__(THREADS, 2)
@@ -326,8 +321,8 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
   up_abs = fmaxf(up_abs, up_abs1);
 
   float *wsm = smem + (size_t)warp * WARP_FLOATS;
-  float *xs0 = wsm, *xs1 = wsm + XS_FLOATS, *ring = wsm + 2 * XS_FLOATS;
-  float2 *cst = reinterpret_cast<float2 *>(ring + RING_FLOATS);
+  float *const xs0 = wsm, *const vs0 = wsm + 2 * XS_FLOATS;  // buffer b at + b * size
+  float2 *cst = reinterpret_cast<float2 *>(wsm + 2 * XS_FLOATS + 2 * VS_FLOATS);
 
   // this warp's contiguous range of tiles (row pair * tiles_per_row + tile)
   const long long nw = (long long)gridDim.x * WARPS;
@@ -343,9 +338,9 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
   cp_async_commit();
   int cur_pair = -1;
   bool pending = false;  // stage B of the previous tile still to run
-  int p_t0 = 0, rb = 0;
-  for (long long id = beg; id < end; ++id, rb ^= 2 * TW) {
-    const int j = (int)(id - beg);
+  int p_t0 = 0;
+  for (long long id = beg; id < end; ++id) {
+    const int b = (int)((id - beg) & 1);
     int npair = pair, ntile = tile + 1;
     if (ntile == tiles_per_row) {
       ntile = 0;
@@ -353,7 +348,8 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
     }
     __syncwarp();  // the previous iteration's reads of the buffers written below are done
     if (id + 1 < end)
-      issue_tile(row_ptr(npair, 0), row_ptr(npair, 1), (j & 1) ? xs0 : xs1, ntile * TW, T, lane);
+      issue_tile(row_ptr(npair, 0), row_ptr(npair, 1), xs0 + (b ^ 1) * XS_FLOATS, ntile * TW, T,
+                 lane);
     cp_async_commit();
     if (pair != cur_pair) {
       // the row pair's SnakeBeta constants (every lane computes the same values)
@@ -383,44 +379,44 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
     }
     cp_async_wait<1>();  // this tile's input has landed (the next one may be in flight)
     __syncwarp();
-    const float *xb = (j & 1) ? xs1 : xs0;
     const int t0 = tile * TW;
-    stage_a(xb, ring, rb, taps, cst, up_abs, lane);
+    const float *xb = xs0 + b * XS_FLOATS;
+    float *vb = vs0 + b * VS_FLOATS, *vo = vs0 + (b ^ 1) * VS_FLOATS;
+    stage_a(xb, vb, vo, taps, cst, up_abs, lane);
     __syncwarp();
     // Replicate padding of the 2x signal: v[m] for m in [-5, -1] is v[0], for
     // m in [2T, 2T + 4] it is v[2T - 1] (slot s = m - 2 t0 + 5; only m up to
-    // 2T + 4 are read).  The slots below 2 TW are fixed here, before the
-    // previous tile's stage B reads the first 10 of them.
+    // 2T + 4 are read).  The slots below 2 TW are fixed here (and mirrored,
+    // below 10), before the previous tile's stage B reads the first 10.
     const bool row_end = tile == tiles_per_row - 1;
     const bool edge_r = T <= t0 + TW + 2;  // the tile's outputs read v[2T..]
     const int s_end = 2 * (T - t0) + 4;    // slot of v[2T - 1]
     if (t0 == 0 || edge_r) {
       if (lane < 5) {
-        if (t0 == 0)
-          *reinterpret_cast<float2 *>(ring + voff(rb + lane)) =
-              *reinterpret_cast<const float2 *>(ring + voff(rb + 5));
-        if (edge_r && s_end + 1 + lane < 2 * TW)
-          *reinterpret_cast<float2 *>(ring + voff(rb + s_end + 1 + lane)) =
-              *reinterpret_cast<const float2 *>(ring + voff(rb + s_end));
+        if (t0 == 0) copy_pair(vb, lane, 5);
+        const int s = s_end + 1 + lane;
+        if (edge_r && s < 2 * TW) {
+          copy_pair(vb, s, s_end);
+          if (s < 10)
+            *reinterpret_cast<float2 *>(vo + voff(s + 2 * TW)) =
+                *reinterpret_cast<const float2 *>(vb + voff(s_end));
+        }
       }
       __syncwarp();
     }
     float *yp = y + (size_t)(2 * pair) * T;
     const bool has_r1 = 2 * pair + 1 < rows;
-    if (pending) stage_b(ring, rb ^ (2 * TW), taps, yp, has_r1, p_t0, T, lane);
+    if (pending) stage_b(vo, taps, yp, has_r1, p_t0, T, lane);
     if (row_end || id + 1 == end) {
       // stage B of this tile now: its last 10 values come from its own window
-      __syncwarp();
-      stage_a_tail(xb, ring, rb, taps, cst, lane);
+      stage_a_tail(xb, vb, taps, cst, lane);
       __syncwarp();
       if (edge_r && lane < 5) {
         const int s = s_end + 1 + lane;
-        if (s >= 2 * TW && s < 2 * TW + 10)
-          *reinterpret_cast<float2 *>(ring + voff((rb + s) & (RING - 1))) =
-              *reinterpret_cast<const float2 *>(ring + voff((rb + s_end) & (RING - 1)));
+        if (s >= 2 * TW && s < VP) copy_pair(vb, s, s_end);
       }
       __syncwarp();
-      stage_b(ring, rb, taps, yp, has_r1, t0, T, lane);
+      stage_b(vb, taps, yp, has_r1, t0, T, lane);
       pending = false;
     } else {
       pending = true;
