@@ -30,8 +30,8 @@ constexpr float kFastLimit = 65536.0f;
 // sin(pi f) for |f| <= 1/2 as f P(f^2), P of degree 4: coefficients of a
 // near-minimax fit of sin(pi f) / f in s = f^2 on [0, 1/4] (least squares on
 // Chebyshev nodes, reweighted by Lawson's iteration towards the minimax
-// error), rounded to float.  Approximation error below 3.4e-9 in sin(pi f);
-// evaluated by Horner's rule in float the total stays within 2e-7.
+// error), rounded to float.  Approximation error 3.4e-9 before and 4.9e-8
+// after the rounding; evaluated by Horner's rule in float, within 2.5e-7.
 namespace sin2p {
 constexpr float kInvPi = 0.31830987334251404f;  // float(1/pi)
 __host__ __device__ constexpr float coef(int j) {

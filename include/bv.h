@@ -123,11 +123,13 @@ bv_status bv_activation1d(const float *x, float *y, int B, int C, int T,
                           const float *up_filter, const float *down_filter,
                           float eps, void *stream);
 
-/* The sin^2 the activation kernel evaluates for SnakeBeta, elementwise on n
- * device floats (out may equal z): exposed so its accuracy can be tested.
- * Method: additive reduction by pi (sin^2 has period pi) with pi split in
- * three floats (Cody & Waite), then the Taylor series of sin to r^13 on
- * |r| <= pi/2, squared; |z| > 65536 uses sinf. */
+/* The scalar sin^2 of the activation kernel, elementwise on n device floats
+ * (out may equal z): exposed so its accuracy can be tested.  The activation
+ * takes it for arguments past its fast path (|a u| > 51472; the fast path
+ * works in units of pi with a degree-4 polynomial and is covered by the
+ * activation's parity tests).  Method: additive reduction by pi (sin^2 has
+ * period pi) with pi split in three floats (Cody & Waite), then the Taylor
+ * series of sin to r^13 on |r| <= pi/2, squared; |z| > 65536 uses sinf. */
 bv_status bv_sin_squared(const float *z, float *out, int64_t n, void *stream);
 
 /* Epilogue fused into the convolutions.  With v = conv(x) + bias:
