@@ -25,6 +25,15 @@ constexpr int SM_PER = 4;        // consecutive outputs per thread
 constexpr int SM_THREADS = SM_T / SM_PER;
 constexpr int SM_MAX_C = 32;
 
+// 4-byte asynchronous copy global -> shared; when !ok nothing is read and the
+// destination is zero-filled (src must still be a valid address)
+__device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool ok) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src),
+               "r"(ok ? 4 : 0)
+               : "memory");
+}
+
 // COUT: output channels rounded up to a multiple of 4; KT: the kernel size
 // when fixed at compile time, 0 for a runtime K
 template <int COUT, int KT>
@@ -43,18 +52,24 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
   const int t0 = blockIdx.x * SM_T, b = blockIdx.y;
   const int tid = threadIdx.x;
 
+  // staging through cp.async, zero-filled where nothing is read: every copy
+  // of the thread is in flight at once instead of one load latency each
   for (int idx = tid; idx < Cin * K * COUT; idx += SM_THREADS) {
     const int o = idx % COUT, ij = idx / COUT;
     const int i = ij / K, j = ij - i * K;
-    ws[idx] = o < Cout ? __ldg(w + ((size_t)o * Cin + i) * K + j) : 0.0f;
+    const bool ok = o < Cout;
+    cp_async4_zfill(ws + idx, ok ? w + ((size_t)o * Cin + i) * K + j : w, ok);
   }
   const float *xb = x + (size_t)b * Cin * T;
   for (int idx = tid; idx < Cin * XW; idx += SM_THREADS) {
     const int i = idx / XW, n = idx - i * XW;
     const int t = t0 - pad + n;
-    xs[idx] = (t >= 0 && t < T && n < SM_T + halo) ? __ldg(xb + (size_t)i * T + t) : 0.0f;
+    const bool ok = t >= 0 && t < T && n < SM_T + halo;
+    cp_async4_zfill(xs + idx, ok ? xb + (size_t)i * T + t : xb, ok);
   }
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
   if (tid < COUT) bias_s[tid] = (bias && tid < Cout) ? __ldg(bias + tid) : 0.0f;
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
   __syncthreads();
 
   const int tl = SM_PER * tid;  // this thread's outputs t0 + tl .. t0 + tl + SM_PER - 1
