@@ -40,6 +40,21 @@ class LaunchTimer {
 
 inline cudaStream_t as_stream(void *s) { return reinterpret_cast<cudaStream_t>(s); }
 
+// 4-byte asynchronous copy global -> shared (cp.async); when !ok nothing is
+// read and the destination is zero-filled (src must still be a valid
+// address).  Staging loops issue these back to back, so all of a thread's
+// copies are in flight at once; cp_async_wait_all() then completes them.
+__device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool ok) {
+  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src),
+               "r"(ok ? 4 : 0)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n" ::: "memory");
+  asm volatile("cp.async.wait_all;\n" ::: "memory");
+}
+
 // [a, a+na) and [b, b+nb) (in floats) overlap?
 inline bool overlaps(const float *a, size_t na, const float *b, size_t nb) {
   const char *a0 = reinterpret_cast<const char *>(a), *b0 = reinterpret_cast<const char *>(b);

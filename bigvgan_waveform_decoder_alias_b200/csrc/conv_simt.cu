@@ -57,23 +57,24 @@ conv1d_simt_kernel(const float *__restrict__ x, const float *__restrict__ w,
     for (int q = 0; q < TN; ++q) acc[i][q] = 0.0f;
 
   for (int i0 = 0; i0 < Cin; i0 += CK) {
-    // stage the input rows (zero outside [0, T) and beyond Cin)
+    // stage the input rows (zero outside [0, T) and beyond Cin) through
+    // cp.async, all of a thread's copies in flight at once
     for (int idx = tid; idx < CK * W; idx += Cfg::THREADS) {
       const int ci = idx / W, n = idx - ci * W;
       const int tin = t0 - pad + n;
-      float v = 0.0f;
-      if (i0 + ci < Cin && tin >= 0 && tin < T) v = __ldg(xb + (size_t)(i0 + ci) * T + tin);
-      xs[idx] = v;
+      const bool ok = i0 + ci < Cin && tin >= 0 && tin < T;
+      cp_async4_zfill(xs + idx, ok ? xb + (size_t)(i0 + ci) * T + tin : xb, ok);
     }
     // stage the weights as [ci][j][m]; global order (m, ci, j) is contiguous in (ci, j)
     const int KC = CK * K;
     for (int idx = tid; idx < BM * KC; idx += Cfg::THREADS) {
       const int m = idx / KC, r = idx - m * KC;
       const int ci = r / K, j = r - ci * K;
-      float v = 0.0f;
-      if (m0 + m < Cout && i0 + ci < Cin) v = __ldg(w + ((size_t)(m0 + m) * Cin + i0 + ci) * K + j);
-      ws[(ci * K + j) * Cfg::WS_PITCH + m] = v;
+      const bool ok = m0 + m < Cout && i0 + ci < Cin;
+      cp_async4_zfill(ws + (ci * K + j) * Cfg::WS_PITCH + m,
+                      ok ? w + ((size_t)(m0 + m) * Cin + i0 + ci) * K + j : w, ok);
     }
+    cp_async_wait_all();
     __syncthreads();
 
     for (int ci = 0; ci < CK; ++ci) {

@@ -25,15 +25,6 @@ constexpr int SM_PER = 4;        // consecutive outputs per thread
 constexpr int SM_THREADS = SM_T / SM_PER;
 constexpr int SM_MAX_C = 32;
 
-// 4-byte asynchronous copy global -> shared; when !ok nothing is read and the
-// destination is zero-filled (src must still be a valid address)
-__device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool ok) {
-  const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src),
-               "r"(ok ? 4 : 0)
-               : "memory");
-}
-
 // COUT: output channels rounded up to a multiple of 4; KT: the kernel size
 // when fixed at compile time, 0 for a runtime K
 template <int COUT, int KT>
@@ -67,9 +58,8 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
     const bool ok = t >= 0 && t < T && n < SM_T + halo;
     cp_async4_zfill(xs + idx, ok ? xb + (size_t)i * T + t : xb, ok);
   }
-  asm volatile("cp.async.commit_group;\n" ::: "memory");
   if (tid < COUT) bias_s[tid] = (bias && tid < Cout) ? __ldg(bias + tid) : 0.0f;
-  asm volatile("cp.async.wait_all;\n" ::: "memory");
+  cp_async_wait_all();
   __syncthreads();
 
   const int tl = SM_PER * tid;  // this thread's outputs t0 + tl .. t0 + tl + SM_PER - 1

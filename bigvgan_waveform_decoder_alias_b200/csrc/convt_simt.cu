@@ -51,22 +51,23 @@ convt_simt_kernel(const float *__restrict__ x, const float *__restrict__ w,
     for (int k = 0; k < TP; ++k) acc[i][k] = 0.0f;
 
   for (int i0 = 0; i0 < Cin; i0 += CK) {
+    // staged through cp.async (zero-filled outside the input and the channels)
     for (int idx = tid; idx < CK * WX; idx += blockDim.x) {
       const int ci = idx / WX, q = idx - ci * WX;
       const int tin = P_lo + q;
-      float v = 0.0f;
-      if (i0 + ci < Cin && tin >= 0 && tin < T) v = __ldg(xb + (size_t)(i0 + ci) * T + tin);
-      xs[idx] = v;
+      const bool ok = i0 + ci < Cin && tin >= 0 && tin < T;
+      cp_async4_zfill(xs + idx, ok ? xb + (size_t)(i0 + ci) * T + tin : xb, ok);
     }
     // w[i, o, j]: contiguous over (o, j) for a fixed i
     const int MK = BM * K;
     for (int idx = tid; idx < CK * MK; idx += blockDim.x) {
       const int ci = idx / MK, rem = idx - ci * MK;
       const int m = rem / K, j = rem - m * K;
-      float v = 0.0f;
-      if (i0 + ci < Cin && m0 + m < Cout) v = __ldg(w + ((size_t)(i0 + ci) * Cout + m0 + m) * K + j);
-      ws[(ci * K + j) * WSP + m] = v;
+      const bool ok = i0 + ci < Cin && m0 + m < Cout;
+      cp_async4_zfill(ws + (ci * K + j) * WSP + m,
+                      ok ? w + ((size_t)(i0 + ci) * Cout + m0 + m) * K + j : w, ok);
     }
+    cp_async_wait_all();
     __syncthreads();
     for (int ci = 0; ci < CK; ++ci) {
       for (int mm = 0; mm < NTAP; ++mm) {
@@ -92,11 +93,19 @@ convt_simt_kernel(const float *__restrict__ x, const float *__restrict__ w,
     __syncthreads();
   }
 
+  // the biases are read before any output is written (a load between the
+  // stores would wait a full round trip each)
+  float bos[TM];
+#pragma unroll
+  for (int i = 0; i < TM; ++i) {
+    const int o = m0 + ty * TM + i;
+    bos[i] = (bias && o < Cout) ? __ldg(bias + o) : 0.0f;
+  }
 #pragma unroll
   for (int i = 0; i < TM; ++i) {
     const int o = m0 + ty * TM + i;
     if (o >= Cout) continue;
-    const float bo = bias ? __ldg(bias + o) : 0.0f;
+    const float bo = bos[i];
     float *yrow = y + ((size_t)b * Cout + o) * Tout;
 #pragma unroll
     for (int k = 0; k < TP; ++k) {
