@@ -32,6 +32,7 @@
 // [-1/2, 1/2] (exact), and sin(pi f) = f P(f^2) with a degree-4 polynomial P
 // (sin2.cuh).  The row's sqrt(inv_b) is folded into P, so v = u + g^2 with
 // g = f P'(f^2): eleven paired instructions per pair of values.
+#include <atomic>
 #include <type_traits>
 
 #include "common.cuh"
@@ -435,19 +436,24 @@ __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restric
     out[i] = sin_squared(z[i]);
 }
 
-// CTAs resident at once for the activation kernel on this device.
+// CTAs resident at once for the activation kernel on the current device
+// (computed once per device; a racing first call computes the same value).
 int persistent_ctas() {
-  static int n = 0;
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int slot = dev >= 0 && dev < kMaxDev ? dev : 0;
+  int n = cache[slot].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0, sms = 148, per_sm = 4;
-    cudaGetDevice(&dev);
+    int sms = 148, per_sm = 2;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_kernel, THREADS,
-                                                      SMEM_BYTES) !=
-            cudaSuccess ||
+                                                      SMEM_BYTES) != cudaSuccess ||
         per_sm < 1)
-      per_sm = 4;
+      per_sm = 2;
     n = sms * per_sm;
+    cache[slot].store(n, std::memory_order_relaxed);
   }
   return n;
 }
@@ -472,13 +478,8 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
   if (n_tiles <= 0) return BV_OK;
   if (rows > 0x7fffffffLL || (rows + 1) / 2 > 0x7fffffffLL / 2)
     return fail(BV_ERR_SHAPE, "activation: too many rows");
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(activation_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_BYTES) != cudaSuccess)
-      return check_launch("activation smem attribute");
-    configured = true;
-  }
+  BV_TRY(ensure_dynamic_smem((const void *)activation_kernel, SMEM_BYTES,
+                             "activation smem attribute"));
   const long long ctas = persistent_ctas();
   const long long need = (n_tiles + WARPS - 1) / WARPS;
   const long long grid = need < ctas ? need : ctas;

@@ -46,6 +46,37 @@ bv_status check_launch(const char *what) {
 
 void count_launch(uint64_t n) { __atomic_fetch_add(&g_launches, n, __ATOMIC_RELAXED); }
 
+namespace {
+struct SmemLimit {
+  int dev;
+  const void *func;
+  size_t bytes;
+};
+std::mutex g_smem_mu;
+std::vector<SmemLimit> g_smem_limits;
+}  // namespace
+
+bv_status ensure_dynamic_smem(const void *func, size_t bytes, const char *what) {
+  if (bytes <= 48 * 1024) return BV_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return check_launch(what);
+  std::lock_guard<std::mutex> lk(g_smem_mu);
+  for (SmemLimit &l : g_smem_limits)
+    if (l.dev == dev && l.func == func) {
+      if (l.bytes >= bytes) return BV_OK;
+      if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+          cudaSuccess)
+        return check_launch(what);
+      l.bytes = bytes;
+      return BV_OK;
+    }
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return check_launch(what);
+  g_smem_limits.push_back({dev, func, bytes});
+  return BV_OK;
+}
+
 // ------------------------------------------------------------ launch timing
 
 namespace {

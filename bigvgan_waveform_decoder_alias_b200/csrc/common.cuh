@@ -20,6 +20,11 @@ bv_status check_launch(const char *what);
 // Counts kernel launches issued by the library.
 void count_launch(uint64_t n = 1);
 
+// Raises `func`'s dynamic shared-memory limit to at least `bytes` on the
+// current device; remembered per (device, kernel), thread-safe.  Nothing to do
+// up to 48 KB.  BV_ERR_CUDA (tagged `what`) if the driver refuses.
+bv_status ensure_dynamic_smem(const void *func, size_t bytes, const char *what);
+
 // Address of the device status word that bounded waits set when they give
 // up (kernels take it as an argument); nullptr if it cannot be resolved.
 int *device_status_ptr();

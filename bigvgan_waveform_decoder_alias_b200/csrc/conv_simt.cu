@@ -155,13 +155,7 @@ bv_status run_conv(const float *x, int B, int Cin, int T, const float *w, const 
   const size_t smem = Cfg::smem_bytes(K, dil);
   if (smem > 227 * 1024) return fail(BV_ERR_UNSUPPORTED, "conv1d: K*dilation too large");
   auto kern = conv1d_simt_kernel<BM, BN, TM, TN, CK>;
-  static size_t configured = 0;  // max dynamic smem set so far for this instance
-  if (smem > 48 * 1024 && smem > configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return check_launch("conv1d smem attribute");
-    configured = smem;
-  }
+  BV_TRY(ensure_dynamic_smem((const void *)kern, smem, "conv1d smem attribute"));
   dim3 grid((y_len + BN - 1) / BN, (Cout + BM - 1) / BM, B);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d: grid too large");
   {

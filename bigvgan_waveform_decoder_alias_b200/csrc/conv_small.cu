@@ -141,13 +141,8 @@ bv_status run_small(const float *x, int B, int Cin, int T, const float *w, const
   const int XW = (SM_T + (K - 1) * dil + 3) & ~3;
   const size_t smem = ((size_t)Cin * K * COUT + (size_t)Cin * XW) * sizeof(float);
   if (smem > 200 * 1024) return fail(BV_ERR_UNSUPPORTED, "conv1d_small: tile too large");
-  static size_t configured = 0;
-  if (smem > 48 * 1024 && smem > configured) {
-    if (cudaFuncSetAttribute(conv1d_small_kernel<COUT, KT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return check_launch("conv1d_small smem attribute");
-    configured = smem;
-  }
+  BV_TRY(ensure_dynamic_smem((const void *)conv1d_small_kernel<COUT, KT>, smem,
+                             "conv1d_small smem attribute"));
   dim3 grid((y_len + SM_T - 1) / SM_T, B);
   if (grid.y > 65535) return fail(BV_ERR_SHAPE, "conv1d_small: grid too large");
   {

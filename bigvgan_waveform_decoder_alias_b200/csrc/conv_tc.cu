@@ -558,13 +558,8 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
                  int Cin, int T, const float *bias, int Cout, int K, int dil, int pad,
                  const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
                  cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(conv1d_tc_kernel<NT, PRESPLIT>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
-      return check_launch("conv1d_tc smem attribute");
-    configured = true;
-  }
+  BV_TRY(ensure_dynamic_smem((const void *)conv1d_tc_kernel<NT, PRESPLIT>, SMEM_BYTES,
+                             "conv1d_tc smem attribute"));
   dim3 grid((y_len + BM - 1) / BM, (Cout + NT - 1) / NT, B * om.phases);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
   conv1d_tc_kernel<NT, PRESPLIT><<<grid, THREADS, SMEM_BYTES, st>>>(
@@ -949,13 +944,8 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
                  int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
                  const OutMap &om, cudaStream_t st) {
-  static bool configured = false;
-  if (!configured) {
-    if (cudaFuncSetAttribute(conv1d_tm_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             TM_SMEM_BYTES) != cudaSuccess)
-      return check_launch("conv1d_tm smem attribute");
-    configured = true;
-  }
+  BV_TRY(ensure_dynamic_smem((const void *)conv1d_tm_kernel<NT>, TM_SMEM_BYTES,
+                             "conv1d_tm smem attribute"));
   dim3 grid(2 * ((y_len + 2 * BM - 1) / (2 * BM)), (Cout + NT - 1) / NT, B * om.phases);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tm: grid too large");
   conv1d_tm_kernel<NT><<<grid, THREADS, TM_SMEM_BYTES, st>>>(

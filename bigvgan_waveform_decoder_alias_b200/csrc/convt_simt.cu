@@ -139,23 +139,11 @@ bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const f
                  4.0 * ((double)B * Cin * T + (double)Cin * Cout * K + (double)B * Cout * Tout));
   if (wide) {
     auto kern = convt_simt_kernel<16, 4>;
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-        return check_launch("convt smem attribute");
-      configured = smem;
-    }
+    BV_TRY(ensure_dynamic_smem((const void *)kern, smem, "convt smem attribute"));
     kern<<<grid, threads, smem, st>>>(x, w, bias, y, Cin, T, Cout, K, S, pad, Tout, NTX, NTAP);
   } else {
     auto kern = convt_simt_kernel<8, 4>;
-    static size_t configured = 0;
-    if (smem > 48 * 1024 && smem > configured) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-        return check_launch("convt smem attribute");
-      configured = smem;
-    }
+    BV_TRY(ensure_dynamic_smem((const void *)kern, smem, "convt smem attribute"));
     kern<<<grid, threads, smem, st>>>(x, w, bias, y, Cin, T, Cout, K, S, pad, Tout, NTX, NTAP);
   }
   count_launch();
