@@ -125,6 +125,25 @@ def test_activation_full_size_sweep_point(nat, oracle, filt):
     assert np.abs(y - want).max() < 1e-4
 
 
+@pytest.mark.parametrize("B,C,T", [(1, 8, 128 * 1200 + 1), (1, 7, 128 * 1500 + 2),
+                                   (2, 3, 128 * 900 + 130)])
+def test_activation_multi_tile_ranges_and_short_last_tiles(nat, oracle, filt, B, C, T):
+    """Enough tiles that warps own several consecutive 128-output tiles (so a
+    tile's down-sampling reads the next tile's first 2x-rate values), rows
+    whose last tile holds 1, 2 or 2 + 128 outputs (the replicate padding then
+    reaches into the previous tile's reads), and odd row counts; every
+    element against the oracle."""
+    s = synth.NormalStream(5000 + C + T)
+    x = s.normal((B, C, T), 0.0, 1.5)
+    la, lb = s.normal((C,), 0.0, 0.3), s.normal((C,), 0.0, 0.3)
+    y = host(nat.bv_activation1d(dev(x), dev(la), dev(lb), filt))
+    want = oracle.activation1d(x, la, lb)
+    assert rel_l2(y, want) < LAYER_TOL
+    tail = slice(T - 300, T)
+    assert rel_l2(y[..., tail], want[..., tail]) < LAYER_TOL
+    assert np.abs(y - want).max() < 1e-4
+
+
 @pytest.mark.parametrize("C,T", [(64, 262144), (1536, 4096), (768, 16384)])
 def test_activation_sweep_shapes_sampled(nat, oracle, filt, C, T):
     s = synth.NormalStream(C + T)
