@@ -47,6 +47,9 @@ def lib():
                                  _f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                  ctypes.c_int, ctypes.c_int, _f32p]
         L.orc_conv_transpose1d.argtypes = L.orc_conv1d.argtypes
+        L.orc_latent_front_end.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                           _f32p, _f32p, _f32p, _f32p, ctypes.c_int,
+                                           ctypes.c_int, _f32p]
         L.orc_conv1d_points.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         _f32p, _f32p, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, ctypes.c_int, _i64p, ctypes.c_int,
@@ -141,6 +144,22 @@ def conv1d(x, w, bias, dilation=1, pad=None, store_f64=False):
     _check(lib().orc_conv1d(_p32(x), B, Cin, T, _p32(w), _p32(b), Cout, K, dilation,
                             pad, int(store_f64), _p32(y)), "conv1d")
     return y
+
+
+def latent_front_end(z, mean, std, w, bias, store_f64=False):
+    """[H3] ``AudioVae::decode`` front end: normalised latents z [C, S, T]
+    (stereo: S = 2) -> per side z std + mean, then ``dec_in_proj`` (one-tap
+    conv, w [Cout, C, 1]) -> [S, Cout, T]."""
+    z, w = _f32(z), _f32(w)
+    C, S, T = z.shape
+    Cout, C2, K = w.shape
+    assert C2 == C and K == 1
+    b = None if bias is None else _f32(bias)
+    out = np.empty((S, Cout, T), np.float32)
+    _check(lib().orc_latent_front_end(_p32(z), C, S, T, _p32(_f32(mean)), _p32(_f32(std)),
+                                      _p32(w), _p32(b), Cout, int(store_f64), _p32(out)),
+           "latent_front_end")
+    return out
 
 
 def conv_transpose1d(x, w, bias, stride, pad=None, store_f64=False):

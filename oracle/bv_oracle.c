@@ -289,6 +289,36 @@ int orc_conv1d(const float *x, int B, int Cin, int T, const float *w,
     return ORC_OK;
 }
 
+/* The latent front end of [H3] `AudioVae::decode`.  The normalised latents
+ * arrive as z [C, S, T] (channel ci of side s at (ci S + s) T + t; the page's
+ * stereo layout has S = 2).  Per side s, in the page's order:
+ *   lat[ci, t] = z[ci, s, t] std[ci] + mean[ci]      (stored as float),
+ *   out[s, o, t] = bias[o] + sum_ci w[o, ci] lat[ci, t]   (`dec_in`).
+ * `dec_in` is the checkpoint's `avae.dec_in_proj` Conv1d, loaded with padding
+ * 0 and dilation 1 ([H3] `AudioVae::from_cmf`); `decode` keeps the length t
+ * after it, so its kernel has one tap: w [Cout, C, 1]. */
+int orc_latent_front_end(const float *z, int C, int S, int T, const float *mean,
+                         const float *std_, const float *w, const float *bias,
+                         int Cout, int store_f64, float *out) {
+    if (C <= 0 || S <= 0 || T <= 0 || Cout <= 0 || !mean || !std_ || !w) return ORC_ERR_ARG;
+    size_t nl = (size_t)S * C * T, no = (size_t)S * Cout * T;
+    double *lat = (double *)malloc(nl * sizeof(double));
+    double *yd = (double *)malloc(no * sizeof(double));
+    double *acc = (double *)malloc((size_t)T * sizeof(double));
+    if (!lat || !yd || !acc) { free(lat); free(yd); free(acc); return ORC_ERR_NOMEM; }
+    for (int s = 0; s < S; ++s)
+        for (int ci = 0; ci < C; ++ci) {
+            const float *zr = z + ((size_t)ci * S + s) * T;
+            double *lr = lat + ((size_t)s * C + ci) * T;
+            for (int t = 0; t < T; ++t)
+                lr[t] = rnd((double)zr[t] * (double)std_[ci] + (double)mean[ci], store_f64);
+        }
+    conv1d_d(lat, S, C, T, w, bias, Cout, 1, 1, 0, yd, acc, store_f64);
+    to_f(yd, out, no);
+    free(lat); free(yd); free(acc);
+    return ORC_OK;
+}
+
 int orc_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,
                          const float *bias, int Cout, int K, int s, int pad,
                          int store_f64, float *y) {

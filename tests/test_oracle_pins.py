@@ -513,3 +513,53 @@ def test_normal_stream_is_a_stream():
     np.testing.assert_array_equal(np.concatenate([x1, x2]), both)
     big = synth.NormalStream(3).normal((200000,)).astype(np.float64)
     assert abs(big.mean()) < 0.01 and abs(big.std() - 1.0) < 0.01
+
+
+# ------------------------------------------------- latent front end (H3 decode)
+
+
+def test_latent_front_end_identity_reads_the_stereo_layout(oracle):
+    """std 1, mean 0 and an identity projection return the latents as they
+    are, side by side: out[s, c, t] = z[c, s, t] -- the [C, 2, T] layout of
+    the audiovae.rs page's `AudioVae::decode` (z[(ci 2 + ch) t + ti])."""
+    rng = np.random.default_rng(5)
+    C, S, T = 6, 2, 11
+    z = rng.standard_normal((C, S, T)).astype(np.float32)
+    w = np.eye(C, dtype=np.float32)[:, :, None]
+    out = oracle.latent_front_end(z, np.zeros(C, np.float32), np.ones(C, np.float32), w, None)
+    np.testing.assert_array_equal(out, z.transpose(1, 0, 2))
+
+
+def test_latent_front_end_affine_denormalisation(oracle):
+    """With an identity projection and a bias: out = z std + mean + bias,
+    channel by channel (the de-normalisation runs before the projection)."""
+    rng = np.random.default_rng(6)
+    C, S, T = 5, 2, 9
+    z = rng.standard_normal((C, S, T)).astype(np.float32)
+    mean = rng.standard_normal(C).astype(np.float32)
+    std = rng.uniform(0.5, 2.0, C).astype(np.float32)
+    bias = rng.standard_normal(C).astype(np.float32)
+    w = np.eye(C, dtype=np.float32)[:, :, None]
+    out = oracle.latent_front_end(z, mean, std, w, bias, store_f64=True).astype(np.float64)
+    lat = z.astype(np.float64) * std[:, None, None] + mean[:, None, None]
+    want = lat.transpose(1, 0, 2) + bias[None, :, None]
+    np.testing.assert_allclose(out, want, rtol=1e-6, atol=1e-6)
+
+
+def test_latent_front_end_projection_matches_torch(oracle):
+    """The projection against torch's float64 conv1d (kernel size 1) of the
+    float-stored de-normalised latents."""
+    import torch
+    rng = np.random.default_rng(7)
+    C, S, T, Cout = 8, 2, 40, 12
+    z = rng.standard_normal((C, S, T)).astype(np.float32)
+    mean = rng.standard_normal(C).astype(np.float32)
+    std = rng.uniform(0.5, 2.0, C).astype(np.float32)
+    w = (0.3 * rng.standard_normal((Cout, C, 1))).astype(np.float32)
+    b = rng.standard_normal(Cout).astype(np.float32)
+    out = oracle.latent_front_end(z, mean, std, w, b)
+    lat = (z.astype(np.float64) * std[:, None, None] + mean[:, None, None]).astype(np.float32)
+    want = torch.nn.functional.conv1d(torch.from_numpy(lat.transpose(1, 0, 2).astype(np.float64)),
+                                      torch.from_numpy(w.astype(np.float64)),
+                                      torch.from_numpy(b.astype(np.float64))).numpy()
+    np.testing.assert_allclose(out, want.astype(np.float32), rtol=2e-6, atol=2e-6)
