@@ -75,6 +75,14 @@ def lib():
                                        ctypes.c_int, _f32p, _f32p, ctypes.c_int,
                                        ctypes.c_double, ctypes.c_int, _f32p, _f32p]
         L.orc_tile_count.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.orc_snake1d.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
+                                  ctypes.c_int, _f32p]
+        L.orc_dav_param_count.restype = ctypes.c_long
+        L.orc_dav_param_count.argtypes = [_i32p]
+        L.orc_dav_hop.restype = ctypes.c_long
+        L.orc_dav_hop.argtypes = [_i32p]
+        L.orc_dav_decode.argtypes = [_i32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
+                                     ctypes.c_int, _f32p]
         _LIB = L
     return _LIB
 
@@ -320,3 +328,62 @@ def decode_tiled(geo, params, z, tile, overlap, tiles=None, filt=None, eps=1e-9,
                                   tile, overlap, lo, hi, _p32(f), _p32(f), len(f), eps,
                                   int(store_f64), _p32(y), _p32(cnt)), "decode_tiled")
     return y, cnt
+
+
+# ------------------------------------------------------- Music-3 DAV decoder
+
+
+def snake1d(x, alpha, store_f64=False):
+    """Plain Snake, alpha used as stored: x + sin^2(alpha x) / (alpha + 1e-9)
+    (the audiovae.rs page's `Snake`)."""
+    x = _f32(x)
+    B, C, T = x.shape
+    y = np.empty_like(x)
+    _check(lib().orc_snake1d(_p32(x), B, C, T, _p32(_f32(alpha)), int(store_f64), _p32(y)),
+           "snake1d")
+    return y
+
+
+def dav_geometry_ints(geo) -> np.ndarray:
+    g = np.zeros(38, np.int32)
+    rates, upk, upch = (list(_get(geo, n)) for n in ("up_rates", "up_kernels", "up_channels"))
+    dil = list(_get(geo, "dilations"))
+    fa = _get(geo, "final_act")
+    g[0], g[1], g[2], g[3], g[4] = (_get(geo, "latent_channels"), _get(geo, "in_channels"),
+                                    _get(geo, "pre_channels"), _get(geo, "pre_kernel"),
+                                    len(rates))
+    g[5:5 + len(rates)] = rates
+    g[13:13 + len(upk)] = upk
+    g[21:21 + len(upch)] = upch
+    g[29] = len(dil)
+    g[30:30 + len(dil)] = dil
+    g[34], g[35], g[36] = (_get(geo, "unit_kernel"), _get(geo, "post_kernel"),
+                           _get(geo, "out_channels"))
+    g[37] = FINAL_ACTS[fa] if isinstance(fa, str) else int(fa)
+    return g
+
+
+def dav_param_count(geo) -> int:
+    g = dav_geometry_ints(geo)
+    return int(lib().orc_dav_param_count(g.ctypes.data_as(_i32p)))
+
+
+def dav_hop(geo) -> int:
+    g = dav_geometry_ints(geo)
+    return int(lib().orc_dav_hop(g.ctypes.data_as(_i32p)))
+
+
+def dav_decode(geo, params, z, store_f64=False):
+    """MiniMax-Music-3 DAV decoder (the audiovae.rs page's `Music3Dav`):
+    z [B, latent_channels, frames] -> [B, out_channels, frames * hop]; the
+    page's 128-channel stereo latent is B = 2 halves of 64."""
+    g = dav_geometry_ints(geo)
+    z, params = _f32(z), _f32(params)
+    if params.size != dav_param_count(geo):
+        raise ValueError(f"params has {params.size} values, geometry needs "
+                         f"{dav_param_count(geo)}")
+    B, _, F = z.shape
+    y = np.empty((B, int(g[36]), F * dav_hop(geo)), np.float32)
+    _check(lib().orc_dav_decode(g.ctypes.data_as(_i32p), _p32(params), _p32(z), B, F,
+                                int(store_f64), _p32(y)), "dav_decode")
+    return y

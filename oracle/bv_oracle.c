@@ -701,3 +701,162 @@ int orc_tile_count(int frames, int tile, int overlap) {
     while (start + tile < frames) { start += tile - overlap; ++n; }
     return n;
 }
+
+/* ------------------------------------------------------ Music-3 DAV decoder */
+
+/* Plain Snake over rows of length n, alpha used as stored ([H3] `Snake`):
+ *   v = x + sin^2(alpha_c x) / (alpha_c + 1e-9). */
+static void snake_rows(double *x, int rows, int C, int n, const float *alpha,
+                       int store_f64) {
+    for (int r = 0; r < rows; ++r) {
+        double a = (double)alpha[r % C];
+        double inv = 1.0 / (a + 1e-9);
+        double *xr = x + (size_t)r * n;
+        for (int t = 0; t < n; ++t) {
+            double s = sin(a * xr[t]);
+            xr[t] = rnd(xr[t] + s * s * inv, store_f64);
+        }
+    }
+}
+
+/* Plain Snake over x [B, C, T] (exported for its pins). */
+int orc_snake1d(const float *x, int B, int C, int T, const float *alpha, int store_f64,
+                float *y) {
+    if (B <= 0 || C <= 0 || T <= 0 || !alpha) return ORC_ERR_ARG;
+    size_t n = (size_t)B * C * T;
+    double *d = to_d(x, n);
+    if (!d) return ORC_ERR_NOMEM;
+    snake_rows(d, B * C, C, T, alpha, store_f64);
+    to_f(d, y, n);
+    free(d);
+    return ORC_OK;
+}
+
+/* DAV geometry, as an int array:
+ *  [0] latent_ch  [1] in_ch (dec_in output)  [2] pre_ch  [3] pre_k  [4] n_up
+ *  [5..12] up_rate[8]  [13..20] up_k[8]  [21..28] up_ch[8]
+ *  [29] n_dil  [30..33] dil[4]  [34] unit_k  [35] post_k  [36] out_ch
+ *  [37] final_act (0 none, 1 clamp, 2 tanh).
+ * Parameters in module order ([H3] `Music3Dav::from_cmf`, `DavStage::load`,
+ * `DavUnit::load`): dec_in w [in, lat, 1], b [in]; conv_pre w [pre, in,
+ * pre_k], b [pre]; per stage i: act alpha [Cin_i]; up w [Cin_i, Cout_i,
+ * up_k_i], b [Cout_i]; per unit u: a1 alpha [C], c1 w [C, C, unit_k], b [C],
+ * a2 alpha [C], c2 w [C, C, 1], b [C]; act_post alpha [C]; conv_post w [out,
+ * C, post_k], b [out].
+ * Wiring ([H3] `Music3Dav::decode`, `DavStage::apply`, `DavUnit::apply`):
+ *  dec_in (one tap, pad 0) -> conv_pre (pad (k-1)/2) -> per stage: Snake ->
+ *  ConvT (pad (k - s)/2) -> units x += c2(Snake(c1(Snake(x)))) with c1
+ *  dilated (pad d (unit_k - 1)/2) and c2 one tap -> Snake -> conv_post
+ *  (pad (k-1)/2) -> final op. */
+enum { D_LAT, D_IN, D_PRE, D_PREK, D_NUP, D_RATE = 5, D_UPK = 13, D_UPCH = 21,
+       D_ND = 29, D_DIL = 30, D_UNITK = 34, D_POSTK = 35, D_OUT = 36, D_FINAL = 37,
+       D_LEN = 38 };
+
+static int dav_ok(const int *g) {
+    if (g[D_LAT] <= 0 || g[D_IN] <= 0 || g[D_PRE] <= 0 || g[D_PREK] <= 0 ||
+        g[D_PREK] % 2 == 0) return 0;
+    if (g[D_NUP] < 0 || g[D_NUP] > 8 || g[D_ND] < 0 || g[D_ND] > 4) return 0;
+    for (int i = 0; i < g[D_NUP]; ++i)
+        if (g[D_RATE + i] <= 0 || g[D_UPK + i] < g[D_RATE + i] || g[D_UPCH + i] <= 0) return 0;
+    for (int u = 0; u < g[D_ND]; ++u) if (g[D_DIL + u] <= 0) return 0;
+    if (g[D_UNITK] <= 0 || g[D_UNITK] % 2 == 0 || g[D_POSTK] <= 0 || g[D_POSTK] % 2 == 0)
+        return 0;
+    return g[D_OUT] > 0;
+}
+
+long orc_dav_param_count(const int *g) {
+    if (!dav_ok(g)) return -1;
+    long n = (long)g[D_IN] * g[D_LAT] + g[D_IN];
+    n += (long)g[D_PRE] * g[D_IN] * g[D_PREK] + g[D_PRE];
+    long cin = g[D_PRE];
+    for (int i = 0; i < g[D_NUP]; ++i) {
+        long c = g[D_UPCH + i];
+        n += cin + cin * c * g[D_UPK + i] + c;
+        n += (long)g[D_ND] * (2 * c + c * c * g[D_UNITK] + c + c * c + c);
+        cin = c;
+    }
+    n += cin + (long)g[D_OUT] * cin * g[D_POSTK] + g[D_OUT];
+    return n;
+}
+
+long orc_dav_hop(const int *g) {
+    long h = 1;
+    for (int i = 0; i < g[D_NUP]; ++i) h *= g[D_RATE + i];
+    return h;
+}
+
+/* z [B, lat, F] -> y [B, out, F hop].  Every ConvT must give exactly s times
+ * its input length (k - 2 pad = s), as the page's `n = n * stride` assumes;
+ * otherwise ORC_ERR_ARG. */
+int orc_dav_decode(const int *g, const float *params, const float *z, int B, int F,
+                   int store_f64, float *y) {
+    if (!dav_ok(g) || B <= 0 || F <= 0) return ORC_ERR_ARG;
+    long hop = orc_dav_hop(g);
+    long L = (long)F * hop;
+    int cmax = g[D_PRE] > g[D_IN] ? g[D_PRE] : g[D_IN];
+    if (g[D_LAT] > cmax) cmax = g[D_LAT];
+    for (int i = 0; i < g[D_NUP]; ++i) {
+        int k = g[D_UPK + i], s = g[D_RATE + i];
+        if (k - 2 * ((k - s) / 2) != s) return ORC_ERR_ARG;
+        if (g[D_UPCH + i] > cmax) cmax = g[D_UPCH + i];
+    }
+    size_t big = (size_t)B * cmax * (size_t)L + 16;
+    double *a = (double *)malloc(big * sizeof(double));
+    double *b = (double *)malloc(big * sizeof(double));
+    double *r = (double *)malloc(big * sizeof(double));
+    double *acc = (double *)malloc(((size_t)L + 64) * sizeof(double));
+    if (!a || !b || !r || !acc) { free(a); free(b); free(r); free(acc); return ORC_ERR_NOMEM; }
+    const float *p = params;
+    size_t nz = (size_t)B * g[D_LAT] * F;
+    for (size_t i = 0; i < nz; ++i) a[i] = (double)z[i];
+    /* dec_in */
+    const float *w = p; p += (size_t)g[D_IN] * g[D_LAT];
+    const float *bb = p; p += g[D_IN];
+    conv1d_d(a, B, g[D_LAT], F, w, bb, g[D_IN], 1, 1, 0, b, acc, store_f64);
+    /* conv_pre */
+    w = p; p += (size_t)g[D_PRE] * g[D_IN] * g[D_PREK];
+    bb = p; p += g[D_PRE];
+    conv1d_d(b, B, g[D_IN], F, w, bb, g[D_PRE], g[D_PREK], 1, (g[D_PREK] - 1) / 2, a, acc,
+             store_f64);
+    int C = g[D_PRE];
+    long n = F;
+    for (int i = 0; i < g[D_NUP]; ++i) {
+        int s = g[D_RATE + i], k = g[D_UPK + i], Co = g[D_UPCH + i];
+        const float *alpha = p; p += C;
+        snake_rows(a, B * C, C, (int)n, alpha, store_f64);
+        w = p; p += (size_t)C * Co * k;
+        bb = p; p += Co;
+        convt1d_d(a, B, C, (int)n, w, bb, Co, k, s, (k - s) / 2, b, acc, store_f64);
+        n *= s;
+        C = Co;
+        size_t nn = (size_t)B * C * n;
+        for (int u = 0; u < g[D_ND]; ++u) {
+            int d = g[D_DIL + u], K = g[D_UNITK];
+            const float *a1 = p; p += C;
+            const float *w1 = p; p += (size_t)C * C * K;
+            const float *b1 = p; p += C;
+            const float *a2 = p; p += C;
+            const float *w2 = p; p += (size_t)C * C;
+            const float *b2 = p; p += C;
+            memcpy(r, b, nn * sizeof(double));
+            snake_rows(r, B * C, C, (int)n, a1, store_f64);
+            conv1d_d(r, B, C, (int)n, w1, b1, C, K, d, d * (K - 1) / 2, a, acc, store_f64);
+            snake_rows(a, B * C, C, (int)n, a2, store_f64);
+            conv1d_d(a, B, C, (int)n, w2, b2, C, 1, 1, 0, r, acc, store_f64);
+            for (size_t q = 0; q < nn; ++q) b[q] = rnd(b[q] + r[q], store_f64);
+        }
+        /* the stage output lives in b; the next stage reads a */
+        memcpy(a, b, nn * sizeof(double));
+    }
+    const float *ap = p; p += C;
+    snake_rows(a, B * C, C, (int)n, ap, store_f64);
+    w = p; p += (size_t)g[D_OUT] * C * g[D_POSTK];
+    bb = p; p += g[D_OUT];
+    conv1d_d(a, B, C, (int)n, w, bb, g[D_OUT], g[D_POSTK], 1, (g[D_POSTK] - 1) / 2, b, acc,
+             store_f64);
+    size_t ny = (size_t)B * g[D_OUT] * L;
+    final_op(b, ny, g[D_FINAL], store_f64);
+    to_f(b, y, ny);
+    free(a); free(b); free(r); free(acc);
+    return ORC_OK;
+}

@@ -563,3 +563,134 @@ def test_latent_front_end_projection_matches_torch(oracle):
                                       torch.from_numpy(w.astype(np.float64)),
                                       torch.from_numpy(b.astype(np.float64))).numpy()
     np.testing.assert_allclose(out, want.astype(np.float32), rtol=2e-6, atol=2e-6)
+
+
+# ----------------------------------------------------- Music-3 DAV decoder
+
+
+def test_snake_closed_forms(oracle):
+    """Plain Snake x + sin^2(a x)/(a + 1e-9) at points where sin^2 is known:
+    a x = pi/2 adds 1/(a + 1e-9), a x = pi adds 0, x = 0 stays 0."""
+    a = np.array([0.5, 1.0, 2.0, 1.7], np.float32)
+    x = np.stack([np.pi / 2 / a, np.pi / a, np.zeros(4), -np.pi / 2 / a], 1)[None].astype(
+        np.float32)
+    y = oracle.snake1d(x, a, store_f64=True).astype(np.float64)
+    xd = x.astype(np.float64)
+    ad = a.astype(np.float64)[:, None]
+    want = np.stack([xd[0, :, 0] + 1 / (ad[:, 0] + 1e-9), xd[0, :, 1], np.zeros(4),
+                     xd[0, :, 3] + 1 / (ad[:, 0] + 1e-9)], 1)
+    np.testing.assert_allclose(y[0], want, rtol=1e-6, atol=1e-7)
+
+
+def _dav_tensors(geo, params):
+    out, off = {}, 0
+    for name, shape, _ in synth.dav_param_layout(geo):
+        n = int(np.prod(shape))
+        out[name] = params[off:off + n].reshape(shape)
+        off += n
+    return out
+
+
+def _dav_inputs(geo, B=2, F_=5, seed=41):
+    s = synth.NormalStream(seed)
+    z = s.normal((B, geo.latent_channels, F_))
+    params = s.normal((synth.dav_param_count(geo),), 0.0, 0.2)
+    t = _dav_tensors(geo, params)
+    for name in t:  # plain Snake alphas are used as stored: keep them near 1
+        if name.endswith(".alpha"):
+            t[name][:] = 1.0 + 0.1 * np.tanh(t[name])
+    return z, params
+
+
+def _torch_dav(geo, params, z):
+    """The DAV decoder composed from torch float64 operators."""
+    t = {k: torch.as_tensor(v, dtype=torch.float64) for k, v in _dav_tensors(geo, params).items()}
+
+    def snake(x, a):
+        a = a[None, :, None]
+        return x + torch.sin(a * x) ** 2 / (a + 1e-9)
+
+    x = F.conv1d(torch.as_tensor(z, dtype=torch.float64), t["dec_in.w"], t["dec_in.b"])
+    x = F.conv1d(x, t["conv_pre.w"], t["conv_pre.b"], padding=(geo.pre_kernel - 1) // 2)
+    for i, (s_, k) in enumerate(zip(geo.up_rates, geo.up_kernels)):
+        x = F.conv_transpose1d(snake(x, t[f"stage{i}.act.alpha"]), t[f"stage{i}.up.w"],
+                               t[f"stage{i}.up.b"], stride=s_, padding=(k - s_) // 2)
+        for u, d in enumerate(geo.dilations):
+            p = f"stage{i}.unit{u}"
+            h = snake(x, t[f"{p}.a1.alpha"])
+            h = F.conv1d(h, t[f"{p}.c1.w"], t[f"{p}.c1.b"], dilation=d,
+                         padding=d * (geo.unit_kernel - 1) // 2)
+            h = F.conv1d(snake(h, t[f"{p}.a2.alpha"]), t[f"{p}.c2.w"], t[f"{p}.c2.b"])
+            x = x + h
+    x = snake(x, t["act_post.alpha"])
+    y = F.conv1d(x, t["conv_post.w"], t["conv_post.b"], padding=(geo.post_kernel - 1) // 2)
+    return torch.tanh(y).numpy() if geo.final_act == "tanh" else y.numpy()
+
+
+def test_dav_param_counts_and_hop(oracle):
+    for geo in (synth.MUSIC3_DAV, synth.tiny_dav_geometry()):
+        assert oracle.dav_param_count(geo) == synth.dav_param_count(geo)
+        assert oracle.dav_hop(geo) == geo.hop
+    # the page's Music3Dav: 512 samples per latent frame, 44.1 kHz
+    assert synth.MUSIC3_DAV.hop == 512 and synth.MUSIC3_DAV.sample_rate == 44100
+
+
+@pytest.mark.parametrize("final_act", ["none", "tanh"])
+def test_dav_matches_torch_composition(oracle, final_act):
+    geo = synth.tiny_dav_geometry(final_act=final_act)
+    z, params = _dav_inputs(geo)
+    y = oracle.dav_decode(geo, params, z, store_f64=True)
+    want = _torch_dav(geo, params, z)
+    assert y.shape == want.shape == (2, 1, z.shape[2] * geo.hop)
+    np.testing.assert_allclose(y, want, rtol=1e-6, atol=1e-6)
+
+
+def test_dav_geometry_and_range(oracle):
+    """The page's Music-3 vocoder test, on the small geometry: a structured
+    latent (0.4 sin(0.13 c + 0.7 t) over the 2 x C stereo channels) decodes
+    to frames x hop samples per side, finite, inside the tanh range, not
+    silent, and the two halves differ."""
+    geo = synth.tiny_dav_geometry()
+    frames, C = 12, geo.latent_channels
+    c = np.arange(2 * C)[:, None]
+    t = np.arange(frames)[None, :]
+    z = (0.4 * np.sin(c * 0.13 + t * 0.7)).reshape(2, C, frames).astype(np.float32)
+    _, params = _dav_inputs(geo)
+    y = oracle.dav_decode(geo, params, z)
+    assert y.shape == (2, 1, frames * geo.hop)
+    assert np.isfinite(y).all() and np.abs(y).max() <= 1.0
+    assert np.sqrt(np.mean(y.astype(np.float64) ** 2)) > 1e-4
+    assert np.abs(y[0] - y[1]).max() > 0
+
+
+def test_dav_residual_identity(oracle):
+    """With every unit's second conv zero, the units add nothing: the decoder
+    is dec_in, conv_pre, (Snake, ConvT) per stage, Snake, conv_post."""
+    geo = synth.tiny_dav_geometry(final_act="none")
+    z, params = _dav_inputs(geo)
+    p = params.copy()
+    off = 0
+    for name, shape, _ in synth.dav_param_layout(geo):
+        n = int(np.prod(shape))
+        if ".c2." in name:
+            p[off:off + n] = 0.0
+        off += n
+    y = oracle.dav_decode(geo, p, z, store_f64=True)
+    t = _dav_tensors(geo, p)
+    x = oracle.conv1d(z, t["dec_in.w"], t["dec_in.b"], 1, 0, store_f64=True)
+    x = oracle.conv1d(x, t["conv_pre.w"], t["conv_pre.b"], 1, 3, store_f64=True)
+    for i, (s_, k) in enumerate(zip(geo.up_rates, geo.up_kernels)):
+        x = oracle.snake1d(x, t[f"stage{i}.act.alpha"], store_f64=True)
+        x = oracle.conv_transpose1d(x, t[f"stage{i}.up.w"], t[f"stage{i}.up.b"], s_,
+                                    (k - s_) // 2, store_f64=True)
+    x = oracle.snake1d(x, t["act_post.alpha"], store_f64=True)
+    want = oracle.conv1d(x, t["conv_post.w"], t["conv_post.b"], 1, 3, store_f64=True)
+    np.testing.assert_allclose(y, want, rtol=1e-5, atol=2e-6)
+
+
+def test_dav_batch_independence(oracle):
+    geo = synth.tiny_dav_geometry()
+    z, params = _dav_inputs(geo)
+    y = oracle.dav_decode(geo, params, z)
+    for b in range(2):
+        np.testing.assert_array_equal(oracle.dav_decode(geo, params, z[b:b + 1]), y[b:b + 1])
