@@ -253,6 +253,107 @@ H3_60S_TILED = DecoderWorkload("h3_decoder_60s_stereo_tiled", H3, 2, 2400, seed=
 DECODER_WORKLOADS = {w.name: w for w in (H3_10S, LTX_VOCODER, H3_60S_TILED)}
 
 
+# ------------------------------------------------ Music-3 DAV decoder
+
+
+@dataclass(frozen=True)
+class DavGeometry:
+    """Shape of a MiniMax-Music-3 DAV decoder: dec_in (one tap) -> conv_pre ->
+    stages of plain Snake, ConvT and residual units at the given dilations
+    -> Snake -> conv_post -> final op."""
+    latent_channels: int
+    in_channels: int
+    pre_channels: int
+    pre_kernel: int
+    up_rates: Tuple[int, ...]
+    up_kernels: Tuple[int, ...]
+    up_channels: Tuple[int, ...]
+    dilations: Tuple[int, ...]
+    unit_kernel: int
+    post_kernel: int
+    out_channels: int
+    final_act: str
+    sample_rate: int
+
+    @property
+    def hop(self) -> int:
+        h = 1
+        for r in self.up_rates:
+            h *= r
+        return h
+
+    def replace(self, **kw) -> "DavGeometry":
+        return dataclasses.replace(self, **kw)
+
+
+def dav_param_layout(g: DavGeometry) -> List[Tuple[str, Tuple[int, ...], str]]:
+    """(name, shape, kind) of every DAV parameter in module order; kind
+    'alpha' is a plain Snake's alpha, used as stored."""
+    out = [("dec_in.w", (g.in_channels, g.latent_channels, 1), "w"),
+           ("dec_in.b", (g.in_channels,), "b"),
+           ("conv_pre.w", (g.pre_channels, g.in_channels, g.pre_kernel), "w"),
+           ("conv_pre.b", (g.pre_channels,), "b")]
+    C = g.pre_channels
+    for i, (k, co) in enumerate(zip(g.up_kernels, g.up_channels)):
+        out += [(f"stage{i}.act.alpha", (C,), "alpha"),
+                (f"stage{i}.up.w", (C, co, k), "w"), (f"stage{i}.up.b", (co,), "b")]
+        C = co
+        for u, _d in enumerate(g.dilations):
+            p = f"stage{i}.unit{u}"
+            out += [(f"{p}.a1.alpha", (C,), "alpha"),
+                    (f"{p}.c1.w", (C, C, g.unit_kernel), "w"), (f"{p}.c1.b", (C,), "b"),
+                    (f"{p}.a2.alpha", (C,), "alpha"),
+                    (f"{p}.c2.w", (C, C, 1), "w"), (f"{p}.c2.b", (C,), "b")]
+    out += [("act_post.alpha", (C,), "alpha"),
+            ("conv_post.w", (g.out_channels, C, g.post_kernel), "w"),
+            ("conv_post.b", (g.out_channels,), "b")]
+    return out
+
+
+def dav_param_count(g: DavGeometry) -> int:
+    return int(sum(int(np.prod(s)) for _, s, _ in dav_param_layout(g)))
+
+
+# Plain Snake alpha of the synthetic DAV decoders: 1 + N(0, 0.1), used as
+# stored (the layers' initial value plus spread).
+ALPHA_MEAN = 1.0
+ALPHA_STD = 0.1
+
+
+def draw_dav_params(stream: "NormalStream", g: DavGeometry) -> np.ndarray:
+    layout = dav_param_layout(g)
+    flat = np.empty(sum(int(np.prod(s)) for _, s, _ in layout), np.float32)
+    off = 0
+    for _, shape, kind in layout:
+        n = int(np.prod(shape))
+        if kind == "alpha":
+            flat[off:off + n] = stream.normal((n,), ALPHA_MEAN, ALPHA_STD)
+        else:
+            flat[off:off + n] = stream.normal((n,), 0.0, WEIGHT_STD if kind == "w" else BIAS_STD)
+        off += n
+    return flat
+
+
+# A DAC-style channel plan for Music-3's DAV decoder (strides 8, 8, 4, 2,
+# dilations 1, 3, 9, 7-tap convs, tanh, 44.1 kHz; the 128-channel latent is a
+# stereo pair of 64): decoder width 1536 halving per stage.
+MUSIC3_DAV = DavGeometry(
+    latent_channels=64, in_channels=64, pre_channels=1536, pre_kernel=7,
+    up_rates=(8, 8, 4, 2), up_kernels=(16, 16, 8, 4), up_channels=(768, 384, 192, 96),
+    dilations=(1, 3, 9), unit_kernel=7, post_kernel=7, out_channels=1, final_act="tanh",
+    sample_rate=44100)
+
+
+def tiny_dav_geometry(**kw) -> DavGeometry:
+    """A small DAV decoder with the same structure, for oracle-speed tests."""
+    base = DavGeometry(
+        latent_channels=8, in_channels=8, pre_channels=48, pre_kernel=7,
+        up_rates=(4, 2, 2), up_kernels=(8, 4, 4), up_channels=(32, 16, 8),
+        dilations=(1, 3, 9), unit_kernel=7, post_kernel=7, out_channels=1, final_act="tanh",
+        sample_rate=44100)
+    return base.replace(**kw)
+
+
 def tiny_geometry(**kw) -> DecoderGeometry:
     """A small decoder with the same structure, for tests the oracle runs in
     seconds (both stride parities, several blocks and dilations)."""
