@@ -253,6 +253,83 @@ H3_60S_TILED = DecoderWorkload("h3_decoder_60s_stereo_tiled", H3, 2, 2400, seed=
 DECODER_WORKLOADS = {w.name: w for w in (H3_10S, LTX_VOCODER, H3_60S_TILED)}
 
 
+# ------------------------------------------ LTX bandwidth-extension tail
+# The extender's mel front end reads two buffers from its checkpoint (the
+# STFT's DFT x window bases and the mel filterbank); none is available here,
+# so they are synthesised as the reference's preprocessing builds them.
+
+
+def stft_basis(n_fft: int) -> np.ndarray:
+    """[2 n_freqs, n_fft] float32, n_freqs = n_fft/2 + 1: rows w[j]
+    cos(2 pi r j / n_fft), then -w[j] sin(2 pi r j / n_fft), w the periodic
+    Hann window 0.5 - 0.5 cos(2 pi j / n_fft) (a one-sided DFT of the
+    windowed frame)."""
+    j = np.arange(n_fft)
+    w = 0.5 - 0.5 * np.cos(2 * np.pi * j / n_fft)
+    r = np.arange(n_fft // 2 + 1)[:, None]
+    ang = 2 * np.pi * r * j[None, :] / n_fft
+    return np.concatenate([w * np.cos(ang), -w * np.sin(ang)]).astype(np.float32)
+
+
+def slaney_mel_basis(sample_rate: int, n_fft: int, n_mels: int, fmin: float,
+                     fmax: float) -> np.ndarray:
+    """[n_mels, n_fft/2 + 1] float32 triangular filters on the Slaney mel
+    scale (linear 3 f / 200 below 1 kHz, logarithmic above, 27 mels per
+    factor 6.4), each scaled by 2 / (upper edge - lower edge) in Hz (Slaney's
+    area normalisation)."""
+    f_min_log, min_log_mel, logstep = 1000.0, 15.0, np.log(6.4) / 27.0
+
+    def hz_to_mel(f):
+        f = np.asarray(f, np.float64)
+        return np.where(f >= f_min_log, min_log_mel + np.log(np.maximum(f, 1e-12) / f_min_log)
+                        / logstep, 3.0 * f / 200.0)
+
+    def mel_to_hz(m):
+        m = np.asarray(m, np.float64)
+        return np.where(m >= min_log_mel, f_min_log * np.exp(logstep * (m - min_log_mel)),
+                        200.0 * m / 3.0)
+
+    freqs = np.linspace(0, sample_rate / 2, n_fft // 2 + 1)
+    pts = mel_to_hz(np.linspace(hz_to_mel(fmin), hz_to_mel(fmax), n_mels + 2))
+    lower = (freqs[None, :] - pts[:-2, None]) / (pts[1:-1] - pts[:-2])[:, None]
+    upper = (pts[2:, None] - freqs[None, :]) / (pts[2:] - pts[1:-1])[:, None]
+    fb = np.maximum(0.0, np.minimum(lower, upper))
+    fb *= (2.0 / (pts[2:] - pts[:-2]))[:, None]
+    return fb.astype(np.float32)
+
+
+@dataclass(frozen=True)
+class BweSpec:
+    """The extender's mel front end and rates: n_fft-sample frames every
+    `hop` samples, n_mels bins over [fmin, fmax] at the input rate, output
+    rate = ratio x input rate."""
+    in_rate: int
+    ratio: int
+    n_fft: int
+    hop: int
+    n_mels: int
+    fmin: float
+    fmax: float
+
+    def bases(self):
+        return (stft_basis(self.n_fft),
+                slaney_mel_basis(self.in_rate, self.n_fft, self.n_mels, self.fmin, self.fmax))
+
+
+LTX_BWE_SPEC = BweSpec(in_rate=16000, ratio=3, n_fft=512, hop=80, n_mels=64, fmin=0.0,
+                       fmax=8000.0)
+
+# The extender generator: BigVGAN v2 on the folded stereo log-mel (2 x 64
+# channels in, 2 out), rates 6, 5, 2, 2, 2 (240 = 3 x the mel hop), no final
+# op (its output is a residual added to the upsampled input).
+LTX_BWE = DecoderGeometry(
+    in_channels=128, pre_channels=512, pre_kernel=7,
+    up_rates=(6, 5, 2, 2, 2), up_kernels=(12, 10, 4, 4, 4),
+    up_channels=(256, 128, 64, 32, 16),
+    block_kernels=(3, 7, 11), dilations=(1, 3, 5),
+    post_kernel=7, out_channels=2, final_act="none", sample_rate=48000)
+
+
 # ------------------------------------------------ Music-3 DAV decoder
 
 

@@ -77,6 +77,17 @@ def lib():
         L.orc_tile_count.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.orc_snake1d.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
                                   ctypes.c_int, _f32p]
+        L.orc_mel_stft.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, _f32p, ctypes.c_int,
+                                   ctypes.c_int, ctypes.c_int, _f32p, ctypes.c_int,
+                                   ctypes.c_int, _f32p]
+        L.orc_mel_frames.restype = ctypes.c_long
+        L.orc_mel_frames.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int]
+        L.orc_hann_sinc_upsample.argtypes = [_f32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, _f32p]
+        L.orc_bwe_tail.argtypes = [_i32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int, _f32p,
+                                   ctypes.c_int, ctypes.c_int, ctypes.c_int, _f32p,
+                                   ctypes.c_int, ctypes.c_int, _f32p, _f32p, ctypes.c_int,
+                                   ctypes.c_int, _f32p]
         L.orc_dav_param_count.restype = ctypes.c_long
         L.orc_dav_param_count.argtypes = [_i32p]
         L.orc_dav_hop.restype = ctypes.c_long
@@ -386,4 +397,55 @@ def dav_decode(geo, params, z, store_f64=False):
     y = np.empty((B, int(g[36]), F * dav_hop(geo)), np.float32)
     _check(lib().orc_dav_decode(g.ctypes.data_as(_i32p), _p32(params), _p32(z), B, F,
                                 int(store_f64), _p32(y)), "dav_decode")
+    return y
+
+
+# --------------------------------------------- LTX bandwidth-extension tail
+
+
+def mel_frames(T, n_fft, hop) -> int:
+    return int(lib().orc_mel_frames(int(T), int(n_fft), int(hop)))
+
+
+def mel_stft(x, basis, mel_basis, hop, store_f64=False):
+    """The ltxaudio.rs page's causal log-mel (`MelStft::forward`): x [C, T],
+    basis [2 n_freqs, n_fft], mel_basis [n_mels, n_freqs] -> the folded
+    [C n_mels, frames] the extender reads."""
+    x, basis, mel_basis = _f32(x), _f32(basis), _f32(mel_basis)
+    C, T = x.shape
+    nf2, L = basis.shape
+    n_mels, nf = mel_basis.shape
+    assert nf2 == 2 * nf
+    frames = mel_frames(T, L, hop)
+    out = np.empty((C * n_mels, frames), np.float32)
+    _check(lib().orc_mel_stft(_p32(x), C, T, _p32(basis), nf, L, hop, _p32(mel_basis), n_mels,
+                              int(store_f64), _p32(out)), "mel_stft")
+    return out
+
+
+def hann_sinc_upsample(x, ratio, store_f64=False):
+    """The ltxaudio.rs page's `hann_sinc_upsample`: x [C, T] -> [C, ratio T]."""
+    x = _f32(x)
+    C, T = x.shape
+    y = np.empty((C, ratio * T), np.float32)
+    _check(lib().orc_hann_sinc_upsample(_p32(x), C, T, ratio, int(store_f64), _p32(y)),
+           "hann_sinc_upsample")
+    return y
+
+
+def bwe_tail(geo, params, low, basis, mel_basis, hop, ratio, filt=None, store_f64=False):
+    """The ltxaudio.rs page's `AudioStack::decode_from_mel` after the first
+    generator: low [C, T] -> clamp(extender(log-mel(low)) + upsample(low)),
+    [C, ratio T]."""
+    g = geometry_ints(geo)
+    low, params = _f32(low), _f32(params)
+    basis, mel_basis = _f32(basis), _f32(mel_basis)
+    C, T = low.shape
+    nf2, L = basis.shape
+    n_mels, nf = mel_basis.shape
+    f = kaiser_sinc() if filt is None else _f32(filt)
+    y = np.empty((C, ratio * T), np.float32)
+    _check(lib().orc_bwe_tail(g.ctypes.data_as(_i32p), _p32(params), _p32(low), C, T,
+                              _p32(basis), nf, L, hop, _p32(mel_basis), n_mels, ratio, _p32(f),
+                              _p32(f), len(f), int(store_f64), _p32(y)), "bwe_tail")
     return y

@@ -860,3 +860,146 @@ int orc_dav_decode(const int *g, const float *params, const float *z, int B, int
     free(a); free(b); free(r); free(acc);
     return ORC_OK;
 }
+
+/* ------------------------------------------- LTX bandwidth-extension tail */
+
+/* The causal log-mel the bandwidth extender is conditioned on ([LTX]
+ * `MelStft::forward`): the signal x [C, T] is left-padded with
+ * L - hop zeros, frame f starts at f hop, frames = (T + L - hop - L)/hop + 1,
+ *   re[r] = sum_j v[j] basis[r, j],  im[r] = sum_j v[j] basis[n_freqs + r, j],
+ *   mag[r] = sqrt(re^2 + im^2)                       (stored as float),
+ *   mel[m] = ln(max(sum_r mel_basis[m, r] mag[r], 1e-5)),
+ * written in the generator's folded layout out[c n_mels + m, f] ([LTX]
+ * `Vocoder::forward` folds (channel, mel) into one channel axis).
+ * basis [2 n_freqs, L] (DFT x window rows), mel_basis [n_mels, n_freqs]. */
+int orc_mel_stft(const float *x, int C, int T, const float *basis, int n_freqs, int L,
+                 int hop, const float *mel_basis, int n_mels, int store_f64, float *out) {
+    if (C <= 0 || T <= 0 || n_freqs <= 0 || L <= 0 || hop <= 0 || n_mels <= 0) return ORC_ERR_ARG;
+    long left = L > hop ? L - hop : 0;
+    long padded = T + left;
+    if (padded < L) return ORC_ERR_ARG;
+    long frames = (padded - L) / hop + 1;
+    double *mag = (double *)malloc((size_t)n_freqs * sizeof(double));
+    if (!mag) return ORC_ERR_NOMEM;
+    for (int c = 0; c < C; ++c)
+        for (long f = 0; f < frames; ++f) {
+            long start = f * hop;
+            for (int r = 0; r < n_freqs; ++r) {
+                double re = 0.0, im = 0.0;
+                for (int j = 0; j < L; ++j) {
+                    long idx = start + j;
+                    double v = 0.0;
+                    if (idx >= left && idx - left < T) v = (double)x[(size_t)c * T + (idx - left)];
+                    re += v * (double)basis[(size_t)r * L + j];
+                    im += v * (double)basis[(size_t)(n_freqs + r) * L + j];
+                }
+                mag[r] = rnd(sqrt(re * re + im * im), store_f64);
+            }
+            for (int m = 0; m < n_mels; ++m) {
+                double acc = 0.0;
+                for (int r = 0; r < n_freqs; ++r)
+                    acc += (double)mel_basis[(size_t)m * n_freqs + r] * mag[r];
+                out[((size_t)c * n_mels + m) * frames + f] =
+                    (float)log(acc > 1e-5 ? acc : 1e-5);
+            }
+        }
+    free(mag);
+    return ORC_OK;
+}
+
+/* Frames of orc_mel_stft for T samples. */
+long orc_mel_frames(int T, int L, int hop) {
+    long left = L > hop ? L - hop : 0;
+    return (T + left - L) / hop + 1;
+}
+
+/* The x ratio Hann-windowed sinc upsampler ([LTX] `hann_sinc_upsample`,
+ * rolloff 0.99, window half-width 6 zero crossings): width = ceil(6/0.99),
+ * k = 2 width ratio + 1 taps
+ *   filt[a] = sinc(ta) cos^2(clamp(ta, -6, 6) pi / 12) 0.99 / ratio,
+ *   ta = (a / ratio - width) 0.99,
+ * then, on x replicate-padded by `width` samples each side (scaled by ratio),
+ * a transposed FIR acc[p ratio + a] += v_p filt[a], trimmed to
+ * [2 width ratio, full - (k - ratio)): ratio T samples per row.
+ * x [C, T] -> y [C, ratio T]. */
+int orc_hann_sinc_upsample(const float *x, int C, int T, int ratio, int store_f64, float *y) {
+    if (C <= 0 || T <= 0 || ratio <= 0) return ORC_ERR_ARG;
+    const double rolloff = 0.99, lpw = 6.0;
+    int width = (int)ceil(lpw / rolloff);
+    int k = 2 * width * ratio + 1;
+    int pad = width;
+    long pad_left = 2L * width * ratio, pad_right = k - ratio;
+    double *filt = (double *)malloc((size_t)k * sizeof(double));
+    long tp = T + 2L * pad;
+    long full = (tp - 1) * ratio + k;
+    double *acc = (double *)malloc((size_t)full * sizeof(double));
+    if (!filt || !acc) { free(filt); free(acc); return ORC_ERR_NOMEM; }
+    for (int a = 0; a < k; ++a) {
+        double ta = ((double)a / ratio - width) * rolloff;
+        double tc = ta < -lpw ? -lpw : (ta > lpw ? lpw : ta);
+        double win = cos(tc * M_PI / lpw / 2.0);
+        win *= win;
+        double s = ta == 0.0 ? 1.0 : sin(M_PI * ta) / (M_PI * ta);
+        filt[a] = (double)(float)(s * win * rolloff / ratio);  /* the page's float taps */
+    }
+    long t2 = full - pad_right - pad_left;
+    for (int c = 0; c < C; ++c) {
+        for (long q = 0; q < full; ++q) acc[q] = 0.0;
+        for (long p = 0; p < tp; ++p) {
+            long src = p - pad;
+            src = src < 0 ? 0 : (src > T - 1 ? T - 1 : src);
+            double v = (double)x[(size_t)c * T + src] * ratio;
+            for (int a = 0; a < k; ++a) acc[p * ratio + a] += v * filt[a];
+        }
+        for (long i = 0; i < t2; ++i) y[(size_t)c * t2 + i] = (float)rnd(acc[pad_left + i], store_f64);
+    }
+    free(filt); free(acc);
+    return ORC_OK;
+}
+
+/* The bandwidth-extension tail ([LTX] `AudioStack::decode_from_mel` after the
+ * first generator): low [C, T] at the input rate is zero-padded to a whole
+ * number of mel hops, its log-mel (orc_mel_stft, folded) drives the extender
+ * (a decoder of geometry g on one row of C n_mels channels, C outputs, no
+ * final op -- its output is a residual), the padded low signal is upsampled
+ * by `ratio` (orc_hann_sinc_upsample), and
+ *   y[c, i] = clamp(residual[c, i] + skip[c, i], -1, 1),  i < ratio T.
+ * g's out_channels must be C, in_channels C n_mels and its hop
+ * ratio x mel hop. */
+int orc_bwe_tail(const int *g, const float *params, const float *low, int C, int T,
+                 const float *basis, int n_freqs, int L, int hop, const float *mel_basis,
+                 int n_mels, int ratio, const float *up, const float *down, int FK,
+                 int store_f64, float *y) {
+    if (!geo_ok(g) || C <= 0 || T <= 0 || ratio <= 0) return ORC_ERR_ARG;
+    if (g[G_IN] != C * n_mels || g[G_OUT] != C) return ORC_ERR_ARG;
+    long ghop = 1;
+    for (int i = 0; i < g[G_NUP]; ++i) ghop *= g[G_RATE + i];
+    if (ghop != (long)ratio * hop) return ORC_ERR_ARG;
+    long Tp = T % hop == 0 ? T : T + hop - T % hop;
+    float *padded = (float *)calloc((size_t)C * Tp, sizeof(float));
+    long frames = orc_mel_frames((int)Tp, L, hop);
+    float *mel = (float *)malloc((size_t)C * n_mels * frames * sizeof(float));
+    float *res = (float *)malloc((size_t)C * frames * ghop * sizeof(float));
+    float *skip = (float *)malloc((size_t)C * ratio * Tp * sizeof(float));
+    int rc = ORC_ERR_NOMEM;
+    if (padded && mel && res && skip) {
+        for (int c = 0; c < C; ++c)
+            memcpy(padded + (size_t)c * Tp, low + (size_t)c * T, (size_t)T * sizeof(float));
+        rc = orc_mel_stft(padded, C, (int)Tp, basis, n_freqs, L, hop, mel_basis, n_mels,
+                          store_f64, mel);
+        if (rc == ORC_OK)
+            rc = orc_decode(g, params, mel, 1, (int)frames, up, down, FK, 1e-9, store_f64, res);
+        if (rc == ORC_OK) rc = orc_hann_sinc_upsample(padded, C, (int)Tp, ratio, store_f64, skip);
+        if (rc == ORC_OK) {
+            long n = (long)ratio * T;
+            long rt = frames * ghop, st = (long)ratio * Tp;
+            for (int c = 0; c < C; ++c)
+                for (long i = 0; i < n; ++i) {
+                    double v = (double)res[(size_t)c * rt + i] + (double)skip[(size_t)c * st + i];
+                    y[(size_t)c * n + i] = (float)(v < -1.0 ? -1.0 : (v > 1.0 ? 1.0 : v));
+                }
+        }
+    }
+    free(padded); free(mel); free(res); free(skip);
+    return rc;
+}

@@ -694,3 +694,90 @@ def test_dav_batch_independence(oracle):
     y = oracle.dav_decode(geo, params, z)
     for b in range(2):
         np.testing.assert_array_equal(oracle.dav_decode(geo, params, z[b:b + 1]), y[b:b + 1])
+
+
+# ---------------------------------------------- LTX bandwidth-extension tail
+
+
+def test_mel_basis_is_torchaudio_slaney():
+    """The synthesised mel filterbank (an input: the checkpoint's is not
+    available) equals torchaudio's Slaney-scale, Slaney-normalised bank."""
+    import torchaudio
+    sp = synth.LTX_BWE_SPEC
+    _, mel = sp.bases()
+    want = torchaudio.functional.melscale_fbanks(sp.n_fft // 2 + 1, sp.fmin, sp.fmax, sp.n_mels,
+                                                 sp.in_rate, norm="slaney",
+                                                 mel_scale="slaney").numpy().T
+    np.testing.assert_allclose(mel, want, rtol=1e-5, atol=1e-7)
+
+
+@pytest.mark.parametrize("n_fft,hop,T", [(512, 80, 1600), (128, 80, 803), (64, 16, 100)])
+def test_mel_stft_matches_torch_stft(oracle, n_fft, hop, T):
+    """The causal log-mel against torch.stft (periodic Hann window, no
+    centring) of the signal left-padded with n_fft - hop zeros, then the mel
+    bank and log(max(., 1e-5)), folded to [C n_mels, frames]."""
+    rng = np.random.default_rng(n_fft + T)
+    x = (0.3 * rng.standard_normal((2, T))).astype(np.float32)
+    basis = synth.stft_basis(n_fft)
+    mel = synth.slaney_mel_basis(16000, n_fft, 24, 0.0, 8000.0)
+    got = oracle.mel_stft(x, basis, mel, hop)
+    xp = torch.nn.functional.pad(torch.as_tensor(x, dtype=torch.float64), (n_fft - hop, 0))
+    S = torch.stft(xp, n_fft=n_fft, hop_length=hop, win_length=n_fft,
+                   window=torch.hann_window(n_fft, periodic=True, dtype=torch.float64),
+                   center=False, return_complex=True).abs()
+    m = torch.log(torch.clamp(torch.as_tensor(mel, dtype=torch.float64) @ S, min=1e-5))
+    want = m.reshape(2 * mel.shape[0], -1).numpy()
+    assert got.shape == want.shape and got.shape[1] == oracle.mel_frames(T, n_fft, hop)
+    np.testing.assert_allclose(got, want, rtol=1e-5, atol=2e-5)
+
+
+@pytest.mark.parametrize("T", [1, 5, 300])
+def test_hann_sinc_upsample_matches_torchaudio(oracle, T):
+    """x3 upsampling against torchaudio's Hann-windowed sinc resampler
+    (lowpass width 6, rolloff 0.99) run on the signal extended by 10
+    replicated samples each side: the page pads by replicating, torchaudio by
+    zeros, so the extension makes the two agree everywhere, edges included."""
+    import torchaudio
+    rng = np.random.default_rng(T)
+    x = rng.standard_normal((2, T)).astype(np.float32)
+    got = oracle.hann_sinc_upsample(x, 3, store_f64=True).astype(np.float64)
+    e = 10
+    xe = np.pad(x.astype(np.float64), ((0, 0), (e, e)), mode="edge")
+    ref = torchaudio.functional.resample(torch.as_tensor(xe), 1, 3, lowpass_filter_width=6,
+                                         rolloff=0.99,
+                                         resampling_method="sinc_interp_hann").numpy()
+    want = ref[:, 3 * e:3 * e + 3 * T]
+    assert got.shape == (2, 3 * T)
+    # the page rounds its taps to float: about 6e-8 of the sum of |taps| x |x|
+    np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-6)
+
+
+def _bwe_tiny():
+    geo = synth.LTX_BWE.replace(in_channels=2 * 16, pre_channels=48,
+                                up_channels=(32, 16, 16, 8, 8))
+    return geo, synth.BweSpec(in_rate=16000, ratio=3, n_fft=128, hop=80, n_mels=16, fmin=0.0,
+                              fmax=8000.0)
+
+
+def test_bwe_tail_is_its_composition(oracle):
+    """clamp(extender(log-mel(padded low)) + upsample(padded low)) over the
+    first 3 T samples, against the oracle's own steps: the low signal zero
+    padded to whole mel hops, the mel front end, one decode of the folded
+    stereo mel (2 outputs, no final op), the x3 skip, the clamped sum."""
+    geo, sp = _bwe_tiny()
+    s = synth.NormalStream(61)
+    T = 8 * sp.hop + 37  # not a whole number of hops
+    low = 0.3 * s.normal((2, T))
+    params = s.normal((synth.param_count(geo),), 0.0, 0.15)
+    basis, mel = sp.bases()
+    y = oracle.bwe_tail(geo, params, low, basis, mel, sp.hop, sp.ratio)
+    Tp = -(-T // sp.hop) * sp.hop
+    padded = np.zeros((2, Tp), np.float32)
+    padded[:, :T] = low
+    m = oracle.mel_stft(padded, basis, mel, sp.hop)
+    res = oracle.decode(geo, params, m[None])[0]
+    skip = oracle.hann_sinc_upsample(padded, sp.ratio)
+    want = np.clip(res[:, :3 * T].astype(np.float64) + skip[:, :3 * T], -1.0, 1.0)
+    assert y.shape == (2, 3 * T)
+    np.testing.assert_allclose(y, want, rtol=1e-6, atol=1e-7)
+    assert np.abs(y).max() <= 1.0 and np.abs(res).max() > 0
