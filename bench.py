@@ -39,13 +39,18 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=synth.H3_10S.name, choices=sorted(synth.DECODER_WORKLOADS))
+    ap.add_argument("--workload", default=synth.H3_60S_TILED.name,
+                    choices=sorted(synth.DECODER_WORKLOADS))
+    ap.add_argument("--activation-sweep", action="store_true",
+                    help="time the activation over the C x T sweep grid (B = 2) instead of "
+                         "the decoder; one JSON line with every shape")
     ap.add_argument("--cpu-sample-frames", type=int, default=40,
                     help="latent frames (one side) of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None,
                     help="time one kernel on one shape instead of the decoder (for profiling): "
                          "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s | "
+                         "actconv:BxCxT:K:d (activation then conv, the decoder's kernels) | "
                          "amp:BxCxT:K (an AMP block, dilations 1, 3, 5)")
     return ap.parse_args()
 
@@ -78,6 +83,18 @@ def run_case(args):
         b = torch.from_numpy(s.normal((Co,), 0, 0.02)).cuda()
         fn = lambda: native.bv_conv_transpose1d(x, w, b, st)  # noqa: E731
         work, unit = 2.0 * B * C * Co * 2 * st * T, "TFLOP/s"
+    elif kind == "actconv":
+        # one AMP-block step on the decoder's kernels: activation -> conv
+        K, d = int(rest[0]), int(rest[1])
+        la = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
+        lb = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
+        w = torch.from_numpy(s.normal((C, C, K), 0, 0.02)).cuda()
+        b = torch.from_numpy(s.normal((C,), 0, 0.02)).cuda()
+        y = torch.empty_like(x)
+        ws = torch.empty(native.lib().bv_act_conv1d_workspace_size(B, C, T, C, K, d) // 4 + 64,
+                         device="cuda")
+        fn = lambda: native.bv_act_conv1d(x, la, lb, filt, w, b, d, y=y, workspace=ws)  # noqa: E731
+        work, unit = 2.0 * B * C * C * K * T, "TFLOP/s"
     elif kind == "amp":
         K = int(rest[0])
         wl = synth.AmpWorkload("case", B, C, T, K, (1, 3, 5), seed=7)
@@ -120,51 +137,107 @@ TF32_PER_BF16 = 1.1 / 2.25
 
 def peaks():
     """Roofline denominators: the measured copy bandwidth and bf16 GEMM
-    rate of this machine's B200s, else the profiling recipe's fallback."""
+    rates of this machine's B200s (a burst, and a seconds-long loop under the
+    power cap with the SM clock it settled at), else the profiling recipe's
+    fallback (1.59 PFLOP/s burst, about 1.4 sustained near 1.3 GHz)."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    out = {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0,
+           "sustained_mhz": 1300.0, "sm_max_mhz": 1965.0, "source": "fallback"}
     if os.path.exists(p):
         with open(p) as fh:
             d = json.load(fh)
-        return {"hbm_gbs": d.get("hbm_gbs", 6650.0), "bf16": d.get("bf16_tflops", 1590.0),
-                "bf16_sustained": d.get("bf16_tflops_sustained", 1400.0),
-                "sm_max_mhz": d.get("sm_max_mhz", 1965.0), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "sm_max_mhz": 1965.0,
-            "source": "fallback"}
+        out["source"] = "measured"
+        out["hbm_gbs"] = float(d.get("hbm_gbs", out["hbm_gbs"]))
+        out["bf16"] = float(d.get("bf16_tflops", out["bf16"]))
+        out["bf16_sustained"] = float(d.get("bf16_tflops_sustained", out["bf16_sustained"]))
+        flat = {}
+
+        def walk(v, pre=""):
+            if isinstance(v, dict):
+                for k, x in v.items():
+                    walk(x, f"{pre}{k}.")
+            elif isinstance(v, (int, float)):
+                flat[pre[:-1]] = float(v)
+        walk(d)
+        for k, v in flat.items():  # the clock the sustained figure was measured at
+            kl = k.lower()
+            if "mhz" in kl and "sustain" in kl and "max" not in kl:
+                out["sustained_mhz"] = v
+            elif "mhz" in kl and "max" in kl:
+                out["sm_max_mhz"] = v
+    return out
+
+
+def tensor_peak(pk, clocks):
+    """Useful 3xTF32 peak for a kernel timed inside a decode: the bf16 figure
+    x the nominal tf32/bf16 ratio / 3 products.  The burst figure applies when
+    the timed region ran at the maximum SM clock with no power capping; under
+    capping or a lower clock, the sustained figure scaled by the measured clock
+    over the clock the sustained figure was taken at.  Returns (peak, source,
+    burst peak)."""
+    burst = pk["bf16"] * TF32_PER_BF16 / 3.0
+    m = (clocks or {}).get("sm_mhz")
+    mx = (clocks or {}).get("sm_max_mhz") or pk["sm_max_mhz"]
+    capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
+    if m is None:
+        return burst, f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s (no clock samples)", burst
+    if not capped and m >= 0.97 * mx:
+        return burst, (f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x tf32/bf16 "
+                       f"{TF32_PER_BF16:.3f} / 3 (3xTF32); SM clock {m:.0f} of {mx:.0f} MHz, "
+                       f"no power cap"), burst
+    peak = pk["bf16_sustained"] * m / pk["sustained_mhz"] * TF32_PER_BF16 / 3.0
+    return peak, (f"{pk['source']} bf16 sustained {pk['bf16_sustained']} TFLOP/s at "
+                  f"{pk['sustained_mhz']:.0f} MHz scaled to the measured {m:.0f} MHz, x tf32/bf16 "
+                  f"{TF32_PER_BF16:.3f} / 3 (3xTF32); power cap {'seen' if capped else 'not seen'}"), \
+        burst
 
 
 # kernel classes that run 3xTF32 on the tensor cores
 TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm")
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of a full decode of the bench workload, per kernel class, for the
-# kernel code as committed with it (profiles/conv1d_tm_traffic_h3_10s.md);
-# a class missing here reports null.
-NCU_TRAFFIC_PER_LAUNCH = {"conv1d_tm": 84.65e6}
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
+# ncu capture of a few launches, per kernel class, for the kernel code named
+# beside it; null for a class without a capture of its current code.
+NCU_TRAFFIC_PER_LAUNCH = {}
 
 
-def roofline_for(name, kd, pk):
+def roofline_for(name, kd, pk, clocks=None):
     """Achieved vs peak for one kernel class; achieved = algorithmic work per
-    launch / average launch time."""
+    launch / average launch time (CUDA events on the launching stream)."""
     t = kd["avg_launch_ms"] / 1000.0
     if name in TENSOR_CLASSES:
         # useful FLOPs of the 3xTF32 conv; the tensor pipe issues 3 TF32 MMAs each
-        peak = pk["bf16_sustained"] * TF32_PER_BF16 / 3.0
+        peak, src, burst = tensor_peak(pk, clocks)
         ach = kd["flops"] / t / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
-                "peak_source": f"{pk['source']} bf16 sustained {pk['bf16_sustained']} TFLOP/s x "
-                               f"tf32/bf16 {TF32_PER_BF16:.3f} / 3 (3xTF32)"}
+                "frac": ach / peak, "frac_of_burst": ach / burst,
+                "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name), "peak_source": src}
+    mhz = (clocks or {}).get("sm_max_mhz") or pk["sm_max_mhz"]
     if kd["flops"] > 0:
-        peak = SMS * FP32_LANES_PER_SM * 2 * pk["sm_max_mhz"] * 1e6 / 1e12
+        peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
         ach = kd["flops"] / t / 1e12
         return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": None,
+                "frac": ach / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
                 "peak_source": f"FP32 pipe: {SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 x "
-                               f"{pk['sm_max_mhz']:.0f} MHz"}
+                               f"{mhz:.0f} MHz"}
     ach = kd["bytes"] / t / 1e9
     return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / pk["hbm_gbs"], "traffic": None,
+            "frac": ach / pk["hbm_gbs"], "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
             "peak_source": f"{pk['source']} hbm_gbs"}
+
+
+def host_cpu():
+    """CPU model and logical core count of this host."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
 
 
 class ClockSampler:
@@ -266,7 +339,7 @@ def run_reference(args, world, rank):
     w = synth.DECODER_WORKLOADS[args.workload]
     import oracle
     z, params = w.make()
-    frames = 3
+    frames = 4
     zs = np.ascontiguousarray(z[:1, :, :frames])
     audio = frames * w.geometry.hop / w.geometry.sample_rate
     for _ in range(args.warmup):
@@ -284,12 +357,57 @@ def run_reference(args, world, rank):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000 * statistics.mean(times), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "batch": 1, "frames": frames},
+        "config": {"workload": w.name, "batch": w.batch, "frames": w.frames,
+                   "tile_frames": w.tile_frames, "overlap_frames": w.overlap_frames,
+                   "timed_sample": {"batch": 1, "frames": frames}},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, **host_cpu()},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_activation_sweep(args):
+    """The activation over the sweep grid: per shape, W warm-up and K timed
+    launches (CUDA events on the launching stream, L2 evicted between
+    launches outside the events); achieved = 8 B per element / median time."""
+    import torch
+    from bigvgan_waveform_decoder_alias_b200 import native
+    torch.cuda.set_device(0)
+    pk = peaks()
+    filt = torch.from_numpy(native.bv_filter_design()).cuda()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, device="cuda")
+    B = 2
+    rows = []
+    with ClockSampler(0) as clk:
+        for C, T in synth.ACT_SWEEP_GRID:
+            # timing only: inputs of the workload's distribution drawn on the
+            # device (the parity tests use the seeded host stream)
+            g = torch.Generator(device="cuda").manual_seed(synth.ACT_SWEEP.seed)
+            x = torch.randn((B, C, T), device="cuda", generator=g)
+            la = torch.randn((C,), device="cuda", generator=g) * synth.SNAKE_STD
+            lb = torch.randn((C,), device="cuda", generator=g) * synth.SNAKE_STD
+            y = torch.empty_like(x)
+            for _ in range(max(args.warmup, 3)):
+                native.bv_activation1d(x, la, lb, filt, y=y)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            for k in range(args.steps):
+                flush.fill_(float(k))
+                ev[k][0].record()
+                native.bv_activation1d(x, la, lb, filt, y=y)
+                ev[k][1].record()
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            gbs = 8.0 * B * C * T / (ms / 1000) / 1e9
+            rows.append({"C": C, "T": T, "ms": ms, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"]})
+            del x, y
+    print(json.dumps({"mode": "activation_sweep", "batch": B, "unit": "GB/s",
+                      "peak": pk["hbm_gbs"], "peak_source": f"{pk['source']} hbm_gbs",
+                      "steps": args.steps, "warmup": args.warmup,
+                      "l2": "evicted between launches (256 MiB write outside the events)",
+                      "shapes": rows, "clocks": clk.summary()}), flush=True)
     return 0
 
 
@@ -298,6 +416,8 @@ def main():
     world, rank, local = dist_init()
     if args.case:
         return run_case(args)
+    if args.activation_sweep:
+        return run_activation_sweep(args)
     if args.impl == "reference":
         return run_reference(args, world, rank)
 
@@ -384,10 +504,11 @@ def main():
     Lb.bv_timing_enable(1)
     Lb.bv_timing_reset()
     prof_steps = min(args.steps, 5)
-    for k in range(prof_steps):
-        flush.fill_(float(k))
-        dec.decode(zd, y=y, workspace=ws)
-    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk_prof:
+        for k in range(prof_steps):
+            flush.fill_(float(k))
+            dec.decode(zd, y=y, workspace=ws)
+        torch.cuda.synchronize()
     Stats = native.KernelStats * 16
     st = Stats()
     n = Lb.bv_timing_read(st, 16)
@@ -401,7 +522,8 @@ def main():
                                     "bytes": s.bytes / max(s.launches, 1),
                                     "avg_launch_ms": s.ms / max(s.launches, 1)}
     pk = peaks()
-    roofs = {name: roofline_for(name, kd, pk) for name, kd in kernels.items()}
+    prof_clocks = clk_prof.summary()
+    roofs = {name: roofline_for(name, kd, pk, prof_clocks) for name, kd in kernels.items()}
     for name, r in roofs.items():
         kernels[name]["roofline"] = r
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
@@ -424,7 +546,7 @@ def main():
         cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
                "sample": f"oracle decode of one side, first {args.cpu_sample_frames} latent "
                          f"frames ({audio:.3f} s of audio) of {w.name}, "
-                         f"{statistics.mean(times):.1f} s"}
+                         f"{statistics.mean(times):.1f} s", **host_cpu()}
 
     if rank == 0:
         line = {
@@ -446,6 +568,7 @@ def main():
             "kernels": kernels,
             "cpu_baseline": cpu,
             "clocks": clk.summary(),
+            "clocks_profiled_pass": prof_clocks,
             "output_finite": finite,
         }
         print(json.dumps(line), flush=True)
