@@ -35,6 +35,7 @@ def test_static_scratch_amp_block_matches_workspace_version():
 
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
     cases = [synth.AMP_BLOCK_C32, synth.AmpWorkload("c96", 2, 96, 3001, 7, (1, 3, 5), seed=5)]
+    params = {}
     for w in cases:
         x, flat = w.make()
         tensors, off = {}, 0
@@ -43,6 +44,7 @@ def test_static_scratch_amp_block_matches_workspace_version():
             tensors[name] = torch.from_numpy(flat[off:off + n].reshape(shape)).cuda()
             off += n
         p = native.amp_params(w.kernel, w.dilations, tensors, filt)
+        params[w.name] = (p, tensors)  # the tensors must outlive the pointers in p
         xd = torch.from_numpy(x).cuda()
         want = native.bv_amp_block(xd, p).cpu().numpy()
         for call in range(2):
@@ -65,11 +67,25 @@ def test_static_scratch_amp_block_matches_workspace_version():
         ref = 0.5 * want.astype(np.float64) + y0.cpu().numpy()
         assert rel_l2(y.cpu().numpy(), ref) < LAYER_TOL
 
-    # more than the static scratch holds: a clear error, output untouched
-    big_t = (1 << 20) // 32 + 1
+    # the 32-channel block's own parameters for the size limits
+    p32, _ = params[synth.AMP_BLOCK_C32.name]
+    limit = 1 << 20  # BV_AMP_STATIC_MAX_ELEMS in include/bv.h
+    # exactly the limit: B * C * T == BV_AMP_STATIC_MAX_ELEMS runs and matches
+    t_max = limit // 32
+    xd = torch.from_numpy(synth.NormalStream(4).normal((1, 32, t_max))).cuda()
+    want = native.bv_amp_block(xd, p32).cpu().numpy()
+    y = torch.full_like(xd, float("nan"))
+    rc = L.bv_amp_block_static(ctypes.c_void_p(xd.data_ptr()), 1, 32, t_max, ctypes.byref(p32),
+                               ctypes.c_void_p(y.data_ptr()), 1.0, 0, stream)
+    assert rc == 0, native.last_error()
+    assert rel_l2(y.cpu().numpy(), want) < LAYER_TOL
+
+    # one element more than the static scratch holds: a clear error, output untouched
+    big_t = t_max + 1
     xd = torch.zeros((1, 32, big_t), device="cuda")
     y = torch.full_like(xd, 7.0)
-    rc = L.bv_amp_block_static(ctypes.c_void_p(xd.data_ptr()), 1, 32, big_t, ctypes.byref(p),
+    rc = L.bv_amp_block_static(ctypes.c_void_p(xd.data_ptr()), 1, 32, big_t, ctypes.byref(p32),
                                ctypes.c_void_p(y.data_ptr()), 1.0, 0, stream)
     assert rc == 3 and "static scratch limit" in native.last_error()
+    torch.cuda.synchronize()
     assert bool((y == 7.0).all())
