@@ -79,12 +79,17 @@ def main():
             nt = oracle.tile_count(w.frames, w.tile_frames, w.overlap_frames)
             starts = [k * step for k in range(nt)]
             # tiles 0-1 fix every sample before tile 2 starts; the last two
-            # tiles fix every sample after tile nt-3 ends
+            # tiles fix every sample after tile nt-3 ends; two middle tiles m,
+            # m+1 fix every sample between the end of tile m-1 and the start
+            # of tile m+2
             head = (0, starts[2] * hop, [starts[1] * hop, w.tile_frames * hop])
             tail_lo = (starts[nt - 3] + w.tile_frames) * hop
             tail = (tail_lo, L, [starts[nt - 1] * hop, (starts[nt - 2] + w.tile_frames) * hop])
-            plans[name] = (positions(L, [head, tail], 4096, w.seed),
-                           [(0, 2), (nt - 2, nt)])
+            m = nt // 2
+            mid = ((starts[m - 1] + w.tile_frames) * hop, starts[m + 2] * hop,
+                   [starts[m + 1] * hop, (starts[m] + w.tile_frames) * hop])
+            plans[name] = (positions(L, [head, mid, tail], 4096, w.seed),
+                           [(0, 2), (m, m + 2), (nt - 2, nt)])
         else:
             plans[name] = (positions(L, [(0, L, [])], 4096, w.seed), [None])
 
