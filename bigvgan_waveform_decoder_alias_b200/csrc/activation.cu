@@ -207,6 +207,9 @@ __device__ __forceinline__ void load_taps(float2 (&F)[12], const float2 *taps) {
 // whose chunks start at 3 L + 1 in the padded layout).  The slots s < 10 are
 // written to the other buffer's slots s + 2 TW too (mirror), where the
 // previous tile's stage B reads them.
+// TAIL: lanes 0-9 also compute the 10 pairs past the tile's end from its own
+// window (as stage_a_tail does), with the taps and constants already loaded.
+template <bool TAIL = false>
 __device__ __forceinline__ void stage_a(const float *xb, float *vb, float *vmirror,
                                         const float2 *taps, const float2 *cst, float up_abs,
                                         int lane) {
@@ -239,13 +242,25 @@ __device__ __forceinline__ void stage_a(const float *xb, float *vb, float *vmirr
       const float2 v1 = snake2<CK>(up2<0>(U2, X + n / 2 + 1), k, cst);
       const float4 o = make_float4(v0.x, v0.y, v1.x, v1.y);
       *reinterpret_cast<float4 *>(vl + 2 * n) = o;
-      if (8 * lane + n < 10) *reinterpret_cast<float4 *>(vmirror + voff(8 * lane + n + 2 * TW)) = o;
+      if (vmirror && 8 * lane + n < 10)
+        *reinterpret_cast<float4 *>(vmirror + voff(8 * lane + n + 2 * TW)) = o;
     }
   };
   if (mx * up_abs * fmaxf(k.A.x, k.A.y) <= kWLimit)
     run(std::false_type{});
   else
     run(std::true_type{});
+  if (TAIL && lane < 10) {
+    // pair s = 2 TW + i, i = lane: lanes 0-4 phase 1 at q = TW + L, lanes
+    // 5-9 phase 0 at q = TW + L - 4 (the layout of stage_a_tail)
+    const int R = lane < 5 ? 1 : 0;
+    const int q = lane < 5 ? TW + lane : TW + lane - 4;
+    float2 xp[6];
+#pragma unroll
+    for (int j = 0; j < 6; ++j) xp[j] = *reinterpret_cast<const float2 *>(xb + xoff(2 + q + R + j));
+    const float2 u = R ? up2<1>(U2, xp) : up2<0>(U2, xp);
+    *reinterpret_cast<float2 *>(vb + voff(2 * q + R - 1)) = snake2<true>(u, k, cst);
+  }
 }
 
 // The 10 pairs s in [2 TW, 2 TW + 10) of a tile, from its own input window:
@@ -298,11 +313,105 @@ __device__ __forceinline__ void copy_pair(float *vb, int dst, int src) {
   *reinterpret_cast<float2 *>(vb + voff(dst)) = *reinterpret_cast<const float2 *>(vb + voff(src));
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
-activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, int C, int T,
-                  int tiles_per_row, long long n_tiles, const float *__restrict__ log_alpha,
-                  const float *__restrict__ log_beta, const float *__restrict__ f_up,
-                  const float *__restrict__ f_dn, float eps) {
+// ---------------------------------------------------------------------------
+// The same activation writing the operand planes of the time-major
+// tensor-core conv instead of [B, C, T]: hi[b, t, c] = tf32(y[b, c, t]) and
+// lo = y - hi, so the activation's output never exists in [B, C, T] form and
+// no separate transpose pass reads it back.
+//
+// A CTA holds two teams of four warps.  A team owns a contiguous range of
+// tasks (8-channel group of one batch row, time tile), group-major; warp k of
+// the team takes the group's row pair k (channels 2k, 2k + 1) and walks the
+// range's tiles exactly as activation_kernel walks a row pair, so consecutive
+// tiles share their 2x-rate values and the SnakeBeta constants are set up
+// once per row pair.  Stage B writes the pair's TW outputs into the team's
+// staging buffer, one region per row pair ([4][RP] floats, time steps as
+// (channel 2k, 2k + 1) pairs); after a named barrier over the team each warp
+// writes a quarter of the tile (32 time steps x 8 channels) to both planes as
+// 32-byte rows, whole sectors.  Two staging buffers alternate, so one
+// barrier per tile orders both the writes before the flush and the flush
+// before the buffer's next use.
+constexpr int TEAM = 4;                 // warps per team (row pairs of a group)
+constexpr int TM_CH = 2 * TEAM;         // channels per group
+constexpr int RP = 2 * TW + 8;          // region pitch: 2 RP = 16 (mod 32) banks apart
+constexpr int STG_FLOATS = TEAM * RP;   // one staging buffer
+constexpr size_t TM_SMEM_BYTES =
+    SMEM_BYTES + (size_t)(WARPS / TEAM) * 2 * STG_FLOATS * sizeof(float);
+static_assert(WARPS % TEAM == 0 && RP % 32 == 8 && STG_FLOATS % 4 == 0, "staging layout");
+
+// Barrier 1 + team over the team's warps (immediate ids, so that the kernel
+// reserves only the barriers it uses).
+__device__ __forceinline__ void team_barrier(int team) {
+  static_assert(WARPS / TEAM == 2, "two teams");
+  if (team == 0)
+    asm volatile("bar.sync 1, %0;\n" ::"n"(32 * TEAM) : "memory");
+  else
+    asm volatile("bar.sync 2, %0;\n" ::"n"(32 * TEAM) : "memory");
+}
+
+// Stage B of row pair k into its staging region: lane L holds t = 4 L + e,
+// stored as (channel 2k, 2k + 1) pairs, two 16-byte stores per lane.
+__device__ __forceinline__ void stage_b_stage(const float *vb, const float2 *taps, float *region,
+                                              int lane) {
+  float2 D2[12];
+  load_taps(D2, taps + 12);
+  float2 W[18];
+  const float *vl = vb + 20 * lane;
+#pragma unroll
+  for (int m = 0; m < 9; ++m) {
+    const float4 v = *reinterpret_cast<const float4 *>(vl + 4 * (m + m / 4));
+    W[2 * m] = make_float2(v.x, v.y);
+    W[2 * m + 1] = make_float2(v.z, v.w);
+  }
+  float2 out[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    float2 acc = mul2(D2[0], W[2 * e]);
+#pragma unroll
+    for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j], acc);
+    out[e] = acc;
+  }
+  float4 *r4 = reinterpret_cast<float4 *>(region + 8 * lane);
+  r4[0] = make_float4(out[0].x, out[0].y, out[1].x, out[1].y);
+  r4[1] = make_float4(out[2].x, out[2].y, out[3].x, out[3].y);
+}
+
+// Warp k's quarter of a staged tile: time steps 32 k .. 32 k + 31, per round
+// 16 time steps x two 4-channel halves (lane pair = one 32-byte row of a
+// plane).  The half's channels are the pairs of regions 2 h and 2 h + 1.
+__device__ __forceinline__ void flush_quarter(const float *sb, float *__restrict__ hi,
+                                              float *__restrict__ lo, size_t obase, int C,
+                                              int t0, int T, int k, int lane) {
+  const int h = lane & 1;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int tl = 32 * k + 16 * r + (lane >> 1), t = t0 + tl;
+    const float2 a = *reinterpret_cast<const float2 *>(sb + (2 * h) * RP + 2 * tl);
+    const float2 c = *reinterpret_cast<const float2 *>(sb + (2 * h + 1) * RP + 2 * tl);
+    if (t < T) {
+      const float v[4] = {a.x, a.y, c.x, c.y};
+      float g[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) g[q] = __uint_as_float(__float_as_uint(v[q]) & 0xFFFFE000u);
+      const size_t o = obase + (size_t)t * C + 4 * h;
+      *reinterpret_cast<float4 *>(hi + o) = make_float4(g[0], g[1], g[2], g[3]);
+      *reinterpret_cast<float4 *>(lo + o) =
+          make_float4(v[0] - g[0], v[1] - g[1], v[2] - g[2], v[3] - g[3]);
+    }
+  }
+}
+
+// The tile walk of both kernels.  TM = false: each warp owns a contiguous
+// range of (row pair, tile) ids, row pair major, and writes y [rows, T].
+// TM = true: each team owns a range of (8-channel group, tile) tasks and
+// warp k walks row pair 4 group + k of them, writing the hi/lo planes
+// [B, T, C] (y = hi).
+template <bool TM>
+__device__ __forceinline__ void activation_walk(
+    const float *__restrict__ x, float *__restrict__ y, float *__restrict__ lo, int rows, int C,
+    int T, int tiles_per_row, long long n_ids, const float *__restrict__ log_alpha,
+    const float *__restrict__ log_beta, const float *__restrict__ f_up,
+    const float *__restrict__ f_dn, float eps) {
   extern __shared__ __align__(16) float smem[];
   __shared__ __align__(16) float2 taps[24];  // 2 f_up, then f_down, as broadcast pairs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -324,28 +433,46 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
   float *wsm = smem + (size_t)warp * WARP_FLOATS;
   float *const xs0 = wsm, *const vs0 = wsm + 2 * XS_FLOATS;  // buffer b at + b * size
   float2 *cst = reinterpret_cast<float2 *>(wsm + 2 * XS_FLOATS + 2 * VS_FLOATS);
+  const int team = warp / TEAM, k = warp % TEAM;
+  float *const stg = smem + (size_t)WARPS * WARP_FLOATS + (size_t)team * 2 * STG_FLOATS;
 
-  // this warp's contiguous range of tiles (row pair * tiles_per_row + tile)
-  const long long nw = (long long)gridDim.x * WARPS;
-  const long long gw = (long long)blockIdx.x * WARPS + warp;
-  const long long beg = gw * n_tiles / nw, end = (gw + 1) * n_tiles / nw;
+  // this warp's (or team's) contiguous range of ids (row pair or group) *
+  // tiles_per_row + tile
+  const long long nw = (long long)gridDim.x * (TM ? WARPS / TEAM : WARPS);
+  const long long gw = (long long)blockIdx.x * (TM ? WARPS / TEAM : WARPS) + (TM ? team : warp);
+  const long long beg = gw * n_ids / nw, end = (gw + 1) * n_ids / nw;
   if (beg >= end) return;
   auto row_ptr = [&](int pr, int which) {
     const int r = 2 * pr + which;
     return x + (size_t)(r < rows ? r : rows - 1) * T;
   };
+  constexpr int kStep = TM ? TEAM : 1;  // row pairs from one id row to the next
   int pair = (int)(beg / tiles_per_row), tile = (int)(beg % tiles_per_row);
+  if (TM) pair = TEAM * pair + k;
   issue_tile(row_ptr(pair, 0), row_ptr(pair, 1), xs0, tile * TW, T, lane);
   cp_async_commit();
   int cur_pair = -1;
   bool pending = false;  // stage B of the previous tile still to run
   int p_t0 = 0;
+  size_t obase = 0;  // TM: plane offset of the group's (b, t = 0, first channel)
+  int n_out = 0;     // TM: staged tiles so far (selects the staging buffer)
+  auto emit = [&](const float *vsrc, int t_out) {
+    if constexpr (TM) {
+      float *sb = stg + (n_out & 1) * STG_FLOATS;
+      ++n_out;
+      stage_b_stage(vsrc, taps, sb + k * RP, lane);
+      team_barrier(team);
+      flush_quarter(sb, y, lo, obase, C, t_out, T, k, lane);
+    } else {
+      stage_b(vsrc, taps, y + (size_t)(2 * pair) * T, 2 * pair + 1 < rows, t_out, T, lane);
+    }
+  };
   for (long long id = beg; id < end; ++id) {
     const int b = (int)((id - beg) & 1);
     int npair = pair, ntile = tile + 1;
     if (ntile == tiles_per_row) {
       ntile = 0;
-      ++npair;
+      npair += kStep;
     }
     __syncwarp();  // the previous iteration's reads of the buffers written below are done
     if (id + 1 < end)
@@ -377,6 +504,10 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
         cf[2 * kIb] = ib0;
         cf[2 * kIb + 1] = ib1;
       }
+      if (TM) {
+        const int row0 = 2 * (pair - k), bb = row0 / C;
+        obase = (size_t)bb * T * C + (row0 - bb * C);
+      }
     }
     cp_async_wait<1>();  // this tile's input has landed (the next one may be in flight)
     __syncwarp();
@@ -405,9 +536,7 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
       }
       __syncwarp();
     }
-    float *yp = y + (size_t)(2 * pair) * T;
-    const bool has_r1 = 2 * pair + 1 < rows;
-    if (pending) stage_b(vo, taps, yp, has_r1, p_t0, T, lane);
+    if (pending) emit(vo, p_t0);
     if (row_end || id + 1 == end) {
       // stage B of this tile now: its last 10 values come from its own window
       stage_a_tail(xb, vb, taps, cst, lane);
@@ -417,7 +546,7 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
         if (s >= 2 * TW && s < VP) copy_pair(vb, s, s_end);
       }
       __syncwarp();
-      stage_b(vb, taps, yp, has_r1, t0, T, lane);
+      emit(vb, t0);
       pending = false;
     } else {
       pending = true;
@@ -427,6 +556,24 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
     tile = ntile;
   }
   cp_async_wait<0>();
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, int C, int T,
+                  int tiles_per_row, long long n_tiles, const float *__restrict__ log_alpha,
+                  const float *__restrict__ log_beta, const float *__restrict__ f_up,
+                  const float *__restrict__ f_dn, float eps) {
+  activation_walk<false>(x, y, nullptr, rows, C, T, tiles_per_row, n_tiles, log_alpha, log_beta,
+                         f_up, f_dn, eps);
+}
+
+__global__ void __launch_bounds__(THREADS, 2)
+activation_tm_kernel(const float *__restrict__ x, float *__restrict__ hi, float *__restrict__ lo,
+                     int rows, int C, int T, int tiles_per_row, long long n_tasks,
+                     const float *__restrict__ log_alpha, const float *__restrict__ log_beta,
+                     const float *__restrict__ f_up, const float *__restrict__ f_dn, float eps) {
+  activation_walk<true>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha, log_beta, f_up,
+                        f_dn, eps);
 }
 
 __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restrict__ out,
@@ -458,7 +605,56 @@ int persistent_ctas() {
   return n;
 }
 
+int persistent_ctas_tm() {
+  constexpr int kMaxDev = 64;
+  static std::atomic<int> cache[kMaxDev];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int slot = dev >= 0 && dev < kMaxDev ? dev : 0;
+  int n = cache[slot].load(std::memory_order_relaxed);
+  if (n == 0) {
+    int sms = 148, per_sm = 2;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_tm_kernel, THREADS,
+                                                      TM_SMEM_BYTES) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    n = sms * per_sm;
+    cache[slot].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
 }  // namespace
+
+bool activation_tm_supported(int C) { return C % TM_CH == 0; }
+
+bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int C, int T,
+                               const float *la, const float *lb, const float *fu, const float *fd,
+                               float eps, cudaStream_t st) {
+  if (!activation_tm_supported(C))
+    return fail(BV_ERR_UNSUPPORTED, "activation_tm: C = %d is not a multiple of %d", C, TM_CH);
+  if (((reinterpret_cast<uintptr_t>(hi) | reinterpret_cast<uintptr_t>(lo)) & 15u) != 0)
+    return fail(BV_ERR_UNSUPPORTED, "activation_tm: planes not 16-byte aligned");
+  const long long rows = (long long)B * C;
+  if (rows > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "activation_tm: too many rows");
+  const int tiles = (T + TW - 1) / TW;
+  const long long n_tasks = rows / TM_CH * tiles;  // (group, tile) tasks
+  if (n_tasks <= 0) return BV_OK;
+  BV_TRY(ensure_dynamic_smem((const void *)activation_tm_kernel, TM_SMEM_BYTES,
+                             "activation_tm smem attribute"));
+  const long long ctas = persistent_ctas_tm();
+  const long long need = (n_tasks + WARPS / TEAM - 1) / (WARPS / TEAM);
+  const long long grid = need < ctas ? need : ctas;
+  {
+    // algorithmic bytes: read x (4 B), write the hi and lo planes (8 B)
+    LaunchTimer tm(st, "activation_tm", 0.0, 12.0 * (double)rows * T);
+    activation_tm_kernel<<<(unsigned)grid, THREADS, TM_SMEM_BYTES, st>>>(
+        x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb, fu, fd, eps);
+  }
+  count_launch();
+  return check_launch("activation_tm_kernel");
+}
 
 bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream_t st) {
   if (n <= 0) return BV_OK;

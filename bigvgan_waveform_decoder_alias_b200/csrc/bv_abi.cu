@@ -1,6 +1,7 @@
 // The C ABI of libbv: argument checks, the filter design, and the host-side
 // orchestration of the AMP block and the decoder.  Every step of the
 // computation runs in the CUDA kernels of this library.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -23,6 +24,13 @@ uint64_t g_launches = 0;
 }  // namespace
 
 __device__ int g_device_status = 0;
+
+namespace {
+constexpr long long kDefaultWaitLimit = 1ll << 26;
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+}  // namespace
+
+long long wait_limit() { return g_wait_limit.load(std::memory_order_relaxed); }
 
 int *device_status_ptr() {
   void *p = nullptr;
@@ -158,6 +166,10 @@ double bessel_i0(double x) {
 double sinc_pi(double v) { return v == 0.0 ? 1.0 : std::sin(M_PI * v) / (M_PI * v); }
 
 }  // namespace
+
+void clear_error() { g_err[0] = 0; }
+bv_status require_device() { return check_device(); }
+
 }  // namespace bv
 
 using namespace bv;
@@ -201,6 +213,10 @@ int bv_timing_read(bv_kernel_stats *out, int max) {
     ++n;
   }
   return n;
+}
+
+long long bv_debug_set_wait_limit(long long polls) {
+  return g_wait_limit.exchange(polls < 0 ? kDefaultWaitLimit : polls);
 }
 
 bv_status bv_sync_status(void *stream) {
@@ -357,20 +373,37 @@ struct AmpSplit {
   bool tm1[BV_MAX_DIL], tm2[BV_MAX_DIL];
 };
 
-// act -> conv with the activation's output in h1: through the time-major
-// planes when the block's scratch and weights are set up for it.
+// One activation followed by one conv (Cin = C, output length Tout): through
+// the time-major planes xhi / xlo when they and tap-major split weights are
+// given, else through h1 ([B, C, T]) and the conv kernels that read it.
+bv_status act_conv_core(const float *in, int B, int C, int T, const float *la, const float *lb,
+                        const float *fu, const float *fd, float eps, const float *w,
+                        const float *bias, int Cout, int K, int dil, int pad, const float *w_split,
+                        bool tm, const Epi &ep, float *out, int Tout, float *h1, float *xhi,
+                        float *xlo, cudaStream_t st) {
+  if (tm && w_split && xhi) {
+    // the activation writes the conv's time-major operand planes itself
+    if (activation_tm_supported(C)) {
+      BV_TRY(launch_activation_tm(in, xhi, xlo, B, C, T, la, lb, fu, fd, eps, st));
+    } else {
+      BV_TRY(launch_activation(in, h1, B, C, T, la, lb, fu, fd, eps, st));
+      BV_TRY(launch_transpose_split(h1, xhi, xlo, B, C, T, st));
+    }
+    return launch_conv1d_tm(xhi, xlo, B, C, T, w_split, bias, Cout, K, dil, pad, ep, out, Tout,
+                            Tout, st);
+  }
+  BV_TRY(launch_activation(in, h1, B, C, T, la, lb, fu, fd, eps, st));
+  return launch_conv1d(h1, B, C, T, w, bias, Cout, K, dil, pad, ep, out, Tout, Tout, st, w_split);
+}
+
+// act -> conv inside an AMP block (length-preserving pad).
 bv_status act_conv(const float *in, int B, int C, int T, const float *la, const float *lb,
                    const bv_amp_params &p, const float *w, const float *bias, const float *w_split,
                    bool tm, int dil, const Epi &ep, float *out, const AmpScratch &s,
                    cudaStream_t st) {
   const int K = p.kernel_size, pad = (K * dil - dil) / 2;
-  BV_TRY(launch_activation(in, s.h1, B, C, T, la, lb, p.up_filter, p.down_filter, 1e-9f, st));
-  if (tm && w_split && s.xhi) {
-    BV_TRY(launch_transpose_split(s.h1, s.xhi, s.xlo, B, C, T, st));
-    return launch_conv1d_tm(s.xhi, s.xlo, B, C, T, w_split, bias, C, K, dil, pad, ep, out, T, T,
-                            st);
-  }
-  return launch_conv1d(s.h1, B, C, T, w, bias, C, K, dil, pad, ep, out, T, T, st, w_split);
+  return act_conv_core(in, B, C, T, la, lb, p.up_filter, p.down_filter, 1e-9f, w, bias, C, K, dil,
+                       pad, w_split, tm, ep, out, T, s.h1, s.xhi, s.xlo, st);
 }
 
 // y = (accumulate ? y : 0) + scale * AMP(x); x, y and the scratch are disjoint.
@@ -493,6 +526,170 @@ bv_status bv_amp_block(const float *x, int B, int C, int T, const bv_amp_params 
 
 }  // extern "C"
 
+// ------------------------------------ one layer on the decoder's own kernels
+
+namespace bv {
+namespace {
+
+// Workspace of bv_act_conv1d: the activation's [B, C, T] output; when the
+// conv qualifies for the time-major tensor-core path, also two [B, T, C]
+// operand planes and the weights split tap-major into tf32 hi / lo.
+struct ActConvPlan {
+  bool tm = false;
+  size_t h1 = 0, plane = 0, split = 0, total = 0;
+};
+
+ActConvPlan act_conv_plan(int B, int C, int T, int Cout, int K, int dil) {
+  ActConvPlan p;
+  const size_t n = (size_t)B * C * T;
+  p.tm = conv1d_tm_supported(C, Cout, K, dil);
+  p.h1 = align_up(n * sizeof(float));
+  if (p.tm) {
+    p.plane = align_up(n * sizeof(float));
+    p.split = align_up(2 * (size_t)tm_cin_pad(C) * Cout * K * sizeof(float));
+  }
+  p.total = p.h1 + 2 * p.plane + p.split;
+  return p;
+}
+
+// Workspace of bv_conv_transpose1d_ws: the time-major planes and the phase
+// weights of the time-major kernel, or the phase weights of the [B, C, T]
+// tensor-core kernel, or nothing (FP32 kernel).
+struct ConvTPlan {
+  int path = 0;  // 2 time-major, 1 [B, C, T] tensor cores, 0 FP32
+  size_t plane = 0, wp = 0, total = 0;
+};
+
+ConvTPlan convt_plan(int B, int Cin, int T, int Cout, int K, int S) {
+  ConvTPlan p;
+  if (conv_transpose1d_tm_supported(Cin, Cout, K, S)) {
+    p.path = 2;
+    p.plane = align_up((size_t)B * Cin * T * sizeof(float));
+    p.wp = align_up(conv_transpose1d_tm_workspace(Cin, Cout, K, S));
+  } else if (conv_transpose1d_tc_supported(Cin, Cout, K, S)) {
+    p.path = 1;
+    p.wp = align_up(conv_transpose1d_tc_workspace(Cin, Cout, K, S));
+  }
+  p.total = 2 * p.plane + p.wp;
+  return p;
+}
+
+}  // namespace
+}  // namespace bv
+
+extern "C" {
+
+size_t bv_act_conv1d_workspace_size(int B, int C, int T, int Cout, int K, int dilation) {
+  if (B < 1 || C < 1 || T < 1 || Cout < 1 || K < 1 || K > 32 || dilation < 1) return 0;
+  return act_conv_plan(B, C, T, Cout, K, dilation).total;
+}
+
+bv_status bv_act_conv1d(const float *x, int B, int C, int T, const float *log_alpha,
+                        const float *log_beta, const float *up_filter, const float *down_filter,
+                        float eps, const float *w, const float *bias, int Cout, int K,
+                        int dilation, int pad, const bv_epilogue *ep, float *y, void *workspace,
+                        size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  if (!x || !y || !w || !log_alpha || !log_beta || !up_filter || !down_filter)
+    return fail(BV_ERR_ARG, "bv_act_conv1d: null pointer");
+  if (B < 1 || C < 1 || T < 1 || Cout < 1 || K < 1 || K > 32 || dilation < 1 || pad < 0)
+    return fail(BV_ERR_SHAPE, "bv_act_conv1d: B=%d C=%d T=%d Cout=%d K=%d d=%d pad=%d", B, C, T,
+                Cout, K, dilation, pad);
+  const long long Tout = (long long)T + 2LL * pad - (long long)dilation * (K - 1);
+  if (Tout < 1 || Tout > 0x7fffffffLL)
+    return fail(BV_ERR_SHAPE, "bv_act_conv1d: output length %lld", Tout);
+  const size_t nin = (size_t)B * C * T, nout = (size_t)B * Cout * Tout;
+  if (nin >= (1ull << 40)) return fail(BV_ERR_SHAPE, "bv_act_conv1d: tensor too large");
+  Epi e{nullptr, 1.0f, 0, 0};
+  if (ep) {
+    e = Epi{ep->residual, ep->scale, ep->accumulate ? 1 : 0, ep->final_act};
+    if (e.final_act < 0 || e.final_act > 2)
+      return fail(BV_ERR_ARG, "bv_act_conv1d: final_act %d", e.final_act);
+  }
+  const ActConvPlan plan = act_conv_plan(B, C, T, Cout, K, dilation);
+  if (!workspace || ws_bytes < plan.total)
+    return fail(BV_ERR_WORKSPACE, "bv_act_conv1d: workspace %zu bytes, need %zu", ws_bytes,
+                plan.total);
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_act_conv1d: workspace not 256-byte aligned");
+  if (!aligned4(x) || !aligned4(y)) return fail(BV_ERR_ARG, "bv_act_conv1d: misaligned pointer");
+  const float *wsf = static_cast<const float *>(workspace);
+  const size_t nws = plan.total / sizeof(float);
+  if (overlaps(x, nin, y, nout) || overlaps(x, nin, wsf, nws) || overlaps(y, nout, wsf, nws))
+    return fail(BV_ERR_ARG, "bv_act_conv1d: x, y and workspace must be disjoint");
+  if (e.residual && ((e.residual != y && overlaps(e.residual, nout, y, nout)) ||
+                     overlaps(e.residual, nout, wsf, nws)))
+    return fail(BV_ERR_ARG, "bv_act_conv1d: residual partially overlaps y or the workspace");
+  BV_TRY(check_device());
+  cudaStream_t st = as_stream(stream);
+  char *w8 = static_cast<char *>(workspace);
+  float *h1 = reinterpret_cast<float *>(w8);
+  float *xhi = nullptr, *xlo = nullptr, *split = nullptr;
+  if (plan.tm) {
+    xhi = reinterpret_cast<float *>(w8 + plan.h1);
+    xlo = reinterpret_cast<float *>(w8 + plan.h1 + plan.plane);
+    split = reinterpret_cast<float *>(w8 + plan.h1 + 2 * plan.plane);
+    SplitTable tab;
+    tab.n = 1;
+    tab.src[0] = w;
+    tab.dst[0] = split;
+    tab.count[0] = (long long)Cout * C * K;
+    tab.cin[0] = C;
+    tab.k[0] = K;
+    BV_TRY(launch_split_weights(tab, st));
+  }
+  return act_conv_core(x, B, C, T, log_alpha, log_beta, up_filter, down_filter, eps, w, bias,
+                       Cout, K, dilation, pad, split, plan.tm, e, y, (int)Tout, h1, xhi, xlo, st);
+}
+
+size_t bv_conv_transpose1d_workspace_size(int B, int Cin, int T, int Cout, int K, int stride) {
+  if (B < 1 || Cin < 1 || T < 1 || Cout < 1 || K < 1 || K > 64 || stride < 1 || stride > 16)
+    return 0;
+  return convt_plan(B, Cin, T, Cout, K, stride).total;
+}
+
+bv_status bv_conv_transpose1d_ws(const float *x, int B, int Cin, int T, const float *w,
+                                 const float *bias, int Cout, int K, int stride, int pad,
+                                 float *y, void *workspace, size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  if (!x || !w || !y) return fail(BV_ERR_ARG, "bv_conv_transpose1d_ws: null pointer");
+  if (B < 1 || Cin < 1 || T < 1 || Cout < 1 || K < 1 || K > 64 || stride < 1 || stride > 16 ||
+      pad < 0)
+    return fail(BV_ERR_SHAPE, "bv_conv_transpose1d_ws: B=%d Cin=%d T=%d Cout=%d K=%d s=%d pad=%d",
+                B, Cin, T, Cout, K, stride, pad);
+  const long long Tout = (long long)(T - 1) * stride + K - 2LL * pad;
+  if (Tout < 1 || Tout > 0x7fffffffLL)
+    return fail(BV_ERR_SHAPE, "bv_conv_transpose1d_ws: output length %lld", Tout);
+  const size_t nin = (size_t)B * Cin * T, nout = (size_t)B * Cout * Tout;
+  const ConvTPlan plan = convt_plan(B, Cin, T, Cout, K, stride);
+  if (plan.total > 0 && (!workspace || ws_bytes < plan.total))
+    return fail(BV_ERR_WORKSPACE, "bv_conv_transpose1d_ws: workspace %zu bytes, need %zu",
+                ws_bytes, plan.total);
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_conv_transpose1d_ws: workspace not 256-byte aligned");
+  const float *wsf = static_cast<const float *>(workspace);
+  const size_t nws = plan.total / sizeof(float);
+  if (overlaps(x, nin, y, nout) || (nws && (overlaps(x, nin, wsf, nws) || overlaps(y, nout, wsf, nws))))
+    return fail(BV_ERR_ARG, "bv_conv_transpose1d_ws: x, y and workspace must be disjoint");
+  BV_TRY(check_device());
+  cudaStream_t st = as_stream(stream);
+  char *w8 = static_cast<char *>(workspace);
+  if (plan.path == 2) {
+    float *xhi = reinterpret_cast<float *>(w8);
+    float *xlo = reinterpret_cast<float *>(w8 + plan.plane);
+    float *wp = reinterpret_cast<float *>(w8 + 2 * plan.plane);
+    BV_TRY(launch_transpose_split(x, xhi, xlo, B, Cin, T, st));
+    return launch_conv_transpose1d_tm(xhi, xlo, B, Cin, T, w, bias, Cout, K, stride, pad, y, wp,
+                                      st);
+  }
+  if (plan.path == 1)
+    return launch_conv_transpose1d_tc(x, B, Cin, T, w, bias, Cout, K, stride, pad, y,
+                                      reinterpret_cast<float *>(w8), st);
+  return launch_conv_transpose1d(x, B, Cin, T, w, bias, Cout, K, stride, pad, y, st);
+}
+
+}  // extern "C"
+
 // --------------------------------------------------------------- decoder
 
 namespace bv {
@@ -525,7 +722,20 @@ bv_status check_config(const bv_decoder_config *c) {
   if (c->tile_frames < 0 || c->overlap_frames < 0 ||
       (c->tile_frames > 0 && c->overlap_frames >= c->tile_frames))
     return fail(BV_ERR_SHAPE, "decoder: tile %d overlap %d", c->tile_frames, c->overlap_frames);
+  if (c->latent_channels < 0)
+    return fail(BV_ERR_SHAPE, "decoder: latent_channels %d", c->latent_channels);
   return BV_OK;
+}
+
+// Channels of the z a decode call takes: normalised latents with the front
+// end, else the decoder's input.
+int z_channels(const bv_decoder_config *c) {
+  return c->latent_channels > 0 ? c->latent_channels : c->in_channels;
+}
+
+// The front end's output [B, in_channels, F] (nothing without a front end).
+size_t front_ws(const bv_decoder_config *c, long long B, long long F) {
+  return c->latent_channels > 0 ? align_up((size_t)B * c->in_channels * F * sizeof(float)) : 0;
 }
 
 long long hop_of(const bv_decoder_config *c) {
@@ -609,8 +819,10 @@ size_t split_ws(const bv_decoder_config *c) {
 }
 
 // Fill `out` with slots in ws (size split_ws) and launch the split kernels.
+// With launch false only the slots are filled in (the weights were split into
+// ws earlier, by bv_decoder_prepare).
 bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w, char *ws,
-                        DecoderSplit *out, cudaStream_t st) {
+                        DecoderSplit *out, cudaStream_t st, bool launch = true) {
   SplitTable tab;
   tab.n = 0;
   bv_status status = BV_OK;
@@ -640,11 +852,11 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
     tab.cin[tab.n] = tm ? Cin : 0;
     tab.k[tab.n] = K;
     if (++tab.n == kMaxSplit) {
-      status = launch_split_weights(tab, st);
+      if (launch) status = launch_split_weights(tab, st);
       tab.n = 0;
     }
   });
-  if (status != BV_OK) return status;
+  if (status != BV_OK || !launch) return status;
   return launch_split_weights(tab, st);
 }
 
@@ -655,16 +867,24 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
 // time-major planes); for blocks 1.. their own outputs, summed into A.
 int core_planes(const bv_decoder_config *c) { return 2 + 5 * c->n_blocks + (c->n_blocks - 1); }
 
-size_t core_ws(const bv_decoder_config *c, long long B, long long F) {
-  return core_planes(c) * align_up((size_t)max_elems(c, B, F) * sizeof(float)) + convt_ws(c);
+// prepared: the transposed convs' phase weights come packed with the
+// prepared weights, so no repack buffer
+size_t core_ws(const bv_decoder_config *c, long long B, long long F, bool prepared = false) {
+  return core_planes(c) * align_up((size_t)max_elems(c, B, F) * sizeof(float)) +
+         (prepared ? 0 : convt_ws(c));
 }
 
 // Streams on which the AMP blocks of a stage run side by side (one per block),
 // created once per device and kept until exit, with the events that fork them
-// from and join them back to the caller's stream.
+// from and join them back to the caller's stream.  `mu` is held from the fork
+// record to the last join wait of a stage, so calls from several host threads
+// on one device enqueue their fork/join sequences one at a time: a stream wait
+// takes the event's state at the time of the wait call, so no call can wait on
+// another call's fork point.  (Their work still shares these streams.)
 struct AuxStreams {
   cudaStream_t s[BV_MAX_BLOCKS];
   cudaEvent_t fork, join[BV_MAX_BLOCKS];
+  std::mutex mu;
   bool ok = false;
 };
 
@@ -717,26 +937,124 @@ TilePlan plan_tiles(const bv_decoder_config *c, int F) {
   return p;
 }
 
-size_t decode_ws(const bv_decoder_config *c, int B, int F) {
+// The decode as units: unit u = k B + b is tile k of side b (an untiled
+// decode is one tile of all `frames`).  Full tiles come first; a shorter last
+// tile, if any, is tile n_tiles - 1.
+struct UnitGeom {
+  int n_tiles = 1, tile_len = 0, step = 0, n_full = 1, last_len = 0;
+  long long pitch = 0;  // samples per unit row: tile_len * hop
+};
+
+UnitGeom unit_geom(const bv_decoder_config *c, int F) {
   const TilePlan tp = plan_tiles(c, F);
-  const long long hop = hop_of(c);
-  if (!tp.tiled) return split_ws(c) + core_ws(c, B, F);
-  size_t s = split_ws(c);
-  const long long rows_full = (long long)B * tp.n_full;
-  s += align_up((size_t)rows_full * c->in_channels * c->tile_frames * sizeof(float));
-  s += align_up((size_t)rows_full * c->out_channels * c->tile_frames * hop * sizeof(float));
-  size_t core = core_ws(c, rows_full, c->tile_frames);
-  if (tp.last_len > 0) {
-    s += align_up((size_t)B * c->in_channels * tp.last_len * sizeof(float));
-    s += align_up((size_t)B * c->out_channels * tp.last_len * hop * sizeof(float));
-    const size_t c2 = core_ws(c, B, tp.last_len);
-    if (c2 > core) core = c2;
+  UnitGeom g;
+  if (tp.tiled) {
+    g.n_tiles = tp.n_tiles;
+    g.tile_len = c->tile_frames;
+    g.step = tp.step;
+    g.n_full = tp.n_full;
+    g.last_len = tp.last_len;
+  } else {
+    g.tile_len = g.step = F;
   }
+  g.pitch = (long long)g.tile_len * hop_of(c);
+  return g;
+}
+
+// Units [u0, u1) split into full-tile units and last-tile units.
+struct UnitRange {
+  long long full_u0 = 0, full_n = 0, last_u0 = 0, last_n = 0;
+};
+
+UnitRange unit_range(const UnitGeom &g, int B, long long u0, long long u1) {
+  UnitRange r;
+  const long long full_units = (long long)g.n_full * B;
+  r.full_u0 = u0;
+  r.full_n = std::max(0LL, std::min(u1, full_units) - u0);
+  r.last_u0 = std::max(u0, full_units);
+  r.last_n = g.last_len > 0 ? std::max(0LL, u1 - r.last_u0) : 0;
+  return r;
+}
+
+// Workspace of decoding a unit range (split weights excluded): the gathered
+// latents of both kinds of unit, and the core buffers of the larger decode.
+size_t units_ws(const bv_decoder_config *c, const UnitGeom &g, const UnitRange &r,
+                bool prepared = false) {
+  size_t s = align_up((size_t)r.full_n * c->in_channels * g.tile_len * sizeof(float)) +
+             align_up((size_t)r.last_n * c->in_channels * g.last_len * sizeof(float));
+  size_t core = r.full_n > 0 ? core_ws(c, r.full_n, g.tile_len, prepared) : 0;
+  if (r.last_n > 0) core = std::max(core, core_ws(c, r.last_n, g.last_len, prepared));
   return s + core;
+}
+
+size_t unit_rows_bytes(const bv_decoder_config *c, const UnitGeom &g, long long n_units) {
+  return align_up((size_t)n_units * c->out_channels * g.pitch * sizeof(float));
+}
+
+// Workspace of a decode; with prepared weights (bv_decoder_prepare) neither
+// the split weights nor the ConvT repack buffer live in it.
+size_t decode_ws(const bv_decoder_config *c, int B, int F, bool prepared = false) {
+  const UnitGeom g = unit_geom(c, F);
+  const size_t sw = prepared ? 0 : split_ws(c);
+  if (g.n_tiles == 1) return sw + front_ws(c, B, F) + core_ws(c, B, F, prepared);
+  const long long n_units = (long long)g.n_tiles * B;
+  return sw + front_ws(c, B, F) + unit_rows_bytes(c, g, n_units) +
+         units_ws(c, g, unit_range(g, B, 0, n_units), prepared);
+}
+
+// The prepared weights: the split weights (split_ws bytes, split_weights'
+// layout), then the packed phase weights of every ConvT stage that runs on a
+// tensor-core kernel.
+size_t prepared_convt_bytes(const bv_decoder_config *c, int i, int Cin) {
+  const int Co = c->up_channels[i], k = c->up_kernel[i], sr = c->up_rate[i];
+  if (conv_transpose1d_tm_supported(Cin, Co, k, sr))
+    return align_up(conv_transpose1d_tm_workspace(Cin, Co, k, sr));
+  if (conv_transpose1d_tc_supported(Cin, Co, k, sr))
+    return align_up(conv_transpose1d_tc_workspace(Cin, Co, k, sr));
+  return 0;
+}
+
+size_t prepared_ws(const bv_decoder_config *c) {
+  size_t s = split_ws(c);
+  int C = c->pre_channels;
+  for (int i = 0; i < c->n_up; ++i) {
+    s += prepared_convt_bytes(c, i, C);
+    C = c->up_channels[i];
+  }
+  return s;
+}
+
+// Slots of the ConvT stages' packed weights in a prepared buffer (nullptr:
+// the stage packs nothing).
+void prepared_convt_slots(const bv_decoder_config *c, const char *base,
+                          const float *out[BV_MAX_UP]) {
+  size_t off = split_ws(c);
+  int C = c->pre_channels;
+  for (int i = 0; i < c->n_up; ++i) {
+    const size_t b = prepared_convt_bytes(c, i, C);
+    out[i] = b ? reinterpret_cast<const float *>(base + off) : nullptr;
+    off += b;
+    C = c->up_channels[i];
+  }
+}
+
+// With the latent front end, z [latent_ch, B, F] -> the decoder's input in
+// the workspace (advanced past it); otherwise z itself.
+bv_status run_front_end(const bv_decoder_config *c, const bv_decoder_weights *w, const float *&z,
+                        int B, int F, char *&ws, cudaStream_t st) {
+  if (c->latent_channels <= 0) return BV_OK;
+  float *zin = reinterpret_cast<float *>(ws);
+  ws += front_ws(c, B, F);
+  BV_TRY(launch_latent_front_end(z, c->latent_channels, B, F, w->latents_mean, w->latents_std,
+                                 w->dec_in_w, w->dec_in_b, c->in_channels, zin, st));
+  z = zin;
+  return BV_OK;
 }
 
 bv_status check_weights(const bv_decoder_config *c, const bv_decoder_weights *w) {
   if (!w) return fail(BV_ERR_ARG, "decoder: null weights");
+  if (c->latent_channels > 0 && (!w->latents_mean || !w->latents_std || !w->dec_in_w))
+    return fail(BV_ERR_ARG, "decoder: null latents_mean / latents_std / dec_in_w");
   if (!w->pre_w || !w->post_w || !w->post_log_alpha || !w->post_log_beta || !w->up_filter ||
       !w->down_filter)
     return fail(BV_ERR_ARG, "decoder: null conv_pre / act_post / conv_post weight or filter");
@@ -755,10 +1073,19 @@ bv_status check_weights(const bv_decoder_config *c, const bv_decoder_weights *w)
   return BV_OK;
 }
 
-// One untiled decode of B rows into y rows of length F*hop.
+// One untiled decode of B rows into y rows of length F*hop, row pitch
+// y_pitch samples.
+// Weights prepared for a decode: split tensor-core weights and, per ConvT
+// stage, its packed phase weights (nullptr: packed into the workspace).
+struct DecoderPrep {
+  DecoderSplit sw;
+  const float *convt[BV_MAX_UP] = {};
+};
+
 bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
-                      const DecoderSplit &sw, const float *z, int B, int F, float *y, char *ws,
-                      cudaStream_t st) {
+                      const DecoderPrep &pp, const float *z, int B, int F, float *y,
+                      long long y_pitch, char *ws, cudaStream_t st) {
+  const DecoderSplit &sw = pp.sw;
   const size_t sz = align_up((size_t)max_elems(c, B, F) * sizeof(float));
   auto plane = [&](int k) { return reinterpret_cast<float *>(ws + (size_t)k * sz); };
   float *A = plane(0);
@@ -774,10 +1101,12 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
   const AmpScratch &s = sb[0];
   float *WP = plane(core_planes(c));  // repacked ConvT weights
   // The blocks of a stage are independent until their mean: they run side by
-  // side on one stream each and their outputs are summed in block order
-  // (bit-identical to accumulating them one after the other).  With the
-  // library's per-kernel timers on they run in order on the caller's stream,
-  // so that every launch's event time is its own.
+  // side on one stream each and their outputs are summed in block order.
+  // With the library's per-kernel timers on they run in order on the
+  // caller's stream, so that every launch's event time is its own, and
+  // accumulate through the epilogue (the same sums in the same order, but the
+  // epilogue fuses scale and add into one multiply-add, so the two paths can
+  // differ in the last bit).
   AuxStreams *aux = (nb > 1 && !g_timing_on.load(std::memory_order_relaxed)) ? aux_streams()
                                                                               : nullptr;
   int C = c->pre_channels, n = F;
@@ -791,17 +1120,26 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
     if (conv_transpose1d_tm_supported(C, Co, k, sr)) {
       // time-major: the stage input goes to block 0's operand planes first
       BV_TRY(launch_transpose_split(A, s.xhi, s.xlo, B, C, n, st));
-      BV_TRY(launch_conv_transpose1d_tm(s.xhi, s.xlo, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr,
-                                        pad, S, WP, st));
-    } else if (conv_transpose1d_tc_supported(C, Co, k, sr))
-      BV_TRY(launch_conv_transpose1d_tc(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S,
-                                        WP, st));
-    else
+      if (pp.convt[i])
+        BV_TRY(launch_conv_transpose1d_tm_packed(s.xhi, s.xlo, B, C, n, pp.convt[i], w->up_b[i],
+                                                 Co, k, sr, pad, S, st));
+      else
+        BV_TRY(launch_conv_transpose1d_tm(s.xhi, s.xlo, B, C, n, w->up_w[i], w->up_b[i], Co, k,
+                                          sr, pad, S, WP, st));
+    } else if (conv_transpose1d_tc_supported(C, Co, k, sr)) {
+      if (pp.convt[i])
+        BV_TRY(launch_conv_transpose1d_tc_packed(A, B, C, n, pp.convt[i], w->up_b[i], Co, k, sr,
+                                                 pad, S, st));
+      else
+        BV_TRY(launch_conv_transpose1d_tc(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S,
+                                          WP, st));
+    } else
       BV_TRY(launch_conv_transpose1d(A, B, C, n, w->up_w[i], w->up_b[i], Co, k, sr, pad, S, st));
     C = Co;
     n = n2;
     const float scale = 1.0f / (float)nb;
     if (aux) {
+      std::lock_guard<std::mutex> enqueue(aux->mu);
       CUDA_TRY(cudaEventRecord(aux->fork, st));
       for (int j = 0; j < nb; ++j) CUDA_TRY(cudaStreamWaitEvent(aux->s[j], aux->fork, 0));
       for (int j = 0; j < nb; ++j)
@@ -824,56 +1162,106 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
   const long long L = (long long)F * hop_of(c);
   Epi fin{nullptr, 1.0f, 0, c->final_act};
   return launch_conv1d(s.h1, B, C, n, w->post_w, w->post_b, c->out_channels, c->post_kernel, 1,
-                       (c->post_kernel - 1) / 2, fin, y, (int)L, (int)L, st, sw.post);
+                       (c->post_kernel - 1) / 2, fin, y, (int)L, (int)y_pitch, st, sw.post);
+}
+
+// Decode units [r.full_u0, ...) into rows of y_units (unit u at row u - u0,
+// out_channels x g.pitch samples each; a last-tile row holds last_len * hop).
+bv_status decode_units_impl(const bv_decoder_config *c, const bv_decoder_weights *w,
+                            const DecoderPrep &sw, const float *z, int B, int F,
+                            const UnitGeom &g, const UnitRange &r, float *y_units, char *ws,
+                            cudaStream_t st) {
+  char *p = ws;
+  float *zf = reinterpret_cast<float *>(p);
+  p += align_up((size_t)r.full_n * c->in_channels * g.tile_len * sizeof(float));
+  float *zl = reinterpret_cast<float *>(p);
+  p += align_up((size_t)r.last_n * c->in_channels * g.last_len * sizeof(float));
+  if (r.full_n > 0) {
+    BV_TRY(launch_gather_tiles(z, zf, B, c->in_channels, F, g.step, g.tile_len, r.full_u0,
+                               r.full_n, st));
+    BV_TRY(decode_core(c, w, sw, zf, (int)r.full_n, g.tile_len, y_units, g.pitch, p, st));
+  }
+  if (r.last_n > 0) {
+    BV_TRY(launch_gather_tiles(z, zl, B, c->in_channels, F, g.step, g.last_len, r.last_u0,
+                               r.last_n, st));
+    float *yl = y_units + (size_t)r.full_n * c->out_channels * g.pitch;
+    BV_TRY(decode_core(c, w, sw, zl, (int)r.last_n, g.last_len, yl, g.pitch, p, st));
+  }
+  return BV_OK;
+}
+
+// The weights a decode reads: from the prepared buffer when the weights carry
+// one, else split into the workspace now (advanced past them).
+bv_status prepare_for_decode(const bv_decoder_config *c, const bv_decoder_weights *w, char *&ws,
+                             DecoderPrep *pp, cudaStream_t st) {
+  if (w->prepared) {
+    char *base = const_cast<char *>(static_cast<const char *>(w->prepared));
+    BV_TRY(split_weights(c, w, base, &pp->sw, st, false));
+    prepared_convt_slots(c, base, pp->convt);
+    return BV_OK;
+  }
+  BV_TRY(split_weights(c, w, ws, &pp->sw, st));
+  ws += split_ws(c);
+  return BV_OK;
+}
+
+// y[b, o, t] = mean over the tiles covering t of their unit rows (all
+// n_tiles B units in y_units, in unit order).
+bv_status stitch_units(const bv_decoder_config *c, const UnitGeom &g, int B, int F,
+                       const float *y_units, float *y, cudaStream_t st) {
+  const long long hop = hop_of(c);
+  TileGroups tg{};
+  tg.n = 0;
+  if (g.n_full > 0) {
+    tg.data[tg.n] = y_units;
+    tg.k0[tg.n] = 0;
+    tg.count[tg.n] = g.n_full;
+    tg.len_samples[tg.n] = (long long)g.tile_len * hop;
+    tg.pitch[tg.n] = g.pitch;
+    ++tg.n;
+  }
+  if (g.last_len > 0) {
+    tg.data[tg.n] = y_units + (size_t)g.n_full * B * c->out_channels * g.pitch;
+    tg.k0[tg.n] = g.n_full;
+    tg.count[tg.n] = 1;
+    tg.len_samples[tg.n] = (long long)g.last_len * hop;
+    tg.pitch[tg.n] = g.pitch;
+    ++tg.n;
+  }
+  tg.max_len_samples = (long long)g.tile_len * hop;
+  return launch_stitch_tiles(tg, y, B, c->out_channels, (long long)F * hop, (int)(g.step * hop),
+                             st);
 }
 
 bv_status decode_impl(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
                       int B, int F, float *y, char *ws, cudaStream_t st) {
-  const TilePlan tp = plan_tiles(c, F);
-  DecoderSplit sw;
-  BV_TRY(split_weights(c, w, ws, &sw, st));
-  ws += split_ws(c);
-  if (!tp.tiled) return decode_core(c, w, sw, z, B, F, y, ws, st);
-  const long long hop = hop_of(c);
-  const int Ft = c->tile_frames;
-  const long long rows_full = (long long)B * tp.n_full;
-  char *p = ws;
-  float *zf = reinterpret_cast<float *>(p);
-  p += align_up((size_t)rows_full * c->in_channels * Ft * sizeof(float));
-  float *yf = reinterpret_cast<float *>(p);
-  p += align_up((size_t)rows_full * c->out_channels * Ft * hop * sizeof(float));
-  float *zl = nullptr, *yl = nullptr;
-  if (tp.last_len > 0) {
-    zl = reinterpret_cast<float *>(p);
-    p += align_up((size_t)B * c->in_channels * tp.last_len * sizeof(float));
-    yl = reinterpret_cast<float *>(p);
-    p += align_up((size_t)B * c->out_channels * tp.last_len * hop * sizeof(float));
-  }
-  TileGroups g{};
-  g.n = 0;
-  if (tp.n_full > 0) {
-    BV_TRY(launch_gather_tiles(z, zf, B, c->in_channels, F, tp.step, Ft, 0, tp.n_full, st));
-    BV_TRY(decode_core(c, w, sw, zf, (int)rows_full, Ft, yf, p, st));
-    g.data[g.n] = yf;
-    g.k0[g.n] = 0;
-    g.count[g.n] = tp.n_full;
-    g.len_samples[g.n] = Ft * hop;
-    ++g.n;
-  }
-  if (tp.last_len > 0) {
-    BV_TRY(launch_gather_tiles(z, zl, B, c->in_channels, F, tp.step, tp.last_len, tp.n_full, 1, st));
-    BV_TRY(decode_core(c, w, sw, zl, B, tp.last_len, yl, p, st));
-    g.data[g.n] = yl;
-    g.k0[g.n] = tp.n_full;
-    g.count[g.n] = 1;
-    g.len_samples[g.n] = tp.last_len * hop;
-    ++g.n;
-  }
-  g.max_len_samples = Ft * hop;
-  return launch_stitch_tiles(g, y, B, c->out_channels, (long long)F * hop, (int)(tp.step * hop), st);
+  const UnitGeom g = unit_geom(c, F);
+  DecoderPrep sw;
+  BV_TRY(prepare_for_decode(c, w, ws, &sw, st));
+  BV_TRY(run_front_end(c, w, z, B, F, ws, st));
+  if (g.n_tiles == 1) return decode_core(c, w, sw, z, B, F, y, (long long)F * hop_of(c), ws, st);
+  // every tile of every side, then the overlap average
+  const long long n_units = (long long)g.n_tiles * B;
+  float *yu = reinterpret_cast<float *>(ws);
+  ws += unit_rows_bytes(c, g, n_units);
+  BV_TRY(decode_units_impl(c, w, sw, z, B, F, g, unit_range(g, B, 0, n_units), yu, ws, st));
+  return stitch_units(c, g, B, F, yu, y, st);
 }
 
 }  // namespace
+
+// The decoder for other parts of the library (the bandwidth-extension tail).
+bv_status decoder_check(const bv_decoder_config *c, const bv_decoder_weights *w) {
+  BV_TRY(check_config(c));
+  return check_weights(c, w);
+}
+size_t decoder_workspace(const bv_decoder_config *c, int B, int F) { return decode_ws(c, B, F); }
+bv_status decoder_run(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                      int B, int F, float *y, char *ws, cudaStream_t st) {
+  return decode_impl(c, w, z, B, F, y, ws, st);
+}
+long long decoder_hop(const bv_decoder_config *c) { return hop_of(c); }
+
 }  // namespace bv
 
 extern "C" {
@@ -970,12 +1358,12 @@ bv_status bv_decode(const bv_decoder_config *c, const bv_decoder_weights *w, con
   if (L > 0x7fffffffLL || max_elems(c, B, frames) > (1LL << 40))
     return fail(BV_ERR_SHAPE, "bv_decode: request too large");
   BV_TRY(check_weights(c, w));
-  const size_t need = decode_ws(c, B, frames);
+  const size_t need = decode_ws(c, B, frames, w->prepared != nullptr);
   if (!workspace || ws_bytes < need)
     return fail(BV_ERR_WORKSPACE, "bv_decode: workspace %zu bytes, need %zu", ws_bytes, need);
   if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
     return fail(BV_ERR_ARG, "bv_decode: workspace not 256-byte aligned");
-  const size_t nz = (size_t)B * c->in_channels * frames, ny = (size_t)B * c->out_channels * L;
+  const size_t nz = (size_t)B * z_channels(c) * frames, ny = (size_t)B * c->out_channels * L;
   const float *wsf = static_cast<const float *>(workspace);
   if (overlaps(z, nz, y, ny) || overlaps(z, nz, wsf, need / 4) || overlaps(y, ny, wsf, need / 4))
     return fail(BV_ERR_ARG, "bv_decode: z, y and workspace must be disjoint");
@@ -983,11 +1371,153 @@ bv_status bv_decode(const bv_decoder_config *c, const bv_decoder_weights *w, con
   return decode_impl(c, w, z, B, frames, y, static_cast<char *>(workspace), as_stream(stream));
 }
 
+bv_status bv_latent_front_end(const float *z, int C, int S, int T, const float *mean,
+                              const float *std_, const float *w, const float *bias, int Cout,
+                              float *out, void *stream) {
+  g_err[0] = 0;
+  if (!z || !mean || !std_ || !w || !out) return fail(BV_ERR_ARG, "bv_latent_front_end: null pointer");
+  if (C < 1 || S < 1 || T < 1 || Cout < 1)
+    return fail(BV_ERR_SHAPE, "bv_latent_front_end: C=%d S=%d T=%d Cout=%d", C, S, T, Cout);
+  if (overlaps(z, (size_t)C * S * T, out, (size_t)S * Cout * T))
+    return fail(BV_ERR_ARG, "bv_latent_front_end: z and out overlap");
+  BV_TRY(check_device());
+  return launch_latent_front_end(z, C, S, T, mean, std_, w, bias, Cout, out, as_stream(stream));
+}
+
+size_t bv_decoder_prepared_size(const bv_decoder_config *c) {
+  clear_error();
+  if (check_config(c) != BV_OK) return 0;
+  return std::max<size_t>(prepared_ws(c), kAlign);
+}
+
+bv_status bv_decoder_prepare(const bv_decoder_config *c, const bv_decoder_weights *w,
+                             void *prepared, size_t bytes, void *stream) {
+  clear_error();
+  BV_TRY(check_config(c));
+  BV_TRY(check_weights(c, w));
+  const size_t need = std::max<size_t>(prepared_ws(c), kAlign);
+  if (!prepared || bytes < need)
+    return fail(BV_ERR_WORKSPACE, "bv_decoder_prepare: %zu bytes, need %zu", bytes, need);
+  if ((reinterpret_cast<uintptr_t>(prepared) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_decoder_prepare: buffer not 256-byte aligned");
+  BV_TRY(check_device());
+  cudaStream_t st = as_stream(stream);
+  char *base = static_cast<char *>(prepared);
+  DecoderSplit sw;
+  BV_TRY(split_weights(c, w, base, &sw, st));
+  const float *slots[BV_MAX_UP] = {};
+  prepared_convt_slots(c, base, slots);
+  int C = c->pre_channels;
+  for (int i = 0; i < c->n_up; ++i) {
+    const int Co = c->up_channels[i], k = c->up_kernel[i], sr = c->up_rate[i];
+    float *wp = const_cast<float *>(slots[i]);
+    if (wp && conv_transpose1d_tm_supported(C, Co, k, sr))
+      BV_TRY(launch_convt_pack_tm(w->up_w[i], C, Co, k, sr, wp, st));
+    else if (wp)
+      BV_TRY(launch_convt_pack_tc(w->up_w[i], C, Co, k, sr, wp, st));
+    C = Co;
+  }
+  return BV_OK;
+}
+
+size_t bv_decode_workspace_size_prepared(const bv_decoder_config *c, int B, int frames) {
+  clear_error();
+  if (check_config(c) != BV_OK) return 0;
+  if (B < 1 || frames < 1) {
+    fail(BV_ERR_SHAPE, "bv_decode_workspace_size_prepared: B=%d frames=%d", B, frames);
+    return 0;
+  }
+  return decode_ws(c, B, frames, true);
+}
+
+int bv_decoder_tile_count(const bv_decoder_config *c, int frames) {
+  if (check_config(c) != BV_OK || frames < 1) return -1;
+  return unit_geom(c, frames).n_tiles;
+}
+
+int64_t bv_decoder_unit_length(const bv_decoder_config *c, int frames) {
+  if (check_config(c) != BV_OK || frames < 1) return -1;
+  return unit_geom(c, frames).pitch;
+}
+
+size_t bv_decode_units_workspace_size(const bv_decoder_config *c, int B, int frames,
+                                      int64_t unit_begin, int64_t unit_end) {
+  g_err[0] = 0;
+  if (check_config(c) != BV_OK) return 0;
+  if (B < 1 || frames < 1) {
+    fail(BV_ERR_SHAPE, "bv_decode_units_workspace_size: B=%d frames=%d", B, frames);
+    return 0;
+  }
+  const UnitGeom g = unit_geom(c, frames);
+  const long long n_units = (long long)g.n_tiles * B;
+  if (unit_begin < 0 || unit_end > n_units || unit_begin >= unit_end) {
+    fail(BV_ERR_SHAPE, "bv_decode_units_workspace_size: units [%lld, %lld) of %lld",
+         (long long)unit_begin, (long long)unit_end, n_units);
+    return 0;
+  }
+  return split_ws(c) + front_ws(c, B, frames) +
+         units_ws(c, g, unit_range(g, B, unit_begin, unit_end));
+}
+
+bv_status bv_decode_units(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                          int B, int frames, int64_t unit_begin, int64_t unit_end,
+                          float *y_units, void *workspace, size_t ws_bytes, void *stream) {
+  g_err[0] = 0;
+  BV_TRY(check_config(c));
+  if (!z || !y_units) return fail(BV_ERR_ARG, "bv_decode_units: null z or y_units");
+  if (B < 1 || frames < 1) return fail(BV_ERR_SHAPE, "bv_decode_units: B=%d frames=%d", B, frames);
+  if ((long long)frames * hop_of(c) > 0x7fffffffLL || max_elems(c, B, frames) > (1LL << 40))
+    return fail(BV_ERR_SHAPE, "bv_decode_units: request too large");
+  const UnitGeom g = unit_geom(c, frames);
+  const long long n_units = (long long)g.n_tiles * B;
+  if (unit_begin < 0 || unit_end > n_units || unit_begin >= unit_end)
+    return fail(BV_ERR_SHAPE, "bv_decode_units: units [%lld, %lld) of %lld", (long long)unit_begin,
+                (long long)unit_end, n_units);
+  BV_TRY(check_weights(c, w));
+  const UnitRange r = unit_range(g, B, unit_begin, unit_end);
+  const bool prepared = w->prepared != nullptr;
+  const size_t need = (prepared ? 0 : split_ws(c)) + front_ws(c, B, frames) +
+                      units_ws(c, g, r, prepared);
+  if (!workspace || ws_bytes < need)
+    return fail(BV_ERR_WORKSPACE, "bv_decode_units: workspace %zu bytes, need %zu", ws_bytes, need);
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return fail(BV_ERR_ARG, "bv_decode_units: workspace not 256-byte aligned");
+  const size_t nz = (size_t)B * z_channels(c) * frames;
+  const size_t ny = (size_t)(unit_end - unit_begin) * c->out_channels * g.pitch;
+  const float *wsf = static_cast<const float *>(workspace);
+  if (overlaps(z, nz, y_units, ny) || overlaps(z, nz, wsf, need / 4) ||
+      overlaps(y_units, ny, wsf, need / 4))
+    return fail(BV_ERR_ARG, "bv_decode_units: z, y_units and workspace must be disjoint");
+  BV_TRY(check_device());
+  cudaStream_t st = as_stream(stream);
+  char *ws = static_cast<char *>(workspace);
+  DecoderPrep sw;
+  BV_TRY(prepare_for_decode(c, w, ws, &sw, st));
+  BV_TRY(run_front_end(c, w, z, B, frames, ws, st));
+  return decode_units_impl(c, w, sw, z, B, frames, g, r, y_units, ws, st);
+}
+
+bv_status bv_stitch_units(const bv_decoder_config *c, int B, int frames, const float *y_units,
+                          float *y, void *stream) {
+  g_err[0] = 0;
+  BV_TRY(check_config(c));
+  if (!y_units || !y) return fail(BV_ERR_ARG, "bv_stitch_units: null y_units or y");
+  if (B < 1 || frames < 1) return fail(BV_ERR_SHAPE, "bv_stitch_units: B=%d frames=%d", B, frames);
+  const UnitGeom g = unit_geom(c, frames);
+  const long long L = (long long)frames * hop_of(c);
+  if (L > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "bv_stitch_units: request too large");
+  const size_t nu = (size_t)g.n_tiles * B * c->out_channels * g.pitch;
+  const size_t ny = (size_t)B * c->out_channels * L;
+  if (overlaps(y_units, nu, y, ny)) return fail(BV_ERR_ARG, "bv_stitch_units: y_units and y overlap");
+  BV_TRY(check_device());
+  return stitch_units(c, g, B, frames, y_units, y, as_stream(stream));
+}
+
 size_t bv_decode_host_workspace_size(const bv_decoder_config *c, int B, int frames) {
   const size_t core = bv_decode_workspace_size(c, B, frames);
   if (core == 0) return 0;
   const long long L = (long long)frames * hop_of(c);
-  return core + align_up((size_t)B * c->in_channels * frames * sizeof(float)) +
+  return core + align_up((size_t)B * z_channels(c) * frames * sizeof(float)) +
          align_up((size_t)B * c->out_channels * L * sizeof(float));
 }
 
@@ -1006,7 +1536,7 @@ bv_status bv_decode_host(const bv_decoder_config *c, const bv_decoder_weights *w
   BV_TRY(check_weights(c, w));
   BV_TRY(check_device());
   const long long L = (long long)frames * hop_of(c);
-  const size_t zb = (size_t)B * c->in_channels * frames * sizeof(float);
+  const size_t zb = (size_t)B * z_channels(c) * frames * sizeof(float);
   const size_t yb = (size_t)B * c->out_channels * L * sizeof(float);
   char *p = static_cast<char *>(workspace);
   float *zd = reinterpret_cast<float *>(p);

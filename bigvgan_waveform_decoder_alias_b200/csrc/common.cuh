@@ -14,6 +14,13 @@ namespace bv {
 // Records a message for bv_last_error() and returns `st`.
 bv_status fail(bv_status st, const char *fmt, ...);
 
+// Clears the calling thread's error message (every ABI entry does first).
+void clear_error();
+
+// BV_OK if the current device is an sm_100 part (checked once per device),
+// else BV_ERR_CUDA.
+bv_status require_device();
+
 // Checks the last launch; BV_ERR_CUDA with the CUDA message on failure.
 bv_status check_launch(const char *what);
 
@@ -28,6 +35,10 @@ bv_status ensure_dynamic_smem(const void *func, size_t bytes, const char *what);
 // Address of the device status word that bounded waits set when they give
 // up (kernels take it as an argument); nullptr if it cannot be resolved.
 int *device_status_ptr();
+
+// Polls after which the tensor-core kernels' bounded waits give up (a kernel
+// argument; bv_debug_set_wait_limit changes it).
+long long wait_limit();
 
 // Per-launch event timing (bv_timing_enable).  Construct right before a
 // launch and let it go out of scope right after it.
@@ -147,6 +158,29 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
                             const float *lb, const float *fu, const float *fd, float eps,
                             cudaStream_t st);
 
+// The activation writing the time-major tensor-core conv's operand planes
+// hi[b, t, c] = tf32(y), lo = y - hi instead of y [B, C, T] (C a multiple of 8;
+// planes 16-byte aligned).
+bool activation_tm_supported(int C);
+bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int C, int T,
+                               const float *la, const float *lb, const float *fu, const float *fd,
+                               float eps, cudaStream_t st);
+
+// Latent front end: z [C, S, T] -> out [S, Cout, T], de-normalised then
+// projected by a one-tap conv w [Cout, C, 1] (+ bias or NULL).
+bv_status launch_latent_front_end(const float *z, int C, int S, int T, const float *mean,
+                                  const float *stdv, const float *w, const float *bias, int Cout,
+                                  float *out, cudaStream_t st);
+
+// The whole decoder (bv_decode without its argument checks): config and
+// weights check, workspace bytes, run (z, y device; ws 256-byte aligned),
+// samples per latent frame.
+bv_status decoder_check(const bv_decoder_config *c, const bv_decoder_weights *w);
+size_t decoder_workspace(const bv_decoder_config *c, int B, int F);
+bv_status decoder_run(const bv_decoder_config *c, const bv_decoder_weights *w, const float *z,
+                      int B, int F, float *y, char *ws, cudaStream_t st);
+long long decoder_hop(const bv_decoder_config *c);
+
 // The activation's sin^2, elementwise (for accuracy tests).
 bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream_t st);
 
@@ -231,6 +265,14 @@ bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B
                                      const float *w, const float *bias, int Cout, int K, int S,
                                      int pad, float *y, float *wp, cudaStream_t st);
 
+// The same with the phase weights packed beforehand (launch_convt_pack_tm
+// writes conv_transpose1d_tm_workspace bytes).
+bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, float *wp,
+                               cudaStream_t st);
+bv_status launch_conv_transpose1d_tm_packed(const float *x_hi, const float *x_lo, int B, int Cin,
+                                            int T, const float *wp, const float *bias, int Cout,
+                                            int K, int S, int pad, float *y, cudaStream_t st);
+
 // [B, C, T] -> time-major planes hi[b, t, c] = tf32(x[b, c, t]),
 // lo = x - hi.
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
@@ -244,6 +286,21 @@ size_t conv_transpose1d_tc_workspace(int Cin, int Cout, int K, int S);
 bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
                                      const float *bias, int Cout, int K, int S, int pad, float *y,
                                      float *wp, cudaStream_t st);
+
+// Narrow ConvTranspose1d on the FP32 pipe (at most 64 input and 32 output
+// channels, stride 1 or 2, at most 4 taps per phase).
+bool conv_transpose1d_small_supported(int Cin, int Cout, int K, int S);
+bv_status launch_conv_transpose1d_small(const float *x, int B, int Cin, int T, const float *w,
+                                        const float *bias, int Cout, int K, int S, int pad,
+                                        float *y, cudaStream_t st);
+
+// The [B, C, T] tensor-core ConvT with its phase weights packed beforehand
+// (launch_convt_pack_tc writes conv_transpose1d_tc_workspace bytes).
+bv_status launch_convt_pack_tc(const float *w, int Cin, int Cout, int K, int S, float *wp,
+                               cudaStream_t st);
+bv_status launch_conv_transpose1d_tc_packed(const float *x, int B, int Cin, int T,
+                                            const float *wp, const float *bias, int Cout, int K,
+                                            int S, int pad, float *y, cudaStream_t st);
 
 // ConvTranspose1d.
 bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const float *w,

@@ -26,9 +26,15 @@
 //   - the epilogue (bias, residual, scale, accumulate, final op) has one
 //     thread per time sample, so global reads and writes are coalesced.
 // Two operand stages overlap conversion with the MMAs.  Every mbarrier wait
-// is bounded; a wait that runs out sets the device status word and the CTA
-// unwinds (its output tile is then unspecified) after freeing its TMEM.
+// is bounded (wait_limit polls, a kernel argument); a wait that runs out sets
+// the device status word and marks the CTA aborted.  Aborting is orderly:
+// each role stops issuing work at its first failed wait, every producer then
+// waits (with a fixed bound) for the copies it issued, the MMA issuer waits
+// for a final commit that covers all its MMAs, and only then is TMEM freed;
+// the output tile is left unspecified.
 #include <cuda.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 
@@ -48,7 +54,7 @@ constexpr int W_TILE = MAX_NT * BK * 4;  // 16 KB: one weight operand tile (at m
 constexpr int THREADS = 256;
 constexpr int CONV_WARP0 = 4;            // warps 4..7 convert, add runs, write out
 constexpr int NCONV = 128;
-constexpr long long WAIT_LIMIT = 1ll << 26;  // try_wait polls before giving up
+constexpr long long DRAIN_LIMIT = 1ll << 22;  // polls for in-flight copies when unwinding
 constexpr int TMEM_COLS = 256;           // two accumulators of up to 128 columns
 constexpr int RUN = 4;                   // chunks accumulated in TMEM before an FP32 add
 constexpr int MAX_K = 32;                // largest kernel size (offset table rows)
@@ -116,37 +122,58 @@ __device__ __forceinline__ bool mbar_test(unsigned bar, unsigned parity) {
 }
 
 struct Ctl {
-  int abort;      // a bounded wait gave up somewhere in the CTA
+  int abort;      // a bounded wait gave up somewhere in the CTA (or its pair)
   unsigned tmem;  // TMEM base address from tcgen05.alloc
 };
 
-// Bounded wait on an mbarrier phase.  On running out it marks the CTA
-// aborted and records the failure in the device status word.
-__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
-                                          int *status, int code) {
+// How a CTA reports a wait that ran out: its own Ctl, the shared::cluster
+// address of its pair peer's abort flag (0 for a lone CTA), the device status
+// word and the poll limit.
+struct WaitCtx {
+  volatile Ctl *ctl;
+  unsigned peer_abort;
+  int *status;
+  long long limit;
+};
+
+__device__ __forceinline__ void raise_abort(const WaitCtx &w, int code) {
+  w.ctl->abort = 1;
+  if (w.peer_abort)
+    asm volatile("st.shared::cluster.u32 [%0], %1;\n" ::"r"(w.peer_abort), "r"(1) : "memory");
+  if (w.status) atomicExch(w.status, code);
+}
+
+// Bounded wait on an mbarrier phase: true once the phase has completed;
+// false after w.limit polls (the CTA and its peer are then marked aborted and
+// the failure recorded in the device status word) or once an abort raised
+// elsewhere in the pair is seen.  A role stops issuing work at its first
+// false.
+__device__ __forceinline__ bool mbar_wait(unsigned bar, unsigned parity, const WaitCtx &w,
+                                          int code) {
   if (mbar_test(bar, parity)) return true;
-  for (long long it = 0; it < WAIT_LIMIT; ++it) {
+  for (long long it = 0; it < w.limit; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 255) == 255 && ctl->abort) return false;
+    if ((it & 255) == 255 && w.ctl->abort) return false;
   }
-  ctl->abort = 1;
-  if (status) atomicExch(status, code);
+  raise_abort(w, code);
   return false;
 }
 
-// Bounded wait that does not return early on abort: used to drain copies that
-// are still in flight before the CTA exits.
+// Wait with a fixed bound that does not return early on abort: used to let
+// the copies and MMAs a role issued finish before the CTA frees TMEM or exits.
 __device__ __forceinline__ void mbar_drain(unsigned bar, unsigned parity) {
-  for (long long it = 0; it < (1ll << 22); ++it)
+  for (long long it = 0; it < DRAIN_LIMIT; ++it)
     if (mbar_try_wait(bar, parity)) return;
 }
 
 // Converter-side wait: lane 0 polls the barrier, the warp follows it, so the
-// polling does not compete with the conversion for shared-memory bandwidth.
-__device__ __forceinline__ void warp_wait(unsigned bar, unsigned parity, volatile Ctl *ctl,
-                                          int *status, int code) {
-  if ((threadIdx.x & 31) == 0) mbar_wait(bar, parity, ctl, status, code);
-  __syncwarp();
+// polling does not compete with the conversion for shared-memory bandwidth;
+// the outcome is the same for every lane.
+__device__ __forceinline__ bool warp_wait(unsigned bar, unsigned parity, const WaitCtx &w,
+                                          int code) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, w, code) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
 __device__ __forceinline__ void cp_async4_zfill(float *dst, const float *src, bool valid) {
@@ -214,7 +241,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
                  const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ x,
                  const float *__restrict__ bias, float *y, int Cin, int T, int Cout, int K,
-                 int dil, int pad, int y_len, int y_pitch, Epi ep, OutMap om, int *status) {
+                 int dil, int pad, int y_len, int y_pitch, Epi ep, OutMap om, int *status,
+                 long long wait_limit) {
   static_assert(NT % 16 == 0 && NT >= 16 && NT <= MAX_NT, "UMMA N for M = 128");
   constexpr int W_BYTES = NT * BK * 4;  // bytes of one weight chunk (TMA box)
   constexpr uint32_t IDESC = make_idesc(NT);
@@ -236,7 +264,9 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
   const unsigned bar_empty = smem_u32(&bars[8]);
   const unsigned bar_run_full = smem_u32(&bars[10]);
   const unsigned bar_run_free = smem_u32(&bars[12]);
+  const unsigned bar_done = smem_u32(&bars[14]);  // every MMA of the CTA has completed
   float *xs = reinterpret_cast<float *>(smem + OFF_X);
+  const WaitCtx wc{&ctl, 0u, status, wait_limit};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.x * BM;
@@ -263,6 +293,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
       mbar_init(bar_run_full + 8 * s, 1);
       mbar_init(bar_run_free + 8 * s, NCONV / 32);
     }
+    mbar_init(bar_done, 1);
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   // chunk m of an x block covers block-local kk = 32 m + e = i K + j
@@ -287,13 +318,13 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
+      int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % NWRING, u = c / NWRING;
-        // After an abort every wait returns at once and the loops run to the end
-        // without blocking, so all roles reach the final barrier.  A raw slot
-        // is free once the converters have split the chunk it held; a
-        // pre-split slot once the MMAs that read it have finished.
-        if (u > 0) mbar_wait(bar_raw_free + 8 * s, (u - 1) & 1, &ctl, status, 101);
+        // A raw slot is free once the converters have split the chunk it
+        // held; a pre-split slot once the MMAs that read it have finished.
+        // On a failed wait no further load is issued.
+        if (u > 0 && !mbar_wait(bar_raw_free + 8 * s, (u - 1) & 1, wc, 101)) break;
         const unsigned dst = smem_u32(smem + (PRESPLIT ? WL::hi(s) : WL::raw(s)));
         mbar_arrive_tx(bar_full_w + 8 * s, PRESPLIT ? 2 * W_BYTES : W_BYTES);
         asm volatile(
@@ -309,9 +340,11 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
               "l"(reinterpret_cast<uint64_t>(&tmap_wlo)), "r"(c * BK), "r"(w_row0),
               "r"(bar_full_w + 8 * s)
               : "memory");
+        issued = c + 1;
       }
-      // drain: the last loads must land before the CTA can exit
-      for (int c = n_chunks - NWRING; c < n_chunks; ++c)
+      // drain: every slot holds at most one load not yet seen complete, the
+      // last one issued into it; it must land before the CTA can exit
+      for (int c = issued - NWRING; c < issued; ++c)
         if (c >= 0) mbar_drain(bar_full_w + 8 * (c % NWRING), (c / NWRING) & 1);
     }
   } else if (warp == 1) {
@@ -322,11 +355,12 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
         const int r = c / RUN, ra = r & 1;
         const bool first = (c % RUN) == 0;
         const bool last = (c % RUN) == RUN - 1 || c == n_chunks - 1;
-        if (first && r >= 2)  // the converters have read this accumulator's run r - 2
-          mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 106);
-        mbar_wait(bar_ready + 8 * s, u & 1, &ctl, status, 102);
+        // the converters have read this accumulator's run r - 2
+        if (first && r >= 2 && !mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, wc, 106))
+          break;
+        if (!mbar_wait(bar_ready + 8 * s, u & 1, wc, 102)) break;
         const int ws = PRESPLIT ? c % NWSLOT : s;  // weight slot of this chunk
-        if (PRESPLIT) mbar_wait(bar_full_w + 8 * ws, (c / NWSLOT) & 1, &ctl, status, 107);
+        if (PRESPLIT && !mbar_wait(bar_full_w + 8 * ws, (c / NWSLOT) & 1, wc, 107)) break;
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
         const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
         const unsigned x_hi = smem_u32(smem + OFF_XHI + s * X_TILE);
@@ -345,6 +379,9 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
         if (PRESPLIT) mma_commit(bar_raw_free + 8 * ws);  // and the weight slot
         if (last) mma_commit(bar_run_full + 8 * ra);
       }
+      // no MMA may still write an accumulator when TMEM is freed
+      mma_commit(bar_done);
+      mbar_drain(bar_done, 0);
     }
   } else if (warp >= CONV_WARP0) {
     // ------------------------------------------------------ converters + sums
@@ -354,6 +391,10 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
     float sum[NT];  // time sample t0 + ct, channels o0 .. o0 + NT - 1: FP32 run sums
 #pragma unroll
     for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
+    // After this warp's first failed wait it does no more work and arrives on
+    // nothing, but keeps walking the chunks so that the four converter warps
+    // take the same named-barrier steps.
+    bool dead = false;
 
     // stage x block blk (channels [CB blk, CB blk + CB)) into xs[blk & 1];
     // channels >= Cin and times outside [0, T) read as zero
@@ -373,7 +414,10 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
     // add finished run p into the sums and hand its accumulator back
     auto promote = [&](int p) {
       const int ra = p & 1;
-      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 105);
+      if (dead || !warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, wc, 105)) {
+        dead = true;
+        return;
+      }
       asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
 #pragma unroll
       for (int c0 = 0; c0 < NT; c0 += 16) {
@@ -411,11 +455,13 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
         cp_async_wait_all();
         conv_bar_sync();  // everyone's copies of this block landed; the old block is free
         ready_blk = blk;
-        if ((blk + 1) * CB < Cin) stage_x(blk + 1);
+        if (!dead && (blk + 1) * CB < Cin) stage_x(blk + 1);
       }
-      if (u > 0) warp_wait(bar_empty + 8 * s, (u - 1) & 1, &ctl, status, 103);
+      if (!dead && u > 0 && !warp_wait(bar_empty + 8 * s, (u - 1) & 1, wc, 103)) dead = true;
+      if (!PRESPLIT && !dead && !warp_wait(bar_full_w + 8 * sr, (c / NRAW) & 1, wc, 104))
+        dead = true;
+      if (dead) continue;
       if (!PRESPLIT) {
-      warp_wait(bar_full_w + 8 * sr, (c / NRAW) & 1, &ctl, status, 104);
       // W: split into hi and lo (elementwise over the swizzled tile)
       const unsigned char *w_raw = smem + WL::raw(sr);
       unsigned char *w_hi = smem + WL::hi(s);
@@ -475,7 +521,7 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
       if (c >= (promoted + 1) * RUN + 1) promote(promoted++);
     }
     cp_async_wait_all();
-    while (promoted < n_runs) promote(promoted++);
+    while (!dead && promoted < n_runs) promote(promoted++);
 
     // ------------------------------------------------------------- epilogue
     // one thread per time sample: for each channel, the warp's 32 lanes touch
@@ -498,14 +544,8 @@ conv1d_tc_kernel(const __grid_constant__ CUtensorMap tmap_w,
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  __syncthreads();
+  __syncthreads();  // the MMA issuer has seen its final commit complete
   if (warp == 1) {
-    // no MMA may still write an accumulator when it is freed
-    if (lane == 0 && n_runs > 0) {
-      mbar_drain(bar_run_full + 8 * ((n_runs - 1) & 1), ((n_runs - 1) >> 1) & 1);
-      if (n_runs > 1) mbar_drain(bar_run_full + 8 * ((n_runs - 2) & 1), ((n_runs - 2) >> 1) & 1);
-    }
-    __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
                  "n"(TMEM_COLS)
@@ -564,7 +604,7 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tc: grid too large");
   conv1d_tc_kernel<NT, PRESPLIT><<<grid, THREADS, SMEM_BYTES, st>>>(
       tmap, tmap_lo, x, bias, y, Cin, T, Cout, K, dil, pad, y_len, y_pitch, ep, om,
-      device_status_ptr());
+      device_status_ptr(), wait_limit());
   return BV_OK;
 }
 
@@ -607,7 +647,7 @@ constexpr int TM_RUN = 2;                              // chunks (up to 4 taps o
 constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
 constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
 constexpr int TM_XSLOTS = 2;                          // x blocks in flight
-constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 + 2;
+constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 + 2 + 1;
 static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
@@ -713,7 +753,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_whi,
                  const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ bias,
                  float *y, int Cin, int Cout, int K, int dil, int pad, int y_len, int y_pitch,
-                 Epi ep, OutMap om, int *status) {
+                 Epi ep, OutMap om, int *status, long long wait_limit, int tpairs, int ntiles,
+                 int n_tiles) {
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= MAX_NT, "UMMA N for M = 256, halves of 16");
   constexpr uint32_t IDESC = make_idesc_pair(NT);
   constexpr unsigned W_TX_TAP = 2u * 2u * (NT / 2) * BK * 4;  // one tap: both CTAs, hi and lo
@@ -721,7 +762,6 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   unsigned char *smem = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ Ctl ctl;
-  __shared__ float bias_s[MAX_NT];  // this tile's biases (0 past Cout or without bias)
   const unsigned rank = cluster_rank();
   const bool leader = (rank == 0);
   const int xrows = BM + (K - 1) * dil;  // rows of one x box
@@ -732,13 +772,14 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + NW * TM_W_SLOT);
   // barriers (the leader's full and run-free barriers serve the pair):
   // x block loaded / consumed (TM_XSLOTS), weight chunk loaded / consumed
-  // (NW slots), run accumulated / run accumulator read (2)
+  // (NW slots), run accumulated / run accumulator read (2), every MMA done
   const unsigned bar_xfull = smem_u32(&bars[0]);
   const unsigned bar_xempty = smem_u32(&bars[TM_XSLOTS]);
   const unsigned bar_wfull = smem_u32(&bars[2 * TM_XSLOTS]);
   const unsigned bar_wempty = smem_u32(&bars[2 * TM_XSLOTS + TM_MAX_WSLOTS]);
   const unsigned bar_run_full = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS]);
   const unsigned bar_run_free = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2]);
+  const unsigned bar_done = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 4]);
   // x slot s, plane (0 hi, 1 lo); weight slot s, tap t of the chunk, plane
   auto x_at = [&](int slot, int plane) { return smem_u32(smem + (2 * slot + plane) * XP); };
   auto w_at = [&](int slot, int tap, int plane) {
@@ -746,18 +787,37 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = (blockIdx.x >> 1) * (2 * BM) + (int)rank * BM;  // this CTA's rows
-  const int o0 = blockIdx.y * NT;
-  const int b = blockIdx.z / om.phases;
-  const int phase = blockIdx.z - b * om.phases;  // weight rows phase Cout .., output offset + phase
+  // The pair walks the tiles cid, cid + P, ... (P pairs in the grid); tile
+  // tau is time pair tau % tpairs, output-channel tile (tau / tpairs) %
+  // ntiles and row-phase bz = tau / (tpairs ntiles).  Every role of both CTAs
+  // walks the same tiles, and the ring, run and phase counters run on across
+  // tiles, so the producers fill the next tile's operands and the MMAs start
+  // on it while the sum warps write the previous one out.
+  const int cid = (int)(blockIdx.x >> 1), P = (int)(gridDim.x >> 1);
+  struct Tile {
+    int t0, o0, b, phase;
+  };
+  auto tile_of = [&](int tau) {
+    Tile tl;
+    const int tp = tau % tpairs, rest = tau / tpairs;
+    const int bz = rest / ntiles;
+    tl.t0 = tp * (2 * BM) + (int)rank * BM;  // this CTA's rows
+    tl.o0 = (rest - bz * ntiles) * NT;
+    tl.b = bz / om.phases;
+    tl.phase = bz - tl.b * om.phases;  // weight rows phase Cout .., output offset + phase
+    return tl;
+  };
   const int n_cb = (Cin + BK - 1) / BK;  // 32-channel blocks (channels past Cin read as 0)
   const int Cpad = n_cb * BK;            // weight row stride per tap
   const int n_tc = (K + 1) / 2;       // chunks per block: taps (0,1), (2,3), ...
   const int n_chunks = n_cb * n_tc;
-  const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;
+  const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;  // per tile
+  // a wait that runs out marks both CTAs of the pair aborted
+  const WaitCtx wc{&ctl, map_to_rank(smem_u32(&ctl.abort), rank ^ 1u), status, wait_limit};
 
   if (threadIdx.x == 0) {
     ctl.abort = 0;
+    mbar_init(bar_done, 1);
     for (int s = 0; s < TM_XSLOTS; ++s) {
       mbar_init(bar_xfull + 8 * s, 1);
       mbar_init(bar_xempty + 8 * s, 1);
@@ -779,8 +839,6 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
   }
-  for (int i = threadIdx.x; i < MAX_NT; i += THREADS)
-    bias_s[i] = (bias && o0 + i < Cout) ? bias[o0 + i] : 0.0f;
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
   cluster_sync();  // both CTAs' barriers exist before anyone signals them
   asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -791,46 +849,62 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     // (a thread of its own, so a block waiting for its slot never holds up
     // the weight stream)
     if (lane == 0) {
-      // after an abort every wait returns at once, so all roles run to the end
-      for (int cb = 0; cb < n_cb; ++cb) {
-        const int xs = cb % TM_XSLOTS, xu = cb / TM_XSLOTS;
-        if (xu > 0) mbar_wait(bar_xempty + 8 * xs, (xu - 1) & 1, &ctl, status, 111);
-        const unsigned fb = bar_xfull + 8 * xs;
-        if (leader) mbar_arrive_tx(fb, X_TX);
-        tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * BK, t0 - pad, b, fb);
-        tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * BK, t0 - pad, b, fb);
+      // a failed wait stops the loads; a slot holds at most one load not yet
+      // seen complete, the last one issued into it (gcb counts the blocks
+      // issued over all tiles)
+      int gcb = 0;
+      bool ok = true;
+      for (int tau = cid; tau < n_tiles && ok; tau += P) {
+        const Tile tl = tile_of(tau);
+        for (int cb = 0; cb < n_cb; ++cb) {
+          const int xs = gcb % TM_XSLOTS, xu = gcb / TM_XSLOTS;
+          if (xu > 0 && !mbar_wait(bar_xempty + 8 * xs, (xu - 1) & 1, wc, 111)) {
+            ok = false;
+            break;
+          }
+          const unsigned fb = bar_xfull + 8 * xs;
+          if (leader) mbar_arrive_tx(fb, X_TX);
+          tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * BK, tl.t0 - pad, tl.b, fb);
+          tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * BK, tl.t0 - pad, tl.b, fb);
+          ++gcb;
+        }
       }
       if (leader)
-        for (int cb = n_cb - TM_XSLOTS; cb < n_cb; ++cb)
-          if (cb >= 0) mbar_drain(bar_xfull + 8 * (cb % TM_XSLOTS), (cb / TM_XSLOTS) & 1);
+        for (int c = gcb - TM_XSLOTS; c < gcb; ++c)
+          if (c >= 0) mbar_drain(bar_xfull + 8 * (c % TM_XSLOTS), (c / TM_XSLOTS) & 1);
     }
   } else if (warp == 0) {
     // ----------------------------------------------- TMA producer: weight chunks
     if (lane == 0) {
-      const int row = phase * Cout + o0 + (int)rank * (NT / 2);
-      int ws = 0, wphase = 0;
-      for (int cb = 0; cb < n_cb; ++cb) {
-        for (int q = 0; q < n_tc; ++q) {
-          if (cb * n_tc + q >= NW) mbar_wait(bar_wempty + 8 * ws, wphase ^ 1, &ctl, status, 112);
-          const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
-          const unsigned fb = bar_wfull + 8 * ws;
-          if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
-          for (int t = 0; t < ntap; ++t) {
-            const int col = (j0 + t) * Cpad + cb * BK;
-            tma_load_2d_pair(w_at(ws, t, 0), &tmap_whi, col, row, fb);
-            tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
-          }
-          if (++ws == NW) {
-            ws = 0;
-            wphase ^= 1;
+      int gc = 0;  // chunks issued over all tiles
+      bool ok = true;
+      for (int tau = cid; tau < n_tiles && ok; tau += P) {
+        const Tile tl = tile_of(tau);
+        const int row = tl.phase * Cout + tl.o0 + (int)rank * (NT / 2);
+        for (int cb = 0; cb < n_cb && ok; ++cb) {
+          for (int q = 0; q < n_tc; ++q) {
+            const int ws = gc % NW, wu = gc / NW;
+            if (wu > 0 && !mbar_wait(bar_wempty + 8 * ws, (wu - 1) & 1, wc, 112)) {
+              ok = false;
+              break;
+            }
+            const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+            const unsigned fb = bar_wfull + 8 * ws;
+            if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
+            for (int t = 0; t < ntap; ++t) {
+              const int col = (j0 + t) * Cpad + cb * BK;
+              tma_load_2d_pair(w_at(ws, t, 0), &tmap_whi, col, row, fb);
+              tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
+            }
+            ++gc;
           }
         }
       }
-      // drain: the pair's last loads land before the leader can exit (the odd
-      // CTA's land before the leader's MMAs read them, which the final
-      // cluster barrier waits for)
+      // drain: the pair's last loads land before the leader can exit (the
+      // leader's full barriers count the odd CTA's bytes too, and the final
+      // cluster barrier holds the odd CTA until then)
       if (leader)
-        for (int c = n_chunks - NW; c < n_chunks; ++c)
+        for (int c = gc - NW; c < gc; ++c)
           if (c >= 0) mbar_drain(bar_wfull + 8 * (c % NW), (c / NW) & 1);
     }
   } else if (warp == 1) {
@@ -838,98 +912,137 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     if (leader && lane == 0) {
       // descriptors are formed once per operand tile and advanced by adding
       // the byte offset / 16 (the start-address field; shared addresses stay
-      // below 256 KB, so the field never carries)
-      int c = 0, ws = 0, wphase = 0;
-      for (int cb = 0; cb < n_cb; ++cb) {
-        const int xs = cb % TM_XSLOTS;
-        mbar_wait(bar_xfull + 8 * xs, (cb / TM_XSLOTS) & 1, &ctl, status, 113);
-        const uint64_t dxh = sw128_desc(x_at(xs, 0)), dxl = sw128_desc(x_at(xs, 1));
-        for (int q = 0; q < n_tc; ++q, ++c) {
-          const int r = c / TM_RUN, ra = r & 1;
-          const bool first = (c % TM_RUN) == 0;
-          const bool last = (c % TM_RUN) == TM_RUN - 1 || c == n_chunks - 1;
-          if (first && r >= 2)  // both CTAs' sum warps have read this accumulator's run r - 2
-            mbar_wait(bar_run_free + 8 * ra, ((r >> 1) - 1) & 1, &ctl, status, 114);
-          mbar_wait(bar_wfull + 8 * ws, wphase, &ctl, status, 115);
-          asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-          const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
-          const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
-          for (int t = 0; t < ntap; ++t) {
-            const uint64_t rows = (uint64_t)((j0 + t) * dil * 8);  // tap's first row, in 16 B
-            const uint64_t ah = dxh + rows, al = dxl + rows;
-            const uint64_t bh = sw128_desc(w_at(ws, t, 0)), bl = sw128_desc(w_at(ws, t, 1));
-#pragma unroll
-            for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes = 2 x 16 B per MMA
-              const uint64_t o = 2 * k;
-              // X_hi is the A operand of two products: read it once
-              mma_tf32_pair<ACol::FILL>(acc, ah + o, bh + o, IDESC,
-                                        (first && t == 0 && k == 0) ? 0u : 1u);
-              mma_tf32_pair<ACol::LASTUSE>(acc, ah + o, bl + o, IDESC, 1u);
-              mma_tf32_pair<ACol::NONE>(acc, al + o, bh + o, IDESC, 1u);
-            }
+      // below 256 KB, so the field never carries).  gcb, gc, gr: x blocks,
+      // weight chunks and runs consumed over all tiles; a run never spans
+      // two tiles.
+      int gcb = 0, gc = 0, gr = 0;
+      bool ok = true;
+      for (int tau = cid; tau < n_tiles && ok; tau += P) {
+        int c = 0;  // chunk within the tile
+        for (int cb = 0; cb < n_cb && ok; ++cb, ++gcb) {
+          const int xs = gcb % TM_XSLOTS;
+          if (!mbar_wait(bar_xfull + 8 * xs, (gcb / TM_XSLOTS) & 1, wc, 113)) {
+            ok = false;
+            break;
           }
-          mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot
-          if (q == n_tc - 1) mma_commit_pair(bar_xempty + 8 * xs);  // and the x slot
-          if (last) mma_commit_pair(bar_run_full + 8 * ra);
-          if (++ws == NW) {
-            ws = 0;
-            wphase ^= 1;
+          const uint64_t dxh = sw128_desc(x_at(xs, 0)), dxl = sw128_desc(x_at(xs, 1));
+          for (int q = 0; q < n_tc; ++q, ++c, ++gc) {
+            const int ra = gr & 1, ws = gc % NW;
+            const bool first = (c % TM_RUN) == 0;
+            const bool last = (c % TM_RUN) == TM_RUN - 1 || c == n_chunks - 1;
+            // both CTAs' sum warps have read this accumulator's run gr - 2
+            if ((first && gr >= 2 &&
+                 !mbar_wait(bar_run_free + 8 * ra, ((gr >> 1) - 1) & 1, wc, 114)) ||
+                !mbar_wait(bar_wfull + 8 * ws, (gc / NW) & 1, wc, 115)) {
+              ok = false;
+              break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+            const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
+            const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+            for (int t = 0; t < ntap; ++t) {
+              const uint64_t rows = (uint64_t)((j0 + t) * dil * 8);  // tap's first row, in 16 B
+              const uint64_t ah = dxh + rows, al = dxl + rows;
+              const uint64_t bh = sw128_desc(w_at(ws, t, 0)), bl = sw128_desc(w_at(ws, t, 1));
+#pragma unroll
+              for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes = 2 x 16 B per MMA
+                const uint64_t o = 2 * k;
+                // X_hi is the A operand of two products: read it once
+                mma_tf32_pair<ACol::FILL>(acc, ah + o, bh + o, IDESC,
+                                          (first && t == 0 && k == 0) ? 0u : 1u);
+                mma_tf32_pair<ACol::LASTUSE>(acc, ah + o, bl + o, IDESC, 1u);
+                mma_tf32_pair<ACol::NONE>(acc, al + o, bh + o, IDESC, 1u);
+              }
+            }
+            mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot
+            if (q == n_tc - 1) mma_commit_pair(bar_xempty + 8 * xs);  // and the x slot
+            if (last) {
+              mma_commit_pair(bar_run_full + 8 * ra);
+              ++gr;
+            }
           }
         }
       }
+      // every MMA issued above has completed before TMEM can be freed
+      mma_commit_pair(bar_done);
+      mbar_drain(bar_done, 0);
     }
   } else if (warp >= CONV_WARP0) {
     // ------------------------------------------------------ run sums + output
     const int ct = threadIdx.x - CONV_WARP0 * 32;  // time row of this thread
     const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
     const unsigned run_free_leader = map_to_rank(bar_run_free, 0);
-    float sum[NT];
+    int gr = 0;  // runs read over all tiles
+    bool alive = true;
+    for (int tau = cid; tau < n_tiles && alive; tau += P) {
+      const Tile tl = tile_of(tau);
+      // this tile's biases, loaded before its runs so that the load latency
+      // hides behind the run waits: lane l holds channels o0 + l + 32 i,
+      // handed to the 16-channel groups by shuffles in the output loop
+      float breg[NT / 32];
 #pragma unroll
-    for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
-    for (int p = 0; p < n_runs; ++p) {
-      const int ra = p & 1;
-      warp_wait(bar_run_full + 8 * ra, (p >> 1) & 1, &ctl, status, 116);
-      asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
-#pragma unroll
-      for (int c0 = 0; c0 < NT; c0 += 16) {
-        uint32_t v[16];
-        const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * MAX_NT + c0);
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-            "%13,%14,%15}, [%16];\n"
-            : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-              "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-              "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-            : "r"(taddr)
-            : "memory");
-        asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
-#pragma unroll
-        for (int e = 0; e < 16; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+      for (int i = 0; i < NT / 32; ++i) {
+        const int o = tl.o0 + lane + 32 * i;
+        breg[i] = (bias && o < Cout) ? __ldg(bias + o) : 0.0f;
       }
-      asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
-    }
-    const int t = t0 + ct;
-    const int p = om.stride * t + om.offset + phase;  // output sample of conv position t
-    if (!ctl.abort && t < y_len && p >= 0 && p < om.len) {
-      // 16 channels at a time: the group's reads, then its writes
-      const size_t base = (size_t)b * Cout * y_pitch + p;
+      float sum[NT];
+#pragma unroll
+      for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
+      for (int p = 0; p < n_runs; ++p, ++gr) {
+        const int ra = gr & 1;
+        if (!warp_wait(bar_run_full + 8 * ra, (gr >> 1) & 1, wc, 116)) {
+          alive = false;
+          break;
+        }
+        asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+#pragma unroll
+        for (int c0 = 0; c0 < NT; c0 += 16) {
+          uint32_t v[16];
+          const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * MAX_NT + c0);
+          asm volatile(
+              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+              "%13,%14,%15}, [%16];\n"
+              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+              : "r"(taddr)
+              : "memory");
+          asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+          for (int e = 0; e < 16; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+        }
+        asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
+      }
+      if (!alive || ctl.abort) break;
+      const int t = tl.t0 + ct;
+      const int p = om.stride * t + om.offset + tl.phase;  // output sample of conv position t
+      const bool in = t < y_len && p >= 0 && p < om.len;
+      const size_t base = (size_t)tl.b * Cout * y_pitch + p;
 #pragma unroll
       for (int g = 0; g < NT; g += 16) {
-        float bb[16];
+        float bb[16];  // every lane of the warp takes part in the shuffles
 #pragma unroll
-        for (int q = 0; q < 16; ++q) bb[q] = bias_s[g + q];
-        epi_group<16>(sum + g, bb, ep, y, base + (size_t)(o0 + g) * y_pitch, (size_t)y_pitch,
-                      Cout - (o0 + g));
+        for (int e = 0; e < 16; ++e) bb[e] = __shfl_sync(0xffffffffu, breg[(g + e) >> 5], (g + e) & 31);
+        // 16 channels at a time: the group's reads, then its writes
+        if (in)
+          epi_group<16>(sum + g, bb, ep, y, base + (size_t)(tl.o0 + g) * y_pitch,
+                        (size_t)y_pitch, Cout - (tl.o0 + g));
       }
     }
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
-  // every MMA of the pair has completed (each CTA's sum warps saw the last
-  // run) and every remote arrive has landed before either CTA frees TMEM or
-  // its shared memory
+  __syncthreads();
+  // After an abort the odd CTA may have loads in flight that the leader's
+  // barriers did not count (issued after the leader stopped); they land in a
+  // few microseconds, so it waits 64 us before it can exit.
+  if (!leader && threadIdx.x == 0 && ctl.abort)
+    for (int i = 0; i < 64; ++i) __nanosleep(1000);
+  // every MMA of the pair has completed (the leader saw its final commit) and
+  // every remote arrive has landed before either CTA frees TMEM or its
+  // shared memory
   cluster_sync();
   if (warp == 1) {
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
@@ -939,6 +1052,23 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   }
 }
 
+// CTA pairs that fit on the device at once (one CTA per SM).
+int tm_pairs() {
+  constexpr int kMaxDev = 64;
+  static int cache[kMaxDev];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int slot = dev >= 0 && dev < kMaxDev ? dev : 0;
+  int n = __atomic_load_n(&cache[slot], __ATOMIC_RELAXED);
+  if (n == 0) {
+    int sms = 148;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    n = sms / 2 > 0 ? sms / 2 : 1;
+    __atomic_store_n(&cache[slot], n, __ATOMIC_RELAXED);
+  }
+  return n;
+}
+
 template <int NT>
 bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
@@ -946,11 +1076,15 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
                  const OutMap &om, cudaStream_t st) {
   BV_TRY(ensure_dynamic_smem((const void *)conv1d_tm_kernel<NT>, TM_SMEM_BYTES,
                              "conv1d_tm smem attribute"));
-  dim3 grid(2 * ((y_len + 2 * BM - 1) / (2 * BM)), (Cout + NT - 1) / NT, B * om.phases);
-  if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "conv1d_tm: grid too large");
-  conv1d_tm_kernel<NT><<<grid, THREADS, TM_SMEM_BYTES, st>>>(
+  // persistent: at most one CTA pair per two SMs, each walking its share of
+  // the (time pair, output-channel tile, row-phase) tiles
+  const long long tpairs = (y_len + 2 * BM - 1) / (2 * BM), ntiles = (Cout + NT - 1) / NT;
+  const long long n_tiles = tpairs * ntiles * (long long)B * om.phases;
+  if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "conv1d_tm: too many tiles");
+  const long long pairs = std::min<long long>(n_tiles, tm_pairs());
+  conv1d_tm_kernel<NT><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
       xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
-      device_status_ptr());
+      device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
   return BV_OK;
 }
 
@@ -1235,11 +1369,9 @@ size_t conv_transpose1d_tc_workspace(int Cin, int Cout, int K, int S) {
   return 2 * (size_t)S * Cout * Cin * convt_taps(K, S) * sizeof(float);  // wp and its lo part
 }
 
-bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
-                                     const float *bias, int Cout, int K, int S, int pad, float *y,
-                                     float *wp, cudaStream_t st) {
+bv_status launch_convt_pack_tc(const float *w, int Cin, int Cout, int K, int S, float *wp,
+                               cudaStream_t st) {
   const int nt = convt_taps(K, S);
-  const int Tout = (T - 1) * S + K - 2 * pad;
   const long long total = (long long)S * Cout * Cin * nt;
   {
     LaunchTimer tm(st, "convt_repack", 0.0, 8.0 * (double)total);
@@ -1248,19 +1380,31 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
         w, wp, wp + total, Cin, Cout, K, S, nt);
   }
   count_launch();
-  bv_status s = check_launch("convt_repack_kernel");
-  if (s != BV_OK) return s;
+  return check_launch("convt_repack_kernel");
+}
+
+bv_status launch_conv_transpose1d_tc_packed(const float *x, int B, int Cin, int T,
+                                            const float *wp, const float *bias, int Cout, int K,
+                                            int S, int pad, float *y, cudaStream_t st) {
+  const int nt = convt_taps(K, S);
+  const int Tout = (T - 1) * S + K - 2 * pad;
   // phase r: conv output P (input-grid index, P < T + nt - 1) lands on sample
-  // S P + r - pad of the output row
+  // S P + r - pad
   const OutMap om{S, -pad, Tout, S};
   const Epi plain{nullptr, 1.0f, 0, 0};
   return launch_tc_impl("conv_transpose1d_tc", x, B, Cin, T, wp, true, S * Cout, bias, Cout,
-                        nt, 1,
-                        nt - 1, plain, y, T + nt - 1, Tout, om,
+                        nt, 1, nt - 1, plain, y, T + nt - 1, Tout, om,
                         2.0 * B * Cin * (double)Cout * K * T,
                         4.0 * ((double)B * Cin * T + (double)Cin * Cout * K +
                                (double)B * Cout * Tout),
                         st);
+}
+
+bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, const float *w,
+                                     const float *bias, int Cout, int K, int S, int pad, float *y,
+                                     float *wp, cudaStream_t st) {
+  BV_TRY(launch_convt_pack_tc(w, Cin, Cout, K, S, wp, st));
+  return launch_conv_transpose1d_tc_packed(x, B, Cin, T, wp, bias, Cout, K, S, pad, y, st);
 }
 
 
@@ -1338,14 +1482,9 @@ size_t conv_transpose1d_tm_workspace(int Cin, int Cout, int K, int S) {
   return 2 * (size_t)S * Cout * tm_cin_pad(Cin) * convt_taps(K, S) * sizeof(float);
 }
 
-bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
-                                     const float *w, const float *bias, int Cout, int K, int S,
-                                     int pad, float *y, float *wp, cudaStream_t st) {
-  if (B <= 0 || T <= 0) return BV_OK;
-  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
-    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
+bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, float *wp,
+                               cudaStream_t st) {
   const int nt = convt_taps(K, S), cp = tm_cin_pad(Cin);
-  const int Tout = (T - 1) * S + K - 2 * pad;
   const long long total = (long long)S * Cout * nt * cp;
   {
     LaunchTimer tm(st, "convt_repack", 0.0, 4.0 * (double)Cin * Cout * K + 8.0 * (double)total);
@@ -1354,7 +1493,17 @@ bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B
         w, wp, wp + total, Cin, Cout, K, S, nt, cp);
   }
   count_launch();
-  BV_TRY(check_launch("convt_repack_tm_kernel"));
+  return check_launch("convt_repack_tm_kernel");
+}
+
+bv_status launch_conv_transpose1d_tm_packed(const float *x_hi, const float *x_lo, int B, int Cin,
+                                            int T, const float *wp, const float *bias, int Cout,
+                                            int K, int S, int pad, float *y, cudaStream_t st) {
+  if (B <= 0 || T <= 0) return BV_OK;
+  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
+    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
+  const int nt = convt_taps(K, S);
+  const int Tout = (T - 1) * S + K - 2 * pad;
   // phase r: conv output P (input-grid index, P < T + nt - 1) lands on sample
   // S P + r - pad of the output row
   return tm_impl("conv_transpose1d_tm", x_hi, x_lo, B, Cin, T, wp, S * Cout, bias, Cout, nt, 1,
@@ -1362,6 +1511,17 @@ bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B
                  2.0 * B * Cin * (double)Cout * K * T,
                  4.0 * ((double)B * Cin * T + (double)Cin * Cout * K + (double)B * Cout * Tout),
                  st);
+}
+
+bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
+                                     const float *w, const float *bias, int Cout, int K, int S,
+                                     int pad, float *y, float *wp, cudaStream_t st) {
+  if (B <= 0 || T <= 0) return BV_OK;
+  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
+    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
+  BV_TRY(launch_convt_pack_tm(w, Cin, Cout, K, S, wp, st));
+  return launch_conv_transpose1d_tm_packed(x_hi, x_lo, B, Cin, T, wp, bias, Cout, K, S, pad, y,
+                                           st);
 }
 
 }  // namespace bv

@@ -122,6 +122,8 @@ bv_status launch_conv_transpose1d(const float *x, int B, int Cin, int T, const f
                                   cudaStream_t st) {
   const int Tout = (T - 1) * S + K - 2 * pad;
   if (B <= 0 || Tout <= 0) return BV_OK;
+  if (conv_transpose1d_small_supported(Cin, Cout, K, S))
+    return launch_conv_transpose1d_small(x, B, Cin, T, w, bias, Cout, K, S, pad, y, st);
   const int NTX = S / gcd_i(S, 32) * 32;  // lcm(S, 32): a multiple of both
   if (NTX > 256) return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d: stride %d", S);
   const int NTY = 256 / NTX;

@@ -8,19 +8,21 @@
 namespace bv {
 namespace {
 
-// zt[(k * B + b), c, f] = z[b, c, start_k + f] for tiles k < n_tiles of length len.
+// zt[j, c, f] = z[b, c, k step + f] for unit u = u0 + j = k B + b (tile k of
+// side b), j < n_units, tiles of length len.
 __global__ void gather_tiles_kernel(const float *__restrict__ z, float *__restrict__ zt, int B,
-                                    int C, int frames, int step, int len, int k0, int n_tiles) {
-  const long long total = (long long)n_tiles * B * C * len;
+                                    int C, int frames, int step, int len, long long u0,
+                                    long long n_units) {
+  const long long total = n_units * C * len;
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
        i += (long long)gridDim.x * blockDim.x) {
     const int f = (int)(i % len);
     long long r = i / len;
     const int c = (int)(r % C);
-    r /= C;
-    const int b = (int)(r % B);
-    const int k = (int)(r / B) + k0;
-    zt[i] = z[((long long)b * C + c) * frames + (long long)k * step + f];
+    const long long u = u0 + r / C;
+    const int b = (int)(u % B);
+    const long long k = u / B;
+    zt[i] = z[((long long)b * C + c) * frames + k * step + f];
   }
 }
 
@@ -51,7 +53,7 @@ __global__ void stitch_tiles_kernel(TileGroups g, float *__restrict__ y, int B, 
         continue;
       }
       const long long row = (k - g.k0[gi]) * B + b;
-      sum += g.data[gi][(row * O + o) * len + (t - start)];
+      sum += g.data[gi][(row * O + o) * g.pitch[gi] + (t - start)];
       ++cnt;
     }
     y[i] = cnt ? sum / (float)cnt : 0.0f;
@@ -84,14 +86,14 @@ bv_status launch_add_parts(float *acc, const Parts &parts, long long n, cudaStre
 }
 
 bv_status launch_gather_tiles(const float *z, float *zt, int B, int C, int frames, int step,
-                              int len, int k0, int n_tiles, cudaStream_t st) {
-  const long long total = (long long)n_tiles * B * C * len;
+                              int len, long long u0, long long n_units, cudaStream_t st) {
+  const long long total = n_units * C * len;
   if (total <= 0) return BV_OK;
   const int threads = 256;
   const long long blocks = (total + threads - 1) / threads;
   LaunchTimer tm(st, "tiles", 0.0, 8.0 * (double)total);
   gather_tiles_kernel<<<(unsigned)(blocks < 148 * 32 ? blocks : 148 * 32), threads, 0, st>>>(
-      z, zt, B, C, frames, step, len, k0, n_tiles);
+      z, zt, B, C, frames, step, len, u0, n_units);
   count_launch();
   return check_launch("gather_tiles_kernel");
 }

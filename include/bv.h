@@ -88,6 +88,17 @@ void bv_timing_reset(void);
  * `stream`. */
 bv_status bv_sync_status(void *stream);
 
+/* Testing hook for the bounded waits.  The tensor-core kernels poll each
+ * mbarrier at most `polls` times (default 2^26) before they give up: the
+ * CTA (and its pair) then stops issuing work, lets the copies and MMAs it
+ * issued finish (each with its own fixed bound), frees its tensor memory,
+ * sets the status word that bv_sync_status reads, and leaves its output
+ * tile unspecified.  polls < 0 restores the default.  Takes effect for
+ * launches enqueued after the call, process-wide; returns the previous
+ * value.  A limit low enough to expire in a normal launch is for tests of
+ * that unwinding only. */
+long long bv_debug_set_wait_limit(long long polls);
+
 /* ------------------------------------------------------------------------
  * Kaiser-windowed sinc lowpass design, on the host.
  * [H3] `kaiser_sinc(cutoff, half_width, k)` and `bessel_i0`, `sinc`:
@@ -177,6 +188,48 @@ bv_status bv_conv_transpose1d(const float *x, int B, int Cin, int T,
                               const float *w, const float *bias, int Cout,
                               int K, int stride, int pad, float *y,
                               void *stream);
+
+/* ------------------------------------------------------------------------
+ * One activation followed by one Conv1d -- the unit step of an AMP block
+ * ([H3] `AmpBlock::apply`: `Activation1d::apply` then `Conv1d::apply`;
+ * [LTX] `AmpBlock::forward`) -- on the kernels the decoder itself runs:
+ *   h = down(snake(up(x)))            (as bv_activation1d, C channels)
+ *   y = epilogue(conv(h; w, bias, K, dilation, pad))   (as bv_conv1d)
+ * x [B, C, T]; log_alpha, log_beta [C]; filters [12]; w [Cout, C, K];
+ * bias [Cout] or NULL; y [B, Cout, T + 2 pad - dilation (K - 1)]; all
+ * device.  When the conv qualifies for the time-major tensor-core path
+ * (C a multiple of 4 with at most a third of channel padding to 32-channel
+ * blocks, Cout >= 40, (K - 1) dilation <= 56) the activation's output is
+ * laid out time-major and the conv runs there, as inside bv_decode.
+ * Workspace: bv_act_conv1d_workspace_size bytes, 256-byte aligned, disjoint
+ * from x, y and the residual.  x must not overlap y; the residual may be y.
+ * Errors: BV_ERR_ARG, BV_ERR_SHAPE (sizes < 1, K > 32, output length < 1),
+ * BV_ERR_WORKSPACE.
+ * ---------------------------------------------------------------------- */
+size_t bv_act_conv1d_workspace_size(int B, int C, int T, int Cout, int K,
+                                    int dilation);
+bv_status bv_act_conv1d(const float *x, int B, int C, int T,
+                        const float *log_alpha, const float *log_beta,
+                        const float *up_filter, const float *down_filter,
+                        float eps, const float *w, const float *bias, int Cout,
+                        int K, int dilation, int pad, const bv_epilogue *ep,
+                        float *y, void *workspace, size_t ws_bytes,
+                        void *stream);
+
+/* bv_conv_transpose1d on the kernels the decoder runs for its upsampling
+ * stages: with the workspace the phases run on the time-major tensor-core
+ * kernel (or the [B, C, T] one) where the shape qualifies, else on the FP32
+ * kernel (then the workspace may be empty).  Arguments, result and errors
+ * as bv_conv_transpose1d, plus BV_ERR_WORKSPACE.  Workspace:
+ * bv_conv_transpose1d_workspace_size bytes, 256-byte aligned, disjoint
+ * from x and y. */
+size_t bv_conv_transpose1d_workspace_size(int B, int Cin, int T, int Cout,
+                                          int K, int stride);
+bv_status bv_conv_transpose1d_ws(const float *x, int B, int Cin, int T,
+                                 const float *w, const float *bias, int Cout,
+                                 int K, int stride, int pad, float *y,
+                                 void *workspace, size_t ws_bytes,
+                                 void *stream);
 
 /* ------------------------------------------------------------------------
  * One AMP (anti-aliased multi-periodicity) residual block, [H3]
@@ -270,6 +323,13 @@ bv_status bv_amp_block_static(const float *x, int B, int C, int T,
  * and trimmed to its own frames * hop samples; where tiles overlap, the
  * samples are averaged over the tiles covering them ([M3] windowed forward).
  * Tiles of equal length are batched into one decode.
+ * Streams and threads: the AMP blocks of a stage run side by side on
+ * library-owned streams (one set per device, forked from and joined back to
+ * `stream` with events).  Calls from several host threads are safe: their
+ * fork/join sequences are enqueued one at a time under a per-device lock,
+ * and their blocks then share those streams.  While a decode is being
+ * captured into a CUDA graph, no other thread may decode on that device
+ * (its blocks would join the capture through the shared streams).
  * ---------------------------------------------------------------------- */
 typedef struct {
   int in_channels;
@@ -288,6 +348,10 @@ typedef struct {
   int final_act;
   int tile_frames;     /* 0: decode the whole latent at once */
   int overlap_frames;  /* < tile_frames */
+  int latent_channels; /* 0: z is the decoder's input [B, in_channels, frames].
+                        * > 0: z holds normalised latents [latent_channels, B,
+                        * frames] that first go through the latent front end
+                        * (bv_latent_front_end) into in_channels */
 } bv_decoder_config;
 
 typedef struct {
@@ -297,7 +361,44 @@ typedef struct {
   const float *post_log_alpha, *post_log_beta; /* [C_last] */
   const float *post_w, *post_b;               /* [out_ch, C_last, post_k], [out_ch] */
   const float *up_filter, *down_filter;       /* [12] each, used by act_post */
+  /* latent front end (used when latent_channels > 0): */
+  const float *latents_mean, *latents_std;    /* [latent_channels] */
+  const float *dec_in_w, *dec_in_b;           /* [in_ch, latent_ch, 1], [in_ch] or NULL */
+  /* NULL, or a buffer bv_decoder_prepare wrote for this config and these
+   * weight pointers: decodes then read the tensor-core weights from it
+   * instead of splitting them into the workspace on every call */
+  const void *prepared;
 } bv_decoder_weights;
+
+/* Prepared weights: the tf32 hi / lo split of every tensor-core conv's
+ * weights (tap-major where the conv runs time-major) and the packed phase
+ * weights of every tensor-core transposed conv, written once into a caller
+ * buffer (device, 256-byte aligned, bv_decoder_prepared_size bytes) and read
+ * by every later decode whose weights point at it (w->prepared).  The buffer
+ * derives from the weight values at the time of the call: re-prepare after
+ * changing them.  A decode with prepared weights needs only
+ * bv_decode_workspace_size_prepared bytes of workspace.  Errors:
+ * BV_ERR_ARG, BV_ERR_SHAPE, BV_ERR_WORKSPACE, BV_ERR_CUDA. */
+size_t bv_decoder_prepared_size(const bv_decoder_config *cfg);
+bv_status bv_decoder_prepare(const bv_decoder_config *cfg,
+                             const bv_decoder_weights *w, void *prepared,
+                             size_t bytes, void *stream);
+size_t bv_decode_workspace_size_prepared(const bv_decoder_config *cfg, int B,
+                                         int frames);
+
+/* The latent front end of [H3] `AudioVae::decode`: normalised latents z
+ * [C, S, T] (channel ci of side s at (ci S + s) T + t; the page's stereo
+ * layout is S = 2) are de-normalised per channel and projected by
+ * `dec_in_proj` ([H3] `AudioVae::from_cmf`: a Conv1d loaded with padding 0
+ * whose output keeps the length, hence one tap):
+ *   lat[s, ci, t] = z[ci, s, t] std[ci] + mean[ci],
+ *   out[s, o, t]  = bias[o] + sum_ci w[o, ci] lat[s, ci, t].
+ * z, mean, std, w [Cout, C, 1], bias [Cout] or NULL, out [S, Cout, T]: device.
+ * out must not overlap z.  Errors: BV_ERR_ARG, BV_ERR_SHAPE (sizes < 1). */
+bv_status bv_latent_front_end(const float *z, int C, int S, int T,
+                              const float *mean, const float *std,
+                              const float *w, const float *bias, int Cout,
+                              float *out, void *stream);
 
 /* Number of floats of the flat parameter vector of `cfg`, in module order:
  *  conv_pre w, b; per stage: ups w, b, then per block, per dilation:
@@ -321,11 +422,146 @@ int64_t bv_decoder_output_length(const bv_decoder_config *cfg, int frames);
  * (0 if the request is invalid; see bv_last_error). */
 size_t bv_decode_workspace_size(const bv_decoder_config *cfg, int B, int frames);
 
-/* z [B, in_channels, frames] -> y [B, out_channels, frames * hop], device.
+/* z [B, in_channels, frames] (or [latent_channels, B, frames] with the
+ * latent front end) -> y [B, out_channels, frames * hop], device.
  * Errors: BV_ERR_ARG, BV_ERR_SHAPE, BV_ERR_WORKSPACE, BV_ERR_CUDA. */
 bv_status bv_decode(const bv_decoder_config *cfg, const bv_decoder_weights *w,
                     const float *z, int B, int frames, float *y,
                     void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * The MiniMax-Music-3 DAV decoder ([H3] page, items `Snake`, `DavUnit`,
+ * `DavStage`, `Music3Dav`):
+ *   dec_in (one-tap Conv1d, latent_channels -> in_channels)
+ *   -> conv_pre (pad (pre_kernel - 1)/2, -> pre_channels)
+ *   -> for each stage i: Snake -> ConvT (rate up_rate[i], kernel
+ *      up_kernel[i], pad (k - s)/2, exactly s samples per input sample,
+ *      -> up_channels[i]) -> for each dilation d: x += c2(Snake(c1(Snake(x))))
+ *      with c1 a unit_kernel-tap conv at dilation d (pad d (unit_kernel-1)/2)
+ *      and c2 a one-tap conv
+ *   -> Snake -> conv_post (pad (post_kernel - 1)/2) -> final_act.
+ * Snake is the plain form with alpha used as stored:
+ *   v = x + sin^2(alpha_c x) / (alpha_c + 1e-9).
+ * The page's 128-channel latent is a stereo pair of 64: z [B = 2, 64, frames]
+ * in this interface (its layout is already [2, 64, frames]); the result is
+ * y [B, out_channels, frames * hop], hop = product of the rates (512 for
+ * strides 8, 8, 4, 2).  Weights are device pointers in PyTorch layouts.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int latent_channels, in_channels, pre_channels, pre_kernel;
+  int n_up;
+  int up_rate[BV_MAX_UP], up_kernel[BV_MAX_UP], up_channels[BV_MAX_UP];
+  int n_dilations;
+  int dilation[BV_MAX_DIL];
+  int unit_kernel, post_kernel, out_channels;
+  int final_act; /* 0 none, 1 clamp [-1, 1], 2 tanh (the page's) */
+} bv_dav_config;
+
+typedef struct {
+  const float *dec_in_w, *dec_in_b;      /* [in, latent, 1], [in] */
+  const float *pre_w, *pre_b;            /* [pre, in, pre_k], [pre] */
+  const float *stage_alpha[BV_MAX_UP];   /* [Cin_i] */
+  const float *up_w[BV_MAX_UP], *up_b[BV_MAX_UP]; /* [Cin_i, Cout_i, k_i], [Cout_i] */
+  const float *a1[BV_MAX_UP][BV_MAX_DIL], *c1_w[BV_MAX_UP][BV_MAX_DIL],
+      *c1_b[BV_MAX_UP][BV_MAX_DIL];     /* [C], [C, C, unit_k], [C] */
+  const float *a2[BV_MAX_UP][BV_MAX_DIL], *c2_w[BV_MAX_UP][BV_MAX_DIL],
+      *c2_b[BV_MAX_UP][BV_MAX_DIL];     /* [C], [C, C, 1], [C] */
+  const float *post_alpha, *post_w, *post_b; /* [C], [out, C, post_k], [out] */
+} bv_dav_weights;
+
+/* Floats of the flat parameter vector in module order: dec_in w, b; conv_pre
+ * w, b; per stage: act alpha, up w, b, then per dilation a1 alpha, c1 w, b,
+ * a2 alpha, c2 w, b; act_post alpha; conv_post w, b.  -1 if cfg is invalid
+ * (including a stage whose kernel does not give exactly `rate` samples per
+ * input sample). */
+int64_t bv_dav_param_count(const bv_dav_config *cfg);
+/* Pointers into a flat DEVICE parameter vector laid out as above. */
+bv_status bv_dav_weights_from_flat(const bv_dav_config *cfg, const float *flat,
+                                   bv_dav_weights *out);
+int64_t bv_dav_output_length(const bv_dav_config *cfg, int frames);
+size_t bv_dav_workspace_size(const bv_dav_config *cfg, int B, int frames);
+/* z [B, latent_channels, frames] -> y [B, out_channels, frames * hop], all
+ * device; z, y and the workspace disjoint.  Errors: BV_ERR_ARG,
+ * BV_ERR_SHAPE, BV_ERR_WORKSPACE, BV_ERR_CUDA. */
+bv_status bv_dav_decode(const bv_dav_config *cfg, const bv_dav_weights *w,
+                        const float *z, int B, int frames, float *y,
+                        void *workspace, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------
+ * The LTX-2.5 bandwidth-extension tail ([LTX] `AudioStack::decode_from_mel`
+ * after the first generator, `MelStft::forward`, `hann_sinc_upsample`).
+ *
+ * bv_mel_stft: the causal log-mel the extender reads.  x [C, T] is
+ * left-padded with n_fft - hop zeros; frame f starts at f hop;
+ *   frames = (T + n_fft - hop - n_fft) / hop + 1   (bv_mel_frames);
+ *   re[r] = sum_j v[j] basis[r, j], im[r] = sum_j v[j] basis[n_freqs + r, j],
+ *   out[c n_mels + m, f] = ln(max(sum_r mel_basis[m, r] |re + i im|, 1e-5)),
+ * the (channel, mel) fold of [LTX] `Vocoder::forward`.  basis [2 n_freqs,
+ * n_fft] (the checkpoint's DFT x window rows), mel_basis [n_mels, n_freqs],
+ * out [C n_mels, frames]; device.
+ *
+ * bv_sinc_upsample: x [C, T] -> y [C, ratio T], the Hann-windowed sinc
+ * interpolator (rolloff 0.99, 6 zero crossings, width = 7 input samples per
+ * side, k = 2 width ratio + 1 float taps), the input replicate-padded by
+ * width samples and scaled by ratio, a transposed FIR trimmed to
+ * [2 width ratio, ...).
+ *
+ * bv_bwe_tail: low [C, T] at the input rate -> y [C, ratio T]:
+ *   padded = low zero-padded to whole hops;
+ *   y = clamp(extender(mel_stft(padded)) + sinc_upsample(padded), -1, 1)
+ * over the first ratio T samples.  The extender is a decoder (cfg, w) run on
+ * one row of C n_mels channels with C outputs (cfg: in_channels = C n_mels,
+ * out_channels = C, final_act 0 as its output is a residual, untiled, no
+ * latent front end, hop = ratio x mel hop).  Errors: BV_ERR_ARG,
+ * BV_ERR_SHAPE, BV_ERR_WORKSPACE, BV_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+int64_t bv_mel_frames(int T, int n_fft, int hop);
+bv_status bv_mel_stft(const float *x, int C, int T, const float *basis,
+                      int n_freqs, int n_fft, int hop, const float *mel_basis,
+                      int n_mels, float *out, void *stream);
+bv_status bv_sinc_upsample(const float *x, int C, int T, int ratio, float *y,
+                           void *stream);
+size_t bv_bwe_tail_workspace_size(const bv_decoder_config *cfg, int C, int T,
+                                  int n_fft, int hop, int n_mels, int ratio);
+bv_status bv_bwe_tail(const bv_decoder_config *cfg, const bv_decoder_weights *w,
+                      const float *low, int C, int T, const float *stft_basis,
+                      int n_fft, int hop, const float *mel_basis, int n_mels,
+                      int ratio, float *y, void *workspace, size_t ws_bytes,
+                      void *stream);
+
+/* ------------------------------------------------------------------------
+ * The decode split into units, for sharding one decode over several GPUs
+ * (each decodes a range of units, the outputs are gathered, one GPU
+ * stitches).  Unit u = k * B + b is tile k of side b, in the tiling bv_decode
+ * uses (an untiled decode is one tile of all `frames` frames).  A unit's row
+ * holds out_channels x bv_decoder_unit_length samples: its tile's decoded
+ * waveform, trimmed to the tile's frames * hop (a shorter last tile fills
+ * only the front of its row; the rest of that row is unspecified).
+ * Decoding every unit and stitching gives bv_decode's result bit for bit
+ * (the units are decoded by the same kernels, rows independently).
+ * ---------------------------------------------------------------------- */
+/* Tiles of the tiling of `frames` (1 when untiled); -1 if invalid. */
+int bv_decoder_tile_count(const bv_decoder_config *cfg, int frames);
+/* Samples per unit row and output channel: tile_frames * hop (frames * hop
+ * when untiled); -1 if invalid. */
+int64_t bv_decoder_unit_length(const bv_decoder_config *cfg, int frames);
+size_t bv_decode_units_workspace_size(const bv_decoder_config *cfg, int B,
+                                      int frames, int64_t unit_begin,
+                                      int64_t unit_end);
+/* Decodes units [unit_begin, unit_end) of z [B, in_channels, frames] into
+ * y_units [unit_end - unit_begin, out_channels, unit length] (unit u at row
+ * u - unit_begin).  Errors as bv_decode; BV_ERR_SHAPE for a unit range
+ * outside [0, tiles * B) or empty. */
+bv_status bv_decode_units(const bv_decoder_config *cfg,
+                          const bv_decoder_weights *w, const float *z, int B,
+                          int frames, int64_t unit_begin, int64_t unit_end,
+                          float *y_units, void *workspace, size_t ws_bytes,
+                          void *stream);
+/* y [B, out_channels, frames * hop] from all tiles * B unit rows in unit
+ * order: each sample the mean of the tiles covering it ([M3] windowed
+ * forward).  y_units and y must not overlap. */
+bv_status bv_stitch_units(const bv_decoder_config *cfg, int B, int frames,
+                          const float *y_units, float *y, void *stream);
 
 /* bv_decode from HOST buffers: copies z_host (pinned for an asynchronous
  * copy) into the workspace, decodes, and copies the waveform back into
