@@ -58,7 +58,11 @@ __host__ __device__ constexpr int xoff(int i) { return 4 * ((i >> 1) + (i >> 2))
 __host__ __device__ constexpr int voff(int s) { return 4 * ((s >> 1) + (s >> 3)) + 2 * (s & 1); }
 constexpr int XS_FLOATS = xoff(XP - 1) + 2;
 constexpr int VS_FLOATS = voff(VP - 1) + 2;
-constexpr int WARP_FLOATS = 2 * XS_FLOATS + 2 * VS_FLOATS + 2 * 10;
+// Per warp: NX input windows (a ring, filled NX - 1 tiles ahead), two 2x-rate
+// buffers and the row pair's SnakeBeta constants.
+__host__ __device__ constexpr int warp_floats(int nx) { return nx * XS_FLOATS + 2 * VS_FLOATS + 2 * 10; }
+constexpr int K1_NX = 2;  // input windows of activation_kernel
+constexpr int WARP_FLOATS = warp_floats(K1_NX);
 constexpr size_t SMEM_BYTES = (size_t)WARPS * WARP_FLOATS * sizeof(float);
 static_assert(TW == 4 * 32, "4 outputs per lane");
 static_assert(XS_FLOATS % 4 == 0 && VS_FLOATS % 4 == 0 && WARP_FLOATS % 4 == 0, "16-byte alignment");
@@ -335,8 +339,11 @@ constexpr int TEAM = 4;                 // warps per team (row pairs of a group)
 constexpr int TM_CH = 2 * TEAM;         // channels per group
 constexpr int RP = 2 * TW + 8;          // region pitch: 2 RP = 16 (mod 32) banks apart
 constexpr int STG_FLOATS = TEAM * RP;   // one staging buffer
+constexpr int TM_NX = 3;                // input windows per warp: two tiles in flight
+constexpr int TM_WARP_FLOATS = warp_floats(TM_NX);
 constexpr size_t TM_SMEM_BYTES =
-    SMEM_BYTES + (size_t)(WARPS / TEAM) * 2 * STG_FLOATS * sizeof(float);
+    ((size_t)WARPS * TM_WARP_FLOATS + (size_t)(WARPS / TEAM) * 2 * STG_FLOATS) * sizeof(float);
+static_assert(TM_WARP_FLOATS % 4 == 0, "16-byte alignment");
 static_assert(WARPS % TEAM == 0 && RP % 32 == 8 && STG_FLOATS % 4 == 0, "staging layout");
 
 // Barrier 1 + team over the team's warps (immediate ids, so that the kernel
@@ -405,8 +412,9 @@ __device__ __forceinline__ void flush_quarter(const float *sb, float *__restrict
 // range of (row pair, tile) ids, row pair major, and writes y [rows, T].
 // TM = true: each team owns a range of (8-channel group, tile) tasks and
 // warp k walks row pair 4 group + k of them, writing the hi/lo planes
-// [B, T, C] (y = hi).
-template <bool TM>
+// [B, T, C] (y = hi).  NX input windows per warp: the copies of the next
+// NX - 1 tiles are in flight while a tile is computed.
+template <bool TM, int NX>
 __device__ __forceinline__ void activation_walk(
     const float *__restrict__ x, float *__restrict__ y, float *__restrict__ lo, int rows, int C,
     int T, int tiles_per_row, long long n_ids, const float *__restrict__ log_alpha,
@@ -430,11 +438,13 @@ __device__ __forceinline__ void activation_walk(
   }
   up_abs = fmaxf(up_abs, up_abs1);
 
-  float *wsm = smem + (size_t)warp * WARP_FLOATS;
-  float *const xs0 = wsm, *const vs0 = wsm + 2 * XS_FLOATS;  // buffer b at + b * size
-  float2 *cst = reinterpret_cast<float2 *>(wsm + 2 * XS_FLOATS + 2 * VS_FLOATS);
+  static_assert(NX >= 2 && NX <= 4, "input ring");
+  constexpr int WF = warp_floats(NX);
+  float *wsm = smem + (size_t)warp * WF;
+  float *const xs0 = wsm, *const vs0 = wsm + NX * XS_FLOATS;  // buffer b at + b * size
+  float2 *cst = reinterpret_cast<float2 *>(wsm + NX * XS_FLOATS + 2 * VS_FLOATS);
   const int team = warp / TEAM, k = warp % TEAM;
-  float *const stg = smem + (size_t)WARPS * WARP_FLOATS + (size_t)team * 2 * STG_FLOATS;
+  float *const stg = smem + (size_t)WARPS * WF + (size_t)team * 2 * STG_FLOATS;
 
   // this warp's (or team's) contiguous range of ids (row pair or group) *
   // tiles_per_row + tile
@@ -449,8 +459,25 @@ __device__ __forceinline__ void activation_walk(
   constexpr int kStep = TM ? TEAM : 1;  // row pairs from one id row to the next
   int pair = (int)(beg / tiles_per_row), tile = (int)(beg % tiles_per_row);
   if (TM) pair = TEAM * pair + k;
-  issue_tile(row_ptr(pair, 0), row_ptr(pair, 1), xs0, tile * TW, T, lane);
-  cp_async_commit();
+  // (fpair, ftile): the tile of id fid = id + NX - 1, whose copies the
+  // iteration of id issues; the prologue issues ids beg .. beg + NX - 2
+  int fpair = pair, ftile = tile;
+  long long fid = beg;
+  auto advance = [&](int &pr, int &tl) {
+    if (++tl == tiles_per_row) {
+      tl = 0;
+      pr += kStep;
+    }
+  };
+#pragma unroll
+  for (int j = 0; j < NX - 1; ++j) {
+    if (fid < end) issue_tile(row_ptr(fpair, 0), row_ptr(fpair, 1), xs0 + j * XS_FLOATS,
+                              ftile * TW, T, lane);
+    cp_async_commit();
+    ++fid;
+    advance(fpair, ftile);
+  }
+  int xslot = 0;  // input window of id (id - beg mod NX)
   int cur_pair = -1;
   bool pending = false;  // stage B of the previous tile still to run
   int p_t0 = 0;
@@ -469,16 +496,19 @@ __device__ __forceinline__ void activation_walk(
   };
   for (long long id = beg; id < end; ++id) {
     const int b = (int)((id - beg) & 1);
-    int npair = pair, ntile = tile + 1;
-    if (ntile == tiles_per_row) {
-      ntile = 0;
-      npair += kStep;
-    }
+    int npair = pair, ntile = tile;
+    advance(npair, ntile);
     __syncwarp();  // the previous iteration's reads of the buffers written below are done
-    if (id + 1 < end)
-      issue_tile(row_ptr(npair, 0), row_ptr(npair, 1), xs0 + (b ^ 1) * XS_FLOATS, ntile * TW, T,
-                 lane);
-    cp_async_commit();
+    {
+      // the window of id + NX - 1 is the one id - 1 used
+      const int fslot = xslot == 0 ? NX - 1 : xslot - 1;
+      if (fid < end)
+        issue_tile(row_ptr(fpair, 0), row_ptr(fpair, 1), xs0 + fslot * XS_FLOATS, ftile * TW, T,
+                   lane);
+      cp_async_commit();
+      ++fid;
+      advance(fpair, ftile);
+    }
     if (pair != cur_pair) {
       // the row pair's SnakeBeta constants (every lane computes the same values)
       cur_pair = pair;
@@ -509,10 +539,11 @@ __device__ __forceinline__ void activation_walk(
         obase = (size_t)bb * T * C + (row0 - bb * C);
       }
     }
-    cp_async_wait<1>();  // this tile's input has landed (the next one may be in flight)
+    cp_async_wait<NX - 1>();  // this tile's input has landed (the next ones may be in flight)
     __syncwarp();
     const int t0 = tile * TW;
-    const float *xb = xs0 + b * XS_FLOATS;
+    const float *xb = xs0 + xslot * XS_FLOATS;
+    xslot = xslot == NX - 1 ? 0 : xslot + 1;
     float *vb = vs0 + b * VS_FLOATS, *vo = vs0 + (b ^ 1) * VS_FLOATS;
     stage_a(xb, vb, vo, taps, cst, up_abs, lane);
     __syncwarp();
@@ -563,8 +594,8 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
                   int tiles_per_row, long long n_tiles, const float *__restrict__ log_alpha,
                   const float *__restrict__ log_beta, const float *__restrict__ f_up,
                   const float *__restrict__ f_dn, float eps) {
-  activation_walk<false>(x, y, nullptr, rows, C, T, tiles_per_row, n_tiles, log_alpha, log_beta,
-                         f_up, f_dn, eps);
+  activation_walk<false, K1_NX>(x, y, nullptr, rows, C, T, tiles_per_row, n_tiles, log_alpha,
+                                log_beta, f_up, f_dn, eps);
 }
 
 __global__ void __launch_bounds__(THREADS, 2)
@@ -572,8 +603,8 @@ activation_tm_kernel(const float *__restrict__ x, float *__restrict__ hi, float 
                      int rows, int C, int T, int tiles_per_row, long long n_tasks,
                      const float *__restrict__ log_alpha, const float *__restrict__ log_beta,
                      const float *__restrict__ f_up, const float *__restrict__ f_dn, float eps) {
-  activation_walk<true>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha, log_beta, f_up,
-                        f_dn, eps);
+  activation_walk<true, TM_NX>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha,
+                               log_beta, f_up, f_dn, eps);
 }
 
 __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restrict__ out,

@@ -876,14 +876,15 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   } else if (warp == 0) {
     // ----------------------------------------------- TMA producer: weight chunks
     if (lane == 0) {
-      int gc = 0;  // chunks issued over all tiles
+      // slot ws of pass wu over the ring (counters, not divisions: this loop
+      // and the MMA issuer's are single threads on the critical path)
+      int ws = 0, wu = 0, gc = 0;  // gc: chunks issued over all tiles
       bool ok = true;
       for (int tau = cid; tau < n_tiles && ok; tau += P) {
         const Tile tl = tile_of(tau);
         const int row = tl.phase * Cout + tl.o0 + (int)rank * (NT / 2);
         for (int cb = 0; cb < n_cb && ok; ++cb) {
           for (int q = 0; q < n_tc; ++q) {
-            const int ws = gc % NW, wu = gc / NW;
             if (wu > 0 && !mbar_wait(bar_wempty + 8 * ws, (wu - 1) & 1, wc, 112)) {
               ok = false;
               break;
@@ -897,6 +898,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
               tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
             }
             ++gc;
+            if (++ws == NW) {
+              ws = 0;
+              ++wu;
+            }
           }
         }
       }
@@ -915,7 +920,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       // below 256 KB, so the field never carries).  gcb, gc, gr: x blocks,
       // weight chunks and runs consumed over all tiles; a run never spans
       // two tiles.
-      int gcb = 0, gc = 0, gr = 0;
+      int gcb = 0, gr = 0, ws = 0;
+      unsigned wphase = 0;
       bool ok = true;
       for (int tau = cid; tau < n_tiles && ok; tau += P) {
         int c = 0;  // chunk within the tile
@@ -926,14 +932,14 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
             break;
           }
           const uint64_t dxh = sw128_desc(x_at(xs, 0)), dxl = sw128_desc(x_at(xs, 1));
-          for (int q = 0; q < n_tc; ++q, ++c, ++gc) {
-            const int ra = gr & 1, ws = gc % NW;
+          for (int q = 0; q < n_tc; ++q, ++c) {
+            const int ra = gr & 1;
             const bool first = (c % TM_RUN) == 0;
             const bool last = (c % TM_RUN) == TM_RUN - 1 || c == n_chunks - 1;
             // both CTAs' sum warps have read this accumulator's run gr - 2
             if ((first && gr >= 2 &&
                  !mbar_wait(bar_run_free + 8 * ra, ((gr >> 1) - 1) & 1, wc, 114)) ||
-                !mbar_wait(bar_wfull + 8 * ws, (gc / NW) & 1, wc, 115)) {
+                !mbar_wait(bar_wfull + 8 * ws, wphase, wc, 115)) {
               ok = false;
               break;
             }
@@ -959,6 +965,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
             if (last) {
               mma_commit_pair(bar_run_full + 8 * ra);
               ++gr;
+            }
+            if (++ws == NW) {
+              ws = 0;
+              wphase ^= 1u;
             }
           }
         }
