@@ -53,3 +53,28 @@ def test_single_rank_and_throughput():
     # 2 replicas, 10 s of audio each per 40 ms step -> 500 audio-s/s for the job
     assert bench.job_throughput(2, 10.0, 40.0) == pytest.approx(500.0)
     assert bench.job_throughput(1, 10.0, 40.0) == pytest.approx(250.0)
+
+
+def test_tensor_peak_follows_the_clocks():
+    """The 3xTF32 roofline denominator: the burst figure at the maximum clock
+    without capping, the sustained figure scaled by the sampled clock under
+    capping or a lower clock, and never more than the burst figure."""
+    sys.path.insert(0, ROOT)
+    import bench
+    pk = {"bf16": 1590.0, "bf16_sustained": 1400.0, "sustained_mhz": 1300.0,
+          "sm_max_mhz": 1965.0, "source": "fallback"}
+    burst = 1590.0 * bench.TF32_PER_BF16 / 3.0
+    peak, _, b = bench.tensor_peak(pk, None)
+    assert peak == pytest.approx(burst) and b == pytest.approx(burst)
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.tensor_peak(pk, full)[0] == pytest.approx(burst)
+    capped_low = {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(pk, capped_low)[0] == pytest.approx(
+        1400.0 * bench.TF32_PER_BF16 / 3.0)
+    # a brief cap at the maximum clock: the scaled sustained figure would
+    # exceed the burst one, so the burst one is taken
+    capped_full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(pk, capped_full)[0] == pytest.approx(burst)
+    slow = {"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []}
+    assert bench.tensor_peak(pk, slow)[0] == pytest.approx(
+        1400.0 * 1000.0 / 1300.0 * bench.TF32_PER_BF16 / 3.0)
