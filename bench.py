@@ -11,6 +11,7 @@ batch on its own GPU (independent replicas, no collective on the data path);
 the step time is the max over ranks.  Prints one JSON line on rank 0.
 """
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -51,7 +52,11 @@ def parse():
                     help="time one kernel on one shape instead of the decoder (for profiling): "
                          "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s | "
                          "actconv:BxCxT:K:d (activation then conv, the decoder's kernels) | "
-                         "amp:BxCxT:K (an AMP block, dilations 1, 3, 5)")
+                         "amp:BxCxT:K (an AMP block, dilations 1, 3, 5) | "
+                         "frontend:CxSxT:Cout (latent de-normalisation + dec_in) | "
+                         "dav:FRAMES (the Music-3 DAV decoder on a stereo latent) | "
+                         "bwe:FRAMES (the LTX bandwidth-extension tail on FRAMES mel hops of "
+                         "stereo 16 kHz input)")
     return ap.parse_args()
 
 
@@ -60,10 +65,46 @@ def run_case(args):
     import torch
     from bigvgan_waveform_decoder_alias_b200 import native
     kind, shape, *rest = args.case.split(":")
-    B, C, T = (int(v) for v in shape.split("x"))
     s = synth.NormalStream(7)
-    x = torch.from_numpy(s.normal((B, C, T))).cuda()
     filt = torch.from_numpy(native.bv_filter_design()).cuda()
+    if kind in ("dav", "bwe"):
+        # whole decoders: the unit is audio-seconds of output per second
+        frames = int(shape)
+        if kind == "dav":
+            geo = synth.MUSIC3_DAV
+            z = torch.from_numpy(s.normal((2, geo.latent_channels, frames))).cuda()
+            dec = native.DavDecoder(geo, synth.draw_dav_params(s, geo))
+            y = dec.decode(z)
+            ws = torch.empty(native.lib().bv_dav_workspace_size(
+                ctypes.byref(dec.cfg), 2, frames) // 4 + 64, device="cuda")
+            fn = lambda: dec.decode(z, y=y, workspace=ws)  # noqa: E731
+            work = frames * geo.hop / geo.sample_rate
+        else:
+            geo, sp = synth.LTX_BWE, synth.LTX_BWE_SPEC
+            low = torch.from_numpy(0.3 * s.normal((2, frames * sp.hop))).cuda()
+            params = synth._draw_params(s, synth.param_layout(geo))
+            basis, mel = sp.bases()
+            tail = native.BweTail(geo, params, sp, basis, mel, filt=filt.cpu().numpy())
+            y = tail(low)
+            ws = torch.empty(native.lib().bv_bwe_tail_workspace_size(
+                ctypes.byref(tail.dec.cfg), 2, frames * sp.hop, sp.n_fft, sp.hop, sp.n_mels,
+                sp.ratio) // 4 + 64, device="cuda")
+            fn = lambda: tail(low, y=y, workspace=ws)  # noqa: E731
+            work = frames * sp.hop / sp.in_rate
+        unit = "audio_s/s"
+        return _time_case(args, native, fn, work, unit)
+    B, C, T = (int(v) for v in shape.split("x"))
+    x = torch.from_numpy(s.normal((B, C, T))).cuda()
+    if kind == "frontend":
+        # z [C, S, T] with S = B sides here: C latent channels x S x T frames
+        Cl, S, Tf, Cout = B, C, T, int(rest[0])
+        mean = torch.from_numpy(s.normal((Cl,), 0.0, 0.5)).cuda()
+        std = torch.from_numpy(np.abs(s.normal((Cl,), 1.0, 0.3)) + 0.1).cuda()
+        w = torch.from_numpy(s.normal((Cout, Cl, 1), 0.0, 0.2)).cuda()
+        b = torch.from_numpy(s.normal((Cout,), 0.0, 0.1)).cuda()
+        out = torch.empty((S, Cout, Tf), device="cuda")
+        fn = lambda: native.bv_latent_front_end(x, mean, std, w, b, out=out)  # noqa: E731
+        return _time_case(args, native, fn, 4.0 * (Cl + Cout) * S * Tf, "GB/s")
     if kind == "activation":
         la = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
         lb = torch.from_numpy(s.normal((C,), 0, 0.1)).cuda()
@@ -114,6 +155,13 @@ def run_case(args):
         work, unit = 2.0 * 6 * B * C * C * K * T, "TFLOP/s"
     else:
         raise SystemExit(f"unknown case {kind}")
+    return _time_case(args, native, fn, work, unit)
+
+
+def _time_case(args, native, fn, work, unit):
+    """W warm-up calls, K calls timed with CUDA events on the current stream
+    (median), then a pass with the library's per-class timers."""
+    import torch
     for _ in range(args.warmup):
         fn()
     torch.cuda.synchronize()
@@ -125,7 +173,7 @@ def run_case(args):
         b_.record()
     torch.cuda.synchronize()
     ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
-    rate = work / (ms / 1000) / (1e9 if unit == "GB/s" else 1e12)
+    rate = work / (ms / 1000) / {"GB/s": 1e9, "TFLOP/s": 1e12}.get(unit, 1.0)
     # a second pass with the library's per-class event timers: the mean time
     # of each kernel class per call (for cases that launch several kernels)
     native.timing_reset()
@@ -551,8 +599,10 @@ def main():
         kernels[name]["roofline"] = r
     dom = max(kernels, key=lambda k: kernels[k]["ms_per_step"]) if kernels else None
     roof = dict(roofs[dom], kernel=dom) if dom else None
-    # the fused activation: algorithmic bytes / time
-    acts = [kernels[k] for k in ("activation",) if k in kernels]
+    # the fused activation, both forms (K1 writes [B, C, T]: 8 B per element;
+    # K1tm writes the conv's hi/lo planes: 12 B): algorithmic bytes / time
+    act_classes = [k for k in ("activation", "activation_tm") if k in kernels]
+    acts = [kernels[k] for k in act_classes]
     act = None
     if acts:
         ms = sum(k["ms_per_step"] for k in acts)
@@ -561,7 +611,7 @@ def main():
         act = {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
                "frac": gbs / pk["hbm_gbs"], "traffic": None,
                "peak_source": f"{pk['source']} hbm_gbs",
-               "kernels": [k for k in ("activation",) if k in kernels]}
+               "kernels": act_classes}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -998,6 +998,15 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       float sum[NT];
 #pragma unroll
       for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
+      // The residual of this thread's output row, 16 channels after each of
+      // the first NT / 16 runs: the loads overlap the wait for the next run
+      // instead of the output loop, and the values join the sum there
+      // ((conv + residual) + bias instead of (conv + bias) + residual).
+      const int t_out = tl.t0 + ct;
+      const int p_out = om.stride * t_out + om.offset + tl.phase;  // output sample
+      const bool in = t_out < y_len && p_out >= 0 && p_out < om.len;
+      const size_t base = (size_t)tl.b * Cout * y_pitch + p_out;
+      const bool fold = ep.residual != nullptr;
       for (int p = 0; p < n_runs; ++p, ++gr) {
         const int ra = gr & 1;
         if (!warp_wait(bar_run_full + 8 * ra, (gr >> 1) & 1, wc, 116)) {
@@ -1024,21 +1033,33 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
+        if (fold && in && p < NT / 16) {
+          const int valid = Cout - (tl.o0 + 16 * p);
+          const float *rp = ep.residual + base + (size_t)(tl.o0 + 16 * p) * y_pitch;
+          float r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = e < valid ? __ldg(rp + (size_t)e * y_pitch) : 0.0f;
+#pragma unroll
+          for (int g = 0; g < NT / 16; ++g)
+            if (g == p) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) sum[16 * g + e] += r[e];
+            }
+        }
       }
       if (!alive || ctl.abort) break;
-      const int t = tl.t0 + ct;
-      const int p = om.stride * t + om.offset + tl.phase;  // output sample of conv position t
-      const bool in = t < y_len && p >= 0 && p < om.len;
-      const size_t base = (size_t)tl.b * Cout * y_pitch + p;
 #pragma unroll
       for (int g = 0; g < NT; g += 16) {
         float bb[16];  // every lane of the warp takes part in the shuffles
 #pragma unroll
         for (int e = 0; e < 16; ++e) bb[e] = __shfl_sync(0xffffffffu, breg[(g + e) >> 5], (g + e) & 31);
-        // 16 channels at a time: the group's reads, then its writes
+        // 16 channels at a time: the group's reads, then its writes (without
+        // the residual where it joined the sum above)
+        Epi eg = ep;
+        if (fold && g / 16 < n_runs) eg.residual = nullptr;
         if (in)
-          epi_group<16>(sum + g, bb, ep, y, base + (size_t)(tl.o0 + g) * y_pitch,
-                        (size_t)y_pitch, Cout - (tl.o0 + g));
+          epi_group<16>(sum + g, bb, eg, y, base + (size_t)(tl.o0 + g) * y_pitch, (size_t)y_pitch,
+                        Cout - (tl.o0 + g));
       }
     }
   }
@@ -1422,9 +1443,11 @@ bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
   // input rows of Cin floats must be 16-byte multiples (TMA strides); a
   // partial last channel block costs padded tensor work, so at most a third.
   // Below 40 output channels (measured on B200 with 24: N = 32 tiles) the
-  // FP32 SIMT kernel is faster.
+  // FP32 SIMT kernel is faster.  A reduction of two channel blocks (a one-tap
+  // conv over 64 channels) already beats the SIMT kernel (measured on the
+  // DAV decoder's 96-channel one-tap convs).
   return Cin % 4 == 0 && 3 * tm_cin_pad(Cin) <= 4 * Cin && Cout >= 40 &&
-         tm_cin_pad(Cin) * K >= 192 && K >= 1 && K <= MAX_K && dil >= 1 &&
+         tm_cin_pad(Cin) * K >= 64 && K >= 1 && K <= MAX_K && dil >= 1 &&
          (K - 1) * dil <= TM_MAX_HALO && encode_fn() != nullptr;
 }
 

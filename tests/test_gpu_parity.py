@@ -535,11 +535,12 @@ def test_act_conv_time_major_activation_ragged(nat, oracle, filt, B, C, T):
 
 
 @pytest.mark.parametrize("C,T,K,d", [(64, 777, 7, 3), (128, 300, 3, 1), (24, 513, 11, 5),
-                                     (100, 257, 5, 2)])
+                                     (100, 257, 5, 2), (96, 1000, 1, 1), (64, 515, 1, 1)])
 def test_act_conv_small_shapes_every_element(nat, oracle, filt, C, T, K, d):
     """bv_act_conv1d on every path (time-major with the fused activation for
-    64 / 128 channels, time-major through a separate transpose for 100, the
-    narrow FP32 kernel for 24), every output against the oracle."""
+    64 / 96 / 128 channels, one-tap convs included, time-major through a
+    separate transpose for 100, the narrow FP32 kernel for 24), every output
+    against the oracle."""
     s = synth.NormalStream(12000 + C + T)
     x = s.normal((2, C, T))
     la, lb = s.normal((C,), 0.0, 0.2), s.normal((C,), 0.0, 0.2)
