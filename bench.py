@@ -263,10 +263,20 @@ def tensor_peak(pk, clocks):
 # kernel classes that run 3xTF32 on the tensor cores
 TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm")
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from an
-# ncu capture of a few launches, per kernel class, for the kernel code named
-# beside it; null for a class without a capture of its current code.
-NCU_TRAFFIC_PER_LAUNCH = {}
+# Measured DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) over
+# the algorithmic bytes, per kernel class, from one ncu capture of every launch
+# of the class's kernel in one decode of the default workload; the bench's
+# `traffic` is this ratio x the class's algorithmic bytes per launch.  A class
+# whose kernel code changed since its capture has no entry (traffic null).
+#   conv1d_tm: conv1d_tm_kernel, all 190 launches of one 60 s stereo decode
+#   (180 AMP convs + 10 transposed convs), 59.70 GB against 43.71 GB
+#   algorithmic; kernel code of the residual fold between runs.
+NCU_TRAFFIC_RATIO = {"conv1d_tm": 1.366}
+
+
+def traffic_for(name, kd):
+    r = NCU_TRAFFIC_RATIO.get(name)
+    return None if r is None else r * kd["bytes"]
 
 
 def roofline_for(name, kd, pk, clocks=None):
@@ -279,18 +289,18 @@ def roofline_for(name, kd, pk, clocks=None):
         ach = kd["flops"] / t / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "frac_of_burst": ach / burst,
-                "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name), "peak_source": src}
+                "traffic": traffic_for(name, kd), "peak_source": src}
     mhz = (clocks or {}).get("sm_max_mhz") or pk["sm_max_mhz"]
     if kd["flops"] > 0:
         peak = SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
         ach = kd["flops"] / t / 1e12
         return {"bound": "alu", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": ach / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
+                "frac": ach / peak, "traffic": traffic_for(name, kd),
                 "peak_source": f"FP32 pipe: {SMS} SMs x {FP32_LANES_PER_SM} lanes x 2 x "
                                f"{mhz:.0f} MHz"}
     ach = kd["bytes"] / t / 1e9
     return {"bound": "hbm", "achieved": ach, "peak": pk["hbm_gbs"], "unit": "GB/s",
-            "frac": ach / pk["hbm_gbs"], "traffic": NCU_TRAFFIC_PER_LAUNCH.get(name),
+            "frac": ach / pk["hbm_gbs"], "traffic": traffic_for(name, kd),
             "peak_source": f"{pk['source']} hbm_gbs"}
 
 
