@@ -184,10 +184,17 @@ __device__ __forceinline__ void issue_tile(const float *__restrict__ x0,
   }
 }
 
+// Four consecutive outputs: one 16-byte store where the row allows it, two
+// 8-byte stores where it is only 8-byte aligned (rows of an even length not a
+// multiple of 4 alternate between the two), else four 4-byte stores.
 __device__ __forceinline__ void store4(float *yr, int t, int T, float o0, float o1, float o2,
                                        float o3) {
-  if (t + 3 < T && ((reinterpret_cast<uintptr_t>(yr + t) & 15u) == 0)) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(yr + t);
+  if (t + 3 < T && (a & 15u) == 0) {
     __stcs(reinterpret_cast<float4 *>(yr + t), make_float4(o0, o1, o2, o3));
+  } else if (t + 3 < T && (a & 7u) == 0) {
+    __stcs(reinterpret_cast<float2 *>(yr + t), make_float2(o0, o1));
+    __stcs(reinterpret_cast<float2 *>(yr + t + 2), make_float2(o2, o3));
   } else {
     if (t < T) yr[t] = o0;
     if (t + 1 < T) yr[t + 1] = o1;

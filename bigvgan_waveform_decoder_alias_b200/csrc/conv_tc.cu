@@ -647,7 +647,14 @@ constexpr int TM_RUN = 2;                              // chunks (up to 4 taps o
 constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
 constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
 constexpr int TM_XSLOTS = 2;                          // x blocks in flight
-constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 + 2 + 1;
+// Run accumulators in TMEM (MAX_NT columns each; all 512 columns: the kernel
+// is alone on its SM, its shared memory leaves room for no other CTA).  With
+// four the issuer can run three runs ahead of the sum warps, which covers a
+// tile's output loop.
+constexpr int TM_ACC = 4;
+constexpr int TM_TMEM_COLS = TM_ACC * MAX_NT;
+static_assert(TM_TMEM_COLS <= 512 && (TM_ACC & (TM_ACC - 1)) == 0, "TMEM accumulators");
+constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC + 1;
 static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
@@ -778,8 +785,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const unsigned bar_wfull = smem_u32(&bars[2 * TM_XSLOTS]);
   const unsigned bar_wempty = smem_u32(&bars[2 * TM_XSLOTS + TM_MAX_WSLOTS]);
   const unsigned bar_run_full = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS]);
-  const unsigned bar_run_free = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2]);
-  const unsigned bar_done = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 4]);
+  const unsigned bar_run_free = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + TM_ACC]);
+  const unsigned bar_done = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC]);
   // x slot s, plane (0 hi, 1 lo); weight slot s, tap t of the chunk, plane
   auto x_at = [&](int slot, int plane) { return smem_u32(smem + (2 * slot + plane) * XP); };
   auto w_at = [&](int slot, int tap, int plane) {
@@ -822,7 +829,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       mbar_init(bar_xfull + 8 * s, 1);
       mbar_init(bar_xempty + 8 * s, 1);
     }
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < TM_ACC; ++s) {
       mbar_init(bar_run_full + 8 * s, 1);
       mbar_init(bar_run_free + 8 * s, 2 * NCONV / 32);  // sum warps of both CTAs
     }
@@ -835,7 +842,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(
                      smem_u32(&ctl.tmem)),
-                 "n"(TMEM_COLS)
+                 "n"(TM_TMEM_COLS)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;\n" ::: "memory");
   }
@@ -933,12 +940,12 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
           }
           const uint64_t dxh = sw128_desc(x_at(xs, 0)), dxl = sw128_desc(x_at(xs, 1));
           for (int q = 0; q < n_tc; ++q, ++c) {
-            const int ra = gr & 1;
+            const int ra = gr & (TM_ACC - 1);
             const bool first = (c % TM_RUN) == 0;
             const bool last = (c % TM_RUN) == TM_RUN - 1 || c == n_chunks - 1;
-            // both CTAs' sum warps have read this accumulator's run gr - 2
-            if ((first && gr >= 2 &&
-                 !mbar_wait(bar_run_free + 8 * ra, ((gr >> 1) - 1) & 1, wc, 114)) ||
+            // both CTAs' sum warps have read this accumulator's run gr - TM_ACC
+            if ((first && gr >= TM_ACC &&
+                 !mbar_wait(bar_run_free + 8 * ra, ((gr / TM_ACC) - 1) & 1, wc, 114)) ||
                 !mbar_wait(bar_wfull + 8 * ws, wphase, wc, 115)) {
               ok = false;
               break;
@@ -1008,27 +1015,33 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       const size_t base = (size_t)tl.b * Cout * y_pitch + p_out;
       const bool fold = ep.residual != nullptr;
       for (int p = 0; p < n_runs; ++p, ++gr) {
-        const int ra = gr & 1;
-        if (!warp_wait(bar_run_full + 8 * ra, (gr >> 1) & 1, wc, 116)) {
+        const int ra = gr & (TM_ACC - 1);
+        if (!warp_wait(bar_run_full + 8 * ra, (gr / TM_ACC) & 1, wc, 116)) {
           alive = false;
           break;
         }
         asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
+        // 32 columns per wait: two loads in flight
 #pragma unroll
-        for (int c0 = 0; c0 < NT; c0 += 16) {
-          uint32_t v[16];
+        for (int c0 = 0; c0 < NT; c0 += 32) {
+          uint32_t v[32];
           const unsigned taddr = tmem + ((unsigned)(32 * q) << 16) + (unsigned)(ra * MAX_NT + c0);
-          asm volatile(
-              "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
-              "%13,%14,%15}, [%16];\n"
-              : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
-                "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
-                "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
-              : "r"(taddr)
-              : "memory");
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
+                "%12,%13,%14,%15}, [%16];\n"
+                : "=r"(v[16 * h + 0]), "=r"(v[16 * h + 1]), "=r"(v[16 * h + 2]),
+                  "=r"(v[16 * h + 3]), "=r"(v[16 * h + 4]), "=r"(v[16 * h + 5]),
+                  "=r"(v[16 * h + 6]), "=r"(v[16 * h + 7]), "=r"(v[16 * h + 8]),
+                  "=r"(v[16 * h + 9]), "=r"(v[16 * h + 10]), "=r"(v[16 * h + 11]),
+                  "=r"(v[16 * h + 12]), "=r"(v[16 * h + 13]), "=r"(v[16 * h + 14]),
+                  "=r"(v[16 * h + 15])
+                : "r"(taddr + 16u * h)
+                : "memory");
           asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
 #pragma unroll
-          for (int e = 0; e < 16; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+          for (int e = 0; e < 32; ++e) sum[c0 + e] += __uint_as_float(v[e]);
         }
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
         __syncwarp();
@@ -1078,7 +1091,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   if (warp == 1) {
     asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;\n" ::"r"(tmem),
-                 "n"(TMEM_COLS)
+                 "n"(TM_TMEM_COLS)
                  : "memory");
   }
 }
