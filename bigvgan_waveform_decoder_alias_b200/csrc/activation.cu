@@ -363,6 +363,11 @@ __device__ __forceinline__ void team_barrier(int team) {
     asm volatile("bar.sync 2, %0;\n" ::"n"(32 * TEAM) : "memory");
 }
 
+// Float offset of time step tl's (channel 2k, 2k + 1) pair in a staging
+// region: 2 tl, with the two 16-byte chunks of every 32-byte lane slot
+// swapped in the upper half of each 16-step block.
+__device__ __forceinline__ int stg_index(int tl) { return (2 * tl) ^ (((tl >> 4) & 1) << 2); }
+
 // Stage B of row pair k into its staging region: lane L holds t = 4 L + e,
 // stored as (channel 2k, 2k + 1) pairs, two 16-byte stores per lane.
 __device__ __forceinline__ void stage_b_stage(const float *vb, const float2 *taps, float *region,
@@ -385,9 +390,12 @@ __device__ __forceinline__ void stage_b_stage(const float *vb, const float2 *tap
     for (int j = 1; j < 12; ++j) acc = fma2(D2[j], W[2 * e + j], acc);
     out[e] = acc;
   }
+  // the two 16-byte chunks of lane L swap places when bit 2 of L is set
+  // (stg_index), so each quarter warp's stores hit 8 distinct bank groups
+  const int s = (lane >> 2) & 1;
   float4 *r4 = reinterpret_cast<float4 *>(region + 8 * lane);
-  r4[0] = make_float4(out[0].x, out[0].y, out[1].x, out[1].y);
-  r4[1] = make_float4(out[2].x, out[2].y, out[3].x, out[3].y);
+  r4[s] = make_float4(out[0].x, out[0].y, out[1].x, out[1].y);
+  r4[1 - s] = make_float4(out[2].x, out[2].y, out[3].x, out[3].y);
 }
 
 // Warp k's quarter of a staged tile: time steps 32 k .. 32 k + 31, per round
@@ -400,8 +408,8 @@ __device__ __forceinline__ void flush_quarter(const float *sb, float *__restrict
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
     const int tl = 32 * k + 16 * r + (lane >> 1), t = t0 + tl;
-    const float2 a = *reinterpret_cast<const float2 *>(sb + (2 * h) * RP + 2 * tl);
-    const float2 c = *reinterpret_cast<const float2 *>(sb + (2 * h + 1) * RP + 2 * tl);
+    const float2 a = *reinterpret_cast<const float2 *>(sb + (2 * h) * RP + stg_index(tl));
+    const float2 c = *reinterpret_cast<const float2 *>(sb + (2 * h + 1) * RP + stg_index(tl));
     if (t < T) {
       const float v[4] = {a.x, a.y, c.x, c.y};
       float g[4];
