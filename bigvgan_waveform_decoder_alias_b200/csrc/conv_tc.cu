@@ -929,10 +929,6 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       // two tiles.
       int gcb = 0, gr = 0, ws = 0;
       unsigned wphase = 0;
-      // the next weight slot was seen loaded by a test in the middle of the
-      // previous chunk's MMAs (whose issue waits on the tensor pipe anyway),
-      // so its wait costs nothing here
-      bool w_ready = false;
       bool ok = true;
       for (int tau = cid; tau < n_tiles && ok; tau += P) {
         int c = 0;  // chunk within the tile
@@ -950,7 +946,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
             // both CTAs' sum warps have read this accumulator's run gr - TM_ACC
             if ((first && gr >= TM_ACC &&
                  !mbar_wait(bar_run_free + 8 * ra, ((gr / TM_ACC) - 1) & 1, wc, 114)) ||
-                (!w_ready && !mbar_wait(bar_wfull + 8 * ws, wphase, wc, 115))) {
+                !mbar_wait(bar_wfull + 8 * ws, wphase, wc, 115)) {
               ok = false;
               break;
             }
@@ -969,10 +965,6 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                                           (first && t == 0 && k == 0) ? 0u : 1u);
                 mma_tf32_pair<ACol::LASTUSE>(acc, ah + o, bl + o, IDESC, 1u);
                 mma_tf32_pair<ACol::NONE>(acc, al + o, bh + o, IDESC, 1u);
-              }
-              if (t == 0) {
-                const int wsn = ws + 1 == NW ? 0 : ws + 1;
-                w_ready = mbar_test(bar_wfull + 8 * wsn, ws + 1 == NW ? wphase ^ 1u : wphase);
               }
             }
             mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot
