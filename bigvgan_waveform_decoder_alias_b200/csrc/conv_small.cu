@@ -13,8 +13,11 @@
 // outside [0, T)) and all the weights, reordered so that the output channels
 // of one (input channel, tap) are contiguous, then each thread accumulates 4
 // consecutive outputs x COUT channels in registers: per (i, j), four reads of
-// x and COUT/4 broadcast 16-byte reads of w feed 4 COUT FMAs.  The common
-// kernel sizes are template arguments, so the tap loop unrolls.
+// x and COUT/4 broadcast 16-byte reads of w feed 4 COUT FMAs, issued as
+// packed pairs over output channels (2p, 2p + 1) against x duplicated into
+// both halves: each half is an ordinary round-to-nearest FMA, so the results
+// are those of scalar FMAs, in half the instructions.  The common kernel
+// sizes are template arguments, so the tap loop unrolls.
 #include "common.cuh"
 
 namespace bv {
@@ -63,11 +66,11 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
   __syncthreads();
 
   const int tl = SM_PER * tid;  // this thread's outputs t0 + tl .. t0 + tl + SM_PER - 1
-  float acc[COUT][SM_PER];
+  float2 acc2[COUT / 2][SM_PER];  // output channels (2p, 2p + 1)
 #pragma unroll
-  for (int o = 0; o < COUT; ++o)
+  for (int o = 0; o < COUT / 2; ++o)
 #pragma unroll
-    for (int e = 0; e < SM_PER; ++e) acc[o][e] = 0.0f;
+    for (int e = 0; e < SM_PER; ++e) acc2[o][e] = make_float2(0.0f, 0.0f);
   for (int i = 0; i < Cin; ++i) {
     const float *xr = xs + i * XW + tl;
     const float4 *wr = reinterpret_cast<const float4 *>(ws + i * K * COUT);
@@ -77,15 +80,17 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
 #pragma unroll
       for (int e = 0; e < SM_PER; ++e) xv[e] = xr[j * dil + e];
       const float4 *wj = wr + j * (COUT / 4);
+      float2 xx[SM_PER];
+#pragma unroll
+      for (int e = 0; e < SM_PER; ++e) xx[e] = make_float2(xv[e], xv[e]);
 #pragma unroll
       for (int o4 = 0; o4 < COUT / 4; ++o4) {
         const float4 wv = wj[o4];
+        const float2 w01 = make_float2(wv.x, wv.y), w23 = make_float2(wv.z, wv.w);
 #pragma unroll
         for (int e = 0; e < SM_PER; ++e) {
-          acc[4 * o4][e] = fmaf(wv.x, xv[e], acc[4 * o4][e]);
-          acc[4 * o4 + 1][e] = fmaf(wv.y, xv[e], acc[4 * o4 + 1][e]);
-          acc[4 * o4 + 2][e] = fmaf(wv.z, xv[e], acc[4 * o4 + 2][e]);
-          acc[4 * o4 + 3][e] = fmaf(wv.w, xv[e], acc[4 * o4 + 3][e]);
+          acc2[2 * o4][e] = __ffma2_rn(w01, xx[e], acc2[2 * o4][e]);
+          acc2[2 * o4 + 1][e] = __ffma2_rn(w23, xx[e], acc2[2 * o4 + 1][e]);
         }
       }
     }
@@ -121,7 +126,8 @@ conv1d_small_kernel(const float *__restrict__ x, const float *__restrict__ w,
         float v[SM_PER];
 #pragma unroll
         for (int e = 0; e < SM_PER; ++e)
-          v[e] = epi_final((acc[o][e] + bias_s[o] + r[q][e]) * ep.scale + a[q][e], ep);
+          v[e] = epi_final(((o & 1 ? acc2[o >> 1][e].y : acc2[o >> 1][e].x) + bias_s[o] + r[q][e]) *
+                               ep.scale + a[q][e], ep);
         if (vec) {
           *reinterpret_cast<float4 *>(y + idx) = make_float4(v[0], v[1], v[2], v[3]);
         } else {
