@@ -270,7 +270,8 @@ TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpo
 # whose kernel code changed since its capture has no entry (traffic null).
 #   conv1d_tm: conv1d_tm_kernel, all 190 launches of one 60 s stereo decode
 #   (180 AMP convs + 10 transposed convs), 59.70 GB against 43.71 GB
-#   algorithmic; kernel code of the residual fold between runs.
+#   algorithmic (one ncu pass per launch); kernel code of commit 5eafb75
+#   (four run accumulators), unchanged since.
 NCU_TRAFFIC_RATIO = {"conv1d_tm": 1.366}
 
 
