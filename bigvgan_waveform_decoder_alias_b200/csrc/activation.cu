@@ -330,37 +330,75 @@ __device__ __forceinline__ void copy_pair(float *vb, int dst, int src) {
 // lo = y - hi, so the activation's output never exists in [B, C, T] form and
 // no separate transpose pass reads it back.
 //
-// A CTA holds two teams of four warps.  A team owns a contiguous range of
-// tasks (8-channel group of one batch row, time tile), group-major; warp k of
-// the team takes the group's row pair k (channels 2k, 2k + 1) and walks the
-// range's tiles exactly as activation_kernel walks a row pair, so consecutive
-// tiles share their 2x-rate values and the SnakeBeta constants are set up
-// once per row pair.  Stage B writes the pair's TW outputs into the team's
-// staging buffer, one region per row pair ([4][RP] floats, time steps as
-// (channel 2k, 2k + 1) pairs); after a named barrier over the team each warp
-// writes a quarter of the tile (32 time steps x 8 channels) to both planes as
-// 32-byte rows, whole sectors.  Two staging buffers alternate, so one
-// barrier per tile orders both the writes before the flush and the flush
-// before the buffer's next use.
-constexpr int TEAM = 4;                 // warps per team (row pairs of a group)
-constexpr int TM_CH = 2 * TEAM;         // channels per group
-constexpr int RP = 2 * TW + 8;          // region pitch: 2 RP = 16 (mod 32) banks apart
-constexpr int STG_FLOATS = TEAM * RP;   // one staging buffer
+// A team of TW_ warps owns a contiguous range of tasks (a group of 2 TW_
+// channels of one batch row, time tile), group-major; warp k of the team
+// takes the group's row pair k (channels 2k, 2k + 1) and walks the range's
+// tiles exactly as activation_kernel walks a row pair, so consecutive tiles
+// share their 2x-rate values and the SnakeBeta constants are set up once per
+// row pair.  Stage B writes the pair's TW outputs into the team's staging
+// buffer, one region per row pair (time steps as (channel 2k, 2k + 1)
+// pairs); after a named barrier over the team each warp writes its share of
+// the tile's time steps, all 2 TW_ channels of each, to both planes.  Two
+// staging buffers alternate, so one barrier per tile orders both the writes
+// before the flush and the flush before the buffer's next use.
+//
+// The flush is what costs: a 16-byte store instruction whose 32 lanes write
+// pieces of many cache lines is paid per line on the SM's write path (with
+// only the hi plane written the kernel ran in 0.65 of the time).  Three team
+// shapes, the widest the channel count allows:
+//   32 channels (C a multiple of 32): one team of 16 warps per CTA; eight
+//     lanes write one time step's 32 channels, a whole aligned 128-byte line
+//     of each plane, four lines per instruction;
+//   16 channels: one team of 8 warps per CTA; 64 bytes, 8 lines;
+//   8 channels: two teams of 4 warps per CTA; 32 bytes, 16 lines.
+template <int TW_>
+struct TeamShape {
+  static constexpr int kWarps = TW_;                  // per team = row pairs per group
+  static constexpr int kCh = 2 * TW_;                 // channels per group
+  static constexpr int kCtaWarps = TW_ < WARPS ? WARPS : TW_;
+  static constexpr int kTeams = kCtaWarps / TW_;
+  static constexpr int kLanesPerStep = TW_ / 2;       // lanes per time step in the flush
+  static constexpr int kStepsPerRound = 32 / kLanesPerStep;
+  static constexpr int kStepsPerWarp = TW / TW_;      // of a tile's TW time steps
+  // region r of a staging buffer: 16-byte aligned, and shifted by 64 / TW_
+  // floats per region pair so that a half warp's 8-byte flush reads (32 / TW_
+  // time steps of each of its TW_ / 2 region pairs) hit distinct banks
+  __host__ __device__ static constexpr int region(int r) {
+    return 2 * TW * r + (64 / TW_) * (r >> 1);
+  }
+  static constexpr int kStgFloats = (region(TW_ - 1) + 2 * TW + 3) / 4 * 4;
+};
 constexpr int TM_NX = 3;                // input windows per warp: two tiles in flight
 constexpr int TM_WARP_FLOATS = warp_floats(TM_NX);
-constexpr size_t TM_SMEM_BYTES =
-    ((size_t)WARPS * TM_WARP_FLOATS + (size_t)(WARPS / TEAM) * 2 * STG_FLOATS) * sizeof(float);
 static_assert(TM_WARP_FLOATS % 4 == 0, "16-byte alignment");
-static_assert(WARPS % TEAM == 0 && RP % 32 == 8 && STG_FLOATS % 4 == 0, "staging layout");
+template <int TW_>
+constexpr size_t tm_smem_bytes() {
+  using S = TeamShape<TW_>;
+  return ((size_t)S::kCtaWarps * TM_WARP_FLOATS + (size_t)S::kTeams * 2 * S::kStgFloats) *
+         sizeof(float);
+}
+static_assert(TeamShape<4>::kTeams == 2 && TeamShape<8>::kTeams == 1 &&
+                  TeamShape<16>::kTeams == 1, "team shapes");
+static_assert(TeamShape<4>::kStepsPerWarp == 2 * TeamShape<4>::kStepsPerRound &&
+                  TeamShape<16>::kStepsPerWarp == 2 * TeamShape<16>::kStepsPerRound,
+              "two flush rounds");
+static_assert(tm_smem_bytes<16>() <= 227 * 1024 && 2 * tm_smem_bytes<8>() <= 228 * 1024 &&
+                  2 * tm_smem_bytes<4>() <= 228 * 1024,
+              "shared memory");
 
 // Barrier 1 + team over the team's warps (immediate ids, so that the kernel
 // reserves only the barriers it uses).
+template <int TW_>
 __device__ __forceinline__ void team_barrier(int team) {
-  static_assert(WARPS / TEAM == 2, "two teams");
-  if (team == 0)
-    asm volatile("bar.sync 1, %0;\n" ::"n"(32 * TEAM) : "memory");
-  else
-    asm volatile("bar.sync 2, %0;\n" ::"n"(32 * TEAM) : "memory");
+  if constexpr (TeamShape<TW_>::kTeams == 1) {
+    asm volatile("bar.sync 1, %0;\n" ::"n"(32 * TW_) : "memory");
+  } else {
+    static_assert(TeamShape<TW_>::kTeams == 2, "two teams");
+    if (team == 0)
+      asm volatile("bar.sync 1, %0;\n" ::"n"(32 * TW_) : "memory");
+    else
+      asm volatile("bar.sync 2, %0;\n" ::"n"(32 * TW_) : "memory");
+  }
 }
 
 // Float offset of time step tl's (channel 2k, 2k + 1) pair in a staging
@@ -398,18 +436,22 @@ __device__ __forceinline__ void stage_b_stage(const float *vb, const float2 *tap
   r4[1 - s] = make_float4(out[2].x, out[2].y, out[3].x, out[3].y);
 }
 
-// Warp k's quarter of a staged tile: time steps 32 k .. 32 k + 31, per round
-// 16 time steps x two 4-channel halves (lane pair = one 32-byte row of a
-// plane).  The half's channels are the pairs of regions 2 h and 2 h + 1.
-__device__ __forceinline__ void flush_quarter(const float *sb, float *__restrict__ hi,
-                                              float *__restrict__ lo, size_t obase, int C,
-                                              int t0, int T, int k, int lane) {
-  const int h = lane & 1;
+// Warp k's share of a staged tile: time steps kStepsPerWarp k .. + kStepsPerWarp
+// - 1, per round kStepsPerRound time steps x the group's 4-channel quarters
+// (kLanesPerStep lanes write one time step's row of a plane).  Quarter h's
+// channels are the pairs of regions 2 h and 2 h + 1.
+template <int TW_>
+__device__ __forceinline__ void flush_share(const float *sb, float *__restrict__ hi,
+                                            float *__restrict__ lo, size_t obase, int C, int t0,
+                                            int T, int k, int lane) {
+  using S = TeamShape<TW_>;
+  const int h = lane % S::kLanesPerStep;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {
-    const int tl = 32 * k + 16 * r + (lane >> 1), t = t0 + tl;
-    const float2 a = *reinterpret_cast<const float2 *>(sb + (2 * h) * RP + stg_index(tl));
-    const float2 c = *reinterpret_cast<const float2 *>(sb + (2 * h + 1) * RP + stg_index(tl));
+    const int tl = S::kStepsPerWarp * k + S::kStepsPerRound * r + lane / S::kLanesPerStep;
+    const int t = t0 + tl;
+    const float2 a = *reinterpret_cast<const float2 *>(sb + S::region(2 * h) + stg_index(tl));
+    const float2 c = *reinterpret_cast<const float2 *>(sb + S::region(2 * h + 1) + stg_index(tl));
     if (t < T) {
       const float v[4] = {a.x, a.y, c.x, c.y};
       float g[4];
@@ -428,8 +470,9 @@ __device__ __forceinline__ void flush_quarter(const float *sb, float *__restrict
 // TM = true: each team owns a range of (8-channel group, tile) tasks and
 // warp k walks row pair 4 group + k of them, writing the hi/lo planes
 // [B, T, C] (y = hi).  NX input windows per warp: the copies of the next
-// NX - 1 tiles are in flight while a tile is computed.
-template <bool TM, int NX>
+// NX - 1 tiles are in flight while a tile is computed.  TW_: warps per team
+// (TM), which also fixes the CTA's warps (TeamShape).
+template <bool TM, int NX, int TW_ = 4>
 __device__ __forceinline__ void activation_walk(
     const float *__restrict__ x, float *__restrict__ y, float *__restrict__ lo, int rows, int C,
     int T, int tiles_per_row, long long n_ids, const float *__restrict__ log_alpha,
@@ -458,22 +501,24 @@ __device__ __forceinline__ void activation_walk(
   float *wsm = smem + (size_t)warp * WF;
   float *const xs0 = wsm, *const vs0 = wsm + NX * XS_FLOATS;  // buffer b at + b * size
   float2 *cst = reinterpret_cast<float2 *>(wsm + NX * XS_FLOATS + 2 * VS_FLOATS);
-  const int team = warp / TEAM, k = warp % TEAM;
-  float *const stg = smem + (size_t)WARPS * WF + (size_t)team * 2 * STG_FLOATS;
+  using S = TeamShape<TW_>;
+  constexpr int CTA_WARPS = TM ? S::kCtaWarps : WARPS;
+  const int team = warp / S::kWarps, k = warp % S::kWarps;
+  float *const stg = smem + (size_t)CTA_WARPS * WF + (size_t)team * 2 * S::kStgFloats;
 
   // this warp's (or team's) contiguous range of ids (row pair or group) *
   // tiles_per_row + tile
-  const long long nw = (long long)gridDim.x * (TM ? WARPS / TEAM : WARPS);
-  const long long gw = (long long)blockIdx.x * (TM ? WARPS / TEAM : WARPS) + (TM ? team : warp);
+  const long long nw = (long long)gridDim.x * (TM ? S::kTeams : WARPS);
+  const long long gw = (long long)blockIdx.x * (TM ? S::kTeams : WARPS) + (TM ? team : warp);
   const long long beg = gw * n_ids / nw, end = (gw + 1) * n_ids / nw;
   if (beg >= end) return;
   auto row_ptr = [&](int pr, int which) {
     const int r = 2 * pr + which;
     return x + (size_t)(r < rows ? r : rows - 1) * T;
   };
-  constexpr int kStep = TM ? TEAM : 1;  // row pairs from one id row to the next
+  constexpr int kStep = TM ? S::kWarps : 1;  // row pairs from one id row to the next
   int pair = (int)(beg / tiles_per_row), tile = (int)(beg % tiles_per_row);
-  if (TM) pair = TEAM * pair + k;
+  if (TM) pair = S::kWarps * pair + k;
   // (fpair, ftile): the tile of id fid = id + NX - 1, whose copies the
   // iteration of id issues; the prologue issues ids beg .. beg + NX - 2
   int fpair = pair, ftile = tile;
@@ -500,11 +545,11 @@ __device__ __forceinline__ void activation_walk(
   int n_out = 0;     // TM: staged tiles so far (selects the staging buffer)
   auto emit = [&](const float *vsrc, int t_out) {
     if constexpr (TM) {
-      float *sb = stg + (n_out & 1) * STG_FLOATS;
+      float *sb = stg + (n_out & 1) * S::kStgFloats;
       ++n_out;
-      stage_b_stage(vsrc, taps, sb + k * RP, lane);
-      team_barrier(team);
-      flush_quarter(sb, y, lo, obase, C, t_out, T, k, lane);
+      stage_b_stage(vsrc, taps, sb + S::region(k), lane);
+      team_barrier<TW_>(team);
+      flush_share<TW_>(sb, y, lo, obase, C, t_out, T, k, lane);
     } else {
       stage_b(vsrc, taps, y + (size_t)(2 * pair) * T, 2 * pair + 1 < rows, t_out, T, lane);
     }
@@ -613,13 +658,17 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
                                 log_beta, f_up, f_dn, eps);
 }
 
-__global__ void __launch_bounds__(THREADS, 2)
+// TW_ = 4: two 4-warp teams per CTA, two CTAs per SM; TW_ = 8: one 8-warp team
+// per CTA, two CTAs per SM; TW_ = 16: one 16-warp team per CTA, one CTA per
+// SM.  Each way 16 warps per SM.
+template <int TW_>
+__global__ void __launch_bounds__(32 * TeamShape<TW_>::kCtaWarps, TW_ == 16 ? 1 : 2)
 activation_tm_kernel(const float *__restrict__ x, float *__restrict__ hi, float *__restrict__ lo,
                      int rows, int C, int T, int tiles_per_row, long long n_tasks,
                      const float *__restrict__ log_alpha, const float *__restrict__ log_beta,
                      const float *__restrict__ f_up, const float *__restrict__ f_dn, float eps) {
-  activation_walk<true, TM_NX>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha,
-                               log_beta, f_up, f_dn, eps);
+  activation_walk<true, TM_NX, TW_>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha,
+                                    log_beta, f_up, f_dn, eps);
 }
 
 __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restrict__ out,
@@ -651,6 +700,7 @@ int persistent_ctas() {
   return n;
 }
 
+template <int TW_>
 int persistent_ctas_tm() {
   constexpr int kMaxDev = 64;
   static std::atomic<int> cache[kMaxDev];
@@ -659,10 +709,11 @@ int persistent_ctas_tm() {
   const int slot = dev >= 0 && dev < kMaxDev ? dev : 0;
   int n = cache[slot].load(std::memory_order_relaxed);
   if (n == 0) {
-    int sms = 148, per_sm = 2;
+    int sms = 148, per_sm = 1;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, activation_tm_kernel, THREADS,
-                                                      TM_SMEM_BYTES) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &per_sm, activation_tm_kernel<TW_>, 32 * TeamShape<TW_>::kCtaWarps,
+            tm_smem_bytes<TW_>()) != cudaSuccess ||
         per_sm < 1)
       per_sm = 1;
     n = sms * per_sm;
@@ -671,35 +722,49 @@ int persistent_ctas_tm() {
   return n;
 }
 
+template <int TW_>
+bv_status run_activation_tm(const float *x, float *hi, float *lo, long long rows, int C, int T,
+                            const float *la, const float *lb, const float *fu, const float *fd,
+                            float eps, cudaStream_t st) {
+  using S = TeamShape<TW_>;
+  const int tiles = (T + TW - 1) / TW;
+  const long long n_tasks = rows / S::kCh * tiles;  // (group, tile) tasks
+  if (n_tasks <= 0) return BV_OK;
+  BV_TRY(ensure_dynamic_smem((const void *)activation_tm_kernel<TW_>, tm_smem_bytes<TW_>(),
+                             "activation_tm smem attribute"));
+  const long long ctas = persistent_ctas_tm<TW_>();
+  const long long need = (n_tasks + S::kTeams - 1) / S::kTeams;
+  const long long grid = need < ctas ? need : ctas;
+  {
+    // algorithmic bytes: read x (4 B), write the hi and lo planes (8 B)
+    LaunchTimer tm(st, "activation_tm", 0.0, 12.0 * (double)rows * T);
+    activation_tm_kernel<TW_><<<(unsigned)grid, 32 * S::kCtaWarps, tm_smem_bytes<TW_>(), st>>>(
+        x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb, fu, fd, eps);
+  }
+  count_launch();
+  return check_launch("activation_tm_kernel");
+}
+
 }  // namespace
 
-bool activation_tm_supported(int C) { return C % TM_CH == 0; }
+bool activation_tm_supported(int C) { return C % TeamShape<4>::kCh == 0; }
 
 bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int C, int T,
                                const float *la, const float *lb, const float *fu, const float *fd,
                                float eps, cudaStream_t st) {
   if (!activation_tm_supported(C))
-    return fail(BV_ERR_UNSUPPORTED, "activation_tm: C = %d is not a multiple of %d", C, TM_CH);
+    return fail(BV_ERR_UNSUPPORTED, "activation_tm: C = %d is not a multiple of %d", C,
+                TeamShape<4>::kCh);
   if (((reinterpret_cast<uintptr_t>(hi) | reinterpret_cast<uintptr_t>(lo)) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "activation_tm: planes not 16-byte aligned");
   const long long rows = (long long)B * C;
   if (rows > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "activation_tm: too many rows");
-  const int tiles = (T + TW - 1) / TW;
-  const long long n_tasks = rows / TM_CH * tiles;  // (group, tile) tasks
-  if (n_tasks <= 0) return BV_OK;
-  BV_TRY(ensure_dynamic_smem((const void *)activation_tm_kernel, TM_SMEM_BYTES,
-                             "activation_tm smem attribute"));
-  const long long ctas = persistent_ctas_tm();
-  const long long need = (n_tasks + WARPS / TEAM - 1) / (WARPS / TEAM);
-  const long long grid = need < ctas ? need : ctas;
-  {
-    // algorithmic bytes: read x (4 B), write the hi and lo planes (8 B)
-    LaunchTimer tm(st, "activation_tm", 0.0, 12.0 * (double)rows * T);
-    activation_tm_kernel<<<(unsigned)grid, THREADS, TM_SMEM_BYTES, st>>>(
-        x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb, fu, fd, eps);
-  }
-  count_launch();
-  return check_launch("activation_tm_kernel");
+  // the widest plane rows per time step the channels allow
+  if (C % TeamShape<16>::kCh == 0)
+    return run_activation_tm<16>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
+  if (C % TeamShape<8>::kCh == 0)
+    return run_activation_tm<8>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
+  return run_activation_tm<4>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
 }
 
 bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream_t st) {

@@ -511,11 +511,12 @@ def test_full_size_conv_transpose_time_major_sampled(nat, oracle, Cin, Cout, S, 
 @pytest.mark.parametrize("B,C,T", [(2, 32, 1), (1, 32, 2), (2, 32, 129), (3, 48, 130),
                                    (2, 64, 257), (1, 32, 1000), (2, 96, 4099), (1, 56, 300)])
 def test_act_conv_time_major_activation_ragged(nat, oracle, filt, B, C, T):
-    """The activation writing the time-major planes (8-channel groups; 56
-    channels: seven groups, the conv's second 32-channel block zero-padded)
-    on ragged and tiny time axes (replicate padding at both ends of a tile),
-    odd batch counts and warps that own less than one channel group; every
-    output."""
+    """The activation writing the time-major planes, both team shapes (32,
+    64, 96 channels: 32-channel groups of one 16-warp team; 48 and 56: 8-channel
+    groups, 56 being seven groups with the conv's second 32-channel block
+    zero-padded) on ragged and tiny time axes (replicate padding at both ends
+    of a tile), odd batch counts and teams that own less than one channel
+    group; every output."""
     s = synth.NormalStream(13000 + B + C + T)
     x = s.normal((B, C, T), 0.0, 1.5)
     la, lb = s.normal((C,), 0.0, 0.3), s.normal((C,), 0.0, 0.3)
