@@ -636,14 +636,20 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
 // CTAs' bytes); one thread of the even CTA issues the MMAs and commits to
 // barriers in both CTAs; four warps per CTA add finished runs into FP32
 // registers and write that CTA's rows of the [B, Cout, T] output with the
-// usual epilogue.  A chunk is two taps of one channel block (24 MMAs), so the
-// per-chunk cost of a barrier wait and a commit in the issuing thread is
+// usual epilogue.  A chunk is TAPS taps of one channel block (12 TAPS MMAs), so
+// the per-chunk cost of a barrier wait and a commit in the issuing thread is
 // spread over twice the tensor work.
 constexpr int TM_MAX_HALO = 56;                       // (K - 1) d the x box can hold
 constexpr int TM_W_PLANE = (MAX_NT / 2) * BK * 4;     // 8 KB: one CTA's half of a weight plane
-constexpr int TM_W_SLOT = 2 * 2 * TM_W_PLANE;         // a chunk: two taps, hi and lo
+// A weight chunk holds TAPS taps (hi and lo planes each); runs are 4 taps of
+// 32 channels (128 kk) whatever the chunk size, so that the tensor core's
+// truncating accumulation stays as short as measured below.  Four-tap chunks
+// for convs of three or more taps (half the barrier waits and commits per
+// MMA: the [8, 384, 10006] K 7 layer 0.745 -> 0.661 ms); two-tap chunks, and
+// so a deeper ring, for shorter ones (the transposed convs' phase convs).
+__host__ __device__ constexpr int tm_w_slot(int taps) { return taps * 2 * TM_W_PLANE; }
+__host__ __device__ constexpr int tm_run(int taps) { return 4 / taps; }  // chunks per run
 constexpr int TM_MAX_WSLOTS = 6;
-constexpr int TM_RUN = 2;                              // chunks (up to 4 taps of 32) per run
 constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
 constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
 constexpr int TM_XSLOTS = 2;                          // x blocks in flight
@@ -659,15 +665,17 @@ static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
 __host__ __device__ constexpr int tm_x_plane(int rows) { return (rows * 128 + 1023) / 1024 * 1024; }
-// Weight ring slots that fit beside the x slots of `rows` rows.
-__host__ __device__ constexpr int tm_w_slots(int rows) {
-  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / TM_W_SLOT <
+// Weight ring slots of `taps`-tap chunks that fit beside the x slots of
+// `rows` rows.
+__host__ __device__ constexpr int tm_w_slots(int rows, int taps) {
+  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / tm_w_slot(taps) <
                  TM_MAX_WSLOTS
-             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / TM_W_SLOT
+             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / tm_w_slot(taps)
              : TM_MAX_WSLOTS;
 }
-static_assert(tm_w_slots(BM + TM_MAX_HALO) >= 4, "weight ring depth");
-static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 4 * TM_W_SLOT + TM_NBARS * 8 <=
+static_assert(tm_w_slots(BM + TM_MAX_HALO, 2) >= 4 && tm_w_slots(BM + TM_MAX_HALO, 4) >= 2,
+              "weight ring depth");
+static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 2 * tm_w_slot(4) + TM_NBARS * 8 <=
                   TM_BUDGET,
               "shared memory layout");
 
@@ -753,7 +761,7 @@ __device__ __forceinline__ void mma_commit_pair(unsigned bar) {
       : "memory");
 }
 
-template <int NT>
+template <int NT, int TAPS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_xlo,
@@ -773,7 +781,9 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const bool leader = (rank == 0);
   const int xrows = BM + (K - 1) * dil;  // rows of one x box
   const int XP = tm_x_plane(xrows);
-  const int NW = tm_w_slots(xrows);
+  static_assert(TAPS == 2 || TAPS == 4, "taps per weight chunk");
+  constexpr int TM_W_SLOT = tm_w_slot(TAPS), TM_RUN = tm_run(TAPS);
+  const int NW = tm_w_slots(xrows, TAPS);
   const unsigned X_TX = 2u * 2u * (unsigned)xrows * 128u;  // both CTAs, hi and lo
   unsigned char *wbase = smem + 2 * TM_XSLOTS * XP;
   uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + NW * TM_W_SLOT);
@@ -816,7 +826,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   };
   const int n_cb = (Cin + BK - 1) / BK;  // 32-channel blocks (channels past Cin read as 0)
   const int Cpad = n_cb * BK;            // weight row stride per tap
-  const int n_tc = (K + 1) / 2;       // chunks per block: taps (0,1), (2,3), ...
+  const int n_tc = (K + TAPS - 1) / TAPS;  // chunks per block: taps 0 .. TAPS - 1, ...
   const int n_chunks = n_cb * n_tc;
   const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;  // per tile
   // a wait that runs out marks both CTAs of the pair aborted
@@ -896,7 +906,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
               ok = false;
               break;
             }
-            const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+            const int j0 = TAPS * q, ntap = (K - j0) < TAPS ? (K - j0) : TAPS;
             const unsigned fb = bar_wfull + 8 * ws;
             if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
             for (int t = 0; t < ntap; ++t) {
@@ -952,7 +962,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
             }
             asm volatile("tcgen05.fence::after_thread_sync;\n" ::: "memory");
             const unsigned acc = tmem + (unsigned)(ra * MAX_NT);
-            const int j0 = 2 * q, ntap = (K - j0) < 2 ? (K - j0) : 2;
+            const int j0 = TAPS * q, ntap = (K - j0) < TAPS ? (K - j0) : TAPS;
             for (int t = 0; t < ntap; ++t) {
               const uint64_t rows = (uint64_t)((j0 + t) * dil * 8);  // tap's first row, in 16 B
               const uint64_t ah = dxh + rows, al = dxl + rows;
@@ -1113,12 +1123,12 @@ int tm_pairs() {
   return n;
 }
 
-template <int NT>
+template <int NT, int TAPS>
 bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
                  int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
                  const OutMap &om, cudaStream_t st) {
-  BV_TRY(ensure_dynamic_smem((const void *)conv1d_tm_kernel<NT>, TM_SMEM_BYTES,
+  BV_TRY(ensure_dynamic_smem((const void *)conv1d_tm_kernel<NT, TAPS>, TM_SMEM_BYTES,
                              "conv1d_tm smem attribute"));
   // persistent: at most one CTA pair per two SMs, each walking its share of
   // the (time pair, output-channel tile, row-phase) tiles
@@ -1126,7 +1136,7 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
   const long long n_tiles = tpairs * ntiles * (long long)B * om.phases;
   if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "conv1d_tm: too many tiles");
   const long long pairs = std::min<long long>(n_tiles, tm_pairs());
-  conv1d_tm_kernel<NT><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
+  conv1d_tm_kernel<NT, TAPS><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
       xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
       device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
   return BV_OK;
@@ -1482,10 +1492,12 @@ bv_status tm_impl(const char *cls, const float *x_hi, const float *x_lo, int B, 
   bv_status s;
   {
     LaunchTimer tm(st, cls, flops, bytes);
-#define BV_TM_CASE(N)                                                                      \
-  case N:                                                                                  \
-    s = run_tm<N>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, \
-                  om, st);                                                                 \
+#define BV_TM_CASE(N)                                                                        \
+  case N:                                                                                    \
+    s = K >= 3 ? run_tm<N, 4>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, \
+                              y_pitch, om, st)                                               \
+               : run_tm<N, 2>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, \
+                              y_pitch, om, st);                                              \
     break;
     switch (nt) {
       BV_TM_CASE(64)
