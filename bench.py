@@ -269,10 +269,10 @@ TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpo
 # `traffic` is this ratio x the class's algorithmic bytes per launch.  A class
 # whose kernel code changed since its capture has no entry (traffic null).
 #   conv1d_tm: conv1d_tm_kernel, all 190 launches of one 60 s stereo decode
-#   (180 AMP convs + 10 transposed convs), 59.70 GB against 43.71 GB
-#   algorithmic (one ncu pass per launch); kernel code of commit 5eafb75
-#   (four run accumulators), unchanged since.
-NCU_TRAFFIC_RATIO = {"conv1d_tm": 1.366}
+#   (180 AMP convs + 10 transposed convs), 59.66 GB against 43.71 GB
+#   algorithmic (one ncu pass per launch); kernel code of commit 591c821
+#   (four-tap weight chunks), unchanged since.
+NCU_TRAFFIC_RATIO = {"conv1d_tm": 1.365}
 
 
 def traffic_for(name, kd):
