@@ -999,6 +999,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     const int ct = threadIdx.x - CONV_WARP0 * 32;  // time row of this thread
     const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
     const unsigned run_free_leader = map_to_rank(bar_run_free, 0);
+    constexpr int NG = NT / 16;                // 16-channel groups of a tile
+    constexpr int FOLD_G = NT < 128 ? 2 : 1;   // residual groups folded per run
     int gr = 0;  // runs read over all tiles
     bool alive = true;
     for (int tau = cid; tau < n_tiles && alive; tau += P) {
@@ -1015,10 +1017,12 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       float sum[NT];
 #pragma unroll
       for (int e = 0; e < NT; ++e) sum[e] = 0.0f;
-      // The residual of this thread's output row, 16 channels after each of
-      // the first NT / 16 runs: the loads overlap the wait for the next run
-      // instead of the output loop, and the values join the sum there
-      // ((conv + residual) + bias instead of (conv + bias) + residual).
+      // The residual of this thread's output row, FOLD_G groups of 16
+      // channels per run for the first runs: a run's loads are issued before
+      // its wait, so their latency hides behind it instead of the output loop,
+      // and the values join the sum after the run's arrive ((conv + residual)
+      // + bias instead of (conv + bias) + residual).  Narrow tiles have few
+      // runs per tile, so they fold two groups a run.
       const int t_out = tl.t0 + ct;
       const int p_out = om.stride * t_out + om.offset + tl.phase;  // output sample
       const bool in = t_out < y_len && p_out >= 0 && p_out < om.len;
@@ -1026,6 +1030,19 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       const bool fold = ep.residual != nullptr;
       for (int p = 0; p < n_runs; ++p, ++gr) {
         const int ra = gr & (TM_ACC - 1);
+        const bool fold_p = fold && in && p * FOLD_G < NG;
+        float r[16 * FOLD_G];
+        if (fold_p) {
+#pragma unroll
+          for (int j = 0; j < FOLD_G; ++j) {
+            const int g = p * FOLD_G + j;
+            const int valid = g < NG ? Cout - (tl.o0 + 16 * g) : 0;
+            const float *rp = ep.residual + base + (size_t)(tl.o0 + 16 * g) * y_pitch;
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              r[16 * j + e] = e < valid ? __ldg(rp + (size_t)e * y_pitch) : 0.0f;
+          }
+        }
         if (!warp_wait(bar_run_full + 8 * ra, (gr / TM_ACC) & 1, wc, 116)) {
           alive = false;
           break;
@@ -1056,18 +1073,15 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(run_free_leader + 8 * ra);
-        if (fold && in && p < NT / 16) {
-          const int valid = Cout - (tl.o0 + 16 * p);
-          const float *rp = ep.residual + base + (size_t)(tl.o0 + 16 * p) * y_pitch;
-          float r[16];
+        if (fold_p) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = e < valid ? __ldg(rp + (size_t)e * y_pitch) : 0.0f;
+          for (int g = 0; g < NG; ++g)
 #pragma unroll
-          for (int g = 0; g < NT / 16; ++g)
-            if (g == p) {
+            for (int j = 0; j < FOLD_G; ++j)
+              if (g == p * FOLD_G + j) {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) sum[16 * g + e] += r[e];
-            }
+                for (int e = 0; e < 16; ++e) sum[16 * g + e] += r[16 * j + e];
+              }
         }
       }
       if (!alive || ctl.abort) break;
@@ -1079,7 +1093,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
         // 16 channels at a time: the group's reads, then its writes (without
         // the residual where it joined the sum above)
         Epi eg = ep;
-        if (fold && g / 16 < n_runs) eg.residual = nullptr;
+        if (fold && g / 16 < n_runs * FOLD_G) eg.residual = nullptr;
         if (in)
           epi_group<16>(sum + g, bb, eg, y, base + (size_t)(tl.o0 + g) * y_pitch, (size_t)y_pitch,
                         Cout - (tl.o0 + g));
