@@ -97,9 +97,12 @@ struct Epi {
 // between stores to y -- a plain load, or even a read-only bias load -- waited
 // a full memory round trip each, which made the output loop of a tensor-core
 // conv tile several times longer than its stores.)
+// epi_values computes the group's outputs into out (entries past `valid`
+// undefined); epi_group also writes them.
 template <int N>
-__device__ __forceinline__ void epi_group(float *v, const float (&bias)[N], const Epi &e,
-                                          float *y, size_t idx0, size_t stride, int valid) {
+__device__ __forceinline__ void epi_values(const float *v, const float (&bias)[N], const Epi &e,
+                                           const float *y, size_t idx0, size_t stride, int valid,
+                                           float (&out)[N]) {
   float r[N], a[N];
   if (e.residual || e.accumulate) {
 #pragma unroll
@@ -113,13 +116,20 @@ __device__ __forceinline__ void epi_group(float *v, const float (&bias)[N], cons
   }
 #pragma unroll
   for (int q = 0; q < N; ++q) {
-    if (q < valid) {
-      float t = (v[q] + bias[q] + r[q]) * e.scale + a[q];
-      if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
-      else if (e.final_act == 2) t = tanhf(t);
-      y[idx0 + q * stride] = t;
-    }
+    float t = (v[q] + bias[q] + r[q]) * e.scale + a[q];
+    if (e.final_act == 1) t = fminf(fmaxf(t, -1.0f), 1.0f);
+    else if (e.final_act == 2) t = tanhf(t);
+    out[q] = t;
   }
+}
+template <int N>
+__device__ __forceinline__ void epi_group(float *v, const float (&bias)[N], const Epi &e,
+                                          float *y, size_t idx0, size_t stride, int valid) {
+  float t[N];
+  epi_values<N>(v, bias, e, y, idx0, stride, valid, t);
+#pragma unroll
+  for (int q = 0; q < N; ++q)
+    if (q < valid) y[idx0 + q * stride] = t[q];
 }
 
 // Two-phase form for a thread that owns many outputs: epi_load folds in

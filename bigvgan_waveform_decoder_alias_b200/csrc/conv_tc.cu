@@ -35,6 +35,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -640,14 +641,16 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
 // the per-chunk cost of a barrier wait and a commit in the issuing thread is
 // spread over twice the tensor work.
 constexpr int TM_MAX_HALO = 56;                       // (K - 1) d the x box can hold
-constexpr int TM_W_PLANE = (MAX_NT / 2) * BK * 4;     // 8 KB: one CTA's half of a weight plane
+// One CTA's half of a weight plane of an NT-channel tile: NT / 2 rows of 32
+// channels (8 KB at NT = 128).
+__host__ __device__ constexpr int tm_w_plane(int nt) { return (nt / 2) * BK * 4; }
 // A weight chunk holds TAPS taps (hi and lo planes each); runs are 4 taps of
 // 32 channels (128 kk) whatever the chunk size, so that the tensor core's
 // truncating accumulation stays as short as measured below.  Four-tap chunks
 // for convs of three or more taps (half the barrier waits and commits per
 // MMA: the [8, 384, 10006] K 7 layer 0.745 -> 0.661 ms); two-tap chunks, and
 // so a deeper ring, for shorter ones (the transposed convs' phase convs).
-__host__ __device__ constexpr int tm_w_slot(int taps) { return taps * 2 * TM_W_PLANE; }
+__host__ __device__ constexpr int tm_w_slot(int taps, int nt) { return taps * 2 * tm_w_plane(nt); }
 __host__ __device__ constexpr int tm_run(int taps) { return 4 / taps; }  // chunks per run
 constexpr int TM_MAX_WSLOTS = 6;
 constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
@@ -663,21 +666,35 @@ static_assert(TM_TMEM_COLS <= 512 && (TM_ACC & (TM_ACC - 1)) == 0, "TMEM accumul
 constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC + 1;
 static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
+// Output staging for the bulk-tensor stores of the output loop: per sum
+// warp two buffers of 16 channels x 32 time steps.
+constexpr int TM_STG_BUF = 16 * 32 * 4;
+constexpr int TM_STG_BYTES = (NCONV / 32) * 2 * TM_STG_BUF;  // 16 KB
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
 __host__ __device__ constexpr int tm_x_plane(int rows) { return (rows * 128 + 1023) / 1024 * 1024; }
-// Weight ring slots of `taps`-tap chunks that fit beside the x slots of
-// `rows` rows.
-__host__ __device__ constexpr int tm_w_slots(int rows, int taps) {
-  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / tm_w_slot(taps) <
+// Weight ring slots of `taps`-tap chunks of an NT-channel tile that fit
+// beside the x slots of `rows` rows and `stg` bytes of output staging.
+__host__ __device__ constexpr int tm_w_slots(int rows, int taps, int nt, int stg) {
+  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows) - stg) /
+                     tm_w_slot(taps, nt) <
                  TM_MAX_WSLOTS
-             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows)) / tm_w_slot(taps)
+             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows) - stg) /
+                   tm_w_slot(taps, nt)
              : TM_MAX_WSLOTS;
 }
-static_assert(tm_w_slots(BM + TM_MAX_HALO, 2) >= 4 && tm_w_slots(BM + TM_MAX_HALO, 4) >= 2,
+// The ring depth the issuer needs: two four-tap or four two-tap chunks.
+__host__ __device__ constexpr int tm_min_wslots(int taps) { return taps == 4 ? 2 : 4; }
+static_assert(tm_w_slots(BM + TM_MAX_HALO, 2, MAX_NT, 0) >= tm_min_wslots(2) &&
+                  tm_w_slots(BM + TM_MAX_HALO, 4, MAX_NT, 0) >= tm_min_wslots(4),
               "weight ring depth");
-static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 2 * tm_w_slot(4) + TM_NBARS * 8 <=
+static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 2 * tm_w_slot(4, MAX_NT) +
+                      TM_NBARS * 8 <=
                   TM_BUDGET,
               "shared memory layout");
+// Below 128 channels the staging always fits beside a full ring.
+static_assert(tm_w_slots(BM + TM_MAX_HALO, 4, 96, TM_STG_BYTES) >= tm_min_wslots(4) &&
+                  tm_w_slots(BM + TM_MAX_HALO, 2, 96, TM_STG_BYTES) >= tm_min_wslots(2),
+              "ring depth with output staging");
 
 // Instruction descriptor for the pair: D f32, A and B tf32, K-major, M = 256.
 __host__ __device__ constexpr uint32_t make_idesc_pair(int nt) {
@@ -761,12 +778,40 @@ __device__ __forceinline__ void mma_commit_pair(unsigned bar) {
       : "memory");
 }
 
-template <int NT, int TAPS>
+// Bulk-tensor store of a staged box (this CTA's shared memory -> global),
+// tracked per thread in bulk groups.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap *map, unsigned src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];\n" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(src)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;\n" ::: "memory");
+}
+// At most N of this thread's bulk groups still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;\n" ::"n"(N) : "memory");
+}
+// Every bulk group of this thread complete (its writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;\n" ::: "memory");
+}
+// Generic-proxy writes to shared memory made visible to the bulk copies.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
+}
+
+template <int NT, int TAPS, bool STG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_xlo,
                  const __grid_constant__ CUtensorMap tmap_whi,
-                 const __grid_constant__ CUtensorMap tmap_wlo, const float *__restrict__ bias,
+                 const __grid_constant__ CUtensorMap tmap_wlo,
+                 const __grid_constant__ CUtensorMap tmap_y, const float *__restrict__ bias,
                  float *y, int Cin, int Cout, int K, int dil, int pad, int y_len, int y_pitch,
                  Epi ep, OutMap om, int *status, long long wait_limit, int tpairs, int ntiles,
                  int n_tiles) {
@@ -782,11 +827,17 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const int xrows = BM + (K - 1) * dil;  // rows of one x box
   const int XP = tm_x_plane(xrows);
   static_assert(TAPS == 2 || TAPS == 4, "taps per weight chunk");
-  constexpr int TM_W_SLOT = tm_w_slot(TAPS), TM_RUN = tm_run(TAPS);
-  const int NW = tm_w_slots(xrows, TAPS);
+  constexpr int TM_W_PLANE = tm_w_plane(NT);
+  constexpr int TM_W_SLOT = tm_w_slot(TAPS, NT), TM_RUN = tm_run(TAPS);
+  // STG: the output loop stages each 16-channel group in shared memory and
+  // writes it with one bulk-tensor store through tmap_y (plain [B, Cout,
+  // y_pitch] outputs whose rows start on 16 bytes; the launcher checked that
+  // the staging leaves the ring its depth)
+  const int NW = tm_w_slots(xrows, TAPS, NT, STG ? TM_STG_BYTES : 0);
   const unsigned X_TX = 2u * 2u * (unsigned)xrows * 128u;  // both CTAs, hi and lo
   unsigned char *wbase = smem + 2 * TM_XSLOTS * XP;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(wbase + NW * TM_W_SLOT);
+  unsigned char *stg_base = wbase + NW * TM_W_SLOT;  // 1024-byte aligned
+  uint64_t *bars = reinterpret_cast<uint64_t *>(stg_base + (STG ? TM_STG_BYTES : 0));
   // barriers (the leader's full and run-free barriers serve the pair):
   // x block loaded / consumed (TM_XSLOTS), weight chunk loaded / consumed
   // (NW slots), run accumulated / run accumulator read (2), every MMA done
@@ -1001,7 +1052,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     const unsigned run_free_leader = map_to_rank(bar_run_free, 0);
     constexpr int NG = NT / 16;                // 16-channel groups of a tile
     constexpr int FOLD_G = NT < 128 ? 2 : 1;   // residual groups folded per run
-    int gr = 0;  // runs read over all tiles
+    int gr = 0;   // runs read over all tiles
+    int sgi = 0;  // staged output groups of this warp over all tiles
     bool alive = true;
     for (int tau = cid; tau < n_tiles && alive; tau += P) {
       const Tile tl = tile_of(tau);
@@ -1094,11 +1146,36 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
         // the residual where it joined the sum above)
         Epi eg = ep;
         if (fold && g / 16 < n_runs * FOLD_G) eg.residual = nullptr;
-        if (in)
-          epi_group<16>(sum + g, bb, eg, y, base + (size_t)(tl.o0 + g) * y_pitch, (size_t)y_pitch,
-                        Cout - (tl.o0 + g));
+        const size_t idx0 = base + (size_t)(tl.o0 + g) * y_pitch;
+        if constexpr (STG) {
+          // staged: the warp's 32 time steps x 16 channels go out in one
+          // bulk store, which clips rows past y_len and channels past Cout
+          float val[16];
+          if (in) epi_values<16>(sum + g, bb, eg, y, idx0, (size_t)y_pitch, Cout - (tl.o0 + g), val);
+          if (tl.o0 + g < Cout && tl.t0 + 32 * q < y_len) {  // warp-uniform
+            float *sb = reinterpret_cast<float *>(stg_base + (2 * q + (sgi & 1)) * TM_STG_BUF);
+            if (sgi >= 2) {  // the store that read this buffer two groups ago is done
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) sb[32 * e + lane] = val[e];
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmap_y, smem_u32(sb), tl.t0 + 32 * q, tl.o0 + g, tl.b);
+              bulk_commit();
+            }
+            ++sgi;
+          }
+        } else if (in) {
+          epi_group<16>(sum + g, bb, eg, y, idx0, (size_t)y_pitch, Cout - (tl.o0 + g));
+        }
       }
     }
+    // the staged stores have written y before the kernel can end
+    if (STG && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
@@ -1137,22 +1214,53 @@ int tm_pairs() {
   return n;
 }
 
+// Output tensor map for the staged output loop: y as [B, Cout, y_pitch]
+// with y_len valid time steps, box 32 time steps x 16 channels.  Returns
+// false (no staging) where the rows do not start on 16 bytes.
+bool encode_y_tm(CUtensorMap *tmap, float *y, int B, int Cout, int y_len, int y_pitch) {
+  if ((reinterpret_cast<uintptr_t>(y) & 15u) != 0 || y_pitch % 4 != 0 || y_len > y_pitch)
+    return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)y_len, (cuuint64_t)Cout, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)y_pitch * sizeof(float),
+                                 (cuuint64_t)y_pitch * Cout * sizeof(float)};
+  const cuuint32_t box[3] = {32, 16, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y, dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                     CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NT, int TAPS>
 bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
                  int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
                  const OutMap &om, cudaStream_t st) {
-  BV_TRY(ensure_dynamic_smem((const void *)conv1d_tm_kernel<NT, TAPS>, TM_SMEM_BYTES,
-                             "conv1d_tm smem attribute"));
+  // Staged output loop for plain outputs (not the transposed convs' phase
+  // interleave) when the staging leaves the weight ring its depth.
+  CUtensorMap ym;
+  const bool plain = om.stride == 1 && om.offset == 0 && om.phases == 1 && om.len == y_len;
+  const bool stg = plain &&
+                   tm_w_slots(BM + (K - 1) * dil, TAPS, NT, TM_STG_BYTES) >= tm_min_wslots(TAPS) &&
+                   encode_y_tm(&ym, y, B, Cout, y_len, y_pitch);
+  if (!stg) std::memset(&ym, 0, sizeof(ym));
+  const void *kern = stg ? (const void *)conv1d_tm_kernel<NT, TAPS, true>
+                         : (const void *)conv1d_tm_kernel<NT, TAPS, false>;
+  BV_TRY(ensure_dynamic_smem(kern, TM_SMEM_BYTES, "conv1d_tm smem attribute"));
   // persistent: at most one CTA pair per two SMs, each walking its share of
   // the (time pair, output-channel tile, row-phase) tiles
   const long long tpairs = (y_len + 2 * BM - 1) / (2 * BM), ntiles = (Cout + NT - 1) / NT;
   const long long n_tiles = tpairs * ntiles * (long long)B * om.phases;
   if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "conv1d_tm: too many tiles");
   const long long pairs = std::min<long long>(n_tiles, tm_pairs());
-  conv1d_tm_kernel<NT, TAPS><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
-      xh, xl, wh, wl, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
-      device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
+  if (stg)
+    conv1d_tm_kernel<NT, TAPS, true><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
+        xh, xl, wh, wl, ym, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
+        device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
+  else
+    conv1d_tm_kernel<NT, TAPS, false><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
+        xh, xl, wh, wl, ym, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
+        device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
   return BV_OK;
 }
 

@@ -536,12 +536,16 @@ def test_act_conv_time_major_activation_ragged(nat, oracle, filt, B, C, T):
 
 
 @pytest.mark.parametrize("C,T,K,d", [(64, 777, 7, 3), (128, 300, 3, 1), (24, 513, 11, 5),
-                                     (100, 257, 5, 2), (96, 1000, 1, 1), (64, 515, 1, 1)])
+                                     (100, 257, 5, 2), (96, 1000, 1, 1), (64, 515, 1, 1),
+                                     (128, 1000, 11, 5), (48, 516, 3, 1)])
 def test_act_conv_small_shapes_every_element(nat, oracle, filt, C, T, K, d):
     """bv_act_conv1d on every path (time-major with the fused activation for
     64 / 96 / 128 channels, one-tap convs included, time-major through a
     separate transpose for 100, the narrow FP32 kernel for 24), every output
-    against the oracle."""
+    against the oracle.  Rows of a multiple of 4 time steps take the staged
+    bulk-store output loop (48 channels: a 16-channel group past Cout; 516:
+    a last time tile of 4 steps), except where the staging does not fit beside
+    the weight ring (128 channels, K 11, dilation 5)."""
     s = synth.NormalStream(12000 + C + T)
     x = s.normal((2, C, T))
     la, lb = s.normal((C,), 0.0, 0.2), s.normal((C,), 0.0, 0.2)
@@ -580,7 +584,7 @@ AMP_SHAPES = [(12, 3001, 11, (1, 3, 5), False), (96, 517, 7, (1, 3, 5), True),
               (130, 64, 3, (2,), False), (16, 5, 7, (1, 3, 5, 7), False),
               (128, 2001, 11, (1, 3, 5), True), (48, 1003, 7, (1, 3, 5), True),
               (64, 300, 3, (1, 3, 5), True), (256, 130, 11, (5,), True),
-              (24, 700, 11, (1, 3, 5), False)]
+              (24, 700, 11, (1, 3, 5), False), (96, 516, 7, (1, 3, 5), True)]
 
 
 @pytest.mark.parametrize("tensor_core", [False, True])
