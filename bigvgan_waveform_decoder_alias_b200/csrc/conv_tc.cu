@@ -645,17 +645,24 @@ constexpr int TM_MAX_HALO = 56;                       // (K - 1) d the x box can
 // channels (8 KB at NT = 128).
 __host__ __device__ constexpr int tm_w_plane(int nt) { return (nt / 2) * BK * 4; }
 // A weight chunk holds TAPS taps (hi and lo planes each); runs are 4 taps of
-// 32 channels (128 kk) whatever the chunk size, so that the tensor core's
-// truncating accumulation stays as short as measured below.  Four-tap chunks
+// 32 channels (128 kk) at 128 channels, 8 taps (256 kk) for narrower tiles,
+// whatever the chunk size, so that the tensor core's truncating accumulation
+// stays short (measured below).  Four-tap chunks
 // for convs of three or more taps (half the barrier waits and commits per
 // MMA: the [8, 384, 10006] K 7 layer 0.745 -> 0.661 ms); two-tap chunks, and
 // so a deeper ring, for shorter ones (the transposed convs' phase convs).
 __host__ __device__ constexpr int tm_w_slot(int taps, int nt) { return taps * 2 * tm_w_plane(nt); }
-__host__ __device__ constexpr int tm_run(int taps) { return 4 / taps; }  // chunks per run
+// Chunks per run: 128 kk at 128 channels; 256 kk for narrower tiles, whose
+// runs are short against the sum warps' fixed cost per run (TMEM reads, the
+// arrive).
+__host__ __device__ constexpr int tm_run(int taps, int nt) { return (nt < MAX_NT ? 8 : 4) / taps; }
 constexpr int TM_MAX_WSLOTS = 6;
 constexpr int TM_BUDGET = 225 * 1024;                 // operand rings + barriers
 constexpr int TM_SMEM_BYTES = TM_BUDGET + 1024;       // room to align the base
-constexpr int TM_XSLOTS = 2;                          // x blocks in flight
+// x blocks in flight: two for 128-channel tiles (their weight chunks fill the
+// rest), up to four for narrower tiles, whose few chunks per tile leave the
+// x stream only a block or two of lead with two.
+constexpr int TM_MAX_XSLOTS = 4;
 // Run accumulators in TMEM (MAX_NT columns each; all 512 columns: the kernel
 // is alone on its SM, its shared memory leaves room for no other CTA).  With
 // four the issuer can run three runs ahead of the sum warps, which covers a
@@ -663,7 +670,7 @@ constexpr int TM_XSLOTS = 2;                          // x blocks in flight
 constexpr int TM_ACC = 4;
 constexpr int TM_TMEM_COLS = TM_ACC * MAX_NT;
 static_assert(TM_TMEM_COLS <= 512 && (TM_ACC & (TM_ACC - 1)) == 0, "TMEM accumulators");
-constexpr int TM_NBARS = 2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC + 1;
+constexpr int TM_NBARS = 2 * TM_MAX_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC + 1;
 static_assert(TM_SMEM_BYTES + 1024 <= 227 * 1024, "shared memory budget");
 
 // Output staging for the bulk-tensor stores of the output loop: per sum
@@ -673,27 +680,31 @@ constexpr int TM_STG_BYTES = (NCONV / 32) * 2 * TM_STG_BUF;  // 16 KB
 // Bytes of one x plane slot for `rows` rows (whole 1024-byte swizzle atoms).
 __host__ __device__ constexpr int tm_x_plane(int rows) { return (rows * 128 + 1023) / 1024 * 1024; }
 // Weight ring slots of `taps`-tap chunks of an NT-channel tile that fit
-// beside the x slots of `rows` rows and `stg` bytes of output staging.
-__host__ __device__ constexpr int tm_w_slots(int rows, int taps, int nt, int stg) {
-  return (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows) - stg) /
-                     tm_w_slot(taps, nt) <
+// beside xs x slots of `rows` rows and `stg` bytes of output staging.
+__host__ __device__ constexpr int tm_w_slots(int rows, int taps, int nt, int stg, int xs) {
+  return (TM_BUDGET - TM_NBARS * 8 - 2 * xs * tm_x_plane(rows) - stg) / tm_w_slot(taps, nt) <
                  TM_MAX_WSLOTS
-             ? (TM_BUDGET - TM_NBARS * 8 - 2 * TM_XSLOTS * tm_x_plane(rows) - stg) /
-                   tm_w_slot(taps, nt)
+             ? (TM_BUDGET - TM_NBARS * 8 - 2 * xs * tm_x_plane(rows) - stg) / tm_w_slot(taps, nt)
              : TM_MAX_WSLOTS;
 }
 // The ring depth the issuer needs: two four-tap or four two-tap chunks.
 __host__ __device__ constexpr int tm_min_wslots(int taps) { return taps == 4 ? 2 : 4; }
-static_assert(tm_w_slots(BM + TM_MAX_HALO, 2, MAX_NT, 0) >= tm_min_wslots(2) &&
-                  tm_w_slots(BM + TM_MAX_HALO, 4, MAX_NT, 0) >= tm_min_wslots(4),
+// x slots of the layout: two at 128 channels, else the most (up to four) that
+// leave the weight ring its depth.
+__host__ __device__ constexpr int tm_x_slots(int rows, int taps, int nt, int stg) {
+  return nt < MAX_NT && tm_w_slots(rows, taps, nt, stg, 4) >= tm_min_wslots(taps)   ? 4
+         : nt < MAX_NT && tm_w_slots(rows, taps, nt, stg, 3) >= tm_min_wslots(taps) ? 3
+                                                                                     : 2;
+}
+static_assert(tm_w_slots(BM + TM_MAX_HALO, 2, MAX_NT, 0, 2) >= tm_min_wslots(2) &&
+                  tm_w_slots(BM + TM_MAX_HALO, 4, MAX_NT, 0, 2) >= tm_min_wslots(4),
               "weight ring depth");
-static_assert(2 * TM_XSLOTS * tm_x_plane(BM + TM_MAX_HALO) + 2 * tm_w_slot(4, MAX_NT) +
-                      TM_NBARS * 8 <=
+static_assert(2 * 2 * tm_x_plane(BM + TM_MAX_HALO) + 2 * tm_w_slot(4, MAX_NT) + TM_NBARS * 8 <=
                   TM_BUDGET,
               "shared memory layout");
 // Below 128 channels the staging always fits beside a full ring.
-static_assert(tm_w_slots(BM + TM_MAX_HALO, 4, 96, TM_STG_BYTES) >= tm_min_wslots(4) &&
-                  tm_w_slots(BM + TM_MAX_HALO, 2, 96, TM_STG_BYTES) >= tm_min_wslots(2),
+static_assert(tm_w_slots(BM + TM_MAX_HALO, 4, 96, TM_STG_BYTES, 2) >= tm_min_wslots(4) &&
+                  tm_w_slots(BM + TM_MAX_HALO, 2, 96, TM_STG_BYTES, 2) >= tm_min_wslots(2),
               "ring depth with output staging");
 
 // Instruction descriptor for the pair: D f32, A and B tf32, K-major, M = 256.
@@ -717,8 +728,14 @@ __device__ __forceinline__ unsigned map_to_rank(unsigned addr, unsigned rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// Relaxed: the arrive publishes no data of this thread's.  Its one use says
+// that this thread's TMEM reads of a run accumulator are complete
+// (tcgen05.wait::ld returned their values, then tcgen05.fence::before_thread_sync),
+// so the MMA issuer may overwrite it; a release would also wait for this
+// thread's outstanding global loads and stores (the residual prefetch, the
+// previous tile's output), about a thousand cycles per run.
 __device__ __forceinline__ void mbar_arrive_remote(unsigned cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr)
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];\n" ::"r"(cluster_addr)
                : "memory");
 }
 // TMA loads of the pair: the destination is this CTA's shared memory, the
@@ -828,26 +845,28 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   const int XP = tm_x_plane(xrows);
   static_assert(TAPS == 2 || TAPS == 4, "taps per weight chunk");
   constexpr int TM_W_PLANE = tm_w_plane(NT);
-  constexpr int TM_W_SLOT = tm_w_slot(TAPS, NT), TM_RUN = tm_run(TAPS);
+  constexpr int TM_W_SLOT = tm_w_slot(TAPS, NT), TM_RUN = tm_run(TAPS, NT);
   // STG: the output loop stages each 16-channel group in shared memory and
   // writes it with one bulk-tensor store through tmap_y (plain [B, Cout,
   // y_pitch] outputs whose rows start on 16 bytes; the launcher checked that
   // the staging leaves the ring its depth)
-  const int NW = tm_w_slots(xrows, TAPS, NT, STG ? TM_STG_BYTES : 0);
+  const int XS = tm_x_slots(xrows, TAPS, NT, STG ? TM_STG_BYTES : 0);
+  const int NW = tm_w_slots(xrows, TAPS, NT, STG ? TM_STG_BYTES : 0, XS);
   const unsigned X_TX = 2u * 2u * (unsigned)xrows * 128u;  // both CTAs, hi and lo
-  unsigned char *wbase = smem + 2 * TM_XSLOTS * XP;
+  unsigned char *wbase = smem + 2 * XS * XP;
   unsigned char *stg_base = wbase + NW * TM_W_SLOT;  // 1024-byte aligned
   uint64_t *bars = reinterpret_cast<uint64_t *>(stg_base + (STG ? TM_STG_BYTES : 0));
   // barriers (the leader's full and run-free barriers serve the pair):
-  // x block loaded / consumed (TM_XSLOTS), weight chunk loaded / consumed
+  // x block loaded / consumed (XS slots), weight chunk loaded / consumed
   // (NW slots), run accumulated / run accumulator read (2), every MMA done
   const unsigned bar_xfull = smem_u32(&bars[0]);
-  const unsigned bar_xempty = smem_u32(&bars[TM_XSLOTS]);
-  const unsigned bar_wfull = smem_u32(&bars[2 * TM_XSLOTS]);
-  const unsigned bar_wempty = smem_u32(&bars[2 * TM_XSLOTS + TM_MAX_WSLOTS]);
-  const unsigned bar_run_full = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS]);
-  const unsigned bar_run_free = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + TM_ACC]);
-  const unsigned bar_done = smem_u32(&bars[2 * TM_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC]);
+  const unsigned bar_xempty = smem_u32(&bars[TM_MAX_XSLOTS]);
+  const unsigned bar_wfull = smem_u32(&bars[2 * TM_MAX_XSLOTS]);
+  const unsigned bar_wempty = smem_u32(&bars[2 * TM_MAX_XSLOTS + TM_MAX_WSLOTS]);
+  const unsigned bar_run_full = smem_u32(&bars[2 * TM_MAX_XSLOTS + 2 * TM_MAX_WSLOTS]);
+  const unsigned bar_run_free =
+      smem_u32(&bars[2 * TM_MAX_XSLOTS + 2 * TM_MAX_WSLOTS + TM_ACC]);
+  const unsigned bar_done = smem_u32(&bars[2 * TM_MAX_XSLOTS + 2 * TM_MAX_WSLOTS + 2 * TM_ACC]);
   // x slot s, plane (0 hi, 1 lo); weight slot s, tap t of the chunk, plane
   auto x_at = [&](int slot, int plane) { return smem_u32(smem + (2 * slot + plane) * XP); };
   auto w_at = [&](int slot, int tap, int plane) {
@@ -886,7 +905,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
   if (threadIdx.x == 0) {
     ctl.abort = 0;
     mbar_init(bar_done, 1);
-    for (int s = 0; s < TM_XSLOTS; ++s) {
+    for (int s = 0; s < XS; ++s) {
       mbar_init(bar_xfull + 8 * s, 1);
       mbar_init(bar_xempty + 8 * s, 1);
     }
@@ -920,12 +939,11 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       // a failed wait stops the loads; a slot holds at most one load not yet
       // seen complete, the last one issued into it (gcb counts the blocks
       // issued over all tiles)
-      int gcb = 0;
+      int gcb = 0, xs = 0, xu = 0;  // slot xs of pass xu over the x ring
       bool ok = true;
       for (int tau = cid; tau < n_tiles && ok; tau += P) {
         const Tile tl = tile_of(tau);
         for (int cb = 0; cb < n_cb; ++cb) {
-          const int xs = gcb % TM_XSLOTS, xu = gcb / TM_XSLOTS;
           if (xu > 0 && !mbar_wait(bar_xempty + 8 * xs, (xu - 1) & 1, wc, 111)) {
             ok = false;
             break;
@@ -935,11 +953,15 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
           tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * BK, tl.t0 - pad, tl.b, fb);
           tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * BK, tl.t0 - pad, tl.b, fb);
           ++gcb;
+          if (++xs == XS) {
+            xs = 0;
+            ++xu;
+          }
         }
       }
       if (leader)
-        for (int c = gcb - TM_XSLOTS; c < gcb; ++c)
-          if (c >= 0) mbar_drain(bar_xfull + 8 * (c % TM_XSLOTS), (c / TM_XSLOTS) & 1);
+        for (int c = gcb - XS; c < gcb; ++c)
+          if (c >= 0) mbar_drain(bar_xfull + 8 * (c % XS), (c / XS) & 1);
     }
   } else if (warp == 0) {
     // ----------------------------------------------- TMA producer: weight chunks
@@ -985,17 +1007,16 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     if (leader && lane == 0) {
       // descriptors are formed once per operand tile and advanced by adding
       // the byte offset / 16 (the start-address field; shared addresses stay
-      // below 256 KB, so the field never carries).  gcb, gc, gr: x blocks,
-      // weight chunks and runs consumed over all tiles; a run never spans
-      // two tiles.
-      int gcb = 0, gr = 0, ws = 0;
-      unsigned wphase = 0;
+      // below 256 KB, so the field never carries).  xs / ws: the x and
+      // weight ring slots with their phases; gr: runs issued over all
+      // tiles (a run never spans two tiles).
+      int gr = 0, ws = 0, xs = 0;
+      unsigned wphase = 0, xphase = 0;
       bool ok = true;
       for (int tau = cid; tau < n_tiles && ok; tau += P) {
         int c = 0;  // chunk within the tile
-        for (int cb = 0; cb < n_cb && ok; ++cb, ++gcb) {
-          const int xs = gcb % TM_XSLOTS;
-          if (!mbar_wait(bar_xfull + 8 * xs, (gcb / TM_XSLOTS) & 1, wc, 113)) {
+        for (int cb = 0; cb < n_cb && ok; ++cb) {
+          if (!mbar_wait(bar_xfull + 8 * xs, xphase, wc, 113)) {
             ok = false;
             break;
           }
@@ -1039,6 +1060,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
               wphase ^= 1u;
             }
           }
+          if (++xs == XS) {
+            xs = 0;
+            xphase ^= 1u;
+          }
         }
       }
       // every MMA issued above has completed before TMEM can be freed
@@ -1051,7 +1076,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     const int q = warp - CONV_WARP0;                // TMEM lane quarter (= rows 32q..)
     const unsigned run_free_leader = map_to_rank(bar_run_free, 0);
     constexpr int NG = NT / 16;                // 16-channel groups of a tile
-    constexpr int FOLD_G = NT < 128 ? 2 : 1;   // residual groups folded per run
+    constexpr int FOLD_G = NT < MAX_NT ? 3 : 1;  // residual groups folded per run
     int gr = 0;   // runs read over all tiles
     int sgi = 0;  // staged output groups of this warp over all tiles
     bool alive = true;
@@ -1074,7 +1099,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
       // its wait, so their latency hides behind it instead of the output loop,
       // and the values join the sum after the run's arrive ((conv + residual)
       // + bias instead of (conv + bias) + residual).  Narrow tiles have few
-      // runs per tile, so they fold two groups a run.
+      // runs per tile, so they fold three groups a run.
       const int t_out = tl.t0 + ct;
       const int p_out = om.stride * t_out + om.offset + tl.phase;  // output sample
       const bool in = t_out < y_len && p_out >= 0 && p_out < om.len;
@@ -1241,7 +1266,7 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
   CUtensorMap ym;
   const bool plain = om.stride == 1 && om.offset == 0 && om.phases == 1 && om.len == y_len;
   const bool stg = plain &&
-                   tm_w_slots(BM + (K - 1) * dil, TAPS, NT, TM_STG_BYTES) >= tm_min_wslots(TAPS) &&
+                   tm_w_slots(BM + (K - 1) * dil, TAPS, NT, TM_STG_BYTES, 2) >= tm_min_wslots(TAPS) &&
                    encode_y_tm(&ym, y, B, Cout, y_len, y_pitch);
   if (!stg) std::memset(&ym, 0, sizeof(ym));
   const void *kern = stg ? (const void *)conv1d_tm_kernel<NT, TAPS, true>
