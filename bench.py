@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--cpu-sample-frames", type=int, default=40,
                     help="latent frames (one side) of the oracle's timed sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tf32-only", action="store_true",
+                    help="decode with every tensor-core conv in 3xTF32 (bv_decoder_config."
+                         "tf32_only); by default the AMP convs that qualify use the fp16 "
+                         "split and the line also reports the 3xTF32 decode")
     ap.add_argument("--case", default=None,
                     help="time one kernel on one shape instead of the decoder (for profiling): "
                          "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s | "
@@ -230,49 +234,55 @@ def peaks():
     return out
 
 
-def tensor_peak(pk, clocks):
-    """Useful 3xTF32 peak for a kernel timed inside a decode: the bf16 figure
-    x the nominal tf32/bf16 ratio / 3 products.  The burst figure applies when
-    the timed region ran at the maximum SM clock with no power capping; under
-    capping or a lower clock, the sustained figure scaled by the measured clock
-    over the clock the sustained figure was taken at.  Returns (peak, source,
-    burst peak).  The scaled figure never exceeds the burst figure: a clock
-    near the maximum with a brief power cap takes the burst peak."""
-    burst = pk["bf16"] * TF32_PER_BF16 / 3.0
+def tensor_peak(pk, clocks, f16=False):
+    """Useful peak of a split-precision conv timed inside a decode: the bf16
+    figure x the nominal ratio of the MMA kind to bf16 (tf32 1.1 / 2.25; fp16
+    1.0) / 3 products.  The burst figure applies when the timed region ran at
+    the maximum SM clock with no power capping; under capping or a lower
+    clock, the sustained figure scaled by the measured clock over the clock the
+    sustained figure was taken at.  Returns (peak, source, burst peak).  The
+    scaled figure never exceeds the burst figure: a clock near the maximum with
+    a brief power cap takes the burst peak."""
+    ratio = 1.0 if f16 else TF32_PER_BF16
+    kind = (f"fp16/bf16 1.0 / 3 (3xF16)" if f16 else
+            f"tf32/bf16 {TF32_PER_BF16:.3f} / 3 (3xTF32)")
+    burst = pk["bf16"] * ratio / 3.0
     m = (clocks or {}).get("sm_mhz")
     mx = (clocks or {}).get("sm_max_mhz") or pk["sm_max_mhz"]
     capped = "sw_power_cap" in (clocks or {}).get("reasons", [])
     if m is None:
-        return burst, f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s (no clock samples)", burst
+        return burst, f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x {kind} (no clock samples)", burst
     if not capped and m >= 0.97 * mx:
-        return burst, (f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x tf32/bf16 "
-                       f"{TF32_PER_BF16:.3f} / 3 (3xTF32); SM clock {m:.0f} of {mx:.0f} MHz, "
-                       f"no power cap"), burst
-    peak = pk["bf16_sustained"] * m / pk["sustained_mhz"] * TF32_PER_BF16 / 3.0
+        return burst, (f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x {kind}; "
+                       f"SM clock {m:.0f} of {mx:.0f} MHz, no power cap"), burst
+    peak = pk["bf16_sustained"] * m / pk["sustained_mhz"] * ratio / 3.0
     if peak >= burst:
-        return burst, (f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x tf32/bf16 "
-                       f"{TF32_PER_BF16:.3f} / 3 (3xTF32); SM clock {m:.0f} of {mx:.0f} MHz, "
+        return burst, (f"{pk['source']} bf16 burst {pk['bf16']} TFLOP/s x {kind}; "
+                       f"SM clock {m:.0f} of {mx:.0f} MHz, "
                        f"power cap {'seen' if capped else 'not seen'} (the sustained figure "
                        f"scaled to this clock would exceed the burst figure)"), burst
     return peak, (f"{pk['source']} bf16 sustained {pk['bf16_sustained']} TFLOP/s at "
-                  f"{pk['sustained_mhz']:.0f} MHz scaled to the measured {m:.0f} MHz, x tf32/bf16 "
-                  f"{TF32_PER_BF16:.3f} / 3 (3xTF32); power cap {'seen' if capped else 'not seen'}"), \
+                  f"{pk['sustained_mhz']:.0f} MHz scaled to the measured {m:.0f} MHz, x {kind}; "
+                  f"power cap {'seen' if capped else 'not seen'}"), \
         burst
 
 
-# kernel classes that run 3xTF32 on the tensor cores
-TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm")
+# kernel classes on the tensor cores: 3xTF32, and the fp16 split
+TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm",
+                  "conv1d_tm_f16")
+F16_CLASSES = ("conv1d_tm_f16",)
 
 # Measured DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) over
 # the algorithmic bytes, per kernel class, from one ncu capture of every launch
 # of the class's kernel in one decode of the default workload; the bench's
 # `traffic` is this ratio x the class's algorithmic bytes per launch.  A class
 # whose kernel code changed since its capture has no entry (traffic null).
-#   conv1d_tm: conv1d_tm_kernel, all 190 launches of one 60 s stereo decode
-#   (180 AMP convs + 10 transposed convs), 59.66 GB against 43.71 GB
-#   algorithmic (one ncu pass per launch); kernel code of commit 591c821
-#   (four-tap weight chunks), unchanged since.
-NCU_TRAFFIC_RATIO = {"conv1d_tm": 1.365}
+#   conv1d_tm_f16: the fp16-split conv1d_tm_kernel instances, all 180 AMP-conv
+#   launches of one 60 s stereo decode, 35.52 GB against 42.01 GB algorithmic
+#   (the algorithmic count takes the operand as 4 B per element; the two fp16
+#   planes are 2 + 2 B); one ncu pass per launch.  The 3xTF32 class's last
+#   capture predates the staged output loop: no entry.
+NCU_TRAFFIC_RATIO = {"conv1d_tm_f16": 0.846}
 
 
 def traffic_for(name, kd):
@@ -285,8 +295,8 @@ def roofline_for(name, kd, pk, clocks=None):
     launch / average launch time (CUDA events on the launching stream)."""
     t = kd["avg_launch_ms"] / 1000.0
     if name in TENSOR_CLASSES:
-        # useful FLOPs of the 3xTF32 conv; the tensor pipe issues 3 TF32 MMAs each
-        peak, src, burst = tensor_peak(pk, clocks)
+        # useful FLOPs of the split conv; the tensor pipe issues 3 MMAs each
+        peak, src, burst = tensor_peak(pk, clocks, f16=name in F16_CLASSES)
         ach = kd["flops"] / t / 1e12
         return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
                 "frac": ach / peak, "frac_of_burst": ach / burst,
@@ -518,7 +528,7 @@ def main():
     if rank > 0:  # each replica decodes its own latent
         z = synth.NormalStream(w.seed + 1000 * rank).normal(z.shape, w.input_mean, w.input_std)
     dec = native.Decoder(w.geometry, params, tile_frames=w.tile_frames,
-                         overlap_frames=w.overlap_frames, device=dev)
+                         overlap_frames=w.overlap_frames, device=dev, tf32_only=args.tf32_only)
     # model load: the tensor-core weights split and packed once
     # (bv_decoder_prepare); every step decodes its own latent in full
     dec.prepare()
@@ -560,6 +570,36 @@ def main():
     value = job_throughput(world, audio_per_step, ms_per_step)
     y_check = y.detach().float()
     finite = bool(torch.isfinite(y_check).all().item())
+
+    # ------------------- the same decode with every conv in 3xTF32, for scale
+    tf32 = None
+    if not args.tf32_only:
+        dec32 = native.Decoder(w.geometry, params, tile_frames=w.tile_frames,
+                               overlap_frames=w.overlap_frames, device=dev, tf32_only=True)
+        dec32.prepare()
+        y32 = torch.empty_like(y)
+        for _ in range(max(args.warmup, 3)):
+            dec32.decode(zd, y=y32, workspace=ws)
+        torch.cuda.synchronize()
+        ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier()
+        with ClockSampler(dev.index) as clk32:
+            for k in range(args.steps):
+                flush.fill_(float(k))
+                ev3[k][0].record(stream)
+                dec32.decode(zd, y=y32, workspace=ws)
+                ev3[k][1].record(stream)
+            torch.cuda.synchronize()
+        barrier()
+        ms32 = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev3), world, dev) / args.steps
+        # the two splits' outputs on the same latent (both against the oracle
+        # in the golden tests)
+        d = (y - y32).double()
+        tf32 = {"value": job_throughput(world, audio_per_step, ms32), "unit": UNIT,
+                "ms_per_step": ms32, "clocks": clk32.summary(),
+                "rel_l2_vs_default": float(d.norm() / y32.double().norm())}
+        del dec32, y32
 
     # -------------------------------------------- end to end through host memory
     zh = torch.from_numpy(z).pin_memory()
@@ -642,7 +682,11 @@ def main():
                        "audio_seconds_per_step": audio_per_step,
                        "sample_rate": w.geometry.sample_rate,
                        "l2": "flushed between steps (256 MiB write outside the timed events)",
-                       "weights": "resident, tf32 split and ConvT packing prepared once at load",
+                       "weights": "resident, split and ConvT packing prepared once at load",
+                       "conv_split": ("3xTF32 throughout" if args.tf32_only else
+                                      "fp16 split (3 products, fp32 accumulate) for the AMP "
+                                      "convs of 48+ channels in multiples of 8, 3xTF32 "
+                                      "elsewhere"),
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int(zh.numel() * 4),
@@ -655,6 +699,7 @@ def main():
             "clocks": clk.summary(),
             "clocks_profiled_pass": prof_clocks,
             "output_finite": finite,
+            "split_3xtf32": tf32,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -440,10 +440,10 @@ __device__ __forceinline__ void stage_b_stage(const float *vb, const float2 *tap
 // - 1, per round kStepsPerRound time steps x the group's 4-channel quarters
 // (kLanesPerStep lanes write one time step's row of a plane).  Quarter h's
 // channels are the pairs of regions 2 h and 2 h + 1.
-template <int TW_>
+template <int TW_, bool F16>
 __device__ __forceinline__ void flush_share(const float *sb, float *__restrict__ hi,
                                             float *__restrict__ lo, size_t obase, int C, int t0,
-                                            int T, int k, int lane) {
+                                            int T, int k, int lane, float &vmax) {
   using S = TeamShape<TW_>;
   const int h = lane % S::kLanesPerStep;
 #pragma unroll
@@ -454,13 +454,31 @@ __device__ __forceinline__ void flush_share(const float *sb, float *__restrict__
     const float2 c = *reinterpret_cast<const float2 *>(sb + S::region(2 * h + 1) + stg_index(tl));
     if (t < T) {
       const float v[4] = {a.x, a.y, c.x, c.y};
-      float g[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) g[q] = __uint_as_float(__float_as_uint(v[q]) & 0xFFFFE000u);
       const size_t o = obase + (size_t)t * C + 4 * h;
-      *reinterpret_cast<float4 *>(hi + o) = make_float4(g[0], g[1], g[2], g[3]);
-      *reinterpret_cast<float4 *>(lo + o) =
-          make_float4(v[0] - g[0], v[1] - g[1], v[2] - g[2], v[3] - g[3]);
+      if constexpr (F16) {
+        // fp16 planes: hi = fp16(v), lo = fp16(v - hi), four channels in 8 bytes
+        vmax = fmaxf(vmax, fmaxf(fmaxf(fabsf(v[0]), fabsf(v[1])), fmaxf(fabsf(v[2]), fabsf(v[3]))));
+        __half2 h2[2], l2[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          h2[q] = __floats2half2_rn(v[2 * q], v[2 * q + 1]);
+          const float2 back = __half22float2(h2[q]);
+          l2[q] = __floats2half2_rn(v[2 * q] - back.x, v[2 * q + 1] - back.y);
+        }
+        *reinterpret_cast<uint2 *>(reinterpret_cast<__half *>(hi) + o) =
+            make_uint2(*reinterpret_cast<const unsigned *>(&h2[0]),
+                       *reinterpret_cast<const unsigned *>(&h2[1]));
+        *reinterpret_cast<uint2 *>(reinterpret_cast<__half *>(lo) + o) =
+            make_uint2(*reinterpret_cast<const unsigned *>(&l2[0]),
+                       *reinterpret_cast<const unsigned *>(&l2[1]));
+      } else {
+        float g[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) g[q] = __uint_as_float(__float_as_uint(v[q]) & 0xFFFFE000u);
+        *reinterpret_cast<float4 *>(hi + o) = make_float4(g[0], g[1], g[2], g[3]);
+        *reinterpret_cast<float4 *>(lo + o) =
+            make_float4(v[0] - g[0], v[1] - g[1], v[2] - g[2], v[3] - g[3]);
+      }
     }
   }
 }
@@ -472,12 +490,12 @@ __device__ __forceinline__ void flush_share(const float *sb, float *__restrict__
 // [B, T, C] (y = hi).  NX input windows per warp: the copies of the next
 // NX - 1 tiles are in flight while a tile is computed.  TW_: warps per team
 // (TM), which also fixes the CTA's warps (TeamShape).
-template <bool TM, int NX, int TW_ = 4>
+template <bool TM, int NX, int TW_ = 4, bool F16 = false>
 __device__ __forceinline__ void activation_walk(
     const float *__restrict__ x, float *__restrict__ y, float *__restrict__ lo, int rows, int C,
     int T, int tiles_per_row, long long n_ids, const float *__restrict__ log_alpha,
     const float *__restrict__ log_beta, const float *__restrict__ f_up,
-    const float *__restrict__ f_dn, float eps) {
+    const float *__restrict__ f_dn, float eps, int *status = nullptr) {
   extern __shared__ __align__(16) float smem[];
   __shared__ __align__(16) float2 taps[24];  // 2 f_up, then f_down, as broadcast pairs
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -543,13 +561,14 @@ __device__ __forceinline__ void activation_walk(
   int p_t0 = 0;
   size_t obase = 0;  // TM: plane offset of the group's (b, t = 0, first channel)
   int n_out = 0;     // TM: staged tiles so far (selects the staging buffer)
+  float vmax = 0.0f;  // F16: the largest |value| written to the fp16 planes
   auto emit = [&](const float *vsrc, int t_out) {
     if constexpr (TM) {
       float *sb = stg + (n_out & 1) * S::kStgFloats;
       ++n_out;
       stage_b_stage(vsrc, taps, sb + S::region(k), lane);
       team_barrier<TW_>(team);
-      flush_share<TW_>(sb, y, lo, obase, C, t_out, T, k, lane);
+      flush_share<TW_, F16>(sb, y, lo, obase, C, t_out, T, k, lane, vmax);
     } else {
       stage_b(vsrc, taps, y + (size_t)(2 * pair) * T, 2 * pair + 1 < rows, t_out, T, lane);
     }
@@ -647,6 +666,9 @@ __device__ __forceinline__ void activation_walk(
     tile = ntile;
   }
   cp_async_wait<0>();
+  // fp16 holds |v| < 65504: a value at or past it marks the output invalid
+  if constexpr (F16)
+    if (!(vmax < 65504.0f) && status) atomicExch(status, kStatusF16Range);
 }
 
 __global__ void __launch_bounds__(THREADS, 2)
@@ -661,14 +683,15 @@ activation_kernel(const float *__restrict__ x, float *__restrict__ y, int rows, 
 // TW_ = 4: two 4-warp teams per CTA, two CTAs per SM; TW_ = 8: one 8-warp team
 // per CTA, two CTAs per SM; TW_ = 16: one 16-warp team per CTA, one CTA per
 // SM.  Each way 16 warps per SM.
-template <int TW_>
+template <int TW_, bool F16>
 __global__ void __launch_bounds__(32 * TeamShape<TW_>::kCtaWarps, TW_ == 16 ? 1 : 2)
 activation_tm_kernel(const float *__restrict__ x, float *__restrict__ hi, float *__restrict__ lo,
                      int rows, int C, int T, int tiles_per_row, long long n_tasks,
                      const float *__restrict__ log_alpha, const float *__restrict__ log_beta,
-                     const float *__restrict__ f_up, const float *__restrict__ f_dn, float eps) {
-  activation_walk<true, TM_NX, TW_>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks, log_alpha,
-                                    log_beta, f_up, f_dn, eps);
+                     const float *__restrict__ f_up, const float *__restrict__ f_dn, float eps,
+                     int *status) {
+  activation_walk<true, TM_NX, TW_, F16>(x, hi, lo, rows, C, T, tiles_per_row, n_tasks,
+                                         log_alpha, log_beta, f_up, f_dn, eps, status);
 }
 
 __global__ void sin_squared_kernel(const float *__restrict__ z, float *__restrict__ out,
@@ -712,7 +735,7 @@ int persistent_ctas_tm() {
     int sms = 148, per_sm = 1;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &per_sm, activation_tm_kernel<TW_>, 32 * TeamShape<TW_>::kCtaWarps,
+            &per_sm, activation_tm_kernel<TW_, false>, 32 * TeamShape<TW_>::kCtaWarps,
             tm_smem_bytes<TW_>()) != cudaSuccess ||
         per_sm < 1)
       per_sm = 1;
@@ -725,21 +748,29 @@ int persistent_ctas_tm() {
 template <int TW_>
 bv_status run_activation_tm(const float *x, float *hi, float *lo, long long rows, int C, int T,
                             const float *la, const float *lb, const float *fu, const float *fd,
-                            float eps, cudaStream_t st) {
+                            float eps, cudaStream_t st, bool f16) {
   using S = TeamShape<TW_>;
   const int tiles = (T + TW - 1) / TW;
   const long long n_tasks = rows / S::kCh * tiles;  // (group, tile) tasks
   if (n_tasks <= 0) return BV_OK;
-  BV_TRY(ensure_dynamic_smem((const void *)activation_tm_kernel<TW_>, tm_smem_bytes<TW_>(),
-                             "activation_tm smem attribute"));
+  BV_TRY(ensure_dynamic_smem(f16 ? (const void *)activation_tm_kernel<TW_, true>
+                                 : (const void *)activation_tm_kernel<TW_, false>,
+                             tm_smem_bytes<TW_>(), "activation_tm smem attribute"));
   const long long ctas = persistent_ctas_tm<TW_>();
   const long long need = (n_tasks + S::kTeams - 1) / S::kTeams;
   const long long grid = need < ctas ? need : ctas;
   {
-    // algorithmic bytes: read x (4 B), write the hi and lo planes (8 B)
-    LaunchTimer tm(st, "activation_tm", 0.0, 12.0 * (double)rows * T);
-    activation_tm_kernel<TW_><<<(unsigned)grid, 32 * S::kCtaWarps, tm_smem_bytes<TW_>(), st>>>(
-        x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb, fu, fd, eps);
+    // algorithmic bytes: read x (4 B), write the hi and lo planes (8 B, or
+    // 4 B in fp16)
+    LaunchTimer tm(st, "activation_tm", 0.0, (f16 ? 8.0 : 12.0) * (double)rows * T);
+    if (f16)
+      activation_tm_kernel<TW_, true><<<(unsigned)grid, 32 * S::kCtaWarps, tm_smem_bytes<TW_>(),
+                                        st>>>(x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb,
+                                              fu, fd, eps, device_status_ptr());
+    else
+      activation_tm_kernel<TW_, false><<<(unsigned)grid, 32 * S::kCtaWarps, tm_smem_bytes<TW_>(),
+                                         st>>>(x, hi, lo, (int)rows, C, T, tiles, n_tasks, la, lb,
+                                               fu, fd, eps, nullptr);
   }
   count_launch();
   return check_launch("activation_tm_kernel");
@@ -751,7 +782,7 @@ bool activation_tm_supported(int C) { return C % TeamShape<4>::kCh == 0; }
 
 bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int C, int T,
                                const float *la, const float *lb, const float *fu, const float *fd,
-                               float eps, cudaStream_t st) {
+                               float eps, cudaStream_t st, bool f16) {
   if (!activation_tm_supported(C))
     return fail(BV_ERR_UNSUPPORTED, "activation_tm: C = %d is not a multiple of %d", C,
                 TeamShape<4>::kCh);
@@ -761,10 +792,10 @@ bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int 
   if (rows > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "activation_tm: too many rows");
   // the widest plane rows per time step the channels allow
   if (C % TeamShape<16>::kCh == 0)
-    return run_activation_tm<16>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
+    return run_activation_tm<16>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st, f16);
   if (C % TeamShape<8>::kCh == 0)
-    return run_activation_tm<8>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
-  return run_activation_tm<4>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st);
+    return run_activation_tm<8>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st, f16);
+  return run_activation_tm<4>(x, hi, lo, rows, C, T, la, lb, fu, fd, eps, st, f16);
 }
 
 bv_status launch_sin_squared(const float *z, float *out, long long n, cudaStream_t st) {

@@ -232,6 +232,8 @@ bv_status bv_sync_status(void *stream) {
     const int zero = 0;
     cudaMemcpyToSymbolAsync(g_device_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, st);
     cudaStreamSynchronize(st);
+    if (h == kStatusF16Range)
+      return fail(BV_ERR_RANGE, "an activation reached fp16's range on the fp16 conv path");
     return fail(BV_ERR_TIMEOUT, "a bounded device wait gave up (code %d)", h);
   }
   return BV_OK;
@@ -371,6 +373,7 @@ struct AmpScratch {
 struct AmpSplit {
   const float *conv1[BV_MAX_DIL], *conv2[BV_MAX_DIL];
   bool tm1[BV_MAX_DIL], tm2[BV_MAX_DIL];
+  bool f16;  // the time-major splits are fp16 (tm_f16_ok and the config allow)
 };
 
 // One activation followed by one conv (Cin = C, output length Tout): through
@@ -380,30 +383,34 @@ bv_status act_conv_core(const float *in, int B, int C, int T, const float *la, c
                         const float *fu, const float *fd, float eps, const float *w,
                         const float *bias, int Cout, int K, int dil, int pad, const float *w_split,
                         bool tm, const Epi &ep, float *out, int Tout, float *h1, float *xhi,
-                        float *xlo, cudaStream_t st) {
+                        float *xlo, cudaStream_t st, bool f16) {
   if (tm && w_split && xhi) {
-    // the activation writes the conv's time-major operand planes itself
+    // the activation writes the conv's time-major operand planes itself, in
+    // fp16 when the weights were split in fp16 (f16: tm_f16_ok(C))
     if (activation_tm_supported(C)) {
-      BV_TRY(launch_activation_tm(in, xhi, xlo, B, C, T, la, lb, fu, fd, eps, st));
+      BV_TRY(launch_activation_tm(in, xhi, xlo, B, C, T, la, lb, fu, fd, eps, st, f16));
     } else {
       BV_TRY(launch_activation(in, h1, B, C, T, la, lb, fu, fd, eps, st));
       BV_TRY(launch_transpose_split(h1, xhi, xlo, B, C, T, st));
     }
     return launch_conv1d_tm(xhi, xlo, B, C, T, w_split, bias, Cout, K, dil, pad, ep, out, Tout,
-                            Tout, st);
+                            Tout, st, f16);
   }
+  // (tap-major split weights, tf32 or fp16, are for the time-major kernel
+  // only: without its planes the conv takes the raw weights)
   BV_TRY(launch_activation(in, h1, B, C, T, la, lb, fu, fd, eps, st));
-  return launch_conv1d(h1, B, C, T, w, bias, Cout, K, dil, pad, ep, out, Tout, Tout, st, w_split);
+  return launch_conv1d(h1, B, C, T, w, bias, Cout, K, dil, pad, ep, out, Tout, Tout, st,
+                       tm ? nullptr : w_split);
 }
 
 // act -> conv inside an AMP block (length-preserving pad).
 bv_status act_conv(const float *in, int B, int C, int T, const float *la, const float *lb,
                    const bv_amp_params &p, const float *w, const float *bias, const float *w_split,
                    bool tm, int dil, const Epi &ep, float *out, const AmpScratch &s,
-                   cudaStream_t st) {
+                   cudaStream_t st, bool f16) {
   const int K = p.kernel_size, pad = (K * dil - dil) / 2;
   return act_conv_core(in, B, C, T, la, lb, p.up_filter, p.down_filter, 1e-9f, w, bias, C, K, dil,
-                       pad, w_split, tm, ep, out, T, s.h1, s.xhi, s.xlo, st);
+                       pad, w_split, tm, ep, out, T, s.h1, s.xhi, s.xlo, st, f16);
 }
 
 // y = (accumulate ? y : 0) + scale * AMP(x); x, y and the scratch are disjoint.
@@ -416,14 +423,14 @@ bv_status run_amp_block(const float *x, int B, int C, int T, const bv_amp_params
     const Epi plain{nullptr, 1.0f, 0, 0};
     BV_TRY(act_conv(src, B, C, T, p.act_log_alpha[2 * u], p.act_log_beta[2 * u], p, p.conv1_w[u],
                     p.conv1_b[u], sp ? sp->conv1[u] : nullptr, sp && sp->tm1[u], p.dilation[u],
-                    plain, s.h2, s, st));
+                    plain, s.h2, s, st, sp && sp->f16));
     // last unit: y (+)= scale (src + conv2(...)); otherwise cur = src + conv2(...),
     // where src may be cur itself
     const bool last = (u == n - 1);
     const Epi res = last ? Epi{src, scale, accumulate, 0} : Epi{src, 1.0f, 0, 0};
     BV_TRY(act_conv(s.h2, B, C, T, p.act_log_alpha[2 * u + 1], p.act_log_beta[2 * u + 1], p,
                     p.conv2_w[u], p.conv2_b[u], sp ? sp->conv2[u] : nullptr, sp && sp->tm2[u], 1,
-                    res, last ? y : s.cur, s, st));
+                    res, last ? y : s.cur, s, st, sp && sp->f16));
   }
   return BV_OK;
 }
@@ -460,8 +467,10 @@ bv_status split_amp_weights(int C, const bv_amp_params &p, char *ws, AmpSplit *o
     tab.count[tab.n] = (long long)C * C * K;
     tab.cin[tab.n] = C;
     tab.k[tab.n] = K;
+    tab.f16[tab.n] = out->f16;
     ++tab.n;
   };
+  out->f16 = tm_f16_ok(C);
   for (int u = 0; u < p.n_dilations; ++u) {
     if (conv1d_tm_supported(C, C, K, p.dilation[u])) add(p.conv1_w[u], &out->conv1[u], &out->tm1[u]);
     if (conv1d_tm_supported(C, C, K, 1)) add(p.conv2_w[u], &out->conv2[u], &out->tm2[u]);
@@ -636,10 +645,12 @@ bv_status bv_act_conv1d(const float *x, int B, int C, int T, const float *log_al
     tab.count[0] = (long long)Cout * C * K;
     tab.cin[0] = C;
     tab.k[0] = K;
+    tab.f16[0] = tm_f16_ok(C);
     BV_TRY(launch_split_weights(tab, st));
   }
   return act_conv_core(x, B, C, T, log_alpha, log_beta, up_filter, down_filter, eps, w, bias,
-                       Cout, K, dilation, pad, split, plan.tm, e, y, (int)Tout, h1, xhi, xlo, st);
+                       Cout, K, dilation, pad, split, plan.tm, e, y, (int)Tout, h1, xhi, xlo, st,
+                       plan.tm && tm_f16_ok(C));
 }
 
 size_t bv_conv_transpose1d_workspace_size(int B, int Cin, int T, int Cout, int K, int stride) {
@@ -724,6 +735,8 @@ bv_status check_config(const bv_decoder_config *c) {
     return fail(BV_ERR_SHAPE, "decoder: tile %d overlap %d", c->tile_frames, c->overlap_frames);
   if (c->latent_channels < 0)
     return fail(BV_ERR_SHAPE, "decoder: latent_channels %d", c->latent_channels);
+  if (c->tf32_only != 0 && c->tf32_only != 1)
+    return fail(BV_ERR_ARG, "decoder: tf32_only %d", c->tf32_only);
   return BV_OK;
 }
 
@@ -851,6 +864,11 @@ bv_status split_weights(const bv_decoder_config *c, const bv_decoder_weights *w,
     tab.count[tab.n] = count;
     tab.cin[tab.n] = tm ? Cin : 0;
     tab.k[tab.n] = K;
+    // the AMP convs' time-major operands come from the activation, in fp16
+    // where tm_f16_ok unless the config asks for 3xTF32 throughout
+    const bool f16 = tm && (kind == 1 || kind == 2) && tm_f16_ok(Cin) && !c->tf32_only;
+    tab.f16[tab.n] = f16;
+    if (kind == 1 || kind == 2) out->amp[i][j].f16 = f16;
     if (++tab.n == kMaxSplit) {
       if (launch) status = launch_split_weights(tab, st);
       tab.n = 0;

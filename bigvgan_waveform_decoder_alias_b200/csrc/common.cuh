@@ -1,6 +1,7 @@
 // Shared host/device helpers of libbv (error state, launch accounting).
 #pragma once
 
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,6 +36,8 @@ bv_status ensure_dynamic_smem(const void *func, size_t bytes, const char *what);
 // Address of the device status word that bounded waits set when they give
 // up (kernels take it as an argument); nullptr if it cannot be resolved.
 int *device_status_ptr();
+// Status word value of an fp16 operand plane written out of range.
+constexpr int kStatusF16Range = 700;
 
 // Polls after which the tensor-core kernels' bounded waits give up (a kernel
 // argument; bv_debug_set_wait_limit changes it).
@@ -170,11 +173,12 @@ bv_status launch_activation(const float *x, float *y, int B, int C, int T, const
 
 // The activation writing the time-major tensor-core conv's operand planes
 // hi[b, t, c] = tf32(y), lo = y - hi instead of y [B, C, T] (C a multiple of 8;
-// planes 16-byte aligned).
+// planes 16-byte aligned).  With f16 the planes hold fp16 values instead:
+// hi = fp16(y), lo = fp16(y - hi), [B, T, C] halves at the same addresses.
 bool activation_tm_supported(int C);
 bv_status launch_activation_tm(const float *x, float *hi, float *lo, int B, int C, int T,
                                const float *la, const float *lb, const float *fu, const float *fd,
-                               float eps, cudaStream_t st);
+                               float eps, cudaStream_t st, bool f16 = false);
 
 // Latent front end: z [C, S, T] -> out [S, Cout, T], de-normalised then
 // projected by a one-tap conv w [Cout, C, 1] (+ bias or NULL).
@@ -232,6 +236,9 @@ struct SplitTable {
   // tap-major entries: src is [rows][cin][k] and dst[o][j cin + i] = src[o][i][j];
   // cin = 0 keeps src's order
   int cin[kMaxSplit], k[kMaxSplit];
+  // tap-major entries in fp16 (tm_f16_split): hi = fp16(s W), lo = fp16(s W - hi)
+  // with s = kTmF16WScale, rows padded to tm_cin_pad_f16(cin) channels per tap
+  unsigned char f16[kMaxSplit];
 };
 bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st);
 
@@ -260,10 +267,20 @@ bool conv1d_tm_supported(int Cin, int Cout, int K, int dil);
 // Channels per tap in the time-major conv's weight rows: Cin rounded up to
 // whole 32-channel blocks (the padding is zero).
 __host__ __device__ constexpr int tm_cin_pad(int cin) { return (cin + 31) / 32 * 32; }
+// The fp16 form of the time-major conv (f16 below): operands split into two
+// fp16 parts (x = hi + lo, W scaled by kTmF16WScale into fp16's normal range,
+// the products accumulated in fp32 and scaled back), 64-channel blocks (a
+// 128-byte fp16 row, the geometry of a 32-channel tf32 row).  Its split
+// weights take at most the bytes of the tf32 split.
+constexpr float kTmF16WScale = 4096.0f;
+__host__ __device__ constexpr int tm_cin_pad_f16(int cin) { return (cin + 63) / 64 * 64; }
+// The time-major convs fed by the time-major activation run in fp16 when
+// Cin allows: rows of 16 bytes and at most a third of padding in the blocks.
+bool tm_f16_ok(int Cin);
 bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
                            const float *w_split, const float *bias, int Cout, int K, int dil,
                            int pad, const Epi &ep, float *y, int y_len, int y_pitch,
-                           cudaStream_t st);
+                           cudaStream_t st, bool f16 = false);
 
 // Transposed conv on the time-major kernel: x_hi / x_lo [B, T, Cin] planes
 // (launch_transpose_split), each of the S output phases an ceil(K/S)-tap conv

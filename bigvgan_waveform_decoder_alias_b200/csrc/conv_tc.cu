@@ -712,6 +712,10 @@ __host__ __device__ constexpr uint32_t make_idesc_pair(int nt) {
   return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(nt >> 3) << 17) |
          ((uint32_t)(256 >> 4) << 24);
 }
+// The same for kind::f16 with A and B fp16 (format 0).
+__host__ __device__ constexpr uint32_t make_idesc_pair_f16(int nt) {
+  return (1u << 4) | ((uint32_t)(nt >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
 
 __device__ __forceinline__ unsigned cluster_rank() {
   unsigned r;
@@ -761,30 +765,27 @@ __device__ __forceinline__ void tma_load_2d_pair(unsigned dst, const CUtensorMap
 // collector buffer, LASTUSE takes A from there (the same descriptor) and frees
 // it, NONE reads A afresh.  Reusing A saves the tensor core one operand read.
 enum class ACol { NONE, FILL, LASTUSE };
-template <ACol C>
+#define BV_MMA_PAIR(KIND, COL)                                                              \
+  asm volatile("{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"                               \
+               " tcgen05.mma.cta_group::2.kind::" KIND COL " [%0], %1, %2, %3, p;\n}\n" ::"r"( \
+                   tmem_d),                                                                 \
+               "l"(a), "l"(b), "r"(idesc), "r"(acc)                                         \
+               : "memory")
+// kind::tf32, or kind::f16 (A and B fp16) with F16.
+template <ACol C, bool F16 = false>
 __device__ __forceinline__ void mma_tf32_pair(unsigned tmem_d, uint64_t a, uint64_t b,
                                               uint32_t idesc, unsigned acc) {
-  if constexpr (C == ACol::FILL)
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::2.kind::tf32.collector::a::fill [%0], %1, %2, %3, p;\n}\n" ::"r"(
-            tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
-  else if constexpr (C == ACol::LASTUSE)
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::2.kind::tf32.collector::a::lastuse [%0], %1, %2, %3, p;\n}\n" ::
-            "r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
-  else
-    asm volatile(
-        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-        " tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n}\n" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(idesc), "r"(acc)
-        : "memory");
+  if constexpr (F16) {
+    if constexpr (C == ACol::FILL) BV_MMA_PAIR("f16", ".collector::a::fill");
+    else if constexpr (C == ACol::LASTUSE) BV_MMA_PAIR("f16", ".collector::a::lastuse");
+    else BV_MMA_PAIR("f16", "");
+  } else {
+    if constexpr (C == ACol::FILL) BV_MMA_PAIR("tf32", ".collector::a::fill");
+    else if constexpr (C == ACol::LASTUSE) BV_MMA_PAIR("tf32", ".collector::a::lastuse");
+    else BV_MMA_PAIR("tf32", "");
+  }
 }
+#undef BV_MMA_PAIR
 // Arrive on the barrier at this offset in both CTAs once the MMAs issued so
 // far have completed.
 __device__ __forceinline__ void mma_commit_pair(unsigned bar) {
@@ -822,7 +823,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
 }
 
-template <int NT, int TAPS, bool STG>
+template <int NT, int TAPS, bool STG, bool F16>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  const __grid_constant__ CUtensorMap tmap_xlo,
@@ -833,7 +834,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                  Epi ep, OutMap om, int *status, long long wait_limit, int tpairs, int ntiles,
                  int n_tiles) {
   static_assert(NT % 32 == 0 && NT >= 32 && NT <= MAX_NT, "UMMA N for M = 256, halves of 16");
-  constexpr uint32_t IDESC = make_idesc_pair(NT);
+  constexpr uint32_t IDESC = F16 ? make_idesc_pair_f16(NT) : make_idesc_pair(NT);
+  // channels per block: one 128-byte operand row (32 tf32 or 64 fp16 values;
+  // an MMA takes 32 bytes of it, K = 8 or 16)
+  constexpr int CB = F16 ? 2 * BK : BK;
   constexpr unsigned W_TX_TAP = 2u * 2u * (NT / 2) * BK * 4;  // one tap: both CTAs, hi and lo
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem = reinterpret_cast<unsigned char *>(
@@ -894,8 +898,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
     tl.phase = bz - tl.b * om.phases;  // weight rows phase Cout .., output offset + phase
     return tl;
   };
-  const int n_cb = (Cin + BK - 1) / BK;  // 32-channel blocks (channels past Cin read as 0)
-  const int Cpad = n_cb * BK;            // weight row stride per tap
+  const int n_cb = (Cin + CB - 1) / CB;  // channel blocks (channels past Cin read as 0)
+  const int Cpad = n_cb * CB;            // weight row stride per tap
   const int n_tc = (K + TAPS - 1) / TAPS;  // chunks per block: taps 0 .. TAPS - 1, ...
   const int n_chunks = n_cb * n_tc;
   const int n_runs = (n_chunks + TM_RUN - 1) / TM_RUN;  // per tile
@@ -950,8 +954,8 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
           }
           const unsigned fb = bar_xfull + 8 * xs;
           if (leader) mbar_arrive_tx(fb, X_TX);
-          tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * BK, tl.t0 - pad, tl.b, fb);
-          tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * BK, tl.t0 - pad, tl.b, fb);
+          tma_load_3d_pair(x_at(xs, 0), &tmap_xhi, cb * CB, tl.t0 - pad, tl.b, fb);
+          tma_load_3d_pair(x_at(xs, 1), &tmap_xlo, cb * CB, tl.t0 - pad, tl.b, fb);
           ++gcb;
           if (++xs == XS) {
             xs = 0;
@@ -983,7 +987,7 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
             const unsigned fb = bar_wfull + 8 * ws;
             if (leader) mbar_arrive_tx(fb, W_TX_TAP * ntap);
             for (int t = 0; t < ntap; ++t) {
-              const int col = (j0 + t) * Cpad + cb * BK;
+              const int col = (j0 + t) * Cpad + cb * CB;
               tma_load_2d_pair(w_at(ws, t, 0), &tmap_whi, col, row, fb);
               tma_load_2d_pair(w_at(ws, t, 1), &tmap_wlo, col, row, fb);
             }
@@ -1040,13 +1044,13 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
               const uint64_t ah = dxh + rows, al = dxl + rows;
               const uint64_t bh = sw128_desc(w_at(ws, t, 0)), bl = sw128_desc(w_at(ws, t, 1));
 #pragma unroll
-              for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 = 32 bytes = 2 x 16 B per MMA
+              for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 or 16 fp16 = 32 B = 2 x 16 B per MMA
                 const uint64_t o = 2 * k;
                 // X_hi is the A operand of two products: read it once
-                mma_tf32_pair<ACol::FILL>(acc, ah + o, bh + o, IDESC,
-                                          (first && t == 0 && k == 0) ? 0u : 1u);
-                mma_tf32_pair<ACol::LASTUSE>(acc, ah + o, bl + o, IDESC, 1u);
-                mma_tf32_pair<ACol::NONE>(acc, al + o, bh + o, IDESC, 1u);
+                mma_tf32_pair<ACol::FILL, F16>(acc, ah + o, bh + o, IDESC,
+                                               (first && t == 0 && k == 0) ? 0u : 1u);
+                mma_tf32_pair<ACol::LASTUSE, F16>(acc, ah + o, bl + o, IDESC, 1u);
+                mma_tf32_pair<ACol::NONE, F16>(acc, al + o, bh + o, IDESC, 1u);
               }
             }
             mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot
@@ -1144,8 +1148,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
                 : "r"(taddr + 16u * h)
                 : "memory");
           asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+          // the fp16 weights carry kTmF16WScale (a power of two: exact)
+          constexpr float kBack = F16 ? 1.0f / kTmF16WScale : 1.0f;
 #pragma unroll
-          for (int e = 0; e < 32; ++e) sum[c0 + e] += __uint_as_float(v[e]);
+          for (int e = 0; e < 32; ++e) sum[c0 + e] = fmaf(__uint_as_float(v[e]), kBack, sum[c0 + e]);
         }
         asm volatile("tcgen05.fence::before_thread_sync;\n" ::: "memory");
         __syncwarp();
@@ -1256,7 +1262,7 @@ bool encode_y_tm(CUtensorMap *tmap, float *y, int B, int Cout, int y_len, int y_
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NT, int TAPS>
+template <int NT, int TAPS, bool F16>
 bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap &wh,
                  const CUtensorMap &wl, int B, int Cin, const float *bias, int Cout, int K,
                  int dil, int pad, const Epi &ep, float *y, int y_len, int y_pitch,
@@ -1269,8 +1275,8 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
                    tm_w_slots(BM + (K - 1) * dil, TAPS, NT, TM_STG_BYTES, 2) >= tm_min_wslots(TAPS) &&
                    encode_y_tm(&ym, y, B, Cout, y_len, y_pitch);
   if (!stg) std::memset(&ym, 0, sizeof(ym));
-  const void *kern = stg ? (const void *)conv1d_tm_kernel<NT, TAPS, true>
-                         : (const void *)conv1d_tm_kernel<NT, TAPS, false>;
+  const void *kern = stg ? (const void *)conv1d_tm_kernel<NT, TAPS, true, F16>
+                         : (const void *)conv1d_tm_kernel<NT, TAPS, false, F16>;
   BV_TRY(ensure_dynamic_smem(kern, TM_SMEM_BYTES, "conv1d_tm smem attribute"));
   // persistent: at most one CTA pair per two SMs, each walking its share of
   // the (time pair, output-channel tile, row-phase) tiles
@@ -1279,25 +1285,29 @@ bv_status run_tm(const CUtensorMap &xh, const CUtensorMap &xl, const CUtensorMap
   if (n_tiles > 0x7fffffffLL) return fail(BV_ERR_SHAPE, "conv1d_tm: too many tiles");
   const long long pairs = std::min<long long>(n_tiles, tm_pairs());
   if (stg)
-    conv1d_tm_kernel<NT, TAPS, true><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
+    conv1d_tm_kernel<NT, TAPS, true, F16><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
         xh, xl, wh, wl, ym, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
         device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
   else
-    conv1d_tm_kernel<NT, TAPS, false><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
+    conv1d_tm_kernel<NT, TAPS, false, F16><<<dim3((unsigned)(2 * pairs)), THREADS, TM_SMEM_BYTES, st>>>(
         xh, xl, wh, wl, ym, bias, y, Cin, Cout, K, dil, pad, y_len, y_pitch, ep, om,
         device_status_ptr(), wait_limit(), (int)tpairs, (int)ntiles, (int)n_tiles);
   return BV_OK;
 }
 
-// [B, T, C] fp32 plane as a 3-D tensor map, box 32 channels x `rows` times.
-bv_status encode_x_tm(CUtensorMap *tmap, const float *x, int B, int C, int T, int rows) {
+// [B, T, C] plane as a 3-D tensor map, box of one 128-byte row (32 fp32 or
+// 64 fp16 channels) x `rows` times.
+bv_status encode_x_tm(CUtensorMap *tmap, const float *x, int B, int C, int T, int rows,
+                      bool f16 = false) {
   if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: input not 16-byte aligned");
+  const cuuint64_t es = f16 ? 2 : 4;
   const cuuint64_t dims[3] = {(cuuint64_t)C, (cuuint64_t)T, (cuuint64_t)B};
-  const cuuint64_t strides[2] = {(cuuint64_t)C * sizeof(float), (cuuint64_t)T * C * sizeof(float)};
-  const cuuint32_t box[3] = {BK, (cuuint32_t)rows, 1};
+  const cuuint64_t strides[2] = {(cuuint64_t)C * es, (cuuint64_t)T * C * es};
+  const cuuint32_t box[3] = {f16 ? 2u * BK : (cuuint32_t)BK, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float *>(x), dims,
+  CUresult r = encode_fn()(tmap, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           3, const_cast<float *>(x), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1320,15 +1330,17 @@ bool conv1d_tc_supported(int Cin, int Cout, int K, int dil) {
 
 namespace {
 
-// Weight tensor map: [rows, Cin K] fp32, box 32 x nt, 128-byte swizzle.
-bv_status encode_w(CUtensorMap *tmap, const float *w, int rows, int KK, int nt) {
+// Weight tensor map: [rows, Cin K] fp32 (fp16 with f16), box one 128-byte
+// row x nt, 128-byte swizzle.
+bv_status encode_w(CUtensorMap *tmap, const float *w, int rows, int KK, int nt, bool f16 = false) {
   if ((reinterpret_cast<uintptr_t>(w) & 15u) != 0)
     return fail(BV_ERR_UNSUPPORTED, "conv1d_tc: weights not 16-byte aligned");
   const cuuint64_t dims[2] = {(cuuint64_t)KK, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)KK * sizeof(float)};
-  const cuuint32_t box[2] = {BK, (cuuint32_t)nt};
+  const cuuint64_t strides[1] = {(cuuint64_t)KK * (f16 ? 2 : 4)};
+  const cuuint32_t box[2] = {f16 ? 2u * BK : (cuuint32_t)BK, (cuuint32_t)nt};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = encode_fn()(tmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float *>(w), dims,
+  CUresult r = encode_fn()(tmap, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                           2, const_cast<float *>(w), dims,
                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1444,12 +1456,16 @@ __global__ void split_weights_kernel(SplitTable tab) {
       // one output row o at a time, 64 input channels per pass: the slice
       // src[o][i0 .. i0 + 64)[0 .. k) is contiguous, and so is each tap's run
       // dst[o][j cp + i0 .. + 64); shared memory turns one into the other.
-      // Rows are padded to cp = tm_cin_pad(cin) channels per tap with zeros.
+      // Rows are padded to cp = tm_cin_pad(cin) channels per tap with zeros
+      // (tm_cin_pad_f16 for the fp16 split, whose hi and lo are halves).
       __shared__ float sl[64 * MAX_K];
-      const int cin = tab.cin[e], k = tab.k[e], cp = tm_cin_pad(cin);
+      const bool f16 = tab.f16[e] != 0;
+      const int cin = tab.cin[e], k = tab.k[e];
+      const int cp = f16 ? tm_cin_pad_f16(cin) : tm_cin_pad(cin);
       const long long row = (long long)cin * k, drow = (long long)cp * k;
       const long long rows = n / row;
       lo = hi + rows * drow;
+      __half *const hi16 = reinterpret_cast<__half *>(hi), *const lo16 = hi16 + rows * drow;
       for (long long o = blockIdx.x; o < rows; o += gridDim.x) {
         for (int i0 = 0; i0 < cin; i0 += 64) {
           const int ni = cin - i0 < 64 ? cin - i0 : 64;
@@ -1458,18 +1474,30 @@ __global__ void split_weights_kernel(SplitTable tab) {
           __syncthreads();
           for (int q = threadIdx.x; q < ni * k; q += blockDim.x) {
             const int j = q / ni, ii = q - j * ni;
-            const float v = sl[ii * k + j], h = tf32_hi(v);
             const long long d = o * drow + (long long)j * cp + i0 + ii;
-            hi[d] = h;
-            lo[d] = v - h;
+            if (f16) {
+              const float v = sl[ii * k + j] * kTmF16WScale;
+              const __half h = __float2half_rn(v);
+              hi16[d] = h;
+              lo16[d] = __float2half_rn(v - __half2float(h));
+            } else {
+              const float v = sl[ii * k + j], h = tf32_hi(v);
+              hi[d] = h;
+              lo[d] = v - h;
+            }
           }
           __syncthreads();
         }
         for (int q = threadIdx.x; q < (cp - cin) * k; q += blockDim.x) {
           const int j = q / (cp - cin), ii = cin + q - j * (cp - cin);
           const long long d = o * drow + (long long)j * cp + ii;
-          hi[d] = 0.0f;
-          lo[d] = 0.0f;
+          if (f16) {
+            hi16[d] = __float2half_rn(0.0f);
+            lo16[d] = __float2half_rn(0.0f);
+          } else {
+            hi[d] = 0.0f;
+            lo[d] = 0.0f;
+          }
         }
       }
     } else if (vec) {
@@ -1612,11 +1640,16 @@ bv_status launch_conv_transpose1d_tc(const float *x, int B, int Cin, int T, cons
 bool conv1d_tm_supported(int Cin, int Cout, int K, int dil) {
   // input rows of Cin floats must be 16-byte multiples (TMA strides); a
   // partial last channel block costs padded tensor work, so at most a third.
-  // Below 40 output channels (measured on B200 with 24: N = 32 tiles) the
-  // FP32 SIMT kernel is faster.  A reduction of two channel blocks (a one-tap
-  // conv over 64 channels) already beats the SIMT kernel (measured on the
-  // DAV decoder's 96-channel one-tap convs).
-  return Cin % 4 == 0 && 3 * tm_cin_pad(Cin) <= 4 * Cin && Cout >= 40 &&
+  // From 40 output channels, or 32 when neither the tile nor the channel
+  // blocks are padded.  Measured on B200 against the FP32 narrow kernel: 24
+  // channels in 32-channel tiles and blocks break even per conv and lose with
+  // the dearer time-major activation (60 s H3 decode 565 -> 560 audio-s/s);
+  // the 32-channel stage of the LTX bandwidth-extension tail gains (10.0 ->
+  // 9.3 ms per 10 s).  A reduction of two channel blocks (a one-tap conv over
+  // 64 channels) already beats the SIMT kernel (measured on the DAV decoder's
+  // 96-channel one-tap convs).
+  return Cin % 4 == 0 && 3 * tm_cin_pad(Cin) <= 4 * Cin &&
+         (Cout >= 40 || (Cout == 32 && Cin % 32 == 0)) &&
          tm_cin_pad(Cin) * K >= 64 && K >= 1 && K <= MAX_K && dil >= 1 &&
          (K - 1) * dil <= TM_MAX_HALO && encode_fn() != nullptr;
 }
@@ -1628,25 +1661,30 @@ namespace {
 bv_status tm_impl(const char *cls, const float *x_hi, const float *x_lo, int B, int Cin, int T,
                   const float *w_split, int w_rows, const float *bias, int Cout, int K, int dil,
                   int pad, const Epi &ep, float *y, int y_len, int y_pitch, const OutMap &om,
-                  double flops, double bytes, cudaStream_t st) {
+                  double flops, double bytes, cudaStream_t st, bool f16 = false) {
   const int nt = pick_nt_pair(Cout);
-  const int KK = tm_cin_pad(Cin) * K;  // tap-major weight row, padded channels
+  // tap-major weight row, padded channels
+  const int KK = (f16 ? tm_cin_pad_f16(Cin) : tm_cin_pad(Cin)) * K;
   CUtensorMap xh, xl, wh, wl;
-  BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T, BM + (K - 1) * dil));
-  BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T, BM + (K - 1) * dil));
-  BV_TRY(encode_w(&wh, w_split, w_rows, KK, nt / 2));  // each CTA of a pair loads half the rows
-  BV_TRY(encode_w(&wl, w_split + (size_t)w_rows * KK, w_rows, KK, nt / 2));
+  BV_TRY(encode_x_tm(&xh, x_hi, B, Cin, T, BM + (K - 1) * dil, f16));
+  BV_TRY(encode_x_tm(&xl, x_lo, B, Cin, T, BM + (K - 1) * dil, f16));
+  // each CTA of a pair loads half the rows; lo follows hi
+  const float *w_lo = reinterpret_cast<const float *>(reinterpret_cast<const char *>(w_split) +
+                                                      (size_t)w_rows * KK * (f16 ? 2 : 4));
+  BV_TRY(encode_w(&wh, w_split, w_rows, KK, nt / 2, f16));
+  BV_TRY(encode_w(&wl, w_lo, w_rows, KK, nt / 2, f16));
   bv_status s;
   {
     LaunchTimer tm(st, cls, flops, bytes);
-#define BV_TM_CASE(N)                                                                        \
-  case N:                                                                                    \
-    s = K >= 3 ? run_tm<N, 4>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, \
-                              y_pitch, om, st)                                               \
-               : run_tm<N, 2>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, \
-                              y_pitch, om, st);                                              \
+#define BV_TM_RUN(N, TP, H)                                                                 \
+  run_tm<N, TP, H>(xh, xl, wh, wl, B, Cin, bias, Cout, K, dil, pad, ep, y, y_len, y_pitch, om, st)
+#define BV_TM_CASE(N)                                                                       \
+  case N:                                                                                   \
+    s = f16 ? (K >= 3 ? BV_TM_RUN(N, 4, true) : BV_TM_RUN(N, 2, true))                      \
+            : (K >= 3 ? BV_TM_RUN(N, 4, false) : BV_TM_RUN(N, 2, false));                   \
     break;
     switch (nt) {
+      BV_TM_CASE(32)
       BV_TM_CASE(64)
       BV_TM_CASE(96)
       BV_TM_CASE(128)
@@ -1654,6 +1692,7 @@ bv_status tm_impl(const char *cls, const float *x_hi, const float *x_lo, int B, 
         return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: tile %d", nt);
     }
 #undef BV_TM_CASE
+#undef BV_TM_RUN
   }
   if (s != BV_OK) return s;
   count_launch();
@@ -1662,21 +1701,27 @@ bv_status tm_impl(const char *cls, const float *x_hi, const float *x_lo, int B, 
 
 }  // namespace
 
+bool tm_f16_ok(int Cin) {
+  return Cin % 8 == 0 && 3 * tm_cin_pad_f16(Cin) <= 4 * Cin && activation_tm_supported(Cin);
+}
+
 bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
                            const float *w_split, const float *bias, int Cout, int K, int dil,
                            int pad, const Epi &ep, float *y, int y_len, int y_pitch,
-                           cudaStream_t st) {
+                           cudaStream_t st, bool f16) {
   if (B <= 0 || y_len <= 0) return BV_OK;
-  if (!conv1d_tm_supported(Cin, Cout, K, dil))
-    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d", Cin, Cout, K);
+  if (!conv1d_tm_supported(Cin, Cout, K, dil) || (f16 && !tm_f16_ok(Cin)))
+    return fail(BV_ERR_UNSUPPORTED, "conv1d_tm: Cin %d Cout %d K %d%s", Cin, Cout, K,
+                f16 ? " (fp16)" : "");
   // algorithmic work: the useful products (Cin K per output), not the padded
   // channel block or the three 3xTF32 terms
   const double outs = (double)B * Cout * y_len;
-  return tm_impl("conv1d_tm", x_hi, x_lo, B, Cin, T, w_split, Cout, bias, Cout, K, dil, pad, ep,
+  return tm_impl(f16 ? "conv1d_tm_f16" : "conv1d_tm", x_hi, x_lo, B, Cin, T, w_split, Cout, bias,
+                 Cout, K, dil, pad, ep,
                  y, y_len, y_pitch, OutMap{1, 0, y_len, 1}, 2.0 * outs * Cin * K,
                  4.0 * ((double)B * Cin * T + (double)Cout * Cin * K +
                         outs * (1 + (ep.residual ? 1 : 0) + ep.accumulate)),
-                 st);
+                 st, f16);
 }
 
 bool conv_transpose1d_tm_supported(int Cin, int Cout, int K, int S) {

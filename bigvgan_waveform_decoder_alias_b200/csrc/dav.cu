@@ -216,6 +216,7 @@ bv_status dav_decode_impl(const bv_dav_config *c, const bv_dav_weights *w, const
       tab.count[tab.n] = (long long)C * C * K;
       tab.cin[tab.n] = C;
       tab.k[tab.n] = K;
+      tab.f16[tab.n] = 0;  // the DAV convs read tf32 planes
       if (++tab.n == kMaxSplit) {
         BV_TRY(launch_split_weights(tab, st));
         tab.n = 0;

@@ -24,7 +24,8 @@ BV_MAX_BLOCKS = 4
 BV_MAX_DIL = 4
 FINAL_ACTS = {"none": 0, "clamp": 1, "tanh": 2}
 STATUS = {0: "BV_OK", 1: "BV_ERR_ARG", 2: "BV_ERR_SHAPE", 3: "BV_ERR_WORKSPACE",
-          4: "BV_ERR_CUDA", 5: "BV_ERR_TIMEOUT", 6: "BV_ERR_UNSUPPORTED"}
+          4: "BV_ERR_CUDA", 5: "BV_ERR_TIMEOUT", 6: "BV_ERR_UNSUPPORTED",
+          7: "BV_ERR_RANGE"}
 
 
 class BVError(RuntimeError):
@@ -60,7 +61,7 @@ class DecoderConfig(ctypes.Structure):
                 ("dilation", ctypes.c_int * BV_MAX_DIL), ("post_kernel", ctypes.c_int),
                 ("out_channels", ctypes.c_int), ("final_act", ctypes.c_int),
                 ("tile_frames", ctypes.c_int), ("overlap_frames", ctypes.c_int),
-                ("latent_channels", ctypes.c_int)]
+                ("latent_channels", ctypes.c_int), ("tf32_only", ctypes.c_int)]
 
 
 class DecoderWeights(ctypes.Structure):
@@ -420,7 +421,8 @@ def bv_amp_block(x, params: AmpParams, y=None, scale=1.0, accumulate=False, work
 # ----------------------------------------------------------------- decoder
 
 
-def decoder_config(g: DecoderGeometry, tile_frames=0, overlap_frames=0) -> DecoderConfig:
+def decoder_config(g: DecoderGeometry, tile_frames=0, overlap_frames=0,
+                   tf32_only=False) -> DecoderConfig:
     c = DecoderConfig()
     c.in_channels, c.pre_channels, c.pre_kernel = g.in_channels, g.pre_channels, g.pre_kernel
     c.n_up = len(g.up_rates)
@@ -435,6 +437,7 @@ def decoder_config(g: DecoderGeometry, tile_frames=0, overlap_frames=0) -> Decod
     c.post_kernel, c.out_channels = g.post_kernel, g.out_channels
     c.final_act = FINAL_ACTS[g.final_act] if isinstance(g.final_act, str) else int(g.final_act)
     c.tile_frames, c.overlap_frames = tile_frames, overlap_frames
+    c.tf32_only = int(bool(tf32_only))
     return c
 
 
@@ -448,12 +451,13 @@ class Decoder:
     `filt` the 12 resampling taps (both filters)."""
 
     def __init__(self, geometry: DecoderGeometry, params, filt=None, tile_frames=0,
-                 overlap_frames=0, device="cuda", front_end=None):
+                 overlap_frames=0, device="cuda", front_end=None, tf32_only=False):
         """front_end: optional (latents_mean, latents_std, dec_in_w, dec_in_b)
         of the latent front end; decode() then takes normalised latents
-        [latent_channels, B, frames]."""
+        [latent_channels, B, frames].  tf32_only: every tensor-core conv in
+        3xTF32 (else the AMP convs that qualify use the fp16 split)."""
         self.geometry = geometry
-        self.cfg = decoder_config(geometry, tile_frames, overlap_frames)
+        self.cfg = decoder_config(geometry, tile_frames, overlap_frames, tf32_only)
         n = bv_decoder_param_count(self.cfg)
         if n < 0:
             raise BVError(2, last_error())

@@ -45,7 +45,9 @@ typedef enum {
   BV_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required */
   BV_ERR_CUDA = 4,        /* a CUDA call failed (message has the CUDA error) */
   BV_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
-  BV_ERR_UNSUPPORTED = 6  /* a valid request this build does not implement */
+  BV_ERR_UNSUPPORTED = 6, /* a valid request this build does not implement */
+  BV_ERR_RANGE = 7        /* an activation reached fp16's range (|v| >= 65504) on
+                             the fp16 time-major path; that output is not valid */
 } bv_status;
 
 #define BV_FILTER_TAPS 12 /* both resampling filters: 12 taps ([H3] FILTER_LEN) */
@@ -84,8 +86,11 @@ int bv_timing_read(bv_kernel_stats *out, int max);
 void bv_timing_reset(void);
 
 /* Reads and clears the device status word that bounded device-side waits
- * set when they give up; returns BV_OK or BV_ERR_TIMEOUT.  Synchronises
- * `stream`. */
+ * set when they give up, and that the activation feeding the fp16 time-major
+ * convs sets when a value reaches |v| >= 65504 (fp16's range: the convs of
+ * channel counts that are multiples of 8 from 48 up take their operands in
+ * two fp16 parts); returns BV_OK, BV_ERR_TIMEOUT or BV_ERR_RANGE.
+ * Synchronises `stream`. */
 bv_status bv_sync_status(void *stream);
 
 /* Testing hook for the bounded waits.  The tensor-core kernels poll each
@@ -352,6 +357,17 @@ typedef struct {
                         * > 0: z holds normalised latents [latent_channels, B,
                         * frames] that first go through the latent front end
                         * (bv_latent_front_end) into in_channels */
+  int tf32_only;       /* 0: the AMP-block convs whose channel count is a
+                        * multiple of 8 from 48 up take their tensor-core
+                        * operands as two fp16 parts (x = hi + lo, W likewise,
+                        * three products accumulated in fp32: 22 significant
+                        * bits per operand as in the tf32 split, rounded
+                        * instead of truncated, at twice the tf32 MMA rate);
+                        * their activations must stay below 65504 in
+                        * magnitude, else bv_sync_status reports BV_ERR_RANGE.
+                        * 1: every tensor-core conv splits into tf32 parts
+                        * (3xTF32, the full f32 range).  Prepared weights
+                        * follow the config they were prepared with. */
 } bv_decoder_config;
 
 typedef struct {

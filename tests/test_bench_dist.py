@@ -78,3 +78,23 @@ def test_tensor_peak_follows_the_clocks():
     slow = {"sm_mhz": 1000.0, "sm_max_mhz": 1965.0, "reasons": []}
     assert bench.tensor_peak(pk, slow)[0] == pytest.approx(
         1400.0 * 1000.0 / 1300.0 * bench.TF32_PER_BF16 / 3.0)
+
+
+def test_tensor_peak_of_the_fp16_split():
+    """The fp16 split conv class takes the bf16 figure at the fp16 rate (1:1
+    with bf16) over its three products, under the same clock rules."""
+    sys.path.insert(0, ROOT)
+    import bench
+    pk = {"bf16": 1590.0, "bf16_sustained": 1400.0, "sustained_mhz": 1300.0,
+          "sm_max_mhz": 1965.0, "source": "fallback"}
+    full = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    peak, src, burst = bench.tensor_peak(pk, full, f16=True)
+    assert peak == pytest.approx(530.0) and burst == pytest.approx(530.0)
+    assert "3xF16" in src
+    capped_low = {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.tensor_peak(pk, capped_low, f16=True)[0] == pytest.approx(1400.0 / 3.0)
+    kd = {"avg_launch_ms": 1.0, "flops": 300e9, "bytes": 1e9}
+    r = bench.roofline_for("conv1d_tm_f16", kd, pk, full)
+    assert r["bound"] == "tensor" and r["frac"] == pytest.approx(300.0 / 530.0)
+    r = bench.roofline_for("conv1d_tm", kd, pk, full)
+    assert r["frac"] == pytest.approx(300.0 / (1590.0 * bench.TF32_PER_BF16 / 3.0))

@@ -36,21 +36,24 @@ def nat():
     return native
 
 
+@pytest.mark.parametrize("tf32_only", [False, True], ids=["default-split", "3xtf32"])
 @pytest.mark.parametrize("name", sorted(synth.DECODER_WORKLOADS))
-def test_full_size_decoder_matches_oracle(nat, name):
+def test_full_size_decoder_matches_oracle(nat, name, tf32_only):
+    """Both conv splits: the default (fp16 parts for the AMP convs that
+    qualify) and 3xTF32 throughout."""
     g = np.load(os.path.join(GOLDEN, f"{name}.npz"))
     w = synth.DECODER_WORKLOADS[name]
     z, params = w.make()
     dec = nat.Decoder(w.geometry, params, tile_frames=w.tile_frames,
-                      overlap_frames=w.overlap_frames)
+                      overlap_frames=w.overlap_frames, tf32_only=tf32_only)
     y = dec.decode(torch.from_numpy(z).cuda()).cpu().numpy()
     L = w.frames * w.geometry.hop
     assert y.shape == (w.batch, 1, L)
     idx, want = g["idx"], g["value"]
     got = y[:, 0, idx]
     err = rel_l2(got, want)
-    print(f"{name}: rel-L2 vs oracle {err:.3e} over {idx.size} positions x {w.batch} rows, "
-          f"max abs {np.abs(got - want).max():.3e}")
+    print(f"{name} ({'3xTF32' if tf32_only else 'default split'}): rel-L2 vs oracle {err:.3e} "
+          f"over {idx.size} positions x {w.batch} rows, max abs {np.abs(got - want).max():.3e}")
     assert err < WAVE_TOL
     for b in range(w.batch):
         assert rel_l2(got[b], want[b]) < WAVE_TOL

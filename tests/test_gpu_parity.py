@@ -329,6 +329,16 @@ TC_CASES = [(64, 64, 3, 1, 200), (128, 128, 3, 1, 1), (128, 128, 7, 3, 5), (96, 
             (48, 48, 11, 5, 77), (64, 40, 3, 1, 300), (96, 112, 7, 1, 130), (80, 80, 3, 1, 9)]
 
 
+# The time-major conv's timer classes: 3xTF32, and the fp16 split that convs
+# fed by the time-major activation take for channel counts that are
+# multiples of 8 from 48 up.
+TM_CLASSES = ("conv1d_tm", "conv1d_tm_f16")
+
+
+def _has_tm(classes):
+    return any(c in classes for c in TM_CLASSES)
+
+
 def _kernel_classes(nat, fn):
     nat.timing(True)
     nat.timing_reset()
@@ -467,7 +477,7 @@ def test_full_size_act_conv_time_major_sampled(nat, oracle, filt, C, T, K, d, re
     classes = _kernel_classes(nat, lambda: out.setdefault("y", nat.bv_act_conv1d(
         xd, dev(la), dev(lb), filt, wd, bd, d, pad, residual=rd)))
     # the activation writes the conv's time-major operands itself
-    assert "conv1d_tm" in classes and "activation_tm" in classes, classes
+    assert "conv1d_tm_f16" in classes and "activation_tm" in classes, classes
     assert "transpose_split" not in classes, classes
     y = host(out["y"])
     h = oracle.activation1d(x, la, lb)  # the conv's input, stored as float
@@ -527,7 +537,8 @@ def test_act_conv_time_major_activation_ragged(nat, oracle, filt, B, C, T):
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault("y", nat.bv_act_conv1d(
         xd, dev(la), dev(lb), filt, dev(w), dev(b), d, 3)))
-    assert "activation_tm" in classes and "conv1d_tm" in classes, classes
+    assert "activation_tm" in classes and _has_tm(classes), classes
+    assert ("conv1d_tm_f16" in classes) == (C >= 48), classes
     y = host(out["y"])
     want = oracle.conv1d(oracle.activation1d(x, la, lb), w, b, d, 3)
     assert y.shape == want.shape
@@ -537,10 +548,10 @@ def test_act_conv_time_major_activation_ragged(nat, oracle, filt, B, C, T):
 
 @pytest.mark.parametrize("C,T,K,d", [(64, 777, 7, 3), (128, 300, 3, 1), (24, 513, 11, 5),
                                      (100, 257, 5, 2), (96, 1000, 1, 1), (64, 515, 1, 1),
-                                     (128, 1000, 11, 5), (48, 516, 3, 1)])
+                                     (128, 1000, 11, 5), (48, 516, 3, 1), (32, 301, 11, 3)])
 def test_act_conv_small_shapes_every_element(nat, oracle, filt, C, T, K, d):
     """bv_act_conv1d on every path (time-major with the fused activation for
-    64 / 96 / 128 channels, one-tap convs included, time-major through a
+    32 / 64 / 96 / 128 channels, one-tap convs included, time-major through a
     separate transpose for 100, the narrow FP32 kernel for 24), every output
     against the oracle.  Rows of a multiple of 4 time steps take the staged
     bulk-store output loop (48 channels: a 16-channel group past Cout; 516:
@@ -584,7 +595,8 @@ AMP_SHAPES = [(12, 3001, 11, (1, 3, 5), False), (96, 517, 7, (1, 3, 5), True),
               (130, 64, 3, (2,), False), (16, 5, 7, (1, 3, 5, 7), False),
               (128, 2001, 11, (1, 3, 5), True), (48, 1003, 7, (1, 3, 5), True),
               (64, 300, 3, (1, 3, 5), True), (256, 130, 11, (5,), True),
-              (24, 700, 11, (1, 3, 5), False), (96, 516, 7, (1, 3, 5), True)]
+              (24, 700, 11, (1, 3, 5), False), (96, 516, 7, (1, 3, 5), True),
+              (32, 520, 7, (1, 3, 5), True)]
 
 
 @pytest.mark.parametrize("tensor_core", [False, True])
@@ -602,7 +614,7 @@ def test_amp_block_shapes(nat, oracle, filt, C, T, K, dils, tm, tensor_core):
     classes = _kernel_classes(nat, lambda: nat.bv_amp_block(dev(x), p, y=yd, scale=0.5,
                                                             accumulate=True,
                                                             tensor_core=tensor_core))
-    assert ("conv1d_tm" in classes) == (tm and tensor_core), classes
+    assert _has_tm(classes) == (tm and tensor_core), classes
     want = 0.5 * oracle.amp_block(x, flat, K, dils).astype(np.float64) + y0
     assert rel_l2(host(yd), want) < LAYER_TOL
 
@@ -660,7 +672,7 @@ def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     assert "conv_transpose1d_tm" in classes, classes
     # the 128/96/48-channel AMP convs run time-major, fed by the activation
     # writing their operand planes; the ConvT inputs are transposed
-    assert "conv1d_tm" in classes and "activation_tm" in classes, classes
+    assert _has_tm(classes) and "activation_tm" in classes, classes
     assert "transpose_split" in classes, classes
     want = oracle.decode(geo, params, z)
     assert rel_l2(host(out["y"]), want) < WAVE_TOL
@@ -993,7 +1005,7 @@ def test_decode_with_prepared_weights(nat, filt):
         # kernel classes are compared there)
         classes = _kernel_classes(nat, lambda: prep.decode(z))
         assert "weight_split" not in classes and "convt_repack" not in classes, classes
-        assert "conv1d_tm" in classes and "conv_transpose1d_tm" in classes, classes
+        assert _has_tm(classes) and "conv_transpose1d_tm" in classes, classes
         n_units = prep.tile_count(13) * 2
         rows = prep.decode_units(z, 0, n_units)
         np.testing.assert_array_equal(host(prep.stitch_units(rows, 2, 13)), want)

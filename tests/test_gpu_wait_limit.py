@@ -72,7 +72,7 @@ def test_wait_limit_zero_reports_timeout_and_context_survives(nat, oracle):
     finally:
         nat.timing(False)
         nat.timing_reset()
-    assert "conv1d_tm" in classes and "conv1d_tc" in classes, classes
+    assert "conv1d_tm_f16" in classes and "conv1d_tc" in classes, classes
     assert _status(nat) == 0
 
     prev = nat.set_wait_limit(0)
@@ -96,3 +96,31 @@ def test_wait_limit_zero_reports_timeout_and_context_survives(nat, oracle):
     y2 = conv().cpu().numpy()
     assert rel_l2(y2, oracle.conv1d(x, w, b, d, pad)) < LAYER_TOL
     assert _status(nat) == 0
+
+
+BV_ERR_RANGE = 7
+
+
+def test_fp16_operand_range_is_reported(nat, oracle):
+    """The fp16 time-major path (64 channels) on activations past fp16's range
+    (inputs of order 1e5; the activation is about its input there): the status
+    word reports BV_ERR_RANGE, and the next call on ordinary inputs is clean and
+    matches the oracle."""
+    s = synth.NormalStream(322)
+    C, T, K, d = 64, 300, 3, 1
+    x = s.normal((2, C, T))
+    la, lb = s.normal((C,), 0.0, 0.1), s.normal((C,), 0.0, 0.1)
+    w = s.normal((C, C, K), 0.0, 0.02)
+    b = s.normal((C,), 0.0, 0.02)
+    filt = torch.from_numpy(nat.bv_filter_design()).cuda()
+    lad, lbd = (torch.from_numpy(a).cuda() for a in (la, lb))
+    wd, bd = torch.from_numpy(w).cuda(), torch.from_numpy(b).cuda()
+    assert _status(nat) == 0
+    big = torch.from_numpy(1.0e5 * x).cuda()
+    nat.bv_act_conv1d(big, lad, lbd, filt, wd, bd, d, 1)
+    assert _status(nat) == BV_ERR_RANGE
+    assert "fp16" in nat.last_error()
+    y = nat.bv_act_conv1d(torch.from_numpy(x).cuda(), lad, lbd, filt, wd, bd, d, 1)
+    assert _status(nat) == 0
+    want = oracle.conv1d(oracle.activation1d(x, la, lb), w, b, d, 1)
+    assert rel_l2(y.cpu().numpy(), want) < LAYER_TOL
