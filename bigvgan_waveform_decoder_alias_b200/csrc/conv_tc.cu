@@ -773,7 +773,7 @@ enum class ACol { NONE, FILL, LASTUSE };
                : "memory")
 // kind::tf32, or kind::f16 (A and B fp16) with F16.
 template <ACol C, bool F16 = false>
-__device__ __forceinline__ void mma_tf32_pair(unsigned tmem_d, uint64_t a, uint64_t b,
+__device__ __forceinline__ void mma_split_pair(unsigned tmem_d, uint64_t a, uint64_t b,
                                               uint32_t idesc, unsigned acc) {
   if constexpr (F16) {
     if constexpr (C == ACol::FILL) BV_MMA_PAIR("f16", ".collector::a::fill");
@@ -1047,10 +1047,10 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
               for (int k = 0; k < BK / 8; ++k) {  // 8 tf32 or 16 fp16 = 32 B = 2 x 16 B per MMA
                 const uint64_t o = 2 * k;
                 // X_hi is the A operand of two products: read it once
-                mma_tf32_pair<ACol::FILL, F16>(acc, ah + o, bh + o, IDESC,
+                mma_split_pair<ACol::FILL, F16>(acc, ah + o, bh + o, IDESC,
                                                (first && t == 0 && k == 0) ? 0u : 1u);
-                mma_tf32_pair<ACol::LASTUSE, F16>(acc, ah + o, bl + o, IDESC, 1u);
-                mma_tf32_pair<ACol::NONE, F16>(acc, al + o, bh + o, IDESC, 1u);
+                mma_split_pair<ACol::LASTUSE, F16>(acc, ah + o, bl + o, IDESC, 1u);
+                mma_split_pair<ACol::NONE, F16>(acc, al + o, bh + o, IDESC, 1u);
               }
             }
             mma_commit_pair(bar_wempty + 8 * ws);  // both CTAs may refill the weight slot

@@ -204,8 +204,11 @@ bv_status bv_conv_transpose1d(const float *x, int B, int Cin, int T,
  * bias [Cout] or NULL; y [B, Cout, T + 2 pad - dilation (K - 1)]; all
  * device.  When the conv qualifies for the time-major tensor-core path
  * (C a multiple of 4 with at most a third of channel padding to 32-channel
- * blocks, Cout >= 40, (K - 1) dilation <= 56) the activation's output is
- * laid out time-major and the conv runs there, as inside bv_decode.
+ * blocks, Cout >= 40 or Cout = 32 with C a multiple of 32, (K - 1) dilation
+ * <= 56) the activation's output is laid out time-major and the conv runs
+ * there, as inside bv_decode: in two fp16 parts where C is a multiple of 8
+ * from 48 up (activations below 65504 in magnitude, else bv_sync_status
+ * reports BV_ERR_RANGE; see bv_decoder_config.tf32_only), else in 3xTF32.
  * Workspace: bv_act_conv1d_workspace_size bytes, 256-byte aligned, disjoint
  * from x, y and the residual.  x must not overlap y; the residual may be y.
  * Errors: BV_ERR_ARG, BV_ERR_SHAPE (sizes < 1, K > 32, output length < 1),
@@ -269,8 +272,9 @@ size_t bv_amp_block_workspace_size(int B, int C, int T);
 
 /* Workspace bytes with which bv_amp_block runs the block's convs on the
  * tensor cores from time-major operands (the path bv_decode takes): room for
- * two [B, T, C] operand planes and the convs' weights split into tf32 hi / lo
- * parts, besides the three [B, C, T] buffers.  Equals
+ * two [B, T, C] operand planes and the convs' weights split into hi / lo
+ * parts (fp16 where C is a multiple of 8 from 48 up, as bv_act_conv1d; else
+ * tf32), besides the three [B, C, T] buffers.  Equals
  * bv_amp_block_workspace_size when no conv of the block qualifies (narrow
  * channel counts, or no tensor-core support); 0 for invalid arguments. */
 size_t bv_amp_block_workspace_size_tc(int B, int C, int T, const bv_amp_params *p);
@@ -386,8 +390,9 @@ typedef struct {
   const void *prepared;
 } bv_decoder_weights;
 
-/* Prepared weights: the tf32 hi / lo split of every tensor-core conv's
- * weights (tap-major where the conv runs time-major) and the packed phase
+/* Prepared weights: the hi / lo split of every tensor-core conv's weights
+ * (tap-major where the conv runs time-major; fp16 parts for the AMP convs the
+ * config's tf32_only leaves on the fp16 split, else tf32) and the packed phase
  * weights of every tensor-core transposed conv, written once into a caller
  * buffer (device, 256-byte aligned, bv_decoder_prepared_size bytes) and read
  * by every later decode whose weights point at it (w->prepared).  The buffer
