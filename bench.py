@@ -269,8 +269,8 @@ def tensor_peak(pk, clocks, f16=False):
 
 # kernel classes on the tensor cores: 3xTF32, and the fp16 split
 TENSOR_CLASSES = ("conv1d_tm", "conv1d_tc", "conv_transpose1d_tc", "conv_transpose1d_tm",
-                  "conv1d_tm_f16")
-F16_CLASSES = ("conv1d_tm_f16",)
+                  "conv1d_tm_f16", "conv_transpose1d_tm_f16")
+F16_CLASSES = ("conv1d_tm_f16", "conv_transpose1d_tm_f16")
 
 # Measured DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) over
 # the algorithmic bytes, per kernel class, from one ncu capture of every launch

@@ -689,9 +689,10 @@ bv_status bv_conv_transpose1d_ws(const float *x, int B, int Cin, int T, const fl
     float *xhi = reinterpret_cast<float *>(w8);
     float *xlo = reinterpret_cast<float *>(w8 + plan.plane);
     float *wp = reinterpret_cast<float *>(w8 + 2 * plan.plane);
-    BV_TRY(launch_transpose_split(x, xhi, xlo, B, Cin, T, st));
+    const bool f16 = tm_f16_ok(Cin);
+    BV_TRY(launch_transpose_split(x, xhi, xlo, B, Cin, T, st, f16));
     return launch_conv_transpose1d_tm(xhi, xlo, B, Cin, T, w, bias, Cout, K, stride, pad, y, wp,
-                                      st);
+                                      st, f16);
   }
   if (plan.path == 1)
     return launch_conv_transpose1d_tc(x, B, Cin, T, w, bias, Cout, K, stride, pad, y,
@@ -1095,6 +1096,10 @@ bv_status check_weights(const bv_decoder_config *c, const bv_decoder_weights *w)
 // y_pitch samples.
 // Weights prepared for a decode: split tensor-core weights and, per ConvT
 // stage, its packed phase weights (nullptr: packed into the workspace).
+// A decoder's transposed conv of Cin input channels takes the fp16 split
+// (where the time-major kernel runs it at all).
+bool convt_f16(const bv_decoder_config *c, int Cin) { return tm_f16_ok(Cin) && !c->tf32_only; }
+
 struct DecoderPrep {
   DecoderSplit sw;
   const float *convt[BV_MAX_UP] = {};
@@ -1136,14 +1141,17 @@ bv_status decode_core(const bv_decoder_config *c, const bv_decoder_weights *w,
     const int pad = (k - sr) / 2;
     const int n2 = (n - 1) * sr + k - 2 * pad;
     if (conv_transpose1d_tm_supported(C, Co, k, sr)) {
-      // time-major: the stage input goes to block 0's operand planes first
-      BV_TRY(launch_transpose_split(A, s.xhi, s.xlo, B, C, n, st));
+      // time-major: the stage input goes to block 0's operand planes first,
+      // in the fp16 split where C allows and the config does not ask for
+      // 3xTF32 (the prepared phase weights were packed by the same rule)
+      const bool f16 = convt_f16(c, C);
+      BV_TRY(launch_transpose_split(A, s.xhi, s.xlo, B, C, n, st, f16));
       if (pp.convt[i])
         BV_TRY(launch_conv_transpose1d_tm_packed(s.xhi, s.xlo, B, C, n, pp.convt[i], w->up_b[i],
-                                                 Co, k, sr, pad, S, st));
+                                                 Co, k, sr, pad, S, st, f16));
       else
         BV_TRY(launch_conv_transpose1d_tm(s.xhi, s.xlo, B, C, n, w->up_w[i], w->up_b[i], Co, k,
-                                          sr, pad, S, WP, st));
+                                          sr, pad, S, WP, st, f16));
     } else if (conv_transpose1d_tc_supported(C, Co, k, sr)) {
       if (pp.convt[i])
         BV_TRY(launch_conv_transpose1d_tc_packed(A, B, C, n, pp.convt[i], w->up_b[i], Co, k, sr,
@@ -1430,7 +1438,7 @@ bv_status bv_decoder_prepare(const bv_decoder_config *c, const bv_decoder_weight
     const int Co = c->up_channels[i], k = c->up_kernel[i], sr = c->up_rate[i];
     float *wp = const_cast<float *>(slots[i]);
     if (wp && conv_transpose1d_tm_supported(C, Co, k, sr))
-      BV_TRY(launch_convt_pack_tm(w->up_w[i], C, Co, k, sr, wp, st));
+      BV_TRY(launch_convt_pack_tm(w->up_w[i], C, Co, k, sr, wp, st, convt_f16(c, C)));
     else if (wp)
       BV_TRY(launch_convt_pack_tc(w->up_w[i], C, Co, k, sr, wp, st));
     C = Co;

@@ -285,25 +285,28 @@ bv_status launch_conv1d_tm(const float *x_hi, const float *x_lo, int B, int Cin,
 // Transposed conv on the time-major kernel: x_hi / x_lo [B, T, Cin] planes
 // (launch_transpose_split), each of the S output phases an ceil(K/S)-tap conv
 // over the input samples with its weights repacked tap-major into wp
-// (conv_transpose1d_tm_workspace bytes).
+// (conv_transpose1d_tm_workspace bytes).  f16: planes and phase weights in
+// the fp16 split (tm_f16_ok(Cin)), as launch_conv1d_tm.
 bool conv_transpose1d_tm_supported(int Cin, int Cout, int K, int S);
 size_t conv_transpose1d_tm_workspace(int Cin, int Cout, int K, int S);
 bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
                                      const float *w, const float *bias, int Cout, int K, int S,
-                                     int pad, float *y, float *wp, cudaStream_t st);
+                                     int pad, float *y, float *wp, cudaStream_t st,
+                                     bool f16 = false);
 
 // The same with the phase weights packed beforehand (launch_convt_pack_tm
-// writes conv_transpose1d_tm_workspace bytes).
+// writes at most conv_transpose1d_tm_workspace bytes, in the same split).
 bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, float *wp,
-                               cudaStream_t st);
+                               cudaStream_t st, bool f16 = false);
 bv_status launch_conv_transpose1d_tm_packed(const float *x_hi, const float *x_lo, int B, int Cin,
                                             int T, const float *wp, const float *bias, int Cout,
-                                            int K, int S, int pad, float *y, cudaStream_t st);
+                                            int K, int S, int pad, float *y, cudaStream_t st,
+                                            bool f16 = false);
 
 // [B, C, T] -> time-major planes hi[b, t, c] = tf32(x[b, c, t]),
-// lo = x - hi.
+// lo = x - hi (f16: fp16(x) and fp16(x - hi), halves at the same addresses).
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
-                                 cudaStream_t st);
+                                 cudaStream_t st, bool f16 = false);
 
 // ConvTranspose1d on the tensor cores: each output phase is an ordinary conv
 // over the input samples with repacked weights (wp: workspace of

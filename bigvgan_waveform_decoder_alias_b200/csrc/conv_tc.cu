@@ -1420,9 +1420,10 @@ __global__ void convt_repack_kernel(const float *__restrict__ w, float *__restri
 
 // Tap-major phase weights for the time-major kernel: wp[r][o][j cp + i] =
 // w[i][o][r + S (nt - 1 - j)] split into tf32 hi / lo (zero past K or Cin).
+// f16: the parts are fp16 of kTmF16WScale W (wp and wp_lo then hold halves)
 __global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__restrict__ wp,
                                        float *__restrict__ wp_lo, int Cin, int Cout, int K, int S,
-                                       int nt, int cp) {
+                                       int nt, int cp, int f16) {
   const long long total = (long long)S * Cout * nt * cp;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -1434,9 +1435,16 @@ __global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__res
     const int r = (int)(rest / Cout);
     const int k = r + S * (nt - 1 - j);
     const float v = (k < K && i < Cin) ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
-    const float h = tf32_hi(v);
-    wp[idx] = h;
-    wp_lo[idx] = v - h;
+    if (f16) {
+      const float vs = v * kTmF16WScale;
+      const __half h = __float2half_rn(vs);
+      reinterpret_cast<__half *>(wp)[idx] = h;
+      reinterpret_cast<__half *>(wp_lo)[idx] = __float2half_rn(vs - __half2float(h));
+    } else {
+      const float h = tf32_hi(v);
+      wp[idx] = h;
+      wp_lo[idx] = v - h;
+    }
   }
 }
 
@@ -1518,7 +1526,9 @@ __global__ void split_weights_kernel(SplitTable tab) {
 }
 
 // hi[b, t, c] = tf32(x[b, c, t]), lo = x - hi: 32 x 32 tiles through shared
-// memory, reads along t and writes along c both coalesced.
+// memory, reads along t and writes along c both coalesced.  F16: fp16 parts,
+// hi = fp16(x), lo = fp16(x - hi).
+template <bool F16>
 __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__restrict__ x,
                                                                float *__restrict__ hi,
                                                                float *__restrict__ lo, int C,
@@ -1538,10 +1548,17 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__res
   for (int r = ty; r < 32; r += 8) {
     const int t = t0 + r;
     if (t < T && c0 + tx < C) {
-      const float v = tile[tx][r], h = tf32_hi(v);
+      const float v = tile[tx][r];
       const size_t idx = ob + (size_t)t * C + c0 + tx;
-      hi[idx] = h;
-      lo[idx] = v - h;
+      if constexpr (F16) {
+        const __half h = __float2half_rn(v);
+        reinterpret_cast<__half *>(hi)[idx] = h;
+        reinterpret_cast<__half *>(lo)[idx] = __float2half_rn(v - __half2float(h));
+      } else {
+        const float h = tf32_hi(v);
+        hi[idx] = h;
+        lo[idx] = v - h;
+      }
     }
   }
 }
@@ -1549,13 +1566,16 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__res
 }  // namespace
 
 bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, int C, int T,
-                                 cudaStream_t st) {
+                                 cudaStream_t st, bool f16) {
   if (B <= 0 || T <= 0) return BV_OK;
   dim3 grid((T + 31) / 32, (C + 31) / 32, B);
   if (grid.y > 65535 || grid.z > 65535) return fail(BV_ERR_SHAPE, "transpose_split: grid");
   {
-    LaunchTimer tm(st, "transpose_split", 0.0, 12.0 * B * C * T);
-    transpose_split_kernel<<<grid, 256, 0, st>>>(x, hi, lo, C, T);
+    LaunchTimer tm(st, "transpose_split", 0.0, (f16 ? 8.0 : 12.0) * B * C * T);
+    if (f16)
+      transpose_split_kernel<true><<<grid, 256, 0, st>>>(x, hi, lo, C, T);
+    else
+      transpose_split_kernel<false><<<grid, 256, 0, st>>>(x, hi, lo, C, T);
   }
   count_launch();
   return check_launch("transpose_split_kernel");
@@ -1733,14 +1753,17 @@ size_t conv_transpose1d_tm_workspace(int Cin, int Cout, int K, int S) {
 }
 
 bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, float *wp,
-                               cudaStream_t st) {
-  const int nt = convt_taps(K, S), cp = tm_cin_pad(Cin);
+                               cudaStream_t st, bool f16) {
+  const int nt = convt_taps(K, S), cp = f16 ? tm_cin_pad_f16(Cin) : tm_cin_pad(Cin);
   const long long total = (long long)S * Cout * nt * cp;
+  // lo follows hi: total values of 4 (tf32) or 2 (fp16) bytes
+  float *wp_lo = reinterpret_cast<float *>(reinterpret_cast<char *>(wp) + total * (f16 ? 2 : 4));
   {
-    LaunchTimer tm(st, "convt_repack", 0.0, 4.0 * (double)Cin * Cout * K + 8.0 * (double)total);
+    LaunchTimer tm(st, "convt_repack", 0.0,
+                   4.0 * (double)Cin * Cout * K + (f16 ? 4.0 : 8.0) * (double)total);
     const long long blocks = (total + 255) / 256;
     convt_repack_tm_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
-        w, wp, wp + total, Cin, Cout, K, S, nt, cp);
+        w, wp, wp_lo, Cin, Cout, K, S, nt, cp, f16 ? 1 : 0);
   }
   count_launch();
   return check_launch("convt_repack_tm_kernel");
@@ -1748,30 +1771,32 @@ bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, 
 
 bv_status launch_conv_transpose1d_tm_packed(const float *x_hi, const float *x_lo, int B, int Cin,
                                             int T, const float *wp, const float *bias, int Cout,
-                                            int K, int S, int pad, float *y, cudaStream_t st) {
+                                            int K, int S, int pad, float *y, cudaStream_t st,
+                                            bool f16) {
   if (B <= 0 || T <= 0) return BV_OK;
-  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
-    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
+  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S) || (f16 && !tm_f16_ok(Cin)))
+    return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d%s", Cin, Cout,
+                f16 ? " (fp16)" : "");
   const int nt = convt_taps(K, S);
   const int Tout = (T - 1) * S + K - 2 * pad;
   // phase r: conv output P (input-grid index, P < T + nt - 1) lands on sample
   // S P + r - pad of the output row
-  return tm_impl("conv_transpose1d_tm", x_hi, x_lo, B, Cin, T, wp, S * Cout, bias, Cout, nt, 1,
-                 nt - 1, Epi{nullptr, 1.0f, 0, 0}, y, T + nt - 1, Tout, OutMap{S, -pad, Tout, S},
-                 2.0 * B * Cin * (double)Cout * K * T,
+  return tm_impl(f16 ? "conv_transpose1d_tm_f16" : "conv_transpose1d_tm", x_hi, x_lo, B, Cin, T,
+                 wp, S * Cout, bias, Cout, nt, 1, nt - 1, Epi{nullptr, 1.0f, 0, 0}, y, T + nt - 1,
+                 Tout, OutMap{S, -pad, Tout, S}, 2.0 * B * Cin * (double)Cout * K * T,
                  4.0 * ((double)B * Cin * T + (double)Cin * Cout * K + (double)B * Cout * Tout),
-                 st);
+                 st, f16);
 }
 
 bv_status launch_conv_transpose1d_tm(const float *x_hi, const float *x_lo, int B, int Cin, int T,
                                      const float *w, const float *bias, int Cout, int K, int S,
-                                     int pad, float *y, float *wp, cudaStream_t st) {
+                                     int pad, float *y, float *wp, cudaStream_t st, bool f16) {
   if (B <= 0 || T <= 0) return BV_OK;
-  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S))
+  if (!conv_transpose1d_tm_supported(Cin, Cout, K, S) || (f16 && !tm_f16_ok(Cin)))
     return fail(BV_ERR_UNSUPPORTED, "conv_transpose1d_tm: Cin %d Cout %d", Cin, Cout);
-  BV_TRY(launch_convt_pack_tm(w, Cin, Cout, K, S, wp, st));
+  BV_TRY(launch_convt_pack_tm(w, Cin, Cout, K, S, wp, st, f16));
   return launch_conv_transpose1d_tm_packed(x_hi, x_lo, B, Cin, T, wp, bias, Cout, K, S, pad, y,
-                                           st);
+                                           st, f16);
 }
 
 }  // namespace bv

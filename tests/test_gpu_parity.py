@@ -333,10 +333,15 @@ TC_CASES = [(64, 64, 3, 1, 200), (128, 128, 3, 1, 1), (128, 128, 7, 3, 5), (96, 
 # fed by the time-major activation take for channel counts that are
 # multiples of 8 from 48 up.
 TM_CLASSES = ("conv1d_tm", "conv1d_tm_f16")
+TMT_CLASSES = ("conv_transpose1d_tm", "conv_transpose1d_tm_f16")
 
 
 def _has_tm(classes):
     return any(c in classes for c in TM_CLASSES)
+
+
+def _has_tmt(classes):
+    return any(c in classes for c in TMT_CLASSES)
 
 
 def _kernel_classes(nat, fn):
@@ -505,7 +510,8 @@ def test_full_size_conv_transpose_time_major_sampled(nat, oracle, Cin, Cout, S, 
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault(
         "y", nat.bv_conv_transpose1d_ws(xd, wd, bd, S, pad)))
-    assert "conv_transpose1d_tm" in classes, classes
+    # every Cin here is a multiple of 8 from 48 up: the fp16 split
+    assert "conv_transpose1d_tm_f16" in classes, classes
     y = host(out["y"])
     Tout = (T - 1) * S + K - 2 * pad
     assert y.shape == (2, Cout, Tout)
@@ -669,7 +675,7 @@ def test_decoder_tensor_core_stages(nat, oracle, filt, frames):
     zd = dev(z)
     out = {}
     classes = _kernel_classes(nat, lambda: out.setdefault("y", dec.decode(zd)))
-    assert "conv_transpose1d_tm" in classes, classes
+    assert "conv_transpose1d_tm_f16" in classes, classes
     # the 128/96/48-channel AMP convs run time-major, fed by the activation
     # writing their operand planes; the ConvT inputs are transposed
     assert _has_tm(classes) and "activation_tm" in classes, classes
@@ -1005,7 +1011,7 @@ def test_decode_with_prepared_weights(nat, filt):
         # kernel classes are compared there)
         classes = _kernel_classes(nat, lambda: prep.decode(z))
         assert "weight_split" not in classes and "convt_repack" not in classes, classes
-        assert _has_tm(classes) and "conv_transpose1d_tm" in classes, classes
+        assert _has_tm(classes) and _has_tmt(classes), classes
         n_units = prep.tile_count(13) * 2
         rows = prep.decode_units(z, 0, n_units)
         np.testing.assert_array_equal(host(prep.stitch_units(rows, 2, 13)), want)
