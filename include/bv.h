@@ -227,7 +227,9 @@ bv_status bv_act_conv1d(const float *x, int B, int C, int T,
 /* bv_conv_transpose1d on the kernels the decoder runs for its upsampling
  * stages: with the workspace the phases run on the time-major tensor-core
  * kernel (or the [B, C, T] one) where the shape qualifies, else on the FP32
- * kernel (then the workspace may be empty).  Arguments, result and errors
+ * kernel (then the workspace may be empty).  The time-major kernel takes the
+ * fp16 split where Cin is a multiple of 8 from 48 up, as bv_act_conv1d
+ * (inputs below 65504 in magnitude), else 3xTF32.  Arguments, result and errors
  * as bv_conv_transpose1d, plus BV_ERR_WORKSPACE.  Workspace:
  * bv_conv_transpose1d_workspace_size bytes, 256-byte aligned, disjoint
  * from x and y. */
@@ -361,9 +363,10 @@ typedef struct {
                         * > 0: z holds normalised latents [latent_channels, B,
                         * frames] that first go through the latent front end
                         * (bv_latent_front_end) into in_channels */
-  int tf32_only;       /* 0: the AMP-block convs whose channel count is a
-                        * multiple of 8 from 48 up take their tensor-core
-                        * operands as two fp16 parts (x = hi + lo, W likewise,
+  int tf32_only;       /* 0: the AMP-block convs and the transposed convs
+                        * whose input channel count is a multiple of 8 from
+                        * 48 up take their tensor-core operands as two fp16
+                        * parts (x = hi + lo, W likewise,
                         * three products accumulated in fp32: 22 significant
                         * bits per operand as in the tf32 split, rounded
                         * instead of truncated, at twice the tf32 MMA rate);
