@@ -1527,12 +1527,13 @@ __global__ void split_weights_kernel(SplitTable tab) {
 
 // hi[b, t, c] = tf32(x[b, c, t]), lo = x - hi: 32 x 32 tiles through shared
 // memory, reads along t and writes along c both coalesced.  F16: fp16 parts,
-// hi = fp16(x), lo = fp16(x - hi).
+// hi = fp16(x), lo = fp16(x - hi); a value at or past fp16's range sets the
+// status word.
 template <bool F16>
 __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__restrict__ x,
                                                                float *__restrict__ hi,
                                                                float *__restrict__ lo, int C,
-                                                               int T) {
+                                                               int T, int *status) {
   __shared__ float tile[32][33];
   const int t0 = blockIdx.x * 32, c0 = blockIdx.y * 32, b = blockIdx.z;
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;  // 8 rows of 32
@@ -1554,6 +1555,7 @@ __global__ void __launch_bounds__(256) transpose_split_kernel(const float *__res
         const __half h = __float2half_rn(v);
         reinterpret_cast<__half *>(hi)[idx] = h;
         reinterpret_cast<__half *>(lo)[idx] = __float2half_rn(v - __half2float(h));
+        if (fabsf(v) >= 65504.0f && status) atomicExch(status, kStatusF16Range);
       } else {
         const float h = tf32_hi(v);
         hi[idx] = h;
@@ -1573,9 +1575,9 @@ bv_status launch_transpose_split(const float *x, float *hi, float *lo, int B, in
   {
     LaunchTimer tm(st, "transpose_split", 0.0, (f16 ? 8.0 : 12.0) * B * C * T);
     if (f16)
-      transpose_split_kernel<true><<<grid, 256, 0, st>>>(x, hi, lo, C, T);
+      transpose_split_kernel<true><<<grid, 256, 0, st>>>(x, hi, lo, C, T, device_status_ptr());
     else
-      transpose_split_kernel<false><<<grid, 256, 0, st>>>(x, hi, lo, C, T);
+      transpose_split_kernel<false><<<grid, 256, 0, st>>>(x, hi, lo, C, T, nullptr);
   }
   count_launch();
   return check_launch("transpose_split_kernel");

@@ -124,3 +124,21 @@ def test_fp16_operand_range_is_reported(nat, oracle):
     assert _status(nat) == 0
     want = oracle.conv1d(oracle.activation1d(x, la, lb), w, b, d, 1)
     assert rel_l2(y.cpu().numpy(), want) < LAYER_TOL
+
+
+def test_fp16_operand_range_is_reported_for_transposed_convs(nat, oracle):
+    """The transposed conv's fp16 planes (64 input channels) from inputs of
+    order 1e5: BV_ERR_RANGE; then ordinary inputs are clean and match."""
+    s = synth.NormalStream(323)
+    Cin, Cout, S, T = 64, 48, 2, 300
+    K, pad = 2 * S, S // 2
+    x = s.normal((2, Cin, T))
+    w = s.normal((Cin, Cout, K), 0.0, 0.02)
+    b = s.normal((Cout,), 0.0, 0.02)
+    wd, bd = torch.from_numpy(w).cuda(), torch.from_numpy(b).cuda()
+    assert _status(nat) == 0
+    nat.bv_conv_transpose1d_ws(torch.from_numpy(1.0e5 * x).cuda(), wd, bd, S, pad)
+    assert _status(nat) == BV_ERR_RANGE
+    y = nat.bv_conv_transpose1d_ws(torch.from_numpy(x).cuda(), wd, bd, S, pad)
+    assert _status(nat) == 0
+    assert rel_l2(y.cpu().numpy(), oracle.conv_transpose1d(x, w, b, S, pad)) < LAYER_TOL
