@@ -1181,7 +1181,9 @@ conv1d_tm_kernel(const __grid_constant__ CUtensorMap tmap_xhi,
         if constexpr (STG) {
           // staged: the warp's 32 time steps x 16 channels go out in one
           // bulk store, which clips rows past y_len and channels past Cout
-          float val[16];
+          float val[16];  // rows past y_len stage zeros (the store clips them)
+#pragma unroll
+          for (int e = 0; e < 16; ++e) val[e] = 0.0f;
           if (in) epi_values<16>(sum + g, bb, eg, y, idx0, (size_t)y_pitch, Cout - (tl.o0 + g), val);
           if (tl.o0 + g < Cout && tl.t0 + 32 * q < y_len) {  // warp-uniform
             float *sb = reinterpret_cast<float *>(stg_base + (2 * q + (sgi & 1)) * TM_STG_BUF);
