@@ -50,8 +50,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tf32-only", action="store_true",
                     help="decode with every tensor-core conv in 3xTF32 (bv_decoder_config."
-                         "tf32_only); by default the AMP convs that qualify use the fp16 "
-                         "split and the line also reports the 3xTF32 decode")
+                         "tf32_only); by default the AMP and transposed convs that qualify use "
+                         "the fp16 split and the line also reports the 3xTF32 decode")
     ap.add_argument("--case", default=None,
                     help="time one kernel on one shape instead of the decoder (for profiling): "
                          "activation:BxCxT | conv1d:BxCxT:K:d | convt:BxCinxT:Cout:s | "
@@ -685,8 +685,8 @@ def main():
                        "weights": "resident, split and ConvT packing prepared once at load",
                        "conv_split": ("3xTF32 throughout" if args.tf32_only else
                                       "fp16 split (3 products, fp32 accumulate) for the AMP "
-                                      "convs of 48+ channels in multiples of 8, 3xTF32 "
-                                      "elsewhere"),
+                                      "and transposed convs of 48+ input channels in "
+                                      "multiples of 8, 3xTF32 elsewhere"),
                        "parallelism": f"replicas x{world}"},
             "e2e": {"value": e2e_value, "unit": UNIT,
                     "h2d_bytes_per_step": int(zh.numel() * 4),
