@@ -115,6 +115,25 @@ def test_decoder_bookkeeping(nat, oracle):
     assert nat.bv_decoder_param_count(cfg) == -1
 
 
+def test_conv_split_flag_is_checked_and_changes_no_sizes(nat):
+    """tf32_only is 0 or 1; the split it selects fits the same buffers (an
+    fp16 split row of 64-channel blocks takes at most the bytes of a tf32 one
+    of 32-channel blocks), so no workspace or prepared size depends on it."""
+    L = nat.lib()
+    for geo in (synth.H3, synth.LTX):
+        a = nat.decoder_config(geo, 200, 16)
+        b = nat.decoder_config(geo, 200, 16, tf32_only=True)
+        assert b.tf32_only == 1 and a.tf32_only == 0
+        for f in (L.bv_decode_workspace_size, L.bv_decode_workspace_size_prepared):
+            assert f(ctypes.byref(a), 2, 2400) == f(ctypes.byref(b), 2, 2400) > 0
+        assert L.bv_decoder_prepared_size(ctypes.byref(a)) == \
+            L.bv_decoder_prepared_size(ctypes.byref(b)) > 0
+    bad = nat.decoder_config(synth.H3)
+    bad.tf32_only = 2
+    assert L.bv_decode_workspace_size(ctypes.byref(bad), 2, 400) == 0
+    assert "tf32_only" in nat.last_error()
+
+
 def test_decode_workspace_grows_with_tiles(nat):
     L = nat.lib()
     untiled = nat.decoder_config(synth.H3)
