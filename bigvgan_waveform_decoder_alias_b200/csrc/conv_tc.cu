@@ -612,8 +612,13 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
 // ---------------------------------------------------------------------------
 // Time-major variant on CTA pairs.  The input arrives as two [B, T, Cin]
 // planes, X_hi = tf32(x) and X_lo = x - X_hi (written by
-// launch_transpose_split), and the weights as tap-major [Cout, K Cin] hi / lo
-// matrices, W'[o, j Cin + i] = w[o, i, j].
+// launch_transpose_split or the time-major activation), and the weights as
+// tap-major [Cout, K Cin] hi / lo matrices, W'[o, j Cin + i] = w[o, i, j].
+// With F16 the same holds with fp16 parts (X_hi = fp16(x), X_lo = fp16(x -
+// X_hi); the weights' parts are of 2^12 W, scaled back in the run sums), a
+// 128-byte operand row holds 64 channels instead of 32, and the MMAs are
+// kind::f16 (K = 16) over the same 32-byte steps: the box geometry, swizzle,
+// descriptors and barriers are those of tf32.
 //
 // Two CTAs of a cluster share each MMA (tcgen05 cta_group::2, M = 256): CTA r
 // of the pair owns time rows t0 + 128 r .. + 127 (its half of the A operand
@@ -621,7 +626,7 @@ bv_status run_tc(const CUtensorMap &tmap, const CUtensorMap &tmap_lo, const floa
 // (its half of the B operand), so each SM fetches half the weight bytes a
 // lone CTA would; the weights are what every time tile re-reads from L2.
 //
-// For each 32-channel block cb, one TMA box per plane brings input rows
+// For each 32-channel (fp16: 64-channel) block cb, one TMA box per plane brings input rows
 // t0 - pad .. t0 - pad + 127 + (K - 1) d (zero outside [0, T), the conv's
 // zero padding) by the block's 32 channels: K-major rows of 128 bytes, the A
 // operand layout.  Tap j's A operand is the same box seen from row j d on:
