@@ -1430,7 +1430,7 @@ __global__ void convt_repack_kernel(const float *__restrict__ w, float *__restri
 // f16: the parts are fp16 of kTmF16WScale W (wp and wp_lo then hold halves)
 __global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__restrict__ wp,
                                        float *__restrict__ wp_lo, int Cin, int Cout, int K, int S,
-                                       int nt, int cp, int f16) {
+                                       int nt, int cp, int f16, int *status) {
   const long long total = (long long)S * Cout * nt * cp;
   for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
@@ -1444,6 +1444,7 @@ __global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__res
     const float v = (k < K && i < Cin) ? w[((size_t)i * Cout + o) * K + k] : 0.0f;
     if (f16) {
       const float vs = v * kTmF16WScale;
+      if (fabsf(vs) >= 65504.0f && status) atomicExch(status, kStatusF16Range);  // |W| >= 16
       const __half h = __float2half_rn(vs);
       reinterpret_cast<__half *>(wp)[idx] = h;
       reinterpret_cast<__half *>(wp_lo)[idx] = __float2half_rn(vs - __half2float(h));
@@ -1457,7 +1458,7 @@ __global__ void convt_repack_tm_kernel(const float *__restrict__ w, float *__res
 
 // dst[0 .. n) = tf32(src), dst[n .. 2n) = src - tf32(src), per table entry
 // (float4 where the entry allows it; tap-major entries reorder as they go)
-__global__ void split_weights_kernel(SplitTable tab) {
+__global__ void split_weights_kernel(SplitTable tab, int *status) {
   for (int e = blockIdx.y; e < tab.n; e += gridDim.y) {
     const float *__restrict__ src = tab.src[e];
     float *__restrict__ hi = tab.dst[e];
@@ -1492,6 +1493,8 @@ __global__ void split_weights_kernel(SplitTable tab) {
             const long long d = o * drow + (long long)j * cp + i0 + ii;
             if (f16) {
               const float v = sl[ii * k + j] * kTmF16WScale;
+              // fp16 holds |2^12 W| < 65504: a weight of 16 or more is reported
+              if (fabsf(v) >= 65504.0f && status) atomicExch(status, kStatusF16Range);
               const __half h = __float2half_rn(v);
               hi16[d] = h;
               lo16[d] = __float2half_rn(v - __half2float(h));
@@ -1597,7 +1600,7 @@ bv_status launch_split_weights(const SplitTable &tab, cudaStream_t st) {
   for (int e = 0; e < tab.n; ++e) bytes += 12.0 * tab.count[e];
   {
     LaunchTimer tm(st, "weight_split", 0.0, bytes);
-    split_weights_kernel<<<dim3(64, tab.n), 256, 0, st>>>(tab);
+    split_weights_kernel<<<dim3(64, tab.n), 256, 0, st>>>(tab, device_status_ptr());
   }
   count_launch();
   return check_launch("split_weights_kernel");
@@ -1772,7 +1775,7 @@ bv_status launch_convt_pack_tm(const float *w, int Cin, int Cout, int K, int S, 
                    4.0 * (double)Cin * Cout * K + (f16 ? 4.0 : 8.0) * (double)total);
     const long long blocks = (total + 255) / 256;
     convt_repack_tm_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, st>>>(
-        w, wp, wp_lo, Cin, Cout, K, S, nt, cp, f16 ? 1 : 0);
+        w, wp, wp_lo, Cin, Cout, K, S, nt, cp, f16 ? 1 : 0, device_status_ptr());
   }
   count_launch();
   return check_launch("convt_repack_tm_kernel");

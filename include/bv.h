@@ -46,8 +46,9 @@ typedef enum {
   BV_ERR_CUDA = 4,        /* a CUDA call failed (message has the CUDA error) */
   BV_ERR_TIMEOUT = 5,     /* a bounded device-side wait gave up */
   BV_ERR_UNSUPPORTED = 6, /* a valid request this build does not implement */
-  BV_ERR_RANGE = 7        /* an activation reached fp16's range (|v| >= 65504) on
-                             the fp16 time-major path; that output is not valid */
+  BV_ERR_RANGE = 7        /* an activation reached fp16's range (|v| >= 65504),
+                             or a weight 16 or more (2^12 |w| >= 65504), on the
+                             fp16 time-major path; that output is not valid */
 } bv_status;
 
 #define BV_FILTER_TAPS 12 /* both resampling filters: 12 taps ([H3] FILTER_LEN) */

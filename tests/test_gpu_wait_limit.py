@@ -142,3 +142,21 @@ def test_fp16_operand_range_is_reported_for_transposed_convs(nat, oracle):
     y = nat.bv_conv_transpose1d_ws(torch.from_numpy(x).cuda(), wd, bd, S, pad)
     assert _status(nat) == 0
     assert rel_l2(y.cpu().numpy(), oracle.conv_transpose1d(x, w, b, S, pad)) < LAYER_TOL
+
+
+def test_fp16_weight_range_is_reported(nat, oracle):
+    """Weights of 16 or more leave fp16's range once scaled by 2^12 for the
+    fp16 split: the split reports BV_ERR_RANGE instead of infinities."""
+    s = synth.NormalStream(324)
+    C, T, K, d = 64, 200, 3, 1
+    x = s.normal((2, C, T))
+    la, lb = s.normal((C,), 0.0, 0.1), s.normal((C,), 0.0, 0.1)
+    w = s.normal((C, C, K), 0.0, 0.02)
+    w[3, 5, 1] = 20.0
+    b = s.normal((C,), 0.0, 0.02)
+    filt = torch.from_numpy(nat.bv_filter_design()).cuda()
+    lad, lbd = (torch.from_numpy(a).cuda() for a in (la, lb))
+    assert _status(nat) == 0
+    nat.bv_act_conv1d(torch.from_numpy(x).cuda(), lad, lbd, filt, torch.from_numpy(w).cuda(),
+                      torch.from_numpy(b).cuda(), d, 1)
+    assert _status(nat) == BV_ERR_RANGE
